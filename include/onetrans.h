@@ -1,0 +1,238 @@
+/*
+ * onetrans.h - C ABI of the OneTrans hot path on B200 (sm_100a).
+ *
+ * The library runs the forward pass of the OneTrans block stack and its
+ * two-stage KV-cached scoring, as described in fun-rec mdbook 7.5, "OneTrans:
+ * Unifying Sequence Modeling and Feature Interaction" (cited below as [FR]),
+ * and in the paper-daily deep reading "OneTrans: Unified Feature Interaction
+ * and Sequence Modeling with One Transformer in Industrial Recommender" ([PD]).
+ *
+ * Conventions shared by every call
+ *  - Every pointer is a DEVICE pointer owned by the caller unless marked
+ *    "host".  The library never allocates device memory: each call takes a
+ *    caller-provided workspace whose size onetrans_workspace_size() reports,
+ *    and the KV cache lives in a caller-provided pool (onetrans_cache_size()).
+ *  - Tensors are dense row-major.  Element type follows the model's mode:
+ *    ONETRANS_BF16 -> bfloat16 storage (fp32 accumulation inside kernels),
+ *    ONETRANS_FP32 -> float32 storage and float32 arithmetic on CUDA cores.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream; inputs must stay valid
+ *    and unmodified until the stream reaches the call's end.
+ *  - Argument and shape errors are detected on the host before any launch and
+ *    leave device memory untouched.  Launch failures return ONETRANS_ERR_CUDA.
+ *  - A model is immutable after creation and may be used from several
+ *    streams at once.  Calls that modify one cache slot must not overlap.
+ *  - Buffers must be 16-byte aligned; the workspace and cache pool 256-byte.
+ */
+#ifndef ONETRANS_H
+#define ONETRANS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ONETRANS_API __attribute__((visibility("default")))
+#else
+#define ONETRANS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ONETRANS_OK = 0,
+  ONETRANS_ERR_INVALID_ARG = -1, /* NULL pointer, bad enum, misaligned buffer */
+  ONETRANS_ERR_SHAPE = -2,       /* sizes inconsistent with the model/schedule */
+  ONETRANS_ERR_UNSUPPORTED = -3, /* e.g. append on a pyramid model */
+  ONETRANS_ERR_CAPACITY = -4,    /* workspace or cache pool too small, slot full */
+  ONETRANS_ERR_CUDA = -5,        /* a CUDA runtime/driver call failed */
+  ONETRANS_ERR_DEVICE_CHECK = -6 /* a kernel's own bounds check fired */
+} onetrans_status;
+
+typedef enum { ONETRANS_BF16 = 0, ONETRANS_FP32 = 1 } onetrans_mode;
+
+/* Model hyper-parameters.  [FR] 7.5.0-7.5.2 fix the structure; the widths,
+ * head count, depth and schedule are the caller's choice.
+ *  d_model % n_heads == 0, d_h = d_model / n_heads in {32, 64, 96, 128}.
+ *  pyramid_q (host, n_layers entries): L'_n, the number of tail rows kept as
+ *    queries by layer n ([FR] 7.5.2, tail index set Q = {L-L'+1..L}).  NULL
+ *    keeps every row.  Must be non-increasing and >= L_NS.
+ *  ns_feat_dim / ns_hidden: F and H of the auto-split MLP (0 if unused).
+ *  n_behaviors / event_dim: per-behavior event MLP used by cache append.
+ *  page_tokens: KV-cache page size in tokens; must be 64. */
+typedef struct {
+  int32_t n_layers, d_model, n_heads, d_ff, L_NS;
+  int32_t ns_feat_dim, ns_hidden;
+  int32_t n_behaviors, event_dim;
+  const int32_t* pyramid_q;
+  float rms_eps;
+  int32_t mode;
+  int32_t page_tokens;
+} onetrans_config;
+
+/* Weights (device pointers, row-major W[out][in]; borrowed: the caller keeps
+ * them alive while the model exists).  Per-layer entries are HOST arrays of
+ * n_layers device pointers.  Mixed parameterization ([FR] 7.5.1): *_S is the
+ * set shared by every S-token, *_NS holds one set per NS-token, stacked.
+ *   g_attn, g_ffn      [d]              RMSNorm gains before attention / FFN
+ *   Wqkv_S             [3d, d]          rows 0..d-1 = W^Q, d..2d-1 = W^K, 2d.. = W^V
+ *   Wqkv_NS            [L_NS, 3d, d]
+ *   Wo                 [d, d]           output projection shared by all tokens
+ *   W1_S, b1_S         [d_ff, d], [d_ff]
+ *   W2_S, b2_S         [d, d_ff], [d]
+ *   W1_NS, b1_NS       [L_NS, d_ff, d], [L_NS, d_ff]
+ *   W2_NS, b2_NS       [L_NS, d, d_ff], [L_NS, d]
+ * Auto-split tokenizer ([FR] 7.5.0, NS-tokens = Split(MLP(Concat(NS)), L_NS)):
+ *   Wa1 [H, F], ba1 [H], Wa2 [L_NS*d, H], ba2 [L_NS*d]      (may be NULL)
+ * Per-behavior event MLP and type identifiers ([FR] 7.5.0, MLP_i and the
+ * timestamp-aware merge): host arrays of n_behaviors device pointers
+ *   Wb1[t] [d, event_dim], bb1[t] [d], Wb2[t] [d, d], bb2[t] [d];
+ *   type_emb [n_behaviors, d]                                  (may be NULL) */
+typedef struct {
+  const void* const* g_attn;
+  const void* const* g_ffn;
+  const void* const* Wqkv_S;
+  const void* const* Wqkv_NS;
+  const void* const* Wo;
+  const void* const* W1_S;
+  const void* const* b1_S;
+  const void* const* W2_S;
+  const void* const* b2_S;
+  const void* const* W1_NS;
+  const void* const* b1_NS;
+  const void* const* W2_NS;
+  const void* const* b2_NS;
+  const void* Wa1;
+  const void* ba1;
+  const void* Wa2;
+  const void* ba2;
+  const void* const* Wb1;
+  const void* const* bb1;
+  const void* const* Wb2;
+  const void* const* bb2;
+  const void* type_emb;
+} onetrans_weights;
+
+typedef struct onetrans_model onetrans_model;
+typedef struct onetrans_cache onetrans_cache;
+
+/* Which call a workspace is sized for. */
+typedef enum {
+  ONETRANS_OP_FORWARD = 0,   /* n = B samples, L = L_S */
+  ONETRANS_OP_STAGE1 = 1,    /* n = U users,   L = L_S */
+  ONETRANS_OP_STAGE2 = 2,    /* n = total candidates, L = cached L_S */
+  ONETRANS_OP_APPEND = 3,    /* n = U users,   L = dL */
+  ONETRANS_OP_AUTOSPLIT = 4  /* n = N feature rows, L unused */
+} onetrans_op;
+
+/* Validate `cfg`/`w` and create a model.  Copies the config and the pointer
+ * tables (not the weights).  Does not touch the GPU. */
+ONETRANS_API onetrans_status onetrans_model_create(const onetrans_config* cfg,
+                                      const onetrans_weights* w,
+                                      onetrans_model** out);
+ONETRANS_API onetrans_status onetrans_model_destroy(onetrans_model* m);
+
+/* Bytes of workspace `op` needs for n rows of length L (see onetrans_op). */
+ONETRANS_API onetrans_status onetrans_workspace_size(const onetrans_model* m, int32_t op,
+                                        int64_t n, int32_t L, size_t* bytes);
+
+/* Query counts of the stack for an input of L0 = L_S + L_NS rows: writes
+ * n_layers values L'_n to `out` (host).  With no pyramid every L'_n = L0.
+ * Returns SHAPE if the schedule does not fit L0 ([FR] 7.5.2). */
+ONETRANS_API onetrans_status onetrans_schedule(const onetrans_model* m, int32_t L_S,
+                                  int32_t* out);
+
+/* ---------------------------------------------------------------- cache --
+ * Paged, append-only KV cache of the S-side keys/values of every layer
+ * ([FR] 7.5.3 Stage I and cross-request caching; [PD] 6.2 on paged
+ * attention).  A page holds page_tokens consecutive tokens of one
+ * (slot, layer) as [K|V][head][token][d_h].  The pool starts with the page
+ * table (int32 [n_slots][n_layers][max_pages]) followed by the pages.  Page
+ * assignment and per-slot lengths are tracked on the host, so capacity errors
+ * never need a device read. */
+ONETRANS_API onetrans_status onetrans_cache_size(const onetrans_model* m, int32_t n_slots,
+                                    int32_t max_L_S, size_t* bytes);
+ONETRANS_API onetrans_status onetrans_cache_init(const onetrans_model* m, void* pool,
+                                    size_t bytes, int32_t n_slots,
+                                    int32_t max_L_S, onetrans_cache** out);
+ONETRANS_API onetrans_status onetrans_cache_destroy(onetrans_cache* c);
+/* Cached S length of `slot` (host); 0 = empty. */
+ONETRANS_API onetrans_status onetrans_cache_length(const onetrans_cache* c, int32_t slot,
+                                      int32_t* len);
+/* Device address of the first element of (slot, layer, kind 0=K/1=V, head,
+ * token): lets callers read back cached rows.  Host-side arithmetic only. */
+ONETRANS_API onetrans_status onetrans_cache_row_ptr(const onetrans_cache* c, int32_t slot,
+                                       int32_t layer, int32_t kind,
+                                       int32_t head, int32_t token,
+                                       void** ptr);
+
+/* ---------------------------------------------------------- entry points --
+ * Auto-split NS tokenizer ([FR] 7.5.0): ns = Split(MLP(feats), L_NS) with
+ * MLP = Linear(F->H) + ba1 -> GELU-tanh -> Linear(H->L_NS*d) + ba2.
+ *   feats     [N, F]
+ *   ns_tokens [L_NS, N, d]  token-major output (token t = MLP columns t*d..) */
+ONETRANS_API onetrans_status onetrans_tokenize_autosplit(const onetrans_model* m,
+                                            const void* feats, int64_t N,
+                                            void* ns_tokens, void* ws,
+                                            size_t ws_bytes, void* stream);
+
+/* Stage I ([FR] 7.5.3): run each user's S-tokens through the stack (pyramid
+ * tail queries included) and store every layer's S-side K/V in cache slot
+ * slots[u] (host array of U slot ids, distinct).  The slot's previous
+ * contents are replaced.  s_tokens [U, L_S, d]. */
+ONETRANS_API onetrans_status onetrans_stage1_encode(const onetrans_model* m,
+                                       onetrans_cache* c, const int32_t* slots,
+                                       int32_t U, const void* s_tokens,
+                                       int32_t L_S, void* ws, size_t ws_bytes,
+                                       void* stream);
+
+/* Stage II ([FR] 7.5.3): score candidates against the cached S side.  User u
+ * owns candidates cand_offsets[u] .. cand_offsets[u+1]-1 (host CSR, U+1
+ * entries) and cache slot slots[u] (host).  Per layer, NS token j of a
+ * candidate attends in one softmax to the slot's cached S keys and its own
+ * NS keys 0..j, then passes through its token-specific FFN.  All slots must
+ * hold the same S length.
+ *   ns_tokens [L_NS, C_tot, d] token-major input; ns_out [L_NS, C_tot, d]. */
+ONETRANS_API onetrans_status onetrans_stage2_score(const onetrans_model* m,
+                                      const onetrans_cache* c,
+                                      const int32_t* slots, int32_t U,
+                                      const int32_t* cand_offsets,
+                                      const void* ns_tokens, void* ns_out,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/* Cross-request append ([FR] 7.5.3): tokenize dL new events per user with the
+ * per-behavior MLP plus type identifier, run only those rows through every
+ * layer (keys: cached + new, causal), and append their K/V to slots[u].
+ * Non-pyramid models only (UNSUPPORTED otherwise).  All slots must hold the
+ * same length.  events [U, dL, event_dim]; types [U, dL] int32 (device). */
+ONETRANS_API onetrans_status onetrans_cache_append(const onetrans_model* m,
+                                      onetrans_cache* c, const int32_t* slots,
+                                      int32_t U, const void* events,
+                                      const int32_t* types, int32_t dL,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/* One-pass forward of the stack on X^(0) = [S-tokens; NS-tokens] ([FR] 7.5.0
+ * eq. for X^(0), 7.5.1, 7.5.2).  x0 [B, L_S + L_NS, d]; out [B, L'_N, d],
+ * the rows the last layer keeps. */
+ONETRANS_API onetrans_status onetrans_forward(const onetrans_model* m, const void* x0,
+                                 int32_t B, int32_t L_S, void* out, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------- plumbing --
+ * Kernel selection for tests: 0 = automatic (tensor-core kernels where the
+ * shape allows), 1 = CUDA-core kernels only.  Process-wide. */
+ONETRANS_API onetrans_status onetrans_set_kernel_policy(int32_t policy);
+/* Reads and clears the device status word that kernels set, instead of
+ * trapping, when a bounds check or a bounded wait fails (0 = no failure).
+ * Synchronizes `stream`. */
+ONETRANS_API onetrans_status onetrans_device_status(void* stream, int32_t* code);
+/* Human-readable name of a status code (static storage). */
+ONETRANS_API const char* onetrans_status_string(int32_t status);
+/* Library version as major*10000 + minor*100 + patch. */
+ONETRANS_API int32_t onetrans_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ONETRANS_H */

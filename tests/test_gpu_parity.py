@@ -1,0 +1,322 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on the same seeded
+inputs.  Tolerance: max-abs-error / RMS(oracle output) <= 2e-2 for bf16
+storage, <= 1e-4 in the float32 mode.  Integer parts (schedule, cache
+indexing, the causal predicate) are checked exactly."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from onetrans_synth import (WORKLOADS, gen_normal, linear_pyramid, random_types,
+                            tiny_raw_inputs)
+from oracle import onetrans as O
+from helpers import EPS, TOL, build, rel_err, shape, to_dev, to_np
+
+import unified_transformer_recommender_b200 as ot  # noqa: E402
+
+
+@pytest.fixture(autouse=True)
+def _policy_reset():
+    yield
+    ot.onetrans_set_kernel_policy(0)
+    assert ot.onetrans_device_status() == 0
+
+
+def tdt(dtype):
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+def run_forward(b, X0):
+    m = b.model
+    L_S = X0.shape[1] - b.shape.L_NS
+    sched = m.schedule(L_S)
+    out = torch.empty(X0.shape[0], sched[-1], b.shape.d, dtype=tdt(b.dtype), device="cuda")
+    ws = m.workspace(ot.OP_FORWARD, X0.shape[0], L_S)
+    ot.onetrans_forward(m, to_dev(X0, tdt(b.dtype)), out, ws)
+    torch.cuda.synchronize()
+    return to_np(out)
+
+
+def run_stage12(b, S, NS_tok, offsets, slots=None):
+    """S: [U, L_S, d]; NS_tok: [L_NS, C, d]; returns (cache obj, ns_out)."""
+    m = b.model
+    U, L_S, d = S.shape
+    slots = list(range(U)) if slots is None else slots
+    cache = ot.Cache(m, max(slots) + 1, L_S + 64)
+    ws1 = m.workspace(ot.OP_STAGE1, U, L_S)
+    ot.onetrans_stage1_encode(m, cache, slots, to_dev(S, tdt(b.dtype)), ws1)
+    C = NS_tok.shape[1]
+    out = torch.empty(b.shape.L_NS, C, d, dtype=tdt(b.dtype), device="cuda")
+    ws2 = m.workspace(ot.OP_STAGE2, C, L_S)
+    ot.onetrans_stage2_score(m, cache, slots, offsets, to_dev(NS_tok, tdt(b.dtype)), out, ws2)
+    torch.cuda.synchronize()
+    return cache, to_np(out)
+
+
+# ------------------------------------------------------------------ tiny --
+
+def test_tiny_fp32_end_to_end():
+    """Tiny workload: intent-order merged S (2 sequences + [SEP]), auto-split
+    NS tokens, one layer, 2 users x 3 candidates, float32 mode."""
+    wl = WORKLOADS["tiny"]
+    sh = wl.shape
+    b = build(sh, wl.seed_weights, "fp32")
+    raw = tiny_raw_inputs(wl.seed_inputs)
+    U, C = wl.users, wl.cands
+    S = np.stack([O.merge_intent_order([raw["seq0"][u], raw["seq1"][u]], b.W) for u in range(U)]).astype(np.float32)
+    feats = raw["feats"]
+    ns = torch.empty(sh.L_NS, U * C, sh.d, dtype=torch.float32, device="cuda")
+    ot.onetrans_tokenize_autosplit(b.model, to_dev(feats, torch.float32), ns,
+                                   b.model.workspace(ot.OP_AUTOSPLIT, U * C))
+    torch.cuda.synchronize()
+    ns_ref = O.autosplit(feats, b.W, sh.L_NS)                     # [N, L_NS, d]
+    assert rel_err(to_np(ns), ns_ref.transpose(1, 0, 2)) <= TOL["fp32"]
+    NS = to_np(ns)                                                 # GPU tokens feed both sides
+    X0 = np.stack([np.concatenate([S[c // C], NS[:, c]]) for c in range(U * C)])
+    got = run_forward(b, X0)
+    ref = O.forward(X0, b.W, sh.L_NS, sh.n_heads, EPS)
+    assert rel_err(got, ref) <= TOL["fp32"]
+    cache, out = run_stage12(b, S, NS, [0, C, 2 * C])
+    for c in range(U * C):
+        kv = O.stage1(S[c // C], b.W, sh.L_NS, sh.n_heads, EPS)
+        r = O.stage2(kv, NS[:, c], b.W, sh.n_heads, EPS)
+        assert rel_err(out[:, c], r) <= TOL["fp32"]
+        np.testing.assert_allclose(out[:, c], ref[c, -sh.L_NS:], rtol=0, atol=1e-4 * np.abs(ref).max())
+
+
+# ------------------------------------------------------- small, bf16/fp32 --
+
+@pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
+def test_forward_pyramid_small(dtype, policy):
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=3)
+    L_S = 290
+    sched = [302, 170, 12]
+    b = build(sh, 101, dtype, pyramid=sched)
+    X0 = gen_normal(5, (3, L_S + sh.L_NS, sh.d), dtype)
+    got = run_forward(b, X0)
+    ref = O.forward(X0, b.W, sh.L_NS, sh.n_heads, EPS, sched)
+    assert got.shape == ref.shape == (3, 12, sh.d)
+    assert rel_err(got, ref) <= TOL[dtype]
+    # the layer updates themselves (output minus the rows it started from)
+    assert rel_err(got - X0[:, -12:], ref - X0[:, -12:]) <= 10 * TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
+def test_forward_no_pyramid_keeps_all_rows(dtype, policy):
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=2)
+    b = build(sh, 102, dtype)
+    X0 = gen_normal(6, (2, 140 + sh.L_NS, sh.d), dtype)
+    got = run_forward(b, X0)
+    ref = O.forward(X0, b.W, sh.L_NS, sh.n_heads, EPS)
+    assert rel_err(got, ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
+def test_stage1_stage2_small_ragged(dtype, policy):
+    """Ragged candidate counts (including a user with none) and slots in a
+    non-identity order; cache rows read back page by page."""
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=3)
+    L_S = 275
+    sched = [287, 150, 12]
+    b = build(sh, 103, dtype, pyramid=sched)
+    U = 3
+    S = gen_normal(7, (U, L_S, sh.d), dtype)
+    counts = [2, 0, 131]
+    offs = np.concatenate([[0], np.cumsum(counts)]).tolist()
+    NS = gen_normal(8, (sh.L_NS, offs[-1], sh.d), dtype)
+    slots = [4, 0, 2]
+    cache, out = run_stage12(b, S, NS, offs, slots)
+    for u in range(U):
+        kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, sched)
+        assert cache.length(slots[u]) == L_S
+        for n, (K, V) in enumerate(kv):
+            got = to_np(cache.gather(slots[u], n, K.shape[0]))
+            assert rel_err(got[0], K) <= TOL[dtype]
+            assert rel_err(got[1], V) <= TOL[dtype]
+        for c in range(offs[u], offs[u + 1]):
+            r = O.stage2(kv, NS[:, c], b.W, sh.n_heads, EPS)
+            assert rel_err(out[:, c], r) <= TOL[dtype], (u, c)
+
+
+@pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
+def test_append_small_crosses_page_boundary(dtype, policy):
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=2)
+    b = build(sh, 104, dtype, event_dim=64)
+    U, L_S, dL = 2, 60, 7
+    S = gen_normal(9, (U, L_S, sh.d), dtype)
+    ev = gen_normal(10, (U, dL, 64), dtype)
+    ty = random_types(11, (U, dL), 3)
+    m = b.model
+    cache = ot.Cache(m, U, 128)
+    ot.onetrans_stage1_encode(m, cache, [1, 0], to_dev(S, tdt(dtype)), m.workspace(ot.OP_STAGE1, U, L_S))
+    ot.onetrans_cache_append(m, cache, [1, 0], to_dev(ev, tdt(dtype)),
+                             torch.from_numpy(ty).cuda(), m.workspace(ot.OP_APPEND, U, dL))
+    torch.cuda.synchronize()
+    NS = gen_normal(12, (sh.L_NS, 4, sh.d), dtype)
+    out = torch.empty(sh.L_NS, 4, sh.d, dtype=tdt(dtype), device="cuda")
+    ot.onetrans_stage2_score(m, cache, [1, 0], [0, 2, 4], to_dev(NS, tdt(dtype)), out,
+                             m.workspace(ot.OP_STAGE2, 4, L_S + dL))
+    torch.cuda.synchronize()
+    out = to_np(out)
+    for u, slot in enumerate([1, 0]):
+        assert cache.length(slot) == L_S + dL
+        new = O.tokenize_events(ev[u], ty[u], b.W)
+        kv = O.append(O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS), new, b.W, sh.n_heads, EPS)
+        for n, (K, V) in enumerate(kv):
+            got = to_np(cache.gather(slot, n, L_S + dL))
+            assert rel_err(got[0], K) <= TOL[dtype]
+            assert rel_err(got[1], V) <= TOL[dtype]
+        for c in range(2 * u, 2 * u + 2):
+            r = O.stage2(kv, NS[:, c], b.W, sh.n_heads, EPS)
+            assert rel_err(out[:, c], r) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
+def test_autosplit_ragged_rows(dtype, policy):
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=1)
+    b = build(sh, 105, dtype)
+    N = 300
+    feats = gen_normal(13, (N, sh.ns_feat), dtype)
+    ns = torch.empty(sh.L_NS, N, sh.d, dtype=tdt(dtype), device="cuda")
+    ot.onetrans_tokenize_autosplit(b.model, to_dev(feats, tdt(dtype)), ns, b.model.workspace(ot.OP_AUTOSPLIT, N))
+    torch.cuda.synchronize()
+    ref = O.autosplit(feats, b.W, sh.L_NS).transpose(1, 0, 2)
+    assert rel_err(to_np(ns), ref) <= TOL[dtype]
+
+
+# --------------------------------------------------------- exact checks --
+
+def test_causal_mask_exact_on_gpu():
+    """Perturbing NS inputs leaves every S output row bit-identical, and
+    perturbing S row t leaves rows < t bit-identical (the kernels are
+    deterministic, so any leak of a masked key shows as a bit change)."""
+    sh = shape(n_layers=2)
+    b = build(sh, 106, "bf16")
+    L_S = 150
+    X0 = gen_normal(14, (2, L_S + sh.L_NS, sh.d), "bf16")
+    base = run_forward(b, X0)
+    X1 = X0.copy()
+    X1[:, L_S:] = gen_normal(15, (2, sh.L_NS, sh.d), "bf16")
+    out1 = run_forward(b, X1)
+    np.testing.assert_array_equal(out1[:, :L_S], base[:, :L_S])
+    assert np.abs(out1[:, L_S:] - base[:, L_S:]).max() > 0
+    X2 = X0.copy()
+    X2[:, 97] += 1.0
+    out2 = run_forward(b, X2)
+    np.testing.assert_array_equal(out2[:, :97], base[:, :97])
+
+
+def test_schedule_query_and_cache_pages_exact():
+    sh = shape(n_layers=6)
+    sched = linear_pyramid(1190, 12, 6)
+    b = build(sh, 107, "bf16", pyramid=sched)
+    assert b.model.schedule(1178) == sched == [1190, 954, 719, 483, 248, 12]
+    cache = ot.Cache(b.model, 3, 1178)
+    S = gen_normal(16, (2, 1178, sh.d), "bf16")
+    ot.onetrans_stage1_encode(b.model, cache, [2, 0], to_dev(S, torch.bfloat16),
+                              b.model.workspace(ot.OP_STAGE1, 2, 1178))
+    torch.cuda.synchronize()
+    s_rows = [1178, 1178, 942, 707, 471, 236]
+    max_pages = (1178 + 63) // 64
+    table = cache.pool[: 3 * 6 * max_pages * 4].view(torch.int32).cpu().numpy().reshape(3, 6, max_pages)
+    seen = set()
+    base = cache.pool.data_ptr()
+    for slot in (2, 0):
+        for n, s in enumerate(s_rows):
+            npg = (s + 63) // 64
+            pages = table[slot, n, :npg]
+            assert (pages >= 0).all() and (table[slot, n, npg:] == -1).all()
+            seen.update(pages.tolist())
+            for t in (0, s - 1):
+                p = cache.row_ptr(slot, n, 1, 3, t) - base
+                page = pages[t // 64]
+                tb = (3 * 6 * max_pages * 4 + 255) // 256 * 256
+                assert p == tb + (page * 2 * sh.d * 64 + ((1 * 4 + 3) * 64 + t % 64) * 64) * 2
+    assert (table[1] == -1).all()
+    assert len(seen) == 2 * sum((s + 63) // 64 for s in s_rows)
+
+
+# ------------------------------------------- full-size workloads, sampled --
+
+def _full(name):
+    wl = WORKLOADS[name]
+    b = build(wl.shape, wl.seed_weights, wl.dtype, pyramid=list(wl.pyramid) if wl.pyramid else None,
+              event_dim=wl.event_dim)
+    return wl, b
+
+
+def test_kv_serving_full_size_sampled():
+    """The benchmark's workload and launch sequence: auto-split of 16 x 512
+    candidates, Stage I of 16 users x 1178, Stage II; oracle on sampled users
+    and candidates."""
+    wl, b = _full("kv_serving")
+    sh, U, C = wl.shape, wl.users, wl.cands
+    S = gen_normal(wl.seed_inputs, (U, wl.L_S, sh.d), "bf16")
+    feats = gen_normal(wl.seed_inputs + 100, (U * C, sh.ns_feat), "bf16")
+    m = b.model
+    ns = torch.empty(sh.L_NS, U * C, sh.d, dtype=torch.bfloat16, device="cuda")
+    ot.onetrans_tokenize_autosplit(m, to_dev(feats, torch.bfloat16), ns, m.workspace(ot.OP_AUTOSPLIT, U * C))
+    torch.cuda.synchronize()
+    NS = to_np(ns)
+    for c in (0, U * C - 1):
+        assert rel_err(NS[:, c], O.autosplit(feats[c:c + 1], b.W, sh.L_NS)[0]) <= TOL["bf16"]
+    cache, out = run_stage12(b, S, NS, [u * C for u in range(U + 1)])
+    for u in (0, U - 1):
+        kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, wl.pyramid)
+        for c in (u * C, u * C + 317, u * C + C - 1):
+            r = O.stage2(kv, NS[:, c], b.W, sh.n_heads, EPS)
+            assert rel_err(out[:, c], r) <= TOL["bf16"]
+
+
+def test_s_forward_full_size_sampled():
+    wl, b = _full("s_forward")
+    sh = wl.shape
+    X0 = gen_normal(wl.seed_inputs, (wl.users, wl.L0, sh.d), "bf16")
+    got = run_forward(b, X0)
+    for u in (0, wl.users - 1):
+        ref = O.forward(X0[u:u + 1], b.W, sh.L_NS, sh.n_heads, EPS, wl.pyramid)[0]
+        assert rel_err(got[u], ref) <= TOL["bf16"]
+
+
+def test_append_full_size_sampled():
+    wl, b = _full("append")
+    sh, U, dL = wl.shape, wl.users, wl.dL
+    m = b.model
+    S = gen_normal(wl.seed_inputs, (U, wl.L_S, sh.d), "bf16")
+    ev = gen_normal(wl.seed_inputs + 200, (U, dL, wl.event_dim), "bf16")
+    ty = random_types(wl.seed_inputs + 300, (U, dL), sh.n_types)
+    cache = ot.Cache(m, U, wl.L_S + dL)
+    ot.onetrans_stage1_encode(m, cache, list(range(U)), to_dev(S, torch.bfloat16),
+                              m.workspace(ot.OP_STAGE1, U, wl.L_S))
+    ot.onetrans_cache_append(m, cache, list(range(U)), to_dev(ev, torch.bfloat16),
+                             torch.from_numpy(ty).cuda(), m.workspace(ot.OP_APPEND, U, dL))
+    C = wl.cands
+    NS = gen_normal(wl.seed_inputs + 400, (sh.L_NS, U * C, sh.d), "bf16")
+    out = torch.empty(sh.L_NS, U * C, sh.d, dtype=torch.bfloat16, device="cuda")
+    ot.onetrans_stage2_score(m, cache, list(range(U)), [u * C for u in range(U + 1)],
+                             to_dev(NS, torch.bfloat16), out, m.workspace(ot.OP_STAGE2, U * C, wl.L_S + dL))
+    torch.cuda.synchronize()
+    out = to_np(out)
+    u = U - 1
+    kv = O.append(O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS),
+                  O.tokenize_events(ev[u], ty[u], b.W), b.W, sh.n_heads, EPS)
+    got = to_np(cache.gather(u, 5, wl.L_S + dL))
+    assert rel_err(got[0], kv[5][0]) <= TOL["bf16"]
+    for c in (u * C, u * C + C - 1):
+        assert rel_err(out[:, c], O.stage2(kv, NS[:, c], b.W, sh.n_heads, EPS)) <= TOL["bf16"]
+
+
+def test_l_forward_full_size_sampled():
+    wl, b = _full("l_forward")
+    sh = wl.shape
+    X0 = gen_normal(wl.seed_inputs, (wl.users, wl.L0, sh.d), "bf16")
+    got = run_forward(b, X0)
+    u = wl.users - 1
+    ref = O.forward(X0[u:u + 1], b.W, sh.L_NS, sh.n_heads, EPS, wl.pyramid)[0]
+    assert rel_err(got[u], ref) <= TOL["bf16"]

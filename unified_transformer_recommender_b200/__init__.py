@@ -1,0 +1,305 @@
+"""Python binding of the OneTrans B200 library (ctypes over include/onetrans.h).
+
+Argument marshalling only: every step of the path runs in the CUDA library
+`libonetrans.so` built in this directory.  PyTorch supplies device memory and
+streams.  Importing this package loads the library and raises if it is
+missing; there is no other implementation behind these calls.
+
+The functions carry the C names (onetrans_forward, onetrans_stage1_encode,
+...).  `Model` and `Cache` own the C handles and the pointer tables.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libonetrans.so")
+
+OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_DEVICE_CHECK = 0, -1, -2, -3, -4, -5, -6
+BF16, FP32 = 0, 1
+OP_FORWARD, OP_STAGE1, OP_STAGE2, OP_APPEND, OP_AUTOSPLIT = 0, 1, 2, 3, 4
+
+SYMBOLS = (
+    "onetrans_model_create", "onetrans_model_destroy", "onetrans_workspace_size",
+    "onetrans_schedule", "onetrans_cache_size", "onetrans_cache_init",
+    "onetrans_cache_destroy", "onetrans_cache_length", "onetrans_cache_row_ptr",
+    "onetrans_tokenize_autosplit", "onetrans_stage1_encode", "onetrans_stage2_score",
+    "onetrans_cache_append", "onetrans_forward", "onetrans_set_kernel_policy",
+    "onetrans_device_status", "onetrans_status_string", "onetrans_version",
+)
+
+
+class OneTransError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m unified_transformer_recommender_b200.build`")
+    return ctypes.CDLL(LIB_PATH)
+
+
+lib = _load()
+
+P = ctypes.c_void_p
+I32 = ctypes.c_int32
+I64 = ctypes.c_int64
+SZ = ctypes.c_size_t
+PP = ctypes.POINTER(ctypes.c_void_p)
+PI32 = ctypes.POINTER(ctypes.c_int32)
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("n_layers", I32), ("d_model", I32), ("n_heads", I32), ("d_ff", I32),
+                ("L_NS", I32), ("ns_feat_dim", I32), ("ns_hidden", I32),
+                ("n_behaviors", I32), ("event_dim", I32), ("pyramid_q", PI32),
+                ("rms_eps", ctypes.c_float), ("mode", I32), ("page_tokens", I32)]
+
+
+_WEIGHT_FIELDS = ("g_attn", "g_ffn", "Wqkv_S", "Wqkv_NS", "Wo", "W1_S", "b1_S", "W2_S",
+                  "b2_S", "W1_NS", "b1_NS", "W2_NS", "b2_NS")
+_TOK_FIELDS = ("Wa1", "ba1", "Wa2", "ba2")
+_BEH_FIELDS = ("Wb1", "bb1", "Wb2", "bb2")
+
+
+class Weights(ctypes.Structure):
+    _fields_ = ([(f, PP) for f in _WEIGHT_FIELDS] + [(f, P) for f in _TOK_FIELDS]
+                + [(f, PP) for f in _BEH_FIELDS] + [("type_emb", P)])
+
+
+def _sig(name, res, *args):
+    fn = getattr(lib, name)
+    fn.restype = res
+    fn.argtypes = list(args)
+    return fn
+
+
+_sig("onetrans_model_create", I32, ctypes.POINTER(Config), ctypes.POINTER(Weights), ctypes.POINTER(P))
+_sig("onetrans_model_destroy", I32, P)
+_sig("onetrans_workspace_size", I32, P, I32, I64, I32, ctypes.POINTER(SZ))
+_sig("onetrans_schedule", I32, P, I32, PI32)
+_sig("onetrans_cache_size", I32, P, I32, I32, ctypes.POINTER(SZ))
+_sig("onetrans_cache_init", I32, P, P, SZ, I32, I32, ctypes.POINTER(P))
+_sig("onetrans_cache_destroy", I32, P)
+_sig("onetrans_cache_length", I32, P, I32, PI32)
+_sig("onetrans_cache_row_ptr", I32, P, I32, I32, I32, I32, I32, ctypes.POINTER(P))
+_sig("onetrans_tokenize_autosplit", I32, P, P, I64, P, P, SZ, P)
+_sig("onetrans_stage1_encode", I32, P, P, PI32, I32, P, I32, P, SZ, P)
+_sig("onetrans_stage2_score", I32, P, P, PI32, I32, PI32, P, P, P, SZ, P)
+_sig("onetrans_cache_append", I32, P, P, PI32, I32, P, P, I32, P, SZ, P)
+_sig("onetrans_forward", I32, P, P, I32, I32, P, P, SZ, P)
+_sig("onetrans_set_kernel_policy", I32, I32)
+_sig("onetrans_device_status", I32, P, PI32)
+_sig("onetrans_status_string", ctypes.c_char_p, I32)
+_sig("onetrans_version", I32)
+
+
+def status_string(s: int) -> str:
+    return lib.onetrans_status_string(int(s)).decode()
+
+
+def _check(fn: str, s: int) -> None:
+    if s != OK:
+        raise OneTransError(fn, s)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _i32(vals: Sequence[int]):
+    arr = (I32 * len(vals))(*[int(v) for v in vals])
+    return arr
+
+
+def onetrans_set_kernel_policy(policy: int) -> None:
+    _check("onetrans_set_kernel_policy", lib.onetrans_set_kernel_policy(int(policy)))
+
+
+def onetrans_device_status(stream=None) -> int:
+    code = I32(0)
+    _check("onetrans_device_status", lib.onetrans_device_status(_stream(stream), ctypes.byref(code)))
+    return code.value
+
+
+class Model:
+    """Owns an onetrans_model handle.  `weights` maps the header's field names
+    to device tensors (per-layer fields: lists of tensors).  The tensors are
+    kept referenced for the model's lifetime."""
+
+    def __init__(self, *, n_layers, d_model, n_heads, d_ff, L_NS, weights: Dict,
+                 pyramid_q: Optional[Sequence[int]] = None, mode: int = BF16,
+                 ns_feat_dim: int = 0, ns_hidden: int = 0, n_behaviors: int = 0,
+                 event_dim: int = 0, rms_eps: float = 1e-6, page_tokens: int = 64):
+        self._keep = []
+        self.dtype = torch.bfloat16 if mode == BF16 else torch.float32
+        self._pyr = _i32(pyramid_q) if pyramid_q is not None else None
+        self.cfg = Config(n_layers, d_model, n_heads, d_ff, L_NS, ns_feat_dim, ns_hidden,
+                          n_behaviors, event_dim,
+                          ctypes.cast(self._pyr, PI32) if self._pyr is not None else None,
+                          rms_eps, mode, page_tokens)
+        w = Weights()
+        for f in _WEIGHT_FIELDS + _BEH_FIELDS:
+            ts = weights.get(f)
+            if ts is None:
+                continue
+            arr = (P * len(ts))(*[_ptr(self._own(t)) for t in ts])
+            self._keep.append(arr)
+            setattr(w, f, ctypes.cast(arr, PP))
+        for f in _TOK_FIELDS + ("type_emb",):
+            t = weights.get(f)
+            if t is not None:
+                setattr(w, f, _ptr(self._own(t)))
+        self._w = w
+        h = P()
+        _check("onetrans_model_create", lib.onetrans_model_create(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(h)))
+        self.handle = h
+        self.n_layers, self.d, self.L_NS = n_layers, d_model, L_NS
+
+    def _own(self, t: torch.Tensor) -> torch.Tensor:
+        if t.dtype != self.dtype or not t.is_contiguous():
+            raise ValueError("weights must be contiguous tensors of the model dtype")
+        self._keep.append(t)
+        return t
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value:
+            lib.onetrans_model_destroy(h)
+            self.handle = None
+
+    def workspace_size(self, op: int, n: int, L: int = 0) -> int:
+        out = SZ(0)
+        _check("onetrans_workspace_size", lib.onetrans_workspace_size(self.handle, op, n, L, ctypes.byref(out)))
+        return out.value
+
+    def workspace(self, op: int, n: int, L: int = 0, device="cuda") -> torch.Tensor:
+        return torch.empty(max(self.workspace_size(op, n, L), 256), dtype=torch.uint8, device=device)
+
+    def schedule(self, L_S: int):
+        out = (I32 * self.n_layers)()
+        _check("onetrans_schedule", lib.onetrans_schedule(self.handle, L_S, out))
+        return list(out)
+
+
+class Cache:
+    """Owns an onetrans_cache handle over a caller-allocated device pool."""
+
+    def __init__(self, model: Model, n_slots: int, max_L_S: int, device="cuda"):
+        size = SZ(0)
+        _check("onetrans_cache_size", lib.onetrans_cache_size(model.handle, n_slots, max_L_S, ctypes.byref(size)))
+        self.pool = torch.empty(size.value, dtype=torch.uint8, device=device)
+        h = P()
+        _check("onetrans_cache_init", lib.onetrans_cache_init(model.handle, self.pool.data_ptr(), size.value,
+                                                                n_slots, max_L_S, ctypes.byref(h)))
+        self.handle, self.model = h, model
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value:
+            lib.onetrans_cache_destroy(h)
+            self.handle = None
+
+    def length(self, slot: int) -> int:
+        out = I32(0)
+        _check("onetrans_cache_length", lib.onetrans_cache_length(self.handle, slot, ctypes.byref(out)))
+        return out.value
+
+    def row_ptr(self, slot, layer, kind, head, token) -> int:
+        out = P()
+        _check("onetrans_cache_row_ptr", lib.onetrans_cache_row_ptr(self.handle, slot, layer, kind, head, token,
+                                                                      ctypes.byref(out)))
+        return out.value
+
+    def gather(self, slot: int, layer: int, length: int) -> torch.Tensor:
+        """Cached [2, length, d] K/V rows of (slot, layer), heads concatenated,
+        read back page by page (device copies)."""
+        m = self.model
+        H = m.cfg.n_heads
+        dh = m.d // H
+        es = 2 if m.dtype == torch.bfloat16 else 4
+        out = torch.empty(2, length, m.d, dtype=m.dtype, device=self.pool.device)
+        base = self.pool.data_ptr()
+        for kind in range(2):
+            for h in range(H):
+                for t0 in range(0, length, m.cfg.page_tokens):
+                    n = min(m.cfg.page_tokens, length - t0)
+                    off = self.row_ptr(slot, layer, kind, h, t0) - base
+                    src = self.pool[off: off + n * dh * es].view(m.dtype).view(n, dh)
+                    out[kind, t0:t0 + n, h * dh:(h + 1) * dh] = src
+        return out
+
+
+# ------------------------------------------------------------- entry points
+
+def onetrans_tokenize_autosplit(model: Model, feats: torch.Tensor, ns_tokens: torch.Tensor,
+                                ws: torch.Tensor, stream=None) -> None:
+    _check("onetrans_tokenize_autosplit", lib.onetrans_tokenize_autosplit(
+        model.handle, _ptr(feats), feats.shape[0], _ptr(ns_tokens), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def onetrans_stage1_encode(model: Model, cache: Cache, slots: Sequence[int], s_tokens: torch.Tensor,
+                           ws: torch.Tensor, stream=None) -> None:
+    sl = _i32(slots)
+    _check("onetrans_stage1_encode", lib.onetrans_stage1_encode(
+        model.handle, cache.handle, sl, len(slots), _ptr(s_tokens), s_tokens.shape[1], _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def onetrans_stage2_score(model: Model, cache: Cache, slots: Sequence[int], cand_offsets: Sequence[int],
+                          ns_tokens: torch.Tensor, ns_out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    sl, co = _i32(slots), _i32(cand_offsets)
+    _check("onetrans_stage2_score", lib.onetrans_stage2_score(
+        model.handle, cache.handle, sl, len(slots), co, _ptr(ns_tokens), _ptr(ns_out), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def onetrans_cache_append(model: Model, cache: Cache, slots: Sequence[int], events: torch.Tensor,
+                          types: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    sl = _i32(slots)
+    _check("onetrans_cache_append", lib.onetrans_cache_append(
+        model.handle, cache.handle, sl, len(slots), _ptr(events), _ptr(types), events.shape[1], _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def onetrans_forward(model: Model, x0: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    _check("onetrans_forward", lib.onetrans_forward(
+        model.handle, _ptr(x0), x0.shape[0], x0.shape[1] - model.L_NS, _ptr(out), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def model_from_arrays(shape, weights: Dict, pyramid_q=None, mode: int = BF16, device="cuda",
+                      event_dim: int = 0) -> Model:
+    """Copy a dict of NumPy weight arrays (the layout of onetrans.h) to the
+    device and create a Model.  `shape` provides n_layers, d, n_heads, d_ff,
+    L_NS, ns_feat, ns_hidden, n_types and eps."""
+    import numpy as np
+    dt = torch.bfloat16 if mode == BF16 else torch.float32
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device=device, dtype=dt)
+
+    tw = {}
+    for k, v in weights.items():
+        if k == "sep":
+            continue
+        tw[k] = [dev(a) for a in v] if isinstance(v, list) else dev(v)
+    n_beh = len(weights.get("Wb1", [])) if event_dim else 0
+    return Model(n_layers=shape.n_layers, d_model=shape.d, n_heads=shape.n_heads, d_ff=shape.d_ff,
+                 L_NS=shape.L_NS, weights=tw, pyramid_q=pyramid_q, mode=mode,
+                 ns_feat_dim=shape.ns_feat, ns_hidden=shape.ns_hidden, n_behaviors=n_beh,
+                 event_dim=event_dim, rms_eps=shape.eps)

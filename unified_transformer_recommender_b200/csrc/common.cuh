@@ -1,0 +1,114 @@
+// Shared descriptors of the OneTrans CUDA library (host and device).
+//
+// Every activation row of the block stack is identified by (b, t): b is the
+// batch index (sample, user or candidate) and t the row within it.  A GEMM
+// tiles one of the two coordinates by 128 rows and fixes the other per CTA:
+//   TILE_ROWS    tiled m = t, fixed g = b      (S rows of one sample/user)
+//   TILE_SAMPLES tiled m = b, fixed g = t      (one NS token across samples;
+//                                               weight group = t - grp_base)
+//   TILE_FLAT    tiled m = b * fold + t        (rows contiguous across users)
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace ot {
+
+enum TileMode : int { TILE_ROWS = 0, TILE_SAMPLES = 1, TILE_FLAT = 2 };
+enum OutKind : int { OUT_ROWS = 0, OUT_KV = 1 };
+enum Act : int { ACT_NONE = 0, ACT_GELU = 1 };
+
+// Address of element (b, t, n) = base + b*sb + t*st + (n / split)*sc + n % split
+// (in elements).  `split` lets one GEMM write column blocks to separate
+// planes (the token-major output of the auto-split tokenizer).
+struct RowMap {
+  void* base;
+  long long sb, st, sc;
+  int split;
+};
+
+// Paged K/V store.  A page holds P tokens of one (sequence, layer) laid out as
+// [kind 0=K,1=V][head][token][d_h].  The page of token `pos` of batch row b is
+//   table ? table[row_off[b] + pos / P] : b * pps + pos / P.
+struct KVStore {
+  void* pool;
+  const int* table;
+  const int* row_off;
+  int P, H, dh, pps;
+  int pos_off;  // written position = t + pos_off
+};
+
+struct GemmDesc {
+  int mode, M, m_lo, G, g_lo, fold;
+  int N, K, n_lo, grp_base;
+  // A element (m, g, k) = A + m*a_sm + g*a_sg + k; extents for the TMA map
+  const void* A;
+  long long a_sm, a_sg, a_mext, a_gext;
+  // W element (grp, n, k) = W + grp*w_sg + (n_lo + n)*K + k
+  const void* W;
+  long long w_sg;
+  int w_rows, w_groups;
+  const void* bias;  // bias[grp*bias_sg + n_lo + n], or null
+  long long bias_sg;
+  int act;
+  int out_kind;
+  RowMap out;
+  RowMap res;    // residual added after bias/activation (base null = none)
+  RowMap rms;    // RMSNorm of the stored output row (base null = none)
+  const void* gamma;
+  float eps;
+  KVStore kv;
+};
+
+struct AttnDesc {
+  int B, H, dh, Lq, q_pos0;  // query t of batch b sits at key position q_pos0 + t
+  RowMap q, o;                // columns: head h occupies [h*dh, (h+1)*dh)
+  KVStore kv;
+  float scale;
+};
+
+// Stage II attention: candidates of one user share the user's cached S keys.
+struct Stage2Desc {
+  int H, dh, L_NS, C_tot, s_len;
+  const int* tiles;    // n_tiles x {user, c0, c1}
+  const void* qkv;     // [L_NS, C_tot, 3d] token-major Q|K|V of the NS rows
+  void* o;             // [L_NS, C_tot, d]
+  KVStore kv;          // row_off indexed by user
+  float scale;
+};
+
+__host__ __device__ inline void row_of(const GemmDesc& d, int m, int g, int& b, int& t) {
+  if (d.mode == TILE_ROWS) { t = m; b = g; }
+  else if (d.mode == TILE_SAMPLES) { b = m; t = g; }
+  else { b = m / d.fold; t = m - b * d.fold; }
+}
+
+__host__ __device__ inline long long rm_off(const RowMap& r, int b, int t, int n) {
+  return (long long)b * r.sb + (long long)t * r.st + (long long)(n / r.split) * r.sc + (n % r.split);
+}
+
+__host__ __device__ inline long long kv_off(const KVStore& kv, int b, int pos, int kind, int head, int e) {
+  int page = kv.table ? kv.table[kv.row_off[b] + pos / kv.P] : b * kv.pps + pos / kv.P;
+  return (long long)page * (2LL * kv.H * kv.P * kv.dh) +
+         ((long long)(kind * kv.H + head) * kv.P + (pos % kv.P)) * kv.dh + e;
+}
+
+template <typename T> __device__ inline float to_f(T v);
+template <> __device__ inline float to_f<float>(float v) { return v; }
+template <> __device__ inline float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ inline T from_f(float v);
+template <> __device__ inline float from_f<float>(float v) { return v; }
+template <> __device__ inline __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// GELU, tanh form (Hendrycks & Gimpel): 0.5 x (1 + tanh(sqrt(2/pi)(x + 0.044715 x^3)))
+__device__ inline float gelu_tanh(float x) {
+  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
+  return 0.5f * x * (1.0f + tanhf(k0 * (x + k1 * x * x * x)));
+}
+
+// Device status word: kernels that detect a bounds or wait failure record a
+// code here instead of trapping; the host reads and clears it.
+__device__ int g_device_status = 0;  // one translation unit holds every kernel
+__device__ inline void flag_error(int code) { atomicCAS(&g_device_status, 0, code); }
+
+}  // namespace ot

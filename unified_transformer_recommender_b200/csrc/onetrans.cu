@@ -1,0 +1,958 @@
+// Host side of the OneTrans C ABI: validation, schedules, workspace carving,
+// paged-cache bookkeeping and the launch sequence of every entry point.
+// All kernels live in this one translation unit (see the included headers).
+#include "onetrans.h"
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "simt.cuh"
+#include "gemm_tc.cuh"
+#include "attn_tc.cuh"
+
+using namespace ot;
+
+// ============================================================== model ====
+struct onetrans_model {
+  onetrans_config cfg;
+  std::vector<int> pyr;
+  int d, H, dh, dff, L_NS, NL, es;
+  bool bf16;
+  std::vector<const void*> g_attn, g_ffn, Wqkv_S, Wqkv_NS, Wo, W1_S, b1_S, W2_S, b2_S, W1_NS,
+      b1_NS, W2_NS, b2_NS, Wb1, bb1, Wb2, bb2;
+  const void *Wa1, *ba1, *Wa2, *ba2, *type_emb;
+};
+
+struct onetrans_cache {
+  const onetrans_model* m;
+  char* pool;
+  size_t bytes;
+  int n_slots, max_L_S, max_pages, n_pages;
+  int* d_table;
+  char* d_pages;
+  std::vector<int> h_table;  // [slot][layer][max_pages], -1 = unassigned
+  std::vector<int> len;      // cached S length per slot
+  std::vector<int> free_pages;
+};
+
+static int g_policy = 0;
+static const int kMaxUsers = 65536;  // users per Stage II call (workspace holds their table rows)
+
+#define OT_TRY(x)                                  \
+  do {                                             \
+    onetrans_status _s = (x);                      \
+    if (_s != ONETRANS_OK) return _s;              \
+  } while (0)
+
+static onetrans_status cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return ONETRANS_OK;
+  return ONETRANS_ERR_CUDA;
+}
+static onetrans_status last_launch() { return cuda_ok(cudaGetLastError()); }
+
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+static long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+// Query count of each layer for an input of L_S S rows.
+static onetrans_status schedule_of(const onetrans_model* m, int L_S, std::vector<int>& Lq) {
+  if (L_S < 0) return ONETRANS_ERR_SHAPE;
+  Lq.assign(m->NL, 0);
+  int L = L_S + m->L_NS;
+  for (int n = 0; n < m->NL; ++n) {
+    int q = m->pyr.empty() ? L : m->pyr[n];
+    if (q < m->L_NS || q > L) return ONETRANS_ERR_SHAPE;
+    Lq[n] = q;
+    L = q;
+  }
+  return ONETRANS_OK;
+}
+
+// S rows per layer (s_n) and S rows among the queries (s'_n) for Stage I.
+static onetrans_status s_rows_of(const onetrans_model* m, int L_S, std::vector<int>& s,
+                                 std::vector<int>& sq) {
+  std::vector<int> Lq;
+  OT_TRY(schedule_of(m, L_S, Lq));
+  s.assign(m->NL, 0);
+  sq.assign(m->NL, 0);
+  int cur = L_S;
+  for (int n = 0; n < m->NL; ++n) {
+    s[n] = cur;
+    sq[n] = Lq[n] - m->L_NS;
+    cur = sq[n];
+  }
+  return ONETRANS_OK;
+}
+
+// Bump allocator over the caller's workspace; with base == null it only sizes.
+struct Carve {
+  char* base;
+  size_t cap, used = 0;
+  bool overflow = false;
+  Carve(void* b, size_t c) : base((char*)b), cap(c) {}
+  void* take(size_t bytes) {
+    used = (used + 255) & ~(size_t)255;
+    void* p = base ? base + used : nullptr;
+    used += bytes;
+    if (base && used > cap) overflow = true;
+    return p;
+  }
+};
+
+static RowMap rmap(const void* base, long long sb, long long st) {
+  RowMap r;
+  r.base = (void*)base;
+  r.sb = sb;
+  r.st = st;
+  r.sc = 0;
+  r.split = 1 << 30;
+  return r;
+}
+
+// Element pointer with an element offset (may be negative relative to a
+// buffer start only when every address the map produces stays in bounds).
+static void* eoff(const void* p, long long elems, int es) { return (char*)p + elems * es; }
+
+static GemmDesc gdesc_base(const onetrans_model* m) {
+  GemmDesc d;
+  std::memset(&d, 0, sizeof(d));
+  d.eps = m->cfg.rms_eps;
+  d.w_groups = 1;
+  d.fold = 1 << 30;
+  return d;
+}
+
+// ============================================================= launches ==
+template <typename T>
+static onetrans_status launch_rms(GemmDesc d, cudaStream_t st) {
+  if (d.M <= 0 || d.G <= 0) return ONETRANS_OK;
+  dim3 grid((unsigned)cdiv(d.M, 8), (unsigned)d.G);
+  rms_rows_kernel<T><<<grid, 256, 0, st>>>(d);
+  return last_launch();
+}
+
+template <typename T>
+static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, cudaStream_t st) {
+  if (d.M <= 0 || d.G <= 0 || d.N <= 0) return ONETRANS_OK;
+  if (cdiv(d.M, 64) > 65535 || d.G > 65535) return ONETRANS_ERR_SHAPE;
+  if (m->bf16 && g_policy == 0 && tc_gemm_supported(d)) {
+    return tc_gemm_launch(d, st);
+  }
+  dim3 grid((unsigned)cdiv(d.N, 64), (unsigned)cdiv(d.M, 64), (unsigned)d.G);
+  gemm_simt_kernel<T><<<grid, 256, 0, st>>>(d);
+  OT_TRY(last_launch());
+  if (d.rms.base) OT_TRY(launch_rms<T>(d, st));
+  return ONETRANS_OK;
+}
+
+template <typename T>
+static onetrans_status launch_attn(const onetrans_model* m, const AttnDesc& a, cudaStream_t st) {
+  if (a.Lq <= 0 || a.B <= 0) return ONETRANS_OK;
+  if (m->bf16 && g_policy == 0 && tc_attn_supported(a)) return tc_attn_launch(a, st);
+  dim3 grid((unsigned)cdiv(a.Lq, 64), (unsigned)a.H, (unsigned)a.B);
+  switch (a.dh) {
+    case 32: attn_simt_kernel<T, 32><<<grid, 64, 0, st>>>(a); break;
+    case 64: attn_simt_kernel<T, 64><<<grid, 64, 0, st>>>(a); break;
+    case 96: attn_simt_kernel<T, 96><<<grid, 64, 0, st>>>(a); break;
+    case 128: attn_simt_kernel<T, 128><<<grid, 64, 0, st>>>(a); break;
+    default: return ONETRANS_ERR_UNSUPPORTED;
+  }
+  return last_launch();
+}
+
+template <typename T>
+static onetrans_status launch_stage2_attn(const onetrans_model* m, const Stage2Desc& a, int n_tiles,
+                                          cudaStream_t st) {
+  if (n_tiles <= 0) return ONETRANS_OK;
+  dim3 grid((unsigned)n_tiles, (unsigned)a.H, (unsigned)a.L_NS);
+  switch (a.dh) {
+    case 32: stage2_attn_simt_kernel<T, 32><<<grid, 64, 0, st>>>(a); break;
+    case 64: stage2_attn_simt_kernel<T, 64><<<grid, 64, 0, st>>>(a); break;
+    case 96: stage2_attn_simt_kernel<T, 96><<<grid, 64, 0, st>>>(a); break;
+    case 128: stage2_attn_simt_kernel<T, 128><<<grid, 64, 0, st>>>(a); break;
+    default: return ONETRANS_ERR_UNSUPPORTED;
+  }
+  return last_launch();
+}
+
+// RMSNorm of `rows` contiguous rows of width d: dst = RMS(src) * gamma.
+template <typename T>
+static onetrans_status rms_flat(const onetrans_model* m, const void* src, void* dst, long long rows,
+                                const void* gamma, cudaStream_t st) {
+  GemmDesc d = gdesc_base(m);
+  d.mode = TILE_FLAT;
+  d.M = (int)rows;
+  d.G = 1;
+  d.N = m->d;
+  d.out = rmap(src, 0, m->d);
+  d.rms = rmap(dst, 0, m->d);
+  d.gamma = gamma;
+  return launch_rms<T>(d, st);
+}
+
+// ================================================================ forward =
+template <typename T>
+static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int B, int L_S, void* out,
+                                    void* ws, size_t ws_bytes, cudaStream_t st, size_t* need) {
+  std::vector<int> Lq;
+  OT_TRY(schedule_of(m, L_S, Lq));
+  const int d = m->d, dff = m->dff, L_NS = m->L_NS, es = m->es, P = m->cfg.page_tokens;
+  const int L0 = L_S + L_NS, Lq1 = Lq[0];
+  const long long pps = cdiv(L0, P);
+  Carve cv(ws, ws_bytes);
+  void* xa = cv.take((size_t)B * Lq1 * d * es);
+  void* xb = cv.take((size_t)B * Lq1 * d * es);
+  void* h = cv.take((size_t)B * L0 * d * es);
+  void* q = cv.take((size_t)B * Lq1 * d * es);
+  void* at = cv.take((size_t)B * Lq1 * d * es);
+  void* xm = cv.take((size_t)B * Lq1 * d * es);
+  void* h2 = cv.take((size_t)B * Lq1 * d * es);
+  void* hid = cv.take((size_t)B * Lq1 * dff * es);
+  void* kvb = cv.take((size_t)B * pps * 2 * d * P * es);
+  if (need) { *need = cv.used; return ONETRANS_OK; }
+  if (cv.overflow) return ONETRANS_ERR_CAPACITY;
+
+  KVStore kv;
+  std::memset(&kv, 0, sizeof(kv));
+  kv.pool = kvb; kv.P = P; kv.H = m->H; kv.dh = m->dh; kv.pps = (int)pps;
+
+  OT_TRY(rms_flat<T>(m, x0, h, (long long)B * L0, m->g_attn[0], st));
+  const void* x_in = x0;
+  int L = L0;
+  for (int n = 0; n < m->NL; ++n) {
+    const int s = L - L_NS, Lqn = Lq[n], sq = Lqn - L_NS, off = L - Lqn;
+    const bool last = n + 1 == m->NL;
+    void* x_next = last ? out : (n % 2 == 0 ? xa : xb);
+    // -- S rows: K,V of all S rows; Q of the tail S rows
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_ROWS; g.M = s; g.m_lo = 0; g.G = B; g.g_lo = 0;
+    g.K = d; g.A = h; g.a_sm = d; g.a_sg = (long long)L * d; g.a_mext = L; g.a_gext = B;
+    g.W = m->Wqkv_S[n]; g.w_rows = 3 * d; g.n_lo = d; g.N = 2 * d;
+    g.out_kind = OUT_KV; g.kv = kv;
+    OT_TRY(launch_gemm<T>(m, g, st));
+    if (sq > 0) {
+      g.m_lo = s - sq; g.M = sq; g.n_lo = 0; g.N = d; g.out_kind = OUT_ROWS;
+      g.out = rmap(eoff(q, -(long long)off * d, es), (long long)Lqn * d, d);
+      OT_TRY(launch_gemm<T>(m, g, st));
+    }
+    // -- NS rows: token j uses its own weights; tile across samples
+    GemmDesc gn = gdesc_base(m);
+    gn.mode = TILE_SAMPLES; gn.M = B; gn.m_lo = 0; gn.G = L_NS; gn.g_lo = s; gn.grp_base = s;
+    gn.K = d; gn.A = h; gn.a_sm = (long long)L * d; gn.a_sg = d; gn.a_mext = B; gn.a_gext = L;
+    gn.W = m->Wqkv_NS[n]; gn.w_sg = 3LL * d * d; gn.w_rows = 3 * d; gn.w_groups = L_NS;
+    gn.n_lo = 0; gn.N = d; gn.out_kind = OUT_ROWS;
+    gn.out = rmap(eoff(q, -(long long)off * d, es), (long long)Lqn * d, d);
+    OT_TRY(launch_gemm<T>(m, gn, st));
+    gn.n_lo = d; gn.N = 2 * d; gn.out_kind = OUT_KV; gn.kv = kv;
+    OT_TRY(launch_gemm<T>(m, gn, st));
+    // -- attention of the Lqn tail queries over keys 0..p
+    AttnDesc a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = B; a.H = m->H; a.dh = m->dh; a.Lq = Lqn; a.q_pos0 = off;
+    a.q = rmap(q, (long long)Lqn * d, d);
+    a.o = rmap(at, (long long)Lqn * d, d);
+    a.kv = kv; a.scale = 1.0f / std::sqrt((float)m->dh);
+    OT_TRY(launch_attn<T>(m, a, st));
+    // -- W^O + residual, then RMSNorm for the FFN (all tail rows share W^O)
+    GemmDesc go = gdesc_base(m);
+    go.mode = TILE_FLAT; go.M = B * Lqn; go.fold = Lqn; go.G = 1;
+    go.K = d; go.A = at; go.a_sm = d; go.a_mext = (long long)B * Lqn; go.a_gext = 1;
+    go.W = m->Wo[n]; go.w_rows = d; go.N = d;
+    go.res = rmap(eoff(x_in, (long long)off * d, es), (long long)L * d, d);
+    go.out = rmap(xm, (long long)Lqn * d, d);
+    go.rms = rmap(h2, (long long)Lqn * d, d);
+    go.gamma = m->g_ffn[n];
+    OT_TRY(launch_gemm<T>(m, go, st));
+    // -- mixed FFN: S tail rows shared, NS rows per token
+    for (int part = 0; part < 2; ++part) {
+      GemmDesc f = gdesc_base(m);
+      if (part == 0) {
+        if (sq <= 0) continue;
+        f.mode = TILE_ROWS; f.M = sq; f.G = B; f.a_sm = d; f.a_sg = (long long)Lqn * d;
+        f.a_mext = Lqn; f.a_gext = B;
+      } else {
+        f.mode = TILE_SAMPLES; f.M = B; f.G = L_NS; f.g_lo = sq; f.grp_base = sq;
+        f.a_sm = (long long)Lqn * d; f.a_sg = d; f.a_mext = B; f.a_gext = Lqn;
+      }
+      f.K = d; f.A = h2;
+      f.W = part ? m->W1_NS[n] : m->W1_S[n]; f.w_rows = dff; f.N = dff;
+      f.w_sg = part ? (long long)dff * d : 0; f.w_groups = part ? L_NS : 1;
+      f.bias = part ? m->b1_NS[n] : m->b1_S[n]; f.bias_sg = part ? dff : 0;
+      f.act = ACT_GELU;
+      f.out = rmap(hid, (long long)Lqn * dff, dff);
+      OT_TRY(launch_gemm<T>(m, f, st));
+      GemmDesc f2 = f;
+      f2.K = dff; f2.A = hid; f2.act = ACT_NONE;
+      if (part == 0) { f2.a_sm = dff; f2.a_sg = (long long)Lqn * dff; }
+      else { f2.a_sm = (long long)Lqn * dff; f2.a_sg = dff; }
+      f2.W = part ? m->W2_NS[n] : m->W2_S[n]; f2.w_rows = d; f2.N = d;
+      f2.w_sg = part ? (long long)d * dff : 0;
+      f2.bias = part ? m->b2_NS[n] : m->b2_S[n]; f2.bias_sg = part ? d : 0;
+      f2.res = rmap(xm, (long long)Lqn * d, d);
+      f2.out = rmap(x_next, (long long)Lqn * d, d);
+      if (!last) { f2.rms = rmap(h, (long long)Lqn * d, d); f2.gamma = m->g_attn[n + 1]; }
+      OT_TRY(launch_gemm<T>(m, f2, st));
+    }
+    x_in = x_next;
+    L = Lqn;
+  }
+  return ONETRANS_OK;
+}
+
+// ============================================================== stage I ==
+static void kv_for_cache(const onetrans_cache* c, int layer, const int* d_row_off, KVStore& kv) {
+  std::memset(&kv, 0, sizeof(kv));
+  kv.pool = c->d_pages;
+  kv.table = c->d_table + (size_t)layer * c->max_pages;
+  kv.row_off = d_row_off;
+  kv.P = c->m->cfg.page_tokens;
+  kv.H = c->m->H;
+  kv.dh = c->m->dh;
+}
+
+static onetrans_status upload_slot_table(onetrans_cache* c, int slot, cudaStream_t st) {
+  const size_t row = (size_t)c->m->NL * c->max_pages;
+  return cuda_ok(cudaMemcpyAsync(c->d_table + slot * row, c->h_table.data() + slot * row,
+                                 row * sizeof(int), cudaMemcpyHostToDevice, st));
+}
+
+template <typename T>
+static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, const int* slots, int U,
+                                   const void* s_tok, int L_S, void* ws, size_t ws_bytes,
+                                   cudaStream_t st, size_t* need) {
+  std::vector<int> s, sq;
+  OT_TRY(s_rows_of(m, L_S, s, sq));
+  const int d = m->d, dff = m->dff, es = m->es;
+  const int sq1 = std::max(sq[0], 0);
+  Carve cv(ws, ws_bytes);
+  void* xa = cv.take((size_t)U * sq1 * d * es);
+  void* xb = cv.take((size_t)U * sq1 * d * es);
+  void* h = cv.take((size_t)U * L_S * d * es);
+  void* q = cv.take((size_t)U * sq1 * d * es);
+  void* at = cv.take((size_t)U * sq1 * d * es);
+  void* xm = cv.take((size_t)U * sq1 * d * es);
+  void* h2 = cv.take((size_t)U * sq1 * d * es);
+  void* hid = cv.take((size_t)U * sq1 * dff * es);
+  int* row_off = (int*)cv.take((size_t)U * sizeof(int));
+  if (need) { *need = cv.used; return ONETRANS_OK; }
+  if (cv.overflow) return ONETRANS_ERR_CAPACITY;
+  if (L_S > c->max_L_S) return ONETRANS_ERR_CAPACITY;
+
+  // page assignment on the host: release the slots' pages, take new ones
+  const int P = m->cfg.page_tokens;
+  long long needed = 0, owned = 0;
+  for (int u = 0; u < U; ++u) {
+    for (int n = 0; n < m->NL; ++n) needed += cdiv(s[n], P);
+    const size_t row = (size_t)slots[u] * m->NL * c->max_pages;
+    for (size_t i = 0; i < (size_t)m->NL * c->max_pages; ++i) owned += c->h_table[row + i] >= 0;
+  }
+  if (needed > (long long)c->free_pages.size() + owned) return ONETRANS_ERR_CAPACITY;
+  std::vector<int> h_row_off(U);
+  for (int u = 0; u < U; ++u) {
+    const size_t row = (size_t)slots[u] * m->NL * c->max_pages;
+    for (size_t i = 0; i < (size_t)m->NL * c->max_pages; ++i) {
+      if (c->h_table[row + i] >= 0) c->free_pages.push_back(c->h_table[row + i]);
+      c->h_table[row + i] = -1;
+    }
+    for (int n = 0; n < m->NL; ++n)
+      for (long long p = 0; p < cdiv(s[n], P); ++p) {
+        c->h_table[row + (size_t)n * c->max_pages + p] = c->free_pages.back();
+        c->free_pages.pop_back();
+      }
+    c->len[slots[u]] = L_S;
+    h_row_off[u] = (int)row;
+    OT_TRY(upload_slot_table(c, slots[u], st));
+  }
+  OT_TRY(cuda_ok(cudaMemcpyAsync(row_off, h_row_off.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
+
+  OT_TRY(rms_flat<T>(m, s_tok, h, (long long)U * L_S, m->g_attn[0], st));
+  const void* x_in = s_tok;
+  for (int n = 0; n < m->NL; ++n) {
+    const int sn = s[n], sqn = sq[n];
+    if (sn <= 0) break;
+    KVStore kv;
+    kv_for_cache(c, n, row_off, kv);
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_FLAT; g.M = U * sn; g.fold = sn; g.G = 1;
+    g.K = d; g.A = h; g.a_sm = d; g.a_mext = (long long)U * sn; g.a_gext = 1;
+    g.W = m->Wqkv_S[n]; g.w_rows = 3 * d; g.n_lo = d; g.N = 2 * d;
+    g.out_kind = OUT_KV; g.kv = kv;
+    OT_TRY(launch_gemm<T>(m, g, st));
+    // the last layer's outputs feed nothing that is cached: only its K/V are needed
+    if (sqn <= 0 || n + 1 == m->NL) break;
+    void* x_next = n % 2 == 0 ? xa : xb;
+    GemmDesc gq = gdesc_base(m);
+    gq.mode = TILE_ROWS; gq.M = sqn; gq.m_lo = sn - sqn; gq.G = U;
+    gq.K = d; gq.A = h; gq.a_sm = d; gq.a_sg = (long long)sn * d; gq.a_mext = sn; gq.a_gext = U;
+    gq.W = m->Wqkv_S[n]; gq.w_rows = 3 * d; gq.n_lo = 0; gq.N = d;
+    gq.out = rmap(eoff(q, -(long long)(sn - sqn) * d, es), (long long)sqn * d, d);
+    OT_TRY(launch_gemm<T>(m, gq, st));
+    AttnDesc a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = U; a.H = m->H; a.dh = m->dh; a.Lq = sqn; a.q_pos0 = sn - sqn;
+    a.q = rmap(q, (long long)sqn * d, d);
+    a.o = rmap(at, (long long)sqn * d, d);
+    a.kv = kv; a.scale = 1.0f / std::sqrt((float)m->dh);
+    OT_TRY(launch_attn<T>(m, a, st));
+    GemmDesc go = gdesc_base(m);
+    go.mode = TILE_FLAT; go.M = U * sqn; go.fold = sqn; go.G = 1;
+    go.K = d; go.A = at; go.a_sm = d; go.a_mext = (long long)U * sqn; go.a_gext = 1;
+    go.W = m->Wo[n]; go.w_rows = d; go.N = d;
+    go.res = rmap(eoff(x_in, (long long)(sn - sqn) * d, es), (long long)sn * d, d);
+    go.out = rmap(xm, (long long)sqn * d, d);
+    go.rms = rmap(h2, (long long)sqn * d, d);
+    go.gamma = m->g_ffn[n];
+    OT_TRY(launch_gemm<T>(m, go, st));
+    GemmDesc f = go;
+    f.res.base = nullptr; f.rms.base = nullptr; f.gamma = nullptr;
+    f.A = h2; f.W = m->W1_S[n]; f.w_rows = dff; f.N = dff; f.bias = m->b1_S[n]; f.act = ACT_GELU;
+    f.out = rmap(hid, (long long)sqn * dff, dff);
+    OT_TRY(launch_gemm<T>(m, f, st));
+    GemmDesc f2 = go;
+    f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.W = m->W2_S[n]; f2.w_rows = d; f2.N = d;
+    f2.bias = m->b2_S[n];
+    f2.res = rmap(xm, (long long)sqn * d, d);
+    f2.out = rmap(x_next, (long long)sqn * d, d);
+    f2.rms = rmap(h, (long long)sqn * d, d);
+    f2.gamma = m->g_attn[n + 1];
+    OT_TRY(launch_gemm<T>(m, f2, st));
+    x_in = x_next;
+  }
+  return ONETRANS_OK;
+}
+
+// ============================================================= stage II ==
+template <typename T>
+static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache* c, const int* slots,
+                                   int U, const int* offs, const void* ns_in, void* ns_out, void* ws,
+                                   size_t ws_bytes, cudaStream_t st, size_t* need, long long C_need,
+                                   int L_S_need) {
+  const int d = m->d, dff = m->dff, L_NS = m->L_NS, es = m->es;
+  const long long C = need ? C_need : offs[U] - offs[0];
+  const int L_S = need ? L_S_need : (U > 0 ? c->len[slots[0]] : 0);
+  std::vector<int> s, sq;
+  OT_TRY(s_rows_of(m, L_S, s, sq));
+  const int TQ = 64;
+  long long max_tiles = need ? cdiv(C, TQ) + std::min<long long>(C, kMaxUsers) : 0;
+  std::vector<int> tiles;
+  if (!need) {
+    for (int u = 0; u < U; ++u)
+      for (int c0 = offs[u]; c0 < offs[u + 1]; c0 += TQ)
+        tiles.insert(tiles.end(), {u, c0 - offs[0], std::min(c0 + TQ, offs[u + 1]) - offs[0]});
+    max_tiles = (long long)tiles.size() / 3;
+  }
+  Carve cv(ws, ws_bytes);
+  void* xa = cv.take((size_t)L_NS * C * d * es);
+  void* xb = cv.take((size_t)L_NS * C * d * es);
+  void* h = cv.take((size_t)L_NS * C * d * es);
+  void* qkv = cv.take((size_t)L_NS * C * 3 * d * es);
+  void* at = cv.take((size_t)L_NS * C * d * es);
+  void* xm = cv.take((size_t)L_NS * C * d * es);
+  void* h2 = cv.take((size_t)L_NS * C * d * es);
+  void* hid = cv.take((size_t)L_NS * C * dff * es);
+  int* row_off = (int*)cv.take((size_t)kMaxUsers * sizeof(int));
+  int* d_tiles = (int*)cv.take((size_t)std::max<long long>(max_tiles, 1) * 3 * sizeof(int));
+  if (need) { *need = cv.used; return ONETRANS_OK; }
+  if (cv.overflow) return ONETRANS_ERR_CAPACITY;
+  if (C == 0) return ONETRANS_OK;
+
+  std::vector<int> h_row_off(U);
+  for (int u = 0; u < U; ++u) h_row_off[u] = slots[u] * m->NL * c->max_pages;
+  OT_TRY(cuda_ok(cudaMemcpyAsync(row_off, h_row_off.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
+  OT_TRY(cuda_ok(cudaMemcpyAsync(d_tiles, tiles.data(), tiles.size() * sizeof(int), cudaMemcpyHostToDevice, st)));
+
+  OT_TRY(rms_flat<T>(m, ns_in, h, (long long)L_NS * C, m->g_attn[0], st));
+  const void* x_in = ns_in;
+  for (int n = 0; n < m->NL; ++n) {
+    const bool last = n + 1 == m->NL;
+    void* x_next = last ? ns_out : (n % 2 == 0 ? xa : xb);
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_SAMPLES; g.M = (int)C; g.G = L_NS; g.g_lo = 0; g.grp_base = 0;
+    g.K = d; g.A = h; g.a_sm = d; g.a_sg = C * d; g.a_mext = C; g.a_gext = L_NS;
+    g.W = m->Wqkv_NS[n]; g.w_sg = 3LL * d * d; g.w_rows = 3 * d; g.w_groups = L_NS;
+    g.n_lo = 0; g.N = 3 * d;
+    g.out = rmap(qkv, 3LL * d, C * 3 * d);
+    OT_TRY(launch_gemm<T>(m, g, st));
+    Stage2Desc a;
+    std::memset(&a, 0, sizeof(a));
+    a.H = m->H; a.dh = m->dh; a.L_NS = L_NS; a.C_tot = (int)C; a.s_len = s[n];
+    a.tiles = d_tiles; a.qkv = qkv; a.o = at;
+    kv_for_cache(c, n, row_off, a.kv);
+    a.scale = 1.0f / std::sqrt((float)m->dh);
+    OT_TRY(launch_stage2_attn<T>(m, a, (int)max_tiles, st));
+    GemmDesc go = gdesc_base(m);
+    go.mode = TILE_FLAT; go.M = (int)(L_NS * C); go.G = 1;
+    go.K = d; go.A = at; go.a_sm = d; go.a_mext = L_NS * C; go.a_gext = 1;
+    go.W = m->Wo[n]; go.w_rows = d; go.N = d;
+    go.res = rmap(x_in, 0, d);
+    go.out = rmap(xm, 0, d);
+    go.rms = rmap(h2, 0, d);
+    go.gamma = m->g_ffn[n];
+    OT_TRY(launch_gemm<T>(m, go, st));
+    GemmDesc f = g;
+    f.A = h2; f.W = m->W1_NS[n]; f.w_sg = (long long)dff * d; f.w_rows = dff; f.N = dff;
+    f.bias = m->b1_NS[n]; f.bias_sg = dff; f.act = ACT_GELU;
+    f.out = rmap(hid, dff, C * dff);
+    OT_TRY(launch_gemm<T>(m, f, st));
+    GemmDesc f2 = g;
+    f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.a_sg = C * dff;
+    f2.W = m->W2_NS[n]; f2.w_sg = (long long)d * dff; f2.w_rows = d; f2.N = d;
+    f2.bias = m->b2_NS[n]; f2.bias_sg = d;
+    f2.res = rmap(xm, d, C * d);
+    f2.out = rmap(x_next, d, C * d);
+    if (!last) { f2.rms = rmap(h, d, C * d); f2.gamma = m->g_attn[n + 1]; }
+    OT_TRY(launch_gemm<T>(m, f2, st));
+    x_in = x_next;
+  }
+  return ONETRANS_OK;
+}
+
+// =============================================================== append ==
+template <typename T>
+static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, const int* slots, int U,
+                                   const void* events, const int* types, int dL, void* ws,
+                                   size_t ws_bytes, cudaStream_t st, size_t* need) {
+  const int d = m->d, dff = m->dff, es = m->es, P = m->cfg.page_tokens;
+  Carve cv(ws, ws_bytes);
+  const long long R = (long long)U * dL;
+  void* xa = cv.take((size_t)R * d * es);
+  void* xb = cv.take((size_t)R * d * es);
+  void* h = cv.take((size_t)R * d * es);
+  void* q = cv.take((size_t)R * d * es);
+  void* at = cv.take((size_t)R * d * es);
+  void* xm = cv.take((size_t)R * d * es);
+  void* h2 = cv.take((size_t)R * d * es);
+  void* hid = cv.take((size_t)R * dff * es);
+  int* row_off = (int*)cv.take((size_t)std::max(U, 1) * sizeof(int));
+  if (need) { *need = cv.used; return ONETRANS_OK; }
+  if (cv.overflow) return ONETRANS_ERR_CAPACITY;
+  if (U == 0 || dL == 0) return ONETRANS_OK;
+  const int s_old = c->len[slots[0]];
+  const int s_new = s_old + dL;
+  if (s_new > c->max_L_S) return ONETRANS_ERR_CAPACITY;
+  // pages for positions [s_old, s_new) of every layer
+  long long needed = 0;
+  for (int u = 0; u < U; ++u) needed += (long long)m->NL * (cdiv(s_new, P) - cdiv(s_old, P));
+  if (needed > (long long)c->free_pages.size()) return ONETRANS_ERR_CAPACITY;
+  std::vector<int> h_row_off(U);
+  for (int u = 0; u < U; ++u) {
+    const size_t row = (size_t)slots[u] * m->NL * c->max_pages;
+    for (int n = 0; n < m->NL; ++n)
+      for (long long p = cdiv(s_old, P); p < cdiv(s_new, P); ++p) {
+        c->h_table[row + (size_t)n * c->max_pages + p] = c->free_pages.back();
+        c->free_pages.pop_back();
+      }
+    c->len[slots[u]] = s_new;
+    h_row_off[u] = (int)row;
+    OT_TRY(upload_slot_table(c, slots[u], st));
+  }
+  OT_TRY(cuda_ok(cudaMemcpyAsync(row_off, h_row_off.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
+
+  EventMLP w;
+  std::memset(&w, 0, sizeof(w));
+  for (int t = 0; t < m->cfg.n_behaviors; ++t) {
+    w.W1[t] = m->Wb1[t]; w.b1[t] = m->bb1[t]; w.W2[t] = m->Wb2[t]; w.b2[t] = m->bb2[t];
+  }
+  w.emb = m->type_emb; w.n_types = m->cfg.n_behaviors; w.e_dim = m->cfg.event_dim; w.d = d;
+  const size_t smem = (size_t)(w.e_dim + d) * sizeof(float);
+  event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>((const T*)events, types, dL, w,
+                                                                         rmap(xa, (long long)dL * d, d));
+  OT_TRY(last_launch());
+  OT_TRY(rms_flat<T>(m, xa, h, R, m->g_attn[0], st));
+  const void* x_in = xa;
+  for (int n = 0; n < m->NL; ++n) {
+    const bool last = n + 1 == m->NL;
+    void* x_next = (n % 2 == 0) ? xb : xa;
+    KVStore kv;
+    kv_for_cache(c, n, row_off, kv);
+    kv.pos_off = s_old;
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_FLAT; g.M = (int)R; g.fold = dL; g.G = 1;
+    g.K = d; g.A = h; g.a_sm = d; g.a_mext = R; g.a_gext = 1;
+    g.W = m->Wqkv_S[n]; g.w_rows = 3 * d; g.n_lo = d; g.N = 2 * d;
+    g.out_kind = OUT_KV; g.kv = kv;
+    OT_TRY(launch_gemm<T>(m, g, st));
+    if (last) break;  // the last layer's outputs feed nothing that is cached
+    g.n_lo = 0; g.N = d; g.out_kind = OUT_ROWS;
+    g.out = rmap(q, (long long)dL * d, d);
+    OT_TRY(launch_gemm<T>(m, g, st));
+    AttnDesc a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = U; a.H = m->H; a.dh = m->dh; a.Lq = dL; a.q_pos0 = s_old;
+    a.q = rmap(q, (long long)dL * d, d);
+    a.o = rmap(at, (long long)dL * d, d);
+    a.kv = kv; a.kv.pos_off = 0; a.scale = 1.0f / std::sqrt((float)m->dh);
+    OT_TRY(launch_attn<T>(m, a, st));
+    GemmDesc go = gdesc_base(m);
+    go.mode = TILE_FLAT; go.M = (int)R; go.fold = dL; go.G = 1;
+    go.K = d; go.A = at; go.a_sm = d; go.a_mext = R; go.a_gext = 1;
+    go.W = m->Wo[n]; go.w_rows = d; go.N = d;
+    go.res = rmap(x_in, (long long)dL * d, d);
+    go.out = rmap(xm, (long long)dL * d, d);
+    go.rms = rmap(h2, (long long)dL * d, d);
+    go.gamma = m->g_ffn[n];
+    OT_TRY(launch_gemm<T>(m, go, st));
+    GemmDesc f = go;
+    f.res.base = nullptr; f.rms.base = nullptr; f.gamma = nullptr;
+    f.A = h2; f.W = m->W1_S[n]; f.w_rows = dff; f.N = dff; f.bias = m->b1_S[n]; f.act = ACT_GELU;
+    f.out = rmap(hid, (long long)dL * dff, dff);
+    OT_TRY(launch_gemm<T>(m, f, st));
+    GemmDesc f2 = go;
+    f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.W = m->W2_S[n]; f2.w_rows = d; f2.N = d;
+    f2.bias = m->b2_S[n];
+    f2.res = rmap(xm, (long long)dL * d, d);
+    f2.out = rmap(x_next, (long long)dL * d, d);
+    f2.rms = rmap(h, (long long)dL * d, d);
+    f2.gamma = m->g_attn[n + 1];
+    OT_TRY(launch_gemm<T>(m, f2, st));
+    x_in = x_next;
+  }
+  return ONETRANS_OK;
+}
+
+// ============================================================ autosplit ==
+template <typename T>
+static onetrans_status autosplit_impl(const onetrans_model* m, const void* feats, long long N, void* out,
+                                      void* ws, size_t ws_bytes, cudaStream_t st, size_t* need) {
+  const int F = m->cfg.ns_feat_dim, Hh = m->cfg.ns_hidden, d = m->d, L_NS = m->L_NS, es = m->es;
+  Carve cv(ws, ws_bytes);
+  void* hid = cv.take((size_t)N * Hh * es);
+  if (need) { *need = cv.used; return ONETRANS_OK; }
+  if (cv.overflow) return ONETRANS_ERR_CAPACITY;
+  if (N == 0) return ONETRANS_OK;
+  GemmDesc g = gdesc_base(m);
+  g.mode = TILE_FLAT; g.M = (int)N; g.G = 1;
+  g.K = F; g.A = feats; g.a_sm = F; g.a_mext = N; g.a_gext = 1;
+  g.W = m->Wa1; g.w_rows = Hh; g.N = Hh; g.bias = m->ba1; g.act = ACT_GELU;
+  g.out = rmap(hid, 0, Hh);
+  OT_TRY(launch_gemm<T>(m, g, st));
+  GemmDesc g2 = g;
+  g2.K = Hh; g2.A = hid; g2.a_sm = Hh; g2.W = m->Wa2; g2.w_rows = L_NS * d; g2.N = L_NS * d;
+  g2.bias = m->ba2; g2.act = ACT_NONE;
+  g2.out = rmap(out, 0, d);
+  g2.out.sc = N * d;
+  g2.out.split = d;
+  return launch_gemm<T>(m, g2, st);
+}
+
+// ============================================================== C ABI ====
+extern "C" {
+
+int32_t onetrans_version(void) { return 100; }
+
+const char* onetrans_status_string(int32_t s) {
+  switch (s) {
+    case ONETRANS_OK: return "ok";
+    case ONETRANS_ERR_INVALID_ARG: return "invalid argument";
+    case ONETRANS_ERR_SHAPE: return "shape mismatch";
+    case ONETRANS_ERR_UNSUPPORTED: return "unsupported";
+    case ONETRANS_ERR_CAPACITY: return "capacity exceeded";
+    case ONETRANS_ERR_CUDA: return "CUDA error";
+    case ONETRANS_ERR_DEVICE_CHECK: return "device-side check failed";
+    default: return "unknown status";
+  }
+}
+
+onetrans_status onetrans_set_kernel_policy(int32_t policy) {
+  if (policy < 0 || policy > 1) return ONETRANS_ERR_INVALID_ARG;
+  g_policy = policy;
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_model_create(const onetrans_config* cfg, const onetrans_weights* w,
+                                      onetrans_model** out) {
+  if (!cfg || !w || !out) return ONETRANS_ERR_INVALID_ARG;
+  *out = nullptr;
+  const int NL = cfg->n_layers, d = cfg->d_model, H = cfg->n_heads;
+  if (NL < 1 || NL > 64 || d < 1 || H < 1 || cfg->d_ff < 1 || cfg->L_NS < 1 || cfg->L_NS > 256)
+    return ONETRANS_ERR_SHAPE;
+  if (d % H) return ONETRANS_ERR_SHAPE;
+  const int dh = d / H;
+  if (dh != 32 && dh != 64 && dh != 96 && dh != 128) return ONETRANS_ERR_UNSUPPORTED;
+  if (cfg->mode != ONETRANS_BF16 && cfg->mode != ONETRANS_FP32) return ONETRANS_ERR_INVALID_ARG;
+  if (cfg->page_tokens != 64) return ONETRANS_ERR_UNSUPPORTED;
+  if (!(cfg->rms_eps > 0.f)) return ONETRANS_ERR_INVALID_ARG;
+  if (cfg->n_behaviors < 0 || cfg->n_behaviors > 8 || cfg->event_dim < 0 || cfg->ns_feat_dim < 0 ||
+      cfg->ns_hidden < 0)
+    return ONETRANS_ERR_SHAPE;
+  if (cfg->event_dim > 4096) return ONETRANS_ERR_UNSUPPORTED;
+  const void* const* per_layer[] = {w->g_attn, w->g_ffn, w->Wqkv_S, w->Wqkv_NS, w->Wo, w->W1_S, w->b1_S,
+                                    w->W2_S, w->b2_S, w->W1_NS, w->b1_NS, w->W2_NS, w->b2_NS};
+  for (auto arr : per_layer) {
+    if (!arr) return ONETRANS_ERR_INVALID_ARG;
+    for (int l = 0; l < NL; ++l)
+      if (!arr[l] || !aligned(arr[l], 16)) return ONETRANS_ERR_INVALID_ARG;
+  }
+  std::vector<int> pyr;
+  if (cfg->pyramid_q) {
+    for (int l = 0; l < NL; ++l) {
+      const int q = cfg->pyramid_q[l];
+      if (q < cfg->L_NS || (l > 0 && q > pyr.back())) return ONETRANS_ERR_SHAPE;
+      pyr.push_back(q);
+    }
+  }
+  onetrans_model* m = new (std::nothrow) onetrans_model();
+  if (!m) return ONETRANS_ERR_CAPACITY;
+  m->cfg = *cfg;
+  m->cfg.pyramid_q = nullptr;
+  m->pyr = pyr;
+  m->d = d; m->H = H; m->dh = dh; m->dff = cfg->d_ff; m->L_NS = cfg->L_NS; m->NL = NL;
+  m->bf16 = cfg->mode == ONETRANS_BF16;
+  m->es = m->bf16 ? 2 : 4;
+  auto cp = [NL](const void* const* a) { return std::vector<const void*>(a, a + NL); };
+  m->g_attn = cp(w->g_attn); m->g_ffn = cp(w->g_ffn); m->Wqkv_S = cp(w->Wqkv_S);
+  m->Wqkv_NS = cp(w->Wqkv_NS); m->Wo = cp(w->Wo); m->W1_S = cp(w->W1_S); m->b1_S = cp(w->b1_S);
+  m->W2_S = cp(w->W2_S); m->b2_S = cp(w->b2_S); m->W1_NS = cp(w->W1_NS); m->b1_NS = cp(w->b1_NS);
+  m->W2_NS = cp(w->W2_NS); m->b2_NS = cp(w->b2_NS);
+  m->Wa1 = w->Wa1; m->ba1 = w->ba1; m->Wa2 = w->Wa2; m->ba2 = w->ba2; m->type_emb = w->type_emb;
+  const int nb = cfg->n_behaviors;
+  if (nb > 0 && w->Wb1 && w->bb1 && w->Wb2 && w->bb2) {
+    m->Wb1.assign(w->Wb1, w->Wb1 + nb); m->bb1.assign(w->bb1, w->bb1 + nb);
+    m->Wb2.assign(w->Wb2, w->Wb2 + nb); m->bb2.assign(w->bb2, w->bb2 + nb);
+  }
+  *out = m;
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_model_destroy(onetrans_model* m) {
+  if (!m) return ONETRANS_ERR_INVALID_ARG;
+  delete m;
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_schedule(const onetrans_model* m, int32_t L_S, int32_t* out) {
+  if (!m || !out) return ONETRANS_ERR_INVALID_ARG;
+  std::vector<int> Lq;
+  OT_TRY(schedule_of(m, L_S, Lq));
+  std::copy(Lq.begin(), Lq.end(), out);
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_workspace_size(const onetrans_model* m, int32_t op, int64_t n, int32_t L,
+                                        size_t* bytes) {
+  if (!m || !bytes) return ONETRANS_ERR_INVALID_ARG;
+  if (n < 0 || n > (1LL << 31) - 1 || L < 0) return ONETRANS_ERR_SHAPE;
+  *bytes = 0;
+  const int nn = (int)n;
+  switch (op) {
+    case ONETRANS_OP_FORWARD:
+      return m->bf16 ? forward_impl<__nv_bfloat16>(m, nullptr, nn, L, nullptr, nullptr, 0, 0, bytes)
+                     : forward_impl<float>(m, nullptr, nn, L, nullptr, nullptr, 0, 0, bytes);
+    case ONETRANS_OP_STAGE1:
+      return m->bf16 ? stage1_impl<__nv_bfloat16>(m, nullptr, nullptr, nn, nullptr, L, nullptr, 0, 0, bytes)
+                     : stage1_impl<float>(m, nullptr, nullptr, nn, nullptr, L, nullptr, 0, 0, bytes);
+    case ONETRANS_OP_STAGE2:
+      return m->bf16 ? stage2_impl<__nv_bfloat16>(m, nullptr, nullptr, 1, nullptr, nullptr, nullptr, nullptr, 0,
+                                                  0, bytes, n, L)
+                     : stage2_impl<float>(m, nullptr, nullptr, 1, nullptr, nullptr, nullptr, nullptr, 0, 0,
+                                          bytes, n, L);
+    case ONETRANS_OP_APPEND:
+      return m->bf16 ? append_impl<__nv_bfloat16>(m, nullptr, nullptr, nn, nullptr, nullptr, L, nullptr, 0, 0,
+                                                  bytes)
+                     : append_impl<float>(m, nullptr, nullptr, nn, nullptr, nullptr, L, nullptr, 0, 0, bytes);
+    case ONETRANS_OP_AUTOSPLIT:
+      return m->bf16 ? autosplit_impl<__nv_bfloat16>(m, nullptr, n, nullptr, nullptr, 0, 0, bytes)
+                     : autosplit_impl<float>(m, nullptr, n, nullptr, nullptr, 0, 0, bytes);
+    default:
+      return ONETRANS_ERR_INVALID_ARG;
+  }
+}
+
+// ---------------------------------------------------------------- cache --
+static void cache_layout(const onetrans_model* m, int n_slots, int max_L_S, int& max_pages, long long& n_pages,
+                         size_t& table_bytes, size_t& page_bytes) {
+  const int P = m->cfg.page_tokens;
+  std::vector<int> s, sq;
+  long long per_slot = 0;
+  max_pages = (int)cdiv(max_L_S, P);
+  if (s_rows_of(m, max_L_S, s, sq) == ONETRANS_OK) {
+    for (int n = 0; n < m->NL; ++n) per_slot += cdiv(s[n], P);
+  } else {
+    per_slot = (long long)m->NL * max_pages;  // no valid schedule at this length: worst case
+  }
+  n_pages = per_slot * n_slots;
+  table_bytes = (((size_t)n_slots * m->NL * max_pages * sizeof(int)) + 255) & ~(size_t)255;
+  page_bytes = (size_t)2 * m->d * P * m->es;
+}
+
+onetrans_status onetrans_cache_size(const onetrans_model* m, int32_t n_slots, int32_t max_L_S, size_t* bytes) {
+  if (!m || !bytes) return ONETRANS_ERR_INVALID_ARG;
+  if (n_slots < 1 || max_L_S < 1) return ONETRANS_ERR_SHAPE;
+  int max_pages;
+  long long n_pages;
+  size_t tb, pb;
+  cache_layout(m, n_slots, max_L_S, max_pages, n_pages, tb, pb);
+  *bytes = tb + (size_t)n_pages * pb;
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_cache_init(const onetrans_model* m, void* pool, size_t bytes, int32_t n_slots,
+                                    int32_t max_L_S, onetrans_cache** out) {
+  if (!m || !pool || !out) return ONETRANS_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!aligned(pool, 256)) return ONETRANS_ERR_INVALID_ARG;
+  if (n_slots < 1 || max_L_S < 1) return ONETRANS_ERR_SHAPE;
+  int max_pages;
+  long long n_pages;
+  size_t tb, pb;
+  cache_layout(m, n_slots, max_L_S, max_pages, n_pages, tb, pb);
+  if (tb + (size_t)n_pages * pb > bytes) return ONETRANS_ERR_CAPACITY;
+  onetrans_cache* c = new (std::nothrow) onetrans_cache();
+  if (!c) return ONETRANS_ERR_CAPACITY;
+  c->m = m; c->pool = (char*)pool; c->bytes = bytes; c->n_slots = n_slots; c->max_L_S = max_L_S;
+  c->max_pages = max_pages; c->n_pages = (int)n_pages;
+  c->d_table = (int*)pool;
+  c->d_pages = (char*)pool + tb;
+  c->h_table.assign((size_t)n_slots * m->NL * max_pages, -1);
+  c->len.assign(n_slots, 0);
+  c->free_pages.resize(n_pages);
+  for (long long i = 0; i < n_pages; ++i) c->free_pages[i] = (int)(n_pages - 1 - i);
+  *out = c;
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_cache_destroy(onetrans_cache* c) {
+  if (!c) return ONETRANS_ERR_INVALID_ARG;
+  delete c;
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_cache_length(const onetrans_cache* c, int32_t slot, int32_t* len) {
+  if (!c || !len) return ONETRANS_ERR_INVALID_ARG;
+  if (slot < 0 || slot >= c->n_slots) return ONETRANS_ERR_SHAPE;
+  *len = c->len[slot];
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_cache_row_ptr(const onetrans_cache* c, int32_t slot, int32_t layer, int32_t kind,
+                                       int32_t head, int32_t token, void** ptr) {
+  if (!c || !ptr) return ONETRANS_ERR_INVALID_ARG;
+  const onetrans_model* m = c->m;
+  if (slot < 0 || slot >= c->n_slots || layer < 0 || layer >= m->NL || kind < 0 || kind > 1 || head < 0 ||
+      head >= m->H || token < 0 || token / m->cfg.page_tokens >= c->max_pages)
+    return ONETRANS_ERR_SHAPE;
+  const int P = m->cfg.page_tokens;
+  const int page = c->h_table[((size_t)slot * m->NL + layer) * c->max_pages + token / P];
+  if (page < 0) return ONETRANS_ERR_SHAPE;
+  const size_t el = (size_t)page * 2 * m->d * P + ((size_t)(kind * m->H + head) * P + token % P) * m->dh;
+  *ptr = c->d_pages + el * m->es;
+  return ONETRANS_OK;
+}
+
+// ---------------------------------------------------------- entry points --
+static onetrans_status check_ws(void* ws) {
+  return (ws && aligned(ws, 256)) ? ONETRANS_OK : ONETRANS_ERR_INVALID_ARG;
+}
+
+onetrans_status onetrans_tokenize_autosplit(const onetrans_model* m, const void* feats, int64_t N,
+                                            void* ns_tokens, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !feats || !ns_tokens || !aligned(feats, 16) || !aligned(ns_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
+  if (N < 0 || N > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
+  if (!m->Wa1 || !m->ba1 || !m->Wa2 || !m->ba2 || m->cfg.ns_feat_dim < 1 || m->cfg.ns_hidden < 1)
+    return ONETRANS_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? autosplit_impl<__nv_bfloat16>(m, feats, N, ns_tokens, ws, ws_bytes, st, nullptr)
+                 : autosplit_impl<float>(m, feats, N, ns_tokens, ws, ws_bytes, st, nullptr);
+}
+
+static onetrans_status check_slots(const onetrans_cache* c, const int32_t* slots, int U) {
+  if (U < 0) return ONETRANS_ERR_SHAPE;
+  if (U > 0 && !slots) return ONETRANS_ERR_INVALID_ARG;
+  std::vector<char> seen(c->n_slots, 0);
+  for (int u = 0; u < U; ++u) {
+    if (slots[u] < 0 || slots[u] >= c->n_slots) return ONETRANS_ERR_SHAPE;
+    if (seen[slots[u]]) return ONETRANS_ERR_INVALID_ARG;
+    seen[slots[u]] = 1;
+  }
+  return ONETRANS_OK;
+}
+
+onetrans_status onetrans_stage1_encode(const onetrans_model* m, onetrans_cache* c, const int32_t* slots,
+                                       int32_t U, const void* s_tokens, int32_t L_S, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  if (!m || !c || c->m != m || !s_tokens || !aligned(s_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
+  OT_TRY(check_slots(c, slots, U));
+  if (L_S < 1) return ONETRANS_ERR_SHAPE;
+  if ((long long)U * L_S > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
+  if (U == 0) return ONETRANS_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? stage1_impl<__nv_bfloat16>(m, c, slots, U, s_tokens, L_S, ws, ws_bytes, st, nullptr)
+                 : stage1_impl<float>(m, c, slots, U, s_tokens, L_S, ws, ws_bytes, st, nullptr);
+}
+
+onetrans_status onetrans_stage2_score(const onetrans_model* m, const onetrans_cache* c, const int32_t* slots,
+                                      int32_t U, const int32_t* cand_offsets, const void* ns_tokens,
+                                      void* ns_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !c || c->m != m || !cand_offsets || !ns_tokens || !ns_out) return ONETRANS_ERR_INVALID_ARG;
+  if (!aligned(ns_tokens, 16) || !aligned(ns_out, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
+  OT_TRY(check_slots(c, slots, U));
+  if (U == 0) return ONETRANS_OK;
+  if (U > kMaxUsers) return ONETRANS_ERR_SHAPE;
+  for (int u = 0; u < U; ++u)
+    if (cand_offsets[u + 1] < cand_offsets[u]) return ONETRANS_ERR_SHAPE;
+  if (cand_offsets[0] != 0) return ONETRANS_ERR_SHAPE;
+  const int L_S = c->len[slots[0]];
+  for (int u = 0; u < U; ++u)
+    if (c->len[slots[u]] != L_S || L_S == 0) return ONETRANS_ERR_SHAPE;
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? stage2_impl<__nv_bfloat16>(m, c, slots, U, cand_offsets, ns_tokens, ns_out, ws, ws_bytes,
+                                              st, nullptr, 0, 0)
+                 : stage2_impl<float>(m, c, slots, U, cand_offsets, ns_tokens, ns_out, ws, ws_bytes, st,
+                                      nullptr, 0, 0);
+}
+
+onetrans_status onetrans_cache_append(const onetrans_model* m, onetrans_cache* c, const int32_t* slots,
+                                      int32_t U, const void* events, const int32_t* types, int32_t dL,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !c || c->m != m) return ONETRANS_ERR_INVALID_ARG;
+  if (!m->pyr.empty()) return ONETRANS_ERR_UNSUPPORTED;
+  if (m->cfg.n_behaviors < 1 || m->cfg.event_dim < 1 || m->Wb1.empty() || !m->type_emb)
+    return ONETRANS_ERR_UNSUPPORTED;
+  if (!events || !types || !aligned(events, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
+  OT_TRY(check_slots(c, slots, U));
+  if (dL < 0) return ONETRANS_ERR_SHAPE;
+  if (U == 0 || dL == 0) return ONETRANS_OK;
+  const int L0 = c->len[slots[0]];
+  for (int u = 0; u < U; ++u)
+    if (c->len[slots[u]] != L0 || L0 == 0) return ONETRANS_ERR_SHAPE;
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? append_impl<__nv_bfloat16>(m, c, slots, U, events, types, dL, ws, ws_bytes, st, nullptr)
+                 : append_impl<float>(m, c, slots, U, events, types, dL, ws, ws_bytes, st, nullptr);
+}
+
+onetrans_status onetrans_forward(const onetrans_model* m, const void* x0, int32_t B, int32_t L_S, void* out,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !x0 || !out || !aligned(x0, 16) || !aligned(out, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
+  if (B < 0 || L_S < 0) return ONETRANS_ERR_SHAPE;
+  if ((long long)B * (L_S + m->L_NS) > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
+  if (B == 0) return ONETRANS_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? forward_impl<__nv_bfloat16>(m, x0, B, L_S, out, ws, ws_bytes, st, nullptr)
+                 : forward_impl<float>(m, x0, B, L_S, out, ws, ws_bytes, st, nullptr);
+}
+
+onetrans_status onetrans_device_status(void* stream, int32_t* code) {
+  if (!code) return ONETRANS_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  int v = 0;
+  OT_TRY(cuda_ok(cudaMemcpyFromSymbolAsync(&v, ot::g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st)));
+  OT_TRY(cuda_ok(cudaStreamSynchronize(st)));
+  *code = v;
+  if (v) {
+    const int zero = 0;
+    OT_TRY(cuda_ok(cudaMemcpyToSymbolAsync(ot::g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st)));
+    OT_TRY(cuda_ok(cudaStreamSynchronize(st)));
+  }
+  return ONETRANS_OK;
+}
+
+}  // extern "C"

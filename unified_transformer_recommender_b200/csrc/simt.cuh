@@ -1,0 +1,290 @@
+// CUDA-core kernels: the float32 mode's whole path, and the fallback for
+// shapes the tensor-core kernels do not take.  Same descriptors and memory
+// layouts as the tensor-core path.
+#pragma once
+#include "common.cuh"
+
+namespace ot {
+
+// ------------------------------------------------------------------ GEMM --
+// C[(b,t), n] = epilogue( sum_k A[(m,g), k] * W[grp][n_lo + n][k] )
+// 64x64 output tile per CTA, 256 threads, 4x4 outputs per thread.
+template <typename T>
+__device__ inline void epilogue_store(const GemmDesc& d, int b, int t, int n, int grp, float v) {
+  if (d.bias) v += to_f(((const T*)d.bias)[grp * d.bias_sg + d.n_lo + n]);
+  if (d.act == ACT_GELU) v = gelu_tanh(v);
+  if (d.res.base) v += to_f(((const T*)d.res.base)[rm_off(d.res, b, t, n)]);
+  if (d.out_kind == OUT_KV) {
+    const int dm = d.kv.H * d.kv.dh;
+    const int kind = n / dm, c = n - kind * dm, head = c / d.kv.dh, e = c - head * d.kv.dh;
+    ((T*)d.kv.pool)[kv_off(d.kv, b, t + d.kv.pos_off, kind, head, e)] = from_f<T>(v);
+  } else {
+    ((T*)d.out.base)[rm_off(d.out, b, t, n)] = from_f<T>(v);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc d) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int n0 = blockIdx.x * 64, m0 = d.m_lo + blockIdx.y * 64, g = d.g_lo + blockIdx.z;
+  const int m_end = d.m_lo + d.M;
+  const int grp = d.mode == TILE_SAMPLES ? g - d.grp_base : 0;
+  const T* A = (const T*)d.A;
+  const T* W = (const T*)d.W + (long long)grp * d.w_sg + (long long)d.n_lo * d.K;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < d.K; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      const int r = i >> 4, kk = i & 15, k = k0 + kk;
+      const int m = m0 + r, n = n0 + r;
+      As[kk][r] = (m < m_end && k < d.K) ? to_f(A[(long long)m * d.a_sm + (long long)g * d.a_sg + k]) : 0.f;
+      Bs[kk][r] = (n < d.N && k < d.K) ? to_f(W[(long long)n * d.K + k]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; w[i] = Bs[kk][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= m_end) continue;
+    int b, t;
+    row_of(d, m, g, b, t);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < d.N) epilogue_store<T>(d, b, t, n, grp, acc[i][j]);
+    }
+  }
+}
+
+// -------------------------------------------------------------- RMSNorm --
+// For every row the descriptor enumerates: dst = src * rsqrt(mean(src^2) + eps) * gamma
+// over N columns; src = d.out, dst = d.rms.  One warp per row.
+template <typename T>
+__global__ void rms_rows_kernel(GemmDesc d) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = d.m_lo + blockIdx.x * (blockDim.x >> 5) + warp;
+  const int g = d.g_lo + blockIdx.y;
+  if (m >= d.m_lo + d.M) return;
+  int b, t;
+  row_of(d, m, g, b, t);
+  const T* src = (const T*)d.out.base;
+  T* dst = (T*)d.rms.base;
+  float ss = 0.f;
+  for (int n = lane; n < d.N; n += 32) {
+    const float v = to_f(src[rm_off(d.out, b, t, n)]);
+    ss += v * v;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = rsqrtf(ss / d.N + d.eps);
+  const T* gm = (const T*)d.gamma;
+  for (int n = lane; n < d.N; n += 32) {
+    const float v = to_f(src[rm_off(d.out, b, t, n)]);
+    dst[rm_off(d.rms, b, t, n)] = from_f<T>(v * r * to_f(gm[n]));
+  }
+}
+
+// ------------------------------------------------------ causal attention --
+constexpr int KT = 32;  // keys staged in shared memory per step
+// Query t of batch b (key position p = q_pos0 + t) attends to keys 0..p of
+// its K/V store.  One thread per query, 64 queries per CTA, keys staged in
+// shared memory KT at a time, online softmax in base 2.
+template <typename T, int DH>
+__global__ void __launch_bounds__(64) attn_simt_kernel(AttnDesc a) {
+  __shared__ float Ks[KT][DH + 1];
+  __shared__ float Vs[KT][DH + 1];
+  __shared__ float Ss[KT][65];
+  const int tid = threadIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int t = blockIdx.x * 64 + tid;
+  const bool valid = t < a.Lq;
+  const int p = a.q_pos0 + t;
+  const int t_last = min(a.Lq, (int)(blockIdx.x + 1) * 64) - 1;
+  const int kmax = a.q_pos0 + t_last;
+  const float qs = a.scale * 1.4426950408889634f;
+  float q[DH], o[DH];
+  const T* qp = (const T*)a.q.base + rm_off(a.q, b, valid ? t : 0, h * DH);
+#pragma unroll
+  for (int e = 0; e < DH; ++e) { q[e] = valid ? to_f(qp[e]) * qs : 0.f; o[e] = 0.f; }
+  float mrow = -INFINITY, lrow = 0.f;
+  const T* pool = (const T*)a.kv.pool;
+  for (int k0 = 0; k0 <= kmax; k0 += KT) {
+    __syncthreads();
+    for (int i = tid; i < KT * DH; i += 64) {
+      const int r = i / DH, e = i - r * DH, pos = k0 + r;
+      float kv = 0.f, vv = 0.f;
+      if (pos <= kmax) {
+        kv = to_f(pool[kv_off(a.kv, b, pos, 0, h, e)]);
+        vv = to_f(pool[kv_off(a.kv, b, pos, 1, h, e)]);
+      }
+      Ks[r][e] = kv;
+      Vs[r][e] = vv;
+    }
+    __syncthreads();
+    float mt = -INFINITY;
+    for (int r = 0; r < KT; ++r) {
+      float s = -INFINITY;
+      if (valid && k0 + r <= p) {
+        s = 0.f;
+#pragma unroll
+        for (int e = 0; e < DH; ++e) s = fmaf(q[e], Ks[r][e], s);
+      }
+      Ss[r][tid] = s;
+      mt = fmaxf(mt, s);
+    }
+    if (!valid || mt == -INFINITY) continue;
+    const float mn = fmaxf(mrow, mt);
+    const float c = exp2f(mrow - mn);
+    lrow *= c;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) o[e] *= c;
+    for (int r = 0; r < KT; ++r) {
+      const float pr = exp2f(Ss[r][tid] - mn);
+      lrow += pr;
+#pragma unroll
+      for (int e = 0; e < DH; ++e) o[e] = fmaf(pr, Vs[r][e], o[e]);
+    }
+    mrow = mn;
+  }
+  if (!valid) return;
+  T* op = (T*)a.o.base + rm_off(a.o, b, t, h * DH);
+  const float inv = 1.f / lrow;
+#pragma unroll
+  for (int e = 0; e < DH; ++e) op[e] = from_f<T>(o[e] * inv);
+}
+
+// ---------------------------------------------------- Stage II attention --
+// NS token j of candidate c (one thread each, all candidates of the CTA from
+// one user) attends in one softmax to the user's s_len cached S keys and to
+// its own NS keys 0..j.
+template <typename T, int DH>
+__global__ void __launch_bounds__(64) stage2_attn_simt_kernel(Stage2Desc a) {
+  __shared__ float Ks[KT][DH + 1];
+  __shared__ float Vs[KT][DH + 1];
+  __shared__ float Ss[KT][65];
+  const int tid = threadIdx.x, h = blockIdx.y, j = blockIdx.z;
+  const int user = a.tiles[blockIdx.x * 3 + 0];
+  const int c = a.tiles[blockIdx.x * 3 + 1] + tid;
+  const bool valid = c < a.tiles[blockIdx.x * 3 + 2];
+  const int d = a.H * DH;
+  const long long rs = 3LL * d;  // row stride of the packed Q|K|V rows
+  const T* qkv = (const T*)a.qkv;
+  const float qs = a.scale * 1.4426950408889634f;
+  float q[DH], o[DH];
+  const T* qp = qkv + ((long long)j * a.C_tot + (valid ? c : 0)) * rs + h * DH;
+#pragma unroll
+  for (int e = 0; e < DH; ++e) { q[e] = valid ? to_f(qp[e]) * qs : 0.f; o[e] = 0.f; }
+  float mrow = -INFINITY, lrow = 0.f;
+  const T* pool = (const T*)a.kv.pool;
+  for (int k0 = 0; k0 < a.s_len; k0 += KT) {
+    __syncthreads();
+    for (int i = tid; i < KT * DH; i += 64) {
+      const int r = i / DH, e = i - r * DH, pos = k0 + r;
+      float kv = 0.f, vv = 0.f;
+      if (pos < a.s_len) {
+        kv = to_f(pool[kv_off(a.kv, user, pos, 0, h, e)]);
+        vv = to_f(pool[kv_off(a.kv, user, pos, 1, h, e)]);
+      }
+      Ks[r][e] = kv;
+      Vs[r][e] = vv;
+    }
+    __syncthreads();
+    float mt = -INFINITY;
+    for (int r = 0; r < KT; ++r) {
+      float s = -INFINITY;
+      if (k0 + r < a.s_len) {
+        s = 0.f;
+#pragma unroll
+        for (int e = 0; e < DH; ++e) s = fmaf(q[e], Ks[r][e], s);
+      }
+      Ss[r][tid] = s;
+      mt = fmaxf(mt, s);
+    }
+    const float mn = fmaxf(mrow, mt);
+    if (mn == -INFINITY) continue;
+    const float cf = exp2f(mrow - mn);
+    lrow *= cf;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) o[e] *= cf;
+    for (int r = 0; r < KT; ++r) {
+      const float pr = exp2f(Ss[r][tid] - mn);
+      lrow += pr;
+#pragma unroll
+      for (int e = 0; e < DH; ++e) o[e] = fmaf(pr, Vs[r][e], o[e]);
+    }
+    mrow = mn;
+  }
+  if (!valid) return;
+  // own NS keys 0..j of this candidate
+  for (int i = 0; i <= j; ++i) {
+    const T* kp = qkv + ((long long)i * a.C_tot + c) * rs + d + h * DH;
+    const T* vp = kp + d;
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) s = fmaf(q[e], to_f(kp[e]), s);
+    const float mn = fmaxf(mrow, s);
+    const float cf = exp2f(mrow - mn), pr = exp2f(s - mn);
+    lrow = lrow * cf + pr;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) o[e] = fmaf(pr, to_f(vp[e]), o[e] * cf);
+    mrow = mn;
+  }
+  T* op = (T*)a.o + ((long long)j * a.C_tot + c) * d + h * DH;
+  const float inv = 1.f / lrow;
+#pragma unroll
+  for (int e = 0; e < DH; ++e) op[e] = from_f<T>(o[e] * inv);
+}
+
+// ------------------------------------------------------ event tokenizer --
+// out(b, t) = W2[ty] gelu(W1[ty] e + b1[ty]) + b2[ty] + type_emb[ty] for each
+// appended event; one CTA per event, one thread per output feature.
+struct EventMLP {
+  const void* W1[8];
+  const void* b1[8];
+  const void* W2[8];
+  const void* b2[8];
+  const void* emb;
+  int n_types, e_dim, d;
+};
+
+template <typename T>
+__global__ void event_tokenize_kernel(const T* ev, const int* types, int dL, EventMLP w, RowMap out) {
+  extern __shared__ float sm[];
+  float* e = sm;              // [e_dim]
+  float* hid = sm + w.e_dim;  // [d]
+  const int row = blockIdx.x, b = row / dL, t = row - b * dL;
+  int ty = types[row];
+  if (ty < 0 || ty >= w.n_types) {
+    if (threadIdx.x == 0) flag_error(3);
+    ty = 0;
+  }
+  for (int i = threadIdx.x; i < w.e_dim; i += blockDim.x) e[i] = to_f(ev[(long long)row * w.e_dim + i]);
+  __syncthreads();
+  const T* W1 = (const T*)w.W1[ty];
+  const T* W2 = (const T*)w.W2[ty];
+  for (int k = threadIdx.x; k < w.d; k += blockDim.x) {
+    float s = to_f(((const T*)w.b1[ty])[k]);
+    for (int i = 0; i < w.e_dim; ++i) s = fmaf(to_f(W1[(long long)k * w.e_dim + i]), e[i], s);
+    hid[k] = gelu_tanh(s);
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < w.d; k += blockDim.x) {
+    float s = to_f(((const T*)w.b2[ty])[k]);
+    for (int i = 0; i < w.d; ++i) s = fmaf(to_f(W2[(long long)k * w.d + i]), hid[i], s);
+    s += to_f(((const T*)w.emb)[(long long)ty * w.d + k]);
+    ((T*)out.base)[rm_off(out, b, t, k)] = from_f<T>(s);
+  }
+}
+
+}  // namespace ot
