@@ -12,9 +12,12 @@
  *    "host".  The library never allocates device memory: each call takes a
  *    caller-provided workspace whose size onetrans_workspace_size() reports,
  *    and the KV cache lives in a caller-provided pool (onetrans_cache_size()).
- *  - Tensors are dense row-major.  Element type follows the model's mode:
- *    ONETRANS_BF16 -> bfloat16 storage (fp32 accumulation inside kernels),
- *    ONETRANS_FP32 -> float32 storage and float32 arithmetic on CUDA cores.
+ *  - Tensors are dense row-major.  Inputs and weights follow the model's
+ *    mode: ONETRANS_BF16 -> bfloat16 (fp32 accumulation inside kernels),
+ *    ONETRANS_FP32 -> float32 with float32 arithmetic on CUDA cores.  The
+ *    outputs of the stack (onetrans_forward's `out`, onetrans_stage2_score's
+ *    `ns_out`) are float32 in both modes; inside, the residual stream is kept
+ *    in float32 and only matrix operands and cached K/V use the mode's type.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Calls are asynchronous on that stream; inputs must stay valid
  *    and unmodified until the stream reaches the call's end.
@@ -54,7 +57,7 @@ typedef enum { ONETRANS_BF16 = 0, ONETRANS_FP32 = 1 } onetrans_mode;
 
 /* Model hyper-parameters.  [FR] 7.5.0-7.5.2 fix the structure; the widths,
  * head count, depth and schedule are the caller's choice.
- *  d_model % n_heads == 0, d_h = d_model / n_heads in {32, 64, 96, 128}.
+ *  d_model % n_heads == 0, d_h = d_model / n_heads in {16, 32, 64, 96, 128}.
  *  pyramid_q (host, n_layers entries): L'_n, the number of tail rows kept as
  *    queries by layer n ([FR] 7.5.2, tail index set Q = {L-L'+1..L}).  NULL
  *    keeps every row.  Must be non-increasing and >= L_NS.
@@ -192,8 +195,9 @@ ONETRANS_API onetrans_status onetrans_stage1_encode(const onetrans_model* m,
  * entries) and cache slot slots[u] (host).  Per layer, NS token j of a
  * candidate attends in one softmax to the slot's cached S keys and its own
  * NS keys 0..j, then passes through its token-specific FFN.  All slots must
- * hold the same S length.
- *   ns_tokens [L_NS, C_tot, d] token-major input; ns_out [L_NS, C_tot, d]. */
+ * hold the same S length; at most 65536 users per call.
+ *   ns_tokens [L_NS, C_tot, d] token-major input;
+ *   ns_out    [L_NS, C_tot, d] float32. */
 ONETRANS_API onetrans_status onetrans_stage2_score(const onetrans_model* m,
                                       const onetrans_cache* c,
                                       const int32_t* slots, int32_t U,
@@ -213,8 +217,8 @@ ONETRANS_API onetrans_status onetrans_cache_append(const onetrans_model* m,
                                       void* ws, size_t ws_bytes, void* stream);
 
 /* One-pass forward of the stack on X^(0) = [S-tokens; NS-tokens] ([FR] 7.5.0
- * eq. for X^(0), 7.5.1, 7.5.2).  x0 [B, L_S + L_NS, d]; out [B, L'_N, d],
- * the rows the last layer keeps. */
+ * eq. for X^(0), 7.5.1, 7.5.2).  x0 [B, L_S + L_NS, d]; out [B, L'_N, d]
+ * float32, the rows the last layer keeps. */
 ONETRANS_API onetrans_status onetrans_forward(const onetrans_model* m, const void* x0,
                                  int32_t B, int32_t L_S, void* out, void* ws,
                                  size_t ws_bytes, void* stream);

@@ -67,7 +67,7 @@ def test_model_create_validation():
     assert FakeModel().status == ot.OK
     assert FakeModel(pyramid=linear_pyramid(1190, 12, 6)).status == ot.OK
     assert FakeModel(H=3).status == ot.ERR_SHAPE                  # d % H
-    assert FakeModel(H=16).status == ot.ERR_UNSUPPORTED           # d_h = 16
+    assert FakeModel(H=32).status == ot.ERR_UNSUPPORTED           # d_h = 8
     assert FakeModel(page=32).status == ot.ERR_UNSUPPORTED
     assert FakeModel(mode=7).status == ot.ERR_INVALID_ARG
     assert FakeModel(null_field="W2_NS").status == ot.ERR_INVALID_ARG

@@ -20,11 +20,14 @@ enum Act : int { ACT_NONE = 0, ACT_GELU = 1 };
 
 // Address of element (b, t, n) = base + b*sb + t*st + (n / split)*sc + n % split
 // (in elements).  `split` lets one GEMM write column blocks to separate
-// planes (the token-major output of the auto-split tokenizer).
+// planes (the token-major output of the auto-split tokenizer).  `f32` marks
+// a float32 tensor (the residual stream and the stack's outputs); otherwise
+// the element type is the model's storage type.
 struct RowMap {
   void* base;
   long long sb, st, sc;
   int split;
+  int f32;
 };
 
 // Paged K/V store.  A page holds P tokens of one (sequence, layer) laid out as
@@ -36,6 +39,7 @@ struct KVStore {
   const int* row_off;
   int P, H, dh, pps;
   int pos_off;  // written position = t + pos_off
+  int n_pages;  // pages in the pool (extent of the page dimension)
 };
 
 struct GemmDesc {
@@ -99,6 +103,14 @@ template <> __device__ inline float to_f<__nv_bfloat16>(__nv_bfloat16 v) { retur
 template <typename T> __device__ inline T from_f(float v);
 template <> __device__ inline float from_f<float>(float v) { return v; }
 template <> __device__ inline __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+template <typename T> __device__ inline float rm_load(const RowMap& r, long long off) {
+  return r.f32 ? ((const float*)r.base)[off] : to_f(((const T*)r.base)[off]);
+}
+template <typename T> __device__ inline void rm_store(const RowMap& r, long long off, float v) {
+  if (r.f32) ((float*)r.base)[off] = v;
+  else ((T*)r.base)[off] = from_f<T>(v);
+}
 
 // GELU, tanh form (Hendrycks & Gimpel): 0.5 x (1 + tanh(sqrt(2/pi)(x + 0.044715 x^3)))
 __device__ inline float gelu_tanh(float x) {

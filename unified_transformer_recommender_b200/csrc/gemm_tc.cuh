@@ -1,6 +1,270 @@
+// Tensor-core GEMM with fused epilogues for the bf16 path (sm_100a).
+//
+//   C[(b,t), n] = epi( sum_k A[(m,g), k] * W[grp][n_lo + n][k] )
+//
+// One CTA computes a 128 x BN output tile.  A and W tiles (64 bf16 of K per
+// row, 128-byte swizzle) are streamed by TMA through a STAGES-deep ring of
+// shared-memory buffers guarded by mbarriers; one thread issues tcgen05.mma
+// (M = 128, N = BN or BN/2, K = 16) into an fp32 accumulator in TMEM; four
+// epilogue warps read the accumulator back with tcgen05.ld (one output row
+// per thread) and apply bias, GELU, residual, the paged K/V store and the
+// RMSNorm of the finished row (when the CTA owns the whole row, BN == N).
+//
+// Warp roles (192 threads): warps 0-3 epilogue, warp 4 TMA producer,
+// warp 5 TMEM allocator and MMA issuer.
 #pragma once
-#include "common.cuh"
+#include <cudaTypedefs.h>
+#include "tc_ptx.cuh"
+
 namespace ot {
-inline bool tc_gemm_supported(const GemmDesc&) { return false; }
-inline onetrans_status tc_gemm_launch(const GemmDesc&, cudaStream_t) { return ONETRANS_ERR_UNSUPPORTED; }
+
+template <int BN>
+struct TcGemmCfg {
+  static constexpr int UN = BN <= 256 ? BN : BN / 2;  // N of one tcgen05.mma
+  static constexpr int NSUB = BN / UN;
+  static constexpr int BOX_N = BN <= 256 ? BN : BN / 2;  // TMA box rows of W (<= 256)
+  static constexpr int STAGES = BN <= 256 ? 4 : 3;
+  static constexpr int A_BYTES = 128 * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = BN <= 128 ? 128 : (BN <= 256 ? 256 : 512);
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmDesc d, const int a_swap) {
+  using C = TcGemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint32_t* tmem_slot = (uint32_t*)(accf + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN;
+  const int mt0 = d.m_lo + blockIdx.y * 128;
+  const int g = d.g_lo + blockIdx.z;
+  const int grp = d.mode == TILE_SAMPLES ? g - d.grp_base : 0;
+  const int KB = d.K / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 5) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % C::STAGES;
+        const uint32_t ph = (kb / C::STAGES) & 1;
+        if (kb >= C::STAGES && !mbar_wait(&empty[s], ph ^ 1)) break;
+        uint8_t* sa = smem + s * C::STAGE_BYTES;
+        uint8_t* sb = sa + C::A_BYTES;
+        mbar_expect_tx(&full[s], C::STAGE_BYTES);
+        if (a_swap) tma_load_3d(&tmA, &full[s], sa, kb * 64, g, mt0);
+        else tma_load_3d(&tmA, &full[s], sa, kb * 64, mt0, g);
+#pragma unroll
+        for (int c = 0; c < BN / C::BOX_N; ++c)
+          tma_load_3d(&tmB, &full[s], sb + c * C::BOX_N * 128, kb * 64, d.n_lo + n0 + c * C::BOX_N, grp);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, C::UN);
+      bool ok = true;
+      for (int kb = 0; kb < KB && ok; ++kb) {
+        const int s = kb % C::STAGES;
+        const uint32_t ph = (kb / C::STAGES) & 1;
+        ok = mbar_wait(&full[s], ph);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+        const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = sdesc_k128(sa + k * 32);
+#pragma unroll
+          for (int j = 0; j < C::NSUB; ++j)
+            umma_bf16(tmem + j * C::UN, ad, sdesc_k128(sb + j * C::UN * 128 + k * 32), idesc,
+                      (kb | k) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const bool done = mbar_wait(accf, 0);
+    tc_fence_after();
+    const int r = warp * 32 + lane;
+    const int m = mt0 + r;
+    const bool valid = done && m < d.m_lo + d.M;
+    int b = 0, t = 0;
+    if (valid) row_of(d, m, g, b, t);
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const __nv_bfloat16* bias = (const __nv_bfloat16*)d.bias;
+    float ss = 0.f;
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+      float v[32];
+      tmem_ld32(trow + c0, v);
+      if (!valid) continue;
+      const int n = n0 + c0;
+      if (bias) {
+        float bv[32];
+        load_bf16x32(bias + (long long)grp * d.bias_sg + d.n_lo + n, bv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] += bv[i];
+      }
+      if (d.act == ACT_GELU) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+      }
+      if (d.res.base) {
+        float rv[32];
+        load_row32(d.res, rm_off(d.res, b, t, n), rv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] += rv[i];
+      }
+      if (d.out_kind == OUT_KV) {
+        const int dm = d.kv.H * d.kv.dh;
+        const int kind = n / dm, cc = n - kind * dm, head = cc / d.kv.dh, e = cc - head * d.kv.dh;
+        store_bf16x32((__nv_bfloat16*)d.kv.pool + kv_off(d.kv, b, t + d.kv.pos_off, kind, head, e), v);
+      } else {
+        store_row32(d.out, rm_off(d.out, b, t, n), v);
+      }
+      if (d.rms.base) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float q = d.out.f32 ? v[i] : __bfloat162float(__float2bfloat16_rn(v[i]));
+          ss += q * q;
+        }
+      }
+    }
+    if (valid && d.rms.base) {
+      // the CTA owns the whole row (BN == N): normalise the stored row
+      const float rr = rsqrtf(ss / d.N + d.eps);
+      const __nv_bfloat16* gm = (const __nv_bfloat16*)d.gamma;
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32], gv[32];
+        load_row32(d.out, rm_off(d.out, b, t, c0), v);
+        load_bf16x32(gm + c0, gv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = v[i] * rr * gv[i];
+        store_row32(d.rms, rm_off(d.rms, b, t, c0), v);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
 }
+
+// ------------------------------------------------------------------ host --
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map: dims (inner, d1, d2), strides in elements for d1, d2.
+inline bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t d1, uint64_t d2,
+                         uint64_t s1, uint64_t s2, uint32_t box0, uint32_t box1, uint32_t box2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {inner, d1, d2};
+  const cuuint64_t strides[2] = {s1 * 2, s2 * 2};
+  const cuuint32_t box[3] = {box0, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int tc_pick_bn(const GemmDesc& d) {
+  if (d.rms.base) return (d.N == 128 || d.N == 256 || d.N == 384) ? d.N : 0;
+  if (d.N % 256 == 0) return 256;
+  if (d.N % 384 == 0) return 384;
+  if (d.N % 128 == 0) return 128;
+  return 0;
+}
+
+inline bool rowmap_vec_ok(const RowMap& r) {
+  return ((uintptr_t)r.base % 16) == 0 && r.sb % 8 == 0 && r.st % 8 == 0 && r.sc % 8 == 0 && r.split % 32 == 0;
+}
+
+inline bool tc_gemm_supported(const GemmDesc& d) {
+  if (d.K <= 0 || d.K % 64 || !tc_pick_bn(d)) return false;
+  if ((uintptr_t)d.A % 16 || (uintptr_t)d.W % 16) return false;
+  if (d.a_sm % 8 || d.a_sg % 8 || d.w_sg % 8) return false;
+  if (d.bias && ((d.bias_sg % 8) || (d.n_lo % 8) || ((uintptr_t)d.bias % 16))) return false;
+  if (d.res.base && !rowmap_vec_ok(d.res)) return false;
+  if (d.rms.base && (!rowmap_vec_ok(d.rms) || (uintptr_t)d.gamma % 16)) return false;
+  if (d.out_kind == OUT_KV) {
+    if (d.kv.dh % 32 || (uintptr_t)d.kv.pool % 16) return false;
+  } else if (!rowmap_vec_ok(d.out)) {
+    return false;
+  }
+  return encode_fn() != nullptr;
+}
+
+template <int BN>
+inline onetrans_status tc_gemm_launch_bn(const GemmDesc& d, cudaStream_t st) {
+  using C = TcGemmCfg<BN>;
+  CUtensorMap ta, tb;
+  const uint64_t mext = (uint64_t)d.a_mext, gext = (uint64_t)d.a_gext;
+  const uint64_t s_m = (uint64_t)d.a_sm, s_g = gext > 1 ? (uint64_t)d.a_sg : mext * (uint64_t)d.a_sm;
+  const int a_swap = (gext > 1 && d.a_sg < d.a_sm) ? 1 : 0;
+  bool ok = a_swap ? make_tmap_3d(&ta, d.A, d.K, gext, mext, s_g, s_m, 64, 1, 128)
+                   : make_tmap_3d(&ta, d.A, d.K, mext, gext, s_m, s_g, 64, 128, 1);
+  const uint64_t wg = (uint64_t)d.w_groups;
+  const uint64_t w_sg = wg > 1 ? (uint64_t)d.w_sg : (uint64_t)d.w_rows * d.K;
+  ok = ok && make_tmap_3d(&tb, d.W, d.K, d.w_rows, wg, d.K, w_sg, 64, C::BOX_N, 1);
+  if (!ok) return ONETRANS_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+      return ONETRANS_ERR_CUDA;
+    attr_set = true;
+  }
+  dim3 grid((unsigned)(d.N / BN), (unsigned)((d.M + 127) / 128), (unsigned)d.G);
+  gemm_tc_kernel<BN><<<grid, 192, C::SMEM, st>>>(ta, tb, d, a_swap);
+  return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
+}
+
+inline onetrans_status tc_gemm_launch(const GemmDesc& d, cudaStream_t st) {
+  switch (tc_pick_bn(d)) {
+    case 128: return tc_gemm_launch_bn<128>(d, st);
+    case 256: return tc_gemm_launch_bn<256>(d, st);
+    case 384: return tc_gemm_launch_bn<384>(d, st);
+    default: return ONETRANS_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace ot

@@ -110,6 +110,13 @@ static RowMap rmap(const void* base, long long sb, long long st) {
   r.st = st;
   r.sc = 0;
   r.split = 1 << 30;
+  r.f32 = 0;
+  return r;
+}
+// Map over a float32 tensor (residual stream, stack outputs).
+static RowMap rmap32(const void* base, long long sb, long long st) {
+  RowMap r = rmap(base, sb, st);
+  r.f32 = 1;
   return r;
 }
 
@@ -155,6 +162,7 @@ static onetrans_status launch_attn(const onetrans_model* m, const AttnDesc& a, c
   if (m->bf16 && g_policy == 0 && tc_attn_supported(a)) return tc_attn_launch(a, st);
   dim3 grid((unsigned)cdiv(a.Lq, 64), (unsigned)a.H, (unsigned)a.B);
   switch (a.dh) {
+    case 16: attn_simt_kernel<T, 16><<<grid, 64, 0, st>>>(a); break;
     case 32: attn_simt_kernel<T, 32><<<grid, 64, 0, st>>>(a); break;
     case 64: attn_simt_kernel<T, 64><<<grid, 64, 0, st>>>(a); break;
     case 96: attn_simt_kernel<T, 96><<<grid, 64, 0, st>>>(a); break;
@@ -170,6 +178,7 @@ static onetrans_status launch_stage2_attn(const onetrans_model* m, const Stage2D
   if (n_tiles <= 0) return ONETRANS_OK;
   dim3 grid((unsigned)n_tiles, (unsigned)a.H, (unsigned)a.L_NS);
   switch (a.dh) {
+    case 16: stage2_attn_simt_kernel<T, 16><<<grid, 64, 0, st>>>(a); break;
     case 32: stage2_attn_simt_kernel<T, 32><<<grid, 64, 0, st>>>(a); break;
     case 64: stage2_attn_simt_kernel<T, 64><<<grid, 64, 0, st>>>(a); break;
     case 96: stage2_attn_simt_kernel<T, 96><<<grid, 64, 0, st>>>(a); break;
@@ -181,14 +190,14 @@ static onetrans_status launch_stage2_attn(const onetrans_model* m, const Stage2D
 
 // RMSNorm of `rows` contiguous rows of width d: dst = RMS(src) * gamma.
 template <typename T>
-static onetrans_status rms_flat(const onetrans_model* m, const void* src, void* dst, long long rows,
-                                const void* gamma, cudaStream_t st) {
+static onetrans_status rms_flat(const onetrans_model* m, const void* src, bool src_f32, void* dst,
+                                long long rows, const void* gamma, cudaStream_t st) {
   GemmDesc d = gdesc_base(m);
   d.mode = TILE_FLAT;
   d.M = (int)rows;
   d.G = 1;
   d.N = m->d;
-  d.out = rmap(src, 0, m->d);
+  d.out = src_f32 ? rmap32(src, 0, m->d) : rmap(src, 0, m->d);
   d.rms = rmap(dst, 0, m->d);
   d.gamma = gamma;
   return launch_rms<T>(d, st);
@@ -204,12 +213,12 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
   const int L0 = L_S + L_NS, Lq1 = Lq[0];
   const long long pps = cdiv(L0, P);
   Carve cv(ws, ws_bytes);
-  void* xa = cv.take((size_t)B * Lq1 * d * es);
-  void* xb = cv.take((size_t)B * Lq1 * d * es);
+  void* xa = cv.take((size_t)B * Lq1 * d * 4);   // residual stream: float32
+  void* xb = cv.take((size_t)B * Lq1 * d * 4);
   void* h = cv.take((size_t)B * L0 * d * es);
   void* q = cv.take((size_t)B * Lq1 * d * es);
   void* at = cv.take((size_t)B * Lq1 * d * es);
-  void* xm = cv.take((size_t)B * Lq1 * d * es);
+  void* xm = cv.take((size_t)B * Lq1 * d * 4);
   void* h2 = cv.take((size_t)B * Lq1 * d * es);
   void* hid = cv.take((size_t)B * Lq1 * dff * es);
   void* kvb = cv.take((size_t)B * pps * 2 * d * P * es);
@@ -218,9 +227,9 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
 
   KVStore kv;
   std::memset(&kv, 0, sizeof(kv));
-  kv.pool = kvb; kv.P = P; kv.H = m->H; kv.dh = m->dh; kv.pps = (int)pps;
+  kv.pool = kvb; kv.P = P; kv.H = m->H; kv.dh = m->dh; kv.pps = (int)pps; kv.n_pages = (int)(B * pps);
 
-  OT_TRY(rms_flat<T>(m, x0, h, (long long)B * L0, m->g_attn[0], st));
+  OT_TRY(rms_flat<T>(m, x0, false, h, (long long)B * L0, m->g_attn[0], st));
   const void* x_in = x0;
   int L = L0;
   for (int n = 0; n < m->NL; ++n) {
@@ -262,8 +271,9 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
     go.mode = TILE_FLAT; go.M = B * Lqn; go.fold = Lqn; go.G = 1;
     go.K = d; go.A = at; go.a_sm = d; go.a_mext = (long long)B * Lqn; go.a_gext = 1;
     go.W = m->Wo[n]; go.w_rows = d; go.N = d;
-    go.res = rmap(eoff(x_in, (long long)off * d, es), (long long)L * d, d);
-    go.out = rmap(xm, (long long)Lqn * d, d);
+    go.res = n == 0 ? rmap(eoff(x_in, (long long)off * d, es), (long long)L * d, d)
+                    : rmap32(eoff(x_in, (long long)off * d, 4), (long long)L * d, d);
+    go.out = rmap32(xm, (long long)Lqn * d, d);
     go.rms = rmap(h2, (long long)Lqn * d, d);
     go.gamma = m->g_ffn[n];
     OT_TRY(launch_gemm<T>(m, go, st));
@@ -292,8 +302,8 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
       f2.W = part ? m->W2_NS[n] : m->W2_S[n]; f2.w_rows = d; f2.N = d;
       f2.w_sg = part ? (long long)d * dff : 0;
       f2.bias = part ? m->b2_NS[n] : m->b2_S[n]; f2.bias_sg = part ? d : 0;
-      f2.res = rmap(xm, (long long)Lqn * d, d);
-      f2.out = rmap(x_next, (long long)Lqn * d, d);
+      f2.res = rmap32(xm, (long long)Lqn * d, d);
+      f2.out = rmap32(x_next, (long long)Lqn * d, d);
       if (!last) { f2.rms = rmap(h, (long long)Lqn * d, d); f2.gamma = m->g_attn[n + 1]; }
       OT_TRY(launch_gemm<T>(m, f2, st));
     }
@@ -312,6 +322,7 @@ static void kv_for_cache(const onetrans_cache* c, int layer, const int* d_row_of
   kv.P = c->m->cfg.page_tokens;
   kv.H = c->m->H;
   kv.dh = c->m->dh;
+  kv.n_pages = c->n_pages;
 }
 
 static onetrans_status upload_slot_table(onetrans_cache* c, int slot, cudaStream_t st) {
@@ -329,12 +340,12 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
   const int d = m->d, dff = m->dff, es = m->es;
   const int sq1 = std::max(sq[0], 0);
   Carve cv(ws, ws_bytes);
-  void* xa = cv.take((size_t)U * sq1 * d * es);
-  void* xb = cv.take((size_t)U * sq1 * d * es);
+  void* xa = cv.take((size_t)U * sq1 * d * 4);   // residual stream: float32
+  void* xb = cv.take((size_t)U * sq1 * d * 4);
   void* h = cv.take((size_t)U * L_S * d * es);
   void* q = cv.take((size_t)U * sq1 * d * es);
   void* at = cv.take((size_t)U * sq1 * d * es);
-  void* xm = cv.take((size_t)U * sq1 * d * es);
+  void* xm = cv.take((size_t)U * sq1 * d * 4);
   void* h2 = cv.take((size_t)U * sq1 * d * es);
   void* hid = cv.take((size_t)U * sq1 * dff * es);
   int* row_off = (int*)cv.take((size_t)U * sizeof(int));
@@ -369,7 +380,7 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
   }
   OT_TRY(cuda_ok(cudaMemcpyAsync(row_off, h_row_off.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
 
-  OT_TRY(rms_flat<T>(m, s_tok, h, (long long)U * L_S, m->g_attn[0], st));
+  OT_TRY(rms_flat<T>(m, s_tok, false, h, (long long)U * L_S, m->g_attn[0], st));
   const void* x_in = s_tok;
   for (int n = 0; n < m->NL; ++n) {
     const int sn = s[n], sqn = sq[n];
@@ -402,8 +413,9 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
     go.mode = TILE_FLAT; go.M = U * sqn; go.fold = sqn; go.G = 1;
     go.K = d; go.A = at; go.a_sm = d; go.a_mext = (long long)U * sqn; go.a_gext = 1;
     go.W = m->Wo[n]; go.w_rows = d; go.N = d;
-    go.res = rmap(eoff(x_in, (long long)(sn - sqn) * d, es), (long long)sn * d, d);
-    go.out = rmap(xm, (long long)sqn * d, d);
+    go.res = n == 0 ? rmap(eoff(x_in, (long long)(sn - sqn) * d, es), (long long)sn * d, d)
+                    : rmap32(eoff(x_in, (long long)(sn - sqn) * d, 4), (long long)sn * d, d);
+    go.out = rmap32(xm, (long long)sqn * d, d);
     go.rms = rmap(h2, (long long)sqn * d, d);
     go.gamma = m->g_ffn[n];
     OT_TRY(launch_gemm<T>(m, go, st));
@@ -415,8 +427,8 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
     GemmDesc f2 = go;
     f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.W = m->W2_S[n]; f2.w_rows = d; f2.N = d;
     f2.bias = m->b2_S[n];
-    f2.res = rmap(xm, (long long)sqn * d, d);
-    f2.out = rmap(x_next, (long long)sqn * d, d);
+    f2.res = rmap32(xm, (long long)sqn * d, d);
+    f2.out = rmap32(x_next, (long long)sqn * d, d);
     f2.rms = rmap(h, (long long)sqn * d, d);
     f2.gamma = m->g_attn[n + 1];
     OT_TRY(launch_gemm<T>(m, f2, st));
@@ -446,12 +458,12 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     max_tiles = (long long)tiles.size() / 3;
   }
   Carve cv(ws, ws_bytes);
-  void* xa = cv.take((size_t)L_NS * C * d * es);
-  void* xb = cv.take((size_t)L_NS * C * d * es);
+  void* xa = cv.take((size_t)L_NS * C * d * 4);   // residual stream: float32
+  void* xb = cv.take((size_t)L_NS * C * d * 4);
   void* h = cv.take((size_t)L_NS * C * d * es);
   void* qkv = cv.take((size_t)L_NS * C * 3 * d * es);
   void* at = cv.take((size_t)L_NS * C * d * es);
-  void* xm = cv.take((size_t)L_NS * C * d * es);
+  void* xm = cv.take((size_t)L_NS * C * d * 4);
   void* h2 = cv.take((size_t)L_NS * C * d * es);
   void* hid = cv.take((size_t)L_NS * C * dff * es);
   int* row_off = (int*)cv.take((size_t)kMaxUsers * sizeof(int));
@@ -465,7 +477,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   OT_TRY(cuda_ok(cudaMemcpyAsync(row_off, h_row_off.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
   OT_TRY(cuda_ok(cudaMemcpyAsync(d_tiles, tiles.data(), tiles.size() * sizeof(int), cudaMemcpyHostToDevice, st)));
 
-  OT_TRY(rms_flat<T>(m, ns_in, h, (long long)L_NS * C, m->g_attn[0], st));
+  OT_TRY(rms_flat<T>(m, ns_in, false, h, (long long)L_NS * C, m->g_attn[0], st));
   const void* x_in = ns_in;
   for (int n = 0; n < m->NL; ++n) {
     const bool last = n + 1 == m->NL;
@@ -488,8 +500,8 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     go.mode = TILE_FLAT; go.M = (int)(L_NS * C); go.G = 1;
     go.K = d; go.A = at; go.a_sm = d; go.a_mext = L_NS * C; go.a_gext = 1;
     go.W = m->Wo[n]; go.w_rows = d; go.N = d;
-    go.res = rmap(x_in, 0, d);
-    go.out = rmap(xm, 0, d);
+    go.res = n == 0 ? rmap(x_in, 0, d) : rmap32(x_in, 0, d);
+    go.out = rmap32(xm, 0, d);
     go.rms = rmap(h2, 0, d);
     go.gamma = m->g_ffn[n];
     OT_TRY(launch_gemm<T>(m, go, st));
@@ -502,8 +514,8 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.a_sg = C * dff;
     f2.W = m->W2_NS[n]; f2.w_sg = (long long)d * dff; f2.w_rows = d; f2.N = d;
     f2.bias = m->b2_NS[n]; f2.bias_sg = d;
-    f2.res = rmap(xm, d, C * d);
-    f2.out = rmap(x_next, d, C * d);
+    f2.res = rmap32(xm, d, C * d);
+    f2.out = rmap32(x_next, d, C * d);
     if (!last) { f2.rms = rmap(h, d, C * d); f2.gamma = m->g_attn[n + 1]; }
     OT_TRY(launch_gemm<T>(m, f2, st));
     x_in = x_next;
@@ -519,12 +531,12 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
   const int d = m->d, dff = m->dff, es = m->es, P = m->cfg.page_tokens;
   Carve cv(ws, ws_bytes);
   const long long R = (long long)U * dL;
-  void* xa = cv.take((size_t)R * d * es);
-  void* xb = cv.take((size_t)R * d * es);
+  void* xa = cv.take((size_t)R * d * 4);   // residual stream: float32
+  void* xb = cv.take((size_t)R * d * 4);
   void* h = cv.take((size_t)R * d * es);
   void* q = cv.take((size_t)R * d * es);
   void* at = cv.take((size_t)R * d * es);
-  void* xm = cv.take((size_t)R * d * es);
+  void* xm = cv.take((size_t)R * d * 4);
   void* h2 = cv.take((size_t)R * d * es);
   void* hid = cv.take((size_t)R * dff * es);
   int* row_off = (int*)cv.take((size_t)std::max(U, 1) * sizeof(int));
@@ -560,9 +572,9 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
   w.emb = m->type_emb; w.n_types = m->cfg.n_behaviors; w.e_dim = m->cfg.event_dim; w.d = d;
   const size_t smem = (size_t)(w.e_dim + d) * sizeof(float);
   event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>((const T*)events, types, dL, w,
-                                                                         rmap(xa, (long long)dL * d, d));
+                                                                         rmap32(xa, (long long)dL * d, d));
   OT_TRY(last_launch());
-  OT_TRY(rms_flat<T>(m, xa, h, R, m->g_attn[0], st));
+  OT_TRY(rms_flat<T>(m, xa, true, h, R, m->g_attn[0], st));
   const void* x_in = xa;
   for (int n = 0; n < m->NL; ++n) {
     const bool last = n + 1 == m->NL;
@@ -591,8 +603,8 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     go.mode = TILE_FLAT; go.M = (int)R; go.fold = dL; go.G = 1;
     go.K = d; go.A = at; go.a_sm = d; go.a_mext = R; go.a_gext = 1;
     go.W = m->Wo[n]; go.w_rows = d; go.N = d;
-    go.res = rmap(x_in, (long long)dL * d, d);
-    go.out = rmap(xm, (long long)dL * d, d);
+    go.res = rmap32(x_in, (long long)dL * d, d);
+    go.out = rmap32(xm, (long long)dL * d, d);
     go.rms = rmap(h2, (long long)dL * d, d);
     go.gamma = m->g_ffn[n];
     OT_TRY(launch_gemm<T>(m, go, st));
@@ -604,8 +616,8 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     GemmDesc f2 = go;
     f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.W = m->W2_S[n]; f2.w_rows = d; f2.N = d;
     f2.bias = m->b2_S[n];
-    f2.res = rmap(xm, (long long)dL * d, d);
-    f2.out = rmap(x_next, (long long)dL * d, d);
+    f2.res = rmap32(xm, (long long)dL * d, d);
+    f2.out = rmap32(x_next, (long long)dL * d, d);
     f2.rms = rmap(h, (long long)dL * d, d);
     f2.gamma = m->g_attn[n + 1];
     OT_TRY(launch_gemm<T>(m, f2, st));
@@ -672,7 +684,7 @@ onetrans_status onetrans_model_create(const onetrans_config* cfg, const onetrans
     return ONETRANS_ERR_SHAPE;
   if (d % H) return ONETRANS_ERR_SHAPE;
   const int dh = d / H;
-  if (dh != 32 && dh != 64 && dh != 96 && dh != 128) return ONETRANS_ERR_UNSUPPORTED;
+  if (dh != 16 && dh != 32 && dh != 64 && dh != 96 && dh != 128) return ONETRANS_ERR_UNSUPPORTED;
   if (cfg->mode != ONETRANS_BF16 && cfg->mode != ONETRANS_FP32) return ONETRANS_ERR_INVALID_ARG;
   if (cfg->page_tokens != 64) return ONETRANS_ERR_UNSUPPORTED;
   if (!(cfg->rms_eps > 0.f)) return ONETRANS_ERR_INVALID_ARG;

@@ -13,13 +13,13 @@ template <typename T>
 __device__ inline void epilogue_store(const GemmDesc& d, int b, int t, int n, int grp, float v) {
   if (d.bias) v += to_f(((const T*)d.bias)[grp * d.bias_sg + d.n_lo + n]);
   if (d.act == ACT_GELU) v = gelu_tanh(v);
-  if (d.res.base) v += to_f(((const T*)d.res.base)[rm_off(d.res, b, t, n)]);
+  if (d.res.base) v += rm_load<T>(d.res, rm_off(d.res, b, t, n));
   if (d.out_kind == OUT_KV) {
     const int dm = d.kv.H * d.kv.dh;
     const int kind = n / dm, c = n - kind * dm, head = c / d.kv.dh, e = c - head * d.kv.dh;
     ((T*)d.kv.pool)[kv_off(d.kv, b, t + d.kv.pos_off, kind, head, e)] = from_f<T>(v);
   } else {
-    ((T*)d.out.base)[rm_off(d.out, b, t, n)] = from_f<T>(v);
+    rm_store<T>(d.out, rm_off(d.out, b, t, n), v);
   }
 }
 
@@ -79,11 +79,9 @@ __global__ void rms_rows_kernel(GemmDesc d) {
   if (m >= d.m_lo + d.M) return;
   int b, t;
   row_of(d, m, g, b, t);
-  const T* src = (const T*)d.out.base;
-  T* dst = (T*)d.rms.base;
   float ss = 0.f;
   for (int n = lane; n < d.N; n += 32) {
-    const float v = to_f(src[rm_off(d.out, b, t, n)]);
+    const float v = rm_load<T>(d.out, rm_off(d.out, b, t, n));
     ss += v * v;
   }
 #pragma unroll
@@ -91,8 +89,8 @@ __global__ void rms_rows_kernel(GemmDesc d) {
   const float r = rsqrtf(ss / d.N + d.eps);
   const T* gm = (const T*)d.gamma;
   for (int n = lane; n < d.N; n += 32) {
-    const float v = to_f(src[rm_off(d.out, b, t, n)]);
-    dst[rm_off(d.rms, b, t, n)] = from_f<T>(v * r * to_f(gm[n]));
+    const float v = rm_load<T>(d.out, rm_off(d.out, b, t, n));
+    rm_store<T>(d.rms, rm_off(d.rms, b, t, n), v * r * to_f(gm[n]));
   }
 }
 
@@ -283,7 +281,7 @@ __global__ void event_tokenize_kernel(const T* ev, const int* types, int dL, Eve
     float s = to_f(((const T*)w.b2[ty])[k]);
     for (int i = 0; i < w.d; ++i) s = fmaf(to_f(W2[(long long)k * w.d + i]), hid[i], s);
     s += to_f(((const T*)w.emb)[(long long)ty * w.d + k]);
-    ((T*)out.base)[rm_off(out, b, t, k)] = from_f<T>(s);
+    rm_store<T>(out, rm_off(out, b, t, k), s);
   }
 }
 
