@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Throughput of the OneTrans hot path on B200: candidates scored per second
+(Stage II over the KV cache) and users encoded per second (Stage I).
+
+One step = auto-split tokenization of every candidate's NS features, Stage I
+of every user's S tokens into the paged KV cache, and Stage II scoring of
+every candidate against its user's cache, all through the C ABI.  Workload
+(default): 6 layers, d=256, 4 heads, FFN 1024, 12 NS tokens, L_S = 1178,
+pyramid query counts 1190 -> 12 (linear), 16 users x 512 candidates, NS
+features 512 wide, bf16 storage.  Other workloads: --workload append (non-
+pyramid cross-request append of 16 events for 256 users, then 128
+candidates each), s_forward / l_forward (one-pass forward).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank serves its own users: no data
+moves between ranks, work per GPU is fixed (weak scaling), the device time
+is the max over ranks.  `--impl reference` times the fp64 CPU oracle on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "candidates scored/sec (Stage II, KV-cached) and users/sec (Stage I) on 1 B200"
+UNIT = "candidates/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="kv_serving",
+                    choices=("kv_serving", "append", "s_forward", "l_forward"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------- dist utils
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def shard_users(n_users_per_rank: int, rank: int):
+    """User ids served by `rank`: a contiguous block of n_users_per_rank.
+    Every rank holds the same count (weak scaling) and no id repeats."""
+    return list(range(rank * n_users_per_rank, (rank + 1) * n_users_per_rank))
+
+
+def max_over_ranks(value: float, pg=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons while the
+    timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[3]) if v.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------- workload
+
+class KVServing:
+    """Auto-split + Stage I + Stage II for U users x C candidates."""
+
+    def __init__(self, rank: int, wl_name: str = "kv_serving"):
+        import torch
+        import unified_transformer_recommender_b200 as ot
+        from onetrans_synth import WORKLOADS, gen_normal, make_weights
+        self.ot, self.torch = ot, torch
+        wl = WORKLOADS[wl_name]
+        self.wl, sh = wl, wl.shape
+        self.U, self.C = wl.users, wl.cands
+        self.W = make_weights(sh, wl.seed_weights, wl.dtype)
+        self.model = ot.model_from_arrays(sh, self.W, pyramid_q=list(wl.pyramid), mode=ot.BF16)
+        seed = wl.seed_inputs + 7919 * rank     # each rank serves different users
+        self.S_h = gen_normal(seed, (self.U, wl.L_S, sh.d), "bf16")
+        self.F_h = gen_normal(seed + 100, (self.U * self.C, sh.ns_feat), "bf16")
+        dev = torch.device("cuda")
+        self.S = torch.from_numpy(self.S_h).to(dev, torch.bfloat16)
+        self.F = torch.from_numpy(self.F_h).to(dev, torch.bfloat16)
+        # pinned host copies for the end-to-end leg
+        self.S_pin = torch.from_numpy(self.S_h).to(torch.bfloat16).pin_memory()
+        self.F_pin = torch.from_numpy(self.F_h).to(torch.bfloat16).pin_memory()
+        m = self.model
+        self.ns = torch.empty(sh.L_NS, self.U * self.C, sh.d, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(sh.L_NS, self.U * self.C, sh.d, dtype=torch.float32, device=dev)
+        self.out_pin = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        self.ws_a = m.workspace(ot.OP_AUTOSPLIT, self.U * self.C)
+        self.ws_1 = m.workspace(ot.OP_STAGE1, self.U, wl.L_S)
+        self.ws_2 = m.workspace(ot.OP_STAGE2, self.U * self.C, wl.L_S)
+        self.cache = ot.Cache(m, self.U, wl.L_S)
+        self.slots = list(range(self.U))
+        self.offs = [u * self.C for u in range(self.U + 1)]
+        self.units = self.U * self.C
+        self.h2d = self.S_h.size * 2 + self.F_h.size * 2
+        self.d2h = self.out.numel() * 4
+
+    def step(self, ev_mid=None, S=None, F=None):
+        ot, m = self.ot, self.model
+        S = self.S if S is None else S
+        F = self.F if F is None else F
+        ot.onetrans_stage1_encode(m, self.cache, self.slots, S, self.ws_1)
+        if ev_mid is not None:
+            ev_mid.record()
+        ot.onetrans_tokenize_autosplit(m, F, self.ns, self.ws_a)
+        ot.onetrans_stage2_score(m, self.cache, self.slots, self.offs, self.ns, self.out, self.ws_2)
+
+    def e2e_step(self):
+        """Inputs from pinned host memory, result back to pinned host memory."""
+        self.S.copy_(self.S_pin, non_blocking=True)
+        self.F.copy_(self.F_pin, non_blocking=True)
+        self.step()
+        self.out_pin.copy_(self.out, non_blocking=True)
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_sample(n_cands: int = 160, seed_shift: int = 0):
+    """Time the fp64 oracle on 1 user's Stage I plus n_cands candidates'
+    auto-split and Stage II; returns (candidates/s of the full workload by
+    linear extrapolation, sample description, threads used)."""
+    from onetrans_synth import WORKLOADS, gen_normal, make_weights
+    from oracle import onetrans as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    wl = WORKLOADS["kv_serving"]
+    sh = wl.shape
+    W = make_weights(sh, wl.seed_weights, "bf16")
+    S = gen_normal(wl.seed_inputs + seed_shift, (1, wl.L_S, sh.d), "bf16")
+    F = gen_normal(wl.seed_inputs + 100 + seed_shift, (n_cands, sh.ns_feat), "bf16")
+    t0 = time.perf_counter()
+    kv = O.stage1(S[0], W, sh.L_NS, sh.n_heads, sh.eps, wl.pyramid)
+    t1 = time.perf_counter()
+    ns = O.autosplit(F, W, sh.L_NS)
+    for c in range(n_cands):
+        O.stage2(kv, ns[c], W, sh.n_heads, sh.eps)
+    t2 = time.perf_counter()
+    per_user, per_cand = t1 - t0, (t2 - t1) / n_cands
+    step_s = wl.users * per_user + wl.users * wl.cands * per_cand
+    desc = (f"oracle fp64: Stage I of 1 user ({per_user:.2f} s) + auto-split and Stage II of {n_cands} "
+            f"candidates ({per_cand * 1e3:.1f} ms each), extrapolated linearly to {wl.users} users x "
+            f"{wl.cands} candidates ({step_s:.0f} s per step)")
+    return wl.users * wl.cands / step_s, desc, cores, t2 - t0
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    vals, samples = [], None
+    for i in range(args.warmup + args.steps):
+        v, desc, cores, secs = oracle_sample(n_cands=8, seed_shift=i)
+        if i >= args.warmup:
+            vals.append(v)
+            samples = desc
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * 8192 / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "kv_serving: 6x256 pyramid 1190->12, 16 users x 1178 S "
+                                                    "tokens, 512 candidates/user, 12 NS tokens from 512 features"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": samples},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    import torch
+    import torch.distributed as dist
+    if ws > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    import unified_transformer_recommender_b200 as ot
+
+    if args.workload != "kv_serving":
+        raise SystemExit("bench.py times the kv_serving workload; other workloads: tests/")
+    wk = KVServing(rank)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")   # > 126 MB L2
+    st = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        wk.step()
+    torch.cuda.synchronize()
+    assert ot.onetrans_device_status() == 0
+
+    # ---- device-timed region: inputs resident in HBM; L2 flushed between steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    ot.onetrans_profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(st)
+        wk.step(ev_mid=evs[i][1])
+        evs[i][2].record(st)
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - t_wall
+    clk = clocks.stop()
+    prof = ot.onetrans_profile_read()
+    ot.onetrans_profile_enable(False)
+    step_ms = [a.elapsed_time(c) for a, _, c in evs]
+    s1_ms = [a.elapsed_time(b) for a, b, _ in evs]
+    total_ms = max_over_ranks(sum(step_ms))
+    s1_total = max_over_ranks(sum(s1_ms))
+    value = wk.units * args.steps * ws / (total_ms / 1e3)
+    users_per_s = wk.U * args.steps * ws / (s1_total / 1e3)
+
+    # ---- end to end through the public API, host buffers
+    for _ in range(2):
+        wk.e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, args.steps // 4)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(e2e_steps):
+        wk.e2e_step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = wk.units * e2e_steps * ws / (e2e_ms / 1e3)
+    assert ot.onetrans_device_status() == 0
+
+    # ---- roofline of the dominant kernel (largest device time in the timed region)
+    pk = peaks()
+    dom_name, dom = max(prof.items(), key=lambda kv: kv[1]["ms"])
+    per_launch_ms = dom["ms"] / dom["launches"]
+    tensor_bound = dom["flops"] / max(dom["bytes"], 1.0) > pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": pk["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops_sustained"],
+                "peak_source": pk["source"] + " bf16 sustained", "traffic": None,
+                "flops_per_launch": dom["flops"] / dom["launches"], "ms_per_launch": per_launch_ms}
+    else:
+        achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"] + " copy", "traffic": None,
+                "bytes_per_launch": dom["bytes"] / dom["launches"], "ms_per_launch": per_launch_ms}
+    kernels = {k: {"launches": v["launches"], "ms": round(v["ms"], 3),
+                   "share": round(v["ms"] / sum(x["ms"] for x in prof.values()), 4),
+                   "TFLOP/s": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1) if v["flops"] else None,
+                   "GB/s": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)}
+               for k, v in sorted(prof.items(), key=lambda kv: -kv[1]["ms"])}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "kv_serving: auto-split + Stage I + Stage II; 6 layers d=256 4 heads FFN 1024, "
+                               "pyramid queries 1190->12 (linear), 16 users x 1178 S tokens, 512 candidates/user, "
+                               "12 NS tokens from 512 features", "users_per_gpu": wk.U,
+                   "candidates_per_gpu": wk.units, "parallelism": f"users sharded over {ws} GPU(s), no collective",
+                   "l2": "512 MB buffer written between timed steps (not timed)"},
+        "users_per_s": users_per_s,
+        "stage1_ms_per_step": s1_total / args.steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wk.h2d, "d2h_bytes_per_step": wk.d2h},
+        "gpu_launches": int(sum(v["launches"] for v in prof.values())),
+        "roofline": roof,
+        "kernels": kernels,
+        "clocks": clk,
+        "wall_s_timed": wall,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, desc, cores, secs = oracle_sample()
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+                                "seconds": round(secs, 1)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -231,6 +231,17 @@ ONETRANS_API onetrans_status onetrans_set_kernel_policy(int32_t policy);
  * trapping, when a bounds check or a bounded wait fails (0 = no failure).
  * Synchronizes `stream`. */
 ONETRANS_API onetrans_status onetrans_device_status(void* stream, int32_t* code);
+/* Per-kernel timing for measurement.  While enabled, every launch is
+ * bracketed by CUDA events on its stream and tagged with its kernel kind and
+ * its algorithmic FLOPs and bytes (each operand and result once).  Enabling
+ * clears earlier records.  onetrans_profile_read synchronizes on the
+ * recorded events and sums one kind: launches, device milliseconds, FLOPs,
+ * bytes; `name` points to static storage. */
+ONETRANS_API onetrans_status onetrans_profile_enable(int32_t on);
+ONETRANS_API int32_t onetrans_profile_kinds(void);
+ONETRANS_API onetrans_status onetrans_profile_read(int32_t kind, const char** name,
+                                                   int64_t* launches, double* ms,
+                                                   double* flops, double* bytes);
 /* Human-readable name of a status code (static storage). */
 ONETRANS_API const char* onetrans_status_string(int32_t status);
 /* Library version as major*10000 + minor*100 + patch. */

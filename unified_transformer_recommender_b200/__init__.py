@@ -30,6 +30,7 @@ SYMBOLS = (
     "onetrans_tokenize_autosplit", "onetrans_stage1_encode", "onetrans_stage2_score",
     "onetrans_cache_append", "onetrans_forward", "onetrans_set_kernel_policy",
     "onetrans_device_status", "onetrans_status_string", "onetrans_version",
+    "onetrans_profile_enable", "onetrans_profile_kinds", "onetrans_profile_read",
 )
 
 
@@ -43,7 +44,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m unified_transformer_recommender_b200.build`")
+            "`python unified_transformer_recommender_b200/build.py`")
     return ctypes.CDLL(LIB_PATH)
 
 
@@ -100,6 +101,10 @@ _sig("onetrans_set_kernel_policy", I32, I32)
 _sig("onetrans_device_status", I32, P, PI32)
 _sig("onetrans_status_string", ctypes.c_char_p, I32)
 _sig("onetrans_version", I32)
+_sig("onetrans_profile_enable", I32, I32)
+_sig("onetrans_profile_kinds", I32)
+_sig("onetrans_profile_read", I32, I32, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(I64),
+     ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double))
 
 
 def status_string(s: int) -> str:
@@ -134,6 +139,24 @@ def onetrans_device_status(stream=None) -> int:
     code = I32(0)
     _check("onetrans_device_status", lib.onetrans_device_status(_stream(stream), ctypes.byref(code)))
     return code.value
+
+
+def onetrans_profile_enable(on: bool) -> None:
+    _check("onetrans_profile_enable", lib.onetrans_profile_enable(1 if on else 0))
+
+
+def onetrans_profile_read() -> dict:
+    """{kernel kind: {launches, ms, flops, bytes}} of the launches recorded
+    since profiling was enabled (kinds with no launch omitted)."""
+    out = {}
+    for k in range(lib.onetrans_profile_kinds()):
+        name, n = ctypes.c_char_p(), I64(0)
+        ms, fl, by = ctypes.c_double(0), ctypes.c_double(0), ctypes.c_double(0)
+        _check("onetrans_profile_read", lib.onetrans_profile_read(k, ctypes.byref(name), ctypes.byref(n),
+                                                                   ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(by)))
+        if n.value:
+            out[name.value.decode()] = {"launches": n.value, "ms": ms.value, "flops": fl.value, "bytes": by.value}
+    return out
 
 
 class Model:

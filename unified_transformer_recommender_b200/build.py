@@ -1,6 +1,6 @@
 """Build the OneTrans CUDA library in-tree for B200 (sm_100a).
 
-    python -m unified_transformer_recommender_b200.build
+    python unified_transformer_recommender_b200/build.py
 
 writes unified_transformer_recommender_b200/libonetrans.so.  nvcc
 cross-compiles, so no GPU is needed to build.

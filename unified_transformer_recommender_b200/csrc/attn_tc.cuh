@@ -1,6 +1,413 @@
+// Tensor-core attention for the bf16 path (sm_100a), head dim 64.
+//
+// One CTA owns 128 queries of one head.  K/V tiles of 128 keys (two 64-token
+// cache pages) are streamed by TMA through a 2-deep shared-memory ring.
+// Per key tile:  S = Q K^T (tcgen05.mma into TMEM, fp32) -> four softmax
+// warps read their query row back (tcgen05.ld: one row per thread, so the
+// row max and row sum stay inside the thread), apply the mask, update the
+// running max / sum (online softmax in base 2), write P = exp2(S - m) as bf16
+// into shared memory -> O_tile = P V (tcgen05.mma, V as an MN-major operand)
+// -> the softmax warps fold O_tile into their register accumulator.
+//
+// Two query kinds share the kernel:
+//  * MODE_CAUSAL  (Stage I, forward, append): query t of sequence b sits at
+//    key position q_pos0 + t and sees keys 0..q_pos0 + t (the pyramid's tail
+//    query set: only the last Lq rows are queries, keys span the layer input).
+//  * MODE_STAGE2: the queries are NS token j of up to 128 candidates of one
+//    user; they see every cached S key of the user (s_len keys) and then,
+//    in the same softmax, their own NS keys 0..j, folded in on CUDA cores.
+//
+// Warp roles (192 threads): warps 0-3 softmax/epilogue, warp 4 TMA, warp 5 MMA.
 #pragma once
-#include "common.cuh"
+#include "tc_ptx.cuh"
+
 namespace ot {
-inline bool tc_attn_supported(const AttnDesc&) { return false; }
-inline onetrans_status tc_attn_launch(const AttnDesc&, cudaStream_t) { return ONETRANS_ERR_UNSUPPORTED; }
+
+enum : int { MODE_CAUSAL = 0, MODE_STAGE2 = 1 };
+
+struct TcAttnArgs {
+  int mode;
+  // causal
+  int Lq, q_pos0;
+  RowMap o;
+  // stage II
+  const int* tiles;           // {user, c0, c1} per blockIdx.x
+  const __nv_bfloat16* qkv;   // [L_NS, C_tot, 3d]
+  __nv_bfloat16* o2;          // [L_NS, C_tot, d]
+  int C_tot, s_len;
+  // shared
+  KVStore kv;
+  int H;
+  float scale_log2;  // 1/sqrt(d_h) * log2(e)
+};
+
+struct AttnCfg {
+  static constexpr int DH = 64, BM = 128, BN = 128;
+  static constexpr int Q_BYTES = BM * DH * 2;     // 16 KB
+  static constexpr int KV_BYTES = BN * DH * 2;    // 16 KB (one of K or V)
+  static constexpr int PAGE_BYTES = 64 * DH * 2;  // one 64-token page of one head
+  static constexpr int STAGES = 2;
+  static constexpr int P_BYTES = BM * BN * 2;     // 32 KB
+  static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + 1024 + 256;
+  static constexpr int TMEM_COLS = 256;           // S: cols 0..127, O tile: 128..191
+};
+
+__device__ inline int kv_page_id(const KVStore& kv, int b, int page_idx) {
+  return kv.table ? kv.table[kv.row_off[b] + page_idx] : b * kv.pps + page_idx;
 }
+
+__global__ void __launch_bounds__(192, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
+                   const TcAttnArgs a) {
+  using C = AttnCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + C::Q_BYTES;                       // [stage][K|V][128 keys][64]
+  uint8_t* sP = sKV + C::STAGES * 2 * C::KV_BYTES;      // [2 key blocks][128 rows][64]
+  uint64_t* bars = (uint64_t*)(sP + C::P_BYTES);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;    // [2]
+  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* o_full = bars + 7;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+
+  // ---- work of this CTA
+  int b, q_row0, n_keys, kmax;   // n_keys: keys the tile loop covers (pre-mask)
+  int user = 0, c0 = 0, c1 = 0, j = 0;
+  if (a.mode == MODE_CAUSAL) {
+    b = blockIdx.z;
+    q_row0 = blockIdx.x * C::BM;
+    const int t_last = min(a.Lq, q_row0 + C::BM) - 1;
+    kmax = a.q_pos0 + t_last;
+    n_keys = kmax + 1;
+  } else {
+    user = a.tiles[blockIdx.x * 3 + 0];
+    c0 = a.tiles[blockIdx.x * 3 + 1];
+    c1 = a.tiles[blockIdx.x * 3 + 2];
+    j = blockIdx.z;
+    b = user;
+    q_row0 = c0;
+    kmax = a.s_len - 1;
+    n_keys = a.s_len;
+  }
+  const int nt = (n_keys + C::BN - 1) / C::BN;
+  const int n_pages_used = (kmax + 1 + 63) / 64;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(&kv_full[0], 1); mbar_init(&kv_full[1], 1);
+    mbar_init(&kv_empty[0], 1); mbar_init(&kv_empty[1], 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmKV);
+  }
+  if (warp == 5) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 128;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nt > 0) {
+      mbar_expect_tx(q_full, C::Q_BYTES);
+      if (a.mode == MODE_CAUSAL) tma_load_3d(&tmQ, q_full, sQ, h * C::DH, q_row0, b);
+      else tma_load_3d(&tmQ, q_full, sQ, h * C::DH, q_row0, j);
+      for (int kt = 0; kt < nt; ++kt) {
+        const int s = kt & 1;
+        if (kt >= 2 && !mbar_wait(&kv_empty[s], ((kt >> 1) - 1) & 1)) break;
+        mbar_expect_tx(&kv_full[s], 4 * C::PAGE_BYTES);
+        uint8_t* sk = sKV + s * 2 * C::KV_BYTES;
+        uint8_t* sv = sk + C::KV_BYTES;
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {
+          const int pi = kt * 2 + hp;
+          // pages past the last used one read as zeros (out-of-range page coordinate)
+          const int pg = pi < n_pages_used ? kv_page_id(a.kv, b, pi) : a.kv.n_pages;
+          tma_load_4d(&tmKV, &kv_full[s], sk + hp * C::PAGE_BYTES, 0, 0, h, pg);
+          tma_load_4d(&tmKV, &kv_full[s], sv + hp * C::PAGE_BYTES, 0, 0, a.H + h, pg);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0 && nt > 0) {
+      constexpr uint32_t id_qk = idesc_bf16(128, 128);
+      constexpr uint32_t id_pv = idesc_bf16(128, 64, false, true);
+      const uint32_t aq = smem_u32(sQ);
+      bool ok = mbar_wait(q_full, 0) && mbar_wait(&kv_full[0], 0);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t ak = smem_u32(sKV);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(tS, sdesc_k128(aq + k * 32), sdesc_k128(ak + k * 32), id_qk, k ? 1u : 0u);
+        umma_commit(s_full);
+      }
+      for (int kt = 0; kt < nt && ok; ++kt) {
+        ok = mbar_wait(p_full, kt & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (kt + 1 < nt) {
+          const int s1 = (kt + 1) & 1;
+          ok = mbar_wait(&kv_full[s1], ((kt + 1) >> 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ak = smem_u32(sKV + s1 * 2 * C::KV_BYTES);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(tS, sdesc_k128(aq + k * 32), sdesc_k128(ak + k * 32), id_qk, k ? 1u : 0u);
+          umma_commit(s_full);
+        }
+        const int s = kt & 1;
+        const uint32_t av = smem_u32(sKV + s * 2 * C::KV_BYTES + C::KV_BYTES);
+        const uint32_t ap = smem_u32(sP);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t pd = sdesc_k128(ap + (kk >> 2) * (128 * 128) + (kk & 3) * 32);
+          const uint64_t vd = sdesc_mn128(av + kk * 2048, 0);
+          umma_bf16(tO, pd, vd, id_pv, kk ? 1u : 0u);
+        }
+        umma_commit(o_full);
+        umma_commit(&kv_empty[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------- softmax + epilogue
+    const int r = warp * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int qpos = a.q_pos0 + q_row0 + r;  // causal: key position of this query
+    float o[64];
+#pragma unroll
+    for (int e = 0; e < 64; ++e) o[e] = 0.f;
+    float m = -INFINITY, l = 0.f;
+    const float sc = a.scale_log2;
+    for (int kt = 0; kt < nt; ++kt) {
+      if (!mbar_wait(s_full, kt & 1)) break;
+      tc_fence_after();
+      const int kbase = kt * C::BN;
+      const int vis_end = a.mode == MODE_CAUSAL ? min(qpos + 1, n_keys) : n_keys;  // keys < vis_end visible
+      // pass 1: masked row max (TMEM is re-read in pass 2 instead of holding 128 scores)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float sv[32];
+        tmem_ld32(tS + lane_base + c * 32, sv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (kbase + c * 32 + i < vis_end) mx = fmaxf(mx, sv[i] * sc);
+      }
+      const float m_new = fmaxf(m, mx);
+      const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m - m_new);
+      const float mref = (m_new == -INFINITY) ? 0.f : m_new;
+      if (kt > 0) {
+        // PV of the previous tile is done: fold it in, and P's buffer is free again
+        if (!mbar_wait(o_full, (kt - 1) & 1)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float ov[32];
+          tmem_ld32(tO + lane_base + c * 32, ov);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[c * 32 + e] = (o[c * 32 + e] + ov[e]) * alpha;
+        }
+      }
+      // pass 2: P = exp2(S - m) as bf16 into the K-major, 128-byte-swizzled A
+      // operand of P.V (row r, key k -> block k/64, 16-byte chunk (k%64)/8 ^ (r%8))
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float sv[32];
+        tmem_ld32(tS + lane_base + c * 32, sv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = (kbase + c * 32 + i < vis_end) ? exp2f(sv[i] * sc - mref) : 0.f;
+          rs += sv[i];
+        }
+        uint8_t* rowp = sP + (c >> 1) * (128 * 128) + r * 128;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int ch = (c & 1) * 4 + q4;
+          uint4 u;
+          __nv_bfloat162* hh = (__nv_bfloat162*)&u;
+#pragma unroll
+          for (int q2 = 0; q2 < 4; ++q2) hh[q2] = __floats2bfloat162_rn(sv[q4 * 8 + 2 * q2], sv[q4 * 8 + 2 * q2 + 1]);
+          *(uint4*)(rowp + ((ch ^ (r & 7)) << 4)) = u;
+        }
+      }
+      l = l * alpha + rs;
+      m = m_new;
+      // keys past the last valid one may hold stale bits: zero their V rows
+      if (kt == nt - 1) {
+        const int key = kbase + r;
+        if (key > kmax) {
+          uint4* vrow = (uint4*)(sKV + (kt & 1) * 2 * C::KV_BYTES + C::KV_BYTES + r * 128);
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) vrow[ch] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (nt > 0 && mbar_wait(o_full, (nt - 1) & 1)) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float ov[32];
+        tmem_ld32(tO + lane_base + c * 32, ov);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[c * 32 + e] += ov[e];
+      }
+    }
+    if (a.mode == MODE_CAUSAL) {
+      const int t = q_row0 + r;
+      if (t < a.Lq) {
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) o[e] *= inv;
+        __nv_bfloat16* dst = (__nv_bfloat16*)a.o.base + rm_off(a.o, b, t, h * 64);
+        store_bf16x32(dst, o);
+        store_bf16x32(dst + 32, o + 32);
+      }
+    } else {
+      const int c = c0 + r;
+      if (c < c1) {
+        // own NS keys 0..j of this candidate, in the same softmax
+        const int d = a.H * 64;
+        const long long rs3 = 3LL * d;
+        float q[64];
+        const __nv_bfloat16* qp = a.qkv + ((long long)j * a.C_tot + c) * rs3 + h * 64;
+        load_bf16x32(qp, q);
+        load_bf16x32(qp + 32, q + 32);
+        for (int i = 0; i <= j; ++i) {
+          const __nv_bfloat16* kp = a.qkv + ((long long)i * a.C_tot + c) * rs3 + d + h * 64;
+          float kv[64];
+          load_bf16x32(kp, kv);
+          load_bf16x32(kp + 32, kv + 32);
+          float s = 0.f;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) s = fmaf(q[e], kv[e], s);
+          s *= sc;
+          const float m_new = fmaxf(m, s);
+          const float alpha = exp2f(m - m_new), p = exp2f(s - m_new);
+          load_bf16x32(kp + d, kv);
+          load_bf16x32(kp + d + 32, kv + 32);
+#pragma unroll
+          for (int e = 0; e < 64; ++e) o[e] = fmaf(p, kv[e], o[e] * alpha);
+          l = l * alpha + p;
+          m = m_new;
+        }
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) o[e] *= inv;
+        __nv_bfloat16* dst = a.o2 + ((long long)j * a.C_tot + c) * d + h * 64;
+        store_bf16x32(dst, o);
+        store_bf16x32(dst + 32, o + 32);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host --
+// 4-D bf16 map over a page pool: (d_h, token, kind*H + head, page).
+inline bool make_tmap_pages(CUtensorMap* map, const KVStore& kv) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)kv.dh, (cuuint64_t)kv.P, (cuuint64_t)(2 * kv.H),
+                              (cuuint64_t)kv.n_pages};
+  const cuuint64_t strides[3] = {(cuuint64_t)kv.dh * 2, (cuuint64_t)kv.P * kv.dh * 2,
+                                 (cuuint64_t)2 * kv.H * kv.P * kv.dh * 2};
+  const cuuint32_t box[4] = {64, 64, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, kv.pool, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool tc_kv_ok(const KVStore& kv) {
+  return kv.dh == 64 && kv.P == 64 && kv.n_pages > 0 && ((uintptr_t)kv.pool % 16) == 0 && encode_fn();
+}
+
+inline bool tc_attn_supported(const AttnDesc& a) {
+  return a.dh == 64 && tc_kv_ok(a.kv) && ((uintptr_t)a.q.base % 16) == 0 && a.q.st % 8 == 0 &&
+         a.q.sb % 8 == 0 && rowmap_vec_ok(a.o) && !a.o.f32;
+}
+
+inline onetrans_status attn_launch_common(const CUtensorMap& tq, const CUtensorMap& tkv, const TcAttnArgs& args,
+                                          dim3 grid, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg::SMEM) !=
+        cudaSuccess)
+      return ONETRANS_ERR_CUDA;
+    attr_set = true;
+  }
+  attn_tc_kernel<<<grid, 192, AttnCfg::SMEM, st>>>(tq, tkv, args);
+  return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
+}
+
+inline onetrans_status tc_attn_launch(const AttnDesc& a, cudaStream_t st) {
+  CUtensorMap tq, tkv;
+  const uint64_t d = (uint64_t)a.H * a.dh;
+  // Q rows of batch b: base + b*sb + t*st, d columns per row
+  if (!make_tmap_3d(&tq, a.q.base, d, (uint64_t)a.Lq, (uint64_t)a.B, (uint64_t)a.q.st,
+                    a.B > 1 ? (uint64_t)a.q.sb : (uint64_t)a.Lq * a.q.st, 64, 128, 1) ||
+      !make_tmap_pages(&tkv, a.kv))
+    return ONETRANS_ERR_CUDA;
+  TcAttnArgs args;
+  memset(&args, 0, sizeof(args));
+  args.mode = MODE_CAUSAL;
+  args.Lq = a.Lq;
+  args.q_pos0 = a.q_pos0;
+  args.o = a.o;
+  args.kv = a.kv;
+  args.H = a.H;
+  args.scale_log2 = a.scale * 1.4426950408889634f;
+  dim3 grid((unsigned)((a.Lq + 127) / 128), (unsigned)a.H, (unsigned)a.B);
+  return attn_launch_common(tq, tkv, args, grid, st);
+}
+
+inline bool tc_stage2_supported(const Stage2Desc& a) {
+  return a.dh == 64 && tc_kv_ok(a.kv) && ((uintptr_t)a.qkv % 16) == 0 && ((uintptr_t)a.o % 16) == 0;
+}
+
+// Stage II: `tiles` holds up to 128 candidates of one user per entry.
+inline onetrans_status tc_stage2_launch(const Stage2Desc& a, int n_tiles, cudaStream_t st) {
+  CUtensorMap tq, tkv;
+  const uint64_t d = (uint64_t)a.H * a.dh;
+  if (!make_tmap_3d(&tq, a.qkv, 3 * d, (uint64_t)a.C_tot, (uint64_t)a.L_NS, 3 * d, (uint64_t)a.C_tot * 3 * d, 64,
+                    128, 1) ||
+      !make_tmap_pages(&tkv, a.kv))
+    return ONETRANS_ERR_CUDA;
+  TcAttnArgs args;
+  memset(&args, 0, sizeof(args));
+  args.mode = MODE_STAGE2;
+  args.tiles = a.tiles;
+  args.qkv = (const __nv_bfloat16*)a.qkv;
+  args.o2 = (__nv_bfloat16*)a.o;
+  args.C_tot = a.C_tot;
+  args.s_len = a.s_len;
+  args.kv = a.kv;
+  args.H = a.H;
+  args.scale_log2 = a.scale * 1.4426950408889634f;
+  dim3 grid((unsigned)n_tiles, (unsigned)a.H, (unsigned)a.L_NS);
+  return attn_launch_common(tq, tkv, args, grid, st);
+}
+
+}  // namespace ot

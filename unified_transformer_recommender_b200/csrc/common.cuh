@@ -73,7 +73,7 @@ struct AttnDesc {
 
 // Stage II attention: candidates of one user share the user's cached S keys.
 struct Stage2Desc {
-  int H, dh, L_NS, C_tot, s_len;
+  int H, dh, L_NS, C_tot, s_len, n_users;
   const int* tiles;    // n_tiles x {user, c0, c1}
   const void* qkv;     // [L_NS, C_tot, 3d] token-major Q|K|V of the NS rows
   void* o;             // [L_NS, C_tot, d]

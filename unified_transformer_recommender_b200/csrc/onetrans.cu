@@ -41,6 +41,57 @@ struct onetrans_cache {
 };
 
 static int g_policy = 0;
+
+// ------------------------------------------------------------ profiling --
+// When enabled, every launch is bracketed by CUDA events on its stream and
+// tagged with a kernel kind and its algorithmic FLOPs and bytes.
+enum ProfKind {
+  PK_GEMM_QKV = 0, PK_GEMM_OPROJ, PK_GEMM_FFN_UP, PK_GEMM_FFN_DOWN, PK_GEMM_AUTOSPLIT, PK_ATTN_CAUSAL,
+  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_COUNT
+};
+static const char* kProfNames[PK_COUNT] = {"gemm_qkv", "gemm_oproj_rms", "gemm_ffn_up_gelu", "gemm_ffn_down_rms",
+                                           "gemm_autosplit", "attn_causal", "attn_stage2", "rmsnorm",
+                                           "tokenize_events"};
+struct ProfRec {
+  int kind;
+  cudaEvent_t e0, e1;
+  double flops, bytes;
+};
+static struct {
+  std::mutex mu;
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+} g_prof;
+
+static cudaEvent_t prof_event() {
+  if (g_prof.used < g_prof.pool.size()) return g_prof.pool[g_prof.used++];
+  cudaEvent_t e;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  g_prof.pool.push_back(e);
+  g_prof.used++;
+  return e;
+}
+
+struct ProfScope {
+  bool on;
+  ProfRec rec;
+  cudaStream_t st;
+  ProfScope(int kind, double flops, double bytes, cudaStream_t s) : on(false), st(s) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (!g_prof.on) return;
+    rec.kind = kind; rec.flops = flops; rec.bytes = bytes;
+    rec.e0 = prof_event(); rec.e1 = prof_event();
+    if (!rec.e0 || !rec.e1) return;
+    on = cudaEventRecord(rec.e0, st) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (cudaEventRecord(rec.e1, st) == cudaSuccess) g_prof.recs.push_back(rec);
+  }
+};
 static const int kMaxUsers = 65536;  // users per Stage II call (workspace holds their table rows)
 
 #define OT_TRY(x)                                  \
@@ -137,15 +188,29 @@ static GemmDesc gdesc_base(const onetrans_model* m) {
 template <typename T>
 static onetrans_status launch_rms(GemmDesc d, cudaStream_t st) {
   if (d.M <= 0 || d.G <= 0) return ONETRANS_OK;
+  ProfScope prof(PK_RMSNORM, 0.0, (double)d.M * d.G * d.N * (sizeof(T) + (d.out.f32 ? 4 : sizeof(T))), st);
   dim3 grid((unsigned)cdiv(d.M, 8), (unsigned)d.G);
   rms_rows_kernel<T><<<grid, 256, 0, st>>>(d);
   return last_launch();
 }
 
+// Algorithmic bytes of one GEMM launch: A, W and every tensor the epilogue
+// reads or writes, each once.
+static double gemm_bytes(const onetrans_model* m, const GemmDesc& d) {
+  const double rows = (double)d.M * d.G, es = m->es;
+  double b = rows * d.K * es + (double)d.N * d.K * es * (d.mode == TILE_SAMPLES ? d.G : 1);
+  b += rows * d.N * (d.out_kind == OUT_KV ? es : (d.out.f32 ? 4 : es));
+  if (d.res.base) b += rows * d.N * (d.res.f32 ? 4 : es);
+  if (d.rms.base) b += rows * d.N * es;
+  return b;
+}
+
 template <typename T>
-static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, cudaStream_t st) {
+static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, cudaStream_t st,
+                                   int kind = PK_GEMM_QKV) {
   if (d.M <= 0 || d.G <= 0 || d.N <= 0) return ONETRANS_OK;
   if (cdiv(d.M, 64) > 65535 || d.G > 65535) return ONETRANS_ERR_SHAPE;
+  ProfScope prof(kind, 2.0 * d.M * d.G * (double)d.N * d.K, gemm_bytes(m, d), st);
   if (m->bf16 && g_policy == 0 && tc_gemm_supported(d)) {
     return tc_gemm_launch(d, st);
   }
@@ -159,6 +224,11 @@ static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, c
 template <typename T>
 static onetrans_status launch_attn(const onetrans_model* m, const AttnDesc& a, cudaStream_t st) {
   if (a.Lq <= 0 || a.B <= 0) return ONETRANS_OK;
+  // visible (query, key) pairs: query t sees q_pos0 + t + 1 keys
+  const double pairs = (double)a.Lq * a.q_pos0 + 0.5 * (double)a.Lq * (a.Lq + 1);
+  const double kv_bytes = 2.0 * (a.q_pos0 + a.Lq) * a.H * a.dh * m->es;
+  ProfScope prof(PK_ATTN_CAUSAL, 4.0 * a.dh * a.H * a.B * pairs,
+                 a.B * (kv_bytes + 2.0 * a.Lq * a.H * a.dh * m->es), st);
   if (m->bf16 && g_policy == 0 && tc_attn_supported(a)) return tc_attn_launch(a, st);
   dim3 grid((unsigned)cdiv(a.Lq, 64), (unsigned)a.H, (unsigned)a.B);
   switch (a.dh) {
@@ -172,10 +242,23 @@ static onetrans_status launch_attn(const onetrans_model* m, const AttnDesc& a, c
   return last_launch();
 }
 
+// Tensor-core Stage II attention takes tiles of up to 128 candidates, the
+// CUDA-core kernel up to 64.
+static bool stage2_tc(const onetrans_model* m, const Stage2Desc& a) {
+  return m->bf16 && g_policy == 0 && tc_stage2_supported(a);
+}
+
 template <typename T>
 static onetrans_status launch_stage2_attn(const onetrans_model* m, const Stage2Desc& a, int n_tiles,
                                           cudaStream_t st) {
   if (n_tiles <= 0) return ONETRANS_OK;
+  // per candidate: token j sees s_len + j + 1 keys; bytes: the users' cached
+  // K/V once each, Q/K/V of the NS rows, the output
+  const double pairs = (double)a.C_tot * (a.L_NS * (double)a.s_len + 0.5 * a.L_NS * (a.L_NS + 1));
+  const double es = m->es;
+  ProfScope prof(PK_ATTN_STAGE2, 4.0 * a.dh * a.H * pairs,
+                 a.n_users * 2.0 * a.s_len * a.H * a.dh * es + (double)a.L_NS * a.C_tot * a.H * a.dh * es * 4, st);
+  if (stage2_tc(m, a)) return tc_stage2_launch(a, n_tiles, st);
   dim3 grid((unsigned)n_tiles, (unsigned)a.H, (unsigned)a.L_NS);
   switch (a.dh) {
     case 16: stage2_attn_simt_kernel<T, 16><<<grid, 64, 0, st>>>(a); break;
@@ -276,7 +359,7 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
     go.out = rmap32(xm, (long long)Lqn * d, d);
     go.rms = rmap(h2, (long long)Lqn * d, d);
     go.gamma = m->g_ffn[n];
-    OT_TRY(launch_gemm<T>(m, go, st));
+    OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     // -- mixed FFN: S tail rows shared, NS rows per token
     for (int part = 0; part < 2; ++part) {
       GemmDesc f = gdesc_base(m);
@@ -294,7 +377,7 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
       f.bias = part ? m->b1_NS[n] : m->b1_S[n]; f.bias_sg = part ? dff : 0;
       f.act = ACT_GELU;
       f.out = rmap(hid, (long long)Lqn * dff, dff);
-      OT_TRY(launch_gemm<T>(m, f, st));
+      OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
       GemmDesc f2 = f;
       f2.K = dff; f2.A = hid; f2.act = ACT_NONE;
       if (part == 0) { f2.a_sm = dff; f2.a_sg = (long long)Lqn * dff; }
@@ -305,7 +388,7 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
       f2.res = rmap32(xm, (long long)Lqn * d, d);
       f2.out = rmap32(x_next, (long long)Lqn * d, d);
       if (!last) { f2.rms = rmap(h, (long long)Lqn * d, d); f2.gamma = m->g_attn[n + 1]; }
-      OT_TRY(launch_gemm<T>(m, f2, st));
+      OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
     }
     x_in = x_next;
     L = Lqn;
@@ -418,12 +501,12 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
     go.out = rmap32(xm, (long long)sqn * d, d);
     go.rms = rmap(h2, (long long)sqn * d, d);
     go.gamma = m->g_ffn[n];
-    OT_TRY(launch_gemm<T>(m, go, st));
+    OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     GemmDesc f = go;
     f.res.base = nullptr; f.rms.base = nullptr; f.gamma = nullptr;
     f.A = h2; f.W = m->W1_S[n]; f.w_rows = dff; f.N = dff; f.bias = m->b1_S[n]; f.act = ACT_GELU;
     f.out = rmap(hid, (long long)sqn * dff, dff);
-    OT_TRY(launch_gemm<T>(m, f, st));
+    OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
     GemmDesc f2 = go;
     f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.W = m->W2_S[n]; f2.w_rows = d; f2.N = d;
     f2.bias = m->b2_S[n];
@@ -431,7 +514,7 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
     f2.out = rmap32(x_next, (long long)sqn * d, d);
     f2.rms = rmap(h, (long long)sqn * d, d);
     f2.gamma = m->g_attn[n + 1];
-    OT_TRY(launch_gemm<T>(m, f2, st));
+    OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
     x_in = x_next;
   }
   return ONETRANS_OK;
@@ -448,15 +531,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   const int L_S = need ? L_S_need : (U > 0 ? c->len[slots[0]] : 0);
   std::vector<int> s, sq;
   OT_TRY(s_rows_of(m, L_S, s, sq));
-  const int TQ = 64;
-  long long max_tiles = need ? cdiv(C, TQ) + std::min<long long>(C, kMaxUsers) : 0;
-  std::vector<int> tiles;
-  if (!need) {
-    for (int u = 0; u < U; ++u)
-      for (int c0 = offs[u]; c0 < offs[u + 1]; c0 += TQ)
-        tiles.insert(tiles.end(), {u, c0 - offs[0], std::min(c0 + TQ, offs[u + 1]) - offs[0]});
-    max_tiles = (long long)tiles.size() / 3;
-  }
+  long long max_tiles = need ? cdiv(C, 64) + std::min<long long>(C, kMaxUsers) : 0;
   Carve cv(ws, ws_bytes);
   void* xa = cv.take((size_t)L_NS * C * d * 4);   // residual stream: float32
   void* xb = cv.take((size_t)L_NS * C * d * 4);
@@ -471,6 +546,19 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   if (need) { *need = cv.used; return ONETRANS_OK; }
   if (cv.overflow) return ONETRANS_ERR_CAPACITY;
   if (C == 0) return ONETRANS_OK;
+
+  // candidate tiles, one user each; the attention kernel decides the tile size
+  Stage2Desc probe;
+  std::memset(&probe, 0, sizeof(probe));
+  probe.H = m->H; probe.dh = m->dh; probe.L_NS = L_NS; probe.C_tot = (int)C;
+  probe.qkv = qkv; probe.o = at;
+  kv_for_cache(c, 0, row_off, probe.kv);
+  const int TQ = stage2_tc(m, probe) ? 128 : 64;
+  std::vector<int> tiles;
+  for (int u = 0; u < U; ++u)
+    for (int c0 = offs[u]; c0 < offs[u + 1]; c0 += TQ)
+      tiles.insert(tiles.end(), {u, c0 - offs[0], std::min(c0 + TQ, offs[u + 1]) - offs[0]});
+  max_tiles = (long long)tiles.size() / 3;
 
   std::vector<int> h_row_off(U);
   for (int u = 0; u < U; ++u) h_row_off[u] = slots[u] * m->NL * c->max_pages;
@@ -491,7 +579,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     OT_TRY(launch_gemm<T>(m, g, st));
     Stage2Desc a;
     std::memset(&a, 0, sizeof(a));
-    a.H = m->H; a.dh = m->dh; a.L_NS = L_NS; a.C_tot = (int)C; a.s_len = s[n];
+    a.H = m->H; a.dh = m->dh; a.L_NS = L_NS; a.C_tot = (int)C; a.s_len = s[n]; a.n_users = U;
     a.tiles = d_tiles; a.qkv = qkv; a.o = at;
     kv_for_cache(c, n, row_off, a.kv);
     a.scale = 1.0f / std::sqrt((float)m->dh);
@@ -504,12 +592,12 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     go.out = rmap32(xm, 0, d);
     go.rms = rmap(h2, 0, d);
     go.gamma = m->g_ffn[n];
-    OT_TRY(launch_gemm<T>(m, go, st));
+    OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     GemmDesc f = g;
     f.A = h2; f.W = m->W1_NS[n]; f.w_sg = (long long)dff * d; f.w_rows = dff; f.N = dff;
     f.bias = m->b1_NS[n]; f.bias_sg = dff; f.act = ACT_GELU;
     f.out = rmap(hid, dff, C * dff);
-    OT_TRY(launch_gemm<T>(m, f, st));
+    OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
     GemmDesc f2 = g;
     f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.a_sg = C * dff;
     f2.W = m->W2_NS[n]; f2.w_sg = (long long)d * dff; f2.w_rows = d; f2.N = d;
@@ -517,7 +605,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     f2.res = rmap32(xm, d, C * d);
     f2.out = rmap32(x_next, d, C * d);
     if (!last) { f2.rms = rmap(h, d, C * d); f2.gamma = m->g_attn[n + 1]; }
-    OT_TRY(launch_gemm<T>(m, f2, st));
+    OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
     x_in = x_next;
   }
   return ONETRANS_OK;
@@ -571,6 +659,8 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
   }
   w.emb = m->type_emb; w.n_types = m->cfg.n_behaviors; w.e_dim = m->cfg.event_dim; w.d = d;
   const size_t smem = (size_t)(w.e_dim + d) * sizeof(float);
+  ProfScope prof_tok(PK_TOKENIZE, 2.0 * R * ((double)w.e_dim * d + (double)d * d),
+                     (double)R * (w.e_dim * m->es + d * 4), st);
   event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>((const T*)events, types, dL, w,
                                                                          rmap32(xa, (long long)dL * d, d));
   OT_TRY(last_launch());
@@ -607,12 +697,12 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     go.out = rmap32(xm, (long long)dL * d, d);
     go.rms = rmap(h2, (long long)dL * d, d);
     go.gamma = m->g_ffn[n];
-    OT_TRY(launch_gemm<T>(m, go, st));
+    OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     GemmDesc f = go;
     f.res.base = nullptr; f.rms.base = nullptr; f.gamma = nullptr;
     f.A = h2; f.W = m->W1_S[n]; f.w_rows = dff; f.N = dff; f.bias = m->b1_S[n]; f.act = ACT_GELU;
     f.out = rmap(hid, (long long)dL * dff, dff);
-    OT_TRY(launch_gemm<T>(m, f, st));
+    OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
     GemmDesc f2 = go;
     f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.W = m->W2_S[n]; f2.w_rows = d; f2.N = d;
     f2.bias = m->b2_S[n];
@@ -620,7 +710,7 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     f2.out = rmap32(x_next, (long long)dL * d, d);
     f2.rms = rmap(h, (long long)dL * d, d);
     f2.gamma = m->g_attn[n + 1];
-    OT_TRY(launch_gemm<T>(m, f2, st));
+    OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
     x_in = x_next;
   }
   return ONETRANS_OK;
@@ -641,14 +731,14 @@ static onetrans_status autosplit_impl(const onetrans_model* m, const void* feats
   g.K = F; g.A = feats; g.a_sm = F; g.a_mext = N; g.a_gext = 1;
   g.W = m->Wa1; g.w_rows = Hh; g.N = Hh; g.bias = m->ba1; g.act = ACT_GELU;
   g.out = rmap(hid, 0, Hh);
-  OT_TRY(launch_gemm<T>(m, g, st));
+  OT_TRY(launch_gemm<T>(m, g, st, PK_GEMM_AUTOSPLIT));
   GemmDesc g2 = g;
   g2.K = Hh; g2.A = hid; g2.a_sm = Hh; g2.W = m->Wa2; g2.w_rows = L_NS * d; g2.N = L_NS * d;
   g2.bias = m->ba2; g2.act = ACT_NONE;
   g2.out = rmap(out, 0, d);
   g2.out.sc = N * d;
   g2.out.split = d;
-  return launch_gemm<T>(m, g2, st);
+  return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
 }
 
 // ============================================================== C ABI ====
@@ -950,6 +1040,33 @@ onetrans_status onetrans_forward(const onetrans_model* m, const void* x0, int32_
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? forward_impl<__nv_bfloat16>(m, x0, B, L_S, out, ws, ws_bytes, st, nullptr)
                  : forward_impl<float>(m, x0, B, L_S, out, ws, ws_bytes, st, nullptr);
+}
+
+onetrans_status onetrans_profile_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.on = on != 0;
+  g_prof.recs.clear();
+  g_prof.used = 0;
+  return ONETRANS_OK;
+}
+
+int32_t onetrans_profile_kinds(void) { return PK_COUNT; }
+
+onetrans_status onetrans_profile_read(int32_t kind, const char** name, int64_t* launches, double* ms,
+                                      double* flops, double* bytes) {
+  if (kind < 0 || kind >= PK_COUNT || !name || !launches || !ms || !flops || !bytes)
+    return ONETRANS_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  *name = kProfNames[kind];
+  *launches = 0; *ms = 0; *flops = 0; *bytes = 0;
+  for (const ProfRec& r : g_prof.recs) {
+    if (r.kind != kind) continue;
+    float t = 0.f;
+    OT_TRY(cuda_ok(cudaEventSynchronize(r.e1)));
+    OT_TRY(cuda_ok(cudaEventElapsedTime(&t, r.e0, r.e1)));
+    *launches += 1; *ms += t; *flops += r.flops; *bytes += r.bytes;
+  }
+  return ONETRANS_OK;
 }
 
 onetrans_status onetrans_device_status(void* stream, int32_t* code) {
