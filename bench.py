@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--workload", default="kv_serving",
                     choices=("kv_serving", "append", "s_forward", "l_forward"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--users", type=int, default=0, help="override users per GPU (small profiling captures)")
+    ap.add_argument("--cands", type=int, default=0, help="override candidates per user (small captures)")
     return ap.parse_args()
 
 
@@ -147,14 +149,14 @@ def peaks():
 class KVServing:
     """Auto-split + Stage I + Stage II for U users x C candidates."""
 
-    def __init__(self, rank: int, wl_name: str = "kv_serving"):
+    def __init__(self, rank: int, wl_name: str = "kv_serving", users: int = 0, cands: int = 0):
         import torch
         import unified_transformer_recommender_b200 as ot
         from onetrans_synth import WORKLOADS, gen_normal, make_weights
         self.ot, self.torch = ot, torch
         wl = WORKLOADS[wl_name]
         self.wl, sh = wl, wl.shape
-        self.U, self.C = wl.users, wl.cands
+        self.U, self.C = users or wl.users, cands or wl.cands
         self.W = make_weights(sh, wl.seed_weights, wl.dtype)
         self.model = ot.model_from_arrays(sh, self.W, pyramid_q=list(wl.pyramid), mode=ot.BF16)
         seed = wl.seed_inputs + 7919 * rank     # each rank serves different users
@@ -271,7 +273,7 @@ def main():
 
     if args.workload != "kv_serving":
         raise SystemExit("bench.py times the kv_serving workload; other workloads: tests/")
-    wk = KVServing(rank)
+    wk = KVServing(rank, users=args.users, cands=args.cands)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")   # > 126 MB L2
     st = torch.cuda.current_stream()
 
@@ -352,8 +354,8 @@ def main():
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "kv_serving: auto-split + Stage I + Stage II; 6 layers d=256 4 heads FFN 1024, "
-                               "pyramid queries 1190->12 (linear), 16 users x 1178 S tokens, 512 candidates/user, "
-                               "12 NS tokens from 512 features", "users_per_gpu": wk.U,
+                               f"pyramid queries 1190->12 (linear), {wk.U} users x 1178 S tokens, {wk.C} "
+                               "candidates/user, 12 NS tokens from 512 features", "users_per_gpu": wk.U,
                    "candidates_per_gpu": wk.units, "parallelism": f"users sharded over {ws} GPU(s), no collective",
                    "l2": "512 MB buffer written between timed steps (not timed)"},
         "users_per_s": users_per_s,
@@ -365,7 +367,7 @@ def main():
         "clocks": clk,
         "wall_s_timed": wall,
     }
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and not (args.users or args.cands):
         v, desc, cores, secs = oracle_sample()
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
                                 "seconds": round(secs, 1)}

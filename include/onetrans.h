@@ -180,6 +180,22 @@ ONETRANS_API onetrans_status onetrans_tokenize_autosplit(const onetrans_model* m
                                             void* ns_tokens, void* ws,
                                             size_t ws_bytes, void* stream);
 
+/* The auto-split tokenizer for callers that cannot allocate device memory:
+ * a plugin inside an inference server whose device memory all belongs to the
+ * server's own pool, or a latency-bound serving loop where a cudaMalloc would
+ * synchronize the device.  Same computation and output as
+ * onetrans_tokenize_autosplit, but no workspace: the hidden layer lives in a
+ * fixed 16 MiB array in the library's own device memory, held by every GPU
+ * that loads the library until the process exits.  N * ns_hidden * element
+ * size must not exceed 16 MiB (N <= 2730 rows at H = 3072 in bf16), else
+ * ONETRANS_ERR_CAPACITY.  The first call on a device looks up the array's
+ * address with that device current; make that first call before any stream
+ * capture.  All calls share the array: calls whose kernels overlap on the GPU
+ * race.  Nothing is allocated.  The pages have no counterpart of this call. */
+ONETRANS_API onetrans_status onetrans_tokenize_autosplit_static(
+    const onetrans_model* m, const void* feats, int64_t N, void* ns_tokens,
+    void* stream);
+
 /* Stage I ([FR] 7.5.3): run each user's S-tokens through the stack (pyramid
  * tail queries included) and store every layer's S-side K/V in cache slot
  * slots[u] (host array of U slot ids, distinct).  The slot's previous

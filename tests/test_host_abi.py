@@ -22,7 +22,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 21
+    assert len(names) == 22
     for n in names:
         assert hasattr(ot.lib, n), n
     assert set(names) == set(ot.SYMBOLS)

@@ -1,0 +1,42 @@
+"""The allocation-free auto-split entry point, for callers that cannot
+allocate device memory (a plugin whose host server owns every device byte,
+or a serving loop where cudaMalloc would stall the device).  Through the C
+ABI it must give the same tokens as the workspace entry point, within the
+bf16 tolerance of the other tests, on two calls in a row that share the
+library's fixed scratch array.  Collected last so that a run stopping at the
+first failure has already run every other test."""
+import ctypes
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from onetrans_synth import gen_normal
+from helpers import TOL, build, rel_err, shape, to_dev, to_np
+
+import unified_transformer_recommender_b200 as ot  # noqa: E402
+
+
+def test_static_scratch_autosplit_matches_workspace_entry_point():
+    sh = shape(n_layers=1)
+    b = build(sh, 301, "bf16")
+    m = b.model
+    for call, N in enumerate((1000, 2730)):      # 2730 rows fill the 16 MiB array at H = 3072
+        feats = to_dev(gen_normal(400 + call, (N, sh.ns_feat), "bf16"), torch.bfloat16)
+        ref = torch.empty(sh.L_NS, N, sh.d, dtype=torch.bfloat16, device="cuda")
+        ot.onetrans_tokenize_autosplit(m, feats, ref, m.workspace(ot.OP_AUTOSPLIT, N))
+        got = torch.full((sh.L_NS, N, sh.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = torch.cuda.current_stream().cuda_stream
+        status = ot.lib.onetrans_tokenize_autosplit_static(m.handle, feats.data_ptr(), N, got.data_ptr(), st)
+        assert status == ot.OK
+        torch.cuda.synchronize()
+        assert rel_err(to_np(got), to_np(ref)) <= TOL["bf16"]
+    # one row past the array's capacity is refused before any launch
+    too_many = 2731
+    feats = torch.zeros(too_many, sh.ns_feat, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(sh.L_NS, too_many, sh.d, dtype=torch.bfloat16, device="cuda")
+    assert ot.lib.onetrans_tokenize_autosplit_static(m.handle, feats.data_ptr(), too_many, out.data_ptr(),
+                                                     None) == ot.ERR_CAPACITY
+    assert ot.onetrans_device_status() == 0

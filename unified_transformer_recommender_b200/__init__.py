@@ -31,6 +31,7 @@ SYMBOLS = (
     "onetrans_cache_append", "onetrans_forward", "onetrans_set_kernel_policy",
     "onetrans_device_status", "onetrans_status_string", "onetrans_version",
     "onetrans_profile_enable", "onetrans_profile_kinds", "onetrans_profile_read",
+    "onetrans_tokenize_autosplit_static",
 )
 
 
@@ -93,6 +94,7 @@ _sig("onetrans_cache_destroy", I32, P)
 _sig("onetrans_cache_length", I32, P, I32, PI32)
 _sig("onetrans_cache_row_ptr", I32, P, I32, I32, I32, I32, I32, ctypes.POINTER(P))
 _sig("onetrans_tokenize_autosplit", I32, P, P, I64, P, P, SZ, P)
+_sig("onetrans_tokenize_autosplit_static", I32, P, P, I64, P, P)
 _sig("onetrans_stage1_encode", I32, P, P, PI32, I32, P, I32, P, SZ, P)
 _sig("onetrans_stage2_score", I32, P, P, PI32, I32, PI32, P, P, P, SZ, P)
 _sig("onetrans_cache_append", I32, P, P, PI32, I32, P, P, I32, P, SZ, P)
@@ -273,6 +275,13 @@ def onetrans_tokenize_autosplit(model: Model, feats: torch.Tensor, ns_tokens: to
                                 ws: torch.Tensor, stream=None) -> None:
     _check("onetrans_tokenize_autosplit", lib.onetrans_tokenize_autosplit(
         model.handle, _ptr(feats), feats.shape[0], _ptr(ns_tokens), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def onetrans_tokenize_autosplit_static(model: Model, feats: torch.Tensor, ns_tokens: torch.Tensor,
+                                       stream=None) -> None:
+    """Auto-split without a workspace (scratch in the library's fixed array)."""
+    _check("onetrans_tokenize_autosplit_static", lib.onetrans_tokenize_autosplit_static(
+        model.handle, _ptr(feats), feats.shape[0], _ptr(ns_tokens), _stream(stream)))
 
 
 def onetrans_stage1_encode(model: Model, cache: Cache, slots: Sequence[int], s_tokens: torch.Tensor,

@@ -1085,3 +1085,66 @@ onetrans_status onetrans_device_status(void* stream, int32_t* code) {
 }
 
 }  // extern "C"
+
+// ================================================= auto-split, no allocation
+// Scratch for the auto-split tokenizer's hidden layer, in the library's own
+// device memory: every GPU that loads the library holds these 16 MiB until
+// the process exits.  All calls share it and it keeps the previous call's
+// contents; nothing needs clearing because the first GEMM writes every
+// element the second GEMM reads.  Calls whose kernels overlap on the GPU
+// (two streams, two host threads) race on it.
+static const size_t kStaticScratchBytes = 16u << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+static std::mutex g_static_mu;
+static void* g_static_ptr[64];  // device address of g_static_scratch, per device
+
+// Device address of the scratch on the current device, looked up once per
+// device (host code cannot pass the symbol itself to a kernel).
+static onetrans_status static_scratch(void** out) {
+  int dev = -1;
+  OT_TRY(cuda_ok(cudaGetDevice(&dev)));
+  if (dev < 0 || dev >= 64) return ONETRANS_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    OT_TRY(cuda_ok(cudaGetSymbolAddress(&p, g_static_scratch)));
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return ONETRANS_OK;
+}
+
+template <typename T>
+static onetrans_status autosplit_with_hidden(const onetrans_model* m, const void* feats, long long N, void* out,
+                                             void* hid, cudaStream_t st) {
+  const int F = m->cfg.ns_feat_dim, Hh = m->cfg.ns_hidden, d = m->d, L_NS = m->L_NS;
+  GemmDesc g = gdesc_base(m);
+  g.mode = TILE_FLAT; g.M = (int)N; g.G = 1;
+  g.K = F; g.A = feats; g.a_sm = F; g.a_mext = N; g.a_gext = 1;
+  g.W = m->Wa1; g.w_rows = Hh; g.N = Hh; g.bias = m->ba1; g.act = ACT_GELU;
+  g.out = rmap(hid, 0, Hh);
+  OT_TRY(launch_gemm<T>(m, g, st, PK_GEMM_AUTOSPLIT));
+  GemmDesc g2 = g;
+  g2.K = Hh; g2.A = hid; g2.a_sm = Hh; g2.W = m->Wa2; g2.w_rows = L_NS * d; g2.N = L_NS * d;
+  g2.bias = m->ba2; g2.act = ACT_NONE;
+  g2.out = rmap(out, 0, d);
+  g2.out.sc = N * d;
+  g2.out.split = d;
+  return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
+}
+
+extern "C" onetrans_status onetrans_tokenize_autosplit_static(const onetrans_model* m, const void* feats,
+                                                              int64_t N, void* ns_tokens, void* stream) {
+  if (!m || !feats || !ns_tokens || !aligned(feats, 16) || !aligned(ns_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
+  if (N < 0 || N > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
+  if (!m->Wa1 || !m->ba1 || !m->Wa2 || !m->ba2 || m->cfg.ns_feat_dim < 1 || m->cfg.ns_hidden < 1)
+    return ONETRANS_ERR_UNSUPPORTED;
+  if ((size_t)N * m->cfg.ns_hidden * m->es > kStaticScratchBytes) return ONETRANS_ERR_CAPACITY;
+  if (N == 0) return ONETRANS_OK;
+  void* hid = nullptr;
+  OT_TRY(static_scratch(&hid));
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? autosplit_with_hidden<__nv_bfloat16>(m, feats, N, ns_tokens, hid, st)
+                 : autosplit_with_hidden<float>(m, feats, N, ns_tokens, hid, st);
+}
