@@ -169,8 +169,8 @@ class KVServing:
         self.S_pin = torch.from_numpy(self.S_h).to(torch.bfloat16).pin_memory()
         self.F_pin = torch.from_numpy(self.F_h).to(torch.bfloat16).pin_memory()
         m = self.model
-        self.ns = torch.empty(sh.L_NS, self.U * self.C, sh.d, dtype=torch.bfloat16, device=dev)
-        self.out = torch.empty(sh.L_NS, self.U * self.C, sh.d, dtype=torch.float32, device=dev)
+        self.ns = torch.empty(self.U * self.C, sh.L_NS, sh.d, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(self.U * self.C, sh.L_NS, sh.d, dtype=torch.float32, device=dev)
         self.out_pin = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
         self.ws_a = m.workspace(ot.OP_AUTOSPLIT, self.U * self.C)
         self.ws_1 = m.workspace(ot.OP_STAGE1, self.U, wl.L_S)

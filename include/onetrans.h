@@ -174,7 +174,7 @@ ONETRANS_API onetrans_status onetrans_cache_row_ptr(const onetrans_cache* c, int
  * Auto-split NS tokenizer ([FR] 7.5.0): ns = Split(MLP(feats), L_NS) with
  * MLP = Linear(F->H) + ba1 -> GELU-tanh -> Linear(H->L_NS*d) + ba2.
  *   feats     [N, F]
- *   ns_tokens [L_NS, N, d]  token-major output (token t = MLP columns t*d..) */
+ *   ns_tokens [N, L_NS, d]  (token t of row i = MLP output columns t*d..t*d+d-1) */
 ONETRANS_API onetrans_status onetrans_tokenize_autosplit(const onetrans_model* m,
                                             const void* feats, int64_t N,
                                             void* ns_tokens, void* ws,
@@ -212,8 +212,8 @@ ONETRANS_API onetrans_status onetrans_stage1_encode(const onetrans_model* m,
  * candidate attends in one softmax to the slot's cached S keys and its own
  * NS keys 0..j, then passes through its token-specific FFN.  All slots must
  * hold the same S length; at most 65536 users per call.
- *   ns_tokens [L_NS, C_tot, d] token-major input;
- *   ns_out    [L_NS, C_tot, d] float32. */
+ *   ns_tokens [C_tot, L_NS, d] (candidate-major, as the tokenizer writes it);
+ *   ns_out    [C_tot, L_NS, d] float32. */
 ONETRANS_API onetrans_status onetrans_stage2_score(const onetrans_model* m,
                                       const onetrans_cache* c,
                                       const int32_t* slots, int32_t U,

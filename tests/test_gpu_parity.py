@@ -39,15 +39,15 @@ def run_forward(b, X0):
 
 
 def run_stage12(b, S, NS_tok, offsets, slots=None):
-    """S: [U, L_S, d]; NS_tok: [L_NS, C, d]; returns (cache obj, ns_out)."""
+    """S: [U, L_S, d]; NS_tok: [C, L_NS, d]; returns (cache obj, ns_out [C, L_NS, d])."""
     m = b.model
     U, L_S, d = S.shape
     slots = list(range(U)) if slots is None else slots
     cache = ot.Cache(m, max(slots) + 1, L_S + 64)
     ws1 = m.workspace(ot.OP_STAGE1, U, L_S)
     ot.onetrans_stage1_encode(m, cache, slots, to_dev(S, tdt(b.dtype)), ws1)
-    C = NS_tok.shape[1]
-    out = torch.empty(b.shape.L_NS, C, d, dtype=torch.float32, device="cuda")
+    C = NS_tok.shape[0]
+    out = torch.empty(C, b.shape.L_NS, d, dtype=torch.float32, device="cuda")
     ws2 = m.workspace(ot.OP_STAGE2, C, L_S)
     ot.onetrans_stage2_score(m, cache, slots, offsets, to_dev(NS_tok, tdt(b.dtype)), out, ws2)
     torch.cuda.synchronize()
@@ -66,16 +66,15 @@ def test_tiny_fp32_end_to_end():
     U, C = wl.users, wl.cands
     S = np.stack([O.merge_intent_order([raw["seq0"][u], raw["seq1"][u]], b.W) for u in range(U)]).astype(np.float32)
     feats = raw["feats"]
-    ns = torch.empty(sh.L_NS, U * C, sh.d, dtype=torch.float32, device="cuda")
+    ns = torch.empty(U * C, sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
     ot.onetrans_tokenize_autosplit(b.model, to_dev(feats, torch.float32), ns,
                                    b.model.workspace(ot.OP_AUTOSPLIT, U * C))
     torch.cuda.synchronize()
-    ns_ref = O.autosplit(feats, b.W, sh.L_NS).transpose(1, 0, 2)  # [L_NS, N, d], oracle's own
+    ns_ref = O.autosplit(feats, b.W, sh.L_NS)                    # [N, L_NS, d], oracle's own
     assert rel_err(to_np(ns), ns_ref) <= TOL["fp32"]
     # each side runs the stack on its own tokens: GPU tokens -> GPU, oracle tokens -> oracle
-    X0_gpu = torch.cat([torch.from_numpy(S).cuda()[torch.arange(U * C) // C],
-                        ns.permute(1, 0, 2)], dim=1).contiguous()
-    X0_ref = np.stack([np.concatenate([S[c // C], ns_ref[:, c]]) for c in range(U * C)])
+    X0_gpu = torch.cat([torch.from_numpy(S).cuda()[torch.arange(U * C) // C], ns], dim=1).contiguous()
+    X0_ref = np.stack([np.concatenate([S[c // C], ns_ref[c]]) for c in range(U * C)])
     out_f = torch.empty(U * C, S.shape[1] + sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
     ot.onetrans_forward(b.model, X0_gpu, out_f, b.model.workspace(ot.OP_FORWARD, U * C, S.shape[1]))
     torch.cuda.synchronize()
@@ -84,15 +83,15 @@ def test_tiny_fp32_end_to_end():
     m = b.model
     cache = ot.Cache(m, U, S.shape[1])
     ot.onetrans_stage1_encode(m, cache, [0, 1], torch.from_numpy(S).cuda(), m.workspace(ot.OP_STAGE1, U, S.shape[1]))
-    out = torch.empty(sh.L_NS, U * C, sh.d, dtype=torch.float32, device="cuda")
+    out = torch.empty(U * C, sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
     ot.onetrans_stage2_score(m, cache, [0, 1], [0, C, 2 * C], ns, out, m.workspace(ot.OP_STAGE2, U * C, S.shape[1]))
     torch.cuda.synchronize()
     out = to_np(out)
     for c in range(U * C):
         kv = O.stage1(S[c // C], b.W, sh.L_NS, sh.n_heads, EPS)
-        r = O.stage2(kv, ns_ref[:, c], b.W, sh.n_heads, EPS)
-        assert rel_err(out[:, c], r) <= TOL["fp32"]
-        assert rel_err(out[:, c], ref[c, -sh.L_NS:]) <= TOL["fp32"]
+        r = O.stage2(kv, ns_ref[c], b.W, sh.n_heads, EPS)
+        assert rel_err(out[c], r) <= TOL["fp32"]
+        assert rel_err(out[c], ref[c, -sh.L_NS:]) <= TOL["fp32"]
 
 
 # ------------------------------------------------------- small, bf16/fp32 --
@@ -137,7 +136,7 @@ def test_stage1_stage2_small_ragged(dtype, policy):
     S = gen_normal(7, (U, L_S, sh.d), dtype)
     counts = [2, 0, 131]
     offs = np.concatenate([[0], np.cumsum(counts)]).tolist()
-    NS = gen_normal(8, (sh.L_NS, offs[-1], sh.d), dtype)
+    NS = gen_normal(8, (offs[-1], sh.L_NS, sh.d), dtype)
     slots = [4, 0, 2]
     cache, out = run_stage12(b, S, NS, offs, slots)
     for u in range(U):
@@ -148,8 +147,8 @@ def test_stage1_stage2_small_ragged(dtype, policy):
             assert rel_err(got[0], K) <= TOL[dtype]
             assert rel_err(got[1], V) <= TOL[dtype]
         for c in range(offs[u], offs[u + 1]):
-            r = O.stage2(kv, NS[:, c], b.W, sh.n_heads, EPS)
-            assert rel_err(out[:, c], r) <= TOL[dtype], (u, c)
+            r = O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)
+            assert rel_err(out[c], r) <= TOL[dtype], (u, c)
 
 
 @pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
@@ -167,8 +166,8 @@ def test_append_small_crosses_page_boundary(dtype, policy):
     ot.onetrans_cache_append(m, cache, [1, 0], to_dev(ev, tdt(dtype)),
                              torch.from_numpy(ty).cuda(), m.workspace(ot.OP_APPEND, U, dL))
     torch.cuda.synchronize()
-    NS = gen_normal(12, (sh.L_NS, 4, sh.d), dtype)
-    out = torch.empty(sh.L_NS, 4, sh.d, dtype=torch.float32, device="cuda")
+    NS = gen_normal(12, (4, sh.L_NS, sh.d), dtype)
+    out = torch.empty(4, sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
     ot.onetrans_stage2_score(m, cache, [1, 0], [0, 2, 4], to_dev(NS, tdt(dtype)), out,
                              m.workspace(ot.OP_STAGE2, 4, L_S + dL))
     torch.cuda.synchronize()
@@ -182,8 +181,8 @@ def test_append_small_crosses_page_boundary(dtype, policy):
             assert rel_err(got[0], K) <= TOL[dtype]
             assert rel_err(got[1], V) <= TOL[dtype]
         for c in range(2 * u, 2 * u + 2):
-            r = O.stage2(kv, NS[:, c], b.W, sh.n_heads, EPS)
-            assert rel_err(out[:, c], r) <= TOL[dtype]
+            r = O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)
+            assert rel_err(out[c], r) <= TOL[dtype]
 
 
 @pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
@@ -193,10 +192,10 @@ def test_autosplit_ragged_rows(dtype, policy):
     b = build(sh, 105, dtype)
     N = 300
     feats = gen_normal(13, (N, sh.ns_feat), dtype)
-    ns = torch.empty(sh.L_NS, N, sh.d, dtype=tdt(dtype), device="cuda")
+    ns = torch.empty(N, sh.L_NS, sh.d, dtype=tdt(dtype), device="cuda")
     ot.onetrans_tokenize_autosplit(b.model, to_dev(feats, tdt(dtype)), ns, b.model.workspace(ot.OP_AUTOSPLIT, N))
     torch.cuda.synchronize()
-    ref = O.autosplit(feats, b.W, sh.L_NS).transpose(1, 0, 2)
+    ref = O.autosplit(feats, b.W, sh.L_NS)
     assert rel_err(to_np(ns), ref) <= TOL[dtype]
 
 
@@ -269,12 +268,12 @@ def test_kv_serving_full_size_sampled():
     S = gen_normal(wl.seed_inputs, (U, wl.L_S, sh.d), "bf16")
     feats = gen_normal(wl.seed_inputs + 100, (U * C, sh.ns_feat), "bf16")
     m = b.model
-    ns = torch.empty(sh.L_NS, U * C, sh.d, dtype=torch.bfloat16, device="cuda")
+    ns = torch.empty(U * C, sh.L_NS, sh.d, dtype=torch.bfloat16, device="cuda")
     ot.onetrans_tokenize_autosplit(m, to_dev(feats, torch.bfloat16), ns, m.workspace(ot.OP_AUTOSPLIT, U * C))
     cache = ot.Cache(m, U, wl.L_S)
     ot.onetrans_stage1_encode(m, cache, list(range(U)), to_dev(S, torch.bfloat16),
                               m.workspace(ot.OP_STAGE1, U, wl.L_S))
-    out = torch.empty(sh.L_NS, U * C, sh.d, dtype=torch.float32, device="cuda")
+    out = torch.empty(U * C, sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
     ot.onetrans_stage2_score(m, cache, list(range(U)), [u * C for u in range(U + 1)], ns, out,
                              m.workspace(ot.OP_STAGE2, U * C, wl.L_S))
     torch.cuda.synchronize()
@@ -283,9 +282,9 @@ def test_kv_serving_full_size_sampled():
         kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, wl.pyramid)
         for c in (u * C, u * C + 317, u * C + C - 1):
             ns_ref = O.autosplit(feats[c:c + 1], b.W, sh.L_NS)[0]     # the oracle's own tokens
-            assert rel_err(NS[:, c], ns_ref) <= TOL["bf16"]
+            assert rel_err(NS[c], ns_ref) <= TOL["bf16"]
             r = O.stage2(kv, ns_ref, b.W, sh.n_heads, EPS)
-            assert rel_err(out[:, c], r) <= TOL["bf16"]
+            assert rel_err(out[c], r) <= TOL["bf16"]
 
 
 def test_s_forward_full_size_sampled():
@@ -311,8 +310,8 @@ def test_append_full_size_sampled():
     ot.onetrans_cache_append(m, cache, list(range(U)), to_dev(ev, torch.bfloat16),
                              torch.from_numpy(ty).cuda(), m.workspace(ot.OP_APPEND, U, dL))
     C = wl.cands
-    NS = gen_normal(wl.seed_inputs + 400, (sh.L_NS, U * C, sh.d), "bf16")
-    out = torch.empty(sh.L_NS, U * C, sh.d, dtype=torch.float32, device="cuda")
+    NS = gen_normal(wl.seed_inputs + 400, (U * C, sh.L_NS, sh.d), "bf16")
+    out = torch.empty(U * C, sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
     ot.onetrans_stage2_score(m, cache, list(range(U)), [u * C for u in range(U + 1)],
                              to_dev(NS, torch.bfloat16), out, m.workspace(ot.OP_STAGE2, U * C, wl.L_S + dL))
     torch.cuda.synchronize()
@@ -323,7 +322,7 @@ def test_append_full_size_sampled():
     got = to_np(cache.gather(u, 5, wl.L_S + dL))
     assert rel_err(got[0], kv[5][0]) <= TOL["bf16"]
     for c in (u * C, u * C + C - 1):
-        assert rel_err(out[:, c], O.stage2(kv, NS[:, c], b.W, sh.n_heads, EPS)) <= TOL["bf16"]
+        assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL["bf16"]
 
 
 def test_l_forward_full_size_sampled():

@@ -25,9 +25,9 @@ def test_static_scratch_autosplit_matches_workspace_entry_point():
     m = b.model
     for call, N in enumerate((1000, 2730)):      # 2730 rows fill the 16 MiB array at H = 3072
         feats = to_dev(gen_normal(400 + call, (N, sh.ns_feat), "bf16"), torch.bfloat16)
-        ref = torch.empty(sh.L_NS, N, sh.d, dtype=torch.bfloat16, device="cuda")
+        ref = torch.empty(N, sh.L_NS, sh.d, dtype=torch.bfloat16, device="cuda")
         ot.onetrans_tokenize_autosplit(m, feats, ref, m.workspace(ot.OP_AUTOSPLIT, N))
-        got = torch.full((sh.L_NS, N, sh.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        got = torch.full((N, sh.L_NS, sh.d), float("nan"), dtype=torch.bfloat16, device="cuda")
         st = torch.cuda.current_stream().cuda_stream
         status = ot.lib.onetrans_tokenize_autosplit_static(m.handle, feats.data_ptr(), N, got.data_ptr(), st)
         assert status == ot.OK
@@ -36,7 +36,7 @@ def test_static_scratch_autosplit_matches_workspace_entry_point():
     # one row past the array's capacity is refused before any launch
     too_many = 2731
     feats = torch.zeros(too_many, sh.ns_feat, dtype=torch.bfloat16, device="cuda")
-    out = torch.empty(sh.L_NS, too_many, sh.d, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(too_many, sh.L_NS, sh.d, dtype=torch.bfloat16, device="cuda")
     assert ot.lib.onetrans_tokenize_autosplit_static(m.handle, feats.data_ptr(), too_many, out.data_ptr(),
                                                      None) == ot.ERR_CAPACITY
     assert ot.onetrans_device_status() == 0

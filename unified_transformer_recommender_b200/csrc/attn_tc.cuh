@@ -1,21 +1,29 @@
 // Tensor-core attention for the bf16 path (sm_100a), head dim 64.
 //
-// One CTA owns 128 queries of one head.  K/V tiles of 128 keys (two 64-token
-// cache pages) are streamed by TMA through a 2-deep shared-memory ring.
-// Per key tile:  S = Q K^T (tcgen05.mma into TMEM, fp32) -> four softmax
-// warps read their query row back (tcgen05.ld: one row per thread, so the
-// row max and row sum stay inside the thread), apply the mask, update the
-// running max / sum (online softmax in base 2), write P = exp2(S - m) as bf16
-// into shared memory -> O_tile = P V (tcgen05.mma, V as an MN-major operand)
-// -> the softmax warps fold O_tile into their register accumulator.
+// One CTA owns 128 query rows of one head.  K/V tiles of 128 keys are
+// streamed by TMA through a 2-deep shared-memory ring.  Per key tile:
+//   S = Q K^T          tcgen05.mma into TMEM (fp32)
+//   softmax            four warps read their query row back with tcgen05.ld
+//                      (one row per thread, so the row max and sum stay in the
+//                      thread), mask, update the running max and sum (online
+//                      softmax in base 2: queries arrive pre-scaled by
+//                      1/sqrt(d_h)*log2(e)), write P = 2^(S - m) as bf16 into
+//                      shared memory
+//   O_tile = P V       tcgen05.mma, V read as an MN-major operand
+//   fold               the softmax warps add O_tile into their registers
+// MMA of tile t+1 overlaps the fold of tile t; two CTAs share an SM so one's
+// softmax overlaps the other's MMAs.
 //
-// Two query kinds share the kernel:
+// Query kinds:
 //  * MODE_CAUSAL  (Stage I, forward, append): query t of sequence b sits at
-//    key position q_pos0 + t and sees keys 0..q_pos0 + t (the pyramid's tail
-//    query set: only the last Lq rows are queries, keys span the layer input).
-//  * MODE_STAGE2: the queries are NS token j of up to 128 candidates of one
-//    user; they see every cached S key of the user (s_len keys) and then,
-//    in the same softmax, their own NS keys 0..j, folded in on CUDA cores.
+//    key position q_pos0 + t and sees keys 0..q_pos0 + t, all from 64-token
+//    KV-cache pages.  Only the tail rows are queries (the pyramid's Q set);
+//    keys span the layer input.
+//  * MODE_STAGE2: rows are NS tokens of up to floor(128/L_NS) candidates of one
+//    user, candidate-major (row r = candidate r / L_NS, token r % L_NS).  They
+//    see every cached S key of the user, then one more key tile holding the
+//    same candidates' own NS keys, masked to (same candidate, token <= own):
+//    one softmax over the union, every product on tensor cores.
 //
 // Warp roles (192 threads): warps 0-3 softmax/epilogue, warp 4 TMA, warp 5 MMA.
 #pragma once
@@ -31,14 +39,12 @@ struct TcAttnArgs {
   int Lq, q_pos0;
   RowMap o;
   // stage II
-  const int* tiles;           // {user, c0, c1} per blockIdx.x
-  const __nv_bfloat16* qkv;   // [L_NS, C_tot, 3d]
-  __nv_bfloat16* o2;          // [L_NS, C_tot, d]
-  int C_tot, s_len;
+  const int* tiles;   // {user, c0, c1} per blockIdx.x
+  __nv_bfloat16* o2;  // [C_tot, L_NS, d]
+  int L_NS, s_len;
   // shared
   KVStore kv;
   int H;
-  float scale_log2;  // 1/sqrt(d_h) * log2(e)
 };
 
 struct AttnCfg {
@@ -48,7 +54,8 @@ struct AttnCfg {
   static constexpr int PAGE_BYTES = 64 * DH * 2;  // one 64-token page of one head
   static constexpr int STAGES = 2;
   static constexpr int P_BYTES = BM * BN * 2;     // 32 KB
-  static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + 1024 + 256;
+  static constexpr int BAR_BYTES = 128;
+  static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + BAR_BYTES;
   static constexpr int TMEM_COLS = 256;           // S: cols 0..127, O tile: 128..191
 };
 
@@ -56,47 +63,60 @@ __device__ inline int kv_page_id(const KVStore& kv, int b, int page_idx) {
   return kv.table ? kv.table[kv.row_off[b] + page_idx] : b * kv.pps + page_idx;
 }
 
-__global__ void __launch_bounds__(192, 1)
+__device__ inline float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+enum : int { kErrSmemAlign = 102 };
+
+__global__ void __launch_bounds__(192, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
-                   const TcAttnArgs a) {
+                   const __grid_constant__ CUtensorMap tmNS, const TcAttnArgs a) {
   using C = AttnCfg;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + C::Q_BYTES;                       // [stage][K|V][128 keys][64]
-  uint8_t* sP = sKV + C::STAGES * 2 * C::KV_BYTES;      // [2 key blocks][128 rows][64]
+  uint8_t* sKV = sQ + C::Q_BYTES;                   // [stage][K|V][128 keys][64]
+  uint8_t* sP = sKV + C::STAGES * 2 * C::KV_BYTES;  // [2 key blocks][128 rows][64]
   uint64_t* bars = (uint64_t*)(sP + C::P_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;
   uint64_t* p_full = bars + 6;
   uint64_t* o_full = bars + 7;
   uint32_t* tmem_slot = (uint32_t*)(bars + 8);
 
+  // the swizzled tiles need 1024-byte alignment; refuse to run without it
+  if (smem_u32(smem) & 1023) {
+    if (threadIdx.x == 0) flag_error(kErrSmemAlign);
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
 
   // ---- work of this CTA
-  int b, q_row0, n_keys, kmax;   // n_keys: keys the tile loop covers (pre-mask)
-  int user = 0, c0 = 0, c1 = 0, j = 0;
+  int b, row0, n_keys_s, kmax, nt, n_rows = C::BM;
+  int c0 = 0;
   if (a.mode == MODE_CAUSAL) {
     b = blockIdx.z;
-    q_row0 = blockIdx.x * C::BM;
-    const int t_last = min(a.Lq, q_row0 + C::BM) - 1;
+    row0 = blockIdx.x * C::BM;
+    const int t_last = min(a.Lq, row0 + C::BM) - 1;
     kmax = a.q_pos0 + t_last;
-    n_keys = kmax + 1;
+    n_keys_s = kmax + 1;
+    nt = (n_keys_s + C::BN - 1) / C::BN;
   } else {
-    user = a.tiles[blockIdx.x * 3 + 0];
+    b = a.tiles[blockIdx.x * 3 + 0];
     c0 = a.tiles[blockIdx.x * 3 + 1];
-    c1 = a.tiles[blockIdx.x * 3 + 2];
-    j = blockIdx.z;
-    b = user;
-    q_row0 = c0;
+    const int c1 = a.tiles[blockIdx.x * 3 + 2];
+    row0 = c0 * a.L_NS;
+    n_rows = (c1 - c0) * a.L_NS;
     kmax = a.s_len - 1;
-    n_keys = a.s_len;
+    n_keys_s = a.s_len;
+    nt = (n_keys_s + C::BN - 1) / C::BN + 1;  // + the tile of own NS keys
   }
-  const int nt = (n_keys + C::BN - 1) / C::BN;
+  const int nt_s = (n_keys_s + C::BN - 1) / C::BN;  // tiles from the KV pages
   const int n_pages_used = (kmax + 1 + 63) / 64;
 
   if (threadIdx.x == 0) {
@@ -111,6 +131,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 4 && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmKV);
+    if (a.mode == MODE_STAGE2) prefetch_tmap(&tmNS);
   }
   if (warp == 5) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
@@ -123,21 +144,28 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0 && nt > 0) {
       mbar_expect_tx(q_full, C::Q_BYTES);
-      if (a.mode == MODE_CAUSAL) tma_load_3d(&tmQ, q_full, sQ, h * C::DH, q_row0, b);
-      else tma_load_3d(&tmQ, q_full, sQ, h * C::DH, q_row0, j);
+      if (a.mode == MODE_CAUSAL) tma_load_3d(&tmQ, q_full, sQ, h * C::DH, row0, b);
+      else tma_load_3d(&tmQ, q_full, sQ, h * C::DH, row0, 0);
       for (int kt = 0; kt < nt; ++kt) {
         const int s = kt & 1;
         if (kt >= 2 && !mbar_wait(&kv_empty[s], ((kt >> 1) - 1) & 1)) break;
-        mbar_expect_tx(&kv_full[s], 4 * C::PAGE_BYTES);
+        mbar_expect_tx(&kv_full[s], 2 * C::KV_BYTES);
         uint8_t* sk = sKV + s * 2 * C::KV_BYTES;
         uint8_t* sv = sk + C::KV_BYTES;
+        if (kt < nt_s) {
 #pragma unroll
-        for (int hp = 0; hp < 2; ++hp) {
-          const int pi = kt * 2 + hp;
-          // pages past the last used one read as zeros (out-of-range page coordinate)
-          const int pg = pi < n_pages_used ? kv_page_id(a.kv, b, pi) : a.kv.n_pages;
-          tma_load_4d(&tmKV, &kv_full[s], sk + hp * C::PAGE_BYTES, 0, 0, h, pg);
-          tma_load_4d(&tmKV, &kv_full[s], sv + hp * C::PAGE_BYTES, 0, 0, a.H + h, pg);
+          for (int hp = 0; hp < 2; ++hp) {
+            const int pi = kt * 2 + hp;
+            // pages past the last used one read as zeros (out-of-range page coordinate)
+            const int pg = pi < n_pages_used ? kv_page_id(a.kv, b, pi) : a.kv.n_pages;
+            tma_load_4d(&tmKV, &kv_full[s], sk + hp * C::PAGE_BYTES, 0, 0, h, pg);
+            tma_load_4d(&tmKV, &kv_full[s], sv + hp * C::PAGE_BYTES, 0, 0, a.H + h, pg);
+          }
+        } else {
+          // own NS keys of this CTA's candidates: the K and V column blocks of the same rows
+          const int d = a.H * C::DH;
+          tma_load_3d(&tmNS, &kv_full[s], sk, d + h * C::DH, row0, 0);
+          tma_load_3d(&tmNS, &kv_full[s], sv, 2 * d + h * C::DH, row0, 0);
         }
       }
     }
@@ -188,32 +216,53 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------- softmax + epilogue
     const int r = warp * 32 + lane;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int qpos = a.q_pos0 + q_row0 + r;  // causal: key position of this query
+    // causal: last visible key of this row; stage II: candidate and token of this row
+    const int qpos = a.q_pos0 + row0 + r;
+    const int cand = a.mode == MODE_STAGE2 ? r / a.L_NS : 0;
+    const int tok = a.mode == MODE_STAGE2 ? r - cand * a.L_NS : 0;
+    // the earliest query of the CTA bounds which tiles need no mask
+    const int qpos_min = a.q_pos0 + row0;
     float o[64];
 #pragma unroll
     for (int e = 0; e < 64; ++e) o[e] = 0.f;
     float m = -INFINITY, l = 0.f;
-    const float sc = a.scale_log2;
     for (int kt = 0; kt < nt; ++kt) {
       if (!mbar_wait(s_full, kt & 1)) break;
       tc_fence_after();
       const int kbase = kt * C::BN;
-      const int vis_end = a.mode == MODE_CAUSAL ? min(qpos + 1, n_keys) : n_keys;  // keys < vis_end visible
-      // pass 1: masked row max (TMEM is re-read in pass 2 instead of holding 128 scores)
+      const bool ns_tile = kt >= nt_s;
+      // visible keys of this row in this tile: [0, vis) for S tiles; NS tile: a
+      // same-candidate run [lo, hi)
+      int lo = 0, hi = C::BN;
+      if (ns_tile) {
+        lo = cand * a.L_NS;
+        hi = (r < n_rows) ? lo + tok + 1 : lo;
+      } else {
+        const int vis_end = a.mode == MODE_CAUSAL ? min(qpos + 1, n_keys_s) : n_keys_s;
+        hi = min(max(vis_end - kbase, 0), C::BN);
+      }
+      const bool full = !ns_tile && (a.mode == MODE_CAUSAL ? (kbase + C::BN - 1 <= qpos_min && kbase + C::BN <= n_keys_s)
+                                                          : (kbase + C::BN <= n_keys_s));
+      // pass 1: row max of the visible logits
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float sv[32];
         tmem_ld32(tS + lane_base + c * 32, sv);
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (kbase + c * 32 + i < vis_end) mx = fmaxf(mx, sv[i] * sc);
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, sv[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= lo && c * 32 + i < hi) mx = fmaxf(mx, sv[i]);
+        }
       }
       const float m_new = fmaxf(m, mx);
-      const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m - m_new);
+      const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m - m_new);
       const float mref = (m_new == -INFINITY) ? 0.f : m_new;
       if (kt > 0) {
-        // PV of the previous tile is done: fold it in, and P's buffer is free again
+        // P.V of the previous tile is done: fold it in; P's buffer is free again
         if (!mbar_wait(o_full, (kt - 1) & 1)) break;
         tc_fence_after();
 #pragma unroll
@@ -224,17 +273,25 @@ __global__ void __launch_bounds__(192, 1)
           for (int e = 0; e < 32; ++e) o[c * 32 + e] = (o[c * 32 + e] + ov[e]) * alpha;
         }
       }
-      // pass 2: P = exp2(S - m) as bf16 into the K-major, 128-byte-swizzled A
+      // pass 2: P = 2^(S - m) as bf16 into the K-major, 128-byte-swizzled A
       // operand of P.V (row r, key k -> block k/64, 16-byte chunk (k%64)/8 ^ (r%8))
       float rs = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float sv[32];
         tmem_ld32(tS + lane_base + c * 32, sv);
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = (kbase + c * 32 + i < vis_end) ? exp2f(sv[i] * sc - mref) : 0.f;
-          rs += sv[i];
+          for (int i = 0; i < 32; ++i) {
+            sv[i] = ex2(sv[i] - mref);
+            rs += sv[i];
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            sv[i] = (c * 32 + i >= lo && c * 32 + i < hi) ? ex2(sv[i] - mref) : 0.f;
+            rs += sv[i];
+          }
         }
         uint8_t* rowp = sP + (c >> 1) * (128 * 128) + r * 128;
 #pragma unroll
@@ -249,14 +306,11 @@ __global__ void __launch_bounds__(192, 1)
       }
       l = l * alpha + rs;
       m = m_new;
-      // keys past the last valid one may hold stale bits: zero their V rows
-      if (kt == nt - 1) {
-        const int key = kbase + r;
-        if (key > kmax) {
-          uint4* vrow = (uint4*)(sKV + (kt & 1) * 2 * C::KV_BYTES + C::KV_BYTES + r * 128);
+      // keys past the last valid cache key may hold stale bits: zero their V rows
+      if (kt == nt_s - 1 && kbase + r > kmax) {
+        uint4* vrow = (uint4*)(sKV + (kt & 1) * 2 * C::KV_BYTES + C::KV_BYTES + r * 128);
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) vrow[ch] = make_uint4(0, 0, 0, 0);
-        }
+        for (int ch = 0; ch < 8; ++ch) vrow[ch] = make_uint4(0, 0, 0, 0);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
@@ -272,51 +326,20 @@ __global__ void __launch_bounds__(192, 1)
         for (int e = 0; e < 32; ++e) o[c * 32 + e] += ov[e];
       }
     }
-    if (a.mode == MODE_CAUSAL) {
-      const int t = q_row0 + r;
-      if (t < a.Lq) {
-        const float inv = 1.f / l;
+    const float inv = 1.f / l;
 #pragma unroll
-        for (int e = 0; e < 64; ++e) o[e] *= inv;
+    for (int e = 0; e < 64; ++e) o[e] *= inv;
+    if (a.mode == MODE_CAUSAL) {
+      const int t = row0 + r;
+      if (t < a.Lq) {
         __nv_bfloat16* dst = (__nv_bfloat16*)a.o.base + rm_off(a.o, b, t, h * 64);
         store_bf16x32(dst, o);
         store_bf16x32(dst + 32, o + 32);
       }
-    } else {
-      const int c = c0 + r;
-      if (c < c1) {
-        // own NS keys 0..j of this candidate, in the same softmax
-        const int d = a.H * 64;
-        const long long rs3 = 3LL * d;
-        float q[64];
-        const __nv_bfloat16* qp = a.qkv + ((long long)j * a.C_tot + c) * rs3 + h * 64;
-        load_bf16x32(qp, q);
-        load_bf16x32(qp + 32, q + 32);
-        for (int i = 0; i <= j; ++i) {
-          const __nv_bfloat16* kp = a.qkv + ((long long)i * a.C_tot + c) * rs3 + d + h * 64;
-          float kv[64];
-          load_bf16x32(kp, kv);
-          load_bf16x32(kp + 32, kv + 32);
-          float s = 0.f;
-#pragma unroll
-          for (int e = 0; e < 64; ++e) s = fmaf(q[e], kv[e], s);
-          s *= sc;
-          const float m_new = fmaxf(m, s);
-          const float alpha = exp2f(m - m_new), p = exp2f(s - m_new);
-          load_bf16x32(kp + d, kv);
-          load_bf16x32(kp + d + 32, kv + 32);
-#pragma unroll
-          for (int e = 0; e < 64; ++e) o[e] = fmaf(p, kv[e], o[e] * alpha);
-          l = l * alpha + p;
-          m = m_new;
-        }
-        const float inv = 1.f / l;
-#pragma unroll
-        for (int e = 0; e < 64; ++e) o[e] *= inv;
-        __nv_bfloat16* dst = a.o2 + ((long long)j * a.C_tot + c) * d + h * 64;
-        store_bf16x32(dst, o);
-        store_bf16x32(dst + 32, o + 32);
-      }
+    } else if (r < n_rows) {
+      __nv_bfloat16* dst = a.o2 + (long long)(row0 + r) * (a.H * 64) + h * 64;
+      store_bf16x32(dst, o);
+      store_bf16x32(dst + 32, o + 32);
     }
   }
   tc_fence_before();
@@ -349,8 +372,8 @@ inline bool tc_attn_supported(const AttnDesc& a) {
          a.q.sb % 8 == 0 && rowmap_vec_ok(a.o) && !a.o.f32;
 }
 
-inline onetrans_status attn_launch_common(const CUtensorMap& tq, const CUtensorMap& tkv, const TcAttnArgs& args,
-                                          dim3 grid, cudaStream_t st) {
+inline onetrans_status attn_launch_common(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tns,
+                                          const TcAttnArgs& args, dim3 grid, cudaStream_t st) {
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg::SMEM) !=
@@ -358,7 +381,7 @@ inline onetrans_status attn_launch_common(const CUtensorMap& tq, const CUtensorM
       return ONETRANS_ERR_CUDA;
     attr_set = true;
   }
-  attn_tc_kernel<<<grid, 192, AttnCfg::SMEM, st>>>(tq, tkv, args);
+  attn_tc_kernel<<<grid, 192, AttnCfg::SMEM, st>>>(tq, tkv, tns, args);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 
@@ -378,36 +401,36 @@ inline onetrans_status tc_attn_launch(const AttnDesc& a, cudaStream_t st) {
   args.o = a.o;
   args.kv = a.kv;
   args.H = a.H;
-  args.scale_log2 = a.scale * 1.4426950408889634f;
   dim3 grid((unsigned)((a.Lq + 127) / 128), (unsigned)a.H, (unsigned)a.B);
-  return attn_launch_common(tq, tkv, args, grid, st);
+  return attn_launch_common(tq, tkv, tkv, args, grid, st);
 }
+
+// Candidates per Stage II tile: whole candidates' NS rows fill at most 128 rows.
+inline int stage2_cands_per_tile(int L_NS) { return L_NS <= 128 ? 128 / L_NS : 0; }
 
 inline bool tc_stage2_supported(const Stage2Desc& a) {
-  return a.dh == 64 && tc_kv_ok(a.kv) && ((uintptr_t)a.qkv % 16) == 0 && ((uintptr_t)a.o % 16) == 0;
+  return a.dh == 64 && stage2_cands_per_tile(a.L_NS) > 0 && tc_kv_ok(a.kv) && ((uintptr_t)a.qkv % 16) == 0 &&
+         ((uintptr_t)a.o % 16) == 0;
 }
 
-// Stage II: `tiles` holds up to 128 candidates of one user per entry.
 inline onetrans_status tc_stage2_launch(const Stage2Desc& a, int n_tiles, cudaStream_t st) {
   CUtensorMap tq, tkv;
   const uint64_t d = (uint64_t)a.H * a.dh;
-  if (!make_tmap_3d(&tq, a.qkv, 3 * d, (uint64_t)a.C_tot, (uint64_t)a.L_NS, 3 * d, (uint64_t)a.C_tot * 3 * d, 64,
-                    128, 1) ||
-      !make_tmap_pages(&tkv, a.kv))
+  const uint64_t rows = (uint64_t)a.C_tot * a.L_NS;
+  // one map serves Q (columns h*64) and the own-NS K/V tile (columns d + h*64, 2d + h*64)
+  if (!make_tmap_3d(&tq, a.qkv, 3 * d, rows, 1, 3 * d, rows * 3 * d, 64, 128, 1) || !make_tmap_pages(&tkv, a.kv))
     return ONETRANS_ERR_CUDA;
   TcAttnArgs args;
   memset(&args, 0, sizeof(args));
   args.mode = MODE_STAGE2;
   args.tiles = a.tiles;
-  args.qkv = (const __nv_bfloat16*)a.qkv;
   args.o2 = (__nv_bfloat16*)a.o;
-  args.C_tot = a.C_tot;
+  args.L_NS = a.L_NS;
   args.s_len = a.s_len;
   args.kv = a.kv;
   args.H = a.H;
-  args.scale_log2 = a.scale * 1.4426950408889634f;
-  dim3 grid((unsigned)n_tiles, (unsigned)a.H, (unsigned)a.L_NS);
-  return attn_launch_common(tq, tkv, args, grid, st);
+  dim3 grid((unsigned)n_tiles, (unsigned)a.H, 1);
+  return attn_launch_common(tq, tkv, tq, args, grid, st);
 }
 
 }  // namespace ot

@@ -62,23 +62,26 @@ struct GemmDesc {
   const void* gamma;
   float eps;
   KVStore kv;
+  int scale_cols;     // output columns n < scale_cols are multiplied by col_scale
+  float col_scale;    // (queries leave the GEMM pre-scaled by 1/sqrt(d_h) * log2(e))
 };
 
+// Queries arrive pre-scaled by 1/sqrt(d_h) * log2(e) (the producing GEMM's
+// epilogue), so q.k is already a base-2 logit.
 struct AttnDesc {
   int B, H, dh, Lq, q_pos0;  // query t of batch b sits at key position q_pos0 + t
   RowMap q, o;                // columns: head h occupies [h*dh, (h+1)*dh)
   KVStore kv;
-  float scale;
 };
 
 // Stage II attention: candidates of one user share the user's cached S keys.
+// Rows are candidate-major: row c*L_NS + j is NS token j of candidate c.
 struct Stage2Desc {
   int H, dh, L_NS, C_tot, s_len, n_users;
   const int* tiles;    // n_tiles x {user, c0, c1}
-  const void* qkv;     // [L_NS, C_tot, 3d] token-major Q|K|V of the NS rows
-  void* o;             // [L_NS, C_tot, d]
+  const void* qkv;     // [C_tot, L_NS, 3d] Q|K|V of the NS rows
+  void* o;             // [C_tot, L_NS, d]
   KVStore kv;          // row_off indexed by user
-  float scale;
 };
 
 __host__ __device__ inline void row_of(const GemmDesc& d, int m, int g, int& b, int& t) {

@@ -141,6 +141,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] += rv[i];
       }
+      if (n < d.scale_cols) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= d.col_scale;
+      }
       if (d.out_kind == OUT_KV) {
         const int dm = d.kv.H * d.kv.dh;
         const int kind = n / dm, cc = n - kind * dm, head = cc / d.kv.dh, e = cc - head * d.kv.dh;

@@ -184,6 +184,13 @@ static GemmDesc gdesc_base(const onetrans_model* m) {
   return d;
 }
 
+// Queries leave their GEMM multiplied by 1/sqrt(d_h) * log2(e): the attention
+// kernels then work on base-2 logits directly.
+static void prescale_q(const onetrans_model* m, GemmDesc& g) {
+  g.scale_cols = m->d;
+  g.col_scale = (float)(1.4426950408889634 / std::sqrt((double)m->dh));
+}
+
 // ============================================================= launches ==
 template <typename T>
 static onetrans_status launch_rms(GemmDesc d, cudaStream_t st) {
@@ -329,6 +336,7 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
     if (sq > 0) {
       g.m_lo = s - sq; g.M = sq; g.n_lo = 0; g.N = d; g.out_kind = OUT_ROWS;
       g.out = rmap(eoff(q, -(long long)off * d, es), (long long)Lqn * d, d);
+      prescale_q(m, g);
       OT_TRY(launch_gemm<T>(m, g, st));
     }
     // -- NS rows: token j uses its own weights; tile across samples
@@ -338,7 +346,9 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
     gn.W = m->Wqkv_NS[n]; gn.w_sg = 3LL * d * d; gn.w_rows = 3 * d; gn.w_groups = L_NS;
     gn.n_lo = 0; gn.N = d; gn.out_kind = OUT_ROWS;
     gn.out = rmap(eoff(q, -(long long)off * d, es), (long long)Lqn * d, d);
+    prescale_q(m, gn);
     OT_TRY(launch_gemm<T>(m, gn, st));
+    gn.scale_cols = 0;
     gn.n_lo = d; gn.N = 2 * d; gn.out_kind = OUT_KV; gn.kv = kv;
     OT_TRY(launch_gemm<T>(m, gn, st));
     // -- attention of the Lqn tail queries over keys 0..p
@@ -347,7 +357,7 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
     a.B = B; a.H = m->H; a.dh = m->dh; a.Lq = Lqn; a.q_pos0 = off;
     a.q = rmap(q, (long long)Lqn * d, d);
     a.o = rmap(at, (long long)Lqn * d, d);
-    a.kv = kv; a.scale = 1.0f / std::sqrt((float)m->dh);
+    a.kv = kv;
     OT_TRY(launch_attn<T>(m, a, st));
     // -- W^O + residual, then RMSNorm for the FFN (all tail rows share W^O)
     GemmDesc go = gdesc_base(m);
@@ -484,13 +494,14 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
     gq.K = d; gq.A = h; gq.a_sm = d; gq.a_sg = (long long)sn * d; gq.a_mext = sn; gq.a_gext = U;
     gq.W = m->Wqkv_S[n]; gq.w_rows = 3 * d; gq.n_lo = 0; gq.N = d;
     gq.out = rmap(eoff(q, -(long long)(sn - sqn) * d, es), (long long)sqn * d, d);
+    prescale_q(m, gq);
     OT_TRY(launch_gemm<T>(m, gq, st));
     AttnDesc a;
     std::memset(&a, 0, sizeof(a));
     a.B = U; a.H = m->H; a.dh = m->dh; a.Lq = sqn; a.q_pos0 = sn - sqn;
     a.q = rmap(q, (long long)sqn * d, d);
     a.o = rmap(at, (long long)sqn * d, d);
-    a.kv = kv; a.scale = 1.0f / std::sqrt((float)m->dh);
+    a.kv = kv;
     OT_TRY(launch_attn<T>(m, a, st));
     GemmDesc go = gdesc_base(m);
     go.mode = TILE_FLAT; go.M = U * sqn; go.fold = sqn; go.G = 1;
@@ -553,7 +564,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   probe.H = m->H; probe.dh = m->dh; probe.L_NS = L_NS; probe.C_tot = (int)C;
   probe.qkv = qkv; probe.o = at;
   kv_for_cache(c, 0, row_off, probe.kv);
-  const int TQ = stage2_tc(m, probe) ? 128 : 64;
+  const int TQ = stage2_tc(m, probe) ? stage2_cands_per_tile(L_NS) : 64;
   std::vector<int> tiles;
   for (int u = 0; u < U; ++u)
     for (int c0 = offs[u]; c0 < offs[u + 1]; c0 += TQ)
@@ -567,22 +578,25 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
 
   OT_TRY(rms_flat<T>(m, ns_in, false, h, (long long)L_NS * C, m->g_attn[0], st));
   const void* x_in = ns_in;
+  const long long Ld = (long long)L_NS * d;   // candidate stride of [C, L_NS, d] rows
   for (int n = 0; n < m->NL; ++n) {
     const bool last = n + 1 == m->NL;
     void* x_next = last ? ns_out : (n % 2 == 0 ? xa : xb);
+    // token j of every candidate through W_NS,j: fixed t = j, tiled over candidates
     GemmDesc g = gdesc_base(m);
     g.mode = TILE_SAMPLES; g.M = (int)C; g.G = L_NS; g.g_lo = 0; g.grp_base = 0;
-    g.K = d; g.A = h; g.a_sm = d; g.a_sg = C * d; g.a_mext = C; g.a_gext = L_NS;
+    g.K = d; g.A = h; g.a_sm = Ld; g.a_sg = d; g.a_mext = C; g.a_gext = L_NS;
     g.W = m->Wqkv_NS[n]; g.w_sg = 3LL * d * d; g.w_rows = 3 * d; g.w_groups = L_NS;
     g.n_lo = 0; g.N = 3 * d;
-    g.out = rmap(qkv, 3LL * d, C * 3 * d);
+    g.out = rmap(qkv, 3LL * Ld, 3LL * d);
+    prescale_q(m, g);
     OT_TRY(launch_gemm<T>(m, g, st));
     Stage2Desc a;
     std::memset(&a, 0, sizeof(a));
     a.H = m->H; a.dh = m->dh; a.L_NS = L_NS; a.C_tot = (int)C; a.s_len = s[n]; a.n_users = U;
     a.tiles = d_tiles; a.qkv = qkv; a.o = at;
     kv_for_cache(c, n, row_off, a.kv);
-    a.scale = 1.0f / std::sqrt((float)m->dh);
+   
     OT_TRY(launch_stage2_attn<T>(m, a, (int)max_tiles, st));
     GemmDesc go = gdesc_base(m);
     go.mode = TILE_FLAT; go.M = (int)(L_NS * C); go.G = 1;
@@ -594,17 +608,18 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     go.gamma = m->g_ffn[n];
     OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     GemmDesc f = g;
+    f.scale_cols = 0;
     f.A = h2; f.W = m->W1_NS[n]; f.w_sg = (long long)dff * d; f.w_rows = dff; f.N = dff;
     f.bias = m->b1_NS[n]; f.bias_sg = dff; f.act = ACT_GELU;
-    f.out = rmap(hid, dff, C * dff);
+    f.out = rmap(hid, (long long)L_NS * dff, dff);
     OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
-    GemmDesc f2 = g;
-    f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.a_sg = C * dff;
+    GemmDesc f2 = f;
+    f2.K = dff; f2.A = hid; f2.a_sm = (long long)L_NS * dff; f2.a_sg = dff; f2.act = ACT_NONE;
     f2.W = m->W2_NS[n]; f2.w_sg = (long long)d * dff; f2.w_rows = d; f2.N = d;
     f2.bias = m->b2_NS[n]; f2.bias_sg = d;
-    f2.res = rmap32(xm, d, C * d);
-    f2.out = rmap32(x_next, d, C * d);
-    if (!last) { f2.rms = rmap(h, d, C * d); f2.gamma = m->g_attn[n + 1]; }
+    f2.res = rmap32(xm, Ld, d);
+    f2.out = rmap32(x_next, Ld, d);
+    if (!last) { f2.rms = rmap(h, Ld, d); f2.gamma = m->g_attn[n + 1]; }
     OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
     x_in = x_next;
   }
@@ -681,13 +696,14 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     if (last) break;  // the last layer's outputs feed nothing that is cached
     g.n_lo = 0; g.N = d; g.out_kind = OUT_ROWS;
     g.out = rmap(q, (long long)dL * d, d);
+    prescale_q(m, g);
     OT_TRY(launch_gemm<T>(m, g, st));
     AttnDesc a;
     std::memset(&a, 0, sizeof(a));
     a.B = U; a.H = m->H; a.dh = m->dh; a.Lq = dL; a.q_pos0 = s_old;
     a.q = rmap(q, (long long)dL * d, d);
     a.o = rmap(at, (long long)dL * d, d);
-    a.kv = kv; a.kv.pos_off = 0; a.scale = 1.0f / std::sqrt((float)m->dh);
+    a.kv = kv; a.kv.pos_off = 0;
     OT_TRY(launch_attn<T>(m, a, st));
     GemmDesc go = gdesc_base(m);
     go.mode = TILE_FLAT; go.M = (int)R; go.fold = dL; go.G = 1;
@@ -735,9 +751,7 @@ static onetrans_status autosplit_impl(const onetrans_model* m, const void* feats
   GemmDesc g2 = g;
   g2.K = Hh; g2.A = hid; g2.a_sm = Hh; g2.W = m->Wa2; g2.w_rows = L_NS * d; g2.N = L_NS * d;
   g2.bias = m->ba2; g2.act = ACT_NONE;
-  g2.out = rmap(out, 0, d);
-  g2.out.sc = N * d;
-  g2.out.split = d;
+  g2.out = rmap(out, 0, (long long)L_NS * d);   // [N, L_NS, d]: token t = columns [t d, (t+1) d)
   return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
 }
 
@@ -1128,9 +1142,7 @@ static onetrans_status autosplit_with_hidden(const onetrans_model* m, const void
   GemmDesc g2 = g;
   g2.K = Hh; g2.A = hid; g2.a_sm = Hh; g2.W = m->Wa2; g2.w_rows = L_NS * d; g2.N = L_NS * d;
   g2.bias = m->ba2; g2.act = ACT_NONE;
-  g2.out = rmap(out, 0, d);
-  g2.out.sc = N * d;
-  g2.out.split = d;
+  g2.out = rmap(out, 0, (long long)L_NS * d);
   return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
 }
 

@@ -14,6 +14,7 @@ __device__ inline void epilogue_store(const GemmDesc& d, int b, int t, int n, in
   if (d.bias) v += to_f(((const T*)d.bias)[grp * d.bias_sg + d.n_lo + n]);
   if (d.act == ACT_GELU) v = gelu_tanh(v);
   if (d.res.base) v += rm_load<T>(d.res, rm_off(d.res, b, t, n));
+  if (n < d.scale_cols) v *= d.col_scale;
   if (d.out_kind == OUT_KV) {
     const int dm = d.kv.H * d.kv.dh;
     const int kind = n / dm, c = n - kind * dm, head = c / d.kv.dh, e = c - head * d.kv.dh;
@@ -110,11 +111,10 @@ __global__ void __launch_bounds__(64) attn_simt_kernel(AttnDesc a) {
   const int p = a.q_pos0 + t;
   const int t_last = min(a.Lq, (int)(blockIdx.x + 1) * 64) - 1;
   const int kmax = a.q_pos0 + t_last;
-  const float qs = a.scale * 1.4426950408889634f;
   float q[DH], o[DH];
   const T* qp = (const T*)a.q.base + rm_off(a.q, b, valid ? t : 0, h * DH);
 #pragma unroll
-  for (int e = 0; e < DH; ++e) { q[e] = valid ? to_f(qp[e]) * qs : 0.f; o[e] = 0.f; }
+  for (int e = 0; e < DH; ++e) { q[e] = valid ? to_f(qp[e]) : 0.f; o[e] = 0.f; }
   float mrow = -INFINITY, lrow = 0.f;
   const T* pool = (const T*)a.kv.pool;
   for (int k0 = 0; k0 <= kmax; k0 += KT) {
@@ -178,11 +178,10 @@ __global__ void __launch_bounds__(64) stage2_attn_simt_kernel(Stage2Desc a) {
   const int d = a.H * DH;
   const long long rs = 3LL * d;  // row stride of the packed Q|K|V rows
   const T* qkv = (const T*)a.qkv;
-  const float qs = a.scale * 1.4426950408889634f;
   float q[DH], o[DH];
-  const T* qp = qkv + ((long long)j * a.C_tot + (valid ? c : 0)) * rs + h * DH;
+  const T* qp = qkv + ((long long)(valid ? c : 0) * a.L_NS + j) * rs + h * DH;
 #pragma unroll
-  for (int e = 0; e < DH; ++e) { q[e] = valid ? to_f(qp[e]) * qs : 0.f; o[e] = 0.f; }
+  for (int e = 0; e < DH; ++e) { q[e] = valid ? to_f(qp[e]) : 0.f; o[e] = 0.f; }
   float mrow = -INFINITY, lrow = 0.f;
   const T* pool = (const T*)a.kv.pool;
   for (int k0 = 0; k0 < a.s_len; k0 += KT) {
@@ -226,7 +225,7 @@ __global__ void __launch_bounds__(64) stage2_attn_simt_kernel(Stage2Desc a) {
   if (!valid) return;
   // own NS keys 0..j of this candidate
   for (int i = 0; i <= j; ++i) {
-    const T* kp = qkv + ((long long)i * a.C_tot + c) * rs + d + h * DH;
+    const T* kp = qkv + ((long long)c * a.L_NS + i) * rs + d + h * DH;
     const T* vp = kp + d;
     float s = 0.f;
 #pragma unroll
@@ -238,7 +237,7 @@ __global__ void __launch_bounds__(64) stage2_attn_simt_kernel(Stage2Desc a) {
     for (int e = 0; e < DH; ++e) o[e] = fmaf(pr, to_f(vp[e]), o[e] * cf);
     mrow = mn;
   }
-  T* op = (T*)a.o + ((long long)j * a.C_tot + c) * d + h * DH;
+  T* op = (T*)a.o + ((long long)c * a.L_NS + j) * d + h * DH;
   const float inv = 1.f / lrow;
 #pragma unroll
   for (int e = 0; e < DH; ++e) op[e] = from_f<T>(o[e] * inv);
