@@ -69,8 +69,6 @@ __device__ inline float ex2(float x) {
   return y;
 }
 
-enum : int { kErrSmemAlign = 102 };
-
 __global__ void __launch_bounds__(192, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                    const __grid_constant__ CUtensorMap tmNS, const TcAttnArgs a) {

@@ -84,10 +84,13 @@ struct Stage2Desc {
   KVStore kv;          // row_off indexed by user
 };
 
+__host__ __device__ inline void row_of_rows(int mode, int fold, int m, int g, int& b, int& t) {
+  if (mode == TILE_ROWS) { t = m; b = g; }
+  else if (mode == TILE_SAMPLES) { b = m; t = g; }
+  else { b = m / fold; t = m - b * fold; }
+}
 __host__ __device__ inline void row_of(const GemmDesc& d, int m, int g, int& b, int& t) {
-  if (d.mode == TILE_ROWS) { t = m; b = g; }
-  else if (d.mode == TILE_SAMPLES) { b = m; t = g; }
-  else { b = m / d.fold; t = m - b * d.fold; }
+  row_of_rows(d.mode, d.fold, m, g, b, t);
 }
 
 __host__ __device__ inline long long rm_off(const RowMap& r, int b, int t, int n) {

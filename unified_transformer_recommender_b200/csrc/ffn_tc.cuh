@@ -1,0 +1,373 @@
+// Fused tail of a OneTrans block for 128 rows (bf16 path, d = 256, sm_100a):
+//
+//   x_mid  = x + W^O a                      (a: attention output row)
+//   h2     = RMSNorm(x_mid) * g_ffn
+//   x_next = x_mid + W2 GELU(W1 h2 + b1) + b2       (mixed FFN: W1, W2 of the
+//                                                     rows' weight group)
+//   h_next = RMSNorm(x_next) * g_next               (next layer's pre-norm)
+//
+// Only a, x, x_next and h_next touch HBM; x_mid and the d_ff-wide hidden
+// layer stay on chip.  TMEM holds D (256 fp32 columns: W^O a, then x_mid,
+// then x_mid + W2 hidden, since the down-projection accumulates on top of
+// x_mid) and two 128-column buffers U0/U1 for hidden chunks.  Shared memory
+// holds the attention tile (reused for h2 as the A operand of the
+// up-projection), two 128-wide hidden chunks (A operand of the
+// down-projection) and a 3-stage ring of weight tiles fed by TMA.
+//
+// Per hidden chunk c (128 units): up(c) -> U[c%2]; the four compute warps
+// apply b1 + GELU and write the chunk to shared memory; down(c) accumulates
+// into D.  up(c+2) is issued right after down(c), so GELU of one chunk
+// overlaps the MMAs of the next.
+//
+// Warp roles (192 threads): warps 0-3 compute (one row per thread), warp 4
+// TMA producer, warp 5 TMEM allocator and MMA issuer.
+#pragma once
+#include "tc_ptx.cuh"
+
+namespace ot {
+
+struct FfnDesc {
+  int mode, M, m_lo, G, g_lo, fold, grp_base;  // row enumeration, as in GemmDesc
+  const void* A;                                // attention rows, bf16 [.., 256]
+  long long a_sm, a_sg, a_mext, a_gext;
+  const void* Wo;                               // [256, 256]
+  const void* W1; long long w1_sg;              // [G][dff, 256]
+  const void* b1; long long b1_sg;              // [G][dff]
+  const void* W2; long long w2_sg;              // [G][256, dff]
+  const void* b2; long long b2_sg;              // [G][256]
+  const void* g_ffn;                            // [256]
+  const void* g_next;                           // [256] or null
+  RowMap res, out, hout;                        // hout.base null = no next-layer norm
+  int dff, w_groups;
+  float eps;
+};
+
+struct FfnCfg {
+  static constexpr int D = 256, BM = 128, HC = 128;  // hidden chunk width
+  static constexpr int A_BYTES = BM * D * 2;         // 64 KB: attention tile, then h2
+  static constexpr int H_BYTES = BM * HC * 2;        // 32 KB per hidden chunk buffer
+  static constexpr int STAGE = 32768;                // one weight stage
+  static constexpr int STAGES = 3;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = A_BYTES + 2 * H_BYTES + STAGES * STAGE + BAR_BYTES;
+  static constexpr int TMEM_COLS = 512;              // D 0..255, U0 256..383, U1 384..511
+};
+
+__device__ inline void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ inline void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 bf16 values of row r into a K-major, 128-byte-swizzled operand tile:
+// columns [col0, col0 + 32) of a tile whose 64-column blocks are blk_bytes apart.
+__device__ inline void st_sw128_32(uint8_t* tile, int blk_bytes, int r, int col0, const float* v) {
+  uint8_t* rowp = tile + (col0 >> 6) * blk_bytes + r * 128;
+  const int ch0 = (col0 & 63) >> 3;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint4 u;
+    __nv_bfloat162* hh = (__nv_bfloat162*)&u;
+#pragma unroll
+    for (int q2 = 0; q2 < 4; ++q2) hh[q2] = __floats2bfloat162_rn(v[q4 * 8 + 2 * q2], v[q4 * 8 + 2 * q2 + 1]);
+    *(uint4*)(rowp + (((ch0 + q4) ^ (r & 7)) << 4)) = u;
+  }
+}
+
+__global__ void __launch_bounds__(192, 1)
+    ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmWo,
+                  const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
+                  const FfnDesc d, const int a_swap) {
+  using C = FfnCfg;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sA = smem;
+  uint8_t* sH = sA + C::A_BYTES;                 // [2][128 rows x 128]
+  uint8_t* sW = sH + 2 * C::H_BYTES;             // [3][32 KB]
+  uint64_t* bars = (uint64_t*)(sW + C::STAGES * C::STAGE);
+  uint64_t* a_full = bars;
+  uint64_t* w_full = bars + 1;    // [3]
+  uint64_t* w_empty = bars + 4;   // [3]
+  uint64_t* d_full = bars + 7;
+  uint64_t* h2_ready = bars + 8;
+  uint64_t* u_full = bars + 9;    // [2]
+  uint64_t* hid_full = bars + 11; // [2]
+  uint64_t* hid_free = bars + 13; // [2]
+  uint64_t* d_done = bars + 15;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 16);
+
+  if (smem_u32(smem) & 1023) {
+    if (threadIdx.x == 0) flag_error(kErrSmemAlign);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt0 = d.m_lo + blockIdx.x * C::BM;
+  const int g = d.g_lo + blockIdx.y;
+  const int grp = d.mode == TILE_SAMPLES ? g - d.grp_base : 0;
+  const int NC = d.dff / C::HC;
+
+  if (threadIdx.x == 0) {
+    mbar_init(a_full, 1);
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&w_full[s], 1); mbar_init(&w_empty[s], 1); }
+    mbar_init(d_full, 1);
+    mbar_init(h2_ready, 128);
+    for (int i = 0; i < 2; ++i) { mbar_init(&u_full[i], 1); mbar_init(&hid_full[i], 128); mbar_init(&hid_free[i], 1); }
+    mbar_init(d_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmA); prefetch_tmap(&tmWo); prefetch_tmap(&tmW1); prefetch_tmap(&tmW2);
+  }
+  if (warp == 5) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tD = tmem, tU0 = tmem + 256;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_expect_tx(a_full, C::A_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb) {
+        if (a_swap) tma_load_3d(&tmA, a_full, sA + kb * 16384, kb * 64, g, mt0);
+        else tma_load_3d(&tmA, a_full, sA + kb * 16384, kb * 64, mt0, g);
+      }
+      int q = 0;  // weight stage counter, in the order the MMA thread consumes them
+      auto stage = [&](int kind, int c, int j) -> bool {
+        const int s = q % C::STAGES;
+        if (q >= C::STAGES && !mbar_wait(&w_empty[s], ((q / C::STAGES) - 1) & 1)) return false;
+        uint8_t* dst = sW + s * C::STAGE;
+        mbar_expect_tx(&w_full[s], C::STAGE);
+        if (kind == 0) {          // W^O k-block j: [256 out x 64]
+          tma_load_3d(&tmWo, &w_full[s], dst, j * 64, 0, 0);
+        } else if (kind == 1) {   // W1 chunk c, k-blocks 2j, 2j+1: [128 hidden x 64] each
+          tma_load_3d(&tmW1, &w_full[s], dst, (2 * j) * 64, c * C::HC, grp);
+          tma_load_3d(&tmW1, &w_full[s], dst + 16384, (2 * j + 1) * 64, c * C::HC, grp);
+        } else {                  // W2 chunk c, k-block j: [256 out x 64 hidden]
+          tma_load_3d(&tmW2, &w_full[s], dst, c * C::HC + j * 64, 0, grp);
+        }
+        ++q;
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; j < 4 && ok; ++j) ok = stage(0, 0, j);
+      for (int c = 0; c < 2 && c < NC && ok; ++c)
+        for (int j = 0; j < 2 && ok; ++j) ok = stage(1, c, j);
+      for (int c = 0; c < NC && ok; ++c) {
+        for (int j = 0; j < 2 && ok; ++j) ok = stage(2, c, j);
+        if (c + 2 < NC)
+          for (int j = 0; j < 2 && ok; ++j) ok = stage(1, c + 2, j);
+      }
+    }
+  } else if (warp == 5) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t id256 = idesc_bf16(128, 256);
+      constexpr uint32_t id128 = idesc_bf16(128, 128);
+      const uint32_t aA = smem_u32(sA), aH = smem_u32(sH), aW = smem_u32(sW);
+      int q = 0;
+      bool ok = mbar_wait(a_full, 0);
+      auto wait_stage = [&](uint32_t& base) -> bool {
+        const int s = q % C::STAGES;
+        if (!mbar_wait(&w_full[s], (q / C::STAGES) & 1)) return false;
+        tc_fence_after();
+        base = aW + s * C::STAGE;
+        return true;
+      };
+      auto free_stage = [&]() { umma_commit(&w_empty[q % C::STAGES]); ++q; };
+      auto up = [&](int c) -> bool {
+        const uint32_t tU = tU0 + (c & 1) * C::HC;
+        for (int j = 0; j < 2; ++j) {
+          uint32_t wb;
+          if (!wait_stage(wb)) return false;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int kb = 2 * j + h;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16(tU, sdesc_k128(aA + kb * 16384 + k * 32), sdesc_k128(wb + h * 16384 + k * 32), id128,
+                        (kb | k) ? 1u : 0u);
+          }
+          free_stage();
+        }
+        umma_commit(&u_full[c & 1]);
+        return true;
+      };
+      // x_mid pre-image: D = a W^O^T
+      for (int j = 0; j < 4 && ok; ++j) {
+        uint32_t wb;
+        ok = wait_stage(wb);
+        if (!ok) break;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(tD, sdesc_k128(aA + j * 16384 + k * 32), sdesc_k128(wb + k * 32), id256, (j | k) ? 1u : 0u);
+        free_stage();
+      }
+      if (ok) umma_commit(d_full);
+      ok = ok && mbar_wait(h2_ready, 0);
+      if (ok) tc_fence_after();
+      for (int c = 0; c < 2 && c < NC && ok; ++c) ok = up(c);
+      for (int c = 0; c < NC && ok; ++c) {
+        ok = mbar_wait(&hid_full[c & 1], (c >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t hb = aH + (c & 1) * C::H_BYTES;
+        for (int j = 0; j < 2 && ok; ++j) {
+          uint32_t wb;
+          ok = wait_stage(wb);
+          if (!ok) break;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(tD, sdesc_k128(hb + j * 16384 + k * 32), sdesc_k128(wb + k * 32), id256, 1u);
+          free_stage();
+        }
+        umma_commit(&hid_free[c & 1]);
+        if (ok && c + 2 < NC) ok = up(c + 2);
+      }
+      umma_commit(d_done);
+    }
+  } else {
+    // ------------------------------------------------------------- compute
+    const int r = warp * 32 + lane;
+    const int m = mt0 + r;
+    const bool valid = m < d.m_lo + d.M;
+    int b = 0, t = 0;
+    if (valid) row_of_rows(d.mode, d.fold, m, g, b, t);
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const __nv_bfloat16* gffn = (const __nv_bfloat16*)d.g_ffn;
+    bool ok = mbar_wait(d_full, 0);
+    tc_fence_after();
+    // x_mid = W^O a + x, written back into D; its RMSNorm becomes h2 in sA
+    float ss = 0.f;
+    for (int c0 = 0; c0 < C::D; c0 += 32) {
+      float v[32];
+      tmem_ld32(tD + lb + c0, v);
+      if (valid) {
+        float rv[32];
+        load_row32(d.res, rm_off(d.res, b, t, c0), rv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] += rv[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ss += v[i] * v[i];
+      tmem_st32(tD + lb + c0, v);
+    }
+    tmem_st_wait();
+    const float rr = rsqrtf(ss / C::D + d.eps);
+    for (int c0 = 0; c0 < C::D; c0 += 32) {
+      float v[32], gv[32];
+      tmem_ld32(tD + lb + c0, v);
+      load_bf16x32(gffn + c0, gv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = v[i] * rr * gv[i];
+      st_sw128_32(sA, 16384, r, c0, v);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    mbar_arrive(h2_ready);
+    // hidden chunks: b1 + GELU into shared memory for the down-projection
+    const __nv_bfloat16* b1 = (const __nv_bfloat16*)d.b1 + (long long)grp * d.b1_sg;
+    for (int c = 0; c < NC && ok; ++c) {
+      ok = mbar_wait(&u_full[c & 1], (c >> 1) & 1);
+      if (ok && c >= 2) ok = mbar_wait(&hid_free[c & 1], ((c >> 1) - 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tU = tU0 + (c & 1) * C::HC;
+      uint8_t* hbuf = sH + (c & 1) * C::H_BYTES;
+      for (int c0 = 0; c0 < C::HC; c0 += 32) {
+        float v[32], bv[32];
+        tmem_ld32(tU + lb + c0, v);
+        load_bf16x32(b1 + c * C::HC + c0, bv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i] + bv[i]);
+        st_sw128_32(hbuf, 16384, r, c0, v);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(&hid_full[c & 1]);
+    }
+    // x_next = D + b2, and the next layer's RMSNorm
+    ok = ok && mbar_wait(d_done, 0);
+    tc_fence_after();
+    const __nv_bfloat16* b2 = (const __nv_bfloat16*)d.b2 + (long long)grp * d.b2_sg;
+    ss = 0.f;
+    for (int c0 = 0; c0 < C::D; c0 += 32) {
+      float v[32], bv[32];
+      tmem_ld32(tD + lb + c0, v);
+      load_bf16x32(b2 + c0, bv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) { v[i] += bv[i]; ss += v[i] * v[i]; }
+      if (valid && ok) store_row32(d.out, rm_off(d.out, b, t, c0), v);
+    }
+    if (d.hout.base) {
+      const float r2 = rsqrtf(ss / C::D + d.eps);
+      const __nv_bfloat16* gn = (const __nv_bfloat16*)d.g_next;
+      for (int c0 = 0; c0 < C::D; c0 += 32) {
+        float v[32], bv[32], gv[32];
+        tmem_ld32(tD + lb + c0, v);
+        load_bf16x32(b2 + c0, bv);
+        load_bf16x32(gn + c0, gv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = (v[i] + bv[i]) * r2 * gv[i];
+        if (valid && ok) store_row32(d.hout, rm_off(d.hout, b, t, c0), v);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host --
+inline bool tc_ffn_supported(const FfnDesc& d) {
+  if (d.dff <= 0 || d.dff % FfnCfg::HC) return false;
+  if ((uintptr_t)d.A % 16 || (uintptr_t)d.Wo % 16 || (uintptr_t)d.W1 % 16 || (uintptr_t)d.W2 % 16) return false;
+  if ((uintptr_t)d.b1 % 16 || (uintptr_t)d.b2 % 16 || (uintptr_t)d.g_ffn % 16) return false;
+  if (d.a_sm % 8 || d.a_sg % 8 || d.b1_sg % 8 || d.b2_sg % 8 || d.w1_sg % 8 || d.w2_sg % 8) return false;
+  if (!rowmap_vec_ok(d.res) || !rowmap_vec_ok(d.out) || !d.out.f32) return false;
+  if (d.hout.base && (!rowmap_vec_ok(d.hout) || d.hout.f32 || (uintptr_t)d.g_next % 16)) return false;
+  return encode_fn() != nullptr;
+}
+
+inline onetrans_status tc_ffn_launch(const FfnDesc& d, cudaStream_t st) {
+  using C = FfnCfg;
+  CUtensorMap ta, two, tw1, tw2;
+  const uint64_t mext = (uint64_t)d.a_mext, gext = (uint64_t)d.a_gext;
+  const uint64_t s_m = (uint64_t)d.a_sm, s_g = gext > 1 ? (uint64_t)d.a_sg : mext * (uint64_t)d.a_sm;
+  const int a_swap = (gext > 1 && d.a_sg < d.a_sm) ? 1 : 0;
+  const uint64_t wg = (uint64_t)d.w_groups;
+  bool ok = a_swap ? make_tmap_3d(&ta, d.A, C::D, gext, mext, s_g, s_m, 64, 1, 128)
+                   : make_tmap_3d(&ta, d.A, C::D, mext, gext, s_m, s_g, 64, 128, 1);
+  ok = ok && make_tmap_3d(&two, d.Wo, C::D, C::D, 1, C::D, (uint64_t)C::D * C::D, 64, 256, 1);
+  ok = ok && make_tmap_3d(&tw1, d.W1, C::D, d.dff, wg, C::D, wg > 1 ? (uint64_t)d.w1_sg : (uint64_t)d.dff * C::D,
+                          64, C::HC, 1);
+  ok = ok && make_tmap_3d(&tw2, d.W2, d.dff, C::D, wg, d.dff, wg > 1 ? (uint64_t)d.w2_sg : (uint64_t)d.dff * C::D,
+                          64, 256, 1);
+  if (!ok) return ONETRANS_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+      return ONETRANS_ERR_CUDA;
+    attr_set = true;
+  }
+  dim3 grid((unsigned)((d.M + C::BM - 1) / C::BM), (unsigned)d.G);
+  ffn_tc_kernel<<<grid, 192, C::SMEM, st>>>(ta, two, tw1, tw2, d, a_swap);
+  return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
+}
+
+}  // namespace ot

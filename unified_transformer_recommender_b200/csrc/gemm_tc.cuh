@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (d.act == ACT_GELU) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+        for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i]);
       }
       if (d.res.base) {
         float rv[32];

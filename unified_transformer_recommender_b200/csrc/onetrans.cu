@@ -14,6 +14,7 @@
 #include "simt.cuh"
 #include "gemm_tc.cuh"
 #include "attn_tc.cuh"
+#include "ffn_tc.cuh"
 
 using namespace ot;
 
@@ -47,11 +48,11 @@ static int g_policy = 0;
 // tagged with a kernel kind and its algorithmic FLOPs and bytes.
 enum ProfKind {
   PK_GEMM_QKV = 0, PK_GEMM_OPROJ, PK_GEMM_FFN_UP, PK_GEMM_FFN_DOWN, PK_GEMM_AUTOSPLIT, PK_ATTN_CAUSAL,
-  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_COUNT
+  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_BLOCK_TAIL, PK_COUNT
 };
 static const char* kProfNames[PK_COUNT] = {"gemm_qkv", "gemm_oproj_rms", "gemm_ffn_up_gelu", "gemm_ffn_down_rms",
                                            "gemm_autosplit", "attn_causal", "attn_stage2", "rmsnorm",
-                                           "tokenize_events"};
+                                           "tokenize_events", "fused_oproj_ffn"};
 struct ProfRec {
   int kind;
   cudaEvent_t e0, e1;
@@ -293,6 +294,41 @@ static onetrans_status rms_flat(const onetrans_model* m, const void* src, bool s
   return launch_rms<T>(d, st);
 }
 
+// ------------------------------------------------------------ block tail --
+// W^O + residual + RMSNorm + mixed FFN + residual (+ the next RMSNorm) over
+// the rows that `f` (the FFN-up GEMM) enumerates.  `res` maps those rows to
+// the block's residual input in f's (b, t) convention.
+static FfnDesc ffn_desc(const onetrans_model* m, const GemmDesc& go, const GemmDesc& f, const GemmDesc& f2,
+                        const RowMap& res) {
+  FfnDesc fd;
+  std::memset(&fd, 0, sizeof(fd));
+  fd.mode = f.mode; fd.M = f.M; fd.m_lo = f.m_lo; fd.G = f.G; fd.g_lo = f.g_lo; fd.fold = f.fold;
+  fd.grp_base = f.grp_base;
+  fd.A = go.A;  // the attention output has the layout of h2
+  fd.a_sm = f.a_sm; fd.a_sg = f.a_sg; fd.a_mext = f.a_mext; fd.a_gext = f.a_gext;
+  fd.Wo = go.W;
+  fd.W1 = f.W; fd.w1_sg = f.w_sg; fd.b1 = f.bias; fd.b1_sg = f.bias_sg;
+  fd.W2 = f2.W; fd.w2_sg = f2.w_sg; fd.b2 = f2.bias; fd.b2_sg = f2.bias_sg;
+  fd.g_ffn = go.gamma; fd.g_next = f2.gamma;
+  fd.res = res; fd.out = f2.out; fd.hout = f2.rms;
+  fd.dff = m->dff; fd.w_groups = f.w_groups; fd.eps = m->cfg.rms_eps;
+  return fd;
+}
+
+static bool use_fused_tail(const onetrans_model* m, const FfnDesc& fd) {
+  return m->bf16 && g_policy == 0 && m->d == FfnCfg::D && tc_ffn_supported(fd);
+}
+
+static onetrans_status launch_fused_tail(const onetrans_model* m, const FfnDesc& fd, cudaStream_t st) {
+  if (fd.M <= 0 || fd.G <= 0) return ONETRANS_OK;
+  const double rows = (double)fd.M * fd.G, d = m->d;
+  ProfScope prof(PK_BLOCK_TAIL, 2.0 * rows * (d * d + 2.0 * d * m->dff),
+                 rows * d * (2.0 + (fd.res.f32 ? 4 : 2) + 4 + (fd.hout.base ? 2 : 0)) +
+                     2.0 * (d * d + (fd.mode == TILE_SAMPLES ? fd.G : 1) * 2.0 * d * m->dff),
+                 st);
+  return tc_ffn_launch(fd, st);
+}
+
 // ================================================================ forward =
 template <typename T>
 static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int B, int L_S, void* out,
@@ -369,8 +405,9 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
     go.out = rmap32(xm, (long long)Lqn * d, d);
     go.rms = rmap(h2, (long long)Lqn * d, d);
     go.gamma = m->g_ffn[n];
-    OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     // -- mixed FFN: S tail rows shared, NS rows per token
+    GemmDesc fs[2], f2s[2];
+    bool has[2] = {false, false};
     for (int part = 0; part < 2; ++part) {
       GemmDesc f = gdesc_base(m);
       if (part == 0) {
@@ -387,7 +424,6 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
       f.bias = part ? m->b1_NS[n] : m->b1_S[n]; f.bias_sg = part ? dff : 0;
       f.act = ACT_GELU;
       f.out = rmap(hid, (long long)Lqn * dff, dff);
-      OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
       GemmDesc f2 = f;
       f2.K = dff; f2.A = hid; f2.act = ACT_NONE;
       if (part == 0) { f2.a_sm = dff; f2.a_sg = (long long)Lqn * dff; }
@@ -398,7 +434,22 @@ static onetrans_status forward_impl(const onetrans_model* m, const void* x0, int
       f2.res = rmap32(xm, (long long)Lqn * d, d);
       f2.out = rmap32(x_next, (long long)Lqn * d, d);
       if (!last) { f2.rms = rmap(h, (long long)Lqn * d, d); f2.gamma = m->g_attn[n + 1]; }
-      OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
+      fs[part] = f; f2s[part] = f2; has[part] = true;
+    }
+    bool fused = true;
+    FfnDesc fds[2];
+    for (int part = 0; part < 2; ++part)
+      if (has[part]) { fds[part] = ffn_desc(m, go, fs[part], f2s[part], go.res); fused = fused && use_fused_tail(m, fds[part]); }
+    if (fused) {
+      for (int part = 0; part < 2; ++part)
+        if (has[part]) OT_TRY(launch_fused_tail(m, fds[part], st));
+    } else {
+      OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
+      for (int part = 0; part < 2; ++part) {
+        if (!has[part]) continue;
+        OT_TRY(launch_gemm<T>(m, fs[part], st, PK_GEMM_FFN_UP));
+        OT_TRY(launch_gemm<T>(m, f2s[part], st, PK_GEMM_FFN_DOWN));
+      }
     }
     x_in = x_next;
     L = Lqn;
@@ -512,12 +563,10 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
     go.out = rmap32(xm, (long long)sqn * d, d);
     go.rms = rmap(h2, (long long)sqn * d, d);
     go.gamma = m->g_ffn[n];
-    OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     GemmDesc f = go;
     f.res.base = nullptr; f.rms.base = nullptr; f.gamma = nullptr;
     f.A = h2; f.W = m->W1_S[n]; f.w_rows = dff; f.N = dff; f.bias = m->b1_S[n]; f.act = ACT_GELU;
     f.out = rmap(hid, (long long)sqn * dff, dff);
-    OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
     GemmDesc f2 = go;
     f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.W = m->W2_S[n]; f2.w_rows = d; f2.N = d;
     f2.bias = m->b2_S[n];
@@ -525,7 +574,14 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
     f2.out = rmap32(x_next, (long long)sqn * d, d);
     f2.rms = rmap(h, (long long)sqn * d, d);
     f2.gamma = m->g_attn[n + 1];
-    OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
+    const FfnDesc fd = ffn_desc(m, go, f, f2, go.res);
+    if (use_fused_tail(m, fd)) {
+      OT_TRY(launch_fused_tail(m, fd, st));
+    } else {
+      OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
+      OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
+      OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
+    }
     x_in = x_next;
   }
   return ONETRANS_OK;
@@ -606,13 +662,11 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     go.out = rmap32(xm, 0, d);
     go.rms = rmap(h2, 0, d);
     go.gamma = m->g_ffn[n];
-    OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     GemmDesc f = g;
     f.scale_cols = 0;
     f.A = h2; f.W = m->W1_NS[n]; f.w_sg = (long long)dff * d; f.w_rows = dff; f.N = dff;
     f.bias = m->b1_NS[n]; f.bias_sg = dff; f.act = ACT_GELU;
     f.out = rmap(hid, (long long)L_NS * dff, dff);
-    OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
     GemmDesc f2 = f;
     f2.K = dff; f2.A = hid; f2.a_sm = (long long)L_NS * dff; f2.a_sg = dff; f2.act = ACT_NONE;
     f2.W = m->W2_NS[n]; f2.w_sg = (long long)d * dff; f2.w_rows = d; f2.N = d;
@@ -620,7 +674,15 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     f2.res = rmap32(xm, Ld, d);
     f2.out = rmap32(x_next, Ld, d);
     if (!last) { f2.rms = rmap(h, Ld, d); f2.gamma = m->g_attn[n + 1]; }
-    OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
+    const RowMap res_bt = n == 0 ? rmap(x_in, Ld, d) : rmap32(x_in, Ld, d);  // (b = candidate, t = token)
+    const FfnDesc fd = ffn_desc(m, go, f, f2, res_bt);
+    if (use_fused_tail(m, fd)) {
+      OT_TRY(launch_fused_tail(m, fd, st));
+    } else {
+      OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
+      OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
+      OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
+    }
     x_in = x_next;
   }
   return ONETRANS_OK;
@@ -713,12 +775,10 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     go.out = rmap32(xm, (long long)dL * d, d);
     go.rms = rmap(h2, (long long)dL * d, d);
     go.gamma = m->g_ffn[n];
-    OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
     GemmDesc f = go;
     f.res.base = nullptr; f.rms.base = nullptr; f.gamma = nullptr;
     f.A = h2; f.W = m->W1_S[n]; f.w_rows = dff; f.N = dff; f.bias = m->b1_S[n]; f.act = ACT_GELU;
     f.out = rmap(hid, (long long)dL * dff, dff);
-    OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
     GemmDesc f2 = go;
     f2.K = dff; f2.A = hid; f2.a_sm = dff; f2.W = m->W2_S[n]; f2.w_rows = d; f2.N = d;
     f2.bias = m->b2_S[n];
@@ -726,7 +786,14 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     f2.out = rmap32(x_next, (long long)dL * d, d);
     f2.rms = rmap(h, (long long)dL * d, d);
     f2.gamma = m->g_attn[n + 1];
-    OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
+    const FfnDesc fd = ffn_desc(m, go, f, f2, go.res);
+    if (use_fused_tail(m, fd)) {
+      OT_TRY(launch_fused_tail(m, fd, st));
+    } else {
+      OT_TRY(launch_gemm<T>(m, go, st, PK_GEMM_OPROJ));
+      OT_TRY(launch_gemm<T>(m, f, st, PK_GEMM_FFN_UP));
+      OT_TRY(launch_gemm<T>(m, f2, st, PK_GEMM_FFN_DOWN));
+    }
     x_in = x_next;
   }
   return ONETRANS_OK;

@@ -9,7 +9,7 @@
 namespace ot {
 
 constexpr uint32_t kSpinLimit = 1u << 24;  // try_wait rounds before a wait gives up
-enum : int { kErrWaitTimeout = 101 };
+enum : int { kErrWaitTimeout = 101, kErrSmemAlign = 102 };
 
 __device__ inline uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -146,6 +146,18 @@ __device__ inline void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// GELU, tanh form, with the hardware tanh approximation (relative error about
+// 2^-11, below the bf16 rounding of the values it produces).
+__device__ inline float tanh_fast(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ inline float gelu_fast(float x) {
+  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
+  return 0.5f * x * (1.0f + tanh_fast(k0 * (x + k1 * x * x * x)));
 }
 
 // -------------------------------------------------------- bf16 vectors --
