@@ -55,7 +55,8 @@ struct AttnCfg {
   static constexpr int STAGES = 2;
   static constexpr int P_BYTES = BM * BN * 2;     // 32 KB
   static constexpr int BAR_BYTES = 128;
-  static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + BAR_BYTES;
+  static constexpr int MAX_PAGES = 128;           // page ids cached in shared memory (8192 keys)
+  static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + BAR_BYTES + MAX_PAGES * 4;
   static constexpr int TMEM_COLS = 256;           // S: cols 0..127, O tile: 128..191
 };
 
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* p_full = bars + 6;
   uint64_t* o_full = bars + 7;
   uint32_t* tmem_slot = (uint32_t*)(bars + 8);
+  int* s_pages = (int*)((uint8_t*)bars + C::BAR_BYTES);
 
   // the swizzled tiles need 1024-byte alignment; refuse to run without it
   if (smem_u32(smem) & 1023) {
@@ -126,10 +128,17 @@ __global__ void __launch_bounds__(192, 2)
     mbar_init(o_full, 1);
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
-    prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmKV);
-    if (a.mode == MODE_STAGE2) prefetch_tmap(&tmNS);
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmKV);
+      if (a.mode == MODE_STAGE2) prefetch_tmap(&tmNS);
+    }
+    // page ids of every key page this CTA reads, fetched once (page ids past
+    // the cached range read as the out-of-range page, which loads zeros)
+    const int n_pg = min(2 * nt_s, C::MAX_PAGES);
+    for (int i = lane; i < n_pg; i += 32) s_pages[i] = i < n_pages_used ? kv_page_id(a.kv, b, i) : a.kv.n_pages;
+    __syncwarp();
   }
   if (warp == 5) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
@@ -154,8 +163,8 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
           for (int hp = 0; hp < 2; ++hp) {
             const int pi = kt * 2 + hp;
-            // pages past the last used one read as zeros (out-of-range page coordinate)
-            const int pg = pi < n_pages_used ? kv_page_id(a.kv, b, pi) : a.kv.n_pages;
+            const int pg = pi < C::MAX_PAGES ? s_pages[pi]
+                                             : (pi < n_pages_used ? kv_page_id(a.kv, b, pi) : a.kv.n_pages);
             tma_load_4d(&tmKV, &kv_full[s], sk + hp * C::PAGE_BYTES, 0, 0, h, pg);
             tma_load_4d(&tmKV, &kv_full[s], sv + hp * C::PAGE_BYTES, 0, 0, a.H + h, pg);
           }

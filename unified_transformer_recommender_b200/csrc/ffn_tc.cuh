@@ -14,6 +14,11 @@
 // up-projection), two 128-wide hidden chunks (A operand of the
 // down-projection) and a 3-stage ring of weight tiles fed by TMA.
 //
+// The residual rows arrive by TMA (staged through the hidden-chunk buffers)
+// and are written into D before W^O a accumulates on top of them; x_next and
+// h_next leave by TMA stores staged through the then idle shared memory.
+// Row geometries TMA cannot express fall back to per-thread loads/stores.
+//
 // Per hidden chunk c (128 units): up(c) -> U[c%2]; the four compute warps
 // apply b1 + GELU and write the chunk to shared memory; down(c) accumulates
 // into D.  up(c+2) is issued right after down(c), so GELU of one chunk
@@ -40,6 +45,14 @@ struct FfnDesc {
   RowMap res, out, hout;                        // hout.base null = no next-layer norm
   int dff, w_groups;
   float eps;
+};
+
+// Which row tensors move by TMA (else per-thread accesses), and whether their
+// maps list the fixed coordinate before the tiled one.
+struct FfnIo {
+  int res_tma, res_swap, res_f32;
+  int out_tma, out_swap;
+  int hout_tma, hout_swap;
 };
 
 struct FfnCfg {
@@ -73,6 +86,42 @@ __device__ inline void tmem_st32(uint32_t taddr, const float* v) {
 }
 __device__ inline void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 32 fp32 values of row r into box `box` of a staging area of [128 rows x
+// 128 B] boxes with the 128-byte swizzle (the layout TMA reads and writes).
+__device__ inline void st_sw128_f32(uint8_t* tile, int box, int r, const float* v) {
+  uint8_t* rowp = tile + box * 16384 + r * 128;
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    *(float4*)(rowp + ((k ^ (r & 7)) << 4)) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+}
+// 128 bytes of row r of a staged box, as 32 fp32 or 64 bf16 (to fp32) values.
+__device__ inline void ld_sw128_f32(const uint8_t* tile, int box, int r, float* v) {
+  const uint8_t* rowp = tile + box * 16384 + r * 128;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float4 f = *(const float4*)(rowp + ((k ^ (r & 7)) << 4));
+    v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
+  }
+}
+__device__ inline void ld_sw128_bf16(const uint8_t* tile, int box, int r, float* v) {
+  const uint8_t* rowp = tile + box * 16384 + r * 128;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint4 u = *(const uint4*)(rowp + ((k ^ (r & 7)) << 4));
+    const __nv_bfloat162* h = (const __nv_bfloat162*)&u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      v[8 * k + 2 * j] = f.x; v[8 * k + 2 * j + 1] = f.y;
+    }
+  }
+}
+__device__ inline void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
 // 32 bf16 values of row r into a K-major, 128-byte-swizzled operand tile:
 // columns [col0, col0 + 32) of a tile whose 64-column blocks are blk_bytes apart.
 __device__ inline void st_sw128_32(uint8_t* tile, int blk_bytes, int r, int col0, const float* v) {
@@ -91,7 +140,8 @@ __device__ inline void st_sw128_32(uint8_t* tile, int blk_bytes, int r, int col0
 __global__ void __launch_bounds__(192, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmWo,
                   const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
-                  const FfnDesc d, const int a_swap) {
+                  const __grid_constant__ CUtensorMap tmRes, const __grid_constant__ CUtensorMap tmOut,
+                  const __grid_constant__ CUtensorMap tmHout, const FfnDesc d, const int a_swap, const FfnIo io) {
   using C = FfnCfg;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sA = smem;
@@ -107,7 +157,10 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* hid_full = bars + 11; // [2]
   uint64_t* hid_free = bars + 13; // [2]
   uint64_t* d_done = bars + 15;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 16);
+  uint64_t* res_full = bars + 16;  // [2]
+  uint64_t* sh_free = bars + 18;
+  uint64_t* res_ready = bars + 19;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 20);
 
   if (smem_u32(smem) & 1023) {
     if (threadIdx.x == 0) flag_error(kErrSmemAlign);
@@ -126,6 +179,9 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(h2_ready, 128);
     for (int i = 0; i < 2; ++i) { mbar_init(&u_full[i], 1); mbar_init(&hid_full[i], 128); mbar_init(&hid_free[i], 1); }
     mbar_init(d_done, 1);
+    mbar_init(&res_full[0], 1); mbar_init(&res_full[1], 1);
+    mbar_init(sh_free, 128);
+    mbar_init(res_ready, 128);
     fence_barrier_init();
   }
   if (warp == 4 && lane == 0) {
@@ -137,6 +193,18 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tD = tmem, tU0 = tmem + 256;
+  // residual boxes: fp32 = 8 boxes of 32 columns in two rounds, bf16 = 4 of 64 in one
+  const int res_rounds = io.res_f32 ? 2 : 1;
+  auto res_round = [&](int k) {
+    mbar_expect_tx(&res_full[k], 4 * 16384);
+    const int bc = io.res_f32 ? 32 : 64;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int col = (k * 4 + i) * bc;
+      if (io.res_swap) tma_load_3d(&tmRes, &res_full[k], sH + i * 16384, col, g, mt0);
+      else tma_load_3d(&tmRes, &res_full[k], sH + i * 16384, col, mt0, g);
+    }
+  };
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -146,6 +214,10 @@ __global__ void __launch_bounds__(192, 1)
       for (int kb = 0; kb < 4; ++kb) {
         if (a_swap) tma_load_3d(&tmA, a_full, sA + kb * 16384, kb * 64, g, mt0);
         else tma_load_3d(&tmA, a_full, sA + kb * 16384, kb * 64, mt0, g);
+      }
+      if (io.res_tma) {
+        prefetch_tmap(&tmRes);
+        res_round(0);
       }
       int q = 0;  // weight stage counter, in the order the MMA thread consumes them
       auto stage = [&](int kind, int c, int j) -> bool {
@@ -165,7 +237,14 @@ __global__ void __launch_bounds__(192, 1)
         return true;
       };
       bool ok = true;
-      for (int j = 0; j < 4 && ok; ++j) ok = stage(0, 0, j);
+      for (int j = 0; j < 3 && ok; ++j) ok = stage(0, 0, j);
+      // the second residual round reuses the staging buffer once it is copied out;
+      // issue it before any weight stage that waits on the MMAs
+      if (io.res_tma && res_rounds == 2 && ok) {
+        ok = mbar_wait(sh_free, 0);
+        if (ok) res_round(1);
+      }
+      if (ok) ok = stage(0, 0, 3);
       for (int c = 0; c < 2 && c < NC && ok; ++c)
         for (int j = 0; j < 2 && ok; ++j) ok = stage(1, c, j);
       for (int c = 0; c < NC && ok; ++c) {
@@ -181,7 +260,7 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t id128 = idesc_bf16(128, 128);
       const uint32_t aA = smem_u32(sA), aH = smem_u32(sH), aW = smem_u32(sW);
       int q = 0;
-      bool ok = mbar_wait(a_full, 0);
+      bool ok = mbar_wait(a_full, 0) && mbar_wait(res_ready, 0);
       auto wait_stage = [&](uint32_t& base) -> bool {
         const int s = q % C::STAGES;
         if (!mbar_wait(&w_full[s], (q / C::STAGES) & 1)) return false;
@@ -208,14 +287,14 @@ __global__ void __launch_bounds__(192, 1)
         umma_commit(&u_full[c & 1]);
         return true;
       };
-      // x_mid pre-image: D = a W^O^T
+      // D holds the residual rows: x_mid = x + a W^O^T accumulates in place
       for (int j = 0; j < 4 && ok; ++j) {
         uint32_t wb;
         ok = wait_stage(wb);
         if (!ok) break;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma_bf16(tD, sdesc_k128(aA + j * 16384 + k * 32), sdesc_k128(wb + k * 32), id256, (j | k) ? 1u : 0u);
+          umma_bf16(tD, sdesc_k128(aA + j * 16384 + k * 32), sdesc_k128(wb + k * 32), id256, 1u);
         free_stage();
       }
       if (ok) umma_commit(d_full);
@@ -250,24 +329,50 @@ __global__ void __launch_bounds__(192, 1)
     if (valid) row_of_rows(d.mode, d.fold, m, g, b, t);
     const uint32_t lb = (uint32_t)(warp * 32) << 16;
     const __nv_bfloat16* gffn = (const __nv_bfloat16*)d.g_ffn;
-    bool ok = mbar_wait(d_full, 0);
+    bool ok = true;
+    // residual rows into D (the W^O product accumulates on top)
+    if (io.res_tma) {
+      for (int k = 0; k < res_rounds && ok; ++k) {
+        ok = mbar_wait(&res_full[k], 0);
+        if (!ok) break;
+#pragma unroll 1
+        for (int i = 0; i < 4; ++i) {
+          float v[64];
+          if (io.res_f32) {
+            ld_sw128_f32(sH, i, r, v);
+            tmem_st32(tD + lb + (k * 4 + i) * 32, v);
+          } else {
+            ld_sw128_bf16(sH, i, r, v);
+            tmem_st32(tD + lb + i * 64, v);
+            tmem_st32(tD + lb + i * 64 + 32, v + 32);
+          }
+        }
+        if (k == 0 && res_rounds == 2) mbar_arrive(sh_free);
+      }
+    } else {
+      float nxt[32];
+      if (valid) load_row32(d.res, rm_off(d.res, b, t, 0), nxt);
+      for (int c0 = 0; c0 < C::D; c0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = valid ? nxt[i] : 0.f;
+        if (valid && c0 + 32 < C::D) load_row32(d.res, rm_off(d.res, b, t, c0 + 32), nxt);
+        tmem_st32(tD + lb + c0, v);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(res_ready);
+    ok = ok && mbar_wait(d_full, 0);
     tc_fence_after();
-    // x_mid = W^O a + x, written back into D; its RMSNorm becomes h2 in sA
+    // D = x_mid; its RMSNorm becomes h2 in sA
     float ss = 0.f;
     for (int c0 = 0; c0 < C::D; c0 += 32) {
       float v[32];
       tmem_ld32(tD + lb + c0, v);
-      if (valid) {
-        float rv[32];
-        load_row32(d.res, rm_off(d.res, b, t, c0), rv);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] += rv[i];
-      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) ss += v[i] * v[i];
-      tmem_st32(tD + lb + c0, v);
     }
-    tmem_st_wait();
     const float rr = rsqrtf(ss / C::D + d.eps);
     for (int c0 = 0; c0 < C::D; c0 += 32) {
       float v[32], gv[32];
@@ -301,7 +406,8 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&hid_full[c & 1]);
     }
-    // x_next = D + b2, and the next layer's RMSNorm
+    // x_next = D + b2, and the next layer's RMSNorm; every MMA is done, so the
+    // whole of shared memory can stage the outputs for TMA stores
     ok = ok && mbar_wait(d_done, 0);
     tc_fence_after();
     const __nv_bfloat16* b2 = (const __nv_bfloat16*)d.b2 + (long long)grp * d.b2_sg;
@@ -312,7 +418,8 @@ __global__ void __launch_bounds__(192, 1)
       load_bf16x32(b2 + c0, bv);
 #pragma unroll
       for (int i = 0; i < 32; ++i) { v[i] += bv[i]; ss += v[i] * v[i]; }
-      if (valid && ok) store_row32(d.out, rm_off(d.out, b, t, c0), v);
+      if (io.out_tma) st_sw128_f32(sA, c0 >> 5, r, v);          // sA + sH: 8 boxes of 32 fp32
+      else if (valid && ok) store_row32(d.out, rm_off(d.out, b, t, c0), v);
     }
     if (d.hout.base) {
       const float r2 = rsqrtf(ss / C::D + d.eps);
@@ -324,7 +431,28 @@ __global__ void __launch_bounds__(192, 1)
         load_bf16x32(gn + c0, gv);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = (v[i] + bv[i]) * r2 * gv[i];
-        if (valid && ok) store_row32(d.hout, rm_off(d.hout, b, t, c0), v);
+        if (io.hout_tma) st_sw128_32(sW, 16384, r, c0, v);          // ring: 4 boxes of 64 bf16
+        else if (valid && ok) store_row32(d.hout, rm_off(d.hout, b, t, c0), v);
+      }
+    }
+    if (io.out_tma || io.hout_tma) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (r == 0 && ok) {
+        if (io.out_tma) {
+          for (int i = 0; i < 8; ++i) {
+            if (io.out_swap) tma_store_3d(&tmOut, sA + i * 16384, i * 32, g, mt0);
+            else tma_store_3d(&tmOut, sA + i * 16384, i * 32, mt0, g);
+          }
+        }
+        if (io.hout_tma && d.hout.base) {
+          for (int i = 0; i < 4; ++i) {
+            if (io.hout_swap) tma_store_3d(&tmHout, sW + i * 16384, i * 64, g, mt0);
+            else tma_store_3d(&tmHout, sW + i * 16384, i * 64, mt0, g);
+          }
+        }
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       }
     }
   }
@@ -344,9 +472,36 @@ inline bool tc_ffn_supported(const FfnDesc& d) {
   return encode_fn() != nullptr;
 }
 
+// TMA map over the rows a FfnDesc enumerates for row map r (element size es,
+// box of bc columns x 128 rows).  False when the rows are not a strided 2-D
+// set (a flattened enumeration whose batches are not back to back).
+inline bool make_rows_tmap(CUtensorMap* map, const FfnDesc& d, const RowMap& r, bool f32, int bc, int& swap) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !r.base || ((uintptr_t)r.base % 16) || r.split < FfnCfg::D) return false;
+  const uint64_t es = f32 ? 4 : 2;
+  const uint64_t m_ext = (uint64_t)(d.m_lo + d.M), g_ext = (uint64_t)(d.g_lo + d.G);
+  uint64_t s_m, s_g;
+  if (d.mode == TILE_ROWS) { s_m = r.st; s_g = r.sb; }
+  else if (d.mode == TILE_SAMPLES) { s_m = r.sb; s_g = r.st; }
+  else {
+    if (d.fold < d.m_lo + d.M && (long long)r.sb != (long long)d.fold * r.st) return false;
+    s_m = r.st; s_g = m_ext * r.st;
+  }
+  if (g_ext == 1) s_g = m_ext * s_m;
+  swap = (g_ext > 1 && s_g < s_m) ? 1 : 0;
+  const cuuint64_t dims[3] = {(cuuint64_t)FfnCfg::D, swap ? g_ext : m_ext, swap ? m_ext : g_ext};
+  const cuuint64_t strides[2] = {(swap ? s_g : s_m) * es, (swap ? s_m : s_g) * es};
+  const cuuint32_t box[3] = {(cuuint32_t)bc, swap ? 1u : 128u, swap ? 128u : 1u};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  if (strides[0] % 16 || strides[1] % 16) return false;
+  return fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, r.base, dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline onetrans_status tc_ffn_launch(const FfnDesc& d, cudaStream_t st) {
   using C = FfnCfg;
-  CUtensorMap ta, two, tw1, tw2;
+  CUtensorMap ta, two, tw1, tw2, tres, tout, thout;
   const uint64_t mext = (uint64_t)d.a_mext, gext = (uint64_t)d.a_gext;
   const uint64_t s_m = (uint64_t)d.a_sm, s_g = gext > 1 ? (uint64_t)d.a_sg : mext * (uint64_t)d.a_sm;
   const int a_swap = (gext > 1 && d.a_sg < d.a_sm) ? 1 : 0;
@@ -359,6 +514,15 @@ inline onetrans_status tc_ffn_launch(const FfnDesc& d, cudaStream_t st) {
   ok = ok && make_tmap_3d(&tw2, d.W2, d.dff, C::D, wg, d.dff, wg > 1 ? (uint64_t)d.w2_sg : (uint64_t)d.dff * C::D,
                           64, 256, 1);
   if (!ok) return ONETRANS_ERR_CUDA;
+  FfnIo io;
+  memset(&io, 0, sizeof(io));
+  io.res_f32 = d.res.f32;
+  io.res_tma = make_rows_tmap(&tres, d, d.res, d.res.f32, d.res.f32 ? 32 : 64, io.res_swap);
+  io.out_tma = make_rows_tmap(&tout, d, d.out, true, 32, io.out_swap);
+  io.hout_tma = d.hout.base ? make_rows_tmap(&thout, d, d.hout, false, 64, io.hout_swap) : 0;
+  if (!io.res_tma) tres = ta;
+  if (!io.out_tma) tout = ta;
+  if (!io.hout_tma) thout = ta;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
@@ -366,7 +530,7 @@ inline onetrans_status tc_ffn_launch(const FfnDesc& d, cudaStream_t st) {
     attr_set = true;
   }
   dim3 grid((unsigned)((d.M + C::BM - 1) / C::BM), (unsigned)d.G);
-  ffn_tc_kernel<<<grid, 192, C::SMEM, st>>>(ta, two, tw1, tw2, d, a_swap);
+  ffn_tc_kernel<<<grid, 192, C::SMEM, st>>>(ta, two, tw1, tw2, tres, tout, thout, d, a_swap, io);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 

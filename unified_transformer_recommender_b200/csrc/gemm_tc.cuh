@@ -23,7 +23,8 @@ struct TcGemmCfg {
   static constexpr int UN = BN <= 256 ? BN : BN / 2;  // N of one tcgen05.mma
   static constexpr int NSUB = BN / UN;
   static constexpr int BOX_N = BN <= 256 ? BN : BN / 2;  // TMA box rows of W (<= 256)
-  static constexpr int STAGES = BN <= 256 ? 4 : 3;
+  // two CTAs per SM for BN <= 256 (one's epilogue overlaps the other's loads and MMAs)
+  static constexpr int STAGES = BN <= 256 ? 2 : 3;
   static constexpr int A_BYTES = 128 * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -32,7 +33,7 @@ struct TcGemmCfg {
 };
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmDesc d, const int a_swap) {
   using C = TcGemmCfg<BN>;
