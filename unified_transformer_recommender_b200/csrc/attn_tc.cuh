@@ -5,14 +5,14 @@
 //   S = Q K^T          tcgen05.mma into TMEM (fp32)
 //   softmax            four warps read their query row back with tcgen05.ld
 //                      (one row per thread, so the row max and sum stay in the
-//                      thread), mask, update the running max and sum (online
-//                      softmax in base 2: queries arrive pre-scaled by
-//                      1/sqrt(d_h)*log2(e)), write P = 2^(S - m) as bf16 into
-//                      shared memory
-//   O_tile = P V       tcgen05.mma, V read as an MN-major operand
-//   fold               the softmax warps add O_tile into their registers
-// MMA of tile t+1 overlaps the fold of tile t; two CTAs share an SM so one's
-// softmax overlaps the other's MMAs.
+//                      thread), mask, and write P = 2^(S - m) as bf16 pairs
+//                      into TMEM (online softmax in base 2: queries arrive
+//                      pre-scaled by 1/sqrt(d_h)*log2(e))
+//   O += P V           tcgen05.mma with P read from TMEM and V from shared
+//                      memory (MN-major); O stays in TMEM for the whole row
+// The running max m is raised only when a tile's max passes it by more than
+// 2^8; then the thread rescales l and the O row in TMEM.  S of tile t+1 is
+// computed while the softmax of tile t runs; two CTAs share an SM.
 //
 // Query kinds:
 //  * MODE_CAUSAL  (Stage I, forward, append): query t of sequence b sits at
@@ -53,11 +53,10 @@ struct AttnCfg {
   static constexpr int KV_BYTES = BN * DH * 2;    // 16 KB (one of K or V)
   static constexpr int PAGE_BYTES = 64 * DH * 2;  // one 64-token page of one head
   static constexpr int STAGES = 2;
-  static constexpr int P_BYTES = BM * BN * 2;     // 32 KB
   static constexpr int BAR_BYTES = 128;
   static constexpr int MAX_PAGES = 128;           // page ids cached in shared memory (8192 keys)
-  static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + BAR_BYTES + MAX_PAGES * 4;
-  static constexpr int TMEM_COLS = 256;           // S: cols 0..127, O tile: 128..191
+  static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + BAR_BYTES + MAX_PAGES * 4;
+  static constexpr int TMEM_COLS = 256;           // S 0..127, O 128..191, P (bf16 pairs) 192..255
 };
 
 __device__ inline int kv_page_id(const KVStore& kv, int b, int page_idx) {
@@ -76,16 +75,16 @@ __global__ void __launch_bounds__(192, 2)
   using C = AttnCfg;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + C::Q_BYTES;                   // [stage][K|V][128 keys][64]
-  uint8_t* sP = sKV + C::STAGES * 2 * C::KV_BYTES;  // [2 key blocks][128 rows][64]
-  uint64_t* bars = (uint64_t*)(sP + C::P_BYTES);
+  uint8_t* sKV = sQ + C::Q_BYTES;  // [stage][K|V][128 keys][64]
+  uint64_t* bars = (uint64_t*)(sKV + C::STAGES * 2 * C::KV_BYTES);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;   // [2]
   uint64_t* kv_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;
   uint64_t* p_full = bars + 6;
-  uint64_t* o_full = bars + 7;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 8);
+  uint64_t* p_free = bars + 7;
+  uint64_t* o_done = bars + 8;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 9);
   int* s_pages = (int*)((uint8_t*)bars + C::BAR_BYTES);
 
   // the swizzled tiles need 1024-byte alignment; refuse to run without it
@@ -125,7 +124,8 @@ __global__ void __launch_bounds__(192, 2)
     mbar_init(&kv_empty[0], 1); mbar_init(&kv_empty[1], 1);
     mbar_init(s_full, 1);
     mbar_init(p_full, 128);
-    mbar_init(o_full, 1);
+    mbar_init(p_free, 1);
+    mbar_init(o_done, 1);
     fence_barrier_init();
   }
   if (warp == 4) {
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  const uint32_t tS = tmem, tO = tmem + 128, tP = tmem + 192;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(192, 2)
         umma_commit(s_full);
       }
       for (int kt = 0; kt < nt && ok; ++kt) {
+        // P of tile kt is in TMEM and S of tile kt has been read
         ok = mbar_wait(p_full, kt & 1);
         if (!ok) break;
         tc_fence_after();
@@ -206,40 +207,38 @@ __global__ void __launch_bounds__(192, 2)
             umma_bf16(tS, sdesc_k128(aq + k * 32), sdesc_k128(ak + k * 32), id_qk, k ? 1u : 0u);
           umma_commit(s_full);
         }
+        // O += P V: P from TMEM (8 columns = 16 keys per step), V from shared memory
         const int s = kt & 1;
         const uint32_t av = smem_u32(sKV + s * 2 * C::KV_BYTES + C::KV_BYTES);
-        const uint32_t ap = smem_u32(sP);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t pd = sdesc_k128(ap + (kk >> 2) * (128 * 128) + (kk & 3) * 32);
-          const uint64_t vd = sdesc_mn128(av + kk * 2048, 0);
-          umma_bf16(tO, pd, vd, id_pv, kk ? 1u : 0u);
-        }
-        umma_commit(o_full);
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(tO, tP + kk * 8, sdesc_mn128(av + kk * 2048, 0), id_pv, (kt | kk) ? 1u : 0u);
+        umma_commit(p_free);
         umma_commit(&kv_empty[s]);
       }
+      umma_commit(o_done);
     }
   } else {
     // ------------------------------------------------- softmax + epilogue
     const int r = warp * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    // causal: last visible key of this row; stage II: candidate and token of this row
-    const int qpos = a.q_pos0 + row0 + r;
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const int qpos = a.q_pos0 + row0 + r;  // causal: last visible key of this row
     const int cand = a.mode == MODE_STAGE2 ? r / a.L_NS : 0;
     const int tok = a.mode == MODE_STAGE2 ? r - cand * a.L_NS : 0;
-    // the earliest query of the CTA bounds which tiles need no mask
-    const int qpos_min = a.q_pos0 + row0;
-    float o[64];
-#pragma unroll
-    for (int e = 0; e < 64; ++e) o[e] = 0.f;
+    const int qpos_min = a.q_pos0 + row0;  // earliest query of the CTA: bounds the unmasked tiles
+    // Running max m is only raised when a tile's max exceeds it by more than
+    // 2^8 (then O and l are rescaled); below that, P = 2^(S - m) <= 256 is
+    // exact enough in bf16 and the final O / l is unchanged.
+    const float kThresh = 8.f;
     float m = -INFINITY, l = 0.f;
-    for (int kt = 0; kt < nt; ++kt) {
-      if (!mbar_wait(s_full, kt & 1)) break;
+    bool ok = true;
+    for (int kt = 0; kt < nt && ok; ++kt) {
+      ok = mbar_wait(s_full, kt & 1);
+      if (!ok) break;
       tc_fence_after();
       const int kbase = kt * C::BN;
       const bool ns_tile = kt >= nt_s;
-      // visible keys of this row in this tile: [0, vis) for S tiles; NS tile: a
-      // same-candidate run [lo, hi)
+      // visible keys of this row in this tile: [lo, hi)
       int lo = 0, hi = C::BN;
       if (ns_tile) {
         lo = cand * a.L_NS;
@@ -250,103 +249,125 @@ __global__ void __launch_bounds__(192, 2)
       }
       const bool full = !ns_tile && (a.mode == MODE_CAUSAL ? (kbase + C::BN - 1 <= qpos_min && kbase + C::BN <= n_keys_s)
                                                           : (kbase + C::BN <= n_keys_s));
-      // pass 1: row max of the visible logits
+      // P of the previous tile must be consumed before this one overwrites it
+      if (kt > 0) {
+        ok = mbar_wait(p_free, (kt - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      float mref = m;
       float mx = -INFINITY;
+      if (m == -INFINITY) {
+        // no visible key seen yet: take this tile's max first
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(tS + lane_base + c * 32, sv);
-        if (full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, sv[i]);
-        } else {
+        for (int c = 0; c < 4; ++c) {
+          float sv[32];
+          tmem_ld32(tS + lb + c * 32, sv);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c * 32 + i >= lo && c * 32 + i < hi) mx = fmaxf(mx, sv[i]);
+            if (full || (c * 32 + i >= lo && c * 32 + i < hi)) mx = fmaxf(mx, sv[i]);
         }
+        mref = (mx == -INFINITY) ? 0.f : mx;
       }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m - m_new);
-      const float mref = (m_new == -INFINITY) ? 0.f : m_new;
-      if (kt > 0) {
-        // P.V of the previous tile is done: fold it in; P's buffer is free again
-        if (!mbar_wait(o_full, (kt - 1) & 1)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float ov[32];
-          tmem_ld32(tO + lane_base + c * 32, ov);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[c * 32 + e] = (o[c * 32 + e] + ov[e]) * alpha;
-        }
-      }
-      // pass 2: P = 2^(S - m) as bf16 into the K-major, 128-byte-swizzled A
-      // operand of P.V (row r, key k -> block k/64, 16-byte chunk (k%64)/8 ^ (r%8))
-      float rs = 0.f;
+      float rs = 0.f, mt = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         float sv[32];
-        tmem_ld32(tS + lane_base + c * 32, sv);
+        tmem_ld32(tS + lb + c * 32, sv);
+        uint32_t pk[16];
         if (full) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
+            mt = fmaxf(mt, sv[i]);
             sv[i] = ex2(sv[i] - mref);
             rs += sv[i];
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            sv[i] = (c * 32 + i >= lo && c * 32 + i < hi) ? ex2(sv[i] - mref) : 0.f;
+            const bool vis = c * 32 + i >= lo && c * 32 + i < hi;
+            mt = vis ? fmaxf(mt, sv[i]) : mt;
+            sv[i] = vis ? ex2(sv[i] - mref) : 0.f;
             rs += sv[i];
           }
         }
-        uint8_t* rowp = sP + (c >> 1) * (128 * 128) + r * 128;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int ch = (c & 1) * 4 + q4;
-          uint4 u;
-          __nv_bfloat162* hh = (__nv_bfloat162*)&u;
-#pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) hh[q2] = __floats2bfloat162_rn(sv[q4 * 8 + 2 * q2], sv[q4 * 8 + 2 * q2 + 1]);
-          *(uint4*)(rowp + ((ch ^ (r & 7)) << 4)) = u;
-        }
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(sv[2 * i], sv[2 * i + 1]);
+        tmem_st16(tP + lb + c * 16, pk);
       }
-      l = l * alpha + rs;
-      m = m_new;
-      // keys past the last valid cache key may hold stale bits: zero their V rows
+      if (m == -INFINITY) {
+        m = (mx == -INFINITY) ? -INFINITY : mref;
+        l = rs;
+      } else if (mt > m + kThresh) {
+        // the tile's max ran far past the reference: redo P with the new max and
+        // rescale what O and l hold (O only has tiles < kt: p_free was awaited)
+        const float m_new = mt, alpha = ex2(m - m_new);
+        rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float sv[32];
+          tmem_ld32(tS + lb + c * 32, sv);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const bool vis = full || (c * 32 + i >= lo && c * 32 + i < hi);
+            sv[i] = vis ? ex2(sv[i] - m_new) : 0.f;
+            rs += sv[i];
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(sv[2 * i], sv[2 * i + 1]);
+          tmem_st16(tP + lb + c * 16, pk);
+        }
+        if (kt > 0) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float ov[32];
+            tmem_ld32(tO + lb + c * 32, ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            uint32_t* ou = (uint32_t*)ov;
+            tmem_st16(tO + lb + c * 32, ou);
+            tmem_st16(tO + lb + c * 32 + 16, ou + 16);
+          }
+        }
+        l = l * alpha + rs;
+        m = m_new;
+      } else {
+        l += rs;
+      }
+      // keys past the last valid cache key may hold stale bits (P is 0 there,
+      // but 0 * NaN is not): zero their V rows before P.V reads them
       if (kt == nt_s - 1 && kbase + r > kmax) {
         uint4* vrow = (uint4*)(sKV + (kt & 1) * 2 * C::KV_BYTES + C::KV_BYTES + r * 128);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) vrow[ch] = make_uint4(0, 0, 0, 0);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    if (nt > 0 && mbar_wait(o_full, (nt - 1) & 1)) {
-      tc_fence_after();
+    ok = ok && mbar_wait(o_done, 0);
+    tc_fence_after();
+    float o[64];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float ov[32];
-        tmem_ld32(tO + lane_base + c * 32, ov);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[c * 32 + e] += ov[e];
-      }
-    }
+    for (int c = 0; c < 2; ++c) tmem_ld32(tO + lb + c * 32, o + c * 32);
     const float inv = 1.f / l;
 #pragma unroll
     for (int e = 0; e < 64; ++e) o[e] *= inv;
-    if (a.mode == MODE_CAUSAL) {
-      const int t = row0 + r;
-      if (t < a.Lq) {
-        __nv_bfloat16* dst = (__nv_bfloat16*)a.o.base + rm_off(a.o, b, t, h * 64);
+    if (ok && nt > 0) {
+      if (a.mode == MODE_CAUSAL) {
+        const int t = row0 + r;
+        if (t < a.Lq) {
+          __nv_bfloat16* dst = (__nv_bfloat16*)a.o.base + rm_off(a.o, b, t, h * 64);
+          store_bf16x32(dst, o);
+          store_bf16x32(dst + 32, o + 32);
+        }
+      } else if (r < n_rows) {
+        __nv_bfloat16* dst = a.o2 + (long long)(row0 + r) * (a.H * 64) + h * 64;
         store_bf16x32(dst, o);
         store_bf16x32(dst + 32, o + 32);
       }
-    } else if (r < n_rows) {
-      __nv_bfloat16* dst = a.o2 + (long long)(row0 + r) * (a.H * 64) + h * 64;
-      store_bf16x32(dst, o);
-      store_bf16x32(dst + 32, o + 32);
     }
   }
   tc_fence_before();

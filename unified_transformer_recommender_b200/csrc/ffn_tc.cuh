@@ -84,7 +84,6 @@ __device__ inline void tmem_st32(uint32_t taddr, const float* v) {
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
-__device__ inline void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 fp32 values of row r into box `box` of a staging area of [128 rows x
 // 128 B] boxes with the 128-byte swizzle (the layout TMA reads and writes).
