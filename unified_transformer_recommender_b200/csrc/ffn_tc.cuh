@@ -24,8 +24,10 @@
 // into D.  up(c+2) is issued right after down(c), so GELU of one chunk
 // overlaps the MMAs of the next.
 //
-// Warp roles (192 threads): warps 0-3 compute (one row per thread), warp 4
-// TMA producer, warp 5 TMEM allocator and MMA issuer.
+// Warp roles (320 threads): warps 0-7 compute (two warps per row quarter:
+// warp w and w+4 share TMEM lanes 32*(w%4).. and split each row's columns,
+// exchanging row sums through shared memory), warp 8 TMA producer, warp 9
+// TMEM allocator and MMA issuer.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -61,7 +63,7 @@ struct FfnCfg {
   static constexpr int H_BYTES = BM * HC * 2;        // 32 KB per hidden chunk buffer
   static constexpr int STAGE = 32768;                // one weight stage
   static constexpr int STAGES = 3;
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int BAR_BYTES = 256 + 1024;        // barriers + per-row partial sums
   static constexpr int SMEM = A_BYTES + 2 * H_BYTES + STAGES * STAGE + BAR_BYTES;
   static constexpr int TMEM_COLS = 512;              // D 0..255, U0 256..383, U1 384..511
 };
@@ -136,7 +138,9 @@ __device__ inline void st_sw128_32(uint8_t* tile, int blk_bytes, int r, int col0
   }
 }
 
-__global__ void __launch_bounds__(192, 1)
+constexpr int kFfnThreads = 320;
+
+__global__ void __launch_bounds__(kFfnThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmWo,
                   const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmW2,
                   const __grid_constant__ CUtensorMap tmRes, const __grid_constant__ CUtensorMap tmOut,
@@ -160,6 +164,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* sh_free = bars + 18;
   uint64_t* res_ready = bars + 19;
   uint32_t* tmem_slot = (uint32_t*)(bars + 20);
+  float* red = (float*)((uint8_t*)bars + 256);  // [2][128] partial row sums
 
   if (smem_u32(smem) & 1023) {
     if (threadIdx.x == 0) flag_error(kErrSmemAlign);
@@ -175,18 +180,18 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(a_full, 1);
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&w_full[s], 1); mbar_init(&w_empty[s], 1); }
     mbar_init(d_full, 1);
-    mbar_init(h2_ready, 128);
-    for (int i = 0; i < 2; ++i) { mbar_init(&u_full[i], 1); mbar_init(&hid_full[i], 128); mbar_init(&hid_free[i], 1); }
+    mbar_init(h2_ready, 256);
+    for (int i = 0; i < 2; ++i) { mbar_init(&u_full[i], 1); mbar_init(&hid_full[i], 256); mbar_init(&hid_free[i], 1); }
     mbar_init(d_done, 1);
     mbar_init(&res_full[0], 1); mbar_init(&res_full[1], 1);
-    mbar_init(sh_free, 128);
-    mbar_init(res_ready, 128);
+    mbar_init(sh_free, 256);
+    mbar_init(res_ready, 256);
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tmap(&tmA); prefetch_tmap(&tmWo); prefetch_tmap(&tmW1); prefetch_tmap(&tmW2);
   }
-  if (warp == 5) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  if (warp == 9) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   };
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_expect_tx(a_full, C::A_BYTES);
@@ -252,7 +257,7 @@ __global__ void __launch_bounds__(192, 1)
           for (int j = 0; j < 2 && ok; ++j) ok = stage(1, c + 2, j);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t id256 = idesc_bf16(128, 256);
@@ -319,15 +324,25 @@ __global__ void __launch_bounds__(192, 1)
       }
       umma_commit(d_done);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------- compute
-    const int r = warp * 32 + lane;
+    const int q4 = warp & 3, wg = warp >> 2;   // row quarter, column half
+    const int r = q4 * 32 + lane;
     const int m = mt0 + r;
     const bool valid = m < d.m_lo + d.M;
     int b = 0, t = 0;
     if (valid) row_of_rows(d.mode, d.fold, m, g, b, t);
-    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const uint32_t lb = (uint32_t)(q4 * 32) << 16;
+    const int cD = wg * (C::D / 2);            // this warp's first column of a d-wide row
     const __nv_bfloat16* gffn = (const __nv_bfloat16*)d.g_ffn;
+    // full-row sum from the two column halves of row r
+    auto row_sum = [&](float part) -> float {
+      red[wg * 128 + r] = part;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float s2 = red[r] + red[128 + r];
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      return s2;
+    };
     bool ok = true;
     // residual rows into D (the W^O product accumulates on top)
     if (io.res_tma) {
@@ -335,7 +350,7 @@ __global__ void __launch_bounds__(192, 1)
         ok = mbar_wait(&res_full[k], 0);
         if (!ok) break;
 #pragma unroll 1
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 2 * wg; i < 2 * wg + 2; ++i) {
           float v[64];
           if (io.res_f32) {
             ld_sw128_f32(sH, i, r, v);
@@ -350,12 +365,12 @@ __global__ void __launch_bounds__(192, 1)
       }
     } else {
       float nxt[32];
-      if (valid) load_row32(d.res, rm_off(d.res, b, t, 0), nxt);
-      for (int c0 = 0; c0 < C::D; c0 += 32) {
+      if (valid) load_row32(d.res, rm_off(d.res, b, t, cD), nxt);
+      for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = valid ? nxt[i] : 0.f;
-        if (valid && c0 + 32 < C::D) load_row32(d.res, rm_off(d.res, b, t, c0 + 32), nxt);
+        if (valid && c0 + 32 < cD + C::D / 2) load_row32(d.res, rm_off(d.res, b, t, c0 + 32), nxt);
         tmem_st32(tD + lb + c0, v);
       }
     }
@@ -366,14 +381,14 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     // D = x_mid; its RMSNorm becomes h2 in sA
     float ss = 0.f;
-    for (int c0 = 0; c0 < C::D; c0 += 32) {
+    for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
       float v[32];
       tmem_ld32(tD + lb + c0, v);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ss += v[i] * v[i];
+      for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
     }
-    const float rr = rsqrtf(ss / C::D + d.eps);
-    for (int c0 = 0; c0 < C::D; c0 += 32) {
+    const float rr = rsqrtf(row_sum(ss) / C::D + d.eps);
+    for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
       float v[32], gv[32];
       tmem_ld32(tD + lb + c0, v);
       load_bf16x32(gffn + c0, gv);
@@ -384,8 +399,10 @@ __global__ void __launch_bounds__(192, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     mbar_arrive(h2_ready);
-    // hidden chunks: b1 + GELU into shared memory for the down-projection
+    // hidden chunks: b1 + GELU into shared memory for the down-projection;
+    // each warp takes half of the chunk's columns
     const __nv_bfloat16* b1 = (const __nv_bfloat16*)d.b1 + (long long)grp * d.b1_sg;
+    const int cH = wg * (C::HC / 2);
     for (int c = 0; c < NC && ok; ++c) {
       ok = mbar_wait(&u_full[c & 1], (c >> 1) & 1);
       if (ok && c >= 2) ok = mbar_wait(&hid_free[c & 1], ((c >> 1) - 1) & 1);
@@ -393,7 +410,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t tU = tU0 + (c & 1) * C::HC;
       uint8_t* hbuf = sH + (c & 1) * C::H_BYTES;
-      for (int c0 = 0; c0 < C::HC; c0 += 32) {
+      for (int c0 = cH; c0 < cH + C::HC / 2; c0 += 32) {
         float v[32], bv[32];
         tmem_ld32(tU + lb + c0, v);
         load_bf16x32(b1 + c * C::HC + c0, bv);
@@ -411,19 +428,19 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const __nv_bfloat16* b2 = (const __nv_bfloat16*)d.b2 + (long long)grp * d.b2_sg;
     ss = 0.f;
-    for (int c0 = 0; c0 < C::D; c0 += 32) {
+    for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
       float v[32], bv[32];
       tmem_ld32(tD + lb + c0, v);
       load_bf16x32(b2 + c0, bv);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) { v[i] += bv[i]; ss += v[i] * v[i]; }
+      for (int i = 0; i < 32; ++i) { v[i] += bv[i]; ss = fmaf(v[i], v[i], ss); }
       if (io.out_tma) st_sw128_f32(sA, c0 >> 5, r, v);          // sA + sH: 8 boxes of 32 fp32
       else if (valid && ok) store_row32(d.out, rm_off(d.out, b, t, c0), v);
     }
     if (d.hout.base) {
-      const float r2 = rsqrtf(ss / C::D + d.eps);
+      const float r2 = rsqrtf(row_sum(ss) / C::D + d.eps);
       const __nv_bfloat16* gn = (const __nv_bfloat16*)d.g_next;
-      for (int c0 = 0; c0 < C::D; c0 += 32) {
+      for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
         float v[32], bv[32], gv[32];
         tmem_ld32(tD + lb + c0, v);
         load_bf16x32(b2 + c0, bv);
@@ -436,8 +453,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (io.out_tma || io.hout_tma) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (r == 0 && ok) {
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (threadIdx.x == 0 && ok) {
         if (io.out_tma) {
           for (int i = 0; i < 8; ++i) {
             if (io.out_swap) tma_store_3d(&tmOut, sA + i * 16384, i * 32, g, mt0);
@@ -457,7 +474,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ host --
@@ -529,7 +546,7 @@ inline onetrans_status tc_ffn_launch(const FfnDesc& d, cudaStream_t st) {
     attr_set = true;
   }
   dim3 grid((unsigned)((d.M + C::BM - 1) / C::BM), (unsigned)d.G);
-  ffn_tc_kernel<<<grid, 192, C::SMEM, st>>>(ta, two, tw1, tw2, tres, tout, thout, d, a_swap, io);
+  ffn_tc_kernel<<<grid, kFfnThreads, C::SMEM, st>>>(ta, two, tw1, tw2, tres, tout, thout, d, a_swap, io);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 

@@ -182,8 +182,10 @@ __device__ inline float tanh_fast(float x) {
   return y;
 }
 __device__ inline float gelu_fast(float x) {
-  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-  return 0.5f * x * (1.0f + tanh_fast(k0 * (x + k1 * x * x * x)));
+  // 0.5 x (1 + tanh(k0 x + k0 k1 x^3)) = hx + hx tanh(x (k0 + k0 k1 x^2)), hx = x / 2
+  const float k0 = 0.7978845608028654f, k01 = 0.7978845608028654f * 0.044715f;
+  const float hx = 0.5f * x;
+  return fmaf(hx, tanh_fast(x * fmaf(k01, x * x, k0)), hx);
 }
 
 // -------------------------------------------------------- bf16 vectors --
