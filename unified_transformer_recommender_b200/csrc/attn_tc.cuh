@@ -150,9 +150,10 @@ __global__ void __launch_bounds__(192, 2)
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && nt > 0) {
+      const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
       mbar_expect_tx(q_full, C::Q_BYTES);
-      if (a.mode == MODE_CAUSAL) tma_load_3d(&tmQ, q_full, sQ, h * C::DH, row0, b);
-      else tma_load_3d(&tmQ, q_full, sQ, h * C::DH, row0, 0);
+      if (a.mode == MODE_CAUSAL) tma_load_3d_hint(&tmQ, q_full, sQ, h * C::DH, row0, b, stream);
+      else tma_load_3d_hint(&tmQ, q_full, sQ, h * C::DH, row0, 0, stream);
       for (int kt = 0; kt < nt; ++kt) {
         const int s = kt & 1;
         if (kt >= 2 && !mbar_wait(&kv_empty[s], ((kt >> 1) - 1) & 1)) break;
@@ -165,14 +166,14 @@ __global__ void __launch_bounds__(192, 2)
             const int pi = kt * 2 + hp;
             const int pg = pi < C::MAX_PAGES ? s_pages[pi]
                                              : (pi < n_pages_used ? kv_page_id(a.kv, b, pi) : a.kv.n_pages);
-            tma_load_4d(&tmKV, &kv_full[s], sk + hp * C::PAGE_BYTES, 0, 0, h, pg);
-            tma_load_4d(&tmKV, &kv_full[s], sv + hp * C::PAGE_BYTES, 0, 0, a.H + h, pg);
+            tma_load_4d_hint(&tmKV, &kv_full[s], sk + hp * C::PAGE_BYTES, 0, 0, h, pg, keep);
+            tma_load_4d_hint(&tmKV, &kv_full[s], sv + hp * C::PAGE_BYTES, 0, 0, a.H + h, pg, keep);
           }
         } else {
           // own NS keys of this CTA's candidates: the K and V column blocks of the same rows
           const int d = a.H * C::DH;
-          tma_load_3d(&tmNS, &kv_full[s], sk, d + h * C::DH, row0, 0);
-          tma_load_3d(&tmNS, &kv_full[s], sv, 2 * d + h * C::DH, row0, 0);
+          tma_load_3d_hint(&tmNS, &kv_full[s], sk, d + h * C::DH, row0, 0, stream);
+          tma_load_3d_hint(&tmNS, &kv_full[s], sv, 2 * d + h * C::DH, row0, 0, stream);
         }
       }
     }

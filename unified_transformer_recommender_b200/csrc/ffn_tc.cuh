@@ -7,22 +7,20 @@
 //   h_next = RMSNorm(x_next) * g_next               (next layer's pre-norm)
 //
 // Only a, x, x_next and h_next touch HBM; x_mid and the d_ff-wide hidden
-// layer stay on chip.  TMEM holds D (256 fp32 columns: W^O a, then x_mid,
-// then x_mid + W2 hidden, since the down-projection accumulates on top of
-// x_mid) and two 128-column buffers U0/U1 for hidden chunks.  Shared memory
-// holds the attention tile (reused for h2 as the A operand of the
-// up-projection), two 128-wide hidden chunks (A operand of the
-// down-projection) and a 3-stage ring of weight tiles fed by TMA.
+// layer stay on chip.  TMEM holds D (256 fp32 columns: the residual rows,
+// then + W^O a = x_mid, then + W2 hidden, since both products accumulate in
+// place), two 64-column buffers U0/U1 for the up-projection of a hidden
+// chunk, and two 32-column buffers H0/H1 for the GELU output of a chunk as
+// packed bf16 pairs, which the down-projection reads as its A operand.
+// Shared memory holds the attention tile (reused for h2 as the A operand of
+// the up-projection) and a 5-stage ring of 32 KB tiles fed by TMA: first the
+// residual rows, then W^O, then W1/W2 chunk by chunk.  x_next and h_next
+// leave by TMA stores staged through the then idle shared memory.  Row
+// geometries TMA cannot express fall back to per-thread loads/stores.
 //
-// The residual rows arrive by TMA (staged through the hidden-chunk buffers)
-// and are written into D before W^O a accumulates on top of them; x_next and
-// h_next leave by TMA stores staged through the then idle shared memory.
-// Row geometries TMA cannot express fall back to per-thread loads/stores.
-//
-// Per hidden chunk c (128 units): up(c) -> U[c%2]; the four compute warps
-// apply b1 + GELU and write the chunk to shared memory; down(c) accumulates
-// into D.  up(c+2) is issued right after down(c), so GELU of one chunk
-// overlaps the MMAs of the next.
+// Per hidden chunk c (64 units): up(c) -> U[c%2]; the compute warps apply
+// b1 + GELU and write H[c%2]; down(c) accumulates into D; up(c+2) follows
+// right after, so GELU of one chunk overlaps the MMAs of the next.
 //
 // Warp roles (320 threads): warps 0-7 compute (two warps per row quarter:
 // warp w and w+4 share TMEM lanes 32*(w%4).. and split each row's columns,
@@ -59,13 +57,12 @@ struct FfnIo {
 
 struct FfnCfg {
   static constexpr int D = 256, BM = 128, HC = 128;  // hidden chunk width
-  static constexpr int A_BYTES = BM * D * 2;         // 64 KB: attention tile, then h2
-  static constexpr int H_BYTES = BM * HC * 2;        // 32 KB per hidden chunk buffer
-  static constexpr int STAGE = 32768;                // one weight stage
-  static constexpr int STAGES = 3;
-  static constexpr int BAR_BYTES = 256 + 1024;        // barriers + per-row partial sums
-  static constexpr int SMEM = A_BYTES + 2 * H_BYTES + STAGES * STAGE + BAR_BYTES;
-  static constexpr int TMEM_COLS = 512;              // D 0..255, U0 256..383, U1 384..511
+  static constexpr int A_BYTES = BM * D * 2;        // 64 KB: attention tile, then h2
+  static constexpr int STAGE = 32768;               // one ring stage
+  static constexpr int STAGES = 5;
+  static constexpr int BAR_BYTES = 256 + 1024;       // barriers + per-row partial sums
+  static constexpr int SMEM = A_BYTES + STAGES * STAGE + BAR_BYTES;
+  static constexpr int TMEM_COLS = 512;  // D 0..255, U0 256..383, U1 384..511 (GELU output packed over U)
 };
 
 __device__ inline void tmem_st32(uint32_t taddr, const float* v) {
@@ -148,22 +145,19 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   using C = FfnCfg;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sA = smem;
-  uint8_t* sH = sA + C::A_BYTES;                 // [2][128 rows x 128]
-  uint8_t* sW = sH + 2 * C::H_BYTES;             // [3][32 KB]
+  uint8_t* sW = sA + C::A_BYTES;  // [STAGES][32 KB]
   uint64_t* bars = (uint64_t*)(sW + C::STAGES * C::STAGE);
   uint64_t* a_full = bars;
-  uint64_t* w_full = bars + 1;    // [3]
-  uint64_t* w_empty = bars + 4;   // [3]
-  uint64_t* d_full = bars + 7;
-  uint64_t* h2_ready = bars + 8;
-  uint64_t* u_full = bars + 9;    // [2]
-  uint64_t* hid_full = bars + 11; // [2]
-  uint64_t* hid_free = bars + 13; // [2]
-  uint64_t* d_done = bars + 15;
-  uint64_t* res_full = bars + 16;  // [2]
-  uint64_t* sh_free = bars + 18;
-  uint64_t* res_ready = bars + 19;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 20);
+  uint64_t* w_full = bars + 1;             // [STAGES]
+  uint64_t* w_empty = w_full + C::STAGES;  // [STAGES]
+  uint64_t* d_full = w_empty + C::STAGES;
+  uint64_t* h2_ready = d_full + 1;
+  uint64_t* u_full = h2_ready + 1;   // [2]
+  uint64_t* hid_full = u_full + 2;   // [2]
+  uint64_t* dn_done = hid_full + 2;  // [2]
+  uint64_t* d_done = dn_done + 2;
+  uint64_t* res_ready = d_done + 1;
+  uint32_t* tmem_slot = (uint32_t*)(res_ready + 1);
   float* red = (float*)((uint8_t*)bars + 256);  // [2][128] partial row sums
 
   if (smem_u32(smem) & 1023) {
@@ -175,21 +169,23 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   const int g = d.g_lo + blockIdx.y;
   const int grp = d.mode == TILE_SAMPLES ? g - d.grp_base : 0;
   const int NC = d.dff / C::HC;
+  // residual stages at the head of the ring: fp32 rows in 4 stages of 64
+  // columns, bf16 rows in 2 stages of 128 columns (two 16 KB boxes each)
+  const int RP = io.res_tma ? (io.res_f32 ? 4 : 2) : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(a_full, 1);
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&w_full[s], 1); mbar_init(&w_empty[s], 1); }
     mbar_init(d_full, 1);
     mbar_init(h2_ready, 256);
-    for (int i = 0; i < 2; ++i) { mbar_init(&u_full[i], 1); mbar_init(&hid_full[i], 256); mbar_init(&hid_free[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&u_full[i], 1); mbar_init(&hid_full[i], 256); mbar_init(&dn_done[i], 1); }
     mbar_init(d_done, 1);
-    mbar_init(&res_full[0], 1); mbar_init(&res_full[1], 1);
-    mbar_init(sh_free, 256);
     mbar_init(res_ready, 256);
     fence_barrier_init();
   }
   if (warp == 8 && lane == 0) {
     prefetch_tmap(&tmA); prefetch_tmap(&tmWo); prefetch_tmap(&tmW1); prefetch_tmap(&tmW2);
+    if (io.res_tma) prefetch_tmap(&tmRes);
   }
   if (warp == 9) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
@@ -197,58 +193,45 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tD = tmem, tU0 = tmem + 256;
-  // residual boxes: fp32 = 8 boxes of 32 columns in two rounds, bf16 = 4 of 64 in one
-  const int res_rounds = io.res_f32 ? 2 : 1;
-  auto res_round = [&](int k) {
-    mbar_expect_tx(&res_full[k], 4 * 16384);
-    const int bc = io.res_f32 ? 32 : 64;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int col = (k * 4 + i) * bc;
-      if (io.res_swap) tma_load_3d(&tmRes, &res_full[k], sH + i * 16384, col, g, mt0);
-      else tma_load_3d(&tmRes, &res_full[k], sH + i * 16384, col, mt0, g);
-    }
-  };
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
       mbar_expect_tx(a_full, C::A_BYTES);
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
-        if (a_swap) tma_load_3d(&tmA, a_full, sA + kb * 16384, kb * 64, g, mt0);
-        else tma_load_3d(&tmA, a_full, sA + kb * 16384, kb * 64, mt0, g);
+        if (a_swap) tma_load_3d_hint(&tmA, a_full, sA + kb * 16384, kb * 64, g, mt0, stream);
+        else tma_load_3d_hint(&tmA, a_full, sA + kb * 16384, kb * 64, mt0, g, stream);
       }
-      if (io.res_tma) {
-        prefetch_tmap(&tmRes);
-        res_round(0);
-      }
-      int q = 0;  // weight stage counter, in the order the MMA thread consumes them
+      int q = 0;  // ring stage counter, in the order the stages are consumed
       auto stage = [&](int kind, int c, int j) -> bool {
         const int s = q % C::STAGES;
         if (q >= C::STAGES && !mbar_wait(&w_empty[s], ((q / C::STAGES) - 1) & 1)) return false;
         uint8_t* dst = sW + s * C::STAGE;
         mbar_expect_tx(&w_full[s], C::STAGE);
-        if (kind == 0) {          // W^O k-block j: [256 out x 64]
-          tma_load_3d(&tmWo, &w_full[s], dst, j * 64, 0, 0);
+        if (kind == 3) {          // residual rows, columns of part j
+          const int bc = io.res_f32 ? 32 : 64;
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx) {
+            const int col = (2 * j + bx) * bc;
+            if (io.res_swap) tma_load_3d_hint(&tmRes, &w_full[s], dst + bx * 16384, col, g, mt0, stream);
+            else tma_load_3d_hint(&tmRes, &w_full[s], dst + bx * 16384, col, mt0, g, stream);
+          }
+        } else if (kind == 0) {   // W^O k-block j: [256 out x 64]
+          tma_load_3d_hint(&tmWo, &w_full[s], dst, j * 64, 0, 0, keep);
         } else if (kind == 1) {   // W1 chunk c, k-blocks 2j, 2j+1: [128 hidden x 64] each
-          tma_load_3d(&tmW1, &w_full[s], dst, (2 * j) * 64, c * C::HC, grp);
-          tma_load_3d(&tmW1, &w_full[s], dst + 16384, (2 * j + 1) * 64, c * C::HC, grp);
-        } else {                  // W2 chunk c, k-block j: [256 out x 64 hidden]
-          tma_load_3d(&tmW2, &w_full[s], dst, c * C::HC + j * 64, 0, grp);
+          tma_load_3d_hint(&tmW1, &w_full[s], dst, (2 * j) * 64, c * C::HC, grp, keep);
+          tma_load_3d_hint(&tmW1, &w_full[s], dst + 16384, (2 * j + 1) * 64, c * C::HC, grp, keep);
+        } else {                  // W2 chunk c, hidden k-block j: [256 out x 64 hidden]
+          tma_load_3d_hint(&tmW2, &w_full[s], dst, c * C::HC + j * 64, 0, grp, keep);
         }
         ++q;
         return true;
       };
       bool ok = true;
-      for (int j = 0; j < 3 && ok; ++j) ok = stage(0, 0, j);
-      // the second residual round reuses the staging buffer once it is copied out;
-      // issue it before any weight stage that waits on the MMAs
-      if (io.res_tma && res_rounds == 2 && ok) {
-        ok = mbar_wait(sh_free, 0);
-        if (ok) res_round(1);
-      }
-      if (ok) ok = stage(0, 0, 3);
+      for (int j = 0; j < RP && ok; ++j) ok = stage(3, 0, j);
+      for (int j = 0; j < 4 && ok; ++j) ok = stage(0, 0, j);
       for (int c = 0; c < 2 && c < NC && ok; ++c)
         for (int j = 0; j < 2 && ok; ++j) ok = stage(1, c, j);
       for (int c = 0; c < NC && ok; ++c) {
@@ -262,9 +245,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     if (lane == 0) {
       constexpr uint32_t id256 = idesc_bf16(128, 256);
       constexpr uint32_t id128 = idesc_bf16(128, 128);
-      const uint32_t aA = smem_u32(sA), aH = smem_u32(sH), aW = smem_u32(sW);
-      int q = 0;
-      bool ok = mbar_wait(a_full, 0) && mbar_wait(res_ready, 0);
+      const uint32_t aA = smem_u32(sA), aW = smem_u32(sW);
+      int q = RP;  // the residual stages are consumed by the compute warps
       auto wait_stage = [&](uint32_t& base) -> bool {
         const int s = q % C::STAGES;
         if (!mbar_wait(&w_full[s], (q / C::STAGES) & 1)) return false;
@@ -291,6 +273,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         umma_commit(&u_full[c & 1]);
         return true;
       };
+      bool ok = mbar_wait(a_full, 0) && mbar_wait(res_ready, 0);
+      if (ok) tc_fence_after();
       // D holds the residual rows: x_mid = x + a W^O^T accumulates in place
       for (int j = 0; j < 4 && ok; ++j) {
         uint32_t wb;
@@ -309,22 +293,23 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         ok = mbar_wait(&hid_full[c & 1], (c >> 1) & 1);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t hb = aH + (c & 1) * C::H_BYTES;
+        // D += H W2c^T: A = the GELU output packed over U[c%2] (16 hidden = 8 columns per step)
+        const uint32_t tH = tU0 + (c & 1) * C::HC;
         for (int j = 0; j < 2 && ok; ++j) {
           uint32_t wb;
           ok = wait_stage(wb);
           if (!ok) break;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tD, sdesc_k128(hb + j * 16384 + k * 32), sdesc_k128(wb + k * 32), id256, 1u);
+          for (int k = 0; k < 4; ++k) umma_bf16_ts(tD, tH + j * 32 + k * 8, sdesc_k128(wb + k * 32), id256, 1u);
           free_stage();
         }
-        umma_commit(&hid_free[c & 1]);
-        if (ok && c + 2 < NC) ok = up(c + 2);
+        umma_commit(&dn_done[c & 1]);
+        // up(c+2) overwrites U[c%2]: let down(c) finish reading it first
+        if (ok && c + 2 < NC) ok = mbar_wait(&dn_done[c & 1], (c >> 1) & 1) && up(c + 2);
       }
       umma_commit(d_done);
     }
-  } else if (warp < 8) {
+  } else {
     // ------------------------------------------------------------- compute
     const int q4 = warp & 3, wg = warp >> 2;   // row quarter, column half
     const int r = q4 * 32 + lane;
@@ -346,22 +331,25 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     bool ok = true;
     // residual rows into D (the W^O product accumulates on top)
     if (io.res_tma) {
-      for (int k = 0; k < res_rounds && ok; ++k) {
-        ok = mbar_wait(&res_full[k], 0);
-        if (!ok) break;
-#pragma unroll 1
-        for (int i = 2 * wg; i < 2 * wg + 2; ++i) {
+      // every compute thread passes each named barrier, even after a failed wait
+      for (int p = 0; p < RP; ++p) {
+        const int s = p % C::STAGES;
+        ok = ok && mbar_wait(&w_full[s], (p / C::STAGES) & 1);
+        if (ok) {
+          const uint8_t* st = sW + s * C::STAGE;
           float v[64];
           if (io.res_f32) {
-            ld_sw128_f32(sH, i, r, v);
-            tmem_st32(tD + lb + (k * 4 + i) * 32, v);
+            ld_sw128_f32(st, wg, r, v);
+            tmem_st32(tD + lb + (2 * p + wg) * 32, v);
           } else {
-            ld_sw128_bf16(sH, i, r, v);
-            tmem_st32(tD + lb + i * 64, v);
-            tmem_st32(tD + lb + i * 64 + 32, v + 32);
+            ld_sw128_bf16(st, wg, r, v);
+            tmem_st32(tD + lb + (2 * p + wg) * 64, v);
+            tmem_st32(tD + lb + (2 * p + wg) * 64 + 32, v + 32);
           }
         }
-        if (k == 0 && res_rounds == 2) mbar_arrive(sh_free);
+        // the stage may be refilled once every compute thread has read it
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (threadIdx.x == 0) mbar_arrive(&w_empty[s]);
       }
     } else {
       float nxt[32];
@@ -399,33 +387,40 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     mbar_arrive(h2_ready);
-    // hidden chunks: b1 + GELU into shared memory for the down-projection;
-    // each warp takes half of the chunk's columns
+    // hidden chunks: b1 + GELU, packed bf16 into H[c%2]; each warp takes half
+    // of the chunk's columns
     const __nv_bfloat16* b1 = (const __nv_bfloat16*)d.b1 + (long long)grp * d.b1_sg;
     const int cH = wg * (C::HC / 2);
-    for (int c = 0; c < NC && ok; ++c) {
-      ok = mbar_wait(&u_full[c & 1], (c >> 1) & 1);
-      if (ok && c >= 2) ok = mbar_wait(&hid_free[c & 1], ((c >> 1) - 1) & 1);
-      if (!ok) break;
+    for (int c = 0; c < NC; ++c) {
+      ok = ok && mbar_wait(&u_full[c & 1], (c >> 1) & 1);
       tc_fence_after();
       const uint32_t tU = tU0 + (c & 1) * C::HC;
-      uint8_t* hbuf = sH + (c & 1) * C::H_BYTES;
-      for (int c0 = cH; c0 < cH + C::HC / 2; c0 += 32) {
-        float v[32], bv[32];
-        tmem_ld32(tU + lb + c0, v);
-        load_bf16x32(b1 + c * C::HC + c0, bv);
+      uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i] + bv[i]);
-        st_sw128_32(hbuf, 16384, r, c0, v);
+      for (int h = 0; h < 2; ++h) {
+        float v[32], bv[32];
+        tmem_ld32(tU + lb + cH + h * 32, v);
+        load_bf16x32(b1 + c * C::HC + cH + h * 32, bv);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[h * 16 + i] = pack_bf16x2(gelu_fast(v[2 * i] + bv[2 * i]), gelu_fast(v[2 * i + 1] + bv[2 * i + 1]));
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // the packed output overwrites U's first half: both column halves must be read first
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      tmem_st16(tU + lb + cH / 2, pk);
+      tmem_st16(tU + lb + cH / 2 + 16, pk + 16);
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&hid_full[c & 1]);
     }
-    // x_next = D + b2, and the next layer's RMSNorm; every MMA is done, so the
-    // whole of shared memory can stage the outputs for TMA stores
+    // x_next = D + b2, and the next layer's RMSNorm; every MMA is done, so
+    // the whole of shared memory can stage the outputs for TMA stores:
+    // x_next in 8 boxes of 32 fp32 columns from offset 0, h_next in 4 boxes
+    // of 64 bf16 columns from offset 128 KB
     ok = ok && mbar_wait(d_done, 0);
     tc_fence_after();
+    uint8_t* stage_x = smem;
+    uint8_t* stage_h = smem + 8 * 16384;
     const __nv_bfloat16* b2 = (const __nv_bfloat16*)d.b2 + (long long)grp * d.b2_sg;
     ss = 0.f;
     for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
@@ -434,7 +429,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       load_bf16x32(b2 + c0, bv);
 #pragma unroll
       for (int i = 0; i < 32; ++i) { v[i] += bv[i]; ss = fmaf(v[i], v[i], ss); }
-      if (io.out_tma) st_sw128_f32(sA, c0 >> 5, r, v);          // sA + sH: 8 boxes of 32 fp32
+      if (io.out_tma) st_sw128_f32(stage_x, c0 >> 5, r, v);
       else if (valid && ok) store_row32(d.out, rm_off(d.out, b, t, c0), v);
     }
     if (d.hout.base) {
@@ -447,7 +442,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         load_bf16x32(gn + c0, gv);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = (v[i] + bv[i]) * r2 * gv[i];
-        if (io.hout_tma) st_sw128_32(sW, 16384, r, c0, v);          // ring: 4 boxes of 64 bf16
+        if (io.hout_tma) st_sw128_32(stage_h, 16384, r, c0, v);
         else if (valid && ok) store_row32(d.hout, rm_off(d.hout, b, t, c0), v);
       }
     }
@@ -457,14 +452,14 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       if (threadIdx.x == 0 && ok) {
         if (io.out_tma) {
           for (int i = 0; i < 8; ++i) {
-            if (io.out_swap) tma_store_3d(&tmOut, sA + i * 16384, i * 32, g, mt0);
-            else tma_store_3d(&tmOut, sA + i * 16384, i * 32, mt0, g);
+            if (io.out_swap) tma_store_3d(&tmOut, stage_x + i * 16384, i * 32, g, mt0);
+            else tma_store_3d(&tmOut, stage_x + i * 16384, i * 32, mt0, g);
           }
         }
         if (io.hout_tma && d.hout.base) {
           for (int i = 0; i < 4; ++i) {
-            if (io.hout_swap) tma_store_3d(&tmHout, sW + i * 16384, i * 64, g, mt0);
-            else tma_store_3d(&tmHout, sW + i * 16384, i * 64, mt0, g);
+            if (io.hout_swap) tma_store_3d(&tmHout, stage_h + i * 16384, i * 64, g, mt0);
+            else tma_store_3d(&tmHout, stage_h + i * 16384, i * 64, mt0, g);
           }
         }
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
@@ -526,7 +521,7 @@ inline onetrans_status tc_ffn_launch(const FfnDesc& d, cudaStream_t st) {
                    : make_tmap_3d(&ta, d.A, C::D, mext, gext, s_m, s_g, 64, 128, 1);
   ok = ok && make_tmap_3d(&two, d.Wo, C::D, C::D, 1, C::D, (uint64_t)C::D * C::D, 64, 256, 1);
   ok = ok && make_tmap_3d(&tw1, d.W1, C::D, d.dff, wg, C::D, wg > 1 ? (uint64_t)d.w1_sg : (uint64_t)d.dff * C::D,
-                          64, C::HC, 1);
+                          64, C::HC, 1);  // one k-block of a hidden chunk: [64 x 64]
   ok = ok && make_tmap_3d(&tw2, d.W2, d.dff, C::D, wg, d.dff, wg > 1 ? (uint64_t)d.w2_sg : (uint64_t)d.dff * C::D,
                           64, 256, 1);
   if (!ok) return ONETRANS_ERR_CUDA;

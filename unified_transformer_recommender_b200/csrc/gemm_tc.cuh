@@ -71,6 +71,7 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
 
   if (warp == 4) {
     if (lane == 0) {
+      const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % C::STAGES;
         const uint32_t ph = (kb / C::STAGES) & 1;
@@ -78,11 +79,11 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
         uint8_t* sa = smem + s * C::STAGE_BYTES;
         uint8_t* sb = sa + C::A_BYTES;
         mbar_expect_tx(&full[s], C::STAGE_BYTES);
-        if (a_swap) tma_load_3d(&tmA, &full[s], sa, kb * 64, g, mt0);
-        else tma_load_3d(&tmA, &full[s], sa, kb * 64, mt0, g);
+        if (a_swap) tma_load_3d_hint(&tmA, &full[s], sa, kb * 64, g, mt0, stream);
+        else tma_load_3d_hint(&tmA, &full[s], sa, kb * 64, mt0, g, stream);
 #pragma unroll
         for (int c = 0; c < BN / C::BOX_N; ++c)
-          tma_load_3d(&tmB, &full[s], sb + c * C::BOX_N * 128, kb * 64, d.n_lo + n0 + c * C::BOX_N, grp);
+          tma_load_3d_hint(&tmB, &full[s], sb + c * C::BOX_N * 128, kb * 64, d.n_lo + n0 + c * C::BOX_N, grp, keep);
       }
     }
   } else if (warp == 5) {

@@ -8,7 +8,7 @@
 
 namespace ot {
 
-constexpr uint32_t kSpinLimit = 1u << 24;  // try_wait rounds before a wait gives up
+constexpr uint32_t kSpinLimit = 1u << 20;  // try_wait rounds before a wait gives up (well over 0.1 s)
 enum : int { kErrWaitTimeout = 101, kErrSmemAlign = 102 };
 
 __device__ inline uint32_t smem_u32(const void* p) {
@@ -62,6 +62,34 @@ __device__ inline void tma_load_4d(const CUtensorMap* map, uint64_t* bar, void* 
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+// Same loads with an L2 eviction-priority hint: tensors many CTAs re-read
+// (weights, cached K/V) stay in L2 ahead of streamed activations.
+__device__ inline uint64_t l2_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ inline uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ inline void tma_load_3d_hint(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1, int c2,
+                                        uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+__device__ inline void tma_load_4d_hint(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1, int c2,
+                                        int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
       : "memory");
 }
 __device__ inline void prefetch_tmap(const CUtensorMap* map) {
