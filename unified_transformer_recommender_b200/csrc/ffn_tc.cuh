@@ -65,76 +65,6 @@ struct FfnCfg {
   static constexpr int TMEM_COLS = 512;  // D 0..255, U0 256..383, U1 384..511 (GELU output packed over U)
 };
 
-__device__ inline void tmem_st32(uint32_t taddr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-}
-
-// 32 fp32 values of row r into box `box` of a staging area of [128 rows x
-// 128 B] boxes with the 128-byte swizzle (the layout TMA reads and writes).
-__device__ inline void st_sw128_f32(uint8_t* tile, int box, int r, const float* v) {
-  uint8_t* rowp = tile + box * 16384 + r * 128;
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    *(float4*)(rowp + ((k ^ (r & 7)) << 4)) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-}
-// 128 bytes of row r of a staged box, as 32 fp32 or 64 bf16 (to fp32) values.
-__device__ inline void ld_sw128_f32(const uint8_t* tile, int box, int r, float* v) {
-  const uint8_t* rowp = tile + box * 16384 + r * 128;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float4 f = *(const float4*)(rowp + ((k ^ (r & 7)) << 4));
-    v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
-  }
-}
-__device__ inline void ld_sw128_bf16(const uint8_t* tile, int box, int r, float* v) {
-  const uint8_t* rowp = tile + box * 16384 + r * 128;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    uint4 u = *(const uint4*)(rowp + ((k ^ (r & 7)) << 4));
-    const __nv_bfloat162* h = (const __nv_bfloat162*)&u;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __bfloat1622float2(h[j]);
-      v[8 * k + 2 * j] = f.x; v[8 * k + 2 * j + 1] = f.y;
-    }
-  }
-}
-__device__ inline void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
-               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
-}
-
-// 32 bf16 values of row r into a K-major, 128-byte-swizzled operand tile:
-// columns [col0, col0 + 32) of a tile whose 64-column blocks are blk_bytes apart.
-__device__ inline void st_sw128_32(uint8_t* tile, int blk_bytes, int r, int col0, const float* v) {
-  uint8_t* rowp = tile + (col0 >> 6) * blk_bytes + r * 128;
-  const int ch0 = (col0 & 63) >> 3;
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    uint4 u;
-    __nv_bfloat162* hh = (__nv_bfloat162*)&u;
-#pragma unroll
-    for (int q2 = 0; q2 < 4; ++q2) hh[q2] = __floats2bfloat162_rn(v[q4 * 8 + 2 * q2], v[q4 * 8 + 2 * q2 + 1]);
-    *(uint4*)(rowp + (((ch0 + q4) ^ (r & 7)) << 4)) = u;
-  }
-}
-
 constexpr int kFfnThreads = 320;
 
 __global__ void __launch_bounds__(kFfnThreads, 1)

@@ -10,6 +10,11 @@
 // per thread) and apply bias, GELU, residual, the paged K/V store and the
 // RMSNorm of the finished row (when the CTA owns the whole row, BN == N).
 //
+// Plain row outputs whose rows TMA can address leave through shared memory
+// (the stage buffers are idle once the accumulator is complete) and TMA
+// stores; K/V pages and outputs that feed the in-epilogue RMSNorm are stored
+// per thread.
+//
 // Warp roles (192 threads): warps 0-3 epilogue, warp 4 TMA producer,
 // warp 5 TMEM allocator and MMA issuer.
 #pragma once
@@ -35,7 +40,8 @@ struct TcGemmCfg {
 template <int BN>
 __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmDesc d, const int a_swap) {
+                   const __grid_constant__ CUtensorMap tmOut, const GemmDesc d, const int a_swap,
+                   const int out_tma, const int out_swap) {
   using C = TcGemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -151,6 +157,10 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
         const int dm = d.kv.H * d.kv.dh;
         const int kind = n / dm, cc = n - kind * dm, head = cc / d.kv.dh, e = cc - head * d.kv.dh;
         store_bf16x32((__nv_bfloat16*)d.kv.pool + kv_off(d.kv, b, t + d.kv.pos_off, kind, head, e), v);
+      } else if (out_tma) {
+        // every MMA is done: the stage buffers stage the tile for TMA stores
+        if (d.out.f32) st_sw128_f32(smem, c0 >> 5, r, v);
+        else st_sw128_32(smem, 16384, r, c0, v);
       } else {
         store_row32(d.out, rm_off(d.out, b, t, n), v);
       }
@@ -160,6 +170,19 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
           const float q = d.out.f32 ? v[i] : __bfloat162float(__float2bfloat16_rn(v[i]));
           ss += q * q;
         }
+      }
+    }
+    if (out_tma) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (threadIdx.x == 0 && done) {
+        const int bc = d.out.f32 ? 32 : 64;
+        for (int i = 0; i < BN / bc; ++i) {
+          if (out_swap) tma_store_3d(&tmOut, smem + i * 16384, n0 + i * bc, g, mt0);
+          else tma_store_3d(&tmOut, smem + i * 16384, n0 + i * bc, mt0, g);
+        }
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       }
     }
     if (valid && d.rms.base) {
@@ -182,36 +205,6 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
 }
 
 // ------------------------------------------------------------------ host --
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-inline EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  }
-  return fn;
-}
-
-// 3-D bf16 tensor map: dims (inner, d1, d2), strides in elements for d1, d2.
-inline bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t d1, uint64_t d2,
-                         uint64_t s1, uint64_t s2, uint32_t box0, uint32_t box1, uint32_t box2) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {inner, d1, d2};
-  const cuuint64_t strides[2] = {s1 * 2, s2 * 2};
-  const cuuint32_t box[3] = {box0, box1, box2};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 inline int tc_pick_bn(const GemmDesc& d) {
   if (d.rms.base) return (d.N == 128 || d.N == 256 || d.N == 384) ? d.N : 0;
   if (d.N % 256 == 0) return 256;
@@ -220,9 +213,6 @@ inline int tc_pick_bn(const GemmDesc& d) {
   return 0;
 }
 
-inline bool rowmap_vec_ok(const RowMap& r) {
-  return ((uintptr_t)r.base % 16) == 0 && r.sb % 8 == 0 && r.st % 8 == 0 && r.sc % 8 == 0 && r.split % 32 == 0;
-}
 
 inline bool tc_gemm_supported(const GemmDesc& d) {
   if (d.K <= 0 || d.K % 64 || !tc_pick_bn(d)) return false;
@@ -239,10 +229,39 @@ inline bool tc_gemm_supported(const GemmDesc& d) {
   return encode_fn() != nullptr;
 }
 
+// TMA map over the plain output rows of a GEMM (columns [0, N)), when the
+// rows form a strided 2-D set and the whole tile fits in the stage buffers.
+inline bool make_gemm_out_tmap(CUtensorMap* map, const GemmDesc& d, int bn, int stage_bytes, int& swap) {
+  const RowMap& r = d.out;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || d.out_kind != OUT_ROWS || d.rms.base || r.split < d.N || ((uintptr_t)r.base % 16)) return false;
+  const uint64_t es = r.f32 ? 4 : 2;
+  if ((uint64_t)128 * bn * es > (uint64_t)stage_bytes) return false;
+  const uint64_t m_ext = (uint64_t)(d.m_lo + d.M), g_ext = (uint64_t)(d.g_lo + d.G);
+  uint64_t s_m, s_g;
+  if (d.mode == TILE_ROWS) { s_m = r.st; s_g = r.sb; }
+  else if (d.mode == TILE_SAMPLES) { s_m = r.sb; s_g = r.st; }
+  else {
+    if (d.fold < d.m_lo + d.M && (long long)r.sb != (long long)d.fold * r.st) return false;
+    s_m = r.st; s_g = m_ext * r.st;
+  }
+  if (g_ext == 1) s_g = m_ext * s_m;
+  swap = (g_ext > 1 && s_g < s_m) ? 1 : 0;
+  const uint32_t bc = r.f32 ? 32 : 64;
+  const cuuint64_t dims[3] = {(cuuint64_t)d.N, swap ? g_ext : m_ext, swap ? m_ext : g_ext};
+  const cuuint64_t strides[2] = {(swap ? s_g : s_m) * es, (swap ? s_m : s_g) * es};
+  const cuuint32_t box[3] = {bc, swap ? 1u : 128u, swap ? 128u : 1u};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  if (strides[0] % 16 || strides[1] % 16) return false;
+  return fn(map, r.f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, r.base, dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN>
 inline onetrans_status tc_gemm_launch_bn(const GemmDesc& d, cudaStream_t st) {
   using C = TcGemmCfg<BN>;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tout;
   const uint64_t mext = (uint64_t)d.a_mext, gext = (uint64_t)d.a_gext;
   const uint64_t s_m = (uint64_t)d.a_sm, s_g = gext > 1 ? (uint64_t)d.a_sg : mext * (uint64_t)d.a_sm;
   const int a_swap = (gext > 1 && d.a_sg < d.a_sm) ? 1 : 0;
@@ -259,8 +278,11 @@ inline onetrans_status tc_gemm_launch_bn(const GemmDesc& d, cudaStream_t st) {
       return ONETRANS_ERR_CUDA;
     attr_set = true;
   }
+  int out_swap = 0;
+  const int out_tma = make_gemm_out_tmap(&tout, d, BN, C::STAGES * C::STAGE_BYTES, out_swap) ? 1 : 0;
+  if (!out_tma) tout = ta;
   dim3 grid((unsigned)(d.N / BN), (unsigned)((d.M + 127) / 128), (unsigned)d.G);
-  gemm_tc_kernel<BN><<<grid, 192, C::SMEM, st>>>(ta, tb, d, a_swap);
+  gemm_tc_kernel<BN><<<grid, 192, C::SMEM, st>>>(ta, tb, tout, d, a_swap, out_tma, out_swap);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 

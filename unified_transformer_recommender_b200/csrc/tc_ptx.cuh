@@ -4,6 +4,7 @@
 // device status word and carries on to its teardown instead of hanging.
 #pragma once
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include "common.cuh"
 
 namespace ot {
@@ -263,6 +264,113 @@ __device__ inline void store_row32(const RowMap& r, long long off, const float* 
   } else {
     store_bf16x32((__nv_bfloat16*)r.base + off, v);
   }
+}
+
+// ------------------------------------------------ staged tiles and stores --
+__device__ inline void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+// 32 fp32 values of row r into box `box` of a staging area of [128 rows x
+// 128 B] boxes with the 128-byte swizzle (the layout TMA reads and writes).
+__device__ inline void st_sw128_f32(uint8_t* tile, int box, int r, const float* v) {
+  uint8_t* rowp = tile + box * 16384 + r * 128;
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    *(float4*)(rowp + ((k ^ (r & 7)) << 4)) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+}
+// 128 bytes of row r of a staged box, as 32 fp32 or 64 bf16 (to fp32) values.
+__device__ inline void ld_sw128_f32(const uint8_t* tile, int box, int r, float* v) {
+  const uint8_t* rowp = tile + box * 16384 + r * 128;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float4 f = *(const float4*)(rowp + ((k ^ (r & 7)) << 4));
+    v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
+  }
+}
+__device__ inline void ld_sw128_bf16(const uint8_t* tile, int box, int r, float* v) {
+  const uint8_t* rowp = tile + box * 16384 + r * 128;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint4 u = *(const uint4*)(rowp + ((k ^ (r & 7)) << 4));
+    const __nv_bfloat162* h = (const __nv_bfloat162*)&u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      v[8 * k + 2 * j] = f.x; v[8 * k + 2 * j + 1] = f.y;
+    }
+  }
+}
+__device__ inline void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+// 32 bf16 values of row r into a K-major, 128-byte-swizzled operand tile:
+// columns [col0, col0 + 32) of a tile whose 64-column blocks are blk_bytes apart.
+__device__ inline void st_sw128_32(uint8_t* tile, int blk_bytes, int r, int col0, const float* v) {
+  uint8_t* rowp = tile + (col0 >> 6) * blk_bytes + r * 128;
+  const int ch0 = (col0 & 63) >> 3;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    uint4 u;
+    __nv_bfloat162* hh = (__nv_bfloat162*)&u;
+#pragma unroll
+    for (int q2 = 0; q2 < 4; ++q2) hh[q2] = __floats2bfloat162_rn(v[q4 * 8 + 2 * q2], v[q4 * 8 + 2 * q2 + 1]);
+    *(uint4*)(rowp + (((ch0 + q4) ^ (r & 7)) << 4)) = u;
+  }
+}
+
+
+// ------------------------------------------------------- host: TMA maps --
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map: dims (inner, d1, d2), strides in elements for d1, d2.
+inline bool make_tmap_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t d1, uint64_t d2,
+                         uint64_t s1, uint64_t s2, uint32_t box0, uint32_t box1, uint32_t box2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {inner, d1, d2};
+  const cuuint64_t strides[2] = {s1 * 2, s2 * 2};
+  const cuuint32_t box[3] = {box0, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool rowmap_vec_ok(const RowMap& r) {
+  return ((uintptr_t)r.base % 16) == 0 && r.sb % 8 == 0 && r.st % 8 == 0 && r.sc % 8 == 0 && r.split % 32 == 0;
 }
 
 }  // namespace ot
