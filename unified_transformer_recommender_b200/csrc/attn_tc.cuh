@@ -250,92 +250,68 @@ __global__ void __launch_bounds__(192, 2)
       }
       const bool full = !ns_tile && (a.mode == MODE_CAUSAL ? (kbase + C::BN - 1 <= qpos_min && kbase + C::BN <= n_keys_s)
                                                           : (kbase + C::BN <= n_keys_s));
+      // the row's 128 scores; keys it may not see become -inf
+      float sv[128];
+      tmem_ld128(tS + lb, sv);
+      if (!full) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) sv[i] = (i >= lo && i < hi) ? sv[i] : -INFINITY;
+      }
+      // tile max over four independent chains
+      float mq0 = sv[0], mq1 = sv[1], mq2 = sv[2], mq3 = sv[3];
+#pragma unroll
+      for (int i = 4; i < 128; i += 4) {
+        mq0 = fmaxf(mq0, sv[i]);
+        mq1 = fmaxf(mq1, sv[i + 1]);
+        mq2 = fmaxf(mq2, sv[i + 2]);
+        mq3 = fmaxf(mq3, sv[i + 3]);
+      }
+      const float mt = fmaxf(fmaxf(mq0, mq1), fmaxf(mq2, mq3));
+      // raise the reference only when this tile passes it by more than 2^kThresh
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mt > m + kThresh) {
+        if (m != -INFINITY) {
+          alpha = ex2(m - mt);
+          rescale = true;
+        }
+        m = mt;
+      }
+      const float mref = (m == -INFINITY) ? 0.f : m;
+      float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const float p0 = ex2(sv[2 * i] - mref), p1 = ex2(sv[2 * i + 1] - mref);
+        const float p2 = ex2(sv[2 * i + 2] - mref), p3 = ex2(sv[2 * i + 3] - mref);
+        ps0 += p0;
+        ps1 += p1;
+        ps2 += p2;
+        ps3 += p3;
+        pk[i] = pack_bf16x2(p0, p1);
+        pk[i + 1] = pack_bf16x2(p2, p3);
+      }
+      l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
       // P of the previous tile must be consumed before this one overwrites it
       if (kt > 0) {
         ok = mbar_wait(p_free, (kt - 1) & 1);
         if (!ok) break;
         tc_fence_after();
       }
-      float mref = m;
-      float mx = -INFINITY;
-      if (m == -INFINITY) {
-        // no visible key seen yet: take this tile's max first
+      if (rescale) {
+        // O holds the tiles before kt (p_free was awaited): bring it to the new max
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float sv[32];
-          tmem_ld32(tS + lb + c * 32, sv);
+        for (int c = 0; c < 2; ++c) {
+          float ov[32];
+          tmem_ld32(tO + lb + c * 32, ov);
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (full || (c * 32 + i >= lo && c * 32 + i < hi)) mx = fmaxf(mx, sv[i]);
+          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+          uint32_t* ou = (uint32_t*)ov;
+          tmem_st16(tO + lb + c * 32, ou);
+          tmem_st16(tO + lb + c * 32 + 16, ou + 16);
         }
-        mref = (mx == -INFINITY) ? 0.f : mx;
       }
-      float rs = 0.f, mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(tS + lb + c * 32, sv);
-        uint32_t pk[16];
-        if (full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            mt = fmaxf(mt, sv[i]);
-            sv[i] = ex2(sv[i] - mref);
-            rs += sv[i];
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const bool vis = c * 32 + i >= lo && c * 32 + i < hi;
-            mt = vis ? fmaxf(mt, sv[i]) : mt;
-            sv[i] = vis ? ex2(sv[i] - mref) : 0.f;
-            rs += sv[i];
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(sv[2 * i], sv[2 * i + 1]);
-        tmem_st16(tP + lb + c * 16, pk);
-      }
-      if (m == -INFINITY) {
-        m = (mx == -INFINITY) ? -INFINITY : mref;
-        l = rs;
-      } else if (mt > m + kThresh) {
-        // the tile's max ran far past the reference: redo P with the new max and
-        // rescale what O and l hold (O only has tiles < kt: p_free was awaited)
-        const float m_new = mt, alpha = ex2(m - m_new);
-        rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float sv[32];
-          tmem_ld32(tS + lb + c * 32, sv);
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const bool vis = full || (c * 32 + i >= lo && c * 32 + i < hi);
-            sv[i] = vis ? ex2(sv[i] - m_new) : 0.f;
-            rs += sv[i];
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(sv[2 * i], sv[2 * i + 1]);
-          tmem_st16(tP + lb + c * 16, pk);
-        }
-        if (kt > 0) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float ov[32];
-            tmem_ld32(tO + lb + c * 32, ov);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-            uint32_t* ou = (uint32_t*)ov;
-            tmem_st16(tO + lb + c * 32, ou);
-            tmem_st16(tO + lb + c * 32 + 16, ou + 16);
-          }
-        }
-        l = l * alpha + rs;
-        m = m_new;
-      } else {
-        l += rs;
-      }
+      tmem_st64(tP + lb, pk);
       // keys past the last valid cache key may hold stale bits (P is 0 there,
       // but 0 * NaN is not): zero their V rows before P.V reads them
       if (kt == nt_s - 1 && kbase + r > kmax) {
