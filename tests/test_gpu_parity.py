@@ -252,6 +252,22 @@ def test_schedule_query_and_cache_pages_exact():
 
 # ------------------------------------------- full-size workloads, sampled --
 
+def test_forward_d384_small():
+    """The wider shape (d = 384, 4 heads of 96, FFN 1536, 16 NS tokens) at a
+    small size: 384-column GEMM tiles (W^O, QKV of 1152 = 3 x 384, the FFN
+    down-projection with the next RMSNorm) and d_h = 96 attention, 3 users x
+    (200 + 16) tokens through a 2-layer pyramid."""
+    sh = shape(n_layers=2, d=384, dff=1536, L_NS=16)
+    L_S = 200
+    pyr = linear_pyramid(L_S + sh.L_NS, sh.L_NS, 2)
+    b = build(sh, 77, "bf16", pyramid=pyr)
+    X0 = gen_normal(78, (3, L_S + sh.L_NS, sh.d), "bf16")
+    got = run_forward(b, X0)
+    for u in range(3):
+        ref = O.forward(X0[u:u + 1], b.W, sh.L_NS, sh.n_heads, EPS, pyr)[0]
+        assert rel_err(got[u], ref) <= TOL["bf16"]
+
+
 def _full(name):
     wl = WORKLOADS[name]
     b = build(wl.shape, wl.seed_weights, wl.dtype, pyramid=list(wl.pyramid) if wl.pyramid else None,
