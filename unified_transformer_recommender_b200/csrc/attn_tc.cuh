@@ -182,14 +182,16 @@ __global__ void __launch_bounds__(192, 2)
     if (lane == 0 && nt > 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, 128);
       constexpr uint32_t id_pv = idesc_bf16(128, 64, false, true);
-      const uint32_t aq = smem_u32(sQ);
+      // base descriptors of Q and of each stage's K and V tiles
+      const uint64_t dq = sdesc_k128(smem_u32(sQ));
+      const uint64_t dk0 = sdesc_k128(smem_u32(sKV)), dk1 = sdesc_k128(smem_u32(sKV + 2 * C::KV_BYTES));
+      const uint64_t dv0 = sdesc_mn128(smem_u32(sKV + C::KV_BYTES), 0);
+      const uint64_t dv1 = sdesc_mn128(smem_u32(sKV + 3 * C::KV_BYTES), 0);
       bool ok = mbar_wait(q_full, 0) && mbar_wait(&kv_full[0], 0);
       if (ok) {
         tc_fence_after();
-        const uint32_t ak = smem_u32(sKV);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16(tS, sdesc_k128(aq + k * 32), sdesc_k128(ak + k * 32), id_qk, k ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) umma_bf16(tS, desc_add(dq, k * 32), desc_add(dk0, k * 32), id_qk, k ? 1u : 0u);
         umma_commit(s_full);
       }
       for (int kt = 0; kt < nt && ok; ++kt) {
@@ -202,18 +204,18 @@ __global__ void __launch_bounds__(192, 2)
           ok = mbar_wait(&kv_full[s1], ((kt + 1) >> 1) & 1);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t ak = smem_u32(sKV + s1 * 2 * C::KV_BYTES);
+          const uint64_t dk = s1 ? dk1 : dk0;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tS, sdesc_k128(aq + k * 32), sdesc_k128(ak + k * 32), id_qk, k ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) umma_bf16(tS, desc_add(dq, k * 32), desc_add(dk, k * 32), id_qk, k ? 1u : 0u);
           umma_commit(s_full);
         }
         // O += P V: P from TMEM (8 columns = 16 keys per step), V from shared memory
         const int s = kt & 1;
-        const uint32_t av = smem_u32(sKV + s * 2 * C::KV_BYTES + C::KV_BYTES);
+        const uint64_t dv = s ? dv1 : dv0;
+        const uint32_t acc0 = kt ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ts(tO, tP + kk * 8, sdesc_mn128(av + kk * 2048, 0), id_pv, (kt | kk) ? 1u : 0u);
+          umma_bf16_ts(tO, tP + kk * 8, desc_add(dv, kk * 2048), id_pv, kk ? 1u : acc0);
         umma_commit(p_free);
         umma_commit(&kv_empty[s]);
       }

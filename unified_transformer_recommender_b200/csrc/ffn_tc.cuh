@@ -7,25 +7,28 @@
 //   h_next = RMSNorm(x_next) * g_next               (next layer's pre-norm)
 //
 // Only a, x, x_next and h_next touch HBM; x_mid and the d_ff-wide hidden
-// layer stay on chip.  TMEM holds D (256 fp32 columns: the residual rows,
-// then + W^O a = x_mid, then + W2 hidden, since both products accumulate in
-// place), two 64-column buffers U0/U1 for the up-projection of a hidden
-// chunk, and two 32-column buffers H0/H1 for the GELU output of a chunk as
-// packed bf16 pairs, which the down-projection reads as its A operand.
-// Shared memory holds the attention tile (reused for h2 as the A operand of
-// the up-projection) and a 5-stage ring of 32 KB tiles fed by TMA: first the
-// residual rows, then W^O, then W1/W2 chunk by chunk.  x_next and h_next
-// leave by TMA stores staged through the then idle shared memory.  Row
-// geometries TMA cannot express fall back to per-thread loads/stores.
+// layer stay on chip.  TMEM (512 columns) holds D (256 fp32 columns: the
+// residual rows, then + W^O a = x_mid, then + W2 hidden, since both products
+// accumulate in place) and U (256 fp32 columns: the up-projection of one
+// 256-unit hidden chunk).  Every product is a 128 x 256 tcgen05.mma, the
+// shape that runs at the tensor pipe's full rate (narrower N issue at about
+// the same cost per instruction).  Shared memory holds the attention tile
+// (reused for h2 as the A operand of the up-projection) and a 5-stage ring of
+// 32 KB tiles fed by TMA: first the residual rows, then W^O, then W1/W2
+// chunk by chunk.  x_next and h_next leave by TMA stores staged through the
+// then idle shared memory.  Row geometries TMA cannot express fall back to
+// per-thread loads/stores.
 //
-// Per hidden chunk c (64 units): up(c) -> U[c%2]; the compute warps apply
-// b1 + GELU and write H[c%2]; down(c) accumulates into D; up(c+2) follows
-// right after, so GELU of one chunk overlaps the MMAs of the next.
+// Per hidden chunk c: up(c) -> U; the compute warps apply b1 + GELU to U in
+// four blocks of 64 units, packing each block's bf16 result over its own
+// columns and signalling it at once, so down(c) (A = the packed hidden
+// block, read from TMEM) runs block by block behind the GELU; up(c+1) follows
+// once down(c) has read U.
 //
-// Warp roles (320 threads): warps 0-7 compute (two warps per row quarter:
-// warp w and w+4 share TMEM lanes 32*(w%4).. and split each row's columns,
-// exchanging row sums through shared memory), warp 8 TMA producer, warp 9
-// TMEM allocator and MMA issuer.
+// Warp roles (576 threads): warps 0-15 compute (four warps per row quarter:
+// warps w, w+4, w+8, w+12 share TMEM lanes 32*(w%4).. and split each row's
+// columns, exchanging row sums through shared memory), warp 16 TMA producer,
+// warp 17 TMEM allocator and MMA issuer.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -56,16 +59,17 @@ struct FfnIo {
 };
 
 struct FfnCfg {
-  static constexpr int D = 256, BM = 128, HC = 128;  // hidden chunk width
+  static constexpr int D = 256, BM = 128, HC = 256;  // hidden chunk width
+  static constexpr int HB = 64;                      // GELU / down-projection block of a chunk
   static constexpr int A_BYTES = BM * D * 2;        // 64 KB: attention tile, then h2
   static constexpr int STAGE = 32768;               // one ring stage
   static constexpr int STAGES = 5;
-  static constexpr int BAR_BYTES = 256 + 1024;       // barriers + per-row partial sums
+  static constexpr int BAR_BYTES = 256 + 2048;       // barriers + per-row partial sums [4][128]
   static constexpr int SMEM = A_BYTES + STAGES * STAGE + BAR_BYTES;
-  static constexpr int TMEM_COLS = 512;  // D 0..255, U0 256..383, U1 384..511 (GELU output packed over U)
+  static constexpr int TMEM_COLS = 512;  // D 0..255, U 256..511 (GELU output packed over U, block by block)
 };
 
-constexpr int kFfnThreads = 320;
+constexpr int kFfnThreads = 576;
 
 __global__ void __launch_bounds__(kFfnThreads, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmWo,
@@ -82,13 +86,13 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   uint64_t* w_empty = w_full + C::STAGES;  // [STAGES]
   uint64_t* d_full = w_empty + C::STAGES;
   uint64_t* h2_ready = d_full + 1;
-  uint64_t* u_full = h2_ready + 1;   // [2]
-  uint64_t* hid_full = u_full + 2;   // [2]
-  uint64_t* dn_done = hid_full + 2;  // [2]
-  uint64_t* d_done = dn_done + 2;
+  uint64_t* u_full = h2_ready + 1;
+  uint64_t* hid_full = u_full + 1;   // [HC / HB]: one per hidden block
+  uint64_t* dn_done = hid_full + C::HC / C::HB;
+  uint64_t* d_done = dn_done + 1;
   uint64_t* res_ready = d_done + 1;
   uint32_t* tmem_slot = (uint32_t*)(res_ready + 1);
-  float* red = (float*)((uint8_t*)bars + 256);  // [2][128] partial row sums
+  float* red = (float*)((uint8_t*)bars + 256);  // [4][128] partial row sums
 
   if (smem_u32(smem) & 1023) {
     if (threadIdx.x == 0) flag_error(kErrSmemAlign);
@@ -107,24 +111,26 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     mbar_init(a_full, 1);
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&w_full[s], 1); mbar_init(&w_empty[s], 1); }
     mbar_init(d_full, 1);
-    mbar_init(h2_ready, 256);
-    for (int i = 0; i < 2; ++i) { mbar_init(&u_full[i], 1); mbar_init(&hid_full[i], 256); mbar_init(&dn_done[i], 1); }
+    mbar_init(h2_ready, 512);
+    mbar_init(u_full, 1);
+    mbar_init(dn_done, 1);
+    for (int i = 0; i < C::HC / C::HB; ++i) mbar_init(&hid_full[i], 512);
     mbar_init(d_done, 1);
-    mbar_init(res_ready, 256);
+    mbar_init(res_ready, 512);
     fence_barrier_init();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 16 && lane == 0) {
     prefetch_tmap(&tmA); prefetch_tmap(&tmWo); prefetch_tmap(&tmW1); prefetch_tmap(&tmW2);
     if (io.res_tma) prefetch_tmap(&tmRes);
   }
-  if (warp == 9) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  if (warp == 17) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tD = tmem, tU0 = tmem + 256;
+  const uint32_t tD = tmem, tU = tmem + 256;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
@@ -150,11 +156,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
           }
         } else if (kind == 0) {   // W^O k-block j: [256 out x 64]
           tma_load_3d_hint(&tmWo, &w_full[s], dst, j * 64, 0, 0, keep);
-        } else if (kind == 1) {   // W1 chunk c, k-blocks 2j, 2j+1: [128 hidden x 64] each
-          tma_load_3d_hint(&tmW1, &w_full[s], dst, (2 * j) * 64, c * C::HC, grp, keep);
-          tma_load_3d_hint(&tmW1, &w_full[s], dst + 16384, (2 * j + 1) * 64, c * C::HC, grp, keep);
-        } else {                  // W2 chunk c, hidden k-block j: [256 out x 64 hidden]
-          tma_load_3d_hint(&tmW2, &w_full[s], dst, c * C::HC + j * 64, 0, grp, keep);
+        } else if (kind == 1) {   // W1 chunk c, k-block j: [256 hidden x 64]
+          tma_load_3d_hint(&tmW1, &w_full[s], dst, j * 64, c * C::HC, grp, keep);
+        } else {                  // W2 chunk c, hidden block j: [256 out x 64 hidden]
+          tma_load_3d_hint(&tmW2, &w_full[s], dst, c * C::HC + j * C::HB, 0, grp, keep);
         }
         ++q;
         return true;
@@ -162,100 +167,97 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       bool ok = true;
       for (int j = 0; j < RP && ok; ++j) ok = stage(3, 0, j);
       for (int j = 0; j < 4 && ok; ++j) ok = stage(0, 0, j);
-      for (int c = 0; c < 2 && c < NC && ok; ++c)
-        for (int j = 0; j < 2 && ok; ++j) ok = stage(1, c, j);
+      for (int j = 0; j < 4 && ok; ++j) ok = stage(1, 0, j);
       for (int c = 0; c < NC && ok; ++c) {
-        for (int j = 0; j < 2 && ok; ++j) ok = stage(2, c, j);
-        if (c + 2 < NC)
-          for (int j = 0; j < 2 && ok; ++j) ok = stage(1, c + 2, j);
+        for (int j = 0; j < C::HC / C::HB && ok; ++j) ok = stage(2, c, j);
+        if (c + 1 < NC)
+          for (int j = 0; j < 4 && ok; ++j) ok = stage(1, c + 1, j);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t id256 = idesc_bf16(128, 256);
-      constexpr uint32_t id128 = idesc_bf16(128, 128);
-      const uint32_t aA = smem_u32(sA), aW = smem_u32(sW);
+      const uint64_t dA = sdesc_k128(smem_u32(sA)), dW = sdesc_k128(smem_u32(sW));
       int q = RP;  // the residual stages are consumed by the compute warps
-      auto wait_stage = [&](uint32_t& base) -> bool {
+      auto wait_stage = [&](uint64_t& base) -> bool {
         const int s = q % C::STAGES;
         if (!mbar_wait(&w_full[s], (q / C::STAGES) & 1)) return false;
         tc_fence_after();
-        base = aW + s * C::STAGE;
+        base = desc_add(dW, s * C::STAGE);
         return true;
       };
       auto free_stage = [&]() { umma_commit(&w_empty[q % C::STAGES]); ++q; };
-      auto up = [&](int c) -> bool {
-        const uint32_t tU = tU0 + (c & 1) * C::HC;
-        for (int j = 0; j < 2; ++j) {
-          uint32_t wb;
+      // U = h2 W1c^T, K = 256 in four staged k-blocks
+      auto up = [&]() -> bool {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint64_t wb;
           if (!wait_stage(wb)) return false;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int kb = 2 * j + h;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_bf16(tU, sdesc_k128(aA + kb * 16384 + k * 32), sdesc_k128(wb + h * 16384 + k * 32), id128,
-                        (kb | k) ? 1u : 0u);
-          }
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(tU, desc_add(dA, j * 16384 + k * 32), desc_add(wb, k * 32), id256, (j | k) ? 1u : 0u);
           free_stage();
         }
-        umma_commit(&u_full[c & 1]);
+        umma_commit(u_full);
         return true;
       };
       bool ok = mbar_wait(a_full, 0) && mbar_wait(res_ready, 0);
       if (ok) tc_fence_after();
       // D holds the residual rows: x_mid = x + a W^O^T accumulates in place
       for (int j = 0; j < 4 && ok; ++j) {
-        uint32_t wb;
+        uint64_t wb;
         ok = wait_stage(wb);
         if (!ok) break;
+        const uint64_t da = desc_add(dA, j * 16384);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16(tD, sdesc_k128(aA + j * 16384 + k * 32), sdesc_k128(wb + k * 32), id256, 1u);
+        for (int k = 0; k < 4; ++k) umma_bf16(tD, desc_add(da, k * 32), desc_add(wb, k * 32), id256, 1u);
         free_stage();
       }
       if (ok) umma_commit(d_full);
       ok = ok && mbar_wait(h2_ready, 0);
       if (ok) tc_fence_after();
-      for (int c = 0; c < 2 && c < NC && ok; ++c) ok = up(c);
+      if (ok) ok = up();
       for (int c = 0; c < NC && ok; ++c) {
-        ok = mbar_wait(&hid_full[c & 1], (c >> 1) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        // D += H W2c^T: A = the GELU output packed over U[c%2] (16 hidden = 8 columns per step)
-        const uint32_t tH = tU0 + (c & 1) * C::HC;
-        for (int j = 0; j < 2 && ok; ++j) {
-          uint32_t wb;
+        // D += H W2c^T block by block as the GELU output appears: in block b
+        // (units 64b..64b+63) units 64b+16k..+15 are packed over U columns
+        // 64b+16k..+7, one k-step each
+        for (int b = 0; b < C::HC / C::HB && ok; ++b) {
+          ok = mbar_wait(&hid_full[b], c & 1);
+          if (!ok) break;
+          tc_fence_after();
+          uint64_t wb;
           ok = wait_stage(wb);
           if (!ok) break;
+          const uint32_t tH = tU + b * C::HB;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) umma_bf16_ts(tD, tH + j * 32 + k * 8, sdesc_k128(wb + k * 32), id256, 1u);
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_ts(tD, tH + k * 16, desc_add(wb, k * 32), id256, 1u);
           free_stage();
         }
-        umma_commit(&dn_done[c & 1]);
-        // up(c+2) overwrites U[c%2]: let down(c) finish reading it first
-        if (ok && c + 2 < NC) ok = mbar_wait(&dn_done[c & 1], (c >> 1) & 1) && up(c + 2);
+        umma_commit(dn_done);
+        // up(c+1) overwrites U: let down(c) finish reading it first
+        if (ok && c + 1 < NC) ok = mbar_wait(dn_done, c & 1) && up();
       }
       umma_commit(d_done);
     }
   } else {
     // ------------------------------------------------------------- compute
-    const int q4 = warp & 3, wg = warp >> 2;   // row quarter, column half
+    const int q4 = warp & 3, wq = warp >> 2;   // row quarter, column quarter
     const int r = q4 * 32 + lane;
     const int m = mt0 + r;
     const bool valid = m < d.m_lo + d.M;
     int b = 0, t = 0;
     if (valid) row_of_rows(d.mode, d.fold, m, g, b, t);
     const uint32_t lb = (uint32_t)(q4 * 32) << 16;
-    const int cD = wg * (C::D / 2);            // this warp's first column of a d-wide row
+    const int cD = wq * (C::D / 4);            // this warp's 64 columns of a d-wide row
     const __nv_bfloat16* gffn = (const __nv_bfloat16*)d.g_ffn;
-    // full-row sum from the two column halves of row r
+    // full-row sum from the four column quarters of row r
     auto row_sum = [&](float part) -> float {
-      red[wg * 128 + r] = part;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      const float s2 = red[r] + red[128 + r];
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      red[wq * 128 + r] = part;
+      asm volatile("bar.sync 1, 512;" ::: "memory");
+      const float s2 = (red[r] + red[128 + r]) + (red[256 + r] + red[384 + r]);
+      asm volatile("bar.sync 1, 512;" ::: "memory");
       return s2;
     };
     bool ok = true;
@@ -265,30 +267,30 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       for (int p = 0; p < RP; ++p) {
         const int s = p % C::STAGES;
         ok = ok && mbar_wait(&w_full[s], (p / C::STAGES) & 1);
-        if (ok) {
-          const uint8_t* st = sW + s * C::STAGE;
+        const uint8_t* st = sW + s * C::STAGE;
+        const int bx = wq & 1;  // box of the stage this warp moves
+        if (ok && io.res_f32 && (p & 1) == (wq >> 1)) {
+          float v[32];
+          ld_sw128_f32(st, bx, r, v);
+          tmem_st32(tD + lb + (2 * p + bx) * 32, v);
+        } else if (ok && !io.res_f32 && p == (wq >> 1)) {
           float v[64];
-          if (io.res_f32) {
-            ld_sw128_f32(st, wg, r, v);
-            tmem_st32(tD + lb + (2 * p + wg) * 32, v);
-          } else {
-            ld_sw128_bf16(st, wg, r, v);
-            tmem_st32(tD + lb + (2 * p + wg) * 64, v);
-            tmem_st32(tD + lb + (2 * p + wg) * 64 + 32, v + 32);
-          }
+          ld_sw128_bf16(st, bx, r, v);
+          tmem_st32(tD + lb + (2 * p + bx) * 64, v);
+          tmem_st32(tD + lb + (2 * p + bx) * 64 + 32, v + 32);
         }
         // the stage may be refilled once every compute thread has read it
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, 512;" ::: "memory");
         if (threadIdx.x == 0) mbar_arrive(&w_empty[s]);
       }
     } else {
-      float nxt[32];
-      if (valid) load_row32(d.res, rm_off(d.res, b, t, cD), nxt);
-      for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
+      for (int c0 = cD; c0 < cD + C::D / 4; c0 += 32) {
         float v[32];
+        if (valid) load_row32(d.res, rm_off(d.res, b, t, c0), v);
+        else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = valid ? nxt[i] : 0.f;
-        if (valid && c0 + 32 < cD + C::D / 2) load_row32(d.res, rm_off(d.res, b, t, c0 + 32), nxt);
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
         tmem_st32(tD + lb + c0, v);
       }
     }
@@ -299,86 +301,114 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     tc_fence_after();
     // D = x_mid; its RMSNorm becomes h2 in sA
     float ss = 0.f;
-    for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
       float v[32];
-      tmem_ld32(tD + lb + c0, v);
+      tmem_ld32(tD + lb + cD + h * 32, v);
 #pragma unroll
       for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
     }
-    const float rr = rsqrtf(row_sum(ss) / C::D + d.eps);
-    for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
-      float v[32], gv[32];
-      tmem_ld32(tD + lb + c0, v);
-      load_bf16x32(gffn + c0, gv);
+    {
+      const float rr = rsqrtf(row_sum(ss) / C::D + d.eps);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = v[i] * rr * gv[i];
-      st_sw128_32(sA, 16384, r, c0, v);
+      for (int h = 0; h < 2; ++h) {
+        float v[32], gv[32];
+        tmem_ld32(tD + lb + cD + h * 32, v);
+        load_bf16x32(gffn + cD + h * 32, gv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = v[i] * rr * gv[i];
+        st_sw128_32(sA, 16384, r, cD + h * 32, v);
+      }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     mbar_arrive(h2_ready);
-    // hidden chunks: b1 + GELU, packed bf16 into H[c%2]; each warp takes half
-    // of the chunk's columns
+    // hidden chunks: b1 + GELU block by block; in each 64-unit block warp wq
+    // takes units 16 wq .. 16 wq + 15 and packs them as bf16 pairs over the
+    // first 8 of the columns it read, then signals the block
     const __nv_bfloat16* b1 = (const __nv_bfloat16*)d.b1 + (long long)grp * d.b1_sg;
-    const int cH = wg * (C::HC / 2);
+    const int cH = wq * (C::HB / 4);
     for (int c = 0; c < NC; ++c) {
-      ok = ok && mbar_wait(&u_full[c & 1], (c >> 1) & 1);
+      // this chunk's b1 (bf16 pairs), fetched before the wait for up(c) so the
+      // wait covers the load latency
+      uint4 bq[C::HC / C::HB][2];
+#pragma unroll
+      for (int bb = 0; bb < C::HC / C::HB; ++bb)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) bq[bb][i] = ((const uint4*)(b1 + c * C::HC + bb * C::HB + cH))[i];
+      ok = ok && mbar_wait(u_full, c & 1);
       tc_fence_after();
-      const uint32_t tU = tU0 + (c & 1) * C::HC;
-      uint32_t pk[32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float v[32], bv[32];
-        tmem_ld32(tU + lb + cH + h * 32, v);
-        load_bf16x32(b1 + c * C::HC + cH + h * 32, bv);
+      for (int bb = 0; bb < C::HC / C::HB; ++bb) {
+        const uint32_t col = tU + lb + bb * C::HB + cH;
+        float v[16];
+        tmem_ld16(col, v);
+        const uint32_t* bu = (const uint32_t*)bq[bb];
+        uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[h * 16 + i] = pack_bf16x2(gelu_fast(v[2 * i] + bv[2 * i]), gelu_fast(v[2 * i + 1] + bv[2 * i + 1]));
+        for (int i = 0; i < 8; ++i) {
+          const float2 bf = __bfloat1622float2(*(const __nv_bfloat162*)&bu[i]);
+          pk[i] = pack_bf16x2(gelu_fast(v[2 * i] + bf.x), gelu_fast(v[2 * i + 1] + bf.y));
+        }
+        tmem_st8(col, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&hid_full[bb]);
       }
-      // the packed output overwrites U's first half: both column halves must be read first
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      tmem_st16(tU + lb + cH / 2, pk);
-      tmem_st16(tU + lb + cH / 2 + 16, pk + 16);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&hid_full[c & 1]);
     }
     // x_next = D + b2, and the next layer's RMSNorm; every MMA is done, so
     // the whole of shared memory can stage the outputs for TMA stores:
     // x_next in 8 boxes of 32 fp32 columns from offset 0, h_next in 4 boxes
     // of 64 bf16 columns from offset 128 KB
+    const __nv_bfloat16* b2 = (const __nv_bfloat16*)d.b2 + (long long)grp * d.b2_sg;
+    const __nv_bfloat16* gn = (const __nv_bfloat16*)d.g_next;
+    // this warp's 64 columns of b2 and g_next into L1 before the wait
+    if (lane < 2) asm volatile("prefetch.global.L1 [%0];" ::"l"(b2 + cD + lane * 32));
+    if (d.hout.base && lane >= 2 && lane < 4) asm volatile("prefetch.global.L1 [%0];" ::"l"(gn + cD + (lane - 2) * 32));
     ok = ok && mbar_wait(d_done, 0);
     tc_fence_after();
     uint8_t* stage_x = smem;
     uint8_t* stage_h = smem + 8 * 16384;
-    const __nv_bfloat16* b2 = (const __nv_bfloat16*)d.b2 + (long long)grp * d.b2_sg;
     ss = 0.f;
-    for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c0 = cD + h * 32;
       float v[32], bv[32];
       tmem_ld32(tD + lb + c0, v);
       load_bf16x32(b2 + c0, bv);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) { v[i] += bv[i]; ss = fmaf(v[i], v[i], ss); }
+      for (int i = 0; i < 32; ++i) {
+        v[i] += bv[i];
+        ss = fmaf(v[i], v[i], ss);
+      }
       if (io.out_tma) st_sw128_f32(stage_x, c0 >> 5, r, v);
       else if (valid && ok) store_row32(d.out, rm_off(d.out, b, t, c0), v);
     }
     if (d.hout.base) {
       const float r2 = rsqrtf(row_sum(ss) / C::D + d.eps);
-      const __nv_bfloat16* gn = (const __nv_bfloat16*)d.g_next;
-      for (int c0 = cD; c0 < cD + C::D / 2; c0 += 32) {
-        float v[32], bv[32], gv[32];
-        tmem_ld32(tD + lb + c0, v);
-        load_bf16x32(b2 + c0, bv);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c0 = cD + h * 32;
+        float v[32], gv[32];
+        if (io.out_tma) {
+          ld_sw128_f32(stage_x, c0 >> 5, r, v);  // x_next as staged above (this thread's own row)
+        } else {
+          float bv[32];
+          tmem_ld32(tD + lb + c0, v);
+          load_bf16x32(b2 + c0, bv);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += bv[i];
+        }
         load_bf16x32(gn + c0, gv);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = (v[i] + bv[i]) * r2 * gv[i];
+        for (int i = 0; i < 32; ++i) v[i] *= r2 * gv[i];
         if (io.hout_tma) st_sw128_32(stage_h, 16384, r, c0, v);
         else if (valid && ok) store_row32(d.hout, rm_off(d.hout, b, t, c0), v);
       }
     }
     if (io.out_tma || io.hout_tma) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      asm volatile("bar.sync 1, 512;" ::: "memory");
       if (threadIdx.x == 0 && ok) {
         if (io.out_tma) {
           for (int i = 0; i < 8; ++i) {
@@ -399,7 +429,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == 17) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ host --
@@ -451,7 +481,7 @@ inline onetrans_status tc_ffn_launch(const FfnDesc& d, cudaStream_t st) {
                    : make_tmap_3d(&ta, d.A, C::D, mext, gext, s_m, s_g, 64, 128, 1);
   ok = ok && make_tmap_3d(&two, d.Wo, C::D, C::D, 1, C::D, (uint64_t)C::D * C::D, 64, 256, 1);
   ok = ok && make_tmap_3d(&tw1, d.W1, C::D, d.dff, wg, C::D, wg > 1 ? (uint64_t)d.w1_sg : (uint64_t)d.dff * C::D,
-                          64, C::HC, 1);  // one k-block of a hidden chunk: [64 x 64]
+                          64, C::HC, 1);  // one k-block of a hidden chunk: [256 x 64]
   ok = ok && make_tmap_3d(&tw2, d.W2, d.dff, C::D, wg, d.dff, wg > 1 ? (uint64_t)d.w2_sg : (uint64_t)d.dff * C::D,
                           64, 256, 1);
   if (!ok) return ONETRANS_ERR_CUDA;

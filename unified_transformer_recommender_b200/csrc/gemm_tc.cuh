@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
   } else if (warp == 5) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, C::UN);
+      const uint64_t d0 = sdesc_k128(smem_u32(smem));  // stage 0's A tile
       bool ok = true;
       for (int kb = 0; kb < KB && ok; ++kb) {
         const int s = kb % C::STAGES;
@@ -102,15 +103,14 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
         ok = mbar_wait(&full[s], ph);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
-        const uint32_t sb = sa + C::A_BYTES;
+        const uint64_t da = desc_add(d0, s * C::STAGE_BYTES);
+        const uint32_t acc0 = kb ? 1u : 0u;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = sdesc_k128(sa + k * 32);
 #pragma unroll
           for (int j = 0; j < C::NSUB; ++j)
-            umma_bf16(tmem + j * C::UN, ad, sdesc_k128(sb + j * C::UN * 128 + k * 32), idesc,
-                      (kb | k) ? 1u : 0u);
+            umma_bf16(tmem + j * C::UN, desc_add(da, k * 32), desc_add(da, C::A_BYTES + j * C::UN * 128 + k * 32),
+                      idesc, k ? 1u : acc0);
         }
         umma_commit(&empty[s]);
       }
