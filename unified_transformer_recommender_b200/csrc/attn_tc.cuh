@@ -84,7 +84,8 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* p_full = bars + 6;
   uint64_t* p_free = bars + 7;
   uint64_t* o_done = bars + 8;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 9);
+  uint64_t* s_free = bars + 9;    // the softmax has read S of the current tile
+  uint32_t* tmem_slot = (uint32_t*)(bars + 10);
   int* s_pages = (int*)((uint8_t*)bars + C::BAR_BYTES);
 
   // the swizzled tiles need 1024-byte alignment; refuse to run without it
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(192, 2)
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
     mbar_init(o_done, 1);
+    mbar_init(s_free, 128);
     fence_barrier_init();
   }
   if (warp == 4) {
@@ -195,13 +197,11 @@ __global__ void __launch_bounds__(192, 2)
         umma_commit(s_full);
       }
       for (int kt = 0; kt < nt && ok; ++kt) {
-        // P of tile kt is in TMEM and S of tile kt has been read
-        ok = mbar_wait(p_full, kt & 1);
-        if (!ok) break;
-        tc_fence_after();
+        // S of tile kt has been read into registers: S of tile kt+1 may
+        // overwrite it while the softmax of tile kt runs
         if (kt + 1 < nt) {
           const int s1 = (kt + 1) & 1;
-          ok = mbar_wait(&kv_full[s1], ((kt + 1) >> 1) & 1);
+          ok = mbar_wait(s_free, kt & 1) && mbar_wait(&kv_full[s1], ((kt + 1) >> 1) & 1);
           if (!ok) break;
           tc_fence_after();
           const uint64_t dk = s1 ? dk1 : dk0;
@@ -209,6 +209,10 @@ __global__ void __launch_bounds__(192, 2)
           for (int k = 0; k < 4; ++k) umma_bf16(tS, desc_add(dq, k * 32), desc_add(dk, k * 32), id_qk, k ? 1u : 0u);
           umma_commit(s_full);
         }
+        // P of tile kt is in TMEM
+        ok = mbar_wait(p_full, kt & 1);
+        if (!ok) break;
+        tc_fence_after();
         // O += P V: P from TMEM (8 columns = 16 keys per step), V from shared memory
         const int s = kt & 1;
         const uint64_t dv = s ? dv1 : dv0;
@@ -255,6 +259,9 @@ __global__ void __launch_bounds__(192, 2)
       // the row's 128 scores; keys it may not see become -inf
       float sv[128];
       tmem_ld128(tS + lb, sv);
+      // S is in registers: release its TMEM columns to the next tile's Q K^T
+      tc_fence_before();
+      mbar_arrive(s_free);
       if (!full) {
 #pragma unroll
         for (int i = 0; i < 128; ++i) sv[i] = (i >= lo && i < hi) ? sv[i] : -INFINITY;
