@@ -52,7 +52,9 @@ struct AttnCfg {
   static constexpr int Q_BYTES = BM * DH * 2;     // 16 KB
   static constexpr int KV_BYTES = BN * DH * 2;    // 16 KB (one of K or V)
   static constexpr int PAGE_BYTES = 64 * DH * 2;  // one 64-token page of one head
-  static constexpr int STAGES = 2;
+  // three K/V stages: the load of tile kt+1 may start while P.V of tile kt-1
+  // still reads its stage (two CTAs of 115 KB share an SM's 228 KB)
+  static constexpr int STAGES = 3;
   static constexpr int BAR_BYTES = 128;
   static constexpr int MAX_PAGES = 128;           // page ids cached in shared memory (8192 keys)
   static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + BAR_BYTES + MAX_PAGES * 4;
@@ -78,14 +80,14 @@ __global__ void __launch_bounds__(192, 2)
   uint8_t* sKV = sQ + C::Q_BYTES;  // [stage][K|V][128 keys][64]
   uint64_t* bars = (uint64_t*)(sKV + C::STAGES * 2 * C::KV_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* p_free = bars + 7;
-  uint64_t* o_done = bars + 8;
-  uint64_t* s_free = bars + 9;    // the softmax has read S of the current tile
-  uint32_t* tmem_slot = (uint32_t*)(bars + 10);
+  uint64_t* kv_full = bars + 1;                // [STAGES]
+  uint64_t* kv_empty = kv_full + C::STAGES;    // [STAGES]
+  uint64_t* s_full = kv_empty + C::STAGES;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* p_free = s_full + 2;
+  uint64_t* o_done = s_full + 3;
+  uint64_t* s_free = s_full + 4;               // the softmax has read S of the current tile
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 5);
   int* s_pages = (int*)((uint8_t*)bars + C::BAR_BYTES);
 
   // the swizzled tiles need 1024-byte alignment; refuse to run without it
@@ -121,8 +123,7 @@ __global__ void __launch_bounds__(192, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(&kv_full[0], 1); mbar_init(&kv_full[1], 1);
-    mbar_init(&kv_empty[0], 1); mbar_init(&kv_empty[1], 1);
+    for (int i = 0; i < C::STAGES; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
     mbar_init(s_full, 1);
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
@@ -157,8 +158,8 @@ __global__ void __launch_bounds__(192, 2)
       if (a.mode == MODE_CAUSAL) tma_load_3d_hint(&tmQ, q_full, sQ, h * C::DH, row0, b, stream);
       else tma_load_3d_hint(&tmQ, q_full, sQ, h * C::DH, row0, 0, stream);
       for (int kt = 0; kt < nt; ++kt) {
-        const int s = kt & 1;
-        if (kt >= 2 && !mbar_wait(&kv_empty[s], ((kt >> 1) - 1) & 1)) break;
+        const int s = kt % C::STAGES;
+        if (kt >= C::STAGES && !mbar_wait(&kv_empty[s], ((kt / C::STAGES) - 1) & 1)) break;
         mbar_expect_tx(&kv_full[s], 2 * C::KV_BYTES);
         uint8_t* sk = sKV + s * 2 * C::KV_BYTES;
         uint8_t* sv = sk + C::KV_BYTES;
@@ -186,9 +187,8 @@ __global__ void __launch_bounds__(192, 2)
       constexpr uint32_t id_pv = idesc_bf16(128, 64, false, true);
       // base descriptors of Q and of each stage's K and V tiles
       const uint64_t dq = sdesc_k128(smem_u32(sQ));
-      const uint64_t dk0 = sdesc_k128(smem_u32(sKV)), dk1 = sdesc_k128(smem_u32(sKV + 2 * C::KV_BYTES));
+      const uint64_t dk0 = sdesc_k128(smem_u32(sKV));                    // stage s: + s * 2 * KV_BYTES
       const uint64_t dv0 = sdesc_mn128(smem_u32(sKV + C::KV_BYTES), 0);
-      const uint64_t dv1 = sdesc_mn128(smem_u32(sKV + 3 * C::KV_BYTES), 0);
       bool ok = mbar_wait(q_full, 0) && mbar_wait(&kv_full[0], 0);
       if (ok) {
         tc_fence_after();
@@ -200,11 +200,11 @@ __global__ void __launch_bounds__(192, 2)
         // S of tile kt has been read into registers: S of tile kt+1 may
         // overwrite it while the softmax of tile kt runs
         if (kt + 1 < nt) {
-          const int s1 = (kt + 1) & 1;
-          ok = mbar_wait(s_free, kt & 1) && mbar_wait(&kv_full[s1], ((kt + 1) >> 1) & 1);
+          const int s1 = (kt + 1) % C::STAGES;
+          ok = mbar_wait(s_free, kt & 1) && mbar_wait(&kv_full[s1], ((kt + 1) / C::STAGES) & 1);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t dk = s1 ? dk1 : dk0;
+          const uint64_t dk = desc_add(dk0, s1 * 2 * C::KV_BYTES);
 #pragma unroll
           for (int k = 0; k < 4; ++k) umma_bf16(tS, desc_add(dq, k * 32), desc_add(dk, k * 32), id_qk, k ? 1u : 0u);
           umma_commit(s_full);
@@ -214,8 +214,8 @@ __global__ void __launch_bounds__(192, 2)
         if (!ok) break;
         tc_fence_after();
         // O += P V: P from TMEM (8 columns = 16 keys per step), V from shared memory
-        const int s = kt & 1;
-        const uint64_t dv = s ? dv1 : dv0;
+        const int s = kt % C::STAGES;
+        const uint64_t dv = desc_add(dv0, s * 2 * C::KV_BYTES);
         const uint32_t acc0 = kt ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(192, 2)
       // keys past the last valid cache key may hold stale bits (P is 0 there,
       // but 0 * NaN is not): zero their V rows before P.V reads them
       if (kt == nt_s - 1 && kbase + r > kmax) {
-        uint4* vrow = (uint4*)(sKV + (kt & 1) * 2 * C::KV_BYTES + C::KV_BYTES + r * 128);
+        uint4* vrow = (uint4*)(sKV + (kt % C::STAGES) * 2 * C::KV_BYTES + C::KV_BYTES + r * 128);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) vrow[ch] = make_uint4(0, 0, 0, 0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
