@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_persist.cuh"
 #include "attn_tc.cuh"
 #include "ffn_tc.cuh"
 
@@ -220,6 +221,10 @@ static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, c
   if (cdiv(d.M, 64) > 65535 || d.G > 65535) return ONETRANS_ERR_SHAPE;
   ProfScope prof(kind, 2.0 * d.M * d.G * (double)d.N * d.K, gemm_bytes(m, d), st);
   if (m->bf16 && g_policy == 0 && tc_gemm_supported(d)) {
+    if (tc_persist_supported(d)) {
+      const onetrans_status r = tc_persist_launch(d, st);
+      if (r != ONETRANS_ERR_UNSUPPORTED) return r;
+    }
     return tc_gemm_launch(d, st);
   }
   dim3 grid((unsigned)cdiv(d.N, 64), (unsigned)cdiv(d.M, 64), (unsigned)d.G);
