@@ -296,7 +296,25 @@ static onetrans_status rms_flat(const onetrans_model* m, const void* src, bool s
   d.out = src_f32 ? rmap32(src, 0, m->d) : rmap(src, 0, m->d);
   d.rms = rmap(dst, 0, m->d);
   d.gamma = gamma;
-  return launch_rms<T>(d, st);
+  const int ch = m->d / 128;
+  const bool aligned = ((uintptr_t)src % 16 == 0) && ((uintptr_t)dst % 16 == 0) && ((uintptr_t)gamma % 16 == 0);
+  if (rows <= 0 || m->d % 128 || ch < 1 || ch > 4 || !aligned) return launch_rms<T>(d, st);
+  ProfScope prof(PK_RMSNORM, 0.0, (double)rows * m->d * (sizeof(T) + (src_f32 ? 4 : sizeof(T))), st);
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  T* y = (T*)dst;
+  const T* gm = (const T*)gamma;
+  const float eps = m->cfg.rms_eps;
+#define OT_RMS_FLAT(CH)                                                                                   \
+  if (src_f32) rms_flat_kernel<T, float, CH><<<blocks, 256, 0, st>>>((const float*)src, y, gm, rows, eps); \
+  else rms_flat_kernel<T, T, CH><<<blocks, 256, 0, st>>>((const T*)src, y, gm, rows, eps);
+  switch (ch) {
+    case 1: OT_RMS_FLAT(1) break;
+    case 2: OT_RMS_FLAT(2) break;
+    case 3: OT_RMS_FLAT(3) break;
+    default: OT_RMS_FLAT(4) break;
+  }
+#undef OT_RMS_FLAT
+  return last_launch();
 }
 
 // ------------------------------------------------------------ block tail --

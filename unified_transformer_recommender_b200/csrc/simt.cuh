@@ -95,6 +95,66 @@ __global__ void rms_rows_kernel(GemmDesc d) {
   }
 }
 
+// RMSNorm of contiguous rows of D = 128 CH elements: dst = src * (mean(src^2)
+// + eps)^-1/2 * gamma.  One warp per row, the row held in registers; each
+// warp-wide access covers 128 consecutive elements (lane l: elements 4l ..
+// 4l+3 of the chunk), so every byte is read and written once, coalesced.
+template <typename T>
+__device__ inline void load4(const T* p, float* v);
+template <>
+__device__ inline void load4<float>(const float* p, float* v) {
+  const float4 f = *(const float4*)p;
+  v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
+template <>
+__device__ inline void load4<__nv_bfloat16>(const __nv_bfloat16* p, float* v) {
+  const uint2 u = *(const uint2*)p;
+  const float2 a = __bfloat1622float2(*(const __nv_bfloat162*)&u.x), b = __bfloat1622float2(*(const __nv_bfloat162*)&u.y);
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+template <typename T>
+__device__ inline void store4(T* p, const float* v);
+template <>
+__device__ inline void store4<float>(float* p, const float* v) {
+  *(float4*)p = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+__device__ inline void store4<__nv_bfloat16>(__nv_bfloat16* p, const float* v) {
+  uint2 u;
+  *(__nv_bfloat162*)&u.x = __floats2bfloat162_rn(v[0], v[1]);
+  *(__nv_bfloat162*)&u.y = __floats2bfloat162_rn(v[2], v[3]);
+  *(uint2*)p = u;
+}
+template <typename T, typename S, int CH>
+__global__ void __launch_bounds__(256) rms_flat_kernel(const S* __restrict__ src, T* __restrict__ dst,
+                                                       const T* __restrict__ gamma, long long rows, float eps) {
+  constexpr int D = CH * 128;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const S* x = src + row * D + lane * 4;
+  float v[CH][4];
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    load4<S>(x + c * 128, v[c]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ss = fmaf(v[c][i], v[c][i], ss);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = rsqrtf(ss / D + eps);
+  T* y = dst + row * D + lane * 4;
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    float gv[4];
+    load4<T>(gamma + c * 128 + lane * 4, gv);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[c][i] *= r * gv[i];
+    store4<T>(y + c * 128, v[c]);
+  }
+}
+
 // ------------------------------------------------------ causal attention --
 constexpr int KT = 32;  // keys staged in shared memory per step
 // Query t of batch b (key position p = q_pos0 + t) attends to keys 0..p of
