@@ -199,6 +199,167 @@ class KVServing:
         self.step()
         self.out_pin.copy_(self.out, non_blocking=True)
 
+    metric, unit = METRIC, UNIT
+
+    def config(self, ws):
+        return {"workload": "kv_serving: auto-split + Stage I + Stage II; 6 layers d=256 4 heads FFN 1024, "
+                            f"pyramid queries 1190->12 (linear), {self.U} users x 1178 S tokens, {self.C} "
+                            "candidates/user, 12 NS tokens from 512 features", "users_per_gpu": self.U,
+                "candidates_per_gpu": self.units, "parallelism": f"users sharded over {ws} GPU(s), no collective",
+                "l2": "512 MB buffer written between timed steps (not timed)"}
+
+    def prepare(self, n_steps: int):
+        pass
+
+    def oracle(self):
+        return oracle_sample()
+
+
+class Append:
+    """Cross-request append for U users (non-pyramid 6 x 256, 1178 cached S
+    tokens each): tokenize dL = 16 new events, append their K/V to every
+    layer's cache, then auto-split and score C candidates per user against
+    the extended cache.  Each step starts from a 1178-token cache: every step
+    gets its own cache, encoded by Stage I before anything is timed (one
+    cache is 1.9 GB at 256 users, so this workload caps its step counts)."""
+
+    max_steps, max_warmup = 10, 3
+
+    metric = "users appended (dL=16 events) and their candidates scored per second on 1 B200"
+    unit = "users/s"
+
+    def __init__(self, rank: int, users: int = 0, cands: int = 0):
+        import torch
+        import unified_transformer_recommender_b200 as ot
+        from onetrans_synth import WORKLOADS, gen_normal, make_weights, random_types
+        self.ot, self.torch = ot, torch
+        wl = WORKLOADS["append"]
+        self.wl, sh = wl, wl.shape
+        self.U, self.C, self.dL = users or wl.users, cands or wl.cands, wl.dL
+        W = make_weights(sh, wl.seed_weights, wl.dtype, event_dim=wl.event_dim)
+        self.model = ot.model_from_arrays(sh, W, pyramid_q=None, mode=ot.BF16, event_dim=wl.event_dim)
+        seed = wl.seed_inputs + 7919 * rank
+        dev = torch.device("cuda")
+        self.S = torch.from_numpy(gen_normal(seed, (self.U, wl.L_S, sh.d), "bf16")).to(dev, torch.bfloat16)
+        self.ev_h = gen_normal(seed + 200, (self.U, self.dL, wl.event_dim), "bf16")
+        self.F_h = gen_normal(seed + 100, (self.U * self.C, sh.ns_feat), "bf16")
+        self.ev = torch.from_numpy(self.ev_h).to(dev, torch.bfloat16)
+        self.ty = torch.from_numpy(random_types(seed + 300, (self.U, self.dL), sh.n_types)).to(dev)
+        self.F = torch.from_numpy(self.F_h).to(dev, torch.bfloat16)
+        self.ev_pin = torch.from_numpy(self.ev_h).to(torch.bfloat16).pin_memory()
+        self.F_pin = torch.from_numpy(self.F_h).to(torch.bfloat16).pin_memory()
+        m = self.model
+        self.caches, self.k = [], 0
+        self.slots = list(range(self.U))
+        self.offs = [u * self.C for u in range(self.U + 1)]
+        self.ns = torch.empty(self.U * self.C, sh.L_NS, sh.d, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(self.U * self.C, sh.L_NS, sh.d, dtype=torch.float32, device=dev)
+        self.out_pin = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        self.ws_1 = m.workspace(ot.OP_STAGE1, self.U, wl.L_S)
+        self.ws_ap = m.workspace(ot.OP_APPEND, self.U, self.dL)
+        self.ws_a = m.workspace(ot.OP_AUTOSPLIT, self.U * self.C)
+        self.ws_2 = m.workspace(ot.OP_STAGE2, self.U * self.C, wl.L_S + self.dL)
+        self.units = self.U
+        self.h2d = self.ev_h.size * 2 + self.F_h.size * 2
+        self.d2h = self.out.numel() * 4
+
+    def config(self, ws):
+        return {"workload": f"append: non-pyramid 6 layers d=256 4 heads FFN 1024, {self.U} users x 1178 cached "
+                            f"S tokens, append dL={self.dL} events (64-wide, 3 behavior types), then "
+                            f"{self.C} candidates/user (12 NS tokens from 512 features) scored over 1194 keys",
+                "users_per_gpu": self.U, "candidates_per_gpu": self.U * self.C,
+                "parallelism": f"users sharded over {ws} GPU(s), no collective",
+                "l2": "512 MB buffer written between timed steps (not timed)"}
+
+    def prepare(self, n_steps: int):
+        """One Stage I-encoded cache per step to come (untimed)."""
+        ot = self.ot
+        for _ in range(n_steps):
+            c = ot.Cache(self.model, self.U, self.wl.L_S + self.dL)
+            ot.onetrans_stage1_encode(self.model, c, self.slots, self.S, self.ws_1)
+            self.caches.append(c)
+        self.torch.cuda.synchronize()
+
+    def step(self, ev_mid=None):
+        ot, m = self.ot, self.model
+        cache = self.caches[self.k]
+        self.k += 1
+        ot.onetrans_cache_append(m, cache, self.slots, self.ev, self.ty, self.ws_ap)
+        if ev_mid is not None:
+            ev_mid.record()
+        ot.onetrans_tokenize_autosplit(m, self.F, self.ns, self.ws_a)
+        ot.onetrans_stage2_score(m, cache, self.slots, self.offs, self.ns, self.out, self.ws_2)
+
+    def e2e_step(self):
+        self.ev.copy_(self.ev_pin, non_blocking=True)
+        self.F.copy_(self.F_pin, non_blocking=True)
+        self.step()
+        self.out_pin.copy_(self.out, non_blocking=True)
+
+    def oracle(self):
+        return oracle_sample_append(self.U, self.C)
+
+
+class Forward:
+    """One-pass forward of B samples through the stack (onetrans_forward):
+    s_forward = 6 x 256, 64 samples of 1178 + 12 tokens, pyramid 1190 -> 12;
+    l_forward = 8 x 384, 256 samples of 2048 + 16 tokens, pyramid 2064 -> 16."""
+
+    unit = "samples/s"
+
+    def __init__(self, name: str, rank: int, users: int = 0):
+        import torch
+        import unified_transformer_recommender_b200 as ot
+        from onetrans_synth import WORKLOADS, gen_normal, make_weights
+        self.ot, self.torch, self.name = ot, torch, name
+        wl = WORKLOADS[name]
+        self.wl, sh = wl, wl.shape
+        self.U = users or wl.users
+        self.metric = f"samples/sec of the one-pass forward ({name}) on 1 B200"
+        W = make_weights(sh, wl.seed_weights, wl.dtype)
+        self.model = ot.model_from_arrays(sh, W, pyramid_q=list(wl.pyramid), mode=ot.BF16)
+        dev = torch.device("cuda")
+        self.X_h = gen_normal(wl.seed_inputs + 7919 * rank, (self.U, wl.L0, sh.d), "bf16")
+        self.X = torch.from_numpy(self.X_h).to(dev, torch.bfloat16)
+        self.X_pin = torch.from_numpy(self.X_h).to(torch.bfloat16).pin_memory()
+        sched = self.model.schedule(wl.L_S)
+        self.out = torch.empty(self.U, sched[-1], sh.d, dtype=torch.float32, device=dev)
+        self.out_pin = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        self.ws = self.model.workspace(ot.OP_FORWARD, self.U, wl.L_S)
+        self.units = self.U
+        self.h2d = self.X_h.size * 2
+        self.d2h = self.out.numel() * 4
+
+    def config(self, ws):
+        sh = self.wl.shape
+        return {"workload": f"{self.name}: {sh.n_layers} layers d={sh.d} {sh.n_heads} heads FFN {sh.d_ff}, "
+                            f"{self.U} samples x ({self.wl.L_S} S + {sh.L_NS} NS tokens), pyramid "
+                            f"{self.wl.pyramid[0]}->{self.wl.pyramid[-1]} (linear)",
+                "samples_per_gpu": self.U, "parallelism": f"samples sharded over {ws} GPU(s), no collective",
+                "l2": "512 MB buffer written between timed steps (not timed)"}
+
+    def prepare(self, n_steps: int):
+        pass
+
+    def step(self, ev_mid=None, X=None):
+        self.ot.onetrans_forward(self.model, self.X if X is None else X, self.out, self.ws)
+
+    def e2e_step(self):
+        self.X.copy_(self.X_pin, non_blocking=True)
+        self.step()
+        self.out_pin.copy_(self.out, non_blocking=True)
+
+    def oracle(self):
+        return oracle_sample_forward(self.name, self.U)
+
+
+def make_workload(name: str, rank: int, users: int = 0, cands: int = 0):
+    if name == "kv_serving":
+        return KVServing(rank, users=users, cands=cands)
+    if name == "append":
+        return Append(rank, users=users, cands=cands)
+    return Forward(name, rank, users=users)
+
 
 # ------------------------------------------------------------- CPU oracle
 
@@ -231,6 +392,58 @@ def oracle_sample(n_cands: int = 160, seed_shift: int = 0):
             f"candidates ({per_cand * 1e3:.1f} ms each), extrapolated linearly to {wl.users} users x "
             f"{wl.cands} candidates ({step_s:.0f} s per step)")
     return wl.users * wl.cands / step_s, desc, cores, t2 - t0
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample_append(users: int, cands: int, n_cands: int = 16):
+    """fp64 oracle on 1 user's append (tokenize dL events, extend every
+    layer's K/V) plus n_cands candidates' auto-split and Stage II, extrapolated
+    linearly to users x cands; returns (users/s, description, threads, s)."""
+    from onetrans_synth import WORKLOADS, gen_normal, make_weights, random_types
+    from oracle import onetrans as O
+    wl = WORKLOADS["append"]
+    sh = wl.shape
+    W = make_weights(sh, wl.seed_weights, "bf16", event_dim=wl.event_dim)
+    S = gen_normal(wl.seed_inputs, (1, wl.L_S, sh.d), "bf16")
+    ev = gen_normal(wl.seed_inputs + 200, (1, wl.dL, wl.event_dim), "bf16")
+    ty = random_types(wl.seed_inputs + 300, (1, wl.dL), sh.n_types)
+    F = gen_normal(wl.seed_inputs + 100, (n_cands, sh.ns_feat), "bf16")
+    kv0 = O.stage1(S[0], W, sh.L_NS, sh.n_heads, sh.eps)
+    t0 = time.perf_counter()
+    kv = O.append(kv0, O.tokenize_events(ev[0], ty[0], W), W, sh.n_heads, sh.eps)
+    t1 = time.perf_counter()
+    ns = O.autosplit(F, W, sh.L_NS)
+    for c in range(n_cands):
+        O.stage2(kv, ns[c], W, sh.n_heads, sh.eps)
+    t2 = time.perf_counter()
+    per_user, per_cand = t1 - t0, (t2 - t1) / n_cands
+    step_s = users * per_user + users * cands * per_cand
+    desc = (f"oracle fp64: append of 1 user ({per_user:.2f} s) + auto-split and Stage II of {n_cands} candidates "
+            f"({per_cand * 1e3:.1f} ms each), extrapolated linearly to {users} users x {cands} candidates")
+    return users / step_s, desc, _oracle_threads(), t2 - t0
+
+
+def oracle_sample_forward(name: str, samples: int):
+    """fp64 oracle forward of 1 sample of the workload; returns (samples/s,
+    description, threads, s)."""
+    from onetrans_synth import WORKLOADS, gen_normal, make_weights
+    from oracle import onetrans as O
+    wl = WORKLOADS[name]
+    sh = wl.shape
+    W = make_weights(sh, wl.seed_weights, "bf16")
+    X = gen_normal(wl.seed_inputs, (1, wl.L0, sh.d), "bf16")
+    t0 = time.perf_counter()
+    O.forward(X, W, sh.L_NS, sh.n_heads, sh.eps, list(wl.pyramid))
+    t1 = time.perf_counter()
+    desc = f"oracle fp64: forward of 1 sample ({t1 - t0:.2f} s); the batch of {samples} scales linearly"
+    return 1.0 / (t1 - t0), desc, _oracle_threads(), t1 - t0
 
 
 def run_reference(args, rank):
@@ -271,9 +484,13 @@ def main():
         torch.cuda.set_device(0)
     import unified_transformer_recommender_b200 as ot
 
-    if args.workload != "kv_serving":
-        raise SystemExit("bench.py times the kv_serving workload; other workloads: tests/")
-    wk = KVServing(rank, users=args.users, cands=args.cands)
+    wk = make_workload(args.workload, rank, users=args.users, cands=args.cands)
+    if hasattr(wk, "max_steps"):
+        args.steps = min(args.steps, wk.max_steps)
+        args.warmup = min(max(args.warmup, 3), wk.max_warmup)
+    e2e_steps = max(3, args.steps // 4)
+    wk.prepare(args.warmup + args.steps + 2 + e2e_steps)
+    mid = {"kv_serving": "stage1", "append": "append"}.get(args.workload)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")   # > 126 MB L2
     st = torch.cuda.current_stream()
 
@@ -303,17 +520,15 @@ def main():
     prof = ot.onetrans_profile_read()
     ot.onetrans_profile_enable(False)
     step_ms = [a.elapsed_time(c) for a, _, c in evs]
-    s1_ms = [a.elapsed_time(b) for a, b, _ in evs]
     total_ms = max_over_ranks(sum(step_ms))
-    s1_total = max_over_ranks(sum(s1_ms))
     value = wk.units * args.steps * ws / (total_ms / 1e3)
-    users_per_s = wk.U * args.steps * ws / (s1_total / 1e3)
+    if mid:
+        s1_total = max_over_ranks(sum(a.elapsed_time(b) for a, b, _ in evs))
 
     # ---- end to end through the public API, host buffers
     for _ in range(2):
         wk.e2e_step()
     torch.cuda.synchronize()
-    e2e_steps = max(3, args.steps // 4)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -350,26 +565,25 @@ def main():
                for k, v in sorted(prof.items(), key=lambda kv: -kv[1]["ms"])}
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "kv_serving: auto-split + Stage I + Stage II; 6 layers d=256 4 heads FFN 1024, "
-                               f"pyramid queries 1190->12 (linear), {wk.U} users x 1178 S tokens, {wk.C} "
-                               "candidates/user, 12 NS tokens from 512 features", "users_per_gpu": wk.U,
-                   "candidates_per_gpu": wk.units, "parallelism": f"users sharded over {ws} GPU(s), no collective",
-                   "l2": "512 MB buffer written between timed steps (not timed)"},
-        "users_per_s": users_per_s,
-        "stage1_ms_per_step": s1_total / args.steps,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wk.h2d, "d2h_bytes_per_step": wk.d2h},
+        "metric": wk.metric, "value": value, "unit": wk.unit, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": wk.config(ws),
+    }
+    if args.workload == "kv_serving":
+        line["users_per_s"] = wk.U * args.steps * ws / (s1_total / 1e3)
+    if mid:
+        line[f"{mid}_ms_per_step"] = s1_total / args.steps
+    line.update({
+        "e2e": {"value": e2e_value, "unit": wk.unit, "h2d_bytes_per_step": wk.h2d, "d2h_bytes_per_step": wk.d2h},
         "gpu_launches": int(sum(v["launches"] for v in prof.values())),
         "roofline": roof,
         "kernels": kernels,
         "clocks": clk,
         "wall_s_timed": wall,
-    }
+    })
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not (args.users or args.cands):
-        v, desc, cores, secs = oracle_sample()
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+        v, desc, cores, secs = wk.oracle()
+        line["cpu_baseline"] = {"value": v, "unit": wk.unit, "cores": cores, "kind": "oracle", "sample": desc,
                                 "seconds": round(secs, 1)}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -759,11 +759,22 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
   }
   w.emb = m->type_emb; w.n_types = m->cfg.n_behaviors; w.e_dim = m->cfg.event_dim; w.d = d;
   const size_t smem = (size_t)(w.e_dim + d) * sizeof(float);
-  ProfScope prof_tok(PK_TOKENIZE, 2.0 * R * ((double)w.e_dim * d + (double)d * d),
-                     (double)R * (w.e_dim * m->es + d * 4), st);
-  event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>((const T*)events, types, dL, w,
-                                                                         rmap32(xa, (long long)dL * d, d));
-  OT_TRY(last_launch());
+  if (R > 0x7fffffff) return ONETRANS_ERR_SHAPE;
+  {
+    // the scope of the profiling record is the tokenizer launch alone
+    ProfScope prof_tok(PK_TOKENIZE, 2.0 * R * ((double)w.e_dim * d + (double)d * d),
+                       (double)R * (w.e_dim * m->es + d * 4), st);
+    bool w_aligned = true;
+    for (int t = 0; t < w.n_types; ++t)
+      w_aligned = w_aligned && (uintptr_t)w.W1[t] % 16 == 0 && (uintptr_t)w.W2[t] % 16 == 0;
+    if (d == kEvD && w.e_dim <= kEvEmax && w.e_dim % 8 == 0 && w_aligned)
+      event_tokenize_tile_kernel<T><<<(unsigned)cdiv(R, kEvBlock), kEvD, 0, st>>>(
+          (const T*)events, types, (int)R, dL, w, rmap32(xa, (long long)dL * d, d));
+    else
+      event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>(
+          (const T*)events, types, dL, w, rmap32(xa, (long long)dL * d, d));
+    OT_TRY(last_launch());
+  }
   OT_TRY(rms_flat<T>(m, xa, true, h, R, m->g_attn[0], st));
   const void* x_in = xa;
   for (int n = 0; n < m->NL; ++n) {

@@ -344,4 +344,96 @@ __global__ void event_tokenize_kernel(const T* ev, const int* types, int dL, Eve
   }
 }
 
+// The same tokenizer for d = 256 and e_dim <= 96, 32 events per CTA: the
+// events' inputs and hidden rows sit in shared memory, each thread owns one
+// output column and streams its weight row once per type while updating the
+// 32 events' accumulators from broadcast shared-memory reads.  Every type's
+// MLP is evaluated for every event of the CTA and the event keeps its own
+// type's result (n_types is small), so there is no data-dependent control flow.
+constexpr int kEvBlock = 32, kEvD = 256, kEvEmax = 96;
+// 8 consecutive weights (16-byte aligned) as fp32
+__device__ inline void load8(const __nv_bfloat16* p, float* v) {
+  const uint4 u = *(const uint4*)p;
+  const __nv_bfloat162* h = (const __nv_bfloat162*)&u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ inline void load8(const float* p, float* v) {
+  const float4 a = *(const float4*)p, b = *(const float4*)(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+// acc[j] += sum_{i < 8} wv[i] * x[j][i0 + i] over the CTA's events
+template <int LD>
+__device__ inline void ev_fma8(float* acc, const float* wv, const float (*x)[LD], int i0) {
+#pragma unroll
+  for (int j = 0; j < kEvBlock; ++j) {
+    const float4 a = *(const float4*)&x[j][i0], b = *(const float4*)&x[j][i0 + 4];
+    float s = acc[j];
+    s = fmaf(wv[0], a.x, s); s = fmaf(wv[1], a.y, s); s = fmaf(wv[2], a.z, s); s = fmaf(wv[3], a.w, s);
+    s = fmaf(wv[4], b.x, s); s = fmaf(wv[5], b.y, s); s = fmaf(wv[6], b.z, s); s = fmaf(wv[7], b.w, s);
+    acc[j] = s;
+  }
+}
+template <typename T>
+__global__ void __launch_bounds__(256) event_tokenize_tile_kernel(const T* ev, const int* types, int R, int dL,
+                                                                  EventMLP w, RowMap out) {
+  __shared__ __align__(16) float se[kEvBlock][kEvEmax];
+  __shared__ __align__(16) float shid[kEvBlock][kEvD];
+  __shared__ int sty[kEvBlock];
+  const int r0 = blockIdx.x * kEvBlock;
+  const int k = threadIdx.x;
+  for (int idx = threadIdx.x; idx < kEvBlock * w.e_dim; idx += blockDim.x) {
+    const int j = idx / w.e_dim, i = idx - j * w.e_dim;
+    se[j][i] = (r0 + j < R) ? to_f(ev[(long long)(r0 + j) * w.e_dim + i]) : 0.f;
+  }
+  if (threadIdx.x < kEvBlock) {
+    int ty = (r0 + threadIdx.x < R) ? types[r0 + threadIdx.x] : 0;
+    if (ty < 0 || ty >= w.n_types) {
+      flag_error(3);
+      ty = 0;
+    }
+    sty[threadIdx.x] = ty;
+  }
+  __syncthreads();
+  float acc[kEvBlock];
+  for (int t = 0; t < w.n_types; ++t) {
+    const T* W1r = (const T*)w.W1[t] + (long long)k * w.e_dim;
+    const float b = to_f(((const T*)w.b1[t])[k]);
+#pragma unroll
+    for (int j = 0; j < kEvBlock; ++j) acc[j] = b;
+    for (int i0 = 0; i0 < w.e_dim; i0 += 8) {
+      float wv[8];
+      load8(W1r + i0, wv);
+      ev_fma8<kEvEmax>(acc, wv, se, i0);
+    }
+#pragma unroll
+    for (int j = 0; j < kEvBlock; ++j)
+      if (sty[j] == t) shid[j][k] = gelu_tanh(acc[j]);
+  }
+  __syncthreads();
+  for (int t = 0; t < w.n_types; ++t) {
+    const T* W2r = (const T*)w.W2[t] + (long long)k * kEvD;
+    const float b = to_f(((const T*)w.b2[t])[k]) + to_f(((const T*)w.emb)[(long long)t * kEvD + k]);
+#pragma unroll
+    for (int j = 0; j < kEvBlock; ++j) acc[j] = b;
+    for (int i0 = 0; i0 < kEvD; i0 += 8) {
+      float wv[8];
+      load8(W2r + i0, wv);
+      ev_fma8<kEvD>(acc, wv, shid, i0);
+    }
+#pragma unroll
+    for (int j = 0; j < kEvBlock; ++j) {
+      const int row = r0 + j;
+      if (sty[j] == t && row < R) {
+        const int bb = row / dL, tt = row - bb * dL;
+        rm_store<T>(out, rm_off(out, bb, tt, k), acc[j]);
+      }
+    }
+  }
+}
+
 }  // namespace ot
