@@ -188,19 +188,31 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         return true;
       };
       auto free_stage = [&]() { umma_commit(&w_empty[q % C::STAGES]); ++q; };
-      // U = h2 W1c^T, K = 256 in four staged k-blocks
-      auto up = [&]() -> bool {
+      // The weight stages of a chunk are waited for ahead of their use (each
+      // barrier wait costs a few hundred cycles here): W2(c) right after
+      // up(c) is issued, while GELU runs; W1(c+1) right after down(c) is
+      // issued, while it runs.  Every awaited stage is freed by MMAs already
+      // issued, so the ring keeps moving.
+      auto wait_ahead = [&](uint64_t* base) -> bool {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          uint64_t wb;
-          if (!wait_stage(wb)) return false;
+          const int qq = q + j, s = qq % C::STAGES;
+          if (!mbar_wait(&w_full[s], (qq / C::STAGES) & 1)) return false;
+          base[j] = desc_add(dW, s * C::STAGE);
+        }
+        tc_fence_after();
+        return true;
+      };
+      // U = h2 W1c^T, K = 256 in four staged k-blocks (stages waited by the caller)
+      auto up = [&](const uint64_t* wb) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            umma_bf16(tU, desc_add(dA, j * 16384 + k * 32), desc_add(wb, k * 32), id256, (j | k) ? 1u : 0u);
+            umma_bf16(tU, desc_add(dA, j * 16384 + k * 32), desc_add(wb[j], k * 32), id256, (j | k) ? 1u : 0u);
           free_stage();
         }
         umma_commit(u_full);
-        return true;
       };
       bool ok = mbar_wait(a_full, 0) && mbar_wait(res_ready, 0);
       if (ok) tc_fence_after();
@@ -215,10 +227,14 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         free_stage();
       }
       if (ok) umma_commit(d_full);
-      ok = ok && mbar_wait(h2_ready, 0);
-      if (ok) tc_fence_after();
-      if (ok) ok = up();
+      uint64_t w1b[4], w2b[4];
+      ok = ok && wait_ahead(w1b) && mbar_wait(h2_ready, 0);
+      if (ok) {
+        tc_fence_after();
+        up(w1b);
+      }
       for (int c = 0; c < NC && ok; ++c) {
+        ok = wait_ahead(w2b);  // W2(c)
         // D += H W2c^T block by block as the GELU output appears: in block b
         // (units 64b..64b+63) units 64b+16k..+15 are packed over U columns
         // 64b+16k..+7, one k-step each
@@ -226,18 +242,21 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
           ok = mbar_wait(&hid_full[b], c & 1);
           if (!ok) break;
           tc_fence_after();
-          uint64_t wb;
-          ok = wait_stage(wb);
-          if (!ok) break;
           const uint32_t tH = tU + b * C::HB;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            umma_bf16_ts(tD, tH + k * 16, desc_add(wb, k * 32), id256, 1u);
+            umma_bf16_ts(tD, tH + k * 16, desc_add(w2b[b], k * 32), id256, 1u);
           free_stage();
         }
         umma_commit(dn_done);
         // up(c+1) overwrites U: let down(c) finish reading it first
-        if (ok && c + 1 < NC) ok = mbar_wait(dn_done, c & 1) && up();
+        if (ok && c + 1 < NC) {
+          ok = wait_ahead(w1b) && mbar_wait(dn_done, c & 1);
+          if (ok) {
+            tc_fence_after();
+            up(w1b);
+          }
+        }
       }
       umma_commit(d_done);
     }
