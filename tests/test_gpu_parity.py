@@ -268,6 +268,30 @@ def test_forward_d384_small():
         assert rel_err(got[u], ref) <= TOL["bf16"]
 
 
+def test_stage1_stage2_d384_small():
+    """Stage I + II of the wider shape (d_h = 96, 16 NS tokens): the
+    two-box head layout in both attention modes, ragged candidate counts
+    (a CTA of 8 candidates' 128 NS rows, a partial one and a user with none)."""
+    sh = shape(n_layers=2, d=384, dff=1536, L_NS=16)
+    L_S = 200
+    sched = [L_S + sh.L_NS, sh.L_NS]
+    b = build(sh, 91, "bf16", pyramid=sched)
+    U = 3
+    S = gen_normal(92, (U, L_S, sh.d), "bf16")
+    counts = [11, 0, 3]
+    offs = np.concatenate([[0], np.cumsum(counts)]).tolist()
+    NS = gen_normal(93, (offs[-1], sh.L_NS, sh.d), "bf16")
+    cache, out = run_stage12(b, S, NS, offs)
+    for u in range(U):
+        kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, sched)
+        for n, (K, V) in enumerate(kv):
+            got = to_np(cache.gather(u, n, K.shape[0]))
+            assert rel_err(got[0], K) <= TOL["bf16"]
+            assert rel_err(got[1], V) <= TOL["bf16"]
+        for c in range(offs[u], offs[u + 1]):
+            assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL["bf16"], (u, c)
+
+
 def _full(name):
     wl = WORKLOADS[name]
     b = build(wl.shape, wl.seed_weights, wl.dtype, pyramid=list(wl.pyramid) if wl.pyramid else None,

@@ -1,4 +1,4 @@
-// Tensor-core attention for the bf16 path (sm_100a), head dim 64.
+// Tensor-core attention for the bf16 path (sm_100a), head dims 64 and 96.
 //
 // One CTA owns 128 query rows of one head.  K/V tiles of 128 keys are
 // streamed by TMA through a 2-deep shared-memory ring.  Per key tile:
@@ -47,18 +47,29 @@ struct TcAttnArgs {
   int H;
 };
 
-struct AttnCfg {
-  static constexpr int DH = 64, BM = 128, BN = 128;
-  static constexpr int Q_BYTES = BM * DH * 2;     // 16 KB
-  static constexpr int KV_BYTES = BN * DH * 2;    // 16 KB (one of K or V)
-  static constexpr int PAGE_BYTES = 64 * DH * 2;  // one 64-token page of one head
+// Head dims 64 and 96.  A row of d_h bf16 is held as NB boxes of 64 columns
+// (128-byte swizzle atoms); for d_h = 96 the second box's columns 96..127
+// are the TMA's zero fill or a neighbouring head's values, which no product
+// reads (Q K^T stops after d_h / 16 k-steps, P.V has N = d_h).
+template <int DH_>
+struct AttnCfgT {
+  static constexpr int DH = DH_, BM = 128, BN = 128;
+  static constexpr int NB = (DH + 63) / 64;
+  static constexpr int BOX_BYTES = 128 * 128;     // 128 rows x 64 bf16
+  static constexpr int Q_BYTES = NB * BOX_BYTES;
+  static constexpr int KV_BYTES = NB * BOX_BYTES; // one of K or V for 128 keys
+  static constexpr int PAGE_BYTES = 64 * 128;     // one 64-token page of one box
+  // d_h = 64: S 0..127, O 128..191, P (bf16 pairs) 192..255, two CTAs per SM;
+  // d_h = 96: S 0..127, O 128..223, P 224..287 of 512 columns, one CTA per SM
+  static constexpr int T_O = 128, T_P = 128 + (DH + 31) / 32 * 32;
+  static constexpr int TMEM_COLS = DH <= 64 ? 256 : 512;
+  static constexpr int CTAS = DH <= 64 ? 2 : 1;
   // three K/V stages: the load of tile kt+1 may start while P.V of tile kt-1
-  // still reads its stage (two CTAs of 115 KB share an SM's 228 KB)
+  // still reads its stage (two CTAs of 115 KB share an SM's 228 KB at d_h = 64)
   static constexpr int STAGES = 3;
   static constexpr int BAR_BYTES = 128;
   static constexpr int MAX_PAGES = 128;           // page ids cached in shared memory (8192 keys)
   static constexpr int SMEM = Q_BYTES + STAGES * 2 * KV_BYTES + BAR_BYTES + MAX_PAGES * 4;
-  static constexpr int TMEM_COLS = 256;           // S 0..127, O 128..191, P (bf16 pairs) 192..255
 };
 
 __device__ inline int kv_page_id(const KVStore& kv, int b, int page_idx) {
@@ -71,13 +82,14 @@ __device__ inline float ex2(float x) {
   return y;
 }
 
-__global__ void __launch_bounds__(192, 2)
+template <int DH>
+__global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                    const __grid_constant__ CUtensorMap tmNS, const TcAttnArgs a) {
-  using C = AttnCfg;
+  using C = AttnCfgT<DH>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + C::Q_BYTES;  // [stage][K|V][128 keys][64]
+  uint8_t* sKV = sQ + C::Q_BYTES;  // [stage][K|V][box][128 keys][64]
   uint64_t* bars = (uint64_t*)(sKV + C::STAGES * 2 * C::KV_BYTES);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;                // [STAGES]
@@ -148,15 +160,20 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128, tP = tmem + 192;
+  const uint32_t tS = tmem, tO = tmem + C::T_O, tP = tmem + C::T_P;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && nt > 0) {
       const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
       mbar_expect_tx(q_full, C::Q_BYTES);
-      if (a.mode == MODE_CAUSAL) tma_load_3d_hint(&tmQ, q_full, sQ, h * C::DH, row0, b, stream);
-      else tma_load_3d_hint(&tmQ, q_full, sQ, h * C::DH, row0, 0, stream);
+#pragma unroll
+      for (int i = 0; i < C::NB; ++i) {
+        if (a.mode == MODE_CAUSAL)
+          tma_load_3d_hint(&tmQ, q_full, sQ + i * C::BOX_BYTES, h * C::DH + i * 64, row0, b, stream);
+        else
+          tma_load_3d_hint(&tmQ, q_full, sQ + i * C::BOX_BYTES, h * C::DH + i * 64, row0, 0, stream);
+      }
       for (int kt = 0; kt < nt; ++kt) {
         const int s = kt % C::STAGES;
         if (kt >= C::STAGES && !mbar_wait(&kv_empty[s], ((kt / C::STAGES) - 1) & 1)) break;
@@ -169,14 +186,21 @@ __global__ void __launch_bounds__(192, 2)
             const int pi = kt * 2 + hp;
             const int pg = pi < C::MAX_PAGES ? s_pages[pi]
                                              : (pi < n_pages_used ? kv_page_id(a.kv, b, pi) : a.kv.n_pages);
-            tma_load_4d_hint(&tmKV, &kv_full[s], sk + hp * C::PAGE_BYTES, 0, 0, h, pg, keep);
-            tma_load_4d_hint(&tmKV, &kv_full[s], sv + hp * C::PAGE_BYTES, 0, 0, a.H + h, pg, keep);
+#pragma unroll
+            for (int i = 0; i < C::NB; ++i) {
+              tma_load_4d_hint(&tmKV, &kv_full[s], sk + i * C::BOX_BYTES + hp * C::PAGE_BYTES, i * 64, 0, h, pg, keep);
+              tma_load_4d_hint(&tmKV, &kv_full[s], sv + i * C::BOX_BYTES + hp * C::PAGE_BYTES, i * 64, 0, a.H + h, pg,
+                               keep);
+            }
           }
         } else {
           // own NS keys of this CTA's candidates: the K and V column blocks of the same rows
           const int d = a.H * C::DH;
-          tma_load_3d_hint(&tmNS, &kv_full[s], sk, d + h * C::DH, row0, 0, stream);
-          tma_load_3d_hint(&tmNS, &kv_full[s], sv, 2 * d + h * C::DH, row0, 0, stream);
+#pragma unroll
+          for (int i = 0; i < C::NB; ++i) {
+            tma_load_3d_hint(&tmNS, &kv_full[s], sk + i * C::BOX_BYTES, d + h * C::DH + i * 64, row0, 0, stream);
+            tma_load_3d_hint(&tmNS, &kv_full[s], sv + i * C::BOX_BYTES, 2 * d + h * C::DH + i * 64, row0, 0, stream);
+          }
         }
       }
     }
@@ -184,16 +208,21 @@ __global__ void __launch_bounds__(192, 2)
     // ----------------------------------------------------------------- MMA
     if (lane == 0 && nt > 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, 128);
-      constexpr uint32_t id_pv = idesc_bf16(128, 64, false, true);
+      constexpr uint32_t id_pv = idesc_bf16(128, C::DH, false, true);
+      constexpr int KS = C::DH / 16;  // k-steps of Q K^T: 4 per 64-column box
       // base descriptors of Q and of each stage's K and V tiles
       const uint64_t dq = sdesc_k128(smem_u32(sQ));
       const uint64_t dk0 = sdesc_k128(smem_u32(sKV));                    // stage s: + s * 2 * KV_BYTES
-      const uint64_t dv0 = sdesc_mn128(smem_u32(sKV + C::KV_BYTES), 0);
+      // V as the MN-major B operand: 64-column boxes (N atoms) BOX_BYTES apart
+      const uint64_t dv0 = sdesc_mn128(smem_u32(sKV + C::KV_BYTES), C::NB > 1 ? C::BOX_BYTES : 0);
       bool ok = mbar_wait(q_full, 0) && mbar_wait(&kv_full[0], 0);
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma_bf16(tS, desc_add(dq, k * 32), desc_add(dk0, k * 32), id_qk, k ? 1u : 0u);
+        for (int k = 0; k < KS; ++k) {
+          const uint32_t off = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;
+          umma_bf16(tS, desc_add(dq, off), desc_add(dk0, off), id_qk, k ? 1u : 0u);
+        }
         umma_commit(s_full);
       }
       for (int kt = 0; kt < nt && ok; ++kt) {
@@ -206,7 +235,10 @@ __global__ void __launch_bounds__(192, 2)
           tc_fence_after();
           const uint64_t dk = desc_add(dk0, s1 * 2 * C::KV_BYTES);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) umma_bf16(tS, desc_add(dq, k * 32), desc_add(dk, k * 32), id_qk, k ? 1u : 0u);
+          for (int k = 0; k < KS; ++k) {
+            const uint32_t off = (k >> 2) * C::BOX_BYTES + (k & 3) * 32;
+            umma_bf16(tS, desc_add(dq, off), desc_add(dk, off), id_qk, k ? 1u : 0u);
+          }
           umma_commit(s_full);
         }
         // P of tile kt is in TMEM
@@ -310,7 +342,7 @@ __global__ void __launch_bounds__(192, 2)
       if (rescale) {
         // O holds the tiles before kt (p_free was awaited): bring it to the new max
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < C::DH / 32; ++c) {
           float ov[32];
           tmem_ld32(tO + lb + c * 32, ov);
 #pragma unroll
@@ -324,9 +356,12 @@ __global__ void __launch_bounds__(192, 2)
       // keys past the last valid cache key may hold stale bits (P is 0 there,
       // but 0 * NaN is not): zero their V rows before P.V reads them
       if (kt == nt_s - 1 && kbase + r > kmax) {
-        uint4* vrow = (uint4*)(sKV + (kt % C::STAGES) * 2 * C::KV_BYTES + C::KV_BYTES + r * 128);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) vrow[ch] = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < C::NB; ++i) {
+          uint4* vrow = (uint4*)(sKV + (kt % C::STAGES) * 2 * C::KV_BYTES + C::KV_BYTES + i * C::BOX_BYTES + r * 128);
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) vrow[ch] = make_uint4(0, 0, 0, 0);
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       tmem_st_wait();
@@ -335,24 +370,23 @@ __global__ void __launch_bounds__(192, 2)
     }
     ok = ok && mbar_wait(o_done, 0);
     tc_fence_after();
-    float o[64];
+    float o[C::DH];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) tmem_ld32(tO + lb + c * 32, o + c * 32);
+    for (int c = 0; c < C::DH / 32; ++c) tmem_ld32(tO + lb + c * 32, o + c * 32);
     const float inv = 1.f / l;
 #pragma unroll
-    for (int e = 0; e < 64; ++e) o[e] *= inv;
+    for (int e = 0; e < C::DH; ++e) o[e] *= inv;
     if (ok && nt > 0) {
+      __nv_bfloat16* dst = nullptr;
       if (a.mode == MODE_CAUSAL) {
         const int t = row0 + r;
-        if (t < a.Lq) {
-          __nv_bfloat16* dst = (__nv_bfloat16*)a.o.base + rm_off(a.o, b, t, h * 64);
-          store_bf16x32(dst, o);
-          store_bf16x32(dst + 32, o + 32);
-        }
+        if (t < a.Lq) dst = (__nv_bfloat16*)a.o.base + rm_off(a.o, b, t, h * C::DH);
       } else if (r < n_rows) {
-        __nv_bfloat16* dst = a.o2 + (long long)(row0 + r) * (a.H * 64) + h * 64;
-        store_bf16x32(dst, o);
-        store_bf16x32(dst + 32, o + 32);
+        dst = a.o2 + (long long)(row0 + r) * (a.H * C::DH) + h * C::DH;
+      }
+      if (dst) {
+#pragma unroll
+        for (int c = 0; c < C::DH / 32; ++c) store_bf16x32(dst + c * 32, o + c * 32);
       }
     }
   }
@@ -378,25 +412,33 @@ inline bool make_tmap_pages(CUtensorMap* map, const KVStore& kv) {
 }
 
 inline bool tc_kv_ok(const KVStore& kv) {
-  return kv.dh == 64 && kv.P == 64 && kv.n_pages > 0 && ((uintptr_t)kv.pool % 16) == 0 && encode_fn();
+  return (kv.dh == 64 || kv.dh == 96) && kv.P == 64 && kv.n_pages > 0 && ((uintptr_t)kv.pool % 16) == 0 && encode_fn();
 }
 
 inline bool tc_attn_supported(const AttnDesc& a) {
-  return a.dh == 64 && tc_kv_ok(a.kv) && ((uintptr_t)a.q.base % 16) == 0 && a.q.st % 8 == 0 &&
+  return (a.dh == 64 || a.dh == 96) && a.kv.dh == a.dh && tc_kv_ok(a.kv) && ((uintptr_t)a.q.base % 16) == 0 && a.q.st % 8 == 0 &&
          a.q.sb % 8 == 0 && rowmap_vec_ok(a.o) && !a.o.f32;
 }
 
-inline onetrans_status attn_launch_common(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tns,
-                                          const TcAttnArgs& args, dim3 grid, cudaStream_t st) {
+template <int DH>
+inline onetrans_status attn_launch_dh(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tns,
+                                      const TcAttnArgs& args, dim3 grid, cudaStream_t st) {
+  using C = AttnCfgT<DH>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg::SMEM) !=
+    if (cudaFuncSetAttribute(attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
         cudaSuccess)
       return ONETRANS_ERR_CUDA;
     attr_set = true;
   }
-  attn_tc_kernel<<<grid, 192, AttnCfg::SMEM, st>>>(tq, tkv, tns, args);
+  attn_tc_kernel<DH><<<grid, 192, C::SMEM, st>>>(tq, tkv, tns, args);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
+}
+
+inline onetrans_status attn_launch_common(const CUtensorMap& tq, const CUtensorMap& tkv, const CUtensorMap& tns,
+                                          const TcAttnArgs& args, int dh, dim3 grid, cudaStream_t st) {
+  if (dh == 96) return attn_launch_dh<96>(tq, tkv, tns, args, grid, st);
+  return attn_launch_dh<64>(tq, tkv, tns, args, grid, st);
 }
 
 inline onetrans_status tc_attn_launch(const AttnDesc& a, cudaStream_t st) {
@@ -416,14 +458,14 @@ inline onetrans_status tc_attn_launch(const AttnDesc& a, cudaStream_t st) {
   args.kv = a.kv;
   args.H = a.H;
   dim3 grid((unsigned)((a.Lq + 127) / 128), (unsigned)a.H, (unsigned)a.B);
-  return attn_launch_common(tq, tkv, tkv, args, grid, st);
+  return attn_launch_common(tq, tkv, tkv, args, a.dh, grid, st);
 }
 
 // Candidates per Stage II tile: whole candidates' NS rows fill at most 128 rows.
 inline int stage2_cands_per_tile(int L_NS) { return L_NS <= 128 ? 128 / L_NS : 0; }
 
 inline bool tc_stage2_supported(const Stage2Desc& a) {
-  return a.dh == 64 && stage2_cands_per_tile(a.L_NS) > 0 && tc_kv_ok(a.kv) && ((uintptr_t)a.qkv % 16) == 0 &&
+  return (a.dh == 64 || a.dh == 96) && a.kv.dh == a.dh && stage2_cands_per_tile(a.L_NS) > 0 && tc_kv_ok(a.kv) && ((uintptr_t)a.qkv % 16) == 0 &&
          ((uintptr_t)a.o % 16) == 0;
 }
 
@@ -444,7 +486,7 @@ inline onetrans_status tc_stage2_launch(const Stage2Desc& a, int n_tiles, cudaSt
   args.kv = a.kv;
   args.H = a.H;
   dim3 grid((unsigned)n_tiles, (unsigned)a.H, 1);
-  return attn_launch_common(tq, tkv, tq, args, grid, st);
+  return attn_launch_common(tq, tkv, tq, args, a.dh, grid, st);
 }
 
 }  // namespace ot
