@@ -35,6 +35,10 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 METRIC = "candidates scored/sec (Stage II, KV-cached) and users/sec (Stage I) on 1 B200"
+# DRAM bytes (read + write) per launch of a kernel kind on the default
+# workload, from one ncu capture of the kernels as committed with this file
+# (profiles/kv_serving_launch_list.md); re-measure when such a kernel changes.
+TRAFFIC_PER_LAUNCH = {"fused_oproj_ffn": 137.8e6}
 UNIT = "candidates/s"
 
 
@@ -585,18 +589,20 @@ def main():
     # ---- roofline of the dominant kernel (largest device time in the timed region)
     pk = peaks()
     dom_name, dom = max(prof.items(), key=lambda kv: kv[1]["ms"])
+    traffic = (TRAFFIC_PER_LAUNCH.get(dom_name)
+               if args.workload == "kv_serving" and not (args.users or args.cands) else None)
     per_launch_ms = dom["ms"] / dom["launches"]
     tensor_bound = dom["flops"] / max(dom["bytes"], 1.0) > pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     if tensor_bound:
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
         roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": pk["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops_sustained"],
-                "peak_source": pk["source"] + " bf16 sustained", "traffic": None,
+                "peak_source": pk["source"] + " bf16 sustained", "traffic": traffic,
                 "flops_per_launch": dom["flops"] / dom["launches"], "ms_per_launch": per_launch_ms}
     else:
         achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"] + " copy", "traffic": None,
+                "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"] + " copy", "traffic": traffic,
                 "bytes_per_launch": dom["bytes"] / dom["launches"], "ms_per_launch": per_launch_ms}
     kernels = {k: {"launches": v["launches"], "ms": round(v["ms"], 3),
                    "share": round(v["ms"] / sum(x["ms"] for x in prof.values()), 4),
