@@ -26,6 +26,9 @@
  *  - A model is immutable after creation and may be used from several
  *    streams at once.  Calls that modify one cache slot must not overlap.
  *  - Buffers must be 16-byte aligned; the workspace and cache pool 256-byte.
+ *  - A call with no work (N = 0, U = 0, B = 0, dL = 0, or no candidates at
+ *    all) checks the model, cache, slots and offsets, returns ONETRANS_OK and
+ *    launches nothing; its data pointers and workspace may then be NULL.
  */
 #ifndef ONETRANS_H
 #define ONETRANS_H

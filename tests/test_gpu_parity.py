@@ -292,6 +292,57 @@ def test_stage1_stage2_d384_small():
             assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL["bf16"], (u, c)
 
 
+def test_zero_work_calls_launch_nothing():
+    """Calls with no work return without error and change nothing: no
+    features, no samples, no users, users without candidates, no appended
+    events (NULL data pointers included)."""
+    sh = shape(n_layers=2)
+    b = build(sh, 121, "bf16", event_dim=64)
+    m = b.model
+    bf = torch.bfloat16
+    empty_ws = torch.empty(0, dtype=torch.uint8, device="cuda")
+    ot.onetrans_tokenize_autosplit(m, torch.empty(0, sh.ns_feat, dtype=bf, device="cuda"),
+                                   torch.empty(0, sh.L_NS, sh.d, dtype=bf, device="cuda"), empty_ws)
+    ot.onetrans_forward(m, torch.empty(0, 40 + sh.L_NS, sh.d, dtype=bf, device="cuda"),
+                        torch.empty(0, 40 + sh.L_NS, sh.d, dtype=torch.float32, device="cuda"), empty_ws)
+    U, L_S = 2, 70
+    cache = ot.Cache(m, U, L_S + 8)
+    ot.onetrans_stage1_encode(m, cache, [], torch.empty(0, L_S, sh.d, dtype=bf, device="cuda"), empty_ws)
+    assert cache.length(0) == 0 and cache.length(1) == 0
+    S = gen_normal(122, (U, L_S, sh.d), "bf16")
+    ot.onetrans_stage1_encode(m, cache, [0, 1], to_dev(S, bf), m.workspace(ot.OP_STAGE1, U, L_S))
+    torch.cuda.synchronize()
+    before = to_np(cache.gather(1, 0, L_S))
+    ot.onetrans_stage2_score(m, cache, [0, 1], [0, 0, 0], torch.empty(0, sh.L_NS, sh.d, dtype=bf, device="cuda"),
+                             torch.empty(0, sh.L_NS, sh.d, dtype=torch.float32, device="cuda"), empty_ws)
+    ot.onetrans_cache_append(m, cache, [0, 1], torch.empty(U, 0, 64, dtype=bf, device="cuda"),
+                             torch.empty(U, 0, dtype=torch.int32, device="cuda"), empty_ws)
+    torch.cuda.synchronize()
+    assert cache.length(0) == L_S and cache.length(1) == L_S
+    np.testing.assert_array_equal(to_np(cache.gather(1, 0, L_S)), before)
+
+
+def test_long_sequence_beyond_cached_page_ids():
+    """8400 cached tokens = 132 pages per layer, past the 128 page ids the
+    attention kernel keeps in shared memory: the remaining ids come from the
+    page table in global memory, in Stage I's causal attention (100 tail
+    queries over up to 8400 keys) and in Stage II."""
+    sh = shape(n_layers=2)
+    L_S = 8400
+    sched = [112, sh.L_NS]
+    b = build(sh, 131, "bf16", pyramid=sched)
+    S = gen_normal(132, (1, L_S, sh.d), "bf16")
+    NS = gen_normal(133, (3, sh.L_NS, sh.d), "bf16")
+    cache, out = run_stage12(b, S, NS, [0, 3])
+    kv = O.stage1(S[0], b.W, sh.L_NS, sh.n_heads, EPS, sched)
+    K0 = to_np(cache.gather(0, 0, L_S))
+    assert rel_err(K0[0], kv[0][0]) <= TOL["bf16"] and rel_err(K0[1], kv[0][1]) <= TOL["bf16"]
+    K1 = to_np(cache.gather(0, 1, kv[1][0].shape[0]))
+    assert rel_err(K1[0], kv[1][0]) <= TOL["bf16"] and rel_err(K1[1], kv[1][1]) <= TOL["bf16"]
+    for c in range(3):
+        assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL["bf16"]
+
+
 def _full(name):
     wl = WORKLOADS[name]
     b = build(wl.shape, wl.seed_weights, wl.dtype, pyramid=list(wl.pyramid) if wl.pyramid else None,

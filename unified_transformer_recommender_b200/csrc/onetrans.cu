@@ -1067,11 +1067,13 @@ static onetrans_status check_ws(void* ws) {
 
 onetrans_status onetrans_tokenize_autosplit(const onetrans_model* m, const void* feats, int64_t N,
                                             void* ns_tokens, void* ws, size_t ws_bytes, void* stream) {
-  if (!m || !feats || !ns_tokens || !aligned(feats, 16) || !aligned(ns_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
-  OT_TRY(check_ws(ws));
+  if (!m) return ONETRANS_ERR_INVALID_ARG;
   if (N < 0 || N > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
   if (!m->Wa1 || !m->ba1 || !m->Wa2 || !m->ba2 || m->cfg.ns_feat_dim < 1 || m->cfg.ns_hidden < 1)
     return ONETRANS_ERR_UNSUPPORTED;
+  if (N == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!feats || !ns_tokens || !aligned(feats, 16) || !aligned(ns_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? autosplit_impl<__nv_bfloat16>(m, feats, N, ns_tokens, ws, ws_bytes, st, nullptr)
                  : autosplit_impl<float>(m, feats, N, ns_tokens, ws, ws_bytes, st, nullptr);
@@ -1092,12 +1094,13 @@ static onetrans_status check_slots(const onetrans_cache* c, const int32_t* slots
 onetrans_status onetrans_stage1_encode(const onetrans_model* m, onetrans_cache* c, const int32_t* slots,
                                        int32_t U, const void* s_tokens, int32_t L_S, void* ws, size_t ws_bytes,
                                        void* stream) {
-  if (!m || !c || c->m != m || !s_tokens || !aligned(s_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
-  OT_TRY(check_ws(ws));
+  if (!m || !c || c->m != m) return ONETRANS_ERR_INVALID_ARG;
   OT_TRY(check_slots(c, slots, U));
   if (L_S < 1) return ONETRANS_ERR_SHAPE;
   if ((long long)U * L_S > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
-  if (U == 0) return ONETRANS_OK;
+  if (U == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!s_tokens || !aligned(s_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? stage1_impl<__nv_bfloat16>(m, c, slots, U, s_tokens, L_S, ws, ws_bytes, st, nullptr)
                  : stage1_impl<float>(m, c, slots, U, s_tokens, L_S, ws, ws_bytes, st, nullptr);
@@ -1106,18 +1109,20 @@ onetrans_status onetrans_stage1_encode(const onetrans_model* m, onetrans_cache* 
 onetrans_status onetrans_stage2_score(const onetrans_model* m, const onetrans_cache* c, const int32_t* slots,
                                       int32_t U, const int32_t* cand_offsets, const void* ns_tokens,
                                       void* ns_out, void* ws, size_t ws_bytes, void* stream) {
-  if (!m || !c || c->m != m || !cand_offsets || !ns_tokens || !ns_out) return ONETRANS_ERR_INVALID_ARG;
-  if (!aligned(ns_tokens, 16) || !aligned(ns_out, 16)) return ONETRANS_ERR_INVALID_ARG;
-  OT_TRY(check_ws(ws));
+  if (!m || !c || c->m != m) return ONETRANS_ERR_INVALID_ARG;
   OT_TRY(check_slots(c, slots, U));
-  if (U == 0) return ONETRANS_OK;
+  if (U == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
   if (U > kMaxUsers) return ONETRANS_ERR_SHAPE;
+  if (!cand_offsets) return ONETRANS_ERR_INVALID_ARG;
   for (int u = 0; u < U; ++u)
     if (cand_offsets[u + 1] < cand_offsets[u]) return ONETRANS_ERR_SHAPE;
   if (cand_offsets[0] != 0) return ONETRANS_ERR_SHAPE;
   const int L_S = c->len[slots[0]];
   for (int u = 0; u < U; ++u)
     if (c->len[slots[u]] != L_S || L_S == 0) return ONETRANS_ERR_SHAPE;
+  if (cand_offsets[U] == 0) return ONETRANS_OK;  // no candidates
+  if (!ns_tokens || !ns_out || !aligned(ns_tokens, 16) || !aligned(ns_out, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? stage2_impl<__nv_bfloat16>(m, c, slots, U, cand_offsets, ns_tokens, ns_out, ws, ws_bytes,
                                               st, nullptr, 0, 0)
@@ -1132,11 +1137,11 @@ onetrans_status onetrans_cache_append(const onetrans_model* m, onetrans_cache* c
   if (!m->pyr.empty()) return ONETRANS_ERR_UNSUPPORTED;
   if (m->cfg.n_behaviors < 1 || m->cfg.event_dim < 1 || m->Wb1.empty() || !m->type_emb)
     return ONETRANS_ERR_UNSUPPORTED;
-  if (!events || !types || !aligned(events, 16)) return ONETRANS_ERR_INVALID_ARG;
-  OT_TRY(check_ws(ws));
   OT_TRY(check_slots(c, slots, U));
   if (dL < 0) return ONETRANS_ERR_SHAPE;
-  if (U == 0 || dL == 0) return ONETRANS_OK;
+  if (U == 0 || dL == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!events || !types || !aligned(events, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
   const int L0 = c->len[slots[0]];
   for (int u = 0; u < U; ++u)
     if (c->len[slots[u]] != L0 || L0 == 0) return ONETRANS_ERR_SHAPE;
@@ -1147,11 +1152,12 @@ onetrans_status onetrans_cache_append(const onetrans_model* m, onetrans_cache* c
 
 onetrans_status onetrans_forward(const onetrans_model* m, const void* x0, int32_t B, int32_t L_S, void* out,
                                  void* ws, size_t ws_bytes, void* stream) {
-  if (!m || !x0 || !out || !aligned(x0, 16) || !aligned(out, 16)) return ONETRANS_ERR_INVALID_ARG;
-  OT_TRY(check_ws(ws));
+  if (!m) return ONETRANS_ERR_INVALID_ARG;
   if (B < 0 || L_S < 0) return ONETRANS_ERR_SHAPE;
   if ((long long)B * (L_S + m->L_NS) > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
-  if (B == 0) return ONETRANS_OK;
+  if (B == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!x0 || !out || !aligned(x0, 16) || !aligned(out, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? forward_impl<__nv_bfloat16>(m, x0, B, L_S, out, ws, ws_bytes, st, nullptr)
                  : forward_impl<float>(m, x0, B, L_S, out, ws, ws_bytes, st, nullptr);
@@ -1249,12 +1255,13 @@ static onetrans_status autosplit_with_hidden(const onetrans_model* m, const void
 
 extern "C" onetrans_status onetrans_tokenize_autosplit_static(const onetrans_model* m, const void* feats,
                                                               int64_t N, void* ns_tokens, void* stream) {
-  if (!m || !feats || !ns_tokens || !aligned(feats, 16) || !aligned(ns_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
+  if (!m) return ONETRANS_ERR_INVALID_ARG;
   if (N < 0 || N > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
   if (!m->Wa1 || !m->ba1 || !m->Wa2 || !m->ba2 || m->cfg.ns_feat_dim < 1 || m->cfg.ns_hidden < 1)
     return ONETRANS_ERR_UNSUPPORTED;
   if ((size_t)N * m->cfg.ns_hidden * m->es > kStaticScratchBytes) return ONETRANS_ERR_CAPACITY;
-  if (N == 0) return ONETRANS_OK;
+  if (N == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!feats || !ns_tokens || !aligned(feats, 16) || !aligned(ns_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
   void* hid = nullptr;
   OT_TRY(static_scratch(&hid));
   cudaStream_t st = (cudaStream_t)stream;
