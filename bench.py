@@ -3,8 +3,9 @@
 (Stage II over the KV cache) and users encoded per second (Stage I).
 
 One step = auto-split tokenization of every candidate's NS features, Stage I
-of every user's S tokens into the paged KV cache, and Stage II scoring of
-every candidate against its user's cache, all through the C ABI.  Workload
+of every user's S tokens into the paged KV cache (the two are independent
+and run on two streams at once), and Stage II scoring of every candidate
+against its user's cache, all through the C ABI.  Workload
 (default): 6 layers, d=256, 4 heads, FFN 1024, 12 NS tokens, L_S = 1178,
 pyramid query counts 1190 -> 12 (linear), 16 users x 512 candidates, NS
 features 512 wide, bf16 storage.  Other workloads: --workload append (non-
@@ -180,6 +181,8 @@ class KVServing:
         self.ws_1 = m.workspace(ot.OP_STAGE1, self.U, wl.L_S)
         self.ws_2 = m.workspace(ot.OP_STAGE2, self.U * self.C, wl.L_S)
         self.cache = ot.Cache(m, self.U, wl.L_S)
+        self.side = torch.cuda.Stream()
+        self.ev_in, self.ev_tok = torch.cuda.Event(), torch.cuda.Event()
         self.slots = list(range(self.U))
         self.offs = [u * self.C for u in range(self.U + 1)]
         self.units = self.U * self.C
@@ -187,11 +190,19 @@ class KVServing:
         self.d2h = self.out.numel() * 4
 
     def step(self, ev_mid=None):
+        """Stage I on the current stream; the candidates' auto-split, which
+        does not depend on it, on a side stream meanwhile (Stage I's short
+        launches leave SMs idle); Stage II once both are done."""
         ot, m = self.ot, self.model
+        main = self.torch.cuda.current_stream()
+        self.ev_in.record(main)
+        self.side.wait_event(self.ev_in)
+        ot.onetrans_tokenize_autosplit(m, self.F, self.ns, self.ws_a, stream=self.side)
+        self.ev_tok.record(self.side)
         ot.onetrans_stage1_encode(m, self.cache, self.slots, self.S, self.ws_1)
         if ev_mid is not None:
             ev_mid.record()
-        ot.onetrans_tokenize_autosplit(m, self.F, self.ns, self.ws_a)
+        main.wait_event(self.ev_tok)
         ot.onetrans_stage2_score(m, self.cache, self.slots, self.offs, self.ns, self.out, self.ws_2)
 
     metric, unit = METRIC, UNIT
@@ -247,6 +258,8 @@ class Append:
         self.F_pin = torch.from_numpy(self.F_h).to(torch.bfloat16).pin_memory()
         m = self.model
         self.caches, self.k = [], 0
+        self.side = torch.cuda.Stream()
+        self.ev_in, self.ev_tok = torch.cuda.Event(), torch.cuda.Event()
         self.slots = list(range(self.U))
         self.offs = [u * self.C for u in range(self.U + 1)]
         self.ns = torch.empty(self.U * self.C, sh.L_NS, sh.d, dtype=torch.bfloat16, device=dev)
@@ -278,13 +291,20 @@ class Append:
         self.torch.cuda.synchronize()
 
     def step(self, ev_mid=None):
+        """The append on the current stream, the candidates' auto-split on a
+        side stream meanwhile, Stage II once both are done."""
         ot, m = self.ot, self.model
         cache = self.caches[self.k]
         self.k += 1
+        main = self.torch.cuda.current_stream()
+        self.ev_in.record(main)
+        self.side.wait_event(self.ev_in)
+        ot.onetrans_tokenize_autosplit(m, self.F, self.ns, self.ws_a, stream=self.side)
+        self.ev_tok.record(self.side)
         ot.onetrans_cache_append(m, cache, self.slots, self.ev, self.ty, self.ws_ap)
         if ev_mid is not None:
             ev_mid.record()
-        ot.onetrans_tokenize_autosplit(m, self.F, self.ns, self.ws_a)
+        main.wait_event(self.ev_tok)
         ot.onetrans_stage2_score(m, cache, self.slots, self.offs, self.ns, self.out, self.ws_2)
 
     def oracle(self):
