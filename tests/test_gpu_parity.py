@@ -352,23 +352,46 @@ def _full(name):
 
 def test_kv_serving_full_size_sampled():
     """The benchmark's workload and launch sequence: auto-split of 16 x 512
-    candidates, Stage I of 16 users x 1178, Stage II; oracle on sampled users
-    and candidates."""
+    candidates on a second stream beside Stage I of 16 users x 1178, then
+    Stage II.  The two-stream runs (repeated, cache rewritten each time) must
+    reproduce a one-stream run bit for bit; the oracle checks sampled users
+    and candidates of it."""
     wl, b = _full("kv_serving")
     sh, U, C = wl.shape, wl.users, wl.cands
     S = gen_normal(wl.seed_inputs, (U, wl.L_S, sh.d), "bf16")
     feats = gen_normal(wl.seed_inputs + 100, (U * C, sh.ns_feat), "bf16")
     m = b.model
+    S_d, F_d = to_dev(S, torch.bfloat16), to_dev(feats, torch.bfloat16)
     ns = torch.empty(U * C, sh.L_NS, sh.d, dtype=torch.bfloat16, device="cuda")
-    ot.onetrans_tokenize_autosplit(m, to_dev(feats, torch.bfloat16), ns, m.workspace(ot.OP_AUTOSPLIT, U * C))
     cache = ot.Cache(m, U, wl.L_S)
-    ot.onetrans_stage1_encode(m, cache, list(range(U)), to_dev(S, torch.bfloat16),
-                              m.workspace(ot.OP_STAGE1, U, wl.L_S))
     out = torch.empty(U * C, sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
-    ot.onetrans_stage2_score(m, cache, list(range(U)), [u * C for u in range(U + 1)], ns, out,
-                             m.workspace(ot.OP_STAGE2, U * C, wl.L_S))
+    ws_a = m.workspace(ot.OP_AUTOSPLIT, U * C)
+    ws_1 = m.workspace(ot.OP_STAGE1, U, wl.L_S)
+    ws_2 = m.workspace(ot.OP_STAGE2, U * C, wl.L_S)
+    slots, offs = list(range(U)), [u * C for u in range(U + 1)]
+
+    ot.onetrans_tokenize_autosplit(m, F_d, ns, ws_a)
+    ot.onetrans_stage1_encode(m, cache, slots, S_d, ws_1)
+    ot.onetrans_stage2_score(m, cache, slots, offs, ns, out, ws_2)
     torch.cuda.synchronize()
-    out, NS = to_np(out), to_np(ns)
+    out_seq, ns_seq = out.clone(), ns.clone()
+
+    main, side = torch.cuda.current_stream(), torch.cuda.Stream()
+    ev_in, ev_tok = torch.cuda.Event(), torch.cuda.Event()
+    for _ in range(3):
+        ns.zero_()
+        out.zero_()
+        ev_in.record(main)
+        side.wait_event(ev_in)
+        ot.onetrans_tokenize_autosplit(m, F_d, ns, ws_a, stream=side)
+        ev_tok.record(side)
+        ot.onetrans_stage1_encode(m, cache, slots, S_d, ws_1)
+        main.wait_event(ev_tok)
+        ot.onetrans_stage2_score(m, cache, slots, offs, ns, out, ws_2)
+        torch.cuda.synchronize()
+        assert torch.equal(ns, ns_seq) and torch.equal(out, out_seq)
+
+    out, NS = to_np(out_seq), to_np(ns_seq)
     for u in (0, U - 1):
         kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, wl.pyramid)
         for c in (u * C, u * C + 317, u * C + C - 1):

@@ -110,6 +110,32 @@ __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
 
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < C::STAGES; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(p_free, 1);
+    mbar_init(o_done, 1);
+    mbar_init(s_free, 128);
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmKV);
+      if (a.mode == MODE_STAGE2) prefetch_tmap(&tmNS);
+    }
+  }
+  if (warp == 5) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + C::T_O, tP = tmem + C::T_P;
+  grid_dep_wait();
+  grid_dep_launch();
+
   // ---- work of this CTA
   int b, row0, n_keys_s, kmax, nt, n_rows = C::BM;
   int c0 = 0;
@@ -133,36 +159,12 @@ __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
   const int nt_s = (n_keys_s + C::BN - 1) / C::BN;  // tiles from the KV pages
   const int n_pages_used = (kmax + 1 + 63) / 64;
 
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int i = 0; i < C::STAGES; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(p_free, 1);
-    mbar_init(o_done, 1);
-    mbar_init(s_free, 128);
-    fence_barrier_init();
-  }
   if (warp == 4) {
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmKV);
-      if (a.mode == MODE_STAGE2) prefetch_tmap(&tmNS);
-    }
     // page ids of every key page this CTA reads, fetched once (page ids past
     // the cached range read as the out-of-range page, which loads zeros)
     const int n_pg = min(2 * nt_s, C::MAX_PAGES);
     for (int i = lane; i < n_pg; i += 32) s_pages[i] = i < n_pages_used ? kv_page_id(a.kv, b, i) : a.kv.n_pages;
     __syncwarp();
-  }
-  if (warp == 5) tmem_alloc(tmem_slot, C::TMEM_COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + C::T_O, tP = tmem + C::T_P;
-
-  if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && nt > 0) {
       const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
@@ -431,7 +433,7 @@ inline onetrans_status attn_launch_dh(const CUtensorMap& tq, const CUtensorMap& 
       return ONETRANS_ERR_CUDA;
     attr_set = true;
   }
-  attn_tc_kernel<DH><<<grid, 192, C::SMEM, st>>>(tq, tkv, tns, args);
+  launch_dependent(attn_tc_kernel<DH>, grid, dim3(192), C::SMEM, st, tq, tkv, tns, args);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 

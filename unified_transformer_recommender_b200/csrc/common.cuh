@@ -9,6 +9,7 @@
 //   TILE_FLAT    tiled m = b * fold + t        (rows contiguous across users)
 #pragma once
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -128,5 +129,35 @@ __device__ inline float gelu_tanh(float x) {
 // code here instead of trapping; the host reads and clears it.
 __device__ int g_device_status = 0;  // one translation unit holds every kernel
 __device__ inline void flag_error(int code) { atomicCAS(&g_device_status, 0, code); }
+
+// Programmatic dependent launch.  Kernels of one call follow each other on a
+// stream; launched with the programmatic-serialization attribute, a kernel's
+// CTAs may start while its predecessor's last CTAs still run.  Each kernel
+// therefore does only local set-up (barrier init, descriptor prefetch, TMEM
+// allocation) before grid_dep_wait(), which returns once the predecessor grid
+// has completed and its memory is visible; every global read or write of
+// data that another kernel produces or consumes comes after it.  A kernel
+// signals grid_dep_launch() only after its own TMEM allocation, so a
+// dependent CTA that allocates before its wait never holds columns that a
+// not-yet-started CTA of the predecessor needs.  Without the launch attribute
+// both instructions are no-ops.
+__device__ inline void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t st, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace ot

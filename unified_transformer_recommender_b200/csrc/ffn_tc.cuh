@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tD = tmem, tU = tmem + 256;
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == 16) {
     // ------------------------------------------------------------ producer
@@ -520,7 +522,7 @@ inline onetrans_status tc_ffn_launch(const FfnDesc& d, cudaStream_t st) {
     attr_set = true;
   }
   dim3 grid((unsigned)((d.M + C::BM - 1) / C::BM), (unsigned)d.G);
-  ffn_tc_kernel<<<grid, kFfnThreads, C::SMEM, st>>>(ta, two, tw1, tw2, tres, tout, thout, d, a_swap, io);
+  launch_dependent(ffn_tc_kernel, grid, dim3(kFfnThreads), C::SMEM, st, ta, two, tw1, tw2, tres, tout, thout, d, a_swap, io);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 

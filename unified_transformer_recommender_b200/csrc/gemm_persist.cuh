@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(PersistCfg::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();
+  grid_dep_launch();
 
   // tile -> (first output column, first row, fixed coordinate), n fastest
   auto coords = [&](int tile, int& n0, int& mt0, int& g) {
@@ -252,8 +254,8 @@ inline onetrans_status tc_persist_launch(const GemmDesc& d, cudaStream_t st) {
   if (n_tiles <= 0) return ONETRANS_OK;
   if (n_tiles > 0x7fffffff) return ONETRANS_ERR_SHAPE;
   const int grid = (int)std::min<long long>(n_tiles, device_sm_count());
-  gemm_persist_kernel<<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, tout, d, a_swap, out_swap, tiles_n, tiles_m,
-                                                         (int)n_tiles);
+  launch_dependent(gemm_persist_kernel, dim3(grid), dim3(C::THREADS), C::SMEM, st, ta, tb, tout, d, a_swap,
+                   out_swap, tiles_n, tiles_m, (int)n_tiles);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 

@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == 4) {
     if (lane == 0) {
@@ -282,7 +284,7 @@ inline onetrans_status tc_gemm_launch_bn(const GemmDesc& d, cudaStream_t st) {
   const int out_tma = make_gemm_out_tmap(&tout, d, BN, C::STAGES * C::STAGE_BYTES, out_swap) ? 1 : 0;
   if (!out_tma) tout = ta;
   dim3 grid((unsigned)(d.N / BN), (unsigned)((d.M + 127) / 128), (unsigned)d.G);
-  gemm_tc_kernel<BN><<<grid, 192, C::SMEM, st>>>(ta, tb, tout, d, a_swap, out_tma, out_swap);
+  launch_dependent(gemm_tc_kernel<BN>, grid, dim3(192), C::SMEM, st, ta, tb, tout, d, a_swap, out_tma, out_swap);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 

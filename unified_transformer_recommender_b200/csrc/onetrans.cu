@@ -305,8 +305,11 @@ static onetrans_status rms_flat(const onetrans_model* m, const void* src, bool s
   const T* gm = (const T*)gamma;
   const float eps = m->cfg.rms_eps;
 #define OT_RMS_FLAT(CH)                                                                                   \
-  if (src_f32) rms_flat_kernel<T, float, CH><<<blocks, 256, 0, st>>>((const float*)src, y, gm, rows, eps); \
-  else rms_flat_kernel<T, T, CH><<<blocks, 256, 0, st>>>((const T*)src, y, gm, rows, eps);
+  if (src_f32)                                                                                            \
+    launch_dependent(rms_flat_kernel<T, float, CH>, dim3(blocks), dim3(256), 0, st, (const float*)src, y, gm, \
+                     rows, eps);                                                                             \
+  else                                                                                                     \
+    launch_dependent(rms_flat_kernel<T, T, CH>, dim3(blocks), dim3(256), 0, st, (const T*)src, y, gm, rows, eps);
   switch (ch) {
     case 1: OT_RMS_FLAT(1) break;
     case 2: OT_RMS_FLAT(2) break;
@@ -768,8 +771,8 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     for (int t = 0; t < w.n_types; ++t)
       w_aligned = w_aligned && (uintptr_t)w.W1[t] % 16 == 0 && (uintptr_t)w.W2[t] % 16 == 0;
     if (d == kEvD && w.e_dim <= kEvEmax && w.e_dim % 8 == 0 && w_aligned)
-      event_tokenize_tile_kernel<T><<<(unsigned)cdiv(R, kEvBlock), kEvD, 0, st>>>(
-          (const T*)events, types, (int)R, dL, w, rmap32(xa, (long long)dL * d, d));
+      launch_dependent(event_tokenize_tile_kernel<T>, dim3((unsigned)cdiv(R, kEvBlock)), dim3(kEvD), 0, st,
+                       (const T*)events, types, (int)R, dL, w, rmap32(xa, (long long)dL * d, d));
     else
       event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>(
           (const T*)events, types, dL, w, rmap32(xa, (long long)dL * d, d));

@@ -129,6 +129,8 @@ template <typename T, typename S, int CH>
 __global__ void __launch_bounds__(256) rms_flat_kernel(const S* __restrict__ src, T* __restrict__ dst,
                                                        const T* __restrict__ gamma, long long rows, float eps) {
   constexpr int D = CH * 128;
+  grid_dep_wait();
+  grid_dep_launch();
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int lane = threadIdx.x & 31;
@@ -384,6 +386,8 @@ __global__ void __launch_bounds__(256) event_tokenize_tile_kernel(const T* ev, c
   __shared__ __align__(16) float se[kEvBlock][kEvEmax];
   __shared__ __align__(16) float shid[kEvBlock][kEvD];
   __shared__ int sty[kEvBlock];
+  grid_dep_wait();
+  grid_dep_launch();
   const int r0 = blockIdx.x * kEvBlock;
   const int k = threadIdx.x;
   for (int idx = threadIdx.x; idx < kEvBlock * w.e_dim; idx += blockDim.x) {
