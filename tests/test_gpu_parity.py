@@ -401,6 +401,37 @@ def test_kv_serving_full_size_sampled():
             assert rel_err(out[c], r) <= TOL["bf16"]
 
 
+def test_kv_serving_pipeline_matches_one_stream():
+    """The benchmark's serving pipeline (batch k+1's auto-split and Stage I on
+    side streams before batch k's Stage II; two banks of cache and NS
+    tokens) reproduces, bit for bit, each batch run alone on one stream."""
+    import bench
+    wk = bench.KVServing(0)
+    m, main, n = wk.model, torch.cuda.current_stream(), 5
+    refs = []
+    cache = ot.Cache(m, wk.U, wk.wl.L_S)
+    ns, out = torch.empty_like(wk.ns[0]), torch.empty_like(wk.out)
+    for i in range(n):
+        wk.set_inputs(i)
+        ot.onetrans_tokenize_autosplit(m, wk.F, ns, wk.ws_a)
+        ot.onetrans_stage1_encode(m, cache, wk.slots, wk.S, wk.ws_1)
+        ot.onetrans_stage2_score(m, cache, wk.slots, wk.offs, ns, out, wk.ws_2)
+        refs.append(out.clone())
+    got = []
+    for i in range(n):
+        wk.set_inputs(i)
+        wk.front(i, main)
+        if i >= 1:
+            wk.back(i - 1, main)
+            got.append(wk.out.clone())
+    wk.back(n - 1, main)
+    got.append(wk.out.clone())
+    torch.cuda.synchronize()
+    for i in range(n):
+        assert torch.equal(got[i], refs[i]), i
+    assert not torch.equal(refs[0], refs[1])
+
+
 def test_s_forward_full_size_sampled():
     wl, b = _full("s_forward")
     sh = wl.shape
