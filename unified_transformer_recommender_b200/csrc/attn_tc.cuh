@@ -82,6 +82,7 @@ __device__ inline float ex2(float x) {
   return y;
 }
 
+
 template <int DH>
 __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
@@ -321,20 +322,29 @@ __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
         m = mt;
       }
       const float mref = (m == -INFINITY) ? 0.f : m;
-      float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;
+      // P = 2^(S - m) pair by pair: the subtraction and the row sums on packed
+      // fp32 pairs (half the issue slots), the exponentials on the MUFU
+      const uint64_t nm2 = f2_pack(-mref, -mref);
+      uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
       uint32_t pk[64];
 #pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        const float p0 = ex2(sv[2 * i] - mref), p1 = ex2(sv[2 * i + 1] - mref);
-        const float p2 = ex2(sv[2 * i + 2] - mref), p3 = ex2(sv[2 * i + 3] - mref);
-        ps0 += p0;
-        ps1 += p1;
-        ps2 += p2;
-        ps3 += p3;
-        pk[i] = pack_bf16x2(p0, p1);
-        pk[i + 1] = pack_bf16x2(p2, p3);
+      for (int i = 0; i < 64; ++i) {
+        const uint64_t x2 = f2_add(f2_pack(sv[2 * i], sv[2 * i + 1]), nm2);
+        float xa, xb;
+        f2_unpack(x2, xa, xb);
+        const uint64_t p2 = f2_pack(ex2(xa), ex2(xb));
+        if (i & 1) acc1 = f2_add(acc1, p2);
+        else acc0 = f2_add(acc0, p2);
+        float pa, pb;
+        f2_unpack(p2, pa, pb);
+        pk[i] = pack_bf16x2(pa, pb);
       }
-      l = l * alpha + ((ps0 + ps1) + (ps2 + ps3));
+      {
+        float s0, s1, s2, s3;
+        f2_unpack(acc0, s0, s1);
+        f2_unpack(acc1, s2, s3);
+        l = l * alpha + ((s0 + s1) + (s2 + s3));
+      }
       // P of the previous tile must be consumed before this one overwrites it
       if (kt > 0) {
         ok = mbar_wait(p_free, (kt - 1) & 1);

@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float2 bf = __bfloat1622float2(*(const __nv_bfloat162*)&bu[i]);
-          pk[i] = pack_bf16x2(gelu_fast(v[2 * i] + bf.x), gelu_fast(v[2 * i + 1] + bf.y));
+          pk[i] = gelu_bias_bf16x2(v[2 * i], v[2 * i + 1], bf.x, bf.y);
         }
         tmem_st8(col, pk);
         tmem_st_wait();

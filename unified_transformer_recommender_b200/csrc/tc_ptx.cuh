@@ -245,6 +245,33 @@ __device__ inline void umma_commit(uint64_t* bar) {
 
 // GELU, tanh form, with the hardware tanh approximation (relative error about
 // 2^-11, below the bf16 rounding of the values it produces).
+// ---- packed fp32 pairs: sm_100 executes add / sub / mul / fma on .f32x2
+// operands (two fp32 lanes in a 64-bit register pair) as one instruction,
+// halving the issue slots of elementwise fp32 work.
+__device__ inline uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ inline void f2_unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ inline uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ inline uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ inline uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 __device__ inline float tanh_fast(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -255,6 +282,19 @@ __device__ inline float gelu_fast(float x) {
   const float k0 = 0.7978845608028654f, k01 = 0.7978845608028654f * 0.044715f;
   const float hx = 0.5f * x;
   return fmaf(hx, tanh_fast(x * fmaf(k01, x * x, k0)), hx);
+}
+// The same for a pair (x0, x1) = (a0 + b0, a1 + b1), returned as bf16x2: the
+// fp32 arithmetic on packed pairs, the two tanh on the MUFU.
+__device__ inline uint32_t gelu_bias_bf16x2(float a0, float a1, float b0, float b1) {
+  const float k0 = 0.7978845608028654f, k01 = 0.7978845608028654f * 0.044715f;
+  const uint64_t x = f2_add(f2_pack(a0, a1), f2_pack(b0, b1));
+  const uint64_t hx = f2_mul(x, f2_pack(0.5f, 0.5f));
+  const uint64_t u = f2_mul(x, f2_fma(f2_pack(k01, k01), f2_mul(x, x), f2_pack(k0, k0)));
+  float u0, u1;
+  f2_unpack(u, u0, u1);
+  float g0, g1;
+  f2_unpack(f2_fma(hx, f2_pack(tanh_fast(u0), tanh_fast(u1)), hx), g0, g1);
+  return pack_bf16x2(g0, g1);
 }
 
 // -------------------------------------------------------- bf16 vectors --
