@@ -76,6 +76,12 @@ __device__ inline int kv_page_id(const KVStore& kv, int b, int page_idx) {
   return kv.table ? kv.table[kv.row_off[b] + page_idx] : b * kv.pps + page_idx;
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input max.f32)
+__device__ inline float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 __device__ inline float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -301,14 +307,14 @@ __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
 #pragma unroll
         for (int i = 0; i < 128; ++i) sv[i] = (i >= lo && i < hi) ? sv[i] : -INFINITY;
       }
-      // tile max over four independent chains
-      float mq0 = sv[0], mq1 = sv[1], mq2 = sv[2], mq3 = sv[3];
+      // tile max over four independent chains of three-input maxima
+      float mq0 = -INFINITY, mq1 = -INFINITY, mq2 = -INFINITY, mq3 = -INFINITY;
 #pragma unroll
-      for (int i = 4; i < 128; i += 4) {
-        mq0 = fmaxf(mq0, sv[i]);
-        mq1 = fmaxf(mq1, sv[i + 1]);
-        mq2 = fmaxf(mq2, sv[i + 2]);
-        mq3 = fmaxf(mq3, sv[i + 3]);
+      for (int i = 0; i < 128; i += 8) {
+        mq0 = fmax3(mq0, sv[i], sv[i + 1]);
+        mq1 = fmax3(mq1, sv[i + 2], sv[i + 3]);
+        mq2 = fmax3(mq2, sv[i + 4], sv[i + 5]);
+        mq3 = fmax3(mq3, sv[i + 6], sv[i + 7]);
       }
       const float mt = fmaxf(fmaxf(mq0, mq1), fmaxf(mq2, mq3));
       // raise the reference only when this tile passes it by more than 2^kThresh
