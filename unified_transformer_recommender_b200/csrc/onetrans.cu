@@ -14,6 +14,7 @@
 #include "simt.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_persist.cuh"
+#include "gemm_bres.cuh"
 #include "attn_tc.cuh"
 #include "ffn_tc.cuh"
 
@@ -221,6 +222,10 @@ static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, c
   if (cdiv(d.M, 64) > 65535 || d.G > 65535) return ONETRANS_ERR_SHAPE;
   ProfScope prof(kind, 2.0 * d.M * d.G * (double)d.N * d.K, gemm_bytes(m, d), st);
   if (m->bf16 && g_policy == 0 && tc_gemm_supported(d)) {
+    if (tc_bres_supported(d)) {
+      const onetrans_status r = tc_bres_launch(d, device_sm_count(), st);
+      if (r != ONETRANS_ERR_UNSUPPORTED) return r;
+    }
     if (tc_persist_supported(d)) {
       const onetrans_status r = tc_persist_launch(d, st);
       if (r != ONETRANS_ERR_UNSUPPORTED) return r;
