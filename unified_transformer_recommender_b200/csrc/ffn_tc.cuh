@@ -405,6 +405,19 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       if (io.out_tma) st_sw128_f32(stage_x, c0 >> 5, r, v);
       else if (valid && ok) store_row32(d.out, rm_off(d.out, b, t, c0), v);
     }
+    // x_next leaves first, so its stores drain while the next layer's
+    // RMSNorm is computed from the staged copy (reads only) into stage_h
+    if (io.out_tma) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("bar.sync 1, 512;" ::: "memory");
+      if (threadIdx.x == 0 && ok) {
+        for (int i = 0; i < 8; ++i) {
+          if (io.out_swap) tma_store_3d(&tmOut, stage_x + i * 16384, i * 32, g, mt0);
+          else tma_store_3d(&tmOut, stage_x + i * 16384, i * 32, mt0, g);
+        }
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+    }
     if (d.hout.base) {
       const float r2 = rsqrtf(row_sum(ss) / C::D + d.eps);
 #pragma unroll
@@ -426,27 +439,20 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         if (io.hout_tma) st_sw128_32(stage_h, 16384, r, c0, v);
         else if (valid && ok) store_row32(d.hout, rm_off(d.hout, b, t, c0), v);
       }
-    }
-    if (io.out_tma || io.hout_tma) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      asm volatile("bar.sync 1, 512;" ::: "memory");
-      if (threadIdx.x == 0 && ok) {
-        if (io.out_tma) {
-          for (int i = 0; i < 8; ++i) {
-            if (io.out_swap) tma_store_3d(&tmOut, stage_x + i * 16384, i * 32, g, mt0);
-            else tma_store_3d(&tmOut, stage_x + i * 16384, i * 32, mt0, g);
-          }
-        }
-        if (io.hout_tma && d.hout.base) {
+      if (io.hout_tma) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("bar.sync 1, 512;" ::: "memory");
+        if (threadIdx.x == 0 && ok) {
           for (int i = 0; i < 4; ++i) {
             if (io.hout_swap) tma_store_3d(&tmHout, stage_h + i * 16384, i * 64, g, mt0);
             else tma_store_3d(&tmHout, stage_h + i * 16384, i * 64, mt0, g);
           }
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         }
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       }
     }
+    // shared memory must stay valid until the stores have read it
+    if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
