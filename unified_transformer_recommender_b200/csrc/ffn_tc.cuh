@@ -251,13 +251,21 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
           free_stage();
         }
         umma_commit(dn_done);
-        // up(c+1) overwrites U: let down(c) finish reading it first
+        // up(c+1) overwrites U: let down(c) finish reading it first, then
+        // issue each k-block as soon as its W1 stage is in (the later stages
+        // arrive while the first k-blocks run)
         if (ok && c + 1 < NC) {
-          ok = wait_ahead(w1b) && mbar_wait(dn_done, c & 1);
-          if (ok) {
-            tc_fence_after();
-            up(w1b);
+          ok = mbar_wait(dn_done, c & 1);
+          for (int j = 0; j < 4 && ok; ++j) {
+            uint64_t wb;
+            ok = wait_stage(wb);
+            if (!ok) break;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16(tU, desc_add(dA, j * 16384 + k * 32), desc_add(wb, k * 32), id256, (j | k) ? 1u : 0u);
+            free_stage();
           }
+          if (ok) umma_commit(u_full);
         }
       }
       umma_commit(d_done);
