@@ -1,7 +1,7 @@
 // Tensor-core attention for the bf16 path (sm_100a), head dims 64 and 96.
 //
 // One CTA owns 128 query rows of one head.  K/V tiles of 128 keys are
-// streamed by TMA through a 2-deep shared-memory ring.  Per key tile:
+// streamed by TMA through a 3-stage shared-memory ring.  Per key tile:
 //   S = Q K^T          tcgen05.mma into TMEM (fp32)
 //   softmax            four warps read their query row back with tcgen05.ld
 //                      (one row per thread, so the row max and sum stay in the

@@ -10,8 +10,10 @@
 // accumulators (256 columns each), so the MMAs of tile i+1 run while eight
 // epilogue warps drain tile i: tcgen05.ld, bias / GELU / column scale, bf16
 // into a shared-memory staging tile, TMA stores.  This hides the load latency
-// and the epilogue that a one-tile-per-CTA kernel pays per tile, which
-// matters most for short K (the QKV projection has K = d = 256: 4 k-blocks).
+// and the epilogue that a one-tile-per-CTA kernel pays per tile.  Row-output
+// GEMMs with K = 256 (the QKV projection) take the weight-resident kernel of
+// gemm_bres.cuh; this one takes the others (the auto-split's K = 512 and
+// 3072 among them).
 //
 // Warp roles (320 threads): warps 0-7 epilogue (warp w and w+4 share TMEM
 // lanes 32*(w%4).. and take one half of the tile's columns each), warp 8
