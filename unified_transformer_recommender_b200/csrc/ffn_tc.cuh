@@ -129,6 +129,41 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tD = tmem, tU = tmem + 256;
+  // Ring stages in the order they are consumed: the residual rows (RP), W^O
+  // (4 k-blocks), W1 of chunk 0 (4), then W2(c) (4) and W1(c+1) (4) chunk by
+  // chunk.  Stage q goes to slot q % STAGES.
+  const int n_stages = RP + 8 + NC * 4 + (NC - 1) * 4;
+  auto issue_stage = [&](int q, uint64_t keep, uint64_t stream) {
+    const int s = q % C::STAGES;
+    uint8_t* dst = sW + s * C::STAGE;
+    mbar_expect_tx(&w_full[s], C::STAGE);
+    if (q < RP) {                    // residual rows, columns of part q
+      const int bc = io.res_f32 ? 32 : 64;
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx) {
+        const int col = (2 * q + bx) * bc;
+        if (io.res_swap) tma_load_3d_hint(&tmRes, &w_full[s], dst + bx * 16384, col, g, mt0, stream);
+        else tma_load_3d_hint(&tmRes, &w_full[s], dst + bx * 16384, col, mt0, g, stream);
+      }
+    } else if (q < RP + 4) {         // W^O k-block j: [256 out x 64]
+      tma_load_3d_hint(&tmWo, &w_full[s], dst, (q - RP) * 64, 0, 0, keep);
+    } else if (q < RP + 8) {         // W1 chunk 0, k-block j: [256 hidden x 64]
+      tma_load_3d_hint(&tmW1, &w_full[s], dst, (q - RP - 4) * 64, 0, grp, keep);
+    } else {
+      const int t = q - RP - 8, c = t >> 3, j = t & 3;
+      if ((t & 7) < 4)               // W2 chunk c, hidden block j: [256 out x 64 hidden]
+        tma_load_3d_hint(&tmW2, &w_full[s], dst, c * C::HC + j * C::HB, 0, grp, keep);
+      else                           // W1 chunk c + 1, k-block j
+        tma_load_3d_hint(&tmW1, &w_full[s], dst, j * 64, (c + 1) * C::HC, grp, keep);
+    }
+  };
+  // The weights, and the residual rows (written at least two launches back),
+  // are final before the previous kernel ends; only the attention rows come
+  // from it.  So the first ring stages load before the wait for that kernel.
+  if (warp == 16 && lane == 0) {
+    const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
+    for (int q = 0; q < C::STAGES && q < n_stages; ++q) issue_stage(q, keep, stream);
+  }
   grid_dep_wait();
   grid_dep_launch();
 
@@ -142,38 +177,10 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         if (a_swap) tma_load_3d_hint(&tmA, a_full, sA + kb * 16384, kb * 64, g, mt0, stream);
         else tma_load_3d_hint(&tmA, a_full, sA + kb * 16384, kb * 64, mt0, g, stream);
       }
-      int q = 0;  // ring stage counter, in the order the stages are consumed
-      auto stage = [&](int kind, int c, int j) -> bool {
+      for (int q = C::STAGES; q < n_stages; ++q) {
         const int s = q % C::STAGES;
-        if (q >= C::STAGES && !mbar_wait(&w_empty[s], ((q / C::STAGES) - 1) & 1)) return false;
-        uint8_t* dst = sW + s * C::STAGE;
-        mbar_expect_tx(&w_full[s], C::STAGE);
-        if (kind == 3) {          // residual rows, columns of part j
-          const int bc = io.res_f32 ? 32 : 64;
-#pragma unroll
-          for (int bx = 0; bx < 2; ++bx) {
-            const int col = (2 * j + bx) * bc;
-            if (io.res_swap) tma_load_3d_hint(&tmRes, &w_full[s], dst + bx * 16384, col, g, mt0, stream);
-            else tma_load_3d_hint(&tmRes, &w_full[s], dst + bx * 16384, col, mt0, g, stream);
-          }
-        } else if (kind == 0) {   // W^O k-block j: [256 out x 64]
-          tma_load_3d_hint(&tmWo, &w_full[s], dst, j * 64, 0, 0, keep);
-        } else if (kind == 1) {   // W1 chunk c, k-block j: [256 hidden x 64]
-          tma_load_3d_hint(&tmW1, &w_full[s], dst, j * 64, c * C::HC, grp, keep);
-        } else {                  // W2 chunk c, hidden block j: [256 out x 64 hidden]
-          tma_load_3d_hint(&tmW2, &w_full[s], dst, c * C::HC + j * C::HB, 0, grp, keep);
-        }
-        ++q;
-        return true;
-      };
-      bool ok = true;
-      for (int j = 0; j < RP && ok; ++j) ok = stage(3, 0, j);
-      for (int j = 0; j < 4 && ok; ++j) ok = stage(0, 0, j);
-      for (int j = 0; j < 4 && ok; ++j) ok = stage(1, 0, j);
-      for (int c = 0; c < NC && ok; ++c) {
-        for (int j = 0; j < C::HC / C::HB && ok; ++j) ok = stage(2, c, j);
-        if (c + 1 < NC)
-          for (int j = 0; j < 4 && ok; ++j) ok = stage(1, c + 1, j);
+        if (!mbar_wait(&w_empty[s], ((q / C::STAGES) - 1) & 1)) break;
+        issue_stage(q, keep, stream);
       }
     }
   } else if (warp == 17) {
