@@ -432,6 +432,42 @@ def test_kv_serving_pipeline_matches_one_stream():
     assert not torch.equal(refs[0], refs[1])
 
 
+def test_append_pipeline_matches_serial():
+    """The benchmark's append pipeline (batch k+1's append and auto-split on
+    side streams before batch k's Stage II, each batch on its own prepared
+    cache) gives, bit for bit, what the same batches give run one after
+    another on one stream."""
+    import bench
+    n = 4
+    wk = bench.Append(0, users=16, cands=32)
+    main = torch.cuda.current_stream()
+    wk.prepare(2 * n)
+    # every batch its own candidates and events, so a batch that read another
+    # batch's bank or cache would show
+    F0, ev0 = wk.F, wk.ev
+    Fs = [torch.roll(F0, 37 * i, 0).contiguous() for i in range(n)]
+    evs = [torch.roll(ev0, i, 0).contiguous() for i in range(n)]
+    serial = []
+    for i in range(n):
+        wk.F, wk.ev = Fs[i], evs[i]
+        wk.front(i, main, serial=True)
+        wk.back(i, main)
+        serial.append(wk.out.clone())
+    got = []
+    for i in range(n):
+        wk.F, wk.ev = Fs[i], evs[i]
+        wk.front(i, main)
+        if i >= 1:
+            wk.back(i - 1, main)
+            got.append(wk.out.clone())
+    wk.back(n - 1, main)
+    got.append(wk.out.clone())
+    torch.cuda.synchronize()
+    for i in range(n):
+        assert torch.equal(got[i], serial[i]), i
+    assert torch.isfinite(serial[0]).all() and not torch.equal(serial[0], serial[1])
+
+
 def test_s_forward_full_size_sampled():
     wl, b = _full("s_forward")
     sh = wl.shape
