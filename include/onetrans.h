@@ -213,8 +213,10 @@ ONETRANS_API onetrans_status onetrans_stage1_encode(const onetrans_model* m,
  * owns candidates cand_offsets[u] .. cand_offsets[u+1]-1 (host CSR, U+1
  * entries) and cache slot slots[u] (host).  Per layer, NS token j of a
  * candidate attends in one softmax to the slot's cached S keys and its own
- * NS keys 0..j, then passes through its token-specific FFN.  All slots must
- * hold the same S length; at most 65536 users per call.
+ * NS keys 0..j, then passes through its token-specific FFN.  Slots may hold
+ * different S lengths (encoded by separate Stage I calls): each user's layers
+ * then see that user's own pyramid schedule of cached keys.  A slot with no
+ * cached sequence is ONETRANS_ERR_SHAPE.  At most 65536 users per call.
  *   ns_tokens [C_tot, L_NS, d] (candidate-major, as the tokenizer writes it);
  *   ns_out    [C_tot, L_NS, d] float32. */
 ONETRANS_API onetrans_status onetrans_stage2_score(const onetrans_model* m,

@@ -151,6 +151,38 @@ def test_stage1_stage2_small_ragged(dtype, policy):
             assert rel_err(out[c], r) <= TOL[dtype], (u, c)
 
 
+@pytest.mark.parametrize("dtype,policy,pyr", [("bf16", 0, None), ("bf16", 0, [150, 80, 12]),
+                                              ("bf16", 1, None), ("fp32", 0, None)])
+def test_stage2_users_of_different_lengths(dtype, policy, pyr):
+    """Users encoded by separate Stage I calls with different S lengths are
+    scored in one Stage II call; each user's layers see its own cached keys
+    (all layers without a pyramid, layer 0 with a fixed-count pyramid)."""
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=3)
+    b = build(sh, 109, dtype, pyramid=pyr)
+    m = b.model
+    Ls = [200, 139, 257]
+    slots = [2, 0, 1]
+    cache = ot.Cache(m, 3, max(Ls) + 64)
+    S = [gen_normal(20 + u, (L, sh.d), dtype) for u, L in enumerate(Ls)]
+    for u, L in enumerate(Ls):
+        ot.onetrans_stage1_encode(m, cache, [slots[u]], to_dev(S[u][None], tdt(dtype)),
+                                  m.workspace(ot.OP_STAGE1, 1, L))
+    counts = [5, 3, 7]
+    offs = np.concatenate([[0], np.cumsum(counts)]).tolist()
+    NS = gen_normal(30, (offs[-1], sh.L_NS, sh.d), dtype)
+    out = torch.empty(offs[-1], sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
+    ot.onetrans_stage2_score(m, cache, slots, offs, to_dev(NS, tdt(dtype)), out,
+                             m.workspace(ot.OP_STAGE2, offs[-1], max(Ls)))
+    torch.cuda.synchronize()
+    out = to_np(out)
+    for u in range(3):
+        assert cache.length(slots[u]) == Ls[u]
+        kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, pyr)
+        for c in range(offs[u], offs[u + 1]):
+            assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL[dtype], (u, c)
+
+
 @pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
 def test_append_small_crosses_page_boundary(dtype, policy):
     ot.onetrans_set_kernel_policy(policy)

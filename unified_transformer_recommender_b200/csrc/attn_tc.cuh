@@ -42,6 +42,7 @@ struct TcAttnArgs {
   const int* tiles;   // {user, c0, c1} per blockIdx.x
   __nv_bfloat16* o2;  // [C_tot, L_NS, d]
   int L_NS, s_len;
+  const int* s_len_u;  // cached S keys per user, or null: s_len for all
   // shared
   KVStore kv;
   int H;
@@ -159,8 +160,8 @@ __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
     const int c1 = a.tiles[blockIdx.x * 3 + 2];
     row0 = c0 * a.L_NS;
     n_rows = (c1 - c0) * a.L_NS;
-    kmax = a.s_len - 1;
-    n_keys_s = a.s_len;
+    n_keys_s = a.s_len_u ? a.s_len_u[b] : a.s_len;
+    kmax = n_keys_s - 1;
     nt = (n_keys_s + C::BN - 1) / C::BN + 1;  // + the tile of own NS keys
   }
   const int nt_s = (n_keys_s + C::BN - 1) / C::BN;  // tiles from the KV pages
@@ -501,6 +502,7 @@ inline onetrans_status tc_stage2_launch(const Stage2Desc& a, int n_tiles, cudaSt
   args.o2 = (__nv_bfloat16*)a.o;
   args.L_NS = a.L_NS;
   args.s_len = a.s_len;
+  args.s_len_u = a.s_len_u;
   args.kv = a.kv;
   args.H = a.H;
   dim3 grid((unsigned)n_tiles, (unsigned)a.H, 1);

@@ -79,6 +79,8 @@ struct AttnDesc {
 // Rows are candidate-major: row c*L_NS + j is NS token j of candidate c.
 struct Stage2Desc {
   int H, dh, L_NS, C_tot, s_len, n_users;
+  const int* s_len_u;  // cached S keys of each user at this layer (device, [n_users]), or null: s_len for all
+  double s_sum;        // sum over candidates of their user's cached S keys (profiling)
   const int* tiles;    // n_tiles x {user, c0, c1}
   const void* qkv;     // [C_tot, L_NS, 3d] Q|K|V of the NS rows
   void* o;             // [C_tot, L_NS, d]

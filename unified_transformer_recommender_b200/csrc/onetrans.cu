@@ -272,7 +272,7 @@ static onetrans_status launch_stage2_attn(const onetrans_model* m, const Stage2D
   if (n_tiles <= 0) return ONETRANS_OK;
   // per candidate: token j sees s_len + j + 1 keys; bytes: the users' cached
   // K/V once each, Q/K/V of the NS rows, the output
-  const double pairs = (double)a.C_tot * (a.L_NS * (double)a.s_len + 0.5 * a.L_NS * (a.L_NS + 1));
+  const double pairs = a.L_NS * a.s_sum + (double)a.C_tot * 0.5 * a.L_NS * (a.L_NS + 1);
   const double es = m->es;
   ProfScope prof(PK_ATTN_STAGE2, 4.0 * a.dh * a.H * pairs,
                  a.n_users * 2.0 * a.s_len * a.H * a.dh * es + (double)a.L_NS * a.C_tot * a.H * a.dh * es * 4, st);
@@ -629,6 +629,27 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   const int L_S = need ? L_S_need : (U > 0 ? c->len[slots[0]] : 0);
   std::vector<int> s, sq;
   OT_TRY(s_rows_of(m, L_S, s, sq));
+  // users may hold different cached lengths: each has its own schedule, so
+  // its cached S keys per layer go into a table [NL][U] the attention reads
+  bool ragged = false;
+  std::vector<int> s_tab_h;
+  std::vector<double> s_sum(m->NL, 0.0);
+  std::vector<int> s_max(m->NL, 0);
+  if (!need) {
+    s_tab_h.assign((size_t)m->NL * U, 0);
+    for (int u = 0; u < U; ++u) {
+      const int Lu = c->len[slots[u]];
+      ragged = ragged || Lu != L_S;
+      std::vector<int> su, squ;
+      OT_TRY(s_rows_of(m, Lu, su, squ));
+      const double cu = (double)(offs[u + 1] - offs[u]);
+      for (int n = 0; n < m->NL; ++n) {
+        s_tab_h[(size_t)n * U + u] = su[n];
+        s_sum[n] += cu * su[n];
+        s_max[n] = std::max(s_max[n], su[n]);
+      }
+    }
+  }
   long long max_tiles = need ? cdiv(C, 64) + std::min<long long>(C, kMaxUsers) : 0;
   Carve cv(ws, ws_bytes);
   void* xa = cv.take((size_t)L_NS * C * d * 4);   // residual stream: float32
@@ -641,6 +662,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   void* hid = cv.take((size_t)L_NS * C * dff * es);
   int* row_off = (int*)cv.take((size_t)kMaxUsers * sizeof(int));
   int* d_tiles = (int*)cv.take((size_t)std::max<long long>(max_tiles, 1) * 3 * sizeof(int));
+  int* d_s_tab = (int*)cv.take((size_t)m->NL * kMaxUsers * sizeof(int));
   if (need) { *need = cv.used; return ONETRANS_OK; }
   if (cv.overflow) return ONETRANS_ERR_CAPACITY;
   if (C == 0) return ONETRANS_OK;
@@ -662,6 +684,8 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   for (int u = 0; u < U; ++u) h_row_off[u] = slots[u] * m->NL * c->max_pages;
   OT_TRY(cuda_ok(cudaMemcpyAsync(row_off, h_row_off.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
   OT_TRY(cuda_ok(cudaMemcpyAsync(d_tiles, tiles.data(), tiles.size() * sizeof(int), cudaMemcpyHostToDevice, st)));
+  if (ragged)
+    OT_TRY(cuda_ok(cudaMemcpyAsync(d_s_tab, s_tab_h.data(), s_tab_h.size() * sizeof(int), cudaMemcpyHostToDevice, st)));
 
   OT_TRY(rms_flat<T>(m, ns_in, false, h, (long long)L_NS * C, m->g_attn[0], st));
   const void* x_in = ns_in;
@@ -680,7 +704,10 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     OT_TRY(launch_gemm<T>(m, g, st));
     Stage2Desc a;
     std::memset(&a, 0, sizeof(a));
-    a.H = m->H; a.dh = m->dh; a.L_NS = L_NS; a.C_tot = (int)C; a.s_len = s[n]; a.n_users = U;
+    a.H = m->H; a.dh = m->dh; a.L_NS = L_NS; a.C_tot = (int)C; a.n_users = U;
+    a.s_len = ragged ? s_max[n] : s[n];
+    a.s_len_u = ragged ? d_s_tab + (size_t)n * U : nullptr;
+    a.s_sum = ragged ? s_sum[n] : (double)C * s[n];
     a.tiles = d_tiles; a.qkv = qkv; a.o = at;
     kv_for_cache(c, n, row_off, a.kv);
    
@@ -1125,9 +1152,8 @@ onetrans_status onetrans_stage2_score(const onetrans_model* m, const onetrans_ca
   for (int u = 0; u < U; ++u)
     if (cand_offsets[u + 1] < cand_offsets[u]) return ONETRANS_ERR_SHAPE;
   if (cand_offsets[0] != 0) return ONETRANS_ERR_SHAPE;
-  const int L_S = c->len[slots[0]];
   for (int u = 0; u < U; ++u)
-    if (c->len[slots[u]] != L_S || L_S == 0) return ONETRANS_ERR_SHAPE;
+    if (c->len[slots[u]] == 0) return ONETRANS_ERR_SHAPE;
   if (cand_offsets[U] == 0) return ONETRANS_OK;  // no candidates
   if (!ns_tokens || !ns_out || !aligned(ns_tokens, 16) || !aligned(ns_out, 16)) return ONETRANS_ERR_INVALID_ARG;
   OT_TRY(check_ws(ws));

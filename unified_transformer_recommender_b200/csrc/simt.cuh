@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(64) stage2_attn_simt_kernel(Stage2Desc a) {
   const int user = a.tiles[blockIdx.x * 3 + 0];
   const int c = a.tiles[blockIdx.x * 3 + 1] + tid;
   const bool valid = c < a.tiles[blockIdx.x * 3 + 2];
+  const int s_len = a.s_len_u ? a.s_len_u[user] : a.s_len;
   const int d = a.H * DH;
   const long long rs = 3LL * d;  // row stride of the packed Q|K|V rows
   const T* qkv = (const T*)a.qkv;
@@ -246,12 +247,12 @@ __global__ void __launch_bounds__(64) stage2_attn_simt_kernel(Stage2Desc a) {
   for (int e = 0; e < DH; ++e) { q[e] = valid ? to_f(qp[e]) : 0.f; o[e] = 0.f; }
   float mrow = -INFINITY, lrow = 0.f;
   const T* pool = (const T*)a.kv.pool;
-  for (int k0 = 0; k0 < a.s_len; k0 += KT) {
+  for (int k0 = 0; k0 < s_len; k0 += KT) {
     __syncthreads();
     for (int i = tid; i < KT * DH; i += 64) {
       const int r = i / DH, e = i - r * DH, pos = k0 + r;
       float kv = 0.f, vv = 0.f;
-      if (pos < a.s_len) {
+      if (pos < s_len) {
         kv = to_f(pool[kv_off(a.kv, user, pos, 0, h, e)]);
         vv = to_f(pool[kv_off(a.kv, user, pos, 1, h, e)]);
       }
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(64) stage2_attn_simt_kernel(Stage2Desc a) {
     float mt = -INFINITY;
     for (int r = 0; r < KT; ++r) {
       float s = -INFINITY;
-      if (k0 + r < a.s_len) {
+      if (k0 + r < s_len) {
         s = 0.f;
 #pragma unroll
         for (int e = 0; e < DH; ++e) s = fmaf(q[e], Ks[r][e], s);
