@@ -229,8 +229,11 @@ ONETRANS_API onetrans_status onetrans_stage2_score(const onetrans_model* m,
 /* Cross-request append ([FR] 7.5.3): tokenize dL new events per user with the
  * per-behavior MLP plus type identifier, run only those rows through every
  * layer (keys: cached + new, causal), and append their K/V to slots[u].
- * Non-pyramid models only (UNSUPPORTED otherwise).  All slots must hold the
- * same length.  events [U, dL, event_dim]; types [U, dL] int32 (device). */
+ * Non-pyramid models only (UNSUPPORTED otherwise).  Slots may hold
+ * different lengths: user u's events take positions len(slots[u]) ..
+ * len(slots[u]) + dL - 1.  A slot with no cached sequence is
+ * ONETRANS_ERR_SHAPE.  events [U, dL, event_dim]; types [U, dL] int32
+ * (device). */
 ONETRANS_API onetrans_status onetrans_cache_append(const onetrans_model* m,
                                       onetrans_cache* c, const int32_t* slots,
                                       int32_t U, const void* events,

@@ -184,6 +184,46 @@ def test_stage2_users_of_different_lengths(dtype, policy, pyr):
 
 
 @pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
+def test_append_users_of_different_lengths(dtype, policy):
+    """One append call for users whose slots hold different lengths: each
+    user's events take the positions after its own cached rows (crossing a
+    page boundary for two of them); cache rows and Stage II scores against
+    the oracle."""
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=2)
+    b = build(sh, 111, dtype, event_dim=64)
+    m = b.model
+    Ls, dL, slots = [60, 45, 62], 7, [0, 2, 1]
+    cache = ot.Cache(m, 3, 128)
+    S = [gen_normal(40 + u, (L, sh.d), dtype) for u, L in enumerate(Ls)]
+    for u, L in enumerate(Ls):
+        ot.onetrans_stage1_encode(m, cache, [slots[u]], to_dev(S[u][None], tdt(dtype)),
+                                  m.workspace(ot.OP_STAGE1, 1, L))
+    ev = gen_normal(50, (3, dL, 64), dtype)
+    ty = random_types(51, (3, dL), 3)
+    ot.onetrans_cache_append(m, cache, slots, to_dev(ev, tdt(dtype)), torch.from_numpy(ty).cuda(),
+                             m.workspace(ot.OP_APPEND, 3, dL))
+    counts = [2, 3, 1]
+    offs = np.concatenate([[0], np.cumsum(counts)]).tolist()
+    NS = gen_normal(52, (offs[-1], sh.L_NS, sh.d), dtype)
+    out = torch.empty(offs[-1], sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
+    ot.onetrans_stage2_score(m, cache, slots, offs, to_dev(NS, tdt(dtype)), out,
+                             m.workspace(ot.OP_STAGE2, offs[-1], max(Ls) + dL))
+    torch.cuda.synchronize()
+    out = to_np(out)
+    for u in range(3):
+        assert cache.length(slots[u]) == Ls[u] + dL
+        new = O.tokenize_events(ev[u], ty[u], b.W)
+        kv = O.append(O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS), new, b.W, sh.n_heads, EPS)
+        for n, (K, V) in enumerate(kv):
+            got = to_np(cache.gather(slots[u], n, Ls[u] + dL))
+            assert rel_err(got[0], K) <= TOL[dtype], (u, n)
+            assert rel_err(got[1], V) <= TOL[dtype], (u, n)
+        for c in range(offs[u], offs[u + 1]):
+            assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL[dtype], (u, c)
+
+
+@pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
 def test_append_small_crosses_page_boundary(dtype, policy):
     ot.onetrans_set_kernel_policy(policy)
     sh = shape(n_layers=2)

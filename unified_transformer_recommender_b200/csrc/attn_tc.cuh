@@ -37,6 +37,7 @@ struct TcAttnArgs {
   int mode;
   // causal
   int Lq, q_pos0;
+  const int* q_pos0_u;  // per batch, or null: q_pos0 for all
   RowMap o;
   // stage II
   const int* tiles;   // {user, c0, c1} per blockIdx.x
@@ -146,12 +147,13 @@ __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
 
   // ---- work of this CTA
   int b, row0, n_keys_s, kmax, nt, n_rows = C::BM;
-  int c0 = 0;
+  int c0 = 0, q_pos0 = a.q_pos0;
   if (a.mode == MODE_CAUSAL) {
     b = blockIdx.z;
+    if (a.q_pos0_u) q_pos0 = a.q_pos0_u[b];
     row0 = blockIdx.x * C::BM;
     const int t_last = min(a.Lq, row0 + C::BM) - 1;
-    kmax = a.q_pos0 + t_last;
+    kmax = q_pos0 + t_last;
     n_keys_s = kmax + 1;
     nt = (n_keys_s + C::BN - 1) / C::BN;
   } else {
@@ -271,10 +273,10 @@ __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
     // ------------------------------------------------- softmax + epilogue
     const int r = warp * 32 + lane;
     const uint32_t lb = (uint32_t)(warp * 32) << 16;
-    const int qpos = a.q_pos0 + row0 + r;  // causal: last visible key of this row
+    const int qpos = q_pos0 + row0 + r;  // causal: last visible key of this row
     const int cand = a.mode == MODE_STAGE2 ? r / a.L_NS : 0;
     const int tok = a.mode == MODE_STAGE2 ? r - cand * a.L_NS : 0;
-    const int qpos_min = a.q_pos0 + row0;  // earliest query of the CTA: bounds the unmasked tiles
+    const int qpos_min = q_pos0 + row0;  // earliest query of the CTA: bounds the unmasked tiles
     // Running max m is only raised when a tile's max exceeds it by more than
     // 2^8 (then O and l are rescaled); below that, P = 2^(S - m) <= 256 is
     // exact enough in bf16 and the final O / l is unchanged.
@@ -473,6 +475,7 @@ inline onetrans_status tc_attn_launch(const AttnDesc& a, cudaStream_t st) {
   args.mode = MODE_CAUSAL;
   args.Lq = a.Lq;
   args.q_pos0 = a.q_pos0;
+  args.q_pos0_u = a.q_pos0_u;
   args.o = a.o;
   args.kv = a.kv;
   args.H = a.H;

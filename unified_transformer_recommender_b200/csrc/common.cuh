@@ -40,6 +40,7 @@ struct KVStore {
   const int* row_off;
   int P, H, dh, pps;
   int pos_off;  // written position = t + pos_off
+  const int* pos_off_u;  // or, when set (device, per batch b): t + pos_off_u[b]
   int n_pages;  // pages in the pool (extent of the page dimension)
 };
 
@@ -71,6 +72,7 @@ struct GemmDesc {
 // epilogue), so q.k is already a base-2 logit.
 struct AttnDesc {
   int B, H, dh, Lq, q_pos0;  // query t of batch b sits at key position q_pos0 + t
+  const int* q_pos0_u;       // or, when set (device, per batch b): q_pos0_u[b] + t
   RowMap q, o;                // columns: head h occupies [h*dh, (h+1)*dh)
   KVStore kv;
 };

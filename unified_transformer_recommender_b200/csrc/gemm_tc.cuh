@@ -158,7 +158,8 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
       if (d.out_kind == OUT_KV) {
         const int dm = d.kv.H * d.kv.dh;
         const int kind = n / dm, cc = n - kind * dm, head = cc / d.kv.dh, e = cc - head * d.kv.dh;
-        store_bf16x32((__nv_bfloat16*)d.kv.pool + kv_off(d.kv, b, t + d.kv.pos_off, kind, head, e), v);
+        const int p0 = d.kv.pos_off_u ? d.kv.pos_off_u[b] : d.kv.pos_off;
+        store_bf16x32((__nv_bfloat16*)d.kv.pool + kv_off(d.kv, b, t + p0, kind, head, e), v);
       } else if (out_tma) {
         // every MMA is done: the stage buffers stage the tile for TMA stores
         if (d.out.f32) st_sw128_f32(smem, c0 >> 5, r, v);

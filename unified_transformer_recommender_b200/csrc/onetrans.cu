@@ -763,29 +763,37 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
   void* h2 = cv.take((size_t)R * d * es);
   void* hid = cv.take((size_t)R * dff * es);
   int* row_off = (int*)cv.take((size_t)std::max(U, 1) * sizeof(int));
+  int* d_pos0 = (int*)cv.take((size_t)std::max(U, 1) * sizeof(int));
   if (need) { *need = cv.used; return ONETRANS_OK; }
   if (cv.overflow) return ONETRANS_ERR_CAPACITY;
   if (U == 0 || dL == 0) return ONETRANS_OK;
-  const int s_old = c->len[slots[0]];
-  const int s_new = s_old + dL;
-  if (s_new > c->max_L_S) return ONETRANS_ERR_CAPACITY;
-  // pages for positions [s_old, s_new) of every layer
-  long long needed = 0;
-  for (int u = 0; u < U; ++u) needed += (long long)m->NL * (cdiv(s_new, P) - cdiv(s_old, P));
+  // user u's new rows take positions [s_old[u], s_old[u] + dL); users may
+  // hold different lengths (then the positions go to the kernels as a table)
+  std::vector<int> s_old(U);
+  bool ragged = false;
+  long long needed = 0, sum_old = 0;
+  for (int u = 0; u < U; ++u) {
+    s_old[u] = c->len[slots[u]];
+    if (s_old[u] + dL > c->max_L_S) return ONETRANS_ERR_CAPACITY;
+    ragged = ragged || s_old[u] != s_old[0];
+    sum_old += s_old[u];
+    needed += (long long)m->NL * (cdiv(s_old[u] + dL, P) - cdiv(s_old[u], P));
+  }
   if (needed > (long long)c->free_pages.size()) return ONETRANS_ERR_CAPACITY;
   std::vector<int> h_row_off(U);
   for (int u = 0; u < U; ++u) {
     const size_t row = (size_t)slots[u] * m->NL * c->max_pages;
     for (int n = 0; n < m->NL; ++n)
-      for (long long p = cdiv(s_old, P); p < cdiv(s_new, P); ++p) {
+      for (long long p = cdiv(s_old[u], P); p < cdiv(s_old[u] + dL, P); ++p) {
         c->h_table[row + (size_t)n * c->max_pages + p] = c->free_pages.back();
         c->free_pages.pop_back();
       }
-    c->len[slots[u]] = s_new;
+    c->len[slots[u]] = s_old[u] + dL;
     h_row_off[u] = (int)row;
     OT_TRY(upload_slot_table(c, slots[u], st));
   }
   OT_TRY(cuda_ok(cudaMemcpyAsync(row_off, h_row_off.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
+  if (ragged) OT_TRY(cuda_ok(cudaMemcpyAsync(d_pos0, s_old.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
 
   EventMLP w;
   std::memset(&w, 0, sizeof(w));
@@ -817,7 +825,8 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     void* x_next = (n % 2 == 0) ? xb : xa;
     KVStore kv;
     kv_for_cache(c, n, row_off, kv);
-    kv.pos_off = s_old;
+    kv.pos_off = s_old[0];
+    kv.pos_off_u = ragged ? d_pos0 : nullptr;
     GemmDesc g = gdesc_base(m);
     g.mode = TILE_FLAT; g.M = (int)R; g.fold = dL; g.G = 1;
     g.K = d; g.A = h; g.a_sm = d; g.a_mext = R; g.a_gext = 1;
@@ -831,10 +840,13 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
     OT_TRY(launch_gemm<T>(m, g, st));
     AttnDesc a;
     std::memset(&a, 0, sizeof(a));
-    a.B = U; a.H = m->H; a.dh = m->dh; a.Lq = dL; a.q_pos0 = s_old;
+    a.B = U; a.H = m->H; a.dh = m->dh; a.Lq = dL;
+    // the mean old length when they differ: used only for the profiling counts
+    a.q_pos0 = ragged ? (int)(sum_old / U) : s_old[0];
+    a.q_pos0_u = ragged ? d_pos0 : nullptr;
     a.q = rmap(q, (long long)dL * d, d);
     a.o = rmap(at, (long long)dL * d, d);
-    a.kv = kv; a.kv.pos_off = 0;
+    a.kv = kv; a.kv.pos_off = 0; a.kv.pos_off_u = nullptr;
     OT_TRY(launch_attn<T>(m, a, st));
     GemmDesc go = gdesc_base(m);
     go.mode = TILE_FLAT; go.M = (int)R; go.fold = dL; go.G = 1;
@@ -1176,9 +1188,8 @@ onetrans_status onetrans_cache_append(const onetrans_model* m, onetrans_cache* c
   if (U == 0 || dL == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
   if (!events || !types || !aligned(events, 16)) return ONETRANS_ERR_INVALID_ARG;
   OT_TRY(check_ws(ws));
-  const int L0 = c->len[slots[0]];
   for (int u = 0; u < U; ++u)
-    if (c->len[slots[u]] != L0 || L0 == 0) return ONETRANS_ERR_SHAPE;
+    if (c->len[slots[u]] == 0) return ONETRANS_ERR_SHAPE;
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? append_impl<__nv_bfloat16>(m, c, slots, U, events, types, dL, ws, ws_bytes, st, nullptr)
                  : append_impl<float>(m, c, slots, U, events, types, dL, ws, ws_bytes, st, nullptr);

@@ -18,7 +18,8 @@ __device__ inline void epilogue_store(const GemmDesc& d, int b, int t, int n, in
   if (d.out_kind == OUT_KV) {
     const int dm = d.kv.H * d.kv.dh;
     const int kind = n / dm, c = n - kind * dm, head = c / d.kv.dh, e = c - head * d.kv.dh;
-    ((T*)d.kv.pool)[kv_off(d.kv, b, t + d.kv.pos_off, kind, head, e)] = from_f<T>(v);
+    ((T*)d.kv.pool)[kv_off(d.kv, b, t + (d.kv.pos_off_u ? d.kv.pos_off_u[b] : d.kv.pos_off), kind, head, e)] =
+        from_f<T>(v);
   } else {
     rm_store<T>(d.out, rm_off(d.out, b, t, n), v);
   }
@@ -170,9 +171,10 @@ __global__ void __launch_bounds__(64) attn_simt_kernel(AttnDesc a) {
   const int tid = threadIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int t = blockIdx.x * 64 + tid;
   const bool valid = t < a.Lq;
-  const int p = a.q_pos0 + t;
+  const int q_pos0 = a.q_pos0_u ? a.q_pos0_u[b] : a.q_pos0;
+  const int p = q_pos0 + t;
   const int t_last = min(a.Lq, (int)(blockIdx.x + 1) * 64) - 1;
-  const int kmax = a.q_pos0 + t_last;
+  const int kmax = q_pos0 + t_last;
   float q[DH], o[DH];
   const T* qp = (const T*)a.q.base + rm_off(a.q, b, valid ? t : 0, h * DH);
 #pragma unroll
