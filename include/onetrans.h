@@ -199,6 +199,20 @@ ONETRANS_API onetrans_status onetrans_tokenize_autosplit_static(
     const onetrans_model* m, const void* feats, int64_t N, void* ns_tokens,
     void* stream);
 
+/* S-side tokenizer, timestamp-aware merge ([FR] 7.5.0): each event is
+ * aligned to d by the MLP of its behavior type (Linear e->d, GELU-tanh,
+ * Linear d->d) plus the type's additive identifier.  The caller lays the
+ * events of a user's behavior sequences out in time order (one flat row per
+ * event); the tokens then feed onetrans_stage1_encode or onetrans_forward.
+ *   events [R, event_dim] (the mode's element type); types [R] int32
+ *   (device, each in 0 .. n_behaviors-1; an out-of-range id sets the device
+ *   status word and is read as 0); tokens [R, d] (the mode's element type).
+ * UNSUPPORTED when the model has no behavior MLPs. */
+ONETRANS_API onetrans_status onetrans_tokenize_events(const onetrans_model* m,
+                                        const void* events,
+                                        const int32_t* types, int64_t R,
+                                        void* tokens, void* stream);
+
 /* Stage I ([FR] 7.5.3): run each user's S-tokens through the stack (pyramid
  * tail queries included) and store every layer's S-side K/V in cache slot
  * slots[u] (host array of U slot ids, distinct).  The slot's previous

@@ -223,6 +223,35 @@ def test_append_users_of_different_lengths(dtype, policy):
             assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL[dtype], (u, c)
 
 
+@pytest.mark.parametrize("dtype,d", [("bf16", 256), ("fp32", 256), ("bf16", 128)])
+def test_tokenize_events_then_stage1(dtype, d):
+    """S-side tokenizer: time-ordered events of several behavior types, each
+    through its type's MLP plus the type identifier, then Stage I on the
+    tokens; tokens and cached K/V against the oracle.  d = 256 takes the
+    tiled kernel, d = 128 the per-event one."""
+    sh = shape(n_layers=2, d=d, H=d // 64)
+    b = build(sh, 113, dtype, event_dim=64)
+    m = b.model
+    U, L = 3, 70
+    ev = gen_normal(60, (U, L, 64), dtype)
+    ty = random_types(61, (U, L), 3)
+    tok = torch.empty(U * L, d, dtype=tdt(dtype), device="cuda")
+    ot.onetrans_tokenize_events(m, to_dev(ev.reshape(U * L, 64), tdt(dtype)),
+                                torch.from_numpy(ty.reshape(-1)).cuda(), tok)
+    torch.cuda.synchronize()
+    assert ot.onetrans_device_status() == 0
+    ref = O.tokenize_events(ev, ty, b.W)
+    assert rel_err(to_np(tok).reshape(U, L, d), ref) <= TOL[dtype]
+    cache = ot.Cache(m, U, L)
+    ot.onetrans_stage1_encode(m, cache, list(range(U)), tok.view(U, L, d), m.workspace(ot.OP_STAGE1, U, L))
+    torch.cuda.synchronize()
+    for u in range(U):
+        kv = O.stage1(to_np(tok).reshape(U, L, d)[u], b.W, sh.L_NS, sh.n_heads, EPS)
+        for n, (K, V) in enumerate(kv):
+            got = to_np(cache.gather(u, n, L))
+            assert rel_err(got[0], K) <= TOL[dtype] and rel_err(got[1], V) <= TOL[dtype], (u, n)
+
+
 @pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
 def test_append_small_crosses_page_boundary(dtype, policy):
     ot.onetrans_set_kernel_policy(policy)

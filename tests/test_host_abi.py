@@ -22,7 +22,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 22
+    assert len(names) == 23
     for n in names:
         assert hasattr(ot.lib, n), n
     assert set(names) == set(ot.SYMBOLS)
@@ -181,6 +181,21 @@ def test_entry_point_argument_errors_before_any_launch():
     st, _, c2 = _cache(fm2, 4, 1178)
     assert ot.lib.onetrans_stage1_encode(fm.h, c2, slots, 2, FAKE, 1178, ws, big, None) == ot.ERR_INVALID_ARG
     ot.lib.onetrans_cache_destroy(c2)
+
+
+def test_tokenize_events_argument_errors_before_any_launch():
+    fm = FakeModel(n_beh=3, event_dim=64)
+    assert fm.status == ot.OK
+    # no events: nothing to do, the data pointers may be NULL
+    assert ot.lib.onetrans_tokenize_events(fm.h, None, None, 0, None, None) == ot.OK
+    assert ot.lib.onetrans_tokenize_events(fm.h, FAKE, FAKE, -1, FAKE, None) == ot.ERR_SHAPE
+    assert ot.lib.onetrans_tokenize_events(fm.h, FAKE + 2, FAKE, 8, FAKE, None) == ot.ERR_INVALID_ARG
+    assert ot.lib.onetrans_tokenize_events(fm.h, FAKE, FAKE, 8, FAKE + 8, None) == ot.ERR_INVALID_ARG
+    assert ot.lib.onetrans_tokenize_events(fm.h, FAKE, None, 8, FAKE, None) == ot.ERR_INVALID_ARG
+    assert ot.lib.onetrans_tokenize_events(None, FAKE, FAKE, 8, FAKE, None) == ot.ERR_INVALID_ARG
+    # a model without behavior MLPs has no event tokenizer
+    fm0 = FakeModel()
+    assert ot.lib.onetrans_tokenize_events(fm0.h, FAKE, FAKE, 8, FAKE, None) == ot.ERR_UNSUPPORTED
 
 
 def test_policy_and_status_strings():

@@ -31,7 +31,7 @@ SYMBOLS = (
     "onetrans_cache_append", "onetrans_forward", "onetrans_set_kernel_policy",
     "onetrans_device_status", "onetrans_status_string", "onetrans_version",
     "onetrans_profile_enable", "onetrans_profile_kinds", "onetrans_profile_read",
-    "onetrans_tokenize_autosplit_static",
+    "onetrans_tokenize_autosplit_static", "onetrans_tokenize_events",
 )
 
 
@@ -98,6 +98,7 @@ _sig("onetrans_tokenize_autosplit_static", I32, P, P, I64, P, P)
 _sig("onetrans_stage1_encode", I32, P, P, PI32, I32, P, I32, P, SZ, P)
 _sig("onetrans_stage2_score", I32, P, P, PI32, I32, PI32, P, P, P, SZ, P)
 _sig("onetrans_cache_append", I32, P, P, PI32, I32, P, P, I32, P, SZ, P)
+_sig("onetrans_tokenize_events", I32, P, P, P, I64, P, P)
 _sig("onetrans_forward", I32, P, P, I32, I32, P, P, SZ, P)
 _sig("onetrans_set_kernel_policy", I32, I32)
 _sig("onetrans_device_status", I32, P, PI32)
@@ -282,6 +283,13 @@ def onetrans_tokenize_autosplit_static(model: Model, feats: torch.Tensor, ns_tok
     """Auto-split without a workspace (scratch in the library's fixed array)."""
     _check("onetrans_tokenize_autosplit_static", lib.onetrans_tokenize_autosplit_static(
         model.handle, _ptr(feats), feats.shape[0], _ptr(ns_tokens), _stream(stream)))
+
+
+def onetrans_tokenize_events(model: Model, events: torch.Tensor, types: torch.Tensor, tokens: torch.Tensor,
+                             stream=None) -> None:
+    """events [R, event_dim], types [R] int32 (device), tokens [R, d]."""
+    _check("onetrans_tokenize_events", lib.onetrans_tokenize_events(
+        model.handle, _ptr(events), _ptr(types), events.shape[0], _ptr(tokens), _stream(stream)))
 
 
 def onetrans_stage1_encode(model: Model, cache: Cache, slots: Sequence[int], s_tokens: torch.Tensor,

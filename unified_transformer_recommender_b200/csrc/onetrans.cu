@@ -747,6 +747,41 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
 }
 
 // =============================================================== append ==
+// The per-behavior MLPs and type embedding of the event tokenizer.
+static EventMLP event_mlp_of(const onetrans_model* m) {
+  EventMLP w;
+  std::memset(&w, 0, sizeof(w));
+  for (int t = 0; t < m->cfg.n_behaviors; ++t) {
+    w.W1[t] = m->Wb1[t]; w.b1[t] = m->bb1[t]; w.W2[t] = m->Wb2[t]; w.b2[t] = m->bb2[t];
+  }
+  w.emb = m->type_emb; w.n_types = m->cfg.n_behaviors; w.e_dim = m->cfg.event_dim; w.d = m->d;
+  return w;
+}
+
+// Tokenize R events (rows of `events`, type ids on the device) into `out`
+// (row (r / dL, r % dL) of the row map).
+template <typename T>
+static onetrans_status launch_event_tokenizer(const onetrans_model* m, const void* events, const int* types,
+                                              long long R, int dL, const RowMap& out, cudaStream_t st) {
+  if (R <= 0) return ONETRANS_OK;
+  if (R > 0x7fffffff) return ONETRANS_ERR_SHAPE;
+  const EventMLP w = event_mlp_of(m);
+  const int d = m->d;
+  const size_t smem = (size_t)(w.e_dim + d) * sizeof(float);
+  // the scope of the profiling record is the tokenizer launch alone
+  ProfScope prof_tok(PK_TOKENIZE, 2.0 * R * ((double)w.e_dim * d + (double)d * d),
+                     (double)R * (w.e_dim * m->es + d * (out.f32 ? 4 : m->es)), st);
+  bool w_aligned = true;
+  for (int t = 0; t < w.n_types; ++t)
+    w_aligned = w_aligned && (uintptr_t)w.W1[t] % 16 == 0 && (uintptr_t)w.W2[t] % 16 == 0;
+  if (d == kEvD && w.e_dim <= kEvEmax && w.e_dim % 8 == 0 && w_aligned)
+    launch_dependent(event_tokenize_tile_kernel<T>, dim3((unsigned)cdiv(R, kEvBlock)), dim3(kEvD), 0, st,
+                     (const T*)events, types, (int)R, dL, w, out);
+  else
+    event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>((const T*)events, types, dL, w, out);
+  return last_launch();
+}
+
 template <typename T>
 static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, const int* slots, int U,
                                    const void* events, const int* types, int dL, void* ws,
@@ -795,29 +830,8 @@ static onetrans_status append_impl(const onetrans_model* m, onetrans_cache* c, c
   OT_TRY(cuda_ok(cudaMemcpyAsync(row_off, h_row_off.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
   if (ragged) OT_TRY(cuda_ok(cudaMemcpyAsync(d_pos0, s_old.data(), U * sizeof(int), cudaMemcpyHostToDevice, st)));
 
-  EventMLP w;
-  std::memset(&w, 0, sizeof(w));
-  for (int t = 0; t < m->cfg.n_behaviors; ++t) {
-    w.W1[t] = m->Wb1[t]; w.b1[t] = m->bb1[t]; w.W2[t] = m->Wb2[t]; w.b2[t] = m->bb2[t];
-  }
-  w.emb = m->type_emb; w.n_types = m->cfg.n_behaviors; w.e_dim = m->cfg.event_dim; w.d = d;
-  const size_t smem = (size_t)(w.e_dim + d) * sizeof(float);
   if (R > 0x7fffffff) return ONETRANS_ERR_SHAPE;
-  {
-    // the scope of the profiling record is the tokenizer launch alone
-    ProfScope prof_tok(PK_TOKENIZE, 2.0 * R * ((double)w.e_dim * d + (double)d * d),
-                       (double)R * (w.e_dim * m->es + d * 4), st);
-    bool w_aligned = true;
-    for (int t = 0; t < w.n_types; ++t)
-      w_aligned = w_aligned && (uintptr_t)w.W1[t] % 16 == 0 && (uintptr_t)w.W2[t] % 16 == 0;
-    if (d == kEvD && w.e_dim <= kEvEmax && w.e_dim % 8 == 0 && w_aligned)
-      launch_dependent(event_tokenize_tile_kernel<T>, dim3((unsigned)cdiv(R, kEvBlock)), dim3(kEvD), 0, st,
-                       (const T*)events, types, (int)R, dL, w, rmap32(xa, (long long)dL * d, d));
-    else
-      event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>(
-          (const T*)events, types, dL, w, rmap32(xa, (long long)dL * d, d));
-    OT_TRY(last_launch());
-  }
+  OT_TRY(launch_event_tokenizer<T>(m, events, types, R, dL, rmap32(xa, (long long)dL * d, d), st));
   OT_TRY(rms_flat<T>(m, xa, true, h, R, m->g_attn[0], st));
   const void* x_in = xa;
   for (int n = 0; n < m->NL; ++n) {
@@ -1193,6 +1207,20 @@ onetrans_status onetrans_cache_append(const onetrans_model* m, onetrans_cache* c
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? append_impl<__nv_bfloat16>(m, c, slots, U, events, types, dL, ws, ws_bytes, st, nullptr)
                  : append_impl<float>(m, c, slots, U, events, types, dL, ws, ws_bytes, st, nullptr);
+}
+
+onetrans_status onetrans_tokenize_events(const onetrans_model* m, const void* events, const int32_t* types,
+                                         int64_t R, void* tokens, void* stream) {
+  if (!m) return ONETRANS_ERR_INVALID_ARG;
+  if (m->cfg.n_behaviors < 1 || m->cfg.event_dim < 1 || m->Wb1.empty() || !m->type_emb)
+    return ONETRANS_ERR_UNSUPPORTED;
+  if (R < 0 || R > 0x7fffffff) return ONETRANS_ERR_SHAPE;
+  if (R == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!events || !types || !tokens || !aligned(events, 16) || !aligned(tokens, 16))
+    return ONETRANS_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? launch_event_tokenizer<__nv_bfloat16>(m, events, types, R, 1, rmap(tokens, m->d, m->d), st)
+                 : launch_event_tokenizer<float>(m, events, types, R, 1, rmap(tokens, m->d, m->d), st);
 }
 
 onetrans_status onetrans_forward(const onetrans_model* m, const void* x0, int32_t B, int32_t L_S, void* out,
