@@ -16,12 +16,14 @@
 //
 // Query kinds:
 //  * MODE_CAUSAL  (Stage I, forward, append): query t of sequence b sits at
-//    key position q_pos0 + t and sees keys 0..q_pos0 + t, all from 64-token
-//    KV-cache pages.  Only the tail rows are queries (the pyramid's Q set);
-//    keys span the layer input.
+//    key position q_pos0 + t (q_pos0_u[b] + t when the sequences' cached
+//    lengths differ, as in an append) and sees keys 0 .. that position, all
+//    from 64-token KV-cache pages.  Only the tail rows are queries (the
+//    pyramid's Q set); keys span the layer input.
 //  * MODE_STAGE2: rows are NS tokens of up to floor(128/L_NS) candidates of one
 //    user, candidate-major (row r = candidate r / L_NS, token r % L_NS).  They
-//    see every cached S key of the user, then one more key tile holding the
+//    see every cached S key of the user (s_len, or s_len_u[user] when users
+//    hold different lengths), then one more key tile holding the
 //    same candidates' own NS keys, masked to (same candidate, token <= own):
 //    one softmax over the union, every product on tensor cores.
 //
