@@ -194,6 +194,9 @@ class Model:
         h = P()
         _check("onetrans_model_create", lib.onetrans_model_create(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(h)))
         self.handle = h
+        # held by the object so that a model collected at interpreter exit,
+        # after the module's globals are cleared, can still be destroyed
+        self._destroy = lib.onetrans_model_destroy
         self.n_layers, self.d, self.L_NS = n_layers, d_model, L_NS
 
     def _own(self, t: torch.Tensor) -> torch.Tensor:
@@ -205,7 +208,7 @@ class Model:
     def __del__(self):
         h = getattr(self, "handle", None)
         if h is not None and h.value:
-            lib.onetrans_model_destroy(h)
+            self._destroy(h)
             self.handle = None
 
     def workspace_size(self, op: int, n: int, L: int = 0) -> int:
@@ -233,11 +236,12 @@ class Cache:
         _check("onetrans_cache_init", lib.onetrans_cache_init(model.handle, self.pool.data_ptr(), size.value,
                                                                 n_slots, max_L_S, ctypes.byref(h)))
         self.handle, self.model = h, model
+        self._destroy = lib.onetrans_cache_destroy
 
     def __del__(self):
         h = getattr(self, "handle", None)
         if h is not None and h.value:
-            lib.onetrans_cache_destroy(h)
+            self._destroy(h)
             self.handle = None
 
     def length(self, slot: int) -> int:
