@@ -314,3 +314,50 @@ def test_flop_counter_attention_matches_brute_force_mask_count():
             pairs += sum(1 for ki in range(L) if ki <= qi)
         L = Lq
     assert f["attn"] == 4 * d * pairs
+
+
+def test_flop_counter_projections_match_torch_flop_counter():
+    """Without a pyramid every row runs every projection; torch's own FLOP
+    counter over the textbook stack's linear layers must give the same count."""
+    from torch.utils.flop_counter import FlopCounterMode
+    shape, W = small_model(n_layers=2)
+    L_S = 8
+    X0 = gen_normal(21, (1, L_S + shape.L_NS, shape.d), "fp32")
+    with FlopCounterMode(display=False) as fc:
+        textbook_stack(X0, W, shape.n_heads, EPS)
+    counts = {str(k): v for k, v in fc.get_flop_counts()["Global"].items()}
+    mm = counts.get("aten.mm", 0) + counts.get("aten.addmm", 0)
+    f = flops.forward_flops(L_S, shape.L_NS, shape.d, shape.d_ff, shape.n_layers)
+    assert f["proj"] == mm
+
+
+@pytest.mark.parametrize("L_S,L_NS,N,L_min", [(13, 3, 3, 3), (40, 4, 5, 9), (7, 2, 1, 2), (30, 6, 4, None)])
+def test_stage_split_flops_add_up_to_one_pass(L_S, L_NS, N, L_min):
+    """[FR] 7.5.3: Stage I (S rows) plus Stage II of one candidate (NS rows)
+    does exactly the one-pass work, pyramid or not (NS rows are the tail, so
+    every layer keeps them).  The auto-split term is one multiply-add per
+    weight entry per candidate."""
+    d, d_ff, F_, H = 16, 48, 10, 24
+    sched = None if L_min is None else linear_pyramid(L_S + L_NS, L_min, N)
+    one = flops.forward_flops(L_S, L_NS, d, d_ff, N, sched)
+    s1 = flops.stage1_flops(L_S, L_NS, d, d_ff, N, sched)
+    s2 = flops.stage2_flops(L_S, L_NS, d, d_ff, N, F_, H, sched)
+    assert s1["proj"] + s2["proj"] == one["proj"]
+    assert s1["attn"] + s2["attn"] == one["attn"]
+    assert s2["tokenize"] == 2 * (H * F_ + L_NS * d * H)   # Wa1 [H, F], Wa2 [L_NS d, H]
+
+
+@pytest.mark.parametrize("L_old,dL,t", [(20, 5, 0), (1, 1, 2), (64, 17, 1)])
+def test_append_flops_equal_the_grown_stage1_minus_the_old(L_old, dL, t):
+    """An append of dL events costs what Stage I of the longer sequence costs
+    beyond Stage I of the old one (non-pyramid); its tokenizer term is one
+    multiply-add per weight entry of the event's per-behavior MLP per event."""
+    shape, W = small_model(n_layers=3)
+    d, N = shape.d, shape.n_layers
+    e = W["Wb1"][t].shape[1]
+    a = flops.append_flops(L_old, dL, d, shape.d_ff, N, e)
+    grown = flops.stage1_flops(L_old + dL, shape.L_NS, d, shape.d_ff, N)
+    old = flops.stage1_flops(L_old, shape.L_NS, d, shape.d_ff, N)
+    assert a["proj"] == grown["proj"] - old["proj"]
+    assert a["attn"] == grown["attn"] - old["attn"]
+    assert a["tokenize"] == 2 * dL * (W["Wb1"][t].size + W["Wb2"][t].size)
