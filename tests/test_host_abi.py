@@ -203,3 +203,27 @@ def test_policy_and_status_strings():
     assert ot.lib.onetrans_set_kernel_policy(0) == ot.OK
     assert ot.status_string(ot.ERR_CAPACITY) == "capacity exceeded"
     assert ot.status_string(123) == "unknown status"
+
+
+def test_model_left_alive_until_interpreter_exit_is_destroyed_cleanly(tmp_path):
+    """A model still referenced by a module global when the interpreter exits
+    is collected after the binding's module globals are cleared; its
+    destructor must still reach the library.  The weights are host tensors:
+    model creation only validates and records their addresses."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = tmp_path / "leave_alive.py"
+    script.write_text(
+        "import sys\n"
+        f"sys.path.insert(0, {root!r})\n"
+        "import unified_transformer_recommender_b200 as ot\n"
+        "from onetrans_synth import ModelShape, make_weights\n"
+        "sh = ModelShape(n_layers=2, d=256, n_heads=4, d_ff=1024, L_NS=2, ns_feat=16,\n"
+        "                ns_hidden=512, behavior_dims=(8,))\n"
+        "MODEL = ot.model_from_arrays(sh, make_weights(sh, 1, 'bf16'), device='cpu')\n"
+        "print('made', bool(MODEL.handle.value))\n")
+    r = subprocess.run([sys.executable, str(script)], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert "made True" in r.stdout
+    assert "Exception ignored" not in r.stderr, r.stderr
