@@ -213,6 +213,27 @@ ONETRANS_API onetrans_status onetrans_tokenize_events(const onetrans_model* m,
                                         const int32_t* types, int64_t R,
                                         void* tokens, void* stream);
 
+/* S-side tokenizer, timestamp-agnostic merge ([FR] 7.5.0): a user's n_seq
+ * behavior sequences, given in intent order (for example purchase, then
+ * add-to-cart, then click), are each aligned to d by their behavior's MLP
+ * (Linear e->d, GELU-tanh, Linear d->d; no type identifier) and laid out one
+ * after another with the learnable [SEP] vector between consecutive ones.
+ *   events [R, event_dim] (the mode's element type, device): the sequences'
+ *     events back to back, R = sum of seq_len;
+ *   seq_len [n_seq] int64, seq_type [n_seq] int32 (host): each sequence's
+ *     length (0 allowed) and behavior id (0 .. n_behaviors-1);
+ *   sep [d] (the mode's element type, device; may be NULL when n_seq = 1);
+ *   tokens [L_S, d] (the mode's element type, device), L_S = R + n_seq - 1:
+ *     sequence i at rows from (sum of earlier lengths) + i, its [SEP] right
+ *     after it.
+ * 1 <= n_seq <= 8, else SHAPE (below 1) or UNSUPPORTED (above 8); a negative
+ * length is SHAPE, an out-of-range behavior id INVALID_ARG, both before any
+ * launch.  UNSUPPORTED when the model has no behavior MLPs. */
+ONETRANS_API onetrans_status onetrans_merge_intent_order(
+    const onetrans_model* m, const void* events, const int64_t* seq_len,
+    const int32_t* seq_type, int32_t n_seq, const void* sep, void* tokens,
+    void* stream);
+
 /* Stage I ([FR] 7.5.3): run each user's S-tokens through the stack (pyramid
  * tail queries included) and store every layer's S-side K/V in cache slot
  * slots[u] (host array of U slot ids, distinct).  The slot's previous

@@ -22,7 +22,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 23
+    assert len(names) == 24
     for n in names:
         assert hasattr(ot.lib, n), n
     assert set(names) == set(ot.SYMBOLS)
@@ -196,6 +196,34 @@ def test_tokenize_events_argument_errors_before_any_launch():
     # a model without behavior MLPs has no event tokenizer
     fm0 = FakeModel()
     assert ot.lib.onetrans_tokenize_events(fm0.h, FAKE, FAKE, 8, FAKE, None) == ot.ERR_UNSUPPORTED
+
+
+def test_merge_intent_order_argument_errors_before_any_launch():
+    fm = FakeModel(n_beh=3, event_dim=64)
+    assert fm.status == ot.OK
+
+    def merge(m, events, lens, types, sep, tokens, n=None):
+        n = len(lens) if n is None else n
+        L = (ot.I64 * max(len(lens), 1))(*lens)
+        T = (ot.I32 * max(len(types), 1))(*types)
+        return ot.lib.onetrans_merge_intent_order(m, events, L, T, n, sep, tokens, None)
+
+    # one empty sequence: no rows at all, nothing launched, pointers may be NULL
+    assert merge(fm.h, None, [0], [1], None, None) == ot.OK
+    assert merge(fm.h, FAKE, [4, 3], [0, 1], FAKE, FAKE, n=0) == ot.ERR_SHAPE
+    assert merge(fm.h, FAKE, [1] * 9, [0] * 9, FAKE, FAKE) == ot.ERR_UNSUPPORTED   # above 8 sequences
+    assert merge(fm.h, FAKE, [4, -1], [0, 1], FAKE, FAKE) == ot.ERR_SHAPE
+    assert merge(fm.h, FAKE, [4, 3], [0, 3], FAKE, FAKE) == ot.ERR_INVALID_ARG     # behavior id out of range
+    assert merge(fm.h, FAKE, [4, 3], [0, -1], FAKE, FAKE) == ot.ERR_INVALID_ARG
+    assert merge(fm.h, FAKE, [4, 3], [0, 1], None, FAKE) == ot.ERR_INVALID_ARG     # two sequences need [SEP]
+    assert merge(fm.h, FAKE + 2, [4, 3], [0, 1], FAKE, FAKE) == ot.ERR_INVALID_ARG
+    assert merge(fm.h, FAKE, [4, 3], [0, 1], FAKE, FAKE + 8) == ot.ERR_INVALID_ARG
+    assert merge(fm.h, None, [4], [0], None, FAKE) == ot.ERR_INVALID_ARG           # events missing
+    assert merge(fm.h, FAKE, [2 ** 31], [0], None, FAKE) == ot.ERR_SHAPE
+    assert ot.lib.onetrans_merge_intent_order(fm.h, FAKE, None, None, 2, FAKE, FAKE, None) == ot.ERR_INVALID_ARG
+    assert merge(None, FAKE, [4, 3], [0, 1], FAKE, FAKE) == ot.ERR_INVALID_ARG
+    fm0 = FakeModel()
+    assert merge(fm0.h, FAKE, [4, 3], [0, 1], FAKE, FAKE) == ot.ERR_UNSUPPORTED
 
 
 def test_policy_and_status_strings():

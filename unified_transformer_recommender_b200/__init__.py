@@ -31,7 +31,7 @@ SYMBOLS = (
     "onetrans_cache_append", "onetrans_forward", "onetrans_set_kernel_policy",
     "onetrans_device_status", "onetrans_status_string", "onetrans_version",
     "onetrans_profile_enable", "onetrans_profile_kinds", "onetrans_profile_read",
-    "onetrans_tokenize_autosplit_static", "onetrans_tokenize_events",
+    "onetrans_tokenize_autosplit_static", "onetrans_tokenize_events", "onetrans_merge_intent_order",
 )
 
 
@@ -57,6 +57,7 @@ I64 = ctypes.c_int64
 SZ = ctypes.c_size_t
 PP = ctypes.POINTER(ctypes.c_void_p)
 PI32 = ctypes.POINTER(ctypes.c_int32)
+PI64 = ctypes.POINTER(ctypes.c_int64)
 
 
 class Config(ctypes.Structure):
@@ -99,6 +100,7 @@ _sig("onetrans_stage1_encode", I32, P, P, PI32, I32, P, I32, P, SZ, P)
 _sig("onetrans_stage2_score", I32, P, P, PI32, I32, PI32, P, P, P, SZ, P)
 _sig("onetrans_cache_append", I32, P, P, PI32, I32, P, P, I32, P, SZ, P)
 _sig("onetrans_tokenize_events", I32, P, P, P, I64, P, P)
+_sig("onetrans_merge_intent_order", I32, P, P, PI64, PI32, I32, P, P, P)
 _sig("onetrans_forward", I32, P, P, I32, I32, P, P, SZ, P)
 _sig("onetrans_set_kernel_policy", I32, I32)
 _sig("onetrans_device_status", I32, P, PI32)
@@ -294,6 +296,19 @@ def onetrans_tokenize_events(model: Model, events: torch.Tensor, types: torch.Te
     """events [R, event_dim], types [R] int32 (device), tokens [R, d]."""
     _check("onetrans_tokenize_events", lib.onetrans_tokenize_events(
         model.handle, _ptr(events), _ptr(types), events.shape[0], _ptr(tokens), _stream(stream)))
+
+
+def onetrans_merge_intent_order(model: Model, events: torch.Tensor, seq_len: Sequence[int],
+                                seq_type: Sequence[int], sep: Optional[torch.Tensor], tokens: torch.Tensor,
+                                stream=None) -> None:
+    """events [sum(seq_len), event_dim] (device), the sequences back to back in
+    intent order; seq_len / seq_type per sequence (host); sep [d] (device);
+    tokens [sum(seq_len) + len(seq_len) - 1, d]."""
+    n = len(seq_len)
+    lens = (I64 * max(n, 1))(*[int(v) for v in seq_len])
+    _check("onetrans_merge_intent_order", lib.onetrans_merge_intent_order(
+        model.handle, _ptr(events), lens, _i32(list(seq_type) or [0]), n, _ptr(sep), _ptr(tokens),
+        _stream(stream)))
 
 
 def onetrans_stage1_encode(model: Model, cache: Cache, slots: Sequence[int], s_tokens: torch.Tensor,

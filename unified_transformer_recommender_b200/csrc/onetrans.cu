@@ -759,13 +759,22 @@ static EventMLP event_mlp_of(const onetrans_model* m) {
 }
 
 // Tokenize R events (rows of `events`, type ids on the device) into `out`
-// (row (r / dL, r % dL) of the row map).
+// (row (r / dL, r % dL) of the row map).  With an intent layout (lay.n > 0)
+// the types come from the layout, output rows are shifted past the [SEP] gaps,
+// one more CTA writes the [SEP] rows, and `emb` decides whether the type
+// identifiers are added.
 template <typename T>
 static onetrans_status launch_event_tokenizer(const onetrans_model* m, const void* events, const int* types,
-                                              long long R, int dL, const RowMap& out, cudaStream_t st) {
-  if (R <= 0) return ONETRANS_OK;
-  if (R > 0x7fffffff) return ONETRANS_ERR_SHAPE;
-  const EventMLP w = event_mlp_of(m);
+                                              long long R, int dL, const RowMap& out, cudaStream_t st,
+                                              const IntentLayout* layout = nullptr, bool emb = true) {
+  IntentLayout lay;
+  std::memset(&lay, 0, sizeof(lay));
+  if (layout) lay = *layout;
+  const int n_sep = lay.n > 1 ? 1 : 0;
+  if (R < 0 || (R == 0 && !n_sep)) return ONETRANS_OK;
+  if (R + lay.n > 0x7fffffff) return ONETRANS_ERR_SHAPE;
+  EventMLP w = event_mlp_of(m);
+  if (!emb) w.emb = nullptr;
   const int d = m->d;
   const size_t smem = (size_t)(w.e_dim + d) * sizeof(float);
   // the scope of the profiling record is the tokenizer launch alone
@@ -775,10 +784,11 @@ static onetrans_status launch_event_tokenizer(const onetrans_model* m, const voi
   for (int t = 0; t < w.n_types; ++t)
     w_aligned = w_aligned && (uintptr_t)w.W1[t] % 16 == 0 && (uintptr_t)w.W2[t] % 16 == 0;
   if (d == kEvD && w.e_dim <= kEvEmax && w.e_dim % 8 == 0 && w_aligned)
-    launch_dependent(event_tokenize_tile_kernel<T>, dim3((unsigned)cdiv(R, kEvBlock)), dim3(kEvD), 0, st,
-                     (const T*)events, types, (int)R, dL, w, out);
+    launch_dependent(event_tokenize_tile_kernel<T>, dim3((unsigned)(cdiv(R, kEvBlock) + n_sep)), dim3(kEvD), 0,
+                     st, (const T*)events, types, (int)R, dL, w, out, lay);
   else
-    event_tokenize_kernel<T><<<(unsigned)R, std::min(d, 512), smem, st>>>((const T*)events, types, dL, w, out);
+    event_tokenize_kernel<T><<<(unsigned)(R + n_sep), std::min(d, 512), smem, st>>>((const T*)events, types, dL,
+                                                                                     w, out, lay);
   return last_launch();
 }
 
@@ -1221,6 +1231,38 @@ onetrans_status onetrans_tokenize_events(const onetrans_model* m, const void* ev
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? launch_event_tokenizer<__nv_bfloat16>(m, events, types, R, 1, rmap(tokens, m->d, m->d), st)
                  : launch_event_tokenizer<float>(m, events, types, R, 1, rmap(tokens, m->d, m->d), st);
+}
+
+onetrans_status onetrans_merge_intent_order(const onetrans_model* m, const void* events,
+                                            const int64_t* seq_len, const int32_t* seq_type, int32_t n_seq,
+                                            const void* sep, void* tokens, void* stream) {
+  if (!m) return ONETRANS_ERR_INVALID_ARG;
+  if (m->cfg.n_behaviors < 1 || m->cfg.event_dim < 1 || m->Wb1.empty()) return ONETRANS_ERR_UNSUPPORTED;
+  if (n_seq < 1) return ONETRANS_ERR_SHAPE;
+  if (n_seq > kMaxIntents) return ONETRANS_ERR_UNSUPPORTED;
+  if (!seq_len || !seq_type) return ONETRANS_ERR_INVALID_ARG;
+  IntentLayout lay;
+  std::memset(&lay, 0, sizeof(lay));
+  lay.n = n_seq;
+  lay.sep = sep;
+  long long R = 0;
+  for (int i = 0; i < n_seq; ++i) {
+    if (seq_len[i] < 0) return ONETRANS_ERR_SHAPE;
+    if (seq_type[i] < 0 || seq_type[i] >= m->cfg.n_behaviors) return ONETRANS_ERR_INVALID_ARG;
+    R += seq_len[i];
+    if (R + n_seq > 0x7fffffff) return ONETRANS_ERR_SHAPE;
+    lay.end[i] = (int)R;
+    lay.type[i] = seq_type[i];
+  }
+  const long long L_S = R + n_seq - 1;
+  if (L_S == 0) return ONETRANS_OK;  // one empty sequence: no work
+  if (!tokens || !aligned(tokens, 16) || (R > 0 && (!events || !aligned(events, 16))) || (n_seq > 1 && !sep))
+    return ONETRANS_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? launch_event_tokenizer<__nv_bfloat16>(m, events, nullptr, R, 1, rmap(tokens, m->d, m->d), st,
+                                                         &lay, false)
+                 : launch_event_tokenizer<float>(m, events, nullptr, R, 1, rmap(tokens, m->d, m->d), st, &lay,
+                                                 false);
 }
 
 onetrans_status onetrans_forward(const onetrans_model* m, const void* x0, int32_t B, int32_t L_S, void* out,

@@ -316,17 +316,63 @@ struct EventMLP {
   const void* b1[8];
   const void* W2[8];
   const void* b2[8];
-  const void* emb;
+  const void* emb;  // [n_types, d] additive type identifiers, or null for none
   int n_types, e_dim, d;
 };
 
+// Intent-order layout of a user's behavior sequences: sequence i holds the
+// flat input rows [end[i-1], end[i]) (end[-1] = 0), all of behavior type[i];
+// its tokens land at output rows shifted by i, so that output row end[i] + i
+// is left for the [SEP] vector after sequence i.  n = 0: no layout (per-row
+// types from the device array, output row = input row).
+constexpr int kMaxIntents = 8;
+struct IntentLayout {
+  int n;
+  int end[kMaxIntents];
+  int type[kMaxIntents];
+  const void* sep;  // [d], written at the n - 1 gap rows
+};
+
+__device__ __forceinline__ int intent_seq_of(const IntentLayout& lay, int row) {
+  int s = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxIntents - 1; ++i) s += (i < lay.n - 1 && lay.end[i] <= row) ? 1 : 0;
+  return s;
+}
+
+__device__ __forceinline__ int intent_type_of(const IntentLayout& lay, int s) {
+  int ty = lay.type[0];
+#pragma unroll
+  for (int i = 1; i < kMaxIntents; ++i) ty = (i == s) ? lay.type[i] : ty;
+  return ty;
+}
+
+// The [SEP] rows of a layout: one CTA, thread k writes column k of each.
 template <typename T>
-__global__ void event_tokenize_kernel(const T* ev, const int* types, int dL, EventMLP w, RowMap out) {
+__device__ __forceinline__ void intent_write_seps(const IntentLayout& lay, int d, int dL, const RowMap& out) {
+#pragma unroll
+  for (int i = 0; i < kMaxIntents - 1; ++i) {
+    if (i + 1 >= lay.n) break;
+    const int orow = lay.end[i] + i, bb = orow / dL, tt = orow - bb * dL;
+    for (int k = threadIdx.x; k < d; k += blockDim.x)
+      rm_store<T>(out, rm_off(out, bb, tt, k), to_f(((const T*)lay.sep)[k]));
+  }
+}
+
+template <typename T>
+__global__ void event_tokenize_kernel(const T* ev, const int* types, int dL, EventMLP w, RowMap out,
+                                      IntentLayout lay) {
   extern __shared__ float sm[];
   float* e = sm;              // [e_dim]
   float* hid = sm + w.e_dim;  // [d]
-  const int row = blockIdx.x, b = row / dL, t = row - b * dL;
-  int ty = types[row];
+  if (lay.n > 1 && blockIdx.x == gridDim.x - 1) {  // the extra block of a layout: its [SEP] rows
+    intent_write_seps<T>(lay, w.d, dL, out);
+    return;
+  }
+  const int row = blockIdx.x;
+  const int seq = lay.n ? intent_seq_of(lay, row) : 0;
+  const int orow = row + seq, b = orow / dL, t = orow - b * dL;
+  int ty = lay.n ? intent_type_of(lay, seq) : types[row];
   if (ty < 0 || ty >= w.n_types) {
     if (threadIdx.x == 0) flag_error(3);
     ty = 0;
@@ -344,7 +390,7 @@ __global__ void event_tokenize_kernel(const T* ev, const int* types, int dL, Eve
   for (int k = threadIdx.x; k < w.d; k += blockDim.x) {
     float s = to_f(((const T*)w.b2[ty])[k]);
     for (int i = 0; i < w.d; ++i) s = fmaf(to_f(W2[(long long)k * w.d + i]), hid[i], s);
-    s += to_f(((const T*)w.emb)[(long long)ty * w.d + k]);
+    if (w.emb) s += to_f(((const T*)w.emb)[(long long)ty * w.d + k]);
     rm_store<T>(out, rm_off(out, b, t, k), s);
   }
 }
@@ -385,12 +431,17 @@ __device__ inline void ev_fma8(float* acc, const float* wv, const float (*x)[LD]
 }
 template <typename T>
 __global__ void __launch_bounds__(256) event_tokenize_tile_kernel(const T* ev, const int* types, int R, int dL,
-                                                                  EventMLP w, RowMap out) {
+                                                                  EventMLP w, RowMap out, IntentLayout lay) {
   __shared__ __align__(16) float se[kEvBlock][kEvEmax];
   __shared__ __align__(16) float shid[kEvBlock][kEvD];
   __shared__ int sty[kEvBlock];
+  __shared__ int sseq[kEvBlock];
   grid_dep_wait();
   grid_dep_launch();
+  if (lay.n > 1 && blockIdx.x == gridDim.x - 1) {  // the extra CTA of a layout: its [SEP] rows
+    intent_write_seps<T>(lay, kEvD, dL, out);
+    return;
+  }
   const int r0 = blockIdx.x * kEvBlock;
   const int k = threadIdx.x;
   for (int idx = threadIdx.x; idx < kEvBlock * w.e_dim; idx += blockDim.x) {
@@ -398,12 +449,15 @@ __global__ void __launch_bounds__(256) event_tokenize_tile_kernel(const T* ev, c
     se[j][i] = (r0 + j < R) ? to_f(ev[(long long)(r0 + j) * w.e_dim + i]) : 0.f;
   }
   if (threadIdx.x < kEvBlock) {
-    int ty = (r0 + threadIdx.x < R) ? types[r0 + threadIdx.x] : 0;
+    const int row = r0 + threadIdx.x;
+    const int seq = (lay.n && row < R) ? intent_seq_of(lay, row) : 0;
+    int ty = row < R ? (lay.n ? intent_type_of(lay, seq) : types[row]) : 0;
     if (ty < 0 || ty >= w.n_types) {
       flag_error(3);
       ty = 0;
     }
     sty[threadIdx.x] = ty;
+    sseq[threadIdx.x] = seq;
   }
   __syncthreads();
   float acc[kEvBlock];
@@ -424,7 +478,7 @@ __global__ void __launch_bounds__(256) event_tokenize_tile_kernel(const T* ev, c
   __syncthreads();
   for (int t = 0; t < w.n_types; ++t) {
     const T* W2r = (const T*)w.W2[t] + (long long)k * kEvD;
-    const float b = to_f(((const T*)w.b2[t])[k]) + to_f(((const T*)w.emb)[(long long)t * kEvD + k]);
+    const float b = to_f(((const T*)w.b2[t])[k]) + (w.emb ? to_f(((const T*)w.emb)[(long long)t * kEvD + k]) : 0.f);
 #pragma unroll
     for (int j = 0; j < kEvBlock; ++j) acc[j] = b;
     for (int i0 = 0; i0 < kEvD; i0 += 8) {
@@ -436,7 +490,7 @@ __global__ void __launch_bounds__(256) event_tokenize_tile_kernel(const T* ev, c
     for (int j = 0; j < kEvBlock; ++j) {
       const int row = r0 + j;
       if (sty[j] == t && row < R) {
-        const int bb = row / dL, tt = row - bb * dL;
+        const int orow = row + sseq[j], bb = orow / dL, tt = orow - bb * dL;
         rm_store<T>(out, rm_off(out, bb, tt, k), acc[j]);
       }
     }
