@@ -29,7 +29,7 @@ Tokenizer weights:
 from __future__ import annotations
 
 import dataclasses
-from typing import Dict, List, Optional
+from typing import Dict, List, Optional, Sequence
 
 import numpy as np
 
@@ -200,6 +200,25 @@ def make_weights(shape: ModelShape, seed: int, dtype: str, event_dim: int = 0,
     W["bb2"] = [nrm(d) for _ in dims]
     W["type_emb"] = nrm(len(dims), d)
     W["sep"] = nrm(d)
+    return W
+
+
+def make_group_weights(d: int, group_dims: Sequence[int], group_hidden: Sequence[int], seed: int,
+                       dtype: str, std: float = 0.02) -> Dict[str, List[np.ndarray]]:
+    """Weights of a group-wise NS tokenizer, one two-layer MLP per feature group:
+    Wg1[g] [h_g, F_g], bg1[g] [h_g], Wg2[g] [d, h_g], bg2[g] [d], drawn group
+    by group from their own seed (the block-stack weights are untouched)."""
+    r = _rng(seed)
+
+    def nrm(*s):
+        return _finish(std * r.standard_normal(size=s, dtype=np.float64), dtype)
+
+    W: Dict[str, List[np.ndarray]] = {"Wg1": [], "bg1": [], "Wg2": [], "bg2": []}
+    for F_g, h_g in zip(group_dims, group_hidden):
+        W["Wg1"].append(nrm(h_g, F_g))
+        W["bg1"].append(nrm(h_g))
+        W["Wg2"].append(nrm(d, h_g))
+        W["bg2"].append(nrm(d))
     return W
 
 

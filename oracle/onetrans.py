@@ -198,6 +198,18 @@ def autosplit(feats: np.ndarray, W: Dict, L_NS: int) -> np.ndarray:
     return y.reshape(n, L_NS, y.shape[1] // L_NS)
 
 
+def tokenize_groupwise(groups: Sequence[np.ndarray], G: Dict) -> np.ndarray:
+    """Group-wise NS tokenizer ([PD] 2.1 "Unified Tokenization"; [LP] 3.1
+    "Non-Sequential Token (NS)"): the non-sequential features come split into
+    semantic groups (user profile, item attributes, ...); group g, its
+    features concatenated, goes through its own two-layer MLP and becomes NS
+    token g.  groups[g]: [N, F_g]; G: Wg1/bg1/Wg2/bg2 lists indexed by group.
+    Returns [N, L_NS, d] with L_NS = the number of groups."""
+    toks = [mlp2(x, G["Wg1"][g], G["bg1"][g], G["Wg2"][g], G["bg2"][g])
+            for g, x in enumerate(groups)]
+    return np.stack(toks, axis=1)
+
+
 def tokenize_events(events: np.ndarray, types: np.ndarray, W: Dict) -> np.ndarray:
     """Per-behavior MLP alignment plus an additive behavior-type identifier
     ([FR] 7.5.0, MLP_i(e_ij) and the timestamp-aware merge's type ids).

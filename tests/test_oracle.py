@@ -16,8 +16,8 @@ import torch
 import torch.nn.functional as F
 
 from onetrans_synth import (ModelShape, WORKLOADS, bf16_round, gen_normal,
-                            linear_pyramid, make_weights, random_types,
-                            tiny_raw_inputs)
+                            linear_pyramid, make_group_weights, make_weights,
+                            random_types, tiny_raw_inputs)
 from oracle import flops, onetrans as O
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -262,6 +262,43 @@ def test_autosplit_equals_concat_mlp_reshape():
         mlp[2].weight.copy_(t64(W["Wa2"])); mlp[2].bias.copy_(t64(W["ba2"]))
         ref = mlp(t64(feats)).view(5, shape.L_NS, shape.d).numpy()
     np.testing.assert_allclose(O.autosplit(feats, W, shape.L_NS), ref, rtol=1e-12, atol=1e-13)
+
+
+GROUP_DIMS, GROUP_HIDDEN = (10, 6, 8, 3), (12, 7, 16, 5)
+
+
+def test_groupwise_tokenizer_is_one_torch_mlp_per_group():
+    """[PD] 2.1, [LP] 3.1: group g through its own MLP gives NS token g."""
+    d = 9
+    G = make_group_weights(d, GROUP_DIMS, GROUP_HIDDEN, 60, "fp32", std=0.3)
+    groups = [gen_normal(61 + g, (5, F_g), "fp32") for g, F_g in enumerate(GROUP_DIMS)]
+    got = O.tokenize_groupwise(groups, G)
+    assert got.shape == (5, len(GROUP_DIMS), d)
+    for g, (F_g, h_g) in enumerate(zip(GROUP_DIMS, GROUP_HIDDEN)):
+        mlp = torch.nn.Sequential(torch.nn.Linear(F_g, h_g), torch.nn.GELU("tanh"),
+                                  torch.nn.Linear(h_g, d)).double()
+        with torch.no_grad():
+            mlp[0].weight.copy_(t64(G["Wg1"][g])); mlp[0].bias.copy_(t64(G["bg1"][g]))
+            mlp[2].weight.copy_(t64(G["Wg2"][g])); mlp[2].bias.copy_(t64(G["bg2"][g]))
+            ref = mlp(t64(groups[g])).numpy()
+        np.testing.assert_allclose(got[:, g], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_groupwise_tokenizer_is_autosplit_with_block_diagonal_weights():
+    """The two NS tokenizers of [PD] 2.1 meet: an auto-split MLP whose layers
+    are block-diagonal by group (group g's inputs feed only its hidden units,
+    which feed only output columns [g d, (g+1) d)) is the group-wise tokenizer,
+    GELU acting elementwise.  Token order and split direction must agree."""
+    from scipy.linalg import block_diag
+    d = 9
+    G = make_group_weights(d, GROUP_DIMS, GROUP_HIDDEN, 62, "fp32", std=0.3)
+    groups = [gen_normal(63 + g, (7, F_g), "fp32") for g, F_g in enumerate(GROUP_DIMS)]
+    W = {"Wa1": block_diag(*G["Wg1"]), "ba1": np.concatenate(G["bg1"]),
+         "Wa2": block_diag(*G["Wg2"]), "ba2": np.concatenate(G["bg2"])}
+    assert W["Wa1"].shape == (sum(GROUP_HIDDEN), sum(GROUP_DIMS))
+    assert W["Wa2"].shape == (len(GROUP_DIMS) * d, sum(GROUP_HIDDEN))
+    split = O.autosplit(np.concatenate(groups, axis=1), W, len(GROUP_DIMS))
+    np.testing.assert_allclose(O.tokenize_groupwise(groups, G), split, rtol=1e-12, atol=1e-14)
 
 
 def test_tokenize_events_per_type_mlp_plus_type_embedding():
