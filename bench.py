@@ -151,6 +151,64 @@ def peaks():
 
 # --------------------------------------------------------------- workload
 
+# ------------------------------------------------- workload descriptions
+# Shared by both arms, so that the reference arm's line names the same
+# metric, unit and config as this arm's.
+
+APPEND_METRIC = "users appended (dL=16 events) and their candidates scored per second on 1 B200"
+
+
+def forward_metric(name: str) -> str:
+    return f"samples/sec of the one-pass forward ({name}) on 1 B200"
+
+
+def kv_serving_config(U: int, C: int, ws: int) -> dict:
+    return {"workload": "kv_serving: auto-split + Stage I + Stage II; 6 layers d=256 4 heads FFN 1024, "
+                        f"pyramid queries 1190->12 (linear), {U} users x 1178 S tokens, {C} "
+                        "candidates/user, 12 NS tokens from 512 features", "users_per_gpu": U,
+            "candidates_per_gpu": U * C, "parallelism": f"users sharded over {ws} GPU(s), no collective",
+            "pipeline": "batch k+1's auto-split and Stage I (two side streams) are issued before batch k's "
+                        "Stage II; two banks of KV cache and NS tokens; the timed span covers the fill "
+                        "and the drain, so every batch counted is complete inside it",
+            "l2": "inputs larger than L2: the timed loops cycle 8 distinct input sets of 17.6 MB (141 MB); "
+                  "no flush between the overlapping steps"}
+
+
+def append_config(U: int, C: int, dL: int, ws: int) -> dict:
+    return {"workload": f"append: non-pyramid 6 layers d=256 4 heads FFN 1024, {U} users x 1178 cached "
+                        f"S tokens, append dL={dL} events (64-wide, 3 behavior types), then "
+                        f"{C} candidates/user (12 NS tokens from 512 features) scored over 1194 keys",
+            "users_per_gpu": U, "candidates_per_gpu": U * C,
+            "parallelism": f"users sharded over {ws} GPU(s), no collective",
+            "pipeline": "batch k+1's append and auto-split (two side streams) are issued before batch k's "
+                        "Stage II; the timed span covers the fill and the drain",
+            "l2": "inputs larger than L2: every step reads its own 1.9 GB cache; no flush between the "
+                  "overlapping steps"}
+
+
+def forward_config(name: str, U: int, ws: int) -> dict:
+    from onetrans_synth import WORKLOADS
+    wl = WORKLOADS[name]
+    sh = wl.shape
+    return {"workload": f"{name}: {sh.n_layers} layers d={sh.d} {sh.n_heads} heads FFN {sh.d_ff}, "
+                        f"{U} samples x ({wl.L_S} S + {sh.L_NS} NS tokens), pyramid "
+                        f"{wl.pyramid[0]}->{wl.pyramid[-1]} (linear)",
+            "samples_per_gpu": U, "parallelism": f"samples sharded over {ws} GPU(s), no collective",
+            "l2": "512 MB buffer written between timed steps (not timed)"}
+
+
+def workload_meta(name: str, ws: int):
+    """(metric, unit, config, units per GPU per step) of a workload at its
+    default size, without building it."""
+    from onetrans_synth import WORKLOADS
+    wl = WORKLOADS[name]
+    if name == "kv_serving":
+        return METRIC, UNIT, kv_serving_config(wl.users, wl.cands, ws), wl.users * wl.cands
+    if name == "append":
+        return APPEND_METRIC, "users/s", append_config(wl.users, wl.cands, wl.dL, ws), wl.users
+    return forward_metric(name), "samples/s", forward_config(name, wl.users, ws), wl.users
+
+
 class KVServing:
     """Auto-split + Stage I + Stage II for U users x C candidates, served as
     a pipeline: batch k's front (the candidates' auto-split on one side
@@ -248,15 +306,7 @@ class KVServing:
     io_names = ("S", "F")       # per-step inputs, uploaded from pinned host copies in the end-to-end leg
 
     def config(self, ws):
-        return {"workload": "kv_serving: auto-split + Stage I + Stage II; 6 layers d=256 4 heads FFN 1024, "
-                            f"pyramid queries 1190->12 (linear), {self.U} users x 1178 S tokens, {self.C} "
-                            "candidates/user, 12 NS tokens from 512 features", "users_per_gpu": self.U,
-                "candidates_per_gpu": self.units, "parallelism": f"users sharded over {ws} GPU(s), no collective",
-                "pipeline": "batch k+1's auto-split and Stage I (two side streams) are issued before batch k's "
-                            "Stage II; two banks of KV cache and NS tokens; the timed span covers the fill "
-                            "and the drain, so every batch counted is complete inside it",
-                "l2": "inputs larger than L2: the timed loops cycle 8 distinct input sets of 17.6 MB (141 MB); "
-                      "no flush between the overlapping steps"}
+        return kv_serving_config(self.U, self.C, ws)
 
     def prepare(self, n_steps: int):
         pass
@@ -281,8 +331,7 @@ class Append:
     max_steps, max_warmup = 10, 3
     io_names = ("ev", "F")
 
-    metric = "users appended (dL=16 events) and their candidates scored per second on 1 B200"
-    unit = "users/s"
+    metric, unit = APPEND_METRIC, "users/s"
 
     def __init__(self, rank: int, users: int = 0, cands: int = 0):
         import torch
@@ -329,15 +378,7 @@ class Append:
         self.d2h = self.out.numel() * 4
 
     def config(self, ws):
-        return {"workload": f"append: non-pyramid 6 layers d=256 4 heads FFN 1024, {self.U} users x 1178 cached "
-                            f"S tokens, append dL={self.dL} events (64-wide, 3 behavior types), then "
-                            f"{self.C} candidates/user (12 NS tokens from 512 features) scored over 1194 keys",
-                "users_per_gpu": self.U, "candidates_per_gpu": self.U * self.C,
-                "parallelism": f"users sharded over {ws} GPU(s), no collective",
-                "pipeline": "batch k+1's append and auto-split (two side streams) are issued before batch k's "
-                            "Stage II; the timed span covers the fill and the drain",
-                "l2": "inputs larger than L2: every step reads its own 1.9 GB cache; no flush between the "
-                      "overlapping steps"}
+        return append_config(self.U, self.C, self.dL, ws)
 
     def prepare(self, n_steps: int):
         """One Stage I-encoded cache per step to come (untimed)."""
@@ -405,7 +446,7 @@ class Forward:
         wl = WORKLOADS[name]
         self.wl, sh = wl, wl.shape
         self.U = users or wl.users
-        self.metric = f"samples/sec of the one-pass forward ({name}) on 1 B200"
+        self.metric = forward_metric(name)
         W = make_weights(sh, wl.seed_weights, wl.dtype)
         self.model = ot.model_from_arrays(sh, W, pyramid_q=list(wl.pyramid), mode=ot.BF16)
         dev = torch.device("cuda")
@@ -421,12 +462,7 @@ class Forward:
         self.d2h = self.out.numel() * 4
 
     def config(self, ws):
-        sh = self.wl.shape
-        return {"workload": f"{self.name}: {sh.n_layers} layers d={sh.d} {sh.n_heads} heads FFN {sh.d_ff}, "
-                            f"{self.U} samples x ({self.wl.L_S} S + {sh.L_NS} NS tokens), pyramid "
-                            f"{self.wl.pyramid[0]}->{self.wl.pyramid[-1]} (linear)",
-                "samples_per_gpu": self.U, "parallelism": f"samples sharded over {ws} GPU(s), no collective",
-                "l2": "512 MB buffer written between timed steps (not timed)"}
+        return forward_config(self.name, self.U, ws)
 
     def prepare(self, n_steps: int):
         pass
@@ -630,22 +666,36 @@ def oracle_sample_forward(name: str, samples: int):
 
 
 def run_reference(args, rank):
+    """The oracle timed on the host cores, each step a bounded sample of the
+    workload extrapolated to its full size; same metric, unit and config as
+    this arm's line.  Rank 0 alone runs it."""
     if rank != 0:
         return
-    vals, samples = [], None
+    from onetrans_synth import WORKLOADS
+    metric, unit, config, units = workload_meta(args.workload, args.gpus)
+    wl = WORKLOADS[args.workload]
+    if args.workload == "kv_serving":
+        def sample(i):
+            return oracle_sample(n_cands=8, seed_shift=i)
+    elif args.workload == "append":
+        def sample(i):
+            return oracle_sample_append(wl.users, wl.cands, n_cands=4)
+    else:
+        def sample(i):
+            return oracle_sample_forward(args.workload, wl.users)
+    vals, samples, cores = [], None, 1
     for i in range(args.warmup + args.steps):
-        v, desc, cores, secs = oracle_sample(n_cands=8, seed_shift=i)
+        v, desc, cores, secs = sample(i)
         if i >= args.warmup:
             vals.append(v)
             samples = desc
     value = statistics.mean(vals)
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * 8192 / value,
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * units / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": "kv_serving: 6x256 pyramid 1190->12, 16 users x 1178 S "
-                                                    "tokens, 512 candidates/user, 12 NS tokens from 512 features"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": samples},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": samples},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
