@@ -325,6 +325,36 @@ def test_intent_order_merge_length_and_sep_position():
     np.testing.assert_array_equal(S[12], np.asarray(W["sep"], dtype=np.float64))
 
 
+@pytest.mark.parametrize("lens", [(5, 0, 7), (0, 0), (9,), (3, 4, 2, 6)])
+def test_intent_order_merge_rows_are_each_sequence_through_its_torch_mlp(lens):
+    """Sequence i's rows are its events through behavior i's MLP (a torch
+    Linear-GELU-Linear), placed after the earlier sequences and their [SEP]s;
+    an empty sequence still gets its [SEP]."""
+    shape, _ = small_model()
+    n = len(lens)
+    dims = tuple(8 + 4 * i for i in range(n))
+    shape = ModelShape(n_layers=1, d=shape.d, n_heads=shape.n_heads, d_ff=shape.d_ff, L_NS=shape.L_NS,
+                       ns_feat=shape.ns_feat, ns_hidden=shape.ns_hidden, behavior_dims=dims)
+    W = make_weights(shape, 70, "fp32", std=0.3)
+    seqs = [gen_normal(71 + i, (L, dims[i]), "fp32") for i, L in enumerate(lens)]
+    S = O.merge_intent_order(seqs, W)
+    assert S.shape == (sum(lens) + n - 1, shape.d)
+    row = 0
+    for i, x in enumerate(seqs):
+        mlp = torch.nn.Sequential(torch.nn.Linear(dims[i], shape.d), torch.nn.GELU("tanh"),
+                                  torch.nn.Linear(shape.d, shape.d)).double()
+        with torch.no_grad():
+            mlp[0].weight.copy_(t64(W["Wb1"][i])); mlp[0].bias.copy_(t64(W["bb1"][i]))
+            mlp[2].weight.copy_(t64(W["Wb2"][i])); mlp[2].bias.copy_(t64(W["bb2"][i]))
+            ref = mlp(t64(x)).numpy()
+        np.testing.assert_allclose(S[row:row + len(x)], ref, rtol=1e-12, atol=1e-13)
+        row += len(x)
+        if i + 1 < n:
+            np.testing.assert_array_equal(S[row], np.asarray(W["sep"], dtype=np.float64))
+            row += 1
+    assert row == S.shape[0]
+
+
 # ------------------------------------------------------------- FLOP counter
 
 def test_flop_counter_reproduces_worked_answers():
