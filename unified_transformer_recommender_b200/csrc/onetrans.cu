@@ -650,7 +650,9 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
       }
     }
   }
-  long long max_tiles = need ? cdiv(C, 64) + std::min<long long>(C, kMaxUsers) : 0;
+  // every candidate tile holds at least one candidate, so C tiles always
+  // suffice; sizing and running carve the same layout
+  const long long tile_cap = std::max<long long>(C, 1);
   Carve cv(ws, ws_bytes);
   void* xa = cv.take((size_t)L_NS * C * d * 4);   // residual stream: float32
   void* xb = cv.take((size_t)L_NS * C * d * 4);
@@ -661,7 +663,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   void* h2 = cv.take((size_t)L_NS * C * d * es);
   void* hid = cv.take((size_t)L_NS * C * dff * es);
   int* row_off = (int*)cv.take((size_t)kMaxUsers * sizeof(int));
-  int* d_tiles = (int*)cv.take((size_t)std::max<long long>(max_tiles, 1) * 3 * sizeof(int));
+  int* d_tiles = (int*)cv.take((size_t)tile_cap * 3 * sizeof(int));
   int* d_s_tab = (int*)cv.take((size_t)m->NL * kMaxUsers * sizeof(int));
   if (need) { *need = cv.used; return ONETRANS_OK; }
   if (cv.overflow) return ONETRANS_ERR_CAPACITY;
@@ -678,7 +680,8 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
   for (int u = 0; u < U; ++u)
     for (int c0 = offs[u]; c0 < offs[u + 1]; c0 += TQ)
       tiles.insert(tiles.end(), {u, c0 - offs[0], std::min(c0 + TQ, offs[u + 1]) - offs[0]});
-  max_tiles = (long long)tiles.size() / 3;
+  const long long n_tiles = (long long)tiles.size() / 3;
+  if (n_tiles > tile_cap) return ONETRANS_ERR_CAPACITY;
 
   std::vector<int> h_row_off(U);
   for (int u = 0; u < U; ++u) h_row_off[u] = slots[u] * m->NL * c->max_pages;
@@ -710,8 +713,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     a.s_sum = ragged ? s_sum[n] : (double)C * s[n];
     a.tiles = d_tiles; a.qkv = qkv; a.o = at;
     kv_for_cache(c, n, row_off, a.kv);
-   
-    OT_TRY(launch_stage2_attn<T>(m, a, (int)max_tiles, st));
+    OT_TRY(launch_stage2_attn<T>(m, a, (int)n_tiles, st));
     GemmDesc go = gdesc_base(m);
     go.mode = TILE_FLAT; go.M = (int)(L_NS * C); go.G = 1;
     go.K = d; go.A = at; go.a_sm = d; go.a_mext = L_NS * C; go.a_gext = 1;
@@ -1351,23 +1353,6 @@ static onetrans_status static_scratch(void** out) {
   return ONETRANS_OK;
 }
 
-template <typename T>
-static onetrans_status autosplit_with_hidden(const onetrans_model* m, const void* feats, long long N, void* out,
-                                             void* hid, cudaStream_t st) {
-  const int F = m->cfg.ns_feat_dim, Hh = m->cfg.ns_hidden, d = m->d, L_NS = m->L_NS;
-  GemmDesc g = gdesc_base(m);
-  g.mode = TILE_FLAT; g.M = (int)N; g.G = 1;
-  g.K = F; g.A = feats; g.a_sm = F; g.a_mext = N; g.a_gext = 1;
-  g.W = m->Wa1; g.w_rows = Hh; g.N = Hh; g.bias = m->ba1; g.act = ACT_GELU;
-  g.out = rmap(hid, 0, Hh);
-  OT_TRY(launch_gemm<T>(m, g, st, PK_GEMM_AUTOSPLIT));
-  GemmDesc g2 = g;
-  g2.K = Hh; g2.A = hid; g2.a_sm = Hh; g2.W = m->Wa2; g2.w_rows = L_NS * d; g2.N = L_NS * d;
-  g2.bias = m->ba2; g2.act = ACT_NONE;
-  g2.out = rmap(out, 0, (long long)L_NS * d);
-  return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
-}
-
 extern "C" onetrans_status onetrans_tokenize_autosplit_static(const onetrans_model* m, const void* feats,
                                                               int64_t N, void* ns_tokens, void* stream) {
   if (!m) return ONETRANS_ERR_INVALID_ARG;
@@ -1377,9 +1362,11 @@ extern "C" onetrans_status onetrans_tokenize_autosplit_static(const onetrans_mod
   if ((size_t)N * m->cfg.ns_hidden * m->es > kStaticScratchBytes) return ONETRANS_ERR_CAPACITY;
   if (N == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
   if (!feats || !ns_tokens || !aligned(feats, 16) || !aligned(ns_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
-  void* hid = nullptr;
-  OT_TRY(static_scratch(&hid));
+  void* scratch = nullptr;
+  OT_TRY(static_scratch(&scratch));
   cudaStream_t st = (cudaStream_t)stream;
-  return m->bf16 ? autosplit_with_hidden<__nv_bfloat16>(m, feats, N, ns_tokens, hid, st)
-                 : autosplit_with_hidden<float>(m, feats, N, ns_tokens, hid, st);
+  // the workspace entry point's body with the scratch array as its workspace:
+  // its capacity check also bounds every access to the array
+  return m->bf16 ? autosplit_impl<__nv_bfloat16>(m, feats, N, ns_tokens, scratch, kStaticScratchBytes, st, nullptr)
+                 : autosplit_impl<float>(m, feats, N, ns_tokens, scratch, kStaticScratchBytes, st, nullptr);
 }
