@@ -129,7 +129,8 @@ typedef enum {
   ONETRANS_OP_STAGE1 = 1,    /* n = U users,   L = L_S */
   ONETRANS_OP_STAGE2 = 2,    /* n = total candidates, L = cached L_S */
   ONETRANS_OP_APPEND = 3,    /* n = U users,   L = dL */
-  ONETRANS_OP_AUTOSPLIT = 4  /* n = N feature rows, L unused */
+  ONETRANS_OP_AUTOSPLIT = 4, /* n = N feature rows, L unused */
+  ONETRANS_OP_GROUPWISE = 5  /* n = N feature rows, L = h_max (padded hidden width) */
 } onetrans_op;
 
 /* Validate `cfg`/`w` and create a model.  Copies the config and the pointer
@@ -182,6 +183,28 @@ ONETRANS_API onetrans_status onetrans_tokenize_autosplit(const onetrans_model* m
                                             const void* feats, int64_t N,
                                             void* ns_tokens, void* ws,
                                             size_t ws_bytes, void* stream);
+
+/* Group-wise NS tokenizer (paper-daily reading "OneTrans: Unified Feature
+ * Interaction and Sequence Modeling with One Transformer in Industrial
+ * Recommender", 2.1 Unified Tokenization; listeners-pseudolab "OneTrans
+ * 정리", 3.1 Non-Sequential Token): the non-sequential features come split
+ * into G = L_NS semantic groups; group g's features go through the group's
+ * own MLP (Linear F_g -> h_g, GELU-tanh, Linear h_g -> d) and give NS token g.
+ * Every group is zero-padded to common widths F_max and h_max (zero feature
+ * columns, zero weight rows and columns, zero bias entries), which leaves
+ * the result unchanged since GELU(0) = 0.
+ *   feats [N, G, F_max]; W1 [G, h_max, F_max]; b1 [G, h_max];
+ *   W2 [G, d, h_max]; b2 [G, d]; ns_tokens [N, G, d] (all device, the mode's
+ *   element type), the layout onetrans_stage2_score takes.
+ * The weights are arguments, not part of the model, and stay the caller's.
+ * G != L_NS, F_max < 1 or h_max < 1 is SHAPE; the workspace holds the hidden
+ * layer (onetrans_workspace_size with ONETRANS_OP_GROUPWISE, n = N,
+ * L = h_max). */
+ONETRANS_API onetrans_status onetrans_tokenize_groupwise(
+    const onetrans_model* m, const void* feats, int64_t N, int32_t G,
+    int32_t F_max, int32_t h_max, const void* W1, const void* b1,
+    const void* W2, const void* b2, void* ns_tokens, void* ws,
+    size_t ws_bytes, void* stream);
 
 /* The auto-split tokenizer for callers that cannot allocate device memory:
  * a plugin inside an inference server whose device memory all belongs to the

@@ -86,3 +86,48 @@ def test_merge_of_one_sequence_is_the_event_tokenizer_without_identifier():
     assert ot.onetrans_device_status() == 0
     emb = to_dev(b.W["type_emb"][t], torch.float32)
     torch.testing.assert_close(merged + emb, plain, rtol=0, atol=1e-5)
+
+
+def pad_groups(groups, G, N, F_max, dtype):
+    """[N, G, F_max] with group g's features in its first F_g columns, zeros after."""
+    out = np.zeros((N, G, F_max), dtype=np.float32)
+    for g, x in enumerate(groups):
+        out[:, g, :x.shape[1]] = x
+    return to_dev(out, tdt(dtype))
+
+
+def pad_weights(Gw, d, F_max, h_max, dtype):
+    G = len(Gw["Wg1"])
+    W1 = np.zeros((G, h_max, F_max), np.float32); b1 = np.zeros((G, h_max), np.float32)
+    W2 = np.zeros((G, d, h_max), np.float32); b2 = np.zeros((G, d), np.float32)
+    for g in range(G):
+        h_g, F_g = Gw["Wg1"][g].shape
+        W1[g, :h_g, :F_g] = Gw["Wg1"][g]; b1[g, :h_g] = Gw["bg1"][g]
+        W2[g, :, :h_g] = Gw["Wg2"][g]; b2[g] = Gw["bg2"][g]
+    return [to_dev(a, tdt(dtype)) for a in (W1, b1, W2, b2)]
+
+
+@pytest.mark.parametrize("dtype,dims,hidden", [
+    ("bf16", (24, 40, 16, 8), (32, 64, 48, 16)),     # F_max = 40: CUDA-core up-projection, tensor-core down
+    ("bf16", (64, 64, 32, 64), (128, 96, 128, 64)),  # F_max = 64, h_max = 128: tensor cores both
+    ("fp32", (24, 40, 16, 8), (32, 64, 48, 16)),
+])
+def test_tokenize_groupwise_matches_oracle(dtype, dims, hidden):
+    from onetrans_synth import make_group_weights
+    G = len(dims)
+    sh = shape(n_layers=1, L_NS=G)
+    b = build(sh, 141, dtype)
+    N, F_max, h_max = 300, max(dims), max(hidden)
+    Gw = make_group_weights(sh.d, dims, hidden, 142, dtype, std=0.1)
+    groups = [gen_normal(143 + g, (N, F_g), dtype) for g, F_g in enumerate(dims)]
+    feats = pad_groups(groups, G, N, F_max, dtype)
+    W1, b1, W2, b2 = pad_weights(Gw, sh.d, F_max, h_max, dtype)
+    tok = torch.full((N, G, sh.d), float("nan"), dtype=tdt(dtype), device="cuda")
+    ws = b.model.workspace(ot.OP_GROUPWISE, N, h_max)
+    ot.onetrans_tokenize_groupwise(b.model, feats, W1, b1, W2, b2, tok, ws)
+    torch.cuda.synchronize()
+    assert ot.onetrans_device_status() == 0
+    ref = O.tokenize_groupwise(groups, Gw)
+    got = to_np(tok)
+    assert not np.isnan(got).any()
+    assert rel_err(got, ref) <= TOL[dtype]

@@ -22,7 +22,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 24
+    assert len(names) == 25
     for n in names:
         assert hasattr(ot.lib, n), n
     assert set(names) == set(ot.SYMBOLS)
@@ -224,6 +224,39 @@ def test_merge_intent_order_argument_errors_before_any_launch():
     assert merge(None, FAKE, [4, 3], [0, 1], FAKE, FAKE) == ot.ERR_INVALID_ARG
     fm0 = FakeModel()
     assert merge(fm0.h, FAKE, [4, 3], [0, 1], FAKE, FAKE) == ot.ERR_UNSUPPORTED
+
+
+def test_tokenize_groupwise_argument_errors_and_workspace_before_any_launch():
+    fm = FakeModel()
+    assert fm.status == ot.OK
+    G = fm.cfg.L_NS
+    gw = ot.lib.onetrans_tokenize_groupwise
+    ws = ctypes.c_void_p(FAKE)
+    big = 1 << 40
+    args = dict(feats=FAKE, N=8, G=G, F=24, h=40, W1=FAKE, b1=FAKE, W2=FAKE, b2=FAKE, tok=FAKE, ws=ws, n=big)
+
+    def call(m=None, **kw):
+        a = dict(args, **kw)
+        return gw(fm.h if m is None else m, a["feats"], a["N"], a["G"], a["F"], a["h"], a["W1"], a["b1"],
+                  a["W2"], a["b2"], a["tok"], a["ws"], a["n"], None)
+
+    assert call(N=0, feats=None, W1=None, tok=None, ws=None) == ot.OK   # no rows: nothing launched
+    assert call(N=-1) == ot.ERR_SHAPE
+    assert call(G=G + 1) == ot.ERR_SHAPE                               # one token per group: G = L_NS
+    assert call(F=0) == ot.ERR_SHAPE
+    assert call(h=0) == ot.ERR_SHAPE
+    for k in ("feats", "W1", "b1", "W2", "b2", "tok"):
+        assert call(**{k: None}) == ot.ERR_INVALID_ARG, k
+    assert call(feats=FAKE + 2) == ot.ERR_INVALID_ARG
+    assert call(W2=FAKE + 8) == ot.ERR_INVALID_ARG
+    assert call(ws=None) == ot.ERR_INVALID_ARG
+    assert call(n=1024) == ot.ERR_CAPACITY                              # hidden layer does not fit
+    assert call(m=ctypes.c_void_p(0)) == ot.ERR_INVALID_ARG
+    # workspace: the [N, G, h_max] hidden layer in the mode's element type
+    out = ot.SZ(0)
+    assert ot.lib.onetrans_workspace_size(fm.h, ot.OP_GROUPWISE, 100, 40, ctypes.byref(out)) == ot.OK
+    assert out.value == 100 * G * 40 * 2
+    assert ot.lib.onetrans_workspace_size(fm.h, ot.OP_GROUPWISE, 100, 0, ctypes.byref(out)) == ot.ERR_SHAPE
 
 
 def test_policy_and_status_strings():

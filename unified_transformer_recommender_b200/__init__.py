@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libonetrans.so")
 
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_DEVICE_CHECK = 0, -1, -2, -3, -4, -5, -6
 BF16, FP32 = 0, 1
-OP_FORWARD, OP_STAGE1, OP_STAGE2, OP_APPEND, OP_AUTOSPLIT = 0, 1, 2, 3, 4
+OP_FORWARD, OP_STAGE1, OP_STAGE2, OP_APPEND, OP_AUTOSPLIT, OP_GROUPWISE = 0, 1, 2, 3, 4, 5
 
 SYMBOLS = (
     "onetrans_model_create", "onetrans_model_destroy", "onetrans_workspace_size",
@@ -32,6 +32,7 @@ SYMBOLS = (
     "onetrans_device_status", "onetrans_status_string", "onetrans_version",
     "onetrans_profile_enable", "onetrans_profile_kinds", "onetrans_profile_read",
     "onetrans_tokenize_autosplit_static", "onetrans_tokenize_events", "onetrans_merge_intent_order",
+    "onetrans_tokenize_groupwise",
 )
 
 
@@ -101,6 +102,7 @@ _sig("onetrans_stage2_score", I32, P, P, PI32, I32, PI32, P, P, P, SZ, P)
 _sig("onetrans_cache_append", I32, P, P, PI32, I32, P, P, I32, P, SZ, P)
 _sig("onetrans_tokenize_events", I32, P, P, P, I64, P, P)
 _sig("onetrans_merge_intent_order", I32, P, P, PI64, PI32, I32, P, P, P)
+_sig("onetrans_tokenize_groupwise", I32, P, P, I64, I32, I32, I32, P, P, P, P, P, P, SZ, P)
 _sig("onetrans_forward", I32, P, P, I32, I32, P, P, SZ, P)
 _sig("onetrans_set_kernel_policy", I32, I32)
 _sig("onetrans_device_status", I32, P, PI32)
@@ -309,6 +311,17 @@ def onetrans_merge_intent_order(model: Model, events: torch.Tensor, seq_len: Seq
     _check("onetrans_merge_intent_order", lib.onetrans_merge_intent_order(
         model.handle, _ptr(events), lens, _i32(list(seq_type) or [0]), n, _ptr(sep), _ptr(tokens),
         _stream(stream)))
+
+
+def onetrans_tokenize_groupwise(model: Model, feats: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor,
+                                W2: torch.Tensor, b2: torch.Tensor, ns_tokens: torch.Tensor, ws: torch.Tensor,
+                                stream=None) -> None:
+    """feats [N, G, F_max]; W1 [G, h_max, F_max], b1 [G, h_max], W2 [G, d, h_max],
+    b2 [G, d] (zero-padded per group); ns_tokens [N, G, d]."""
+    N, G, F_max = feats.shape
+    _check("onetrans_tokenize_groupwise", lib.onetrans_tokenize_groupwise(
+        model.handle, _ptr(feats), N, G, F_max, W1.shape[1], _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2),
+        _ptr(ns_tokens), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def onetrans_stage1_encode(model: Model, cache: Cache, slots: Sequence[int], s_tokens: torch.Tensor,

@@ -929,6 +929,36 @@ static onetrans_status autosplit_impl(const onetrans_model* m, const void* feats
   return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
 }
 
+// Group-wise NS tokenizer: group g of every row through its own two-layer MLP
+// (zero-padded to common widths F_max -> h_max -> d), token g = its output.
+// Two grouped GEMMs: group g is the fixed coordinate that selects the weight
+// set, the rows are tiled as samples; the hidden layer [N, G, h_max] lives in
+// the workspace.
+template <typename T>
+static onetrans_status groupwise_impl(const onetrans_model* m, const void* feats, long long N, int F_max,
+                                      int h_max, const void* W1, const void* b1, const void* W2, const void* b2,
+                                      void* out, void* ws, size_t ws_bytes, cudaStream_t st, size_t* need) {
+  const int G = m->L_NS, d = m->d, es = m->es;
+  Carve cv(ws, ws_bytes);
+  void* hid = cv.take((size_t)N * G * h_max * es);
+  if (need) { *need = cv.used; return ONETRANS_OK; }
+  if (cv.overflow) return ONETRANS_ERR_CAPACITY;
+  if (N == 0) return ONETRANS_OK;
+  GemmDesc g = gdesc_base(m);
+  g.mode = TILE_SAMPLES; g.M = (int)N; g.G = G; g.g_lo = 0; g.grp_base = 0;
+  g.K = F_max; g.A = feats; g.a_sm = (long long)G * F_max; g.a_sg = F_max; g.a_mext = N; g.a_gext = G;
+  g.W = W1; g.w_sg = (long long)h_max * F_max; g.w_rows = h_max; g.w_groups = G; g.n_lo = 0; g.N = h_max;
+  g.bias = b1; g.bias_sg = h_max; g.act = ACT_GELU;
+  g.out = rmap(hid, (long long)G * h_max, h_max);
+  OT_TRY(launch_gemm<T>(m, g, st, PK_GEMM_AUTOSPLIT));
+  GemmDesc g2 = g;
+  g2.K = h_max; g2.A = hid; g2.a_sm = (long long)G * h_max; g2.a_sg = h_max;
+  g2.W = W2; g2.w_sg = (long long)d * h_max; g2.w_rows = d; g2.N = d;
+  g2.bias = b2; g2.bias_sg = d; g2.act = ACT_NONE;
+  g2.out = rmap(out, (long long)G * d, d);   // [N, G, d]
+  return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
+}
+
 // ============================================================== C ABI ====
 extern "C" {
 
@@ -1047,6 +1077,12 @@ onetrans_status onetrans_workspace_size(const onetrans_model* m, int32_t op, int
     case ONETRANS_OP_AUTOSPLIT:
       return m->bf16 ? autosplit_impl<__nv_bfloat16>(m, nullptr, n, nullptr, nullptr, 0, 0, bytes)
                      : autosplit_impl<float>(m, nullptr, n, nullptr, nullptr, 0, 0, bytes);
+    case ONETRANS_OP_GROUPWISE:
+      if (L < 1) return ONETRANS_ERR_SHAPE;
+      return m->bf16 ? groupwise_impl<__nv_bfloat16>(m, nullptr, n, 1, L, nullptr, nullptr, nullptr, nullptr,
+                                                     nullptr, nullptr, 0, 0, bytes)
+                     : groupwise_impl<float>(m, nullptr, n, 1, L, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                             nullptr, 0, 0, bytes);
     default:
       return ONETRANS_ERR_INVALID_ARG;
   }
@@ -1150,6 +1186,24 @@ onetrans_status onetrans_tokenize_autosplit(const onetrans_model* m, const void*
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? autosplit_impl<__nv_bfloat16>(m, feats, N, ns_tokens, ws, ws_bytes, st, nullptr)
                  : autosplit_impl<float>(m, feats, N, ns_tokens, ws, ws_bytes, st, nullptr);
+}
+
+onetrans_status onetrans_tokenize_groupwise(const onetrans_model* m, const void* feats, int64_t N,
+                                            int32_t G, int32_t F_max, int32_t h_max, const void* W1,
+                                            const void* b1, const void* W2, const void* b2, void* ns_tokens,
+                                            void* ws, size_t ws_bytes, void* stream) {
+  if (!m) return ONETRANS_ERR_INVALID_ARG;
+  if (N < 0 || N > (1LL << 31) - 1 || G != m->L_NS || F_max < 1 || h_max < 1) return ONETRANS_ERR_SHAPE;
+  if (N == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!feats || !W1 || !b1 || !W2 || !b2 || !ns_tokens) return ONETRANS_ERR_INVALID_ARG;
+  if (!aligned(feats, 16) || !aligned(ns_tokens, 16) || !aligned(W1, 16) || !aligned(W2, 16))
+    return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? groupwise_impl<__nv_bfloat16>(m, feats, N, F_max, h_max, W1, b1, W2, b2, ns_tokens, ws,
+                                                 ws_bytes, st, nullptr)
+                 : groupwise_impl<float>(m, feats, N, F_max, h_max, W1, b1, W2, b2, ns_tokens, ws, ws_bytes, st,
+                                         nullptr);
 }
 
 static onetrans_status check_slots(const onetrans_cache* c, const int32_t* slots, int U) {
