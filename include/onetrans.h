@@ -267,6 +267,19 @@ ONETRANS_API onetrans_status onetrans_stage1_encode(const onetrans_model* m,
                                        int32_t L_S, void* ws, size_t ws_bytes,
                                        void* stream);
 
+/* Stage I for users of different lengths in one call: user u's lens[u]
+ * (host) S-tokens lie back to back in s_tokens [sum of lens, d], in the
+ * order of slots.  Each run of consecutive users with one length is one
+ * onetrans_stage1_encode pass over its slice (ordering users by length makes
+ * fewer passes).  Every check a pass can fail (length against the pool, the
+ * schedule, the workspace, page capacity over the runs in order) is made for
+ * all runs before the first launch.  A workspace sized for
+ * ONETRANS_OP_STAGE1 with n = U, L = the largest length is enough. */
+ONETRANS_API onetrans_status onetrans_stage1_encode_ragged(
+    const onetrans_model* m, onetrans_cache* c, const int32_t* slots,
+    int32_t U, const void* s_tokens, const int32_t* lens, void* ws,
+    size_t ws_bytes, void* stream);
+
 /* Stage II ([FR] 7.5.3): score candidates against the cached S side.  User u
  * owns candidates cand_offsets[u] .. cand_offsets[u+1]-1 (host CSR, U+1
  * entries) and cache slot slots[u] (host).  Per layer, NS token j of a

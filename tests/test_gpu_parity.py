@@ -183,6 +183,45 @@ def test_stage2_users_of_different_lengths(dtype, policy, pyr):
             assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL[dtype], (u, c)
 
 
+@pytest.mark.parametrize("dtype,policy,pyr", [("bf16", 0, None), ("bf16", 0, [150, 80, 12]),
+                                              ("bf16", 1, None), ("fp32", 0, None)])
+def test_stage1_ragged_one_call(dtype, policy, pyr):
+    """One Stage I call for users of different lengths (runs of equal lengths
+    among them): every layer's cached K/V of every user against the oracle's
+    Stage I of that user alone, then one Stage II call over all of them."""
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=3)
+    b = build(sh, 151, dtype, pyramid=pyr)
+    m = b.model
+    Ls = [200, 200, 139, 257, 257, 140]
+    slots = [4, 0, 2, 1, 5, 3]
+    cache = ot.Cache(m, len(Ls), max(Ls))
+    S = [gen_normal(160 + u, (L, sh.d), dtype) for u, L in enumerate(Ls)]
+    packed = to_dev(np.concatenate(S, axis=0), tdt(dtype))
+    ot.onetrans_stage1_encode_ragged(m, cache, slots, Ls, packed, m.workspace(ot.OP_STAGE1, len(Ls), max(Ls)))
+    torch.cuda.synchronize()
+    assert ot.onetrans_device_status() == 0
+    kvs = []
+    for u, L in enumerate(Ls):
+        assert cache.length(slots[u]) == L
+        kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, pyr)
+        kvs.append(kv)
+        for n, (K, V) in enumerate(kv):
+            got = to_np(cache.gather(slots[u], n, K.shape[0]))
+            assert rel_err(got[0], K) <= TOL[dtype] and rel_err(got[1], V) <= TOL[dtype], (u, n)
+    counts = [2, 3, 1, 2, 2, 3]
+    offs = np.concatenate([[0], np.cumsum(counts)]).tolist()
+    NS = gen_normal(170, (offs[-1], sh.L_NS, sh.d), dtype)
+    out = torch.empty(offs[-1], sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
+    ot.onetrans_stage2_score(m, cache, slots, offs, to_dev(NS, tdt(dtype)), out,
+                             m.workspace(ot.OP_STAGE2, offs[-1], max(Ls)))
+    torch.cuda.synchronize()
+    out = to_np(out)
+    for u in range(len(Ls)):
+        for c in range(offs[u], offs[u + 1]):
+            assert rel_err(out[c], O.stage2(kvs[u], NS[c], b.W, sh.n_heads, EPS)) <= TOL[dtype], (u, c)
+
+
 @pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
 def test_append_users_of_different_lengths(dtype, policy):
     """One append call for users whose slots hold different lengths: each

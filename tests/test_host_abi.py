@@ -22,7 +22,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 25
+    assert len(names) == 26
     for n in names:
         assert hasattr(ot.lib, n), n
     assert set(names) == set(ot.SYMBOLS)
@@ -257,6 +257,36 @@ def test_tokenize_groupwise_argument_errors_and_workspace_before_any_launch():
     assert ot.lib.onetrans_workspace_size(fm.h, ot.OP_GROUPWISE, 100, 40, ctypes.byref(out)) == ot.OK
     assert out.value == 100 * G * 40 * 2
     assert ot.lib.onetrans_workspace_size(fm.h, ot.OP_GROUPWISE, 100, 0, ctypes.byref(out)) == ot.ERR_SHAPE
+
+
+def test_stage1_ragged_checks_every_run_before_any_launch():
+    """Without a GPU any launch fails with a CUDA error: a call whose first run
+    is valid and whose second is not must return the second run's error and
+    leave every slot as it was."""
+    sched = linear_pyramid(1190, 12, 6)
+    fm = FakeModel(pyramid=sched)
+    st, size, c = _cache(fm, 4, 1178)
+    assert st == ot.OK
+    ws, big = FAKE, 1 << 40
+    enc = ot.lib.onetrans_stage1_encode_ragged
+
+    def call(slots, lens, ws_bytes=big, s_tok=FAKE, lens_ptr=True):
+        S = (ot.I32 * len(slots))(*slots)
+        Lp = (ot.I32 * len(lens))(*lens) if lens_ptr else None
+        return enc(fm.h, c, S, len(slots), s_tok, Lp, ws, ws_bytes, None)
+
+    assert enc(fm.h, c, None, 0, None, None, None, 0, None) == ot.OK      # no users: nothing launched
+    assert call([0, 1], [1178, 1178], lens_ptr=False) == ot.ERR_INVALID_ARG
+    assert call([0, 1], [1178, 0]) == ot.ERR_SHAPE
+    assert call([0, 0], [1178, 1178]) == ot.ERR_INVALID_ARG              # a slot twice
+    assert call([0, 1], [1178, 500]) == ot.ERR_SHAPE                     # second run: schedule does not fit
+    assert call([0, 1], [1178, 1179]) == ot.ERR_CAPACITY                 # second run: longer than the pool's rows
+    assert call([0, 1], [1178, 1100], ws_bytes=1024) == ot.ERR_CAPACITY  # workspace
+    assert call([0, 1], [1178, 1100], s_tok=FAKE + 2) == ot.ERR_INVALID_ARG
+    ln = ot.I32(-1)
+    for slot in range(4):
+        assert ot.lib.onetrans_cache_length(c, slot, ctypes.byref(ln)) == ot.OK and ln.value == 0
+    ot.lib.onetrans_cache_destroy(c)
 
 
 def test_policy_and_status_strings():

@@ -27,7 +27,8 @@ SYMBOLS = (
     "onetrans_model_create", "onetrans_model_destroy", "onetrans_workspace_size",
     "onetrans_schedule", "onetrans_cache_size", "onetrans_cache_init",
     "onetrans_cache_destroy", "onetrans_cache_length", "onetrans_cache_row_ptr",
-    "onetrans_tokenize_autosplit", "onetrans_stage1_encode", "onetrans_stage2_score",
+    "onetrans_tokenize_autosplit", "onetrans_stage1_encode", "onetrans_stage1_encode_ragged",
+    "onetrans_stage2_score",
     "onetrans_cache_append", "onetrans_forward", "onetrans_set_kernel_policy",
     "onetrans_device_status", "onetrans_status_string", "onetrans_version",
     "onetrans_profile_enable", "onetrans_profile_kinds", "onetrans_profile_read",
@@ -98,6 +99,7 @@ _sig("onetrans_cache_row_ptr", I32, P, I32, I32, I32, I32, I32, ctypes.POINTER(P
 _sig("onetrans_tokenize_autosplit", I32, P, P, I64, P, P, SZ, P)
 _sig("onetrans_tokenize_autosplit_static", I32, P, P, I64, P, P)
 _sig("onetrans_stage1_encode", I32, P, P, PI32, I32, P, I32, P, SZ, P)
+_sig("onetrans_stage1_encode_ragged", I32, P, P, PI32, I32, P, PI32, P, SZ, P)
 _sig("onetrans_stage2_score", I32, P, P, PI32, I32, PI32, P, P, P, SZ, P)
 _sig("onetrans_cache_append", I32, P, P, PI32, I32, P, P, I32, P, SZ, P)
 _sig("onetrans_tokenize_events", I32, P, P, P, I64, P, P)
@@ -330,6 +332,14 @@ def onetrans_stage1_encode(model: Model, cache: Cache, slots: Sequence[int], s_t
     _check("onetrans_stage1_encode", lib.onetrans_stage1_encode(
         model.handle, cache.handle, sl, len(slots), _ptr(s_tokens), s_tokens.shape[1], _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def onetrans_stage1_encode_ragged(model: Model, cache: Cache, slots: Sequence[int], lens: Sequence[int],
+                                  s_tokens: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    """s_tokens [sum(lens), d]: user u's lens[u] rows back to back, in the order of slots."""
+    _check("onetrans_stage1_encode_ragged", lib.onetrans_stage1_encode_ragged(
+        model.handle, cache.handle, _i32(slots), len(slots), _ptr(s_tokens), _i32(list(lens) or [0]), _ptr(ws),
+        ws.numel(), _stream(stream)))
 
 
 def onetrans_stage2_score(model: Model, cache: Cache, slots: Sequence[int], cand_offsets: Sequence[int],

@@ -1233,6 +1233,64 @@ onetrans_status onetrans_stage1_encode(const onetrans_model* m, onetrans_cache* 
                  : stage1_impl<float>(m, c, slots, U, s_tokens, L_S, ws, ws_bytes, st, nullptr);
 }
 
+onetrans_status onetrans_stage1_encode_ragged(const onetrans_model* m, onetrans_cache* c, const int32_t* slots,
+                                              int32_t U, const void* s_tokens, const int32_t* lens, void* ws,
+                                              size_t ws_bytes, void* stream) {
+  if (!m || !c || c->m != m) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_slots(c, slots, U));
+  if (U == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!lens) return ONETRANS_ERR_INVALID_ARG;
+  long long R = 0;
+  for (int u = 0; u < U; ++u) {
+    if (lens[u] < 1) return ONETRANS_ERR_SHAPE;
+    R += lens[u];
+  }
+  if (R > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
+  if (!s_tokens || !aligned(s_tokens, 16)) return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
+  // runs of consecutive users of one length: each is one uniform Stage I pass
+  std::vector<std::pair<int, int>> runs;  // (first user, users)
+  for (int u = 0; u < U;) {
+    int v = u;
+    while (v < U && lens[v] == lens[u]) ++v;
+    runs.push_back({u, v - u});
+    u = v;
+  }
+  // everything a pass can refuse is checked for every run before the first
+  // launch; a run frees its slots' old pages before taking new ones, so page
+  // capacity must hold for every prefix of the runs, in order
+  const int P = m->cfg.page_tokens;
+  const long long free0 = (long long)c->free_pages.size();
+  long long need_pages = 0, owned_pages = 0;
+  for (const auto& r : runs) {
+    const int L = lens[r.first];
+    if (L > c->max_L_S) return ONETRANS_ERR_CAPACITY;
+    if ((long long)r.second * L > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
+    std::vector<int> s, sq;
+    OT_TRY(s_rows_of(m, L, s, sq));
+    size_t need = 0;
+    OT_TRY(m->bf16 ? stage1_impl<__nv_bfloat16>(m, c, slots + r.first, r.second, nullptr, L, nullptr, 0, 0, &need)
+                   : stage1_impl<float>(m, c, slots + r.first, r.second, nullptr, L, nullptr, 0, 0, &need));
+    if (need > ws_bytes) return ONETRANS_ERR_CAPACITY;
+    for (int u = r.first; u < r.first + r.second; ++u) {
+      for (int n = 0; n < m->NL; ++n) need_pages += cdiv(s[n], P);
+      const size_t row = (size_t)slots[u] * m->NL * c->max_pages;
+      for (size_t i = 0; i < (size_t)m->NL * c->max_pages; ++i) owned_pages += c->h_table[row + i] >= 0;
+    }
+    if (need_pages > free0 + owned_pages) return ONETRANS_ERR_CAPACITY;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  long long off = 0;
+  for (const auto& r : runs) {
+    const int L = lens[r.first];
+    const void* tok = eoff(s_tokens, off * m->d, m->es);
+    OT_TRY(m->bf16 ? stage1_impl<__nv_bfloat16>(m, c, slots + r.first, r.second, tok, L, ws, ws_bytes, st, nullptr)
+                   : stage1_impl<float>(m, c, slots + r.first, r.second, tok, L, ws, ws_bytes, st, nullptr));
+    off += (long long)r.second * L;
+  }
+  return ONETRANS_OK;
+}
+
 onetrans_status onetrans_stage2_score(const onetrans_model* m, const onetrans_cache* c, const int32_t* slots,
                                       int32_t U, const int32_t* cand_offsets, const void* ns_tokens,
                                       void* ns_out, void* ws, size_t ws_bytes, void* stream) {
