@@ -323,9 +323,19 @@ ONETRANS_API onetrans_status onetrans_forward(const onetrans_model* m, const voi
  * shape allows), 1 = CUDA-core kernels only.  Process-wide. */
 ONETRANS_API onetrans_status onetrans_set_kernel_policy(int32_t policy);
 /* Reads and clears the device status word that kernels set, instead of
- * trapping, when a bounds check or a bounded wait fails (0 = no failure).
- * Synchronizes `stream`. */
+ * trapping, when a bounds check or a bounded wait fails.  *code: 0 = no
+ * failure, 101 = an mbarrier wait gave up (its kernel drained and returned),
+ * 102 = dynamic shared memory not 1024-byte aligned (the kernel returned
+ * without work), 3 = a CUDA-core kernel's bounds check skipped an access.
+ * Returns ONETRANS_ERR_DEVICE_CHECK when *code != 0.  Synchronizes `stream`. */
 ONETRANS_API onetrans_status onetrans_device_status(void* stream, int32_t* code);
+/* Exercises the failure path of the bounded waits without a GPU fault: one
+ * thread waits on an mbarrier that nothing arrives at, with the wait every
+ * tensor-core kernel uses, limited to spin_limit try_wait rounds (1 ..
+ * 2^20, else INVALID_ARG).  The wait gives up, records code 101 in the
+ * device status word and the kernel returns; onetrans_device_status then
+ * reports it. */
+ONETRANS_API onetrans_status onetrans_selftest_bounded_wait(int32_t spin_limit, void* stream);
 /* Per-kernel timing for measurement.  While enabled, every launch is
  * bracketed by CUDA events on its stream and tagged with its kernel kind and
  * its algorithmic FLOPs and bytes (each operand and result once).  Enabling

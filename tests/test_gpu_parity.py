@@ -11,7 +11,7 @@ pytestmark = pytest.mark.gpu
 from onetrans_synth import (WORKLOADS, gen_normal, linear_pyramid, random_types,
                             tiny_raw_inputs)
 from oracle import onetrans as O
-from helpers import EPS, TOL, build, rel_err, shape, to_dev, to_np
+from helpers import EPS, TOL, build, rel_err, run_forward, run_stage12, shape, tdt, to_dev, to_np
 
 import unified_transformer_recommender_b200 as ot  # noqa: E402
 
@@ -21,37 +21,6 @@ def _policy_reset():
     yield
     ot.onetrans_set_kernel_policy(0)
     assert ot.onetrans_device_status() == 0
-
-
-def tdt(dtype):
-    return torch.bfloat16 if dtype == "bf16" else torch.float32
-
-
-def run_forward(b, X0):
-    m = b.model
-    L_S = X0.shape[1] - b.shape.L_NS
-    sched = m.schedule(L_S)
-    out = torch.empty(X0.shape[0], sched[-1], b.shape.d, dtype=torch.float32, device="cuda")
-    ws = m.workspace(ot.OP_FORWARD, X0.shape[0], L_S)
-    ot.onetrans_forward(m, to_dev(X0, tdt(b.dtype)), out, ws)
-    torch.cuda.synchronize()
-    return to_np(out)
-
-
-def run_stage12(b, S, NS_tok, offsets, slots=None):
-    """S: [U, L_S, d]; NS_tok: [C, L_NS, d]; returns (cache obj, ns_out [C, L_NS, d])."""
-    m = b.model
-    U, L_S, d = S.shape
-    slots = list(range(U)) if slots is None else slots
-    cache = ot.Cache(m, max(slots) + 1, L_S + 64)
-    ws1 = m.workspace(ot.OP_STAGE1, U, L_S)
-    ot.onetrans_stage1_encode(m, cache, slots, to_dev(S, tdt(b.dtype)), ws1)
-    C = NS_tok.shape[0]
-    out = torch.empty(C, b.shape.L_NS, d, dtype=torch.float32, device="cuda")
-    ws2 = m.workspace(ot.OP_STAGE2, C, L_S)
-    ot.onetrans_stage2_score(m, cache, slots, offsets, to_dev(NS_tok, tdt(b.dtype)), out, ws2)
-    torch.cuda.synchronize()
-    return cache, to_np(out)
 
 
 # ------------------------------------------------------------------ tiny --

@@ -22,7 +22,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 26
+    assert len(names) == 27
     for n in names:
         assert hasattr(ot.lib, n), n
     assert set(names) == set(ot.SYMBOLS)
@@ -290,6 +290,8 @@ def test_stage1_ragged_checks_every_run_before_any_launch():
 
 
 def test_policy_and_status_strings():
+    assert ot.lib.onetrans_selftest_bounded_wait(0, None) == ot.ERR_INVALID_ARG
+    assert ot.lib.onetrans_selftest_bounded_wait((1 << 20) + 1, None) == ot.ERR_INVALID_ARG
     assert ot.lib.onetrans_set_kernel_policy(2) == ot.ERR_INVALID_ARG
     assert ot.lib.onetrans_set_kernel_policy(0) == ot.OK
     assert ot.status_string(ot.ERR_CAPACITY) == "capacity exceeded"

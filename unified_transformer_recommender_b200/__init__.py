@@ -33,7 +33,7 @@ SYMBOLS = (
     "onetrans_device_status", "onetrans_status_string", "onetrans_version",
     "onetrans_profile_enable", "onetrans_profile_kinds", "onetrans_profile_read",
     "onetrans_tokenize_autosplit_static", "onetrans_tokenize_events", "onetrans_merge_intent_order",
-    "onetrans_tokenize_groupwise",
+    "onetrans_tokenize_groupwise", "onetrans_selftest_bounded_wait",
 )
 
 
@@ -108,6 +108,7 @@ _sig("onetrans_tokenize_groupwise", I32, P, P, I64, I32, I32, I32, P, P, P, P, P
 _sig("onetrans_forward", I32, P, P, I32, I32, P, P, SZ, P)
 _sig("onetrans_set_kernel_policy", I32, I32)
 _sig("onetrans_device_status", I32, P, PI32)
+_sig("onetrans_selftest_bounded_wait", I32, I32, P)
 _sig("onetrans_status_string", ctypes.c_char_p, I32)
 _sig("onetrans_version", I32)
 _sig("onetrans_profile_enable", I32, I32)
@@ -145,9 +146,16 @@ def onetrans_set_kernel_policy(policy: int) -> None:
 
 
 def onetrans_device_status(stream=None) -> int:
+    """Reads and clears the device status word: 0, or the failed check's code."""
     code = I32(0)
-    _check("onetrans_device_status", lib.onetrans_device_status(_stream(stream), ctypes.byref(code)))
+    s = lib.onetrans_device_status(_stream(stream), ctypes.byref(code))
+    if s != ERR_DEVICE_CHECK:
+        _check("onetrans_device_status", s)
     return code.value
+
+
+def onetrans_selftest_bounded_wait(spin_limit: int, stream=None) -> None:
+    _check("onetrans_selftest_bounded_wait", lib.onetrans_selftest_bounded_wait(int(spin_limit), _stream(stream)))
 
 
 def onetrans_profile_enable(on: bool) -> None:

@@ -959,6 +959,20 @@ static onetrans_status groupwise_impl(const onetrans_model* m, const void* feats
   return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
 }
 
+// Failure path of the bounded waits, without a fault: one thread waits on an
+// mbarrier that nothing arrives at, with the same wait the tensor-core
+// kernels use but limited to `limit` rounds; the wait gives up, records
+// kErrWaitTimeout in the device status word, and the kernel returns.
+__global__ void selftest_wait_kernel(uint32_t limit) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_limited(&bar, 0, limit);
+}
+
 // ============================================================== C ABI ====
 extern "C" {
 
@@ -1430,8 +1444,15 @@ onetrans_status onetrans_device_status(void* stream, int32_t* code) {
     const int zero = 0;
     OT_TRY(cuda_ok(cudaMemcpyToSymbolAsync(ot::g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st)));
     OT_TRY(cuda_ok(cudaStreamSynchronize(st)));
+    return ONETRANS_ERR_DEVICE_CHECK;
   }
   return ONETRANS_OK;
+}
+
+onetrans_status onetrans_selftest_bounded_wait(int32_t spin_limit, void* stream) {
+  if (spin_limit < 1 || (uint32_t)spin_limit > ot::kSpinLimit) return ONETRANS_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint32_t)spin_limit);
+  return last_launch();
 }
 
 }  // extern "C"

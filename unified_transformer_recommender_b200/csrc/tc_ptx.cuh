@@ -41,12 +41,16 @@ __device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Waits for the phase with the given parity to complete; false on timeout.
-__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+// Waits for the phase with the given parity to complete, for at most `limit`
+// try_wait rounds; on timeout records kErrWaitTimeout and returns false.
+__device__ inline bool mbar_wait_limited(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   flag_error(kErrWaitTimeout);
   return false;
+}
+__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_limited(bar, parity, kSpinLimit);
 }
 
 // ------------------------------------------------------------------ TMA --
