@@ -11,8 +11,10 @@
 //   O += P V           tcgen05.mma with P read from TMEM and V from shared
 //                      memory (MN-major); O stays in TMEM for the whole row
 // The running max m is raised only when a tile's max passes it by more than
-// 2^8; then the thread rescales l and the O row in TMEM.  S of tile t+1 is
-// computed while the softmax of tile t runs; two CTAs share an SM.
+// 2^8; then the thread rescales l, and its warp the O rows in TMEM (a
+// warp-collective load and store, alpha = 1 for rows that keep their max).
+// S of tile t+1 is computed while the softmax of tile t runs; two CTAs share
+// an SM.
 //
 // Query kinds:
 //  * MODE_CAUSAL  (Stage I, forward, append): query t of sequence b sits at
@@ -362,7 +364,9 @@ __global__ void __launch_bounds__(192, AttnCfgT<DH>::CTAS)
         if (!ok) break;
         tc_fence_after();
       }
-      if (rescale) {
+      // tcgen05.ld/st are warp-collective: the whole warp rescales when any
+      // of its rows does (alpha stays exactly 1 for the others)
+      if (__any_sync(0xffffffffu, rescale)) {
         // O holds the tiles before kt (p_free was awaited): bring it to the new max
 #pragma unroll
         for (int c = 0; c < C::DH / 32; ++c) {
