@@ -20,6 +20,24 @@ def rel_err(got, ref) -> float:
     return float(np.max(np.abs(got - ref)) / rms)
 
 
+# A value the bf16 path stores in bf16 (the K/V cache, tokenizer outputs)
+# carries, besides the computation's error, its own rounding (half an ulp,
+# 2^-9 of its magnitude) and that of the bf16 operand it was computed from:
+# its bar adds STORE_ULP * |x| per element to TOL * RMS.  Float32 outputs
+# (the stack's final rows) keep the plain bar.
+STORE_ULP = {"bf16": 2.0 ** -8, "fp32": 0.0}
+
+
+def stored_err(got, ref, dtype) -> float:
+    """max_i |got_i - ref_i| / (RMS(ref) + |ref_i| * STORE_ULP / TOL): at most
+    TOL[dtype] exactly when every element is within TOL * RMS + STORE_ULP * |ref_i|."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    rms = np.sqrt(np.mean(ref * ref))
+    return float(np.max(np.abs(got - ref) / (rms + np.abs(ref) * STORE_ULP[dtype] / TOL[dtype])))
+
+
 def shape(n_layers=2, d=256, H=4, dff=1024, L_NS=12, F=512, Hh=None, n_types=3):
     return ModelShape(n_layers=n_layers, d=d, n_heads=H, d_ff=dff, L_NS=L_NS, ns_feat=F,
                       ns_hidden=Hh if Hh is not None else L_NS * d,

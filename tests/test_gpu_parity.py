@@ -11,7 +11,7 @@ pytestmark = pytest.mark.gpu
 from onetrans_synth import (WORKLOADS, gen_normal, linear_pyramid, random_types,
                             tiny_raw_inputs)
 from oracle import onetrans as O
-from helpers import EPS, TOL, build, rel_err, run_forward, run_stage12, shape, tdt, to_dev, to_np
+from helpers import EPS, TOL, build, rel_err, run_forward, run_stage12, shape, stored_err, tdt, to_dev, to_np
 
 import unified_transformer_recommender_b200 as ot  # noqa: E402
 
@@ -113,8 +113,8 @@ def test_stage1_stage2_small_ragged(dtype, policy):
         assert cache.length(slots[u]) == L_S
         for n, (K, V) in enumerate(kv):
             got = to_np(cache.gather(slots[u], n, K.shape[0]))
-            assert rel_err(got[0], K) <= TOL[dtype]
-            assert rel_err(got[1], V) <= TOL[dtype]
+            assert stored_err(got[0], K, dtype) <= TOL[dtype]
+            assert stored_err(got[1], V, dtype) <= TOL[dtype]
         for c in range(offs[u], offs[u + 1]):
             r = O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)
             assert rel_err(out[c], r) <= TOL[dtype], (u, c)
@@ -177,7 +177,7 @@ def test_stage1_ragged_one_call(dtype, policy, pyr):
         kvs.append(kv)
         for n, (K, V) in enumerate(kv):
             got = to_np(cache.gather(slots[u], n, K.shape[0]))
-            assert rel_err(got[0], K) <= TOL[dtype] and rel_err(got[1], V) <= TOL[dtype], (u, n)
+            assert stored_err(got[0], K, dtype) <= TOL[dtype] and stored_err(got[1], V, dtype) <= TOL[dtype], (u, n)
     counts = [2, 3, 1, 2, 2, 3]
     offs = np.concatenate([[0], np.cumsum(counts)]).tolist()
     NS = gen_normal(170, (offs[-1], sh.L_NS, sh.d), dtype)
@@ -225,8 +225,8 @@ def test_append_users_of_different_lengths(dtype, policy):
         kv = O.append(O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS), new, b.W, sh.n_heads, EPS)
         for n, (K, V) in enumerate(kv):
             got = to_np(cache.gather(slots[u], n, Ls[u] + dL))
-            assert rel_err(got[0], K) <= TOL[dtype], (u, n)
-            assert rel_err(got[1], V) <= TOL[dtype], (u, n)
+            assert stored_err(got[0], K, dtype) <= TOL[dtype], (u, n)
+            assert stored_err(got[1], V, dtype) <= TOL[dtype], (u, n)
         for c in range(offs[u], offs[u + 1]):
             assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL[dtype], (u, c)
 
@@ -249,7 +249,7 @@ def test_tokenize_events_then_stage1(dtype, d):
     torch.cuda.synchronize()
     assert ot.onetrans_device_status() == 0
     ref = O.tokenize_events(ev, ty, b.W)
-    assert rel_err(to_np(tok).reshape(U, L, d), ref) <= TOL[dtype]
+    assert stored_err(to_np(tok).reshape(U, L, d), ref, dtype) <= TOL[dtype]
     cache = ot.Cache(m, U, L)
     ot.onetrans_stage1_encode(m, cache, list(range(U)), tok.view(U, L, d), m.workspace(ot.OP_STAGE1, U, L))
     torch.cuda.synchronize()
@@ -257,7 +257,7 @@ def test_tokenize_events_then_stage1(dtype, d):
         kv = O.stage1(ref[u], b.W, sh.L_NS, sh.n_heads, EPS)   # the oracle's own tokens
         for n, (K, V) in enumerate(kv):
             got = to_np(cache.gather(u, n, L))
-            assert rel_err(got[0], K) <= TOL[dtype] and rel_err(got[1], V) <= TOL[dtype], (u, n)
+            assert stored_err(got[0], K, dtype) <= TOL[dtype] and stored_err(got[1], V, dtype) <= TOL[dtype], (u, n)
 
 
 @pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
@@ -287,8 +287,8 @@ def test_append_small_crosses_page_boundary(dtype, policy):
         kv = O.append(O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS), new, b.W, sh.n_heads, EPS)
         for n, (K, V) in enumerate(kv):
             got = to_np(cache.gather(slot, n, L_S + dL))
-            assert rel_err(got[0], K) <= TOL[dtype]
-            assert rel_err(got[1], V) <= TOL[dtype]
+            assert stored_err(got[0], K, dtype) <= TOL[dtype]
+            assert stored_err(got[1], V, dtype) <= TOL[dtype]
         for c in range(2 * u, 2 * u + 2):
             r = O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)
             assert rel_err(out[c], r) <= TOL[dtype]
@@ -305,7 +305,7 @@ def test_autosplit_ragged_rows(dtype, policy):
     ot.onetrans_tokenize_autosplit(b.model, to_dev(feats, tdt(dtype)), ns, b.model.workspace(ot.OP_AUTOSPLIT, N))
     torch.cuda.synchronize()
     ref = O.autosplit(feats, b.W, sh.L_NS)
-    assert rel_err(to_np(ns), ref) <= TOL[dtype]
+    assert stored_err(to_np(ns), ref, dtype) <= TOL[dtype]
 
 
 # --------------------------------------------------------- exact checks --
@@ -395,8 +395,8 @@ def test_stage1_stage2_d384_small():
         kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, sched)
         for n, (K, V) in enumerate(kv):
             got = to_np(cache.gather(u, n, K.shape[0]))
-            assert rel_err(got[0], K) <= TOL["bf16"]
-            assert rel_err(got[1], V) <= TOL["bf16"]
+            assert stored_err(got[0], K, "bf16") <= TOL["bf16"]
+            assert stored_err(got[1], V, "bf16") <= TOL["bf16"]
         for c in range(offs[u], offs[u + 1]):
             assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL["bf16"], (u, c)
 
@@ -445,9 +445,9 @@ def test_long_sequence_beyond_cached_page_ids():
     cache, out = run_stage12(b, S, NS, [0, 3])
     kv = O.stage1(S[0], b.W, sh.L_NS, sh.n_heads, EPS, sched)
     K0 = to_np(cache.gather(0, 0, L_S))
-    assert rel_err(K0[0], kv[0][0]) <= TOL["bf16"] and rel_err(K0[1], kv[0][1]) <= TOL["bf16"]
+    assert stored_err(K0[0], kv[0][0], "bf16") <= TOL["bf16"] and stored_err(K0[1], kv[0][1], "bf16") <= TOL["bf16"]
     K1 = to_np(cache.gather(0, 1, kv[1][0].shape[0]))
-    assert rel_err(K1[0], kv[1][0]) <= TOL["bf16"] and rel_err(K1[1], kv[1][1]) <= TOL["bf16"]
+    assert stored_err(K1[0], kv[1][0], "bf16") <= TOL["bf16"] and stored_err(K1[1], kv[1][1], "bf16") <= TOL["bf16"]
     for c in range(3):
         assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL["bf16"]
 
@@ -505,7 +505,7 @@ def test_kv_serving_full_size_sampled():
         kv = O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS, wl.pyramid)
         for c in (u * C, u * C + 317, u * C + C - 1):
             ns_ref = O.autosplit(feats[c:c + 1], b.W, sh.L_NS)[0]     # the oracle's own tokens
-            assert rel_err(NS[c], ns_ref) <= TOL["bf16"]
+            assert stored_err(NS[c], ns_ref, "bf16") <= TOL["bf16"]
             r = O.stage2(kv, ns_ref, b.W, sh.n_heads, EPS)
             assert rel_err(out[c], r) <= TOL["bf16"]
 
@@ -610,7 +610,7 @@ def test_append_full_size_sampled():
     kv = O.append(O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS),
                   O.tokenize_events(ev[u], ty[u], b.W), b.W, sh.n_heads, EPS)
     got = to_np(cache.gather(u, 5, wl.L_S + dL))
-    assert rel_err(got[0], kv[5][0]) <= TOL["bf16"]
+    assert stored_err(got[0], kv[5][0], "bf16") <= TOL["bf16"]
     for c in (u * C, u * C + C - 1):
         assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL["bf16"]
 
