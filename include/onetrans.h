@@ -94,7 +94,11 @@ typedef struct {
  * Per-behavior event MLP and type identifiers ([FR] 7.5.0, MLP_i and the
  * timestamp-aware merge): host arrays of n_behaviors device pointers
  *   Wb1[t] [d, event_dim], bb1[t] [d], Wb2[t] [d, d], bb2[t] [d];
- *   type_emb [n_behaviors, d]                                  (may be NULL) */
+ *   type_emb [n_behaviors, d]                                  (may be NULL)
+ * Optional scoring head on the final NS states, the compact representation
+ * the stack hands downstream ([FR] 7.5.2): logit = w_head . vec(h_NS) +
+ * b_head, vec() token-major (token t = entries t*d .. t*d + d - 1):
+ *   w_head [L_NS*d], b_head [1]                                (may be NULL) */
 typedef struct {
   const void* const* g_attn;
   const void* const* g_ffn;
@@ -118,6 +122,8 @@ typedef struct {
   const void* const* Wb2;
   const void* const* bb2;
   const void* type_emb;
+  const void* w_head;
+  const void* b_head;
 } onetrans_weights;
 
 typedef struct onetrans_model onetrans_model;
@@ -289,13 +295,17 @@ ONETRANS_API onetrans_status onetrans_stage1_encode_ragged(
  * then see that user's own pyramid schedule of cached keys.  A slot with no
  * cached sequence is ONETRANS_ERR_SHAPE.  At most 65536 users per call.
  *   ns_tokens [C_tot, L_NS, d] (candidate-major, as the tokenizer writes it);
- *   ns_out    [C_tot, L_NS, d] float32. */
+ *   ns_out    [C_tot, L_NS, d] float32;
+ *   logits    [C_tot] float32 or NULL: w_head . vec(ns_out[c]) + b_head per
+ *             candidate; non-NULL needs the model's head weights
+ *             (ONETRANS_ERR_UNSUPPORTED otherwise). */
 ONETRANS_API onetrans_status onetrans_stage2_score(const onetrans_model* m,
                                       const onetrans_cache* c,
                                       const int32_t* slots, int32_t U,
                                       const int32_t* cand_offsets,
                                       const void* ns_tokens, void* ns_out,
-                                      void* ws, size_t ws_bytes, void* stream);
+                                      float* logits, void* ws, size_t ws_bytes,
+                                      void* stream);
 
 /* Cross-request append ([FR] 7.5.3): tokenize dL new events per user with the
  * per-behavior MLP plus type identifier, run only those rows through every

@@ -25,6 +25,7 @@ Tokenizer weights:
   Wa1 [H, F], ba1 [H], Wa2 [L_NS*d, H], ba2 [L_NS*d]   auto-split MLP
   Wb1[t] [d, e_t], bb1[t] [d], Wb2[t] [d, d], bb2[t] [d] per-behavior MLP
   type_emb [n_types, d], sep [d]
+  w_head [L_NS*d], b_head [1]                          optional scoring head
 """
 from __future__ import annotations
 
@@ -200,6 +201,9 @@ def make_weights(shape: ModelShape, seed: int, dtype: str, event_dim: int = 0,
     W["bb2"] = [nrm(d) for _ in dims]
     W["type_emb"] = nrm(len(dims), d)
     W["sep"] = nrm(d)
+    # drawn last, so every weight above keeps the values of earlier versions
+    W["w_head"] = nrm(L_NS * d)
+    W["b_head"] = nrm(1)
     return W
 
 

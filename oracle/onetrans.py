@@ -240,6 +240,17 @@ def merge_intent_order(seqs: List[np.ndarray], W: Dict) -> np.ndarray:
     return np.concatenate(parts, axis=0)
 
 
+def score_head(h_ns: np.ndarray, W: Dict) -> np.ndarray:
+    """Optional scoring head on the final NS states.  The pages hand the final
+    NS rows downstream as the compact representation of the candidate
+    ([FR] 7.5.2) and give no head; the reading here is one linear unit over
+    their concatenation: logit = w_head . vec(h_NS) + b_head, vec() taking
+    token 0's d entries first.  h_ns: [..., L_NS, d].  Returns [...]."""
+    h = _f(h_ns)
+    flat = h.reshape(h.shape[:-2] + (h.shape[-2] * h.shape[-1],))
+    return flat @ _f(W["w_head"]) + _f(W["b_head"])[0]
+
+
 # --------------------------------------------------------------------------
 # Two-stage KV-cached serving
 # --------------------------------------------------------------------------

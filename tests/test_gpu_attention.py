@@ -157,6 +157,39 @@ def test_stage2_ragged_users_many_tiles(policy):
             assert rel_err(out[c], O.stage2(kv, NS[c], b.W, sh.n_heads, EPS)) <= TOL["bf16"], (u, c)
 
 
+@pytest.mark.parametrize("dtype,policy", [("bf16", 0), ("bf16", 1), ("fp32", 0)])
+def test_stage2_scoring_head(dtype, policy):
+    """Stage II with the optional head (logit = w_head . vec(final NS rows) +
+    b_head): against the oracle's head on its own Stage II output, and against
+    the GPU's own final rows dotted on the host in fp64, which leaves only the
+    kernel's fp32 summation order."""
+    ot.onetrans_set_kernel_policy(policy)
+    sh = shape(n_layers=2)
+    b = build(sh, 236, dtype, std=attn_std(sh.d))
+    m = b.model
+    L_S, counts = 170, [3, 46]
+    S = gen_normal(237, (2, L_S, sh.d), dtype)
+    offs = np.concatenate([[0], np.cumsum(counts)]).tolist()
+    C = offs[-1]
+    NS = gen_normal(238, (C, sh.L_NS, sh.d), dtype)
+    cache = ot.Cache(m, 2, L_S)
+    ot.onetrans_stage1_encode(m, cache, [0, 1], to_dev(S, tdt(dtype)), m.workspace(ot.OP_STAGE1, 2, L_S))
+    out = torch.empty(C, sh.L_NS, sh.d, dtype=torch.float32, device="cuda")
+    logits = torch.full((C,), float("nan"), dtype=torch.float32, device="cuda")
+    ot.onetrans_stage2_score(m, cache, [0, 1], offs, to_dev(NS, tdt(dtype)), out,
+                             m.workspace(ot.OP_STAGE2, C, L_S), logits=logits)
+    torch.cuda.synchronize()
+    got, rows = to_np(logits), to_np(out)
+    w = b.W["w_head"].astype(np.float64)
+    terms = rows.reshape(C, -1).astype(np.float64) * w
+    own = terms.sum(axis=1) + float(b.W["b_head"][0])
+    assert np.all(np.abs(got - own) <= 1e-5 * np.abs(terms).sum(axis=1) + 1e-6)
+    kvs = [O.stage1(S[u], b.W, sh.L_NS, sh.n_heads, EPS) for u in range(2)]
+    ref = np.array([O.score_head(O.stage2(kvs[u], NS[c], b.W, sh.n_heads, EPS), b.W)
+                    for u in range(2) for c in range(offs[u], offs[u + 1])])
+    assert rel_err(got, ref) <= TOL[dtype]
+
+
 # ------------------------------------------------ lazy rescale of the max
 
 RESCALE_GAP = 8.0    # the kernels raise their running max only past this many base-2 units

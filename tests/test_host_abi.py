@@ -33,7 +33,7 @@ class FakeModel:
     """A model handle whose weight pointers are fake device addresses."""
 
     def __init__(self, n_layers=6, d=256, H=4, dff=1024, L_NS=12, pyramid=None, mode=ot.BF16,
-                 page=64, n_beh=0, event_dim=0, F=512, Hh=3072, align=256, null_field=None):
+                 page=64, n_beh=0, event_dim=0, F=512, Hh=3072, align=256, null_field=None, head=()):
         self.arrs = []
         self.pyr = (ot.I32 * len(pyramid))(*pyramid) if pyramid else None
         self.cfg = ot.Config(n_layers, d, H, dff, L_NS, F, Hh, n_beh, event_dim,
@@ -54,6 +54,8 @@ class FakeModel:
                 self.arrs.append(arr)
                 setattr(w, f, ctypes.cast(arr, ot.PP))
             w.type_emb = addr
+        for f, a in zip(ot._HEAD_FIELDS, head):   # (w_head, b_head) addresses, None to leave one out
+            setattr(w, f, a)
         self.w = w
         self.h = ot.P()
         self.status = ot.lib.onetrans_model_create(ctypes.byref(self.cfg), ctypes.byref(w), ctypes.byref(self.h))
@@ -167,9 +169,11 @@ def test_entry_point_argument_errors_before_any_launch():
     assert ot.lib.onetrans_stage1_encode(fm.h, c, slots, 2, FAKE, 500, ws, big, None) == ot.ERR_SHAPE
     # Stage II on empty slots / bad CSR
     offs = (ot.I32 * 3)(0, 5, 9)
-    assert ot.lib.onetrans_stage2_score(fm.h, c, slots, 2, offs, FAKE, FAKE, ws, big, None) == ot.ERR_SHAPE
+    assert ot.lib.onetrans_stage2_score(fm.h, c, slots, 2, offs, FAKE, FAKE, None, ws, big, None) == ot.ERR_SHAPE
     offs_bad = (ot.I32 * 3)(0, 5, 3)
-    assert ot.lib.onetrans_stage2_score(fm.h, c, slots, 2, offs_bad, FAKE, FAKE, ws, big, None) == ot.ERR_SHAPE
+    assert ot.lib.onetrans_stage2_score(fm.h, c, slots, 2, offs_bad, FAKE, FAKE, None, ws, big, None) == ot.ERR_SHAPE
+    # logits asked of a model without the scoring head
+    assert ot.lib.onetrans_stage2_score(fm.h, c, slots, 2, offs, FAKE, FAKE, FAKE, ws, big, None) == ot.ERR_UNSUPPORTED
     # misaligned workspace / inputs
     assert ot.lib.onetrans_forward(fm.h, FAKE, 2, 1178, FAKE, FAKE + 16, big, None) == ot.ERR_INVALID_ARG
     assert ot.lib.onetrans_forward(fm.h, FAKE + 2, 2, 1178, FAKE, ws, big, None) == ot.ERR_INVALID_ARG
@@ -320,3 +324,10 @@ def test_model_left_alive_until_interpreter_exit_is_destroyed_cleanly(tmp_path):
     assert r.returncode == 0, r.stderr
     assert "made True" in r.stdout
     assert "Exception ignored" not in r.stderr, r.stderr
+
+
+def test_scoring_head_weights_come_in_pairs():
+    assert FakeModel(head=(FAKE, FAKE + 256)).status == ot.OK
+    assert FakeModel(head=(FAKE, None)).status == ot.ERR_INVALID_ARG
+    assert FakeModel(head=(None, FAKE)).status == ot.ERR_INVALID_ARG
+    assert FakeModel(head=(FAKE + 4, FAKE)).status == ot.ERR_INVALID_ARG     # w_head not 16-byte aligned

@@ -264,6 +264,25 @@ def test_autosplit_equals_concat_mlp_reshape():
     np.testing.assert_allclose(O.autosplit(feats, W, shape.L_NS), ref, rtol=1e-12, atol=1e-13)
 
 
+def test_score_head_is_a_linear_unit_over_token_major_concatenation():
+    """The optional head: logit = w_head . vec(h_NS) + b_head.  A one-hot
+    w_head at t*d + k reads entry (t, k), which fixes the concatenation
+    order (token-major); random weights match torch's linear layer over the
+    row-major flattened rows."""
+    shape, W = small_model()
+    h = gen_normal(60, (4, shape.L_NS, shape.d), "fp32")
+    W = dict(W)
+    for t, k in ((0, 0), (1, 5), (shape.L_NS - 1, shape.d - 1)):
+        W["w_head"] = np.zeros(shape.L_NS * shape.d)
+        W["w_head"][t * shape.d + k] = 1.0
+        W["b_head"] = np.array([0.25])
+        np.testing.assert_array_equal(O.score_head(h, W), h[:, t, k].astype(np.float64) + 0.25)
+    W["w_head"] = gen_normal(61, (shape.L_NS * shape.d,), "fp32")
+    W["b_head"] = gen_normal(62, (1,), "fp32")
+    ref = F.linear(t64(h).reshape(4, -1), t64(W["w_head"])[None], t64(W["b_head"]))[:, 0].numpy()
+    np.testing.assert_allclose(O.score_head(h, W), ref, rtol=1e-12, atol=1e-12)
+
+
 GROUP_DIMS, GROUP_HIDDEN = (10, 6, 8, 3), (12, 7, 16, 5)
 
 

@@ -72,12 +72,13 @@ class Config(ctypes.Structure):
 _WEIGHT_FIELDS = ("g_attn", "g_ffn", "Wqkv_S", "Wqkv_NS", "Wo", "W1_S", "b1_S", "W2_S",
                   "b2_S", "W1_NS", "b1_NS", "W2_NS", "b2_NS")
 _TOK_FIELDS = ("Wa1", "ba1", "Wa2", "ba2")
+_HEAD_FIELDS = ("w_head", "b_head")
 _BEH_FIELDS = ("Wb1", "bb1", "Wb2", "bb2")
 
 
 class Weights(ctypes.Structure):
     _fields_ = ([(f, PP) for f in _WEIGHT_FIELDS] + [(f, P) for f in _TOK_FIELDS]
-                + [(f, PP) for f in _BEH_FIELDS] + [("type_emb", P)])
+                + [(f, PP) for f in _BEH_FIELDS] + [("type_emb", P)] + [(f, P) for f in _HEAD_FIELDS])
 
 
 def _sig(name, res, *args):
@@ -100,7 +101,7 @@ _sig("onetrans_tokenize_autosplit", I32, P, P, I64, P, P, SZ, P)
 _sig("onetrans_tokenize_autosplit_static", I32, P, P, I64, P, P)
 _sig("onetrans_stage1_encode", I32, P, P, PI32, I32, P, I32, P, SZ, P)
 _sig("onetrans_stage1_encode_ragged", I32, P, P, PI32, I32, P, PI32, P, SZ, P)
-_sig("onetrans_stage2_score", I32, P, P, PI32, I32, PI32, P, P, P, SZ, P)
+_sig("onetrans_stage2_score", I32, P, P, PI32, I32, PI32, P, P, P, P, SZ, P)
 _sig("onetrans_cache_append", I32, P, P, PI32, I32, P, P, I32, P, SZ, P)
 _sig("onetrans_tokenize_events", I32, P, P, P, I64, P, P)
 _sig("onetrans_merge_intent_order", I32, P, P, PI64, PI32, I32, P, P, P)
@@ -200,7 +201,7 @@ class Model:
             arr = (P * len(ts))(*[_ptr(self._own(t)) for t in ts])
             self._keep.append(arr)
             setattr(w, f, ctypes.cast(arr, PP))
-        for f in _TOK_FIELDS + ("type_emb",):
+        for f in _TOK_FIELDS + ("type_emb",) + _HEAD_FIELDS:
             t = weights.get(f)
             if t is not None:
                 setattr(w, f, _ptr(self._own(t)))
@@ -351,11 +352,14 @@ def onetrans_stage1_encode_ragged(model: Model, cache: Cache, slots: Sequence[in
 
 
 def onetrans_stage2_score(model: Model, cache: Cache, slots: Sequence[int], cand_offsets: Sequence[int],
-                          ns_tokens: torch.Tensor, ns_out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+                          ns_tokens: torch.Tensor, ns_out: torch.Tensor, ws: torch.Tensor, stream=None,
+                          logits: Optional[torch.Tensor] = None) -> None:
+    """ns_tokens [C, L_NS, d]; ns_out [C, L_NS, d] float32; logits [C] float32
+    or None (needs the model's w_head / b_head)."""
     sl, co = _i32(slots), _i32(cand_offsets)
     _check("onetrans_stage2_score", lib.onetrans_stage2_score(
-        model.handle, cache.handle, sl, len(slots), co, _ptr(ns_tokens), _ptr(ns_out), _ptr(ws), ws.numel(),
-        _stream(stream)))
+        model.handle, cache.handle, sl, len(slots), co, _ptr(ns_tokens), _ptr(ns_out), _ptr(logits), _ptr(ws),
+        ws.numel(), _stream(stream)))
 
 
 def onetrans_cache_append(model: Model, cache: Cache, slots: Sequence[int], events: torch.Tensor,

@@ -28,7 +28,7 @@ struct onetrans_model {
   bool bf16;
   std::vector<const void*> g_attn, g_ffn, Wqkv_S, Wqkv_NS, Wo, W1_S, b1_S, W2_S, b2_S, W1_NS,
       b1_NS, W2_NS, b2_NS, Wb1, bb1, Wb2, bb2;
-  const void *Wa1, *ba1, *Wa2, *ba2, *type_emb;
+  const void *Wa1, *ba1, *Wa2, *ba2, *type_emb, *w_head, *b_head;
 };
 
 struct onetrans_cache {
@@ -50,11 +50,11 @@ static int g_policy = 0;
 // tagged with a kernel kind and its algorithmic FLOPs and bytes.
 enum ProfKind {
   PK_GEMM_QKV = 0, PK_GEMM_OPROJ, PK_GEMM_FFN_UP, PK_GEMM_FFN_DOWN, PK_GEMM_AUTOSPLIT, PK_ATTN_CAUSAL,
-  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_BLOCK_TAIL, PK_COUNT
+  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_BLOCK_TAIL, PK_HEAD, PK_COUNT
 };
 static const char* kProfNames[PK_COUNT] = {"gemm_qkv", "gemm_oproj_rms", "gemm_ffn_up_gelu", "gemm_ffn_down_rms",
                                            "gemm_autosplit", "attn_causal", "attn_stage2", "rmsnorm",
-                                           "tokenize_events", "fused_oproj_ffn"};
+                                           "tokenize_events", "fused_oproj_ffn", "score_head"};
 struct ProfRec {
   int kind;
   cudaEvent_t e0, e1;
@@ -618,11 +618,25 @@ static onetrans_status stage1_impl(const onetrans_model* m, onetrans_cache* c, c
   return ONETRANS_OK;
 }
 
+// ========================================================= scoring head ==
+// logit[c] = w_head . vec(final NS rows of candidate c) + b_head.
+template <typename T>
+static onetrans_status launch_head(const onetrans_model* m, const float* h, long long C, float* logits,
+                                   cudaStream_t st) {
+  if (C <= 0) return ONETRANS_OK;
+  const int n = m->L_NS * m->d;
+  ProfScope prof(PK_HEAD, 2.0 * C * n, (double)C * (n * 4.0 + 4.0) + (double)n * m->es, st);
+  const unsigned blocks = (unsigned)cdiv(C, 8);
+  launch_dependent(head_logits_kernel<T>, dim3(blocks), dim3(256), 0, st, h, (const T*)m->w_head,
+                   (const T*)m->b_head, n, C, logits);
+  return last_launch();
+}
+
 // ============================================================= stage II ==
 template <typename T>
 static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache* c, const int* slots,
-                                   int U, const int* offs, const void* ns_in, void* ns_out, void* ws,
-                                   size_t ws_bytes, cudaStream_t st, size_t* need, long long C_need,
+                                   int U, const int* offs, const void* ns_in, void* ns_out, float* logits,
+                                   void* ws, size_t ws_bytes, cudaStream_t st, size_t* need, long long C_need,
                                    int L_S_need) {
   const int d = m->d, dff = m->dff, L_NS = m->L_NS, es = m->es;
   const long long C = need ? C_need : offs[U] - offs[0];
@@ -745,6 +759,7 @@ static onetrans_status stage2_impl(const onetrans_model* m, const onetrans_cache
     }
     x_in = x_next;
   }
+  if (logits) OT_TRY(launch_head<T>(m, (const float*)ns_out, C, logits, st));
   return ONETRANS_OK;
 }
 
@@ -1021,6 +1036,8 @@ onetrans_status onetrans_model_create(const onetrans_config* cfg, const onetrans
     for (int l = 0; l < NL; ++l)
       if (!arr[l] || !aligned(arr[l], 16)) return ONETRANS_ERR_INVALID_ARG;
   }
+  if ((w->w_head != nullptr) != (w->b_head != nullptr) || (w->w_head && !aligned(w->w_head, 16)))
+    return ONETRANS_ERR_INVALID_ARG;
   std::vector<int> pyr;
   if (cfg->pyramid_q) {
     for (int l = 0; l < NL; ++l) {
@@ -1043,6 +1060,7 @@ onetrans_status onetrans_model_create(const onetrans_config* cfg, const onetrans
   m->W2_S = cp(w->W2_S); m->b2_S = cp(w->b2_S); m->W1_NS = cp(w->W1_NS); m->b1_NS = cp(w->b1_NS);
   m->W2_NS = cp(w->W2_NS); m->b2_NS = cp(w->b2_NS);
   m->Wa1 = w->Wa1; m->ba1 = w->ba1; m->Wa2 = w->Wa2; m->ba2 = w->ba2; m->type_emb = w->type_emb;
+  m->w_head = w->w_head; m->b_head = w->b_head;
   const int nb = cfg->n_behaviors;
   if (nb > 0 && w->Wb1 && w->bb1 && w->Wb2 && w->bb2) {
     m->Wb1.assign(w->Wb1, w->Wb1 + nb); m->bb1.assign(w->bb1, w->bb1 + nb);
@@ -1080,10 +1098,10 @@ onetrans_status onetrans_workspace_size(const onetrans_model* m, int32_t op, int
       return m->bf16 ? stage1_impl<__nv_bfloat16>(m, nullptr, nullptr, nn, nullptr, L, nullptr, 0, 0, bytes)
                      : stage1_impl<float>(m, nullptr, nullptr, nn, nullptr, L, nullptr, 0, 0, bytes);
     case ONETRANS_OP_STAGE2:
-      return m->bf16 ? stage2_impl<__nv_bfloat16>(m, nullptr, nullptr, 1, nullptr, nullptr, nullptr, nullptr, 0,
-                                                  0, bytes, n, L)
-                     : stage2_impl<float>(m, nullptr, nullptr, 1, nullptr, nullptr, nullptr, nullptr, 0, 0,
-                                          bytes, n, L);
+      return m->bf16 ? stage2_impl<__nv_bfloat16>(m, nullptr, nullptr, 1, nullptr, nullptr, nullptr, nullptr,
+                                                  nullptr, 0, 0, bytes, n, L)
+                     : stage2_impl<float>(m, nullptr, nullptr, 1, nullptr, nullptr, nullptr, nullptr, nullptr, 0,
+                                          0, bytes, n, L);
     case ONETRANS_OP_APPEND:
       return m->bf16 ? append_impl<__nv_bfloat16>(m, nullptr, nullptr, nn, nullptr, nullptr, L, nullptr, 0, 0,
                                                   bytes)
@@ -1307,10 +1325,11 @@ onetrans_status onetrans_stage1_encode_ragged(const onetrans_model* m, onetrans_
 
 onetrans_status onetrans_stage2_score(const onetrans_model* m, const onetrans_cache* c, const int32_t* slots,
                                       int32_t U, const int32_t* cand_offsets, const void* ns_tokens,
-                                      void* ns_out, void* ws, size_t ws_bytes, void* stream) {
+                                      void* ns_out, float* logits, void* ws, size_t ws_bytes, void* stream) {
   if (!m || !c || c->m != m) return ONETRANS_ERR_INVALID_ARG;
   OT_TRY(check_slots(c, slots, U));
   if (U == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (logits && !m->w_head) return ONETRANS_ERR_UNSUPPORTED;
   if (U > kMaxUsers) return ONETRANS_ERR_SHAPE;
   if (!cand_offsets) return ONETRANS_ERR_INVALID_ARG;
   for (int u = 0; u < U; ++u)
@@ -1320,11 +1339,12 @@ onetrans_status onetrans_stage2_score(const onetrans_model* m, const onetrans_ca
     if (c->len[slots[u]] == 0) return ONETRANS_ERR_SHAPE;
   if (cand_offsets[U] == 0) return ONETRANS_OK;  // no candidates
   if (!ns_tokens || !ns_out || !aligned(ns_tokens, 16) || !aligned(ns_out, 16)) return ONETRANS_ERR_INVALID_ARG;
+  if (logits && !aligned(logits, 4)) return ONETRANS_ERR_INVALID_ARG;
   OT_TRY(check_ws(ws));
   cudaStream_t st = (cudaStream_t)stream;
-  return m->bf16 ? stage2_impl<__nv_bfloat16>(m, c, slots, U, cand_offsets, ns_tokens, ns_out, ws, ws_bytes,
-                                              st, nullptr, 0, 0)
-                 : stage2_impl<float>(m, c, slots, U, cand_offsets, ns_tokens, ns_out, ws, ws_bytes, st,
+  return m->bf16 ? stage2_impl<__nv_bfloat16>(m, c, slots, U, cand_offsets, ns_tokens, ns_out, logits, ws,
+                                              ws_bytes, st, nullptr, 0, 0)
+                 : stage2_impl<float>(m, c, slots, U, cand_offsets, ns_tokens, ns_out, logits, ws, ws_bytes, st,
                                       nullptr, 0, 0);
 }
 

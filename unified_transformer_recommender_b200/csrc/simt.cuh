@@ -498,3 +498,36 @@ __global__ void __launch_bounds__(256) event_tokenize_tile_kernel(const T* ev, c
 }
 
 }  // namespace ot
+
+namespace ot {
+
+// ------------------------------------------------------------ scoring head --
+// logit[c] = w . vec(h[c]) + b over the n = L_NS * d float32 entries of
+// candidate c's final NS rows (token-major, as the stack writes them).  One
+// warp per candidate, 16-byte loads of h, fp32 accumulation, a shuffle
+// reduction.  HBM-bound: n * 4 bytes read per candidate (the rows were just
+// written by the last layer, so mostly from L2).
+template <typename T>
+__global__ void __launch_bounds__(256) head_logits_kernel(const float* __restrict__ h, const T* __restrict__ w,
+                                                          const T* __restrict__ b, int n, long long C,
+                                                          float* __restrict__ logits) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int lane = threadIdx.x & 31;
+  const long long c = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (c >= C) return;
+  const float4* hr = (const float4*)(h + c * (long long)n);
+  float acc = 0.f;
+  for (int i = lane; i < n / 4; i += 32) {
+    const float4 x = hr[i];
+    acc = fmaf(x.x, to_f(w[4 * i + 0]), acc);
+    acc = fmaf(x.y, to_f(w[4 * i + 1]), acc);
+    acc = fmaf(x.z, to_f(w[4 * i + 2]), acc);
+    acc = fmaf(x.w, to_f(w[4 * i + 3]), acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) logits[c] = acc + to_f(b[0]);
+}
+
+}  // namespace ot
