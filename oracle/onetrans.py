@@ -340,3 +340,153 @@ def append(cache: List[tuple], new_S: np.ndarray, W: Dict, n_heads: int,
         x = x1 + mixed_ffn_rows(rmsnorm(x1, W["g_ffn"][l], eps), W, l, s,
                                 range(s_old, s))
     return out
+
+
+# --------------------------------------------------------------------------
+# Backward pass (training: gradients of the block stack)
+# --------------------------------------------------------------------------
+#
+# The pages train the stack end to end and speed it up by recomputing
+# activations in the backward pass ([FR] 7.5.3 system optimizations; [PD]
+# 4.3, the "+ mixed precision + recomputation" row).  The oracle gives the
+# exact gradient by the chain rule, step by step in reverse order of
+# `block`; it keeps each layer's input and recomputes the layer's
+# intermediates, the recomputation scheme itself.  The upstream gradient dY
+# of the stack's output defines the loss: L = sum(dY * Y).
+
+_GRAD_KEYS = ("g_attn", "g_ffn", "Wqkv_S", "Wqkv_NS", "Wo", "W1_S", "b1_S", "W2_S",
+              "b2_S", "W1_NS", "b1_NS", "W2_NS", "b2_NS")
+
+
+def rmsnorm_backward(x: np.ndarray, g: np.ndarray, eps: float, dy: np.ndarray):
+    """Gradients of y = x r g, r = (mean(x^2) + eps)^(-1/2), over rows x.
+    Returns (dx, dg): dx = r (g dy) - x r^3 sum(g dy x) / d, dg = sum_rows dy x r."""
+    x, g, dy = _f(x), _f(g), _f(dy)
+    d = x.shape[-1]
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    gy = dy * g
+    dx = r * gy - x * r ** 3 * np.sum(gy * x, axis=-1, keepdims=True) / d
+    dg = np.sum(dy * x * r, axis=tuple(range(x.ndim - 1)))
+    return dx, dg
+
+
+def gelu_tanh_grad(x: np.ndarray) -> np.ndarray:
+    """d/dx of 0.5 x (1 + tanh(c (x + 0.044715 x^3))), c = sqrt(2/pi)."""
+    x = _f(x)
+    c = np.sqrt(2.0 / np.pi)
+    t = np.tanh(c * (x + 0.044715 * x ** 3))
+    return 0.5 * (1.0 + t) + 0.5 * x * (1.0 - t * t) * c * (1.0 + 3 * 0.044715 * x * x)
+
+
+def masked_attention_backward(q, k, v, q_pos, n_heads: int, do: np.ndarray):
+    """Gradients of masked_attention with respect to q, k, v for the output
+    gradient do [Lq, d].  Per head, with P the softmax of the masked scores:
+    dV = P^T dO, dP = dO V^T, dS = P (dP - rowsum(dP P)), dQ = dS K / sqrt(d_h),
+    dK = dS^T Q / sqrt(d_h)."""
+    q, k, v, do = _f(q), _f(k), _f(v), _f(do)
+    Lq, d = q.shape
+    Lk = k.shape[0]
+    dh = d // n_heads
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    visible = np.arange(Lk)[None, :] <= np.asarray(q_pos)[:, None]
+    for h in range(n_heads):
+        sl = slice(h * dh, (h + 1) * dh)
+        s = np.where(visible, q[:, sl] @ k[:, sl].T / np.sqrt(dh), -np.inf)
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p = p / p.sum(axis=1, keepdims=True)
+        dv[:, sl] = p.T @ do[:, sl]
+        dp = do[:, sl] @ v[:, sl].T
+        ds = p * (dp - np.sum(dp * p, axis=1, keepdims=True))
+        dq[:, sl] = ds @ k[:, sl] / np.sqrt(dh)
+        dk[:, sl] = ds.T @ q[:, sl] / np.sqrt(dh)
+    return dq, dk, dv
+
+
+def _zero_grads(W: Dict, l: int) -> Dict:
+    return {key: np.zeros(np.shape(W[key][l])) for key in _GRAD_KEYS}
+
+
+def block_backward(x: np.ndarray, W: Dict, l: int, L_NS: int, Lq: int, n_heads: int,
+                   eps: float, dy: np.ndarray):
+    """Gradient of `block` (one sample, layer l) for the output gradient
+    dy [Lq, d].  Recomputes the block's intermediates from its input x [L, d]
+    and returns (dx [L, d], grads of layer l's weights keyed like W)."""
+    x, dy = _f(x), _f(dy)
+    L, d = x.shape
+    n_S = L - L_NS
+    tail = list(range(L - Lq, L))
+    G = _zero_grads(W, l)
+    # ---- recompute the forward
+    h = rmsnorm(x, W["g_attn"][l], eps)
+    _, k, v = qkv_rows(h, W, l, n_S, range(L))
+    q, _, _ = qkv_rows(h, W, l, n_S, tail)
+    a = masked_attention(q, k, v, np.asarray(tail), n_heads)
+    x1 = x[tail] + a @ _f(W["Wo"][l]).T
+    h2 = rmsnorm(x1, W["g_ffn"][l], eps)
+    # ---- y = x1 + MixedFFN(h2): per row, the row's weight set
+    dx1 = dy.copy()
+    dh2 = np.empty_like(h2)
+    for t, i in enumerate(tail):
+        _, W1, b1, W2, _ = _row_weights(W, l, n_S, i)
+        u = _f(W1) @ h2[t] + _f(b1)
+        z = gelu_tanh(u)
+        du = (_f(W2).T @ dy[t]) * gelu_tanh_grad(u)
+        dh2[t] = _f(W1).T @ du
+        if i < n_S:
+            G["W2_S"] += np.outer(dy[t], z); G["b2_S"] += dy[t]
+            G["W1_S"] += np.outer(du, h2[t]); G["b1_S"] += du
+        else:
+            j = i - n_S
+            G["W2_NS"][j] += np.outer(dy[t], z); G["b2_NS"][j] += dy[t]
+            G["W1_NS"][j] += np.outer(du, h2[t]); G["b1_NS"][j] += du
+    dxn, G["g_ffn"] = rmsnorm_backward(x1, W["g_ffn"][l], eps, dh2)
+    dx1 += dxn
+    # ---- x1 = x[tail] + W^O a
+    G["Wo"] = dx1.T @ a
+    da = dx1 @ _f(W["Wo"][l])
+    dx = np.zeros_like(x)
+    dx[tail] += dx1
+    # ---- attention, then (q, k, v) = W_i^{Q,K,V} h_i per row
+    dq, dk, dv = masked_attention_backward(q, k, v, np.asarray(tail), n_heads, da)
+    dqkv = np.zeros((L, 3 * d))
+    dqkv[tail, :d] = dq
+    dqkv[:, d:2 * d] = dk
+    dqkv[:, 2 * d:] = dv
+    dh = np.empty_like(h)
+    for i in range(L):
+        Wi = _f(W["Wqkv_S"][l] if i < n_S else W["Wqkv_NS"][l][i - n_S])
+        dh[i] = Wi.T @ dqkv[i]
+        if i < n_S:
+            G["Wqkv_S"] += np.outer(dqkv[i], h[i])
+        else:
+            G["Wqkv_NS"][i - n_S] += np.outer(dqkv[i], h[i])
+    dxh, G["g_attn"] = rmsnorm_backward(x, W["g_attn"][l], eps, dh)
+    dx += dxh
+    return dx, G
+
+
+def forward_backward(X0: np.ndarray, W: Dict, L_NS: int, n_heads: int, eps: float,
+                     schedule: Optional[Sequence[int]], dY: np.ndarray):
+    """Forward of the stack keeping only each layer's input, then the
+    backward layer by layer, recomputing each layer from its input.
+    X0 [B, L0, d], dY [B, L'_N, d].  Returns (Y, dX0, dW) with dW[key] a list
+    over layers, summed over the batch."""
+    X0, dY = _f(X0), _f(dY)
+    N = len(W["Wo"])
+    dW = {key: [np.zeros(np.shape(W[key][l])) for l in range(N)] for key in _GRAD_KEYS}
+    Y, dX = [], []
+    for b in range(X0.shape[0]):
+        xs = [X0[b]]
+        for l in range(N):
+            Lq = xs[-1].shape[0] if schedule is None else int(schedule[l])
+            xs.append(block(xs[-1], W, l, L_NS, Lq, n_heads, eps))
+        Y.append(xs[-1])
+        g = dY[b]
+        for l in reversed(range(N)):
+            Lq = xs[l + 1].shape[0]
+            g, G = block_backward(xs[l], W, l, L_NS, Lq, n_heads, eps, g)
+            for key in _GRAD_KEYS:
+                dW[key][l] += G[key]
+        dX.append(g)
+    return np.stack(Y), np.stack(dX), dW
