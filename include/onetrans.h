@@ -126,6 +126,26 @@ typedef struct {
   const void* b_head;
 } onetrans_weights;
 
+/* Weight gradients (float32 device pointers, laid out like onetrans_weights'
+ * block-stack fields: per-layer fields are HOST arrays of n_layers device
+ * pointers; each gradient has its weight's shape).  Written, not
+ * accumulated, by onetrans_forward_backward. */
+typedef struct {
+  float* const* g_attn;
+  float* const* g_ffn;
+  float* const* Wqkv_S;
+  float* const* Wqkv_NS;
+  float* const* Wo;
+  float* const* W1_S;
+  float* const* b1_S;
+  float* const* W2_S;
+  float* const* b2_S;
+  float* const* W1_NS;
+  float* const* b1_NS;
+  float* const* W2_NS;
+  float* const* b2_NS;
+} onetrans_grads;
+
 typedef struct onetrans_model onetrans_model;
 typedef struct onetrans_cache onetrans_cache;
 
@@ -136,7 +156,8 @@ typedef enum {
   ONETRANS_OP_STAGE2 = 2,    /* n = total candidates, L = cached L_S */
   ONETRANS_OP_APPEND = 3,    /* n = U users,   L = dL */
   ONETRANS_OP_AUTOSPLIT = 4, /* n = N feature rows, L unused */
-  ONETRANS_OP_GROUPWISE = 5  /* n = N feature rows, L = h_max (padded hidden width) */
+  ONETRANS_OP_GROUPWISE = 5, /* n = N feature rows, L = h_max (padded hidden width) */
+  ONETRANS_OP_TRAIN = 6      /* n = B samples, L = L_S (onetrans_forward_backward) */
 } onetrans_op;
 
 /* Validate `cfg`/`w` and create a model.  Copies the config and the pointer
@@ -327,6 +348,24 @@ ONETRANS_API onetrans_status onetrans_cache_append(const onetrans_model* m,
 ONETRANS_API onetrans_status onetrans_forward(const onetrans_model* m, const void* x0,
                                  int32_t B, int32_t L_S, void* out, void* ws,
                                  size_t ws_bytes, void* stream);
+
+/* Training step of the stack (the pages train it end to end and cut training
+ * time and memory with mixed precision and activation recomputation: [FR]
+ * 7.5.3 system optimizations; paper-daily 4.3, the "+ mixed precision +
+ * recomputation" row).  Forward over x0 [B, L_S + L_NS, d] (the mode's
+ * type) keeping only each layer's input, then the backward layer by layer,
+ * each layer's intermediates recomputed from its input.  The loss gradient
+ * enters as dy [B, L'_N, d] float32, the gradient of the output out
+ * [B, L'_N, d] float32 (the rows onetrans_forward returns).  Writes out,
+ * dx0 [B, L_S + L_NS, d] float32 (gradient of x0) and every weight gradient
+ * of `grads`.  In BF16 mode every matrix operand is bf16 with float32
+ * accumulation and every gradient float32; FP32 mode is float32
+ * throughout.  Workspace: ONETRANS_OP_TRAIN with n = B, L = L_S. */
+ONETRANS_API onetrans_status onetrans_forward_backward(const onetrans_model* m, const void* x0,
+                                          int32_t B, int32_t L_S, const float* dy,
+                                          float* out, float* dx0,
+                                          const onetrans_grads* grads, void* ws,
+                                          size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------- plumbing --
  * Kernel selection for tests: 0 = automatic (tensor-core kernels where the

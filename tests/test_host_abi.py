@@ -22,7 +22,7 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 27
+    assert len(names) == 28
     for n in names:
         assert hasattr(ot.lib, n), n
     assert set(names) == set(ot.SYMBOLS)
@@ -331,3 +331,27 @@ def test_scoring_head_weights_come_in_pairs():
     assert FakeModel(head=(FAKE, None)).status == ot.ERR_INVALID_ARG
     assert FakeModel(head=(None, FAKE)).status == ot.ERR_INVALID_ARG
     assert FakeModel(head=(FAKE + 4, FAKE)).status == ot.ERR_INVALID_ARG     # w_head not 16-byte aligned
+
+
+def test_forward_backward_argument_errors_before_any_launch():
+    sched = linear_pyramid(1190, 12, 6)
+    fm = FakeModel(pyramid=sched)
+    g = ot.Grads()
+    arrs = []
+    for f in ot._WEIGHT_FIELDS:
+        arr = (ot.P * 6)(*[FAKE + i * 256 for i in range(6)])
+        arrs.append(arr)
+        setattr(g, f, ctypes.cast(arr, ot.PP))
+    fb = ot.lib.onetrans_forward_backward
+    big = 1 << 40
+    assert fb(fm.h, FAKE, 2, 1178, FAKE, FAKE, FAKE, None, FAKE, big, None) == ot.ERR_INVALID_ARG   # no grads
+    assert fb(fm.h, None, 0, 1178, None, None, None, ctypes.byref(g), None, 0, None) == ot.OK   # no samples
+    assert fb(fm.h, FAKE, 2, 900, FAKE, FAKE, FAKE, ctypes.byref(g), FAKE, big, None) == ot.ERR_SHAPE  # schedule
+    assert fb(fm.h, FAKE + 2, 2, 1178, FAKE, FAKE, FAKE, ctypes.byref(g), FAKE, big, None) == ot.ERR_INVALID_ARG
+    assert fb(fm.h, FAKE, 2, 1178, FAKE, FAKE, None, ctypes.byref(g), FAKE, big, None) == ot.ERR_INVALID_ARG
+    assert fb(fm.h, FAKE, 2, 1178, FAKE, FAKE, FAKE, ctypes.byref(g), FAKE, 1024, None) == ot.ERR_CAPACITY
+    arrs[4][3] = FAKE + 4                                              # Wo gradient of layer 3 misaligned
+    assert fb(fm.h, FAKE, 2, 1178, FAKE, FAKE, FAKE, ctypes.byref(g), FAKE, big, None) == ot.ERR_INVALID_ARG
+    out = ot.SZ(0)
+    assert ot.lib.onetrans_workspace_size(fm.h, ot.OP_TRAIN, 2, 1178, ctypes.byref(out)) == ot.OK
+    assert out.value > 2 * 1190 * 256 * 4 * 5                       # at least the kept layer inputs

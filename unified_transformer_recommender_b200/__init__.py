@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libonetrans.so")
 
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_DEVICE_CHECK = 0, -1, -2, -3, -4, -5, -6
 BF16, FP32 = 0, 1
-OP_FORWARD, OP_STAGE1, OP_STAGE2, OP_APPEND, OP_AUTOSPLIT, OP_GROUPWISE = 0, 1, 2, 3, 4, 5
+OP_FORWARD, OP_STAGE1, OP_STAGE2, OP_APPEND, OP_AUTOSPLIT, OP_GROUPWISE, OP_TRAIN = 0, 1, 2, 3, 4, 5, 6
 
 SYMBOLS = (
     "onetrans_model_create", "onetrans_model_destroy", "onetrans_workspace_size",
@@ -33,7 +33,7 @@ SYMBOLS = (
     "onetrans_device_status", "onetrans_status_string", "onetrans_version",
     "onetrans_profile_enable", "onetrans_profile_kinds", "onetrans_profile_read",
     "onetrans_tokenize_autosplit_static", "onetrans_tokenize_events", "onetrans_merge_intent_order",
-    "onetrans_tokenize_groupwise", "onetrans_selftest_bounded_wait",
+    "onetrans_tokenize_groupwise", "onetrans_selftest_bounded_wait", "onetrans_forward_backward",
 )
 
 
@@ -81,6 +81,11 @@ class Weights(ctypes.Structure):
                 + [(f, PP) for f in _BEH_FIELDS] + [("type_emb", P)] + [(f, P) for f in _HEAD_FIELDS])
 
 
+class Grads(ctypes.Structure):
+    """onetrans_grads: per-layer host arrays of float32 device pointers."""
+    _fields_ = [(f, PP) for f in _WEIGHT_FIELDS]
+
+
 def _sig(name, res, *args):
     fn = getattr(lib, name)
     fn.restype = res
@@ -107,6 +112,7 @@ _sig("onetrans_tokenize_events", I32, P, P, P, I64, P, P)
 _sig("onetrans_merge_intent_order", I32, P, P, PI64, PI32, I32, P, P, P)
 _sig("onetrans_tokenize_groupwise", I32, P, P, I64, I32, I32, I32, P, P, P, P, P, P, SZ, P)
 _sig("onetrans_forward", I32, P, P, I32, I32, P, P, SZ, P)
+_sig("onetrans_forward_backward", I32, P, P, I32, I32, P, P, P, P, P, SZ, P)
 _sig("onetrans_set_kernel_policy", I32, I32)
 _sig("onetrans_device_status", I32, P, PI32)
 _sig("onetrans_selftest_bounded_wait", I32, I32, P)
@@ -397,3 +403,20 @@ def model_from_arrays(shape, weights: Dict, pyramid_q=None, mode: int = BF16, de
                  L_NS=shape.L_NS, weights=tw, pyramid_q=pyramid_q, mode=mode,
                  ns_feat_dim=shape.ns_feat, ns_hidden=shape.ns_hidden, n_behaviors=n_beh,
                  event_dim=event_dim, rms_eps=shape.eps)
+
+
+def onetrans_forward_backward(model: Model, x0: torch.Tensor, dy: torch.Tensor, out: torch.Tensor,
+                              dx0: torch.Tensor, grads: Dict[str, Sequence[torch.Tensor]], ws: torch.Tensor,
+                              stream=None) -> None:
+    """x0 [B, L_S + L_NS, d] (model dtype); dy, out [B, L'_N, d] and dx0 [B, L_S + L_NS, d] float32;
+    grads maps each block-stack weight name to per-layer float32 tensors of the weight's shape."""
+    B, L0, _ = x0.shape
+    g = Grads()
+    keep = []
+    for f in _WEIGHT_FIELDS:
+        arr = (P * model.n_layers)(*[_ptr(t) for t in grads[f]])
+        keep.append(arr)
+        setattr(g, f, ctypes.cast(arr, PP))
+    _check("onetrans_forward_backward", lib.onetrans_forward_backward(
+        model.handle, _ptr(x0), B, L0 - model.L_NS, _ptr(dy), _ptr(out), _ptr(dx0), ctypes.byref(g), _ptr(ws),
+        ws.numel(), _stream(stream)))

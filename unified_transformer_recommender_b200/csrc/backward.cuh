@@ -1,0 +1,281 @@
+// Kernels of the training path: the backward pass of the block stack with
+// activation recomputation.  The contractions themselves run on the GEMM
+// kernels of the forward path (tcgen05 where the shape allows); these
+// kernels supply what the forward kernels do not: operand transposes (the
+// backward's GEMMs contract over rows, so their operands are the forward's
+// rows transposed, K-major, zero-padded to a multiple of 64 rows), column
+// sums (bias and gain gradients), the RMSNorm and GELU backward steps, and
+// attention forward / backward on rows recomputed from the layer input.
+#pragma once
+#include "common.cuh"
+
+namespace ot {
+
+// Row r of group g of a gathered row set: src + g*gs + (r / T)*sb + (r % T)*st
+// (T rows per sample, sample stride sb, row stride st).
+struct RowSet {
+  long long gs, sb, st;
+  int T, R;  // rows per sample, rows in the set
+};
+
+__device__ inline long long rowset_off(const RowSet& s, int g, int r) {
+  const int b = r / s.T, t = r - b * s.T;
+  return (long long)g * s.gs + (long long)b * s.sb + (long long)t * s.st;
+}
+
+// dst[g][c][r] = src row r of group g, column c (r < R), 0 for R <= r < R_pad:
+// the K-major operand of a GEMM that contracts over rows.  32 x 32 tiles
+// through shared memory, so both the reads and the writes are coalesced.
+template <typename Ti, typename To>
+__global__ void __launch_bounds__(256) transpose_rows_kernel(const Ti* __restrict__ src, RowSet s, int C,
+                                                             To* __restrict__ dst, int R_pad) {
+  __shared__ float tile[32][33];
+  const int g = blockIdx.z, c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty + 8 * i, c = c0 + tx;
+    tile[ty + 8 * i][tx] = (r < s.R && c < C) ? to_f(src[rowset_off(s, g, r) + c]) : 0.f;
+  }
+  __syncthreads();
+  To* out = dst + (long long)g * C * R_pad;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = c0 + ty + 8 * i, r = r0 + tx;
+    if (c < C && r < R_pad) out[(long long)c * R_pad + r] = from_f<To>(tile[tx][ty + 8 * i]);
+  }
+}
+
+// dst[g * dst_gs + c] = sum over the set's rows r of src row r, column c.
+// 32 columns per CTA, 8 row lanes per column, fixed summation order.
+__global__ void __launch_bounds__(256) colsum_kernel(const float* __restrict__ src, RowSet s, int C,
+                                                     float* __restrict__ dst, long long dst_gs) {
+  __shared__ float part[8][33];
+  const int g = blockIdx.y, tx = threadIdx.x & 31, ty = threadIdx.x >> 5, c = blockIdx.x * 32 + tx;
+  float acc = 0.f;
+  if (c < C)
+    for (int r = ty; r < s.R; r += 8) acc += src[rowset_off(s, g, r) + c];
+  part[ty][tx] = acc;
+  __syncthreads();
+  if (ty == 0 && c < C) {
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t += part[i][tx];
+    dst[(long long)g * dst_gs + c] = t;
+  }
+}
+
+// RMSNorm backward for y = x r g, r = (mean(x^2) + eps)^(-1/2), one warp per
+// row (rows (b, t) through x's and dx's sample and row strides, `fold` rows
+// per sample):  dx += r g dy - x r^3 sum(g dy x) / d, and pg = dy x r, the
+// row's share of dg (summed over rows by colsum_kernel).
+template <typename Tx, typename T>
+__global__ void __launch_bounds__(256) rms_backward_kernel(const Tx* __restrict__ x, long long x_sb, long long x_st,
+                                                           const T* __restrict__ gamma, const float* __restrict__ dy,
+                                                           float* __restrict__ dx, long long dx_sb, long long dx_st,
+                                                           float* __restrict__ pg, int rows, int fold, int d, float eps) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int b = row / fold, t = row - b * fold;
+  const Tx* xr = x + b * x_sb + t * x_st;
+  const float* dyr = dy + (long long)row * d;
+  float ss = 0.f, sg = 0.f;
+  for (int k = lane; k < d; k += 32) {
+    const float xv = to_f(xr[k]), gy = to_f(gamma[k]) * dyr[k];
+    ss = fmaf(xv, xv, ss);
+    sg = fmaf(gy, xv, sg);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    sg += __shfl_xor_sync(0xffffffffu, sg, o);
+  }
+  const float r = rsqrtf(ss / d + eps);
+  const float c3 = r * r * r * sg / d;
+  float* dxr = dx + b * dx_sb + t * dx_st;
+  float* pgr = pg + (long long)row * d;
+  for (int k = lane; k < d; k += 32) {
+    const float xv = to_f(xr[k]), g = to_f(gamma[k]), dv = dyr[k];
+    dxr[k] += r * g * dv - xv * c3;
+    pgr[k] = dv * xv * r;
+  }
+}
+
+// d/du of GELU-tanh: 0.5 (1 + tanh(v)) + 0.5 u (1 - tanh^2(v)) c (1 + 3 a u^2),
+// v = c (u + a u^3), c = sqrt(2/pi), a = 0.044715.
+__device__ inline float gelu_tanh_grad(float u) {
+  const float c = 0.7978845608028654f, a = 0.044715f;
+  const float th = tanhf(c * (u + a * u * u * u));
+  return 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * a * u * u);
+}
+
+// z = GELU(u) in the storage type (the FFN's hidden layer, recomputed).
+template <typename T>
+__global__ void gelu_forward_kernel(const float* __restrict__ u, T* __restrict__ z, long long n) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) z[i] = from_f<T>(gelu_tanh(u[i]));
+}
+
+// du = dz * GELU'(u): float32 (its column sums are db1) and the storage type
+// (the operand of the next GEMMs).
+template <typename T>
+__global__ void gelu_backward_kernel(const float* __restrict__ dz, const float* __restrict__ u,
+                                     float* __restrict__ du32, T* __restrict__ du, long long n) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    const float v = dz[i] * gelu_tanh_grad(u[i]);
+    du32[i] = v;
+    du[i] = from_f<T>(v);
+  }
+}
+
+template <typename T>
+__global__ void cast_kernel(const float* __restrict__ src, T* __restrict__ dst, long long n) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = from_f<T>(src[i]);
+}
+
+// ------------------------------------------------ attention on plain rows --
+// qkv [B, L, 3d] (q | k | v of every row, q unscaled); the Lq queries are the
+// tail rows L - Lq .. L - 1, query t at key position L - Lq + t sees keys
+// 0 .. that position.  One thread per (query or key, head), 64 per CTA.
+struct AttnRows {
+  const void* qkv;
+  int B, L, Lq, H, d;
+};
+
+__device__ inline long long qkv_off(const AttnRows& a, int b, int row, int part, int h, int dh) {
+  return ((long long)b * a.L + row) * 3 * a.d + (long long)part * a.d + (long long)h * dh;
+}
+
+// a = softmax(q k^T / sqrt(d_h)) v over the visible keys, and the row's
+// log-sum-exp (natural units) for the backward.
+template <typename T, int DH>
+__global__ void __launch_bounds__(64) attn_rows_forward_kernel(AttnRows a, T* __restrict__ out, float* __restrict__ lse) {
+  const int t = blockIdx.x * 64 + threadIdx.x, h = blockIdx.y, b = blockIdx.z;
+  if (t >= a.Lq) return;
+  const T* qkv = (const T*)a.qkv;
+  const int p = a.L - a.Lq + t;
+  const float sc = rsqrtf((float)DH) * 1.4426950408889634f;   // base-2 logits
+  float q[DH], o[DH];
+  const T* qr = qkv + qkv_off(a, b, p, 0, h, DH);
+#pragma unroll
+  for (int e = 0; e < DH; ++e) { q[e] = to_f(qr[e]) * sc; o[e] = 0.f; }
+  float m = -INFINITY, l = 0.f;
+  for (int j = 0; j <= p; ++j) {
+    const T* kr = qkv + qkv_off(a, b, j, 1, h, DH);
+    const T* vr = qkv + qkv_off(a, b, j, 2, h, DH);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) s = fmaf(q[e], to_f(kr[e]), s);
+    if (s > m) {
+      const float c = exp2f(m - s);
+      l *= c;
+#pragma unroll
+      for (int e = 0; e < DH; ++e) o[e] *= c;
+      m = s;
+    }
+    const float w = exp2f(s - m);
+    l += w;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) o[e] = fmaf(w, to_f(vr[e]), o[e]);
+  }
+  T* orow = out + ((long long)b * a.Lq + t) * a.d + (long long)h * DH;
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int e = 0; e < DH; ++e) orow[e] = from_f<T>(o[e] * inv);
+  lse[((long long)b * a.H + h) * a.Lq + t] = (m + log2f(l)) * 0.6931471805599453f;
+}
+
+// Per query row: D = dO . O, then dQ = sum_j P_j (dO . v_j - D) k_j / sqrt(d_h)
+// with P_j = exp(q . k_j / sqrt(d_h) - lse).  dq goes to dqkv's q columns.
+template <typename T, int DH>
+__global__ void __launch_bounds__(64) attn_rows_dq_kernel(AttnRows a, const float* __restrict__ dout,
+                                                          const T* __restrict__ out, const float* __restrict__ lse,
+                                                          float* __restrict__ Dr, float* __restrict__ dqkv) {
+  const int t = blockIdx.x * 64 + threadIdx.x, h = blockIdx.y, b = blockIdx.z;
+  if (t >= a.Lq) return;
+  const T* qkv = (const T*)a.qkv;
+  const int p = a.L - a.Lq + t;
+  const float isq = rsqrtf((float)DH);
+  const long long ro = ((long long)b * a.Lq + t) * a.d + (long long)h * DH;
+  float q[DH], g[DH], dq[DH];
+  float D = 0.f;
+  const T* qr = qkv + qkv_off(a, b, p, 0, h, DH);
+#pragma unroll
+  for (int e = 0; e < DH; ++e) {
+    q[e] = to_f(qr[e]) * isq;
+    g[e] = dout[ro + e];
+    D = fmaf(g[e], to_f(out[ro + e]), D);
+    dq[e] = 0.f;
+  }
+  const long long si = ((long long)b * a.H + h) * a.Lq + t;
+  const float ls = lse[si];
+  Dr[si] = D;
+  for (int j = 0; j <= p; ++j) {
+    const T* kr = qkv + qkv_off(a, b, j, 1, h, DH);
+    const T* vr = qkv + qkv_off(a, b, j, 2, h, DH);
+    float s = 0.f, dp = 0.f;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) {
+      s = fmaf(q[e], to_f(kr[e]), s);
+      dp = fmaf(g[e], to_f(vr[e]), dp);
+    }
+    const float ds = __expf(s - ls) * (dp - D) * isq;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) dq[e] = fmaf(ds, to_f(kr[e]), dq[e]);
+  }
+  float* dst = dqkv + ((long long)b * a.L + p) * 3 * a.d + (long long)h * DH;
+#pragma unroll
+  for (int e = 0; e < DH; ++e) dst[e] = dq[e];
+}
+
+// Per key row j: dV = sum_t P_tj dO_t, dK = sum_t P_tj (dO_t . v_j - D_t) q_t / sqrt(d_h)
+// over the queries t that see key j.  dk, dv go to dqkv's k and v columns.
+template <typename T, int DH>
+__global__ void __launch_bounds__(64) attn_rows_dkdv_kernel(AttnRows a, const float* __restrict__ dout,
+                                                            const float* __restrict__ lse, const float* __restrict__ Dr,
+                                                            float* __restrict__ dqkv) {
+  const int j = blockIdx.x * 64 + threadIdx.x, h = blockIdx.y, b = blockIdx.z;
+  if (j >= a.L) return;
+  const T* qkv = (const T*)a.qkv;
+  const float isq = rsqrtf((float)DH);
+  float k[DH], v[DH], dk[DH], dv[DH];
+  const T* kr = qkv + qkv_off(a, b, j, 1, h, DH);
+  const T* vr = qkv + qkv_off(a, b, j, 2, h, DH);
+#pragma unroll
+  for (int e = 0; e < DH; ++e) {
+    k[e] = to_f(kr[e]) * isq;
+    v[e] = to_f(vr[e]);
+    dk[e] = 0.f;
+    dv[e] = 0.f;
+  }
+  const int q0 = a.L - a.Lq;
+  for (int t = max(0, j - q0); t < a.Lq; ++t) {
+    const T* qr = qkv + qkv_off(a, b, q0 + t, 0, h, DH);
+    const float* gr = dout + ((long long)b * a.Lq + t) * a.d + (long long)h * DH;
+    float s = 0.f, dp = 0.f;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) {
+      s = fmaf(to_f(qr[e]), k[e], s);
+      dp = fmaf(gr[e], v[e], dp);
+    }
+    const long long si = ((long long)b * a.H + h) * a.Lq + t;
+    const float pr = __expf(s - lse[si]);
+    const float ds = pr * (dp - Dr[si]) * isq;
+#pragma unroll
+    for (int e = 0; e < DH; ++e) {
+      dv[e] = fmaf(pr, gr[e], dv[e]);
+      dk[e] = fmaf(ds, to_f(qr[e]), dk[e]);
+    }
+  }
+  float* dst = dqkv + ((long long)b * a.L + j) * 3 * a.d + (long long)h * DH;
+#pragma unroll
+  for (int e = 0; e < DH; ++e) {
+    dst[a.d + e] = dk[e];
+    dst[2 * a.d + e] = dv[e];
+  }
+}
+
+}  // namespace ot

@@ -17,6 +17,7 @@
 #include "gemm_bres.cuh"
 #include "attn_tc.cuh"
 #include "ffn_tc.cuh"
+#include "backward.cuh"
 
 using namespace ot;
 
@@ -50,11 +51,12 @@ static int g_policy = 0;
 // tagged with a kernel kind and its algorithmic FLOPs and bytes.
 enum ProfKind {
   PK_GEMM_QKV = 0, PK_GEMM_OPROJ, PK_GEMM_FFN_UP, PK_GEMM_FFN_DOWN, PK_GEMM_AUTOSPLIT, PK_ATTN_CAUSAL,
-  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_BLOCK_TAIL, PK_HEAD, PK_COUNT
+  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_BLOCK_TAIL, PK_HEAD, PK_TRAIN, PK_COUNT
 };
 static const char* kProfNames[PK_COUNT] = {"gemm_qkv", "gemm_oproj_rms", "gemm_ffn_up_gelu", "gemm_ffn_down_rms",
                                            "gemm_autosplit", "attn_causal", "attn_stage2", "rmsnorm",
-                                           "tokenize_events", "fused_oproj_ffn", "score_head"};
+                                           "tokenize_events", "fused_oproj_ffn", "score_head",
+                                           "train_gemm"};
 struct ProfRec {
   int kind;
   cudaEvent_t e0, e1;
@@ -974,6 +976,336 @@ static onetrans_status groupwise_impl(const onetrans_model* m, const void* feats
   return launch_gemm<T>(m, g2, st, PK_GEMM_AUTOSPLIT);
 }
 
+// ============================================================== training ==
+// The backward pass of the stack with activation recomputation: the forward
+// keeps only each layer's input; the backward recomputes a layer's
+// intermediates from its input, then runs the chain rule in reverse order of
+// the block.  Contractions run on the forward path's GEMM kernels: a GEMM
+// over rows (dX = dY W) takes the transposed weights, a GEMM that reduces
+// over rows (dW = dY^T X) takes both operands transposed (K-major), zero-
+// padded to a multiple of 64 rows.
+static long long pad64(long long r) { return (r + 63) / 64 * 64; }
+
+template <typename Ti, typename To>
+static onetrans_status launch_transpose(const void* src, const RowSet& s, int G, int C, void* dst, int R_pad,
+                                        cudaStream_t st) {
+  if (G <= 0 || C <= 0 || R_pad <= 0) return ONETRANS_OK;
+  dim3 grid((unsigned)cdiv(C, 32), (unsigned)cdiv(R_pad, 32), (unsigned)G);
+  transpose_rows_kernel<Ti, To><<<grid, 256, 0, st>>>((const Ti*)src, s, C, (To*)dst, R_pad);
+  return last_launch();
+}
+
+static onetrans_status launch_colsum(const float* src, const RowSet& s, int G, int C, float* dst, long long dst_gs,
+                                     cudaStream_t st) {
+  if (G <= 0 || C <= 0) return ONETRANS_OK;
+  colsum_kernel<<<dim3((unsigned)cdiv(C, 32), (unsigned)G), 256, 0, st>>>(src, s, C, dst, dst_gs);
+  return last_launch();
+}
+
+static RowSet rowset(long long gs, long long sb, long long st, int T, int R) {
+  RowSet r;
+  r.gs = gs; r.sb = sb; r.st = st; r.T = T; r.R = R;
+  return r;
+}
+
+template <typename T>
+static onetrans_status launch_cast(const float* src, void* dst, long long n, cudaStream_t st) {
+  if (n <= 0) return ONETRANS_OK;
+  cast_kernel<T><<<(unsigned)cdiv(n, 256), 256, 0, st>>>(src, (T*)dst, n);
+  return last_launch();
+}
+
+// Rows (b, t), t in [t_lo, t_hi) of a buffer with a_rows rows per sample: rows
+// t < t_s use the shared S weights W_S [N, K], rows t >= t_s the set of NS
+// token t - t_s of W_NS [L_NS, N, K].  A element (b, t, k) = A + b*a_samp +
+// t*a_row + k; output rows through `out`; optional bias sets and residual.
+template <typename T>
+static onetrans_status mixed_rows_gemm(const onetrans_model* m, const void* A, long long a_row, long long a_samp,
+                                       int a_rows, int B, int t_lo, int t_s, int t_hi, const void* W_S,
+                                       const void* W_NS, int K, int N, RowMap out, cudaStream_t st,
+                                       const void* bias_S = nullptr, const void* bias_NS = nullptr,
+                                       RowMap res = RowMap{}) {
+  if (t_s > t_lo) {
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_ROWS; g.M = t_s - t_lo; g.m_lo = t_lo; g.G = B; g.g_lo = 0;
+    g.K = K; g.A = A; g.a_sm = a_row; g.a_sg = a_samp; g.a_mext = a_rows; g.a_gext = B;
+    g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S;
+    g.out = out; g.res = res;
+    OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
+  }
+  if (t_hi > t_s) {
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_SAMPLES; g.M = B; g.G = t_hi - t_s; g.g_lo = t_s; g.grp_base = t_s;
+    g.K = K; g.A = A; g.a_sm = a_samp; g.a_sg = a_row; g.a_mext = B; g.a_gext = a_rows;
+    g.W = W_NS; g.w_sg = (long long)N * K; g.w_rows = N; g.w_groups = t_hi - t_s; g.N = N;
+    g.bias = bias_NS; g.bias_sg = bias_NS ? N : 0;
+    g.out = out; g.res = res;
+    OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
+  }
+  return ONETRANS_OK;
+}
+
+// Weight gradient dW [N_out, K_in] = sum over a row set of dY^T X, the S set
+// over all its rows and each NS set over its token's rows (one per sample).
+// dY rows: src_y (float32) with y_cols columns starting at y_col0; X rows:
+// src_x (storage type or float32) with x_cols columns.
+struct GradRows {
+  const void* p;     // element (b, t, c) = p + b*samp + t*row + c
+  long long row, samp;
+  bool f32;
+};
+
+template <typename T>
+static onetrans_status weight_grad(const onetrans_model* m, GradRows Y, GradRows X, int N_out, int K_in, int B,
+                                   int t_lo, int t_s, int t_hi, float* dW_S, float* dW_NS, void* opA, void* opW,
+                                   cudaStream_t st) {
+  const int es = m->es;
+  auto transpose = [&](const GradRows& s, const RowSet& rs, int G, int C, void* dst, int R_pad) {
+    if (s.f32) return launch_transpose<float, T>(s.p, rs, G, C, dst, R_pad, st);
+    return launch_transpose<T, T>(s.p, rs, G, C, dst, R_pad, st);
+  };
+  if (t_s > t_lo && dW_S) {
+    const int Tn = t_s - t_lo, R = B * Tn;
+    const int Rp = (int)pad64(R);
+    const RowSet ry = rowset(0, Y.samp, Y.row, Tn, R), rx = rowset(0, X.samp, X.row, Tn, R);
+    GradRows y0 = Y, x0 = X;
+    y0.p = (const char*)Y.p + t_lo * Y.row * (Y.f32 ? 4 : es);
+    x0.p = (const char*)X.p + t_lo * X.row * (X.f32 ? 4 : es);
+    OT_TRY(transpose(y0, ry, 1, N_out, opA, Rp));
+    OT_TRY(transpose(x0, rx, 1, K_in, opW, Rp));
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_FLAT; g.M = N_out; g.G = 1;
+    g.K = Rp; g.A = opA; g.a_sm = Rp; g.a_mext = N_out; g.a_gext = 1;
+    g.W = opW; g.w_rows = K_in; g.N = K_in;
+    g.out = rmap32(dW_S, 0, K_in);
+    OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
+  }
+  if (t_hi > t_s && dW_NS) {
+    const int G = t_hi - t_s, Bp = (int)pad64(B);
+    const RowSet ry = rowset(Y.row, Y.samp, 0, 1, B), rx = rowset(X.row, X.samp, 0, 1, B);
+    GradRows y0 = Y, x0 = X;
+    y0.p = (const char*)Y.p + t_s * Y.row * (Y.f32 ? 4 : es);
+    x0.p = (const char*)X.p + t_s * X.row * (X.f32 ? 4 : es);
+    OT_TRY(transpose(y0, ry, G, N_out, opA, Bp));
+    OT_TRY(transpose(x0, rx, G, K_in, opW, Bp));
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_SAMPLES; g.M = N_out; g.G = G; g.g_lo = 0; g.grp_base = 0;
+    g.K = Bp; g.A = opA; g.a_sm = Bp; g.a_sg = (long long)N_out * Bp; g.a_mext = N_out; g.a_gext = G;
+    g.W = opW; g.w_sg = (long long)K_in * Bp; g.w_rows = K_in; g.w_groups = G; g.N = K_in;
+    g.out = rmap32(dW_NS, K_in, (long long)N_out * K_in);
+    OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
+  }
+  return ONETRANS_OK;
+}
+
+// Bias gradient: column sums of float32 rows, the S set over all its rows and
+// each NS set over its token's rows.
+static onetrans_status bias_grad(const float* rows, long long row, long long samp, int C, int B, int t_lo, int t_s,
+                                 int t_hi, float* db_S, float* db_NS, cudaStream_t st) {
+  if (t_s > t_lo && db_S)
+    OT_TRY(launch_colsum(rows + t_lo * row, rowset(0, samp, row, t_s - t_lo, B * (t_s - t_lo)), 1, C, db_S, 0, st));
+  if (t_hi > t_s && db_NS)
+    OT_TRY(launch_colsum(rows + t_s * row, rowset(row, samp, 0, 1, B), t_hi - t_s, C, db_NS, C, st));
+  return ONETRANS_OK;
+}
+
+template <typename T, typename Tx>
+static onetrans_status launch_rms_backward(const void* x, long long x_sb, long long x_st, const void* gamma,
+                                           const float* dy, float* dx, long long dx_sb, long long dx_st, float* pg,
+                                           int rows, int fold, int d, float eps, cudaStream_t st) {
+  if (rows <= 0) return ONETRANS_OK;
+  rms_backward_kernel<Tx, T><<<(unsigned)cdiv(rows, 8), 256, 0, st>>>((const Tx*)x, x_sb, x_st, (const T*)gamma, dy,
+                                                                      dx, dx_sb, dx_st, pg, rows, fold, d, eps);
+  return last_launch();
+}
+
+template <typename T>
+static onetrans_status launch_attn_rows(const onetrans_model* m, int stage, const AttnRows& a, void* out,
+                                        float* lse, const float* dout, float* Dr, float* dqkv, cudaStream_t st) {
+  const int dh = m->dh;
+#define OT_ATTN_ROWS(DH)                                                                                   \
+  if (stage == 0) {                                                                                         \
+    attn_rows_forward_kernel<T, DH><<<dim3((unsigned)cdiv(a.Lq, 64), a.H, a.B), 64, 0, st>>>(a, (T*)out, lse); \
+  } else if (stage == 1) {                                                                                  \
+    attn_rows_dq_kernel<T, DH><<<dim3((unsigned)cdiv(a.Lq, 64), a.H, a.B), 64, 0, st>>>(a, dout, (const T*)out, \
+                                                                                         lse, Dr, dqkv);    \
+  } else {                                                                                                  \
+    attn_rows_dkdv_kernel<T, DH><<<dim3((unsigned)cdiv(a.L, 64), a.H, a.B), 64, 0, st>>>(a, dout, lse, Dr, dqkv); \
+  }
+  switch (dh) {
+    case 16: OT_ATTN_ROWS(16) break;
+    case 32: OT_ATTN_ROWS(32) break;
+    case 64: OT_ATTN_ROWS(64) break;
+    case 96: OT_ATTN_ROWS(96) break;
+    case 128: OT_ATTN_ROWS(128) break;
+    default: return ONETRANS_ERR_UNSUPPORTED;
+  }
+#undef OT_ATTN_ROWS
+  return last_launch();
+}
+
+template <typename T>
+static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B, int L_S, const float* dy,
+                                  float* out, float* dx0, const onetrans_grads* gr, void* ws, size_t ws_bytes,
+                                  cudaStream_t st, size_t* need) {
+  std::vector<int> Lq;
+  OT_TRY(schedule_of(m, L_S, Lq));
+  const int d = m->d, dff = m->dff, L_NS = m->L_NS, NL = m->NL, es = m->es, H = m->H;
+  const int L0 = L_S + L_NS;
+  std::vector<int> Ln(NL);  // input rows of each layer
+  Ln[0] = L0;
+  for (int n = 1; n < NL; ++n) Ln[n] = Lq[n - 1];
+  const int Lq0 = Lq[0];
+  const long long Mmax = pad64((long long)B * L0);
+  const long long op_elems = std::max<long long>(Mmax, (long long)L_NS * pad64(B)) * std::max(3 * d, dff);
+  const long long wt_elems = (long long)(1 + L_NS) * std::max(3 * d, dff) * d;
+  Carve cv(ws, ws_bytes);
+  std::vector<float*> X(NL, nullptr);   // float32 inputs of layers 1 .. NL-1
+  for (int n = 1; n < NL; ++n) X[n] = (float*)cv.take((size_t)B * Ln[n] * d * 4);
+  void* h = cv.take((size_t)B * L0 * d * es);
+  void* qkv = cv.take((size_t)B * L0 * 3 * d * es);
+  void* a = cv.take((size_t)B * Lq0 * d * es);
+  float* lse = (float*)cv.take((size_t)B * H * Lq0 * 4);
+  float* Dr = (float*)cv.take((size_t)B * H * Lq0 * 4);
+  float* x1 = (float*)cv.take((size_t)B * Lq0 * d * 4);
+  void* h2 = cv.take((size_t)B * Lq0 * d * es);
+  float* u = (float*)cv.take((size_t)B * Lq0 * dff * 4);
+  void* z = cv.take((size_t)B * Lq0 * dff * es);
+  float* gbuf[2] = {(float*)cv.take((size_t)B * L0 * d * 4), (float*)cv.take((size_t)B * L0 * d * 4)};
+  float* dx1 = (float*)cv.take((size_t)B * Lq0 * d * 4);
+  void* rowT = cv.take((size_t)B * L0 * 3 * d * es);   // a float32 gradient cast to the storage type
+  float* dz = (float*)cv.take((size_t)B * Lq0 * dff * 4);
+  float* du32 = (float*)cv.take((size_t)B * Lq0 * dff * 4);
+  void* du = cv.take((size_t)B * Lq0 * dff * es);
+  float* dh2 = (float*)cv.take((size_t)B * Lq0 * d * 4);
+  float* da = (float*)cv.take((size_t)B * Lq0 * d * 4);
+  float* dqkv = (float*)cv.take((size_t)B * L0 * 3 * d * 4);
+  float* dh = (float*)cv.take((size_t)B * L0 * d * 4);
+  float* pg = (float*)cv.take((size_t)B * L0 * d * 4);
+  void* opA = cv.take((size_t)op_elems * es);
+  void* opW = cv.take((size_t)op_elems * es);
+  void* wT = cv.take((size_t)wt_elems * es);
+  if (need) { *need = cv.used; return ONETRANS_OK; }
+  if (cv.overflow) return ONETRANS_ERR_CAPACITY;
+
+  // transposed weights of one layer's S set and NS sets: [N_out, K_in] -> [K_in, N_out]
+  auto weights_T = [&](const void* W_S, const void* W_NS, int N_out, int K_in, void*& S_T, void*& NS_T) {
+    S_T = wT;
+    NS_T = (char*)wT + (size_t)N_out * K_in * es;
+    OT_TRY((launch_transpose<T, T>(W_S, rowset(0, 0, K_in, N_out, N_out), 1, K_in, S_T, N_out, st)));
+    if (W_NS)
+      OT_TRY((launch_transpose<T, T>(W_NS, rowset((long long)N_out * K_in, 0, K_in, N_out, N_out), L_NS, K_in, NS_T,
+                                    N_out, st)));
+    return ONETRANS_OK;
+  };
+
+  // recompute layer n's intermediates from its input x_in (L rows per sample)
+  auto recompute = [&](int n, const void* x_in, bool x_f32) -> onetrans_status {
+    const int L = Ln[n], Lqn = Lq[n], s = L - L_NS, sq = Lqn - L_NS, off = L - Lqn;
+    if (x_f32) OT_TRY(rms_flat<T>(m, x_in, true, h, (long long)B * L, m->g_attn[n], st));
+    else OT_TRY(rms_flat<T>(m, x_in, false, h, (long long)B * L, m->g_attn[n], st));
+    // q | k | v of every row (q unscaled)
+    OT_TRY(mixed_rows_gemm<T>(m, h, d, (long long)L * d, L, B, 0, s, L, m->Wqkv_S[n], m->Wqkv_NS[n], d, 3 * d,
+                              rmap(qkv, (long long)L * 3 * d, 3 * d), st));
+    AttnRows ar;
+    ar.qkv = qkv; ar.B = B; ar.L = L; ar.Lq = Lqn; ar.H = H; ar.d = d;
+    OT_TRY(launch_attn_rows<T>(m, 0, ar, a, lse, nullptr, nullptr, nullptr, st));
+    // x1 = x[tail] + W^O a, h2 = RMSNorm(x1)
+    GemmDesc go = gdesc_base(m);
+    go.mode = TILE_FLAT; go.M = B * Lqn; go.fold = Lqn; go.G = 1;
+    go.K = d; go.A = a; go.a_sm = d; go.a_mext = (long long)B * Lqn; go.a_gext = 1;
+    go.W = m->Wo[n]; go.w_rows = d; go.N = d;
+    go.res = x_f32 ? rmap32(eoff(x_in, (long long)off * d, 4), (long long)L * d, d)
+                   : rmap(eoff(x_in, (long long)off * d, es), (long long)L * d, d);
+    go.out = rmap32(x1, (long long)Lqn * d, d);
+    go.rms = rmap(h2, (long long)Lqn * d, d);
+    go.gamma = m->g_ffn[n];
+    OT_TRY(launch_gemm<T>(m, go, st, PK_TRAIN));
+    // u = W1 h2 + b1 (float32), z = GELU(u)
+    OT_TRY(mixed_rows_gemm<T>(m, h2, d, (long long)Lqn * d, Lqn, B, 0, sq, Lqn, m->W1_S[n], m->W1_NS[n], d, dff,
+                              rmap32(u, (long long)Lqn * dff, dff), st, m->b1_S[n], m->b1_NS[n]));
+    const long long nz = (long long)B * Lqn * dff;
+    gelu_forward_kernel<T><<<(unsigned)cdiv(nz, 256), 256, 0, st>>>(u, (T*)z, nz);
+    return last_launch();
+  };
+
+  // ---- forward, keeping each layer's input
+  for (int n = 0; n < NL; ++n) {
+    const int Lqn = Lq[n], sq = Lqn - L_NS;
+    OT_TRY(recompute(n, n == 0 ? x0 : (const void*)X[n], n > 0));
+    float* y = n + 1 == NL ? out : X[n + 1];
+    OT_TRY(mixed_rows_gemm<T>(m, z, dff, (long long)Lqn * dff, Lqn, B, 0, sq, Lqn, m->W2_S[n], m->W2_NS[n], dff, d,
+                              rmap32(y, (long long)Lqn * d, d), st, m->b2_S[n], m->b2_NS[n],
+                              rmap32(x1, (long long)Lqn * d, d)));
+  }
+
+  // ---- backward, layer by layer
+  const float* g_cur = dy;   // gradient of layer n's output, [B, Lq[n], d]
+  for (int n = NL - 1; n >= 0; --n) {
+    const int L = Ln[n], Lqn = Lq[n], s = L - L_NS, sq = Lqn - L_NS, off = L - Lqn;
+    const bool x_f32 = n > 0;
+    const void* x_in = n == 0 ? x0 : (const void*)X[n];
+    float* g_in = n == 0 ? dx0 : gbuf[n % 2];   // gradient of layer n's input, [B, L, d]
+    OT_TRY(recompute(n, x_in, x_f32));
+    const long long Md = (long long)Lqn * d, Mf = (long long)Lqn * dff;
+    // y = x1 + W2 z + b2
+    OT_TRY(bias_grad(g_cur, d, Md, d, B, 0, sq, Lqn, gr->b2_S[n], gr->b2_NS[n], st));
+    OT_TRY(weight_grad<T>(m, GradRows{g_cur, d, Md, true}, GradRows{z, dff, Mf, false}, d, dff, B, 0, sq, Lqn,
+                          gr->W2_S[n], gr->W2_NS[n], opA, opW, st));
+    void *wS, *wNS;
+    OT_TRY(launch_cast<T>(g_cur, rowT, (long long)B * Md, st));
+    OT_TRY(weights_T(m->W2_S[n], m->W2_NS[n], d, dff, wS, wNS));
+    OT_TRY(mixed_rows_gemm<T>(m, rowT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap32(dz, Mf, dff), st));
+    // z = GELU(u), u = W1 h2 + b1
+    const long long nz = (long long)B * Mf;
+    gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 256), 256, 0, st>>>(dz, u, du32, (T*)du, nz);
+    OT_TRY(last_launch());
+    OT_TRY(bias_grad(du32, dff, Mf, dff, B, 0, sq, Lqn, gr->b1_S[n], gr->b1_NS[n], st));
+    OT_TRY(weight_grad<T>(m, GradRows{du, dff, Mf, false}, GradRows{h2, d, Md, false}, dff, d, B, 0, sq, Lqn,
+                          gr->W1_S[n], gr->W1_NS[n], opA, opW, st));
+    OT_TRY(weights_T(m->W1_S[n], m->W1_NS[n], dff, d, wS, wNS));
+    OT_TRY(mixed_rows_gemm<T>(m, du, dff, Mf, Lqn, B, 0, sq, Lqn, wS, wNS, dff, d, rmap32(dh2, Md, d), st));
+    // h2 = RMSNorm(x1; g_ffn), x1 = x[tail] + W^O a
+    OT_TRY(cuda_ok(cudaMemcpyAsync(dx1, g_cur, (size_t)B * Md * 4, cudaMemcpyDeviceToDevice, st)));
+    OT_TRY((launch_rms_backward<T, float>(x1, Md, d, m->g_ffn[n], dh2, dx1, Md, d, pg, B * Lqn, Lqn, d,
+                                         m->cfg.rms_eps, st)));
+    OT_TRY(launch_colsum(pg, rowset(0, Md, d, Lqn, B * Lqn), 1, d, gr->g_ffn[n], 0, st));
+    OT_TRY(weight_grad<T>(m, GradRows{dx1, d, Md, true}, GradRows{a, d, Md, false}, d, d, B, 0, Lqn, Lqn,
+                          gr->Wo[n], nullptr, opA, opW, st));
+    OT_TRY(launch_cast<T>(dx1, rowT, (long long)B * Md, st));
+    OT_TRY(weights_T(m->Wo[n], nullptr, d, d, wS, wNS));
+    OT_TRY(mixed_rows_gemm<T>(m, rowT, d, Md, Lqn, B, 0, Lqn, Lqn, wS, nullptr, d, d, rmap32(da, Md, d), st));
+    // the residual: the tail rows of the input receive dx1, the others start at 0
+    OT_TRY(cuda_ok(cudaMemsetAsync(g_in, 0, (size_t)B * L * d * 4, st)));
+    OT_TRY(cuda_ok(cudaMemcpy2DAsync(g_in + (size_t)off * d, (size_t)L * d * 4, dx1, (size_t)Md * 4, (size_t)Md * 4,
+                                     B, cudaMemcpyDeviceToDevice, st)));
+    // attention: dq, dk, dv of the recomputed rows
+    OT_TRY(cuda_ok(cudaMemsetAsync(dqkv, 0, (size_t)B * L * 3 * d * 4, st)));
+    AttnRows ar;
+    ar.qkv = qkv; ar.B = B; ar.L = L; ar.Lq = Lqn; ar.H = H; ar.d = d;
+    OT_TRY(launch_attn_rows<T>(m, 1, ar, a, lse, da, Dr, dqkv, st));
+    OT_TRY(launch_attn_rows<T>(m, 2, ar, a, lse, da, Dr, dqkv, st));
+    // (q, k, v) = W_i^{QKV} h_i
+    const long long Mq = (long long)L * 3 * d;
+    OT_TRY(weight_grad<T>(m, GradRows{dqkv, 3 * d, Mq, true}, GradRows{h, d, (long long)L * d, false}, 3 * d, d,
+                          B, 0, s, L, gr->Wqkv_S[n], gr->Wqkv_NS[n], opA, opW, st));
+    OT_TRY(launch_cast<T>(dqkv, rowT, (long long)B * Mq, st));
+    OT_TRY(weights_T(m->Wqkv_S[n], m->Wqkv_NS[n], 3 * d, d, wS, wNS));
+    OT_TRY(mixed_rows_gemm<T>(m, rowT, 3 * d, Mq, L, B, 0, s, L, wS, wNS, 3 * d, d,
+                              rmap32(dh, (long long)L * d, d), st));
+    // h = RMSNorm(x; g_attn)
+    if (x_f32)
+      OT_TRY((launch_rms_backward<T, float>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
+                                           B * L, L, d, m->cfg.rms_eps, st)));
+    else
+      OT_TRY((launch_rms_backward<T, T>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
+                                       B * L, L, d, m->cfg.rms_eps, st)));
+    OT_TRY(launch_colsum(pg, rowset(0, (long long)L * d, d, L, B * L), 1, d, gr->g_attn[n], 0, st));
+    g_cur = g_in;
+  }
+  return ONETRANS_OK;
+}
+
 // Failure path of the bounded waits, without a fault: one thread waits on an
 // mbarrier that nothing arrives at, with the same wait the tensor-core
 // kernels use but limited to `limit` rounds; the wait gives up, records
@@ -1109,6 +1441,10 @@ onetrans_status onetrans_workspace_size(const onetrans_model* m, int32_t op, int
     case ONETRANS_OP_AUTOSPLIT:
       return m->bf16 ? autosplit_impl<__nv_bfloat16>(m, nullptr, n, nullptr, nullptr, 0, 0, bytes)
                      : autosplit_impl<float>(m, nullptr, n, nullptr, nullptr, 0, 0, bytes);
+    case ONETRANS_OP_TRAIN:
+      return m->bf16 ? train_impl<__nv_bfloat16>(m, nullptr, nn, L, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0,
+                                                 bytes)
+                     : train_impl<float>(m, nullptr, nn, L, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, bytes);
     case ONETRANS_OP_GROUPWISE:
       if (L < 1) return ONETRANS_ERR_SHAPE;
       return m->bf16 ? groupwise_impl<__nv_bfloat16>(m, nullptr, n, 1, L, nullptr, nullptr, nullptr, nullptr,
@@ -1424,6 +1760,31 @@ onetrans_status onetrans_forward(const onetrans_model* m, const void* x0, int32_
   cudaStream_t st = (cudaStream_t)stream;
   return m->bf16 ? forward_impl<__nv_bfloat16>(m, x0, B, L_S, out, ws, ws_bytes, st, nullptr)
                  : forward_impl<float>(m, x0, B, L_S, out, ws, ws_bytes, st, nullptr);
+}
+
+onetrans_status onetrans_forward_backward(const onetrans_model* m, const void* x0, int32_t B, int32_t L_S,
+                                          const float* dy, float* out, float* dx0, const onetrans_grads* grads,
+                                          void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !grads) return ONETRANS_ERR_INVALID_ARG;
+  if (B < 0 || L_S < 0) return ONETRANS_ERR_SHAPE;
+  if ((long long)B * (L_S + m->L_NS) * 3 * m->d > (1LL << 31) - 1) return ONETRANS_ERR_SHAPE;
+  float* const* per_layer[] = {grads->g_attn, grads->g_ffn, grads->Wqkv_S, grads->Wqkv_NS, grads->Wo,
+                               grads->W1_S, grads->b1_S, grads->W2_S, grads->b2_S, grads->W1_NS,
+                               grads->b1_NS, grads->W2_NS, grads->b2_NS};
+  for (auto arr : per_layer) {
+    if (!arr) return ONETRANS_ERR_INVALID_ARG;
+    for (int l = 0; l < m->NL; ++l)
+      if (!arr[l] || !aligned(arr[l], 16)) return ONETRANS_ERR_INVALID_ARG;
+  }
+  std::vector<int> Lq;
+  OT_TRY(schedule_of(m, L_S, Lq));
+  if (B == 0) return ONETRANS_OK;  // no work: the data pointers may be NULL
+  if (!x0 || !dy || !out || !dx0 || !aligned(x0, 16) || !aligned(dy, 16) || !aligned(out, 16) || !aligned(dx0, 16))
+    return ONETRANS_ERR_INVALID_ARG;
+  OT_TRY(check_ws(ws));
+  cudaStream_t st = (cudaStream_t)stream;
+  return m->bf16 ? train_impl<__nv_bfloat16>(m, x0, B, L_S, dy, out, dx0, grads, ws, ws_bytes, st, nullptr)
+                 : train_impl<float>(m, x0, B, L_S, dy, out, dx0, grads, ws, ws_bytes, st, nullptr);
 }
 
 onetrans_status onetrans_profile_enable(int32_t on) {
