@@ -16,6 +16,7 @@ from helpers import EPS, TOL, attn_std, build, rel_err, shape, tdt, to_dev, to_n
 
 import unified_transformer_recommender_b200 as ot  # noqa: E402
 
+GRAD_TOL = {"bf16": 2e-2, "fp32": 1e-4}
 KEYS = ("g_attn", "g_ffn", "Wqkv_S", "Wqkv_NS", "Wo", "W1_S", "b1_S", "W2_S", "b2_S", "W1_NS", "b1_NS",
         "W2_NS", "b2_NS")
 
@@ -59,10 +60,11 @@ def test_forward_backward_matches_oracle(dtype, policy, d, pyr):
     dY = gen_normal(252, (2, n_out, sh.d), "fp32")
     out, dx0, grads = run_train(b, X0, dY)
     Y, dX, dW = O.forward_backward(X0, b.W, sh.L_NS, sh.n_heads, EPS, sched, dY)
-    tol = TOL[dtype]
-    assert rel_err(out, Y) <= tol
-    assert rel_err(dx0, dX) <= tol
+    assert rel_err(out, Y) <= TOL[dtype]
+    errs = {"dx0": rel_err(dx0, dX)}
     for k in KEYS:
         for l in range(sh.n_layers):
             assert np.isfinite(grads[k][l]).all(), (k, l)
-            assert rel_err(grads[k][l], dW[k][l]) <= tol, (k, l, rel_err(grads[k][l], dW[k][l]))
+            errs[f"{k}[{l}]"] = rel_err(grads[k][l], dW[k][l])
+    bad = {k: e for k, e in errs.items() if not e <= GRAD_TOL[dtype]}
+    assert not bad, (bad, errs)

@@ -1064,6 +1064,8 @@ static onetrans_status weight_grad(const onetrans_model* m, GradRows Y, GradRows
     if (s.f32) return launch_transpose<float, T>(s.p, rs, G, C, dst, R_pad, st);
     return launch_transpose<T, T>(s.p, rs, G, C, dst, R_pad, st);
   };
+  // a set with no rows (the S set of a layer that keeps only NS rows) has a zero gradient
+  if (t_s == t_lo && dW_S) OT_TRY(cuda_ok(cudaMemsetAsync(dW_S, 0, (size_t)N_out * K_in * 4, st)));
   if (t_s > t_lo && dW_S) {
     const int Tn = t_s - t_lo, R = B * Tn;
     const int Rp = (int)pad64(R);
@@ -1102,6 +1104,7 @@ static onetrans_status weight_grad(const onetrans_model* m, GradRows Y, GradRows
 // each NS set over its token's rows.
 static onetrans_status bias_grad(const float* rows, long long row, long long samp, int C, int B, int t_lo, int t_s,
                                  int t_hi, float* db_S, float* db_NS, cudaStream_t st) {
+  if (t_s == t_lo && db_S) OT_TRY(cuda_ok(cudaMemsetAsync(db_S, 0, (size_t)C * 4, st)));
   if (t_s > t_lo && db_S)
     OT_TRY(launch_colsum(rows + t_lo * row, rowset(0, samp, row, t_s - t_lo, B * (t_s - t_lo)), 1, C, db_S, 0, st));
   if (t_hi > t_s && db_NS)
