@@ -1,9 +1,18 @@
 """The training step (forward keeping each layer's input, backward with each
 layer recomputed from it) through the C ABI against the oracle's backward:
-the output, the input gradient and every weight gradient, each within
-max-abs-error / RMS <= 2e-2 (bf16 operands, float32 accumulation and
-gradients) or 1e-4 (float32 mode).  Weights at std 1/sqrt(d), so attention
-is far from uniform and its backward matters."""
+the output, the input gradient and every weight gradient.  Weights at std
+1/sqrt(d), so attention is far from uniform and its backward matters.
+
+Bars.  Float32 mode: max-abs-error / RMS <= 1e-4 for every tensor, element
+by element.  BF16 mode (bf16 operands of every contraction, float32
+accumulation and gradients): the output within max-abs-error / RMS <= 2e-2
+like the forward; the gradients within ||got - ref|| / ||ref|| <= 2e-2.  A
+gradient that sums only a few rows (an NS set's weights sum one row per
+sample) keeps the rounding of its two bf16 operands element by element, up
+to 0.14 of the RMS on these inputs in a CPU emulation of exactly those
+rounding points, while the norm-wise error stays near 5e-3; a dropped term
+or a wrong row still moves it well past 2e-2.  A gradient whose reference
+is exactly zero (the S set of a layer that keeps only NS rows) must be zero."""
 import numpy as np
 import pytest
 
@@ -16,7 +25,14 @@ from helpers import EPS, TOL, attn_std, build, rel_err, shape, tdt, to_dev, to_n
 
 import unified_transformer_recommender_b200 as ot  # noqa: E402
 
-GRAD_TOL = {"bf16": 2e-2, "fp32": 1e-4}
+def grad_err(got, ref, dtype) -> float:
+    """fp32: max-abs-error / RMS; bf16: ||got - ref|| / ||ref||."""
+    if dtype == "fp32":
+        return rel_err(got, ref)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.linalg.norm(np.asarray(got, dtype=np.float64) - ref) / np.linalg.norm(ref))
+
+
 KEYS = ("g_attn", "g_ffn", "Wqkv_S", "Wqkv_NS", "Wo", "W1_S", "b1_S", "W2_S", "b2_S", "W1_NS", "b1_NS",
         "W2_NS", "b2_NS")
 
@@ -61,10 +77,13 @@ def test_forward_backward_matches_oracle(dtype, policy, d, pyr):
     out, dx0, grads = run_train(b, X0, dY)
     Y, dX, dW = O.forward_backward(X0, b.W, sh.L_NS, sh.n_heads, EPS, sched, dY)
     assert rel_err(out, Y) <= TOL[dtype]
-    errs = {"dx0": rel_err(dx0, dX)}
+    errs = {"dx0": grad_err(dx0, dX, dtype)}
     for k in KEYS:
         for l in range(sh.n_layers):
             assert np.isfinite(grads[k][l]).all(), (k, l)
-            errs[f"{k}[{l}]"] = rel_err(grads[k][l], dW[k][l])
-    bad = {k: e for k, e in errs.items() if not e <= GRAD_TOL[dtype]}
+            if not np.any(dW[k][l]):
+                assert not np.any(grads[k][l]), (k, l)
+                continue
+            errs[f"{k}[{l}]"] = grad_err(grads[k][l], dW[k][l], dtype)
+    bad = {k: e for k, e in errs.items() if not e <= TOL[dtype]}
     assert not bad, (bad, errs)
