@@ -74,7 +74,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="kv_serving",
-                    choices=("kv_serving", "append", "s_forward", "l_forward"))
+                    choices=("kv_serving", "append", "s_forward", "l_forward", "train"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--users", type=int, default=0, help="override users per GPU (small profiling captures)")
     ap.add_argument("--cands", type=int, default=0, help="override candidates per user (small captures)")
@@ -221,10 +221,29 @@ def forward_config(name: str, U: int, ws: int) -> dict:
             "l2": "512 MB buffer written between timed steps (not timed)"}
 
 
+ALU_KERNELS = ("train_attn_rows",)   # kernel kinds that run on the CUDA cores' FMA pipes
+TRAIN_METRIC = "samples/sec of the training step (forward + backward with recomputation) on 1 B200"
+TRAIN_SAMPLES = 8
+
+
+def train_config(U: int, ws: int) -> dict:
+    from onetrans_synth import WORKLOADS
+    wl = WORKLOADS["s_forward"]
+    sh = wl.shape
+    return {"workload": f"train: the s_forward model ({sh.n_layers} layers d={sh.d} {sh.n_heads} heads FFN "
+                        f"{sh.d_ff}, pyramid {wl.pyramid[0]}->{wl.pyramid[-1]}), {U} samples x ({wl.L_S} S + "
+                        f"{sh.L_NS} NS tokens): forward keeping each layer's input, backward with every layer "
+                        "recomputed; bf16 operands, float32 gradients of the input and of every weight",
+            "samples_per_gpu": U, "parallelism": f"samples sharded over {ws} GPU(s), no collective",
+            "l2": "512 MB buffer written between timed steps (not timed)"}
+
+
 def workload_meta(name: str, ws: int):
     """(metric, unit, config, units per GPU per step) of a workload at its
     default size, without building it."""
     from onetrans_synth import WORKLOADS
+    if name == "train":
+        return TRAIN_METRIC, "samples/s", train_config(TRAIN_SAMPLES, ws), TRAIN_SAMPLES
     wl = WORKLOADS[name]
     if name == "kv_serving":
         return METRIC, UNIT, kv_serving_config(wl.users, wl.cands, ws), wl.users * wl.cands
@@ -498,6 +517,57 @@ class Forward:
         return oracle_sample_forward(self.name, self.U)
 
 
+class Train:
+    """Training step of the s_forward model (onetrans_forward_backward) on
+    TRAIN_SAMPLES samples: an upstream gradient dY of the output in, the
+    output, dX0 and every weight gradient out."""
+
+    unit = "samples/s"
+    io_names = ("X", "dY")
+
+    def __init__(self, rank: int, users: int = 0):
+        import torch
+        import unified_transformer_recommender_b200 as ot
+        from onetrans_synth import WORKLOADS, gen_normal, make_weights
+        self.ot, self.torch = ot, torch
+        wl = WORKLOADS["s_forward"]
+        self.wl, sh = wl, wl.shape
+        self.U = users or TRAIN_SAMPLES
+        self.metric = TRAIN_METRIC
+        self.W = make_weights(sh, wl.seed_weights, wl.dtype)
+        self.model = ot.model_from_arrays(sh, self.W, pyramid_q=list(wl.pyramid), mode=ot.BF16)
+        dev = torch.device("cuda")
+        self.X_h = gen_normal(wl.seed_inputs + 7919 * rank, (self.U, wl.L0, sh.d), "bf16")
+        self.dY_h = gen_normal(wl.seed_inputs + 17 + 7919 * rank, (self.U, sh.L_NS, sh.d), "fp32")
+        self.X = torch.from_numpy(self.X_h).to(dev, torch.bfloat16)
+        self.dY = torch.from_numpy(self.dY_h).to(dev)
+        self.X_pin = torch.from_numpy(self.X_h).to(torch.bfloat16).pin_memory()
+        self.dY_pin = torch.from_numpy(self.dY_h).pin_memory()
+        self.out = torch.empty(self.U, sh.L_NS, sh.d, dtype=torch.float32, device=dev)
+        self.out_pin = torch.empty(self.out.shape, dtype=torch.float32).pin_memory()
+        self.dX = torch.empty(self.U, wl.L0, sh.d, dtype=torch.float32, device=dev)
+        keys = ("g_attn", "g_ffn", "Wqkv_S", "Wqkv_NS", "Wo", "W1_S", "b1_S", "W2_S", "b2_S", "W1_NS", "b1_NS",
+                "W2_NS", "b2_NS")
+        self.grads = {k: [torch.empty(tuple(self.W[k][l].shape), dtype=torch.float32, device=dev)
+                          for l in range(sh.n_layers)] for k in keys}
+        self.ws = self.model.workspace(ot.OP_TRAIN, self.U, wl.L_S)
+        self.units = self.U
+        self.h2d = self.X_h.size * 2 + self.dY_h.size * 4
+        self.d2h = self.out.numel() * 4
+
+    def config(self, ws):
+        return train_config(self.U, ws)
+
+    def prepare(self, n_steps: int):
+        pass
+
+    def step(self, ev_mid=None):
+        self.ot.onetrans_forward_backward(self.model, self.X, self.dY, self.out, self.dX, self.grads, self.ws)
+
+    def oracle(self):
+        return oracle_sample_train(self.U)
+
+
 class E2EPipeline:
     """End-to-end leg: every step uploads its inputs from pinned host memory
     and downloads its result to pinned host memory, through the public API.
@@ -601,6 +671,8 @@ def make_workload(name: str, rank: int, users: int = 0, cands: int = 0):
         return KVServing(rank, users=users, cands=cands)
     if name == "append":
         return Append(rank, users=users, cands=cands)
+    if name == "train":
+        return Train(rank, users=users)
     return Forward(name, rank, users=users)
 
 
@@ -689,6 +761,25 @@ def oracle_sample_forward(name: str, samples: int):
     return 1.0 / (t1 - t0), desc, _oracle_threads(), t1 - t0
 
 
+def oracle_sample_train(samples: int):
+    """fp64 oracle training step (forward keeping each layer's input, backward
+    with recomputation) of 1 sample of the train workload; returns (samples/s,
+    description, threads, s)."""
+    from onetrans_synth import WORKLOADS, gen_normal, make_weights
+    from oracle import onetrans as O
+    wl = WORKLOADS["s_forward"]
+    sh = wl.shape
+    W = make_weights(sh, wl.seed_weights, "bf16")
+    X = gen_normal(wl.seed_inputs, (1, wl.L0, sh.d), "bf16")
+    dY = gen_normal(wl.seed_inputs + 17, (1, sh.L_NS, sh.d), "fp32")
+    t0 = time.perf_counter()
+    O.forward_backward(X, W, sh.L_NS, sh.n_heads, sh.eps, list(wl.pyramid), dY)
+    t1 = time.perf_counter()
+    desc = (f"oracle fp64: training step of 1 sample ({t1 - t0:.2f} s); the batch of {samples} scales "
+            "linearly")
+    return 1.0 / (t1 - t0), desc, _oracle_threads(), t1 - t0
+
+
 def run_reference(args, rank):
     """The oracle timed on the host cores, each step a bounded sample of the
     workload extrapolated to its full size; same metric, unit and config as
@@ -697,13 +788,16 @@ def run_reference(args, rank):
         return
     from onetrans_synth import WORKLOADS
     metric, unit, config, units = workload_meta(args.workload, args.gpus)
-    wl = WORKLOADS[args.workload]
+    wl = WORKLOADS.get(args.workload)
     if args.workload == "kv_serving":
         def sample(i):
             return oracle_sample(n_cands=8, seed_shift=i)
     elif args.workload == "append":
         def sample(i):
             return oracle_sample_append(wl.users, wl.cands, n_cands=4)
+    elif args.workload == "train":
+        def sample(i):
+            return oracle_sample_train(TRAIN_SAMPLES)
     else:
         def sample(i):
             return oracle_sample_forward(args.workload, wl.users)
@@ -838,7 +932,19 @@ def main():
     # the per-kernel times are single launches of well under a millisecond,
     # timed one by one: the burst figure of the measured GEMM peak applies
     tensor_bound = dom["flops"] / max(dom["bytes"], 1.0) > pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
-    if tensor_bound:
+    if dom_name in ALU_KERNELS:
+        # CUDA-core float32 arithmetic: SMs x 128 FMA lanes x 2 FLOP x the SM
+        # clock measured under load (median of the samples)
+        sm_count = torch.cuda.get_device_properties(0).multi_processor_count
+        mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
+        peak = sm_count * 128 * 2 * mhz * 1e6 / 1e12
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        roof = {"bound": "alu", "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "peak_source": f"{sm_count} SMs x 128 fp32 FMA lanes x 2 FLOP x {mhz:.0f} MHz (measured clock)",
+                "traffic": traffic, "flops_per_launch": dom["flops"] / dom["launches"],
+                "ms_per_launch": per_launch_ms}
+    elif tensor_bound:
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
         roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": pk["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],

@@ -16,7 +16,7 @@ from onetrans_synth import WORKLOADS
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.mark.parametrize("workload", ["kv_serving", "append", "s_forward", "l_forward"])
+@pytest.mark.parametrize("workload", ["kv_serving", "append", "s_forward", "l_forward", "train"])
 def test_reference_line_names_the_workload_of_the_cuda_arm(workload):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                         "--steps", "1", "--warmup", "0", "--workload", workload],

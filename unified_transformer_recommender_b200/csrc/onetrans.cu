@@ -51,12 +51,13 @@ static int g_policy = 0;
 // tagged with a kernel kind and its algorithmic FLOPs and bytes.
 enum ProfKind {
   PK_GEMM_QKV = 0, PK_GEMM_OPROJ, PK_GEMM_FFN_UP, PK_GEMM_FFN_DOWN, PK_GEMM_AUTOSPLIT, PK_ATTN_CAUSAL,
-  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_BLOCK_TAIL, PK_HEAD, PK_TRAIN, PK_COUNT
+  PK_ATTN_STAGE2, PK_RMSNORM, PK_TOKENIZE, PK_BLOCK_TAIL, PK_HEAD, PK_TRAIN, PK_TRAIN_ATTN, PK_TRAIN_ELEM,
+  PK_COUNT
 };
 static const char* kProfNames[PK_COUNT] = {"gemm_qkv", "gemm_oproj_rms", "gemm_ffn_up_gelu", "gemm_ffn_down_rms",
                                            "gemm_autosplit", "attn_causal", "attn_stage2", "rmsnorm",
                                            "tokenize_events", "fused_oproj_ffn", "score_head",
-                                           "train_gemm"};
+                                           "train_gemm", "train_attn_rows", "train_elementwise"};
 struct ProfRec {
   int kind;
   cudaEvent_t e0, e1;
@@ -990,6 +991,7 @@ template <typename Ti, typename To>
 static onetrans_status launch_transpose(const void* src, const RowSet& s, int G, int C, void* dst, int R_pad,
                                         cudaStream_t st) {
   if (G <= 0 || C <= 0 || R_pad <= 0) return ONETRANS_OK;
+  ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * ((double)s.R * sizeof(Ti) + (double)R_pad * sizeof(To)), st);
   dim3 grid((unsigned)cdiv(C, 32), (unsigned)cdiv(R_pad, 32), (unsigned)G);
   transpose_rows_kernel<Ti, To><<<grid, 256, 0, st>>>((const Ti*)src, s, C, (To*)dst, R_pad);
   return last_launch();
@@ -998,6 +1000,7 @@ static onetrans_status launch_transpose(const void* src, const RowSet& s, int G,
 static onetrans_status launch_colsum(const float* src, const RowSet& s, int G, int C, float* dst, long long dst_gs,
                                      cudaStream_t st) {
   if (G <= 0 || C <= 0) return ONETRANS_OK;
+  ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * (s.R + 1) * 4.0, st);
   colsum_kernel<<<dim3((unsigned)cdiv(C, 32), (unsigned)G), 256, 0, st>>>(src, s, C, dst, dst_gs);
   return last_launch();
 }
@@ -1011,6 +1014,7 @@ static RowSet rowset(long long gs, long long sb, long long st, int T, int R) {
 template <typename T>
 static onetrans_status launch_cast(const float* src, void* dst, long long n, cudaStream_t st) {
   if (n <= 0) return ONETRANS_OK;
+  ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)n * (4.0 + sizeof(T)), st);
   cast_kernel<T><<<(unsigned)cdiv(n, 256), 256, 0, st>>>(src, (T*)dst, n);
   return last_launch();
 }
@@ -1117,6 +1121,7 @@ static onetrans_status launch_rms_backward(const void* x, long long x_sb, long l
                                            const float* dy, float* dx, long long dx_sb, long long dx_st, float* pg,
                                            int rows, int fold, int d, float eps, cudaStream_t st) {
   if (rows <= 0) return ONETRANS_OK;
+  ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)rows * d * (sizeof(Tx) + 4.0 + 8.0 + 4.0), st);
   rms_backward_kernel<Tx, T><<<(unsigned)cdiv(rows, 8), 256, 0, st>>>((const Tx*)x, x_sb, x_st, (const T*)gamma, dy,
                                                                       dx, dx_sb, dx_st, pg, rows, fold, d, eps);
   return last_launch();
@@ -1126,6 +1131,11 @@ template <typename T>
 static onetrans_status launch_attn_rows(const onetrans_model* m, int stage, const AttnRows& a, void* out,
                                         float* lse, const float* dout, float* Dr, float* dqkv, cudaStream_t st) {
   const int dh = m->dh;
+  // visible (query, key) pairs x heads; FLOPs per pair: forward 2 x 2 d_h (q.k, p v), dq 3 x 2 d_h,
+  // dk,dv 4 x 2 d_h; bytes: the q|k|v rows read once, the outputs written once
+  const double pairs = (double)a.B * a.H * ((double)a.Lq * (a.L - a.Lq) + 0.5 * (double)a.Lq * (a.Lq + 1));
+  const double fl = pairs * 2.0 * dh * (stage == 0 ? 2 : stage == 1 ? 3 : 4);
+  ProfScope prof(PK_TRAIN_ATTN, fl, (double)a.B * a.L * 3 * a.d * m->es + (double)a.B * a.Lq * a.d * 4, st);
 #define OT_ATTN_ROWS(DH)                                                                                   \
   if (stage == 0) {                                                                                         \
     attn_rows_forward_kernel<T, DH><<<dim3((unsigned)cdiv(a.Lq, 64), a.H, a.B), 64, 0, st>>>(a, (T*)out, lse); \
@@ -1228,6 +1238,7 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     OT_TRY(mixed_rows_gemm<T>(m, h2, d, (long long)Lqn * d, Lqn, B, 0, sq, Lqn, m->W1_S[n], m->W1_NS[n], d, dff,
                               rmap32(u, (long long)Lqn * dff, dff), st, m->b1_S[n], m->b1_NS[n]));
     const long long nz = (long long)B * Lqn * dff;
+    ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + es), st);
     gelu_forward_kernel<T><<<(unsigned)cdiv(nz, 256), 256, 0, st>>>(u, (T*)z, nz);
     return last_launch();
   };
@@ -1261,7 +1272,10 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     OT_TRY(mixed_rows_gemm<T>(m, rowT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap32(dz, Mf, dff), st));
     // z = GELU(u), u = W1 h2 + b1
     const long long nz = (long long)B * Mf;
-    gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 256), 256, 0, st>>>(dz, u, du32, (T*)du, nz);
+    {
+      ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (12.0 + es), st);
+      gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 256), 256, 0, st>>>(dz, u, du32, (T*)du, nz);
+    }
     OT_TRY(last_launch());
     OT_TRY(bias_grad(du32, dff, Mf, dff, B, 0, sq, Lqn, gr->b1_S[n], gr->b1_NS[n], st));
     OT_TRY(weight_grad<T>(m, GradRows{du, dff, Mf, false}, GradRows{h2, d, Md, false}, dff, d, B, 0, sq, Lqn,
