@@ -36,35 +36,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 METRIC = "candidates scored/sec (Stage II, KV-cached) and users/sec (Stage I) on 1 B200"
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
-# kernel kind on the default workload, recorded from one ncu capture, with
-# the SHA-256 prefix of the kernel's sources at capture time.  The line
-# reports the recorded figure only while the sources still hash the same;
-# after a change of the kernel it reports null until the counters are taken
-# again.
-RECORDED_TRAFFIC = {
-    "fused_oproj_ffn": {"bytes_per_launch": 137.6e6, "sources": ("ffn_tc.cuh", "tc_ptx.cuh", "common.cuh"),
-                        "sha256_16": None, "captured": "2026-12-02"},
-}
 UNIT = "candidates/s"
-
-
-def sources_sha16(names) -> str:
-    import hashlib
-    h = hashlib.sha256()
-    for n in names:
-        with open(os.path.join(ROOT, "unified_transformer_recommender_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()[:16]
-
-
-def recorded_traffic(kernel: str):
-    """The recorded DRAM bytes per launch of `kernel`, or None when none was
-    recorded or its sources changed since."""
-    rec = RECORDED_TRAFFIC.get(kernel)
-    if not rec or not rec["sha256_16"] or sources_sha16(rec["sources"]) != rec["sha256_16"]:
-        return None
-    return rec["bytes_per_launch"]
 
 
 def parse():
@@ -926,8 +898,10 @@ def main():
     # ---- roofline of the dominant kernel (largest device time in the timed region)
     pk = peaks()
     dom_name, dom = max(prof.items(), key=lambda kv: kv[1]["ms"])
-    traffic = (recorded_traffic(dom_name)
-               if args.workload == "kv_serving" and not (args.users or args.cands) else None)
+    # DRAM bytes per launch come from ncu captures of single launches, which
+    # this run does not make; the line's mean over Stage I and Stage II
+    # launches has no captured counterpart
+    traffic = None
     per_launch_ms = dom["ms"] / dom["launches"]
     # the per-kernel times are single launches of well under a millisecond,
     # timed one by one: the burst figure of the measured GEMM peak applies
