@@ -1,0 +1,489 @@
+// Tensor-core attention of the training step (sm_100a, d_h = 64), on the
+// rows the backward recomputes: qkv [B, L, 3d] (q | k | v of every row, q
+// unscaled, bf16); the Lq queries are the tail rows L - Lq .. L - 1, query t
+// at key position L - Lq + t sees keys 0 .. that position.
+//
+//  * attn_train_q_kernel<false> (forward): one CTA per 128 queries of one
+//    head; per 128-key tile S = Q K^T (tcgen05, TMEM), online softmax in
+//    base 2 with the lazy rescale, O += P V with P from TMEM; writes the
+//    output rows and each row's log-sum-exp for the backward.
+//  * attn_train_q_kernel<true> (dQ): per key tile S = Q K^T and dP = dO V^T,
+//    then P = exp(S / sqrt(d_h) - lse) and dS = P (dP - D) per row (D =
+//    dO . O), dQ += dS K with dS from TMEM; dQ / sqrt(d_h) into dqkv.
+//  * attn_train_kv_kernel (dK, dV): one CTA per 128 keys of one head; per
+//    128-query tile S^T = K Q^T and dP^T = V dO^T, then P^T and dS^T per
+//    key row, dV += P^T dO and dK += dS^T Q with P^T, dS^T from TMEM.
+//
+// Roles (192 threads): warps 0-3 own one TMEM lane (row) each, warp 4 loads
+// tiles by TMA through a 2-stage ring, warp 5 issues the MMAs.  Every wait is
+// bounded (a timeout sets the device status word and the CTA drains).  One
+// CTA per SM: all 512 TMEM columns.
+#pragma once
+#include "tc_ptx.cuh"
+
+namespace ot {
+
+struct TrainAttnArgs {
+  int B, L, Lq, H, d;
+  const float* lse;      // [B, H, Lq] log-sum-exp, natural units (dQ, dK/dV)
+  float* lse_out;        // forward: written
+  const float* Dr;       // [B, H, Lq] dO . O per query row (dQ, dK/dV)
+  __nv_bfloat16* o;      // forward: output rows [B, Lq, d]
+  float* dqkv;           // [B, L, 3d]: dq into the q columns, dk / dv into k / v
+};
+
+struct TrainAttnCfg {
+  static constexpr int DH = 64, BM = 128, BN = 128, BOX = 16384, STAGES = 2;
+  static constexpr int BAR_BYTES = 256;
+  // 6 tiles of 16 KB; the request is raised to 120 KB so that one CTA runs per
+  // SM (each takes all 512 TMEM columns)
+  static constexpr int SMEM = 6 * BOX + BAR_BYTES;
+  static constexpr int SMEM_REQ = 120 * 1024;
+};
+
+__device__ inline float ex2_t(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ inline float fmax3_t(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+template <bool DQ>
+__global__ void __launch_bounds__(192, 1)
+    attn_train_q_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
+                        const TrainAttnArgs a) {
+  using C = TrainAttnCfg;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sQ = smem;
+  uint8_t* sDO = smem + C::BOX;
+  uint8_t* sKV = smem + 2 * C::BOX;   // [stage][K | V]
+  uint64_t* bars = (uint64_t*)(smem + 6 * C::BOX);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;              // [STAGES]
+  uint64_t* kv_empty = kv_full + C::STAGES;  // [STAGES]
+  uint64_t* s_full = kv_empty + C::STAGES;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* p_free = s_full + 3;
+  uint64_t* o_done = s_full + 4;
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 5);
+  if (smem_u32(smem) & 1023) {
+    if (threadIdx.x == 0) flag_error(kErrSmemAlign);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * C::BM, h = blockIdx.y, b = blockIdx.z;
+  const int q_off = a.L - a.Lq;
+  const int t_last = min(a.Lq, t0 + C::BM) - 1;
+  const int nt = (q_off + t_last + 1 + C::BN - 1) / C::BN;   // key tiles
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < C::STAGES; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(p_free, 1);
+    mbar_init(o_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmQKV);
+    if (DQ) prefetch_tmap(&tmDO);
+  }
+  if (warp == 5) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tX = tmem + 128, tP = tmem + 256, tQ = tmem + 320;  // tX: O (forward) or dP
+  grid_dep_wait();
+  grid_dep_launch();
+
+  if (warp == 4) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      mbar_expect_tx(q_full, (DQ ? 2 : 1) * C::BOX);
+      tma_load_3d(&tmQKV, q_full, sQ, h * C::DH, q_off + t0, b);
+      if (DQ) tma_load_3d(&tmDO, q_full, sDO, h * C::DH, t0, b);
+      for (int kt = 0; kt < nt; ++kt) {
+        const int s = kt % C::STAGES;
+        if (kt >= C::STAGES && !mbar_wait(&kv_empty[s], ((kt / C::STAGES) - 1) & 1)) break;
+        mbar_expect_tx(&kv_full[s], 2 * C::BOX);
+        uint8_t* sk = sKV + s * 2 * C::BOX;
+        tma_load_3d(&tmQKV, &kv_full[s], sk, a.d + h * C::DH, kt * C::BN, b);
+        tma_load_3d(&tmQKV, &kv_full[s], sk + C::BOX, 2 * a.d + h * C::DH, kt * C::BN, b);
+      }
+    }
+  } else if (warp == 5) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t id_ss = idesc_bf16(128, 128);
+      constexpr uint32_t id_ts = idesc_bf16(128, C::DH, false, true);
+      const uint64_t dq = sdesc_k128(smem_u32(sQ)), ddo = sdesc_k128(smem_u32(sDO));
+      const uint64_t dk0 = sdesc_k128(smem_u32(sKV)), dv0 = sdesc_k128(smem_u32(sKV + C::BOX));
+      // K (dQ += dS K) or V (O += P V) as the MN-major B operand
+      const uint64_t db0 = sdesc_mn128(smem_u32(sKV + (DQ ? 0 : C::BOX)), 0);
+      auto issue_s = [&](int kt) {
+        const int s = kt % C::STAGES;
+        const uint64_t dk = desc_add(dk0, s * 2 * C::BOX), dv = desc_add(dv0, s * 2 * C::BOX);
+#pragma unroll
+        for (int k = 0; k < C::DH / 16; ++k) umma_bf16(tS, desc_add(dq, k * 32), desc_add(dk, k * 32), id_ss, k ? 1u : 0u);
+        if (DQ) {
+#pragma unroll
+          for (int k = 0; k < C::DH / 16; ++k)
+            umma_bf16(tX, desc_add(ddo, k * 32), desc_add(dv, k * 32), id_ss, k ? 1u : 0u);
+        }
+        umma_commit(s_full);
+      };
+      bool ok = mbar_wait(q_full, 0) && mbar_wait(&kv_full[0], 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int kt = 0; kt < nt && ok; ++kt) {
+        // S (and dP) of tile kt are in registers: tile kt+1's may overwrite them
+        if (kt + 1 < nt) {
+          ok = mbar_wait(s_free, kt & 1) && mbar_wait(&kv_full[(kt + 1) % C::STAGES], ((kt + 1) / C::STAGES) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(kt + 1);
+        }
+        ok = mbar_wait(p_full, kt & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t db = desc_add(db0, (kt % C::STAGES) * 2 * C::BOX);
+        const uint32_t acc = DQ ? tQ : tX;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(acc, tP + kk * 8, desc_add(db, kk * 2048), id_ts, (kt || kk) ? 1u : 0u);
+        umma_commit(p_free);
+        umma_commit(&kv_empty[kt % C::STAGES]);
+      }
+      umma_commit(o_done);
+    }
+  } else {
+    // ------------------------------------------------- softmax + epilogue
+    const int r = warp * 32 + lane;
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const int t = t0 + r, pos = q_off + t;
+    const bool row_ok = t < a.Lq;
+    const float c = 1.4426950408889634f * 0.125f;   // log2(e) / sqrt(64): base-2 logits
+    const long long si = ((long long)b * a.H + h) * a.Lq + t;
+    float lse2 = 0.f, Dv = 0.f;
+    if (DQ && row_ok) {
+      lse2 = a.lse[si] * 1.4426950408889634f;
+      Dv = a.Dr[si];
+    }
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int kt = 0; kt < nt && ok; ++kt) {
+      ok = mbar_wait(s_full, kt & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const int kbase = kt * C::BN;
+      const int hi = row_ok ? min(max(pos + 1 - kbase, 0), C::BN) : 0;   // visible keys: [0, hi)
+      if (!DQ) {
+        float sv[128];
+        tmem_ld128(tS + lb, sv);
+        tc_fence_before();
+        mbar_arrive(s_free);
+#pragma unroll
+        for (int i = 0; i < 128; ++i) sv[i] = i < hi ? sv[i] * c : -INFINITY;
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; i += 8) {
+          m0 = fmax3_t(m0, sv[i], sv[i + 1]);
+          m1 = fmax3_t(m1, sv[i + 2], sv[i + 3]);
+          m2 = fmax3_t(m2, sv[i + 4], sv[i + 5]);
+          m3 = fmax3_t(m3, sv[i + 6], sv[i + 7]);
+        }
+        const float mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mt > m + 8.f) {
+          if (m != -INFINITY) {
+            alpha = ex2_t(m - mt);
+            rescale = true;
+          }
+          m = mt;
+        }
+        const float mref = m == -INFINITY ? 0.f : m;
+        float s0 = 0.f, s1 = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float pa = ex2_t(sv[2 * i] - mref), pb = ex2_t(sv[2 * i + 1] - mref);
+          s0 += pa;
+          s1 += pb;
+          pk[i] = pack_bf16x2(pa, pb);
+        }
+        l = l * alpha + (s0 + s1);
+        if (kt > 0) {
+          ok = mbar_wait(p_free, (kt - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        // tcgen05.ld/st are warp-collective: the warp rescales when any row does
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int cc = 0; cc < C::DH / 32; ++cc) {
+            float ov[32];
+            tmem_ld32(tX + lb + cc * 32, ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(tX + lb + cc * 32, ov);
+          }
+        }
+        tmem_st64(tP + lb, pk);
+      } else {
+        // P and dS need the previous tile's dQ MMA to be done with TMEM's P
+        if (kt > 0) {
+          ok = mbar_wait(p_free, (kt - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          float sv[32], dp[32];
+          tmem_ld32(tS + lb + qq * 32, sv);
+          tmem_ld32(tX + lb + qq * 32, dp);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = qq * 32 + 2 * i;
+            const float pa = c0 < hi ? ex2_t(fmaf(sv[2 * i], c, -lse2)) : 0.f;
+            const float pb = c0 + 1 < hi ? ex2_t(fmaf(sv[2 * i + 1], c, -lse2)) : 0.f;
+            pk[i] = pack_bf16x2(pa * (dp[2 * i] - Dv), pb * (dp[2 * i + 1] - Dv));
+          }
+          tmem_st16(tP + lb + qq * 16, pk);
+        }
+        tc_fence_before();
+        mbar_arrive(s_free);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    ok = ok && mbar_wait(o_done, 0);
+    tc_fence_after();
+    float o[C::DH];
+#pragma unroll
+    for (int cc = 0; cc < C::DH / 32; ++cc) tmem_ld32((DQ ? tQ : tX) + lb + cc * 32, o + cc * 32);
+    if (ok && row_ok) {
+      if (!DQ) {
+        const float inv = 1.f / l;
+#pragma unroll
+        for (int e = 0; e < C::DH; ++e) o[e] *= inv;
+        __nv_bfloat16* dst = a.o + ((long long)b * a.Lq + t) * a.d + h * C::DH;
+#pragma unroll
+        for (int cc = 0; cc < C::DH / 32; ++cc) store_bf16x32(dst + cc * 32, o + cc * 32);
+        a.lse_out[si] = (m + log2f(l)) * 0.6931471805599453f;
+      } else {
+        float* dst = a.dqkv + ((long long)b * a.L + pos) * 3 * a.d + h * C::DH;
+#pragma unroll
+        for (int e = 0; e < C::DH; e += 4)
+          *(float4*)(dst + e) = make_float4(o[e] * 0.125f, o[e + 1] * 0.125f, o[e + 2] * 0.125f, o[e + 3] * 0.125f);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+__global__ void __launch_bounds__(192, 1)
+    attn_train_kv_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
+                         const TrainAttnArgs a) {
+  using C = TrainAttnCfg;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + C::BOX;
+  uint8_t* sQD = smem + 2 * C::BOX;   // [stage][Q | dO]
+  uint64_t* bars = (uint64_t*)(smem + 6 * C::BOX);
+  uint64_t* kv_ready = bars;
+  uint64_t* qd_full = bars + 1;              // [STAGES]
+  uint64_t* qd_empty = qd_full + C::STAGES;  // [STAGES]
+  uint64_t* s_full = qd_empty + C::STAGES;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* p_free = s_full + 3;
+  uint64_t* o_done = s_full + 4;
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 5);
+  if (smem_u32(smem) & 1023) {
+    if (threadIdx.x == 0) flag_error(kErrSmemAlign);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = blockIdx.x * C::BN, h = blockIdx.y, b = blockIdx.z;
+  const int q_off = a.L - a.Lq;
+  const int it0 = max(0, j0 - q_off) / C::BM;            // first query tile that sees a key of this tile
+  const int nq = (a.Lq + C::BM - 1) / C::BM - it0;       // query tiles
+  if (threadIdx.x == 0) {
+    mbar_init(kv_ready, 1);
+    for (int i = 0; i < C::STAGES; ++i) { mbar_init(&qd_full[i], 1); mbar_init(&qd_empty[i], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(p_free, 1);
+    mbar_init(o_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmQKV);
+    prefetch_tmap(&tmDO);
+  }
+  if (warp == 5) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tDP = tmem + 128, tP = tmem + 256, tDS = tmem + 320, tDV = tmem + 384,
+                 tDK = tmem + 448;
+  grid_dep_wait();
+  grid_dep_launch();
+
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_expect_tx(kv_ready, 2 * C::BOX);
+      tma_load_3d(&tmQKV, kv_ready, sK, a.d + h * C::DH, j0, b);
+      tma_load_3d(&tmQKV, kv_ready, sV, 2 * a.d + h * C::DH, j0, b);
+      for (int i = 0; i < nq; ++i) {
+        const int s = i % C::STAGES, q0 = (it0 + i) * C::BM;
+        if (i >= C::STAGES && !mbar_wait(&qd_empty[s], ((i / C::STAGES) - 1) & 1)) break;
+        mbar_expect_tx(&qd_full[s], 2 * C::BOX);
+        uint8_t* sq = sQD + s * 2 * C::BOX;
+        tma_load_3d(&tmQKV, &qd_full[s], sq, h * C::DH, q_off + q0, b);
+        tma_load_3d(&tmDO, &qd_full[s], sq + C::BOX, h * C::DH, q0, b);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t id_ss = idesc_bf16(128, 128);
+      constexpr uint32_t id_ts = idesc_bf16(128, C::DH, false, true);
+      const uint64_t dk = sdesc_k128(smem_u32(sK)), dv = sdesc_k128(smem_u32(sV));
+      const uint64_t dq0 = sdesc_k128(smem_u32(sQD)), ddo0 = sdesc_k128(smem_u32(sQD + C::BOX));
+      const uint64_t mq0 = sdesc_mn128(smem_u32(sQD), 0), mdo0 = sdesc_mn128(smem_u32(sQD + C::BOX), 0);
+      bool ok = mbar_wait(kv_ready, 0);
+      for (int i = 0; i < nq && ok; ++i) {
+        const int s = i % C::STAGES;
+        ok = mbar_wait(&qd_full[s], (i / C::STAGES) & 1);
+        if (ok && i > 0) ok = mbar_wait(s_free, (i - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t so = s * 2 * C::BOX;
+        // S^T = K Q^T and dP^T = V dO^T: keys on the TMEM lanes, queries on the columns
+#pragma unroll
+        for (int k = 0; k < C::DH / 16; ++k)
+          umma_bf16(tS, desc_add(dk, k * 32), desc_add(desc_add(dq0, so), k * 32), id_ss, k ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < C::DH / 16; ++k)
+          umma_bf16(tDP, desc_add(dv, k * 32), desc_add(desc_add(ddo0, so), k * 32), id_ss, k ? 1u : 0u);
+        umma_commit(s_full);
+        ok = mbar_wait(p_full, i & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // dV += P^T dO, dK += dS^T Q: A from TMEM (16 queries per step), B MN-major
+        const uint64_t mdo = desc_add(mdo0, so), mq = desc_add(mq0, so);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(tDV, tP + kk * 8, desc_add(mdo, kk * 2048), id_ts, (i || kk) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(tDK, tDS + kk * 8, desc_add(mq, kk * 2048), id_ts, (i || kk) ? 1u : 0u);
+        umma_commit(p_free);
+        umma_commit(&qd_empty[s]);
+      }
+      umma_commit(o_done);
+    }
+  } else {
+    const int r = warp * 32 + lane;
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const int j = j0 + r;
+    const bool key_ok = j < a.L;
+    const float c = 1.4426950408889634f * 0.125f;
+    const float* lse = a.lse + ((long long)b * a.H + h) * a.Lq;
+    const float* Dr = a.Dr + ((long long)b * a.H + h) * a.Lq;
+    bool ok = true;
+    for (int i = 0; i < nq && ok; ++i) {
+      const int q0 = (it0 + i) * C::BM;
+      ok = mbar_wait(s_full, i & 1);
+      if (ok && i > 0) ok = mbar_wait(p_free, (i - 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      // query column cc sees this key when q_off + q0 + cc >= j, and exists when q0 + cc < Lq
+      const int lo = key_ok ? min(max(j - q_off - q0, 0), C::BM) : C::BM;
+      const int hi = min(max(a.Lq - q0, 0), C::BM);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        float sv[32], dp[32];
+        tmem_ld32(tS + lb + qq * 32, sv);
+        tmem_ld32(tDP + lb + qq * 32, dp);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float p2[2], d2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int cc = qq * 32 + 2 * e + u;
+            const bool vis = cc >= lo && cc < hi;
+            const float ls = vis ? lse[q0 + cc] * 1.4426950408889634f : 0.f;
+            const float D = vis ? Dr[q0 + cc] : 0.f;
+            const float p = vis ? ex2_t(fmaf(sv[2 * e + u], c, -ls)) : 0.f;
+            p2[u] = p;
+            d2[u] = p * (dp[2 * e + u] - D);
+          }
+          pk[e] = pack_bf16x2(p2[0], p2[1]);
+          dk[e] = pack_bf16x2(d2[0], d2[1]);
+        }
+        tmem_st16(tP + lb + qq * 16, pk);
+        tmem_st16(tDS + lb + qq * 16, dk);
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    ok = ok && mbar_wait(o_done, 0);
+    tc_fence_after();
+    float dv[C::DH], dkv[C::DH];
+#pragma unroll
+    for (int cc = 0; cc < C::DH / 32; ++cc) {
+      tmem_ld32(tDV + lb + cc * 32, dv + cc * 32);
+      tmem_ld32(tDK + lb + cc * 32, dkv + cc * 32);
+    }
+    if (ok && key_ok) {
+      float* dst = a.dqkv + ((long long)b * a.L + j) * 3 * a.d + h * C::DH;
+#pragma unroll
+      for (int e = 0; e < C::DH; e += 4) {
+        *(float4*)(dst + a.d + e) = make_float4(dkv[e] * 0.125f, dkv[e + 1] * 0.125f, dkv[e + 2] * 0.125f,
+                                                dkv[e + 3] * 0.125f);
+        *(float4*)(dst + 2 * a.d + e) = make_float4(dv[e], dv[e + 1], dv[e + 2], dv[e + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+// D = dO . O per (sample, head, query row): the row term of the softmax's
+// backward.  One thread per (row, head).
+__global__ void attn_train_delta_kernel(const float* __restrict__ dO, const __nv_bfloat16* __restrict__ O, float* Dr,
+                                        int B, int Lq, int H, int dh) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)B * Lq * H) return;
+  const int h = (int)(i % H);
+  const long long bt = i / H;
+  const int t = (int)(bt % Lq), b = (int)(bt / Lq);
+  const long long off = bt * H * dh + (long long)h * dh;
+  float acc = 0.f;
+  for (int e = 0; e < dh; ++e) acc = fmaf(dO[off + e], __bfloat162float(O[off + e]), acc);
+  Dr[((long long)b * H + h) * Lq + t] = acc;
+}
+
+}  // namespace ot

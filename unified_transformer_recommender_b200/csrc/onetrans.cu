@@ -18,6 +18,7 @@
 #include "attn_tc.cuh"
 #include "ffn_tc.cuh"
 #include "backward.cuh"
+#include "attn_train.cuh"
 
 using namespace ot;
 
@@ -1157,6 +1158,51 @@ static onetrans_status launch_attn_rows(const onetrans_model* m, int stage, cons
   return last_launch();
 }
 
+// Tensor-core attention of the training step (bf16, d_h = 64): stage 0 the
+// forward with log-sum-exp, 1 dQ, 2 dK and dV.
+static bool train_attn_tc(const onetrans_model* m) {
+  return m->bf16 && g_policy == 0 && m->dh == TrainAttnCfg::DH && m->d % 64 == 0 && encode_fn() != nullptr;
+}
+
+static onetrans_status launch_attn_train_tc(const onetrans_model* m, int stage, const AttnRows& ar, void* o,
+                                            float* lse, float* Dr, const void* dOb, float* dqkv, cudaStream_t st) {
+  using C = TrainAttnCfg;
+  const int d = ar.d;
+  CUtensorMap tq, tdo;
+  if (!make_tmap_3d(&tq, ar.qkv, 3 * (uint64_t)d, ar.L, ar.B, 3 * (uint64_t)d, (uint64_t)ar.L * 3 * d, 64, 128, 1))
+    return ONETRANS_ERR_CUDA;
+  if (stage > 0) {
+    if (!make_tmap_3d(&tdo, dOb, d, ar.Lq, ar.B, d, (uint64_t)ar.Lq * d, 64, 128, 1)) return ONETRANS_ERR_CUDA;
+  } else {
+    tdo = tq;
+  }
+  TrainAttnArgs ta;
+  std::memset(&ta, 0, sizeof(ta));
+  ta.B = ar.B; ta.L = ar.L; ta.Lq = ar.Lq; ta.H = ar.H; ta.d = d;
+  ta.lse = lse; ta.lse_out = lse; ta.Dr = Dr; ta.o = (__nv_bfloat16*)o; ta.dqkv = dqkv;
+  const double pairs = (double)ar.B * ar.H * ((double)ar.Lq * (ar.L - ar.Lq) + 0.5 * (double)ar.Lq * (ar.Lq + 1));
+  ProfScope prof(PK_TRAIN_ATTN, pairs * 2.0 * C::DH * (stage == 0 ? 2 : stage == 1 ? 3 : 4),
+                 (double)ar.B * ar.L * 3 * d * 2 + (double)ar.B * ar.Lq * d * 4, st);
+  static bool attr[3] = {false, false, false};
+  if (!attr[stage]) {
+    cudaError_t e = stage == 0 ? cudaFuncSetAttribute(attn_train_q_kernel<false>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_REQ)
+                    : stage == 1 ? cudaFuncSetAttribute(attn_train_q_kernel<true>,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_REQ)
+                                 : cudaFuncSetAttribute(attn_train_kv_kernel,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_REQ);
+    if (e != cudaSuccess) return ONETRANS_ERR_CUDA;
+    attr[stage] = true;
+  }
+  if (stage == 0)
+    attn_train_q_kernel<false><<<dim3((unsigned)cdiv(ar.Lq, C::BM), ar.H, ar.B), 192, C::SMEM_REQ, st>>>(tq, tdo, ta);
+  else if (stage == 1)
+    attn_train_q_kernel<true><<<dim3((unsigned)cdiv(ar.Lq, C::BM), ar.H, ar.B), 192, C::SMEM_REQ, st>>>(tq, tdo, ta);
+  else
+    attn_train_kv_kernel<<<dim3((unsigned)cdiv(ar.L, C::BN), ar.H, ar.B), 192, C::SMEM_REQ, st>>>(tq, tdo, ta);
+  return last_launch();
+}
+
 template <typename T>
 static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B, int L_S, const float* dy,
                                   float* out, float* dx0, const onetrans_grads* gr, void* ws, size_t ws_bytes,
@@ -1198,7 +1244,9 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
   void* opA = cv.take((size_t)op_elems * es);
   void* opW = cv.take((size_t)op_elems * es);
   void* wT = cv.take((size_t)wt_elems * es);
+  void* dOb = cv.take((size_t)B * Lq0 * d * es);   // the attention output's gradient in the storage type
   if (need) { *need = cv.used; return ONETRANS_OK; }
+  const bool tc_attn = train_attn_tc(m);
   if (cv.overflow) return ONETRANS_ERR_CAPACITY;
 
   // transposed weights of one layer's S set and NS sets: [N_out, K_in] -> [K_in, N_out]
@@ -1222,7 +1270,8 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
                               rmap(qkv, (long long)L * 3 * d, 3 * d), st));
     AttnRows ar;
     ar.qkv = qkv; ar.B = B; ar.L = L; ar.Lq = Lqn; ar.H = H; ar.d = d;
-    OT_TRY(launch_attn_rows<T>(m, 0, ar, a, lse, nullptr, nullptr, nullptr, st));
+    if (tc_attn) OT_TRY(launch_attn_train_tc(m, 0, ar, a, lse, nullptr, nullptr, nullptr, st));
+    else OT_TRY(launch_attn_rows<T>(m, 0, ar, a, lse, nullptr, nullptr, nullptr, st));
     // x1 = x[tail] + W^O a, h2 = RMSNorm(x1)
     GemmDesc go = gdesc_base(m);
     go.mode = TILE_FLAT; go.M = B * Lqn; go.fold = Lqn; go.G = 1;
@@ -1300,8 +1349,18 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     OT_TRY(cuda_ok(cudaMemsetAsync(dqkv, 0, (size_t)B * L * 3 * d * 4, st)));
     AttnRows ar;
     ar.qkv = qkv; ar.B = B; ar.L = L; ar.Lq = Lqn; ar.H = H; ar.d = d;
-    OT_TRY(launch_attn_rows<T>(m, 1, ar, a, lse, da, Dr, dqkv, st));
-    OT_TRY(launch_attn_rows<T>(m, 2, ar, a, lse, da, Dr, dqkv, st));
+    if (tc_attn) {
+      OT_TRY(launch_cast<T>(da, dOb, (long long)B * Md, st));
+      const long long nd = (long long)B * Lqn * H;
+      attn_train_delta_kernel<<<(unsigned)cdiv(nd, 256), 256, 0, st>>>(da, (const __nv_bfloat16*)a, Dr, B, Lqn, H,
+                                                                        m->dh);
+      OT_TRY(last_launch());
+      OT_TRY(launch_attn_train_tc(m, 1, ar, a, lse, Dr, dOb, dqkv, st));
+      OT_TRY(launch_attn_train_tc(m, 2, ar, a, lse, Dr, dOb, dqkv, st));
+    } else {
+      OT_TRY(launch_attn_rows<T>(m, 1, ar, a, lse, da, Dr, dqkv, st));
+      OT_TRY(launch_attn_rows<T>(m, 2, ar, a, lse, da, Dr, dqkv, st));
+    }
     // (q, k, v) = W_i^{QKV} h_i
     const long long Mq = (long long)L * 3 * d;
     OT_TRY(weight_grad<T>(m, GradRows{dqkv, 3 * d, Mq, true}, GradRows{h, d, (long long)L * d, false}, 3 * d, d,
