@@ -23,12 +23,14 @@ __device__ inline long long rowset_off(const RowSet& s, int g, int r) {
   return (long long)g * s.gs + (long long)b * s.sb + (long long)t * s.st;
 }
 
-// dst[g][c][r] = src row r of group g, column c (r < R), 0 for R <= r < R_pad:
-// the K-major operand of a GEMM that contracts over rows.  32 x 32 tiles
-// through shared memory, so both the reads and the writes are coalesced.
+// The K-major operand of a GEMM that contracts over rows: row r of group g,
+// column c goes to dst[g][r / Kc][c][r % Kc] (R_pad = chunks x Kc; 0 for
+// R <= r < R_pad), so that each chunk of Kc rows is its own K-major matrix
+// (Kc = R_pad: one chunk).  32 x 32 tiles through shared memory, so both the
+// reads and the writes are coalesced.
 template <typename Ti, typename To>
 __global__ void __launch_bounds__(256) transpose_rows_kernel(const Ti* __restrict__ src, RowSet s, int C,
-                                                             To* __restrict__ dst, int R_pad) {
+                                                             To* __restrict__ dst, int R_pad, int Kc) {
   __shared__ float tile[32][33];
   const int g = blockIdx.z, c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -42,26 +44,42 @@ __global__ void __launch_bounds__(256) transpose_rows_kernel(const Ti* __restric
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int c = c0 + ty + 8 * i, r = r0 + tx;
-    if (c < C && r < R_pad) out[(long long)c * R_pad + r] = from_f<To>(tile[tx][ty + 8 * i]);
+    if (c < C && r < R_pad) {
+      const int ch = r / Kc;
+      out[(long long)ch * C * Kc + (long long)c * Kc + (r - ch * Kc)] = from_f<To>(tile[tx][ty + 8 * i]);
+    }
   }
 }
 
-// dst[g * dst_gs + c] = sum over the set's rows r of src row r, column c.
-// 32 columns per CTA, 8 row lanes per column, fixed summation order.
+// out[i] = sum over the chunks k of part[k * n + i], in chunk order.
+__global__ void chunk_sum_kernel(const float* __restrict__ part, int chunks, long long n, float* __restrict__ out,
+                                 long long out_stride, long long n_inner) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float acc = 0.f;
+  for (int k = 0; k < chunks; ++k) acc += part[(long long)k * n + i];
+  out[(i / n_inner) * out_stride + i % n_inner] = acc;
+}
+
+// Column sums in two passes with a fixed order: this kernel sums chunk
+// blockIdx.z (kColChunk rows) of group g's rows into part[g][chunk][c], 32
+// columns per CTA and 8 row lanes per column; chunk_sum_kernel adds the chunks.
+constexpr int kColChunk = 256;
 __global__ void __launch_bounds__(256) colsum_kernel(const float* __restrict__ src, RowSet s, int C,
-                                                     float* __restrict__ dst, long long dst_gs) {
-  __shared__ float part[8][33];
-  const int g = blockIdx.y, tx = threadIdx.x & 31, ty = threadIdx.x >> 5, c = blockIdx.x * 32 + tx;
+                                                     float* __restrict__ part) {
+  __shared__ float red[8][33];
+  const int g = blockIdx.y, ch = blockIdx.z, tx = threadIdx.x & 31, ty = threadIdx.x >> 5, c = blockIdx.x * 32 + tx;
+  const int r_end = min(s.R, (ch + 1) * kColChunk);
   float acc = 0.f;
   if (c < C)
-    for (int r = ty; r < s.R; r += 8) acc += src[rowset_off(s, g, r) + c];
-  part[ty][tx] = acc;
+    for (int r = ch * kColChunk + ty; r < r_end; r += 8) acc += src[rowset_off(s, g, r) + c];
+  red[ty][tx] = acc;
   __syncthreads();
   if (ty == 0 && c < C) {
     float t = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) t += part[i][tx];
-    dst[(long long)g * dst_gs + c] = t;
+    for (int i = 0; i < 8; ++i) t += red[i][tx];
+    part[((long long)ch * gridDim.y + g) * C + c] = t;
   }
 }
 

@@ -979,6 +979,7 @@ static onetrans_status groupwise_impl(const onetrans_model* m, const void* feats
 }
 
 // ============================================================== training ==
+static long long pad64(long long r) { return (r + 63) / 64 * 64; }
 // The backward pass of the stack with activation recomputation: the forward
 // keeps only each layer's input; the backward recomputes a layer's
 // intermediates from its input, then runs the chain rule in reverse order of
@@ -986,24 +987,46 @@ static onetrans_status groupwise_impl(const onetrans_model* m, const void* feats
 // over rows (dX = dY W) takes the transposed weights, a GEMM that reduces
 // over rows (dW = dY^T X) takes both operands transposed (K-major), zero-
 // padded to a multiple of 64 rows.
-static long long pad64(long long r) { return (r + 63) / 64 * 64; }
-
 template <typename Ti, typename To>
 static onetrans_status launch_transpose(const void* src, const RowSet& s, int G, int C, void* dst, int R_pad,
-                                        cudaStream_t st) {
+                                        cudaStream_t st, int Kc = 0) {
   if (G <= 0 || C <= 0 || R_pad <= 0) return ONETRANS_OK;
   ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * ((double)s.R * sizeof(Ti) + (double)R_pad * sizeof(To)), st);
   dim3 grid((unsigned)cdiv(C, 32), (unsigned)cdiv(R_pad, 32), (unsigned)G);
-  transpose_rows_kernel<Ti, To><<<grid, 256, 0, st>>>((const Ti*)src, s, C, (To*)dst, R_pad);
+  transpose_rows_kernel<Ti, To><<<grid, 256, 0, st>>>((const Ti*)src, s, C, (To*)dst, R_pad, Kc > 0 ? Kc : R_pad);
   return last_launch();
 }
 
-static onetrans_status launch_colsum(const float* src, const RowSet& s, int G, int C, float* dst, long long dst_gs,
-                                     cudaStream_t st) {
-  if (G <= 0 || C <= 0) return ONETRANS_OK;
-  ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * (s.R + 1) * 4.0, st);
-  colsum_kernel<<<dim3((unsigned)cdiv(C, 32), (unsigned)G), 256, 0, st>>>(src, s, C, dst, dst_gs);
+static onetrans_status launch_chunk_sum(const float* part, int chunks, long long n, float* out, long long out_stride,
+                                        long long n_inner, cudaStream_t st) {
+  if (n <= 0) return ONETRANS_OK;
+  ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)n * (chunks + 1) * 4.0, st);
+  chunk_sum_kernel<<<(unsigned)cdiv(n, 256), 256, 0, st>>>(part, chunks, n, out, out_stride, n_inner);
   return last_launch();
+}
+
+// Column sums of G row sets into dst[g * dst_gs + c]: chunks of kColChunk
+// rows in parallel into `part` (workspace), then the chunks added in order.
+static onetrans_status launch_colsum(const float* src, const RowSet& s, int G, int C, float* dst, long long dst_gs,
+                                     float* part, cudaStream_t st) {
+  if (G <= 0 || C <= 0) return ONETRANS_OK;
+  const int chunks = (int)std::max<long long>(1, cdiv(s.R, kColChunk));
+  {
+    ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * (s.R + chunks) * 4.0, st);
+    colsum_kernel<<<dim3((unsigned)cdiv(C, 32), (unsigned)G, (unsigned)chunks), 256, 0, st>>>(src, s, C, part);
+    OT_TRY(last_launch());
+  }
+  return launch_chunk_sum(part, chunks, (long long)G * C, dst, dst_gs, C, st);
+}
+
+// Row chunks of a weight-gradient GEMM: enough (weight tile, chunk) CTAs to
+// fill two waves of 148 SMs, chunks a multiple of 64 rows.
+constexpr int kSplitCtas = 296;
+static void split_rows(int R, int N_out, int K_in, int& chunks, int& Kc) {
+  const int tiles = (int)(cdiv(N_out, 128) * cdiv(K_in, 256));
+  const int want = std::max(1, std::min(kSplitCtas / std::max(tiles, 1), (int)(pad64(R) / 64)));
+  Kc = (int)pad64(cdiv(R, want));
+  chunks = (int)cdiv(R, Kc);
 }
 
 static RowSet rowset(long long gs, long long sb, long long st, int T, int R) {
@@ -1060,32 +1083,51 @@ struct GradRows {
   bool f32;
 };
 
+// Scratch of the training step's reductions (workspace): the operand
+// transposes, the row chunks' partial weight gradients, the column sums'
+// partial sums.
+struct TrainScratch {
+  void *opA, *opW;
+  float *split_part, *col_part;
+};
+
 template <typename T>
 static onetrans_status weight_grad(const onetrans_model* m, GradRows Y, GradRows X, int N_out, int K_in, int B,
-                                   int t_lo, int t_s, int t_hi, float* dW_S, float* dW_NS, void* opA, void* opW,
+                                   int t_lo, int t_s, int t_hi, float* dW_S, float* dW_NS, const TrainScratch& sc,
                                    cudaStream_t st) {
+  void *opA = sc.opA, *opW = sc.opW;
   const int es = m->es;
-  auto transpose = [&](const GradRows& s, const RowSet& rs, int G, int C, void* dst, int R_pad) {
-    if (s.f32) return launch_transpose<float, T>(s.p, rs, G, C, dst, R_pad, st);
-    return launch_transpose<T, T>(s.p, rs, G, C, dst, R_pad, st);
+  auto transpose = [&](const GradRows& s, const RowSet& rs, int G, int C, void* dst, int R_pad, int Kc) {
+    if (s.f32) return launch_transpose<float, T>(s.p, rs, G, C, dst, R_pad, st, Kc);
+    return launch_transpose<T, T>(s.p, rs, G, C, dst, R_pad, st, Kc);
   };
   // a set with no rows (the S set of a layer that keeps only NS rows) has a zero gradient
   if (t_s == t_lo && dW_S) OT_TRY(cuda_ok(cudaMemsetAsync(dW_S, 0, (size_t)N_out * K_in * 4, st)));
   if (t_s > t_lo && dW_S) {
+    // the reduction over rows is split into row chunks, each its own K-major
+    // pair of operands: a grouped GEMM gives one partial gradient per chunk,
+    // added in chunk order
     const int Tn = t_s - t_lo, R = B * Tn;
-    const int Rp = (int)pad64(R);
+    int chunks, Kc;
+    split_rows(R, N_out, K_in, chunks, Kc);
+    const int Rp = chunks * Kc;
     const RowSet ry = rowset(0, Y.samp, Y.row, Tn, R), rx = rowset(0, X.samp, X.row, Tn, R);
     GradRows y0 = Y, x0 = X;
     y0.p = (const char*)Y.p + t_lo * Y.row * (Y.f32 ? 4 : es);
     x0.p = (const char*)X.p + t_lo * X.row * (X.f32 ? 4 : es);
-    OT_TRY(transpose(y0, ry, 1, N_out, opA, Rp));
-    OT_TRY(transpose(x0, rx, 1, K_in, opW, Rp));
+    OT_TRY(transpose(y0, ry, 1, N_out, opA, Rp, Kc));
+    OT_TRY(transpose(x0, rx, 1, K_in, opW, Rp, Kc));
     GemmDesc g = gdesc_base(m);
-    g.mode = TILE_FLAT; g.M = N_out; g.G = 1;
-    g.K = Rp; g.A = opA; g.a_sm = Rp; g.a_mext = N_out; g.a_gext = 1;
-    g.W = opW; g.w_rows = K_in; g.N = K_in;
-    g.out = rmap32(dW_S, 0, K_in);
+    g.mode = TILE_SAMPLES; g.M = N_out; g.G = chunks; g.g_lo = 0; g.grp_base = 0;
+    g.K = Kc; g.A = opA; g.a_sm = Kc; g.a_sg = (long long)N_out * Kc; g.a_mext = N_out; g.a_gext = chunks;
+    g.W = opW; g.w_sg = (long long)K_in * Kc; g.w_rows = K_in; g.w_groups = chunks; g.N = K_in;
+    float* out = chunks > 1 ? sc.split_part : dW_S;
+    g.out = rmap32(out, K_in, (long long)N_out * K_in);
     OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
+    if (chunks > 1) {
+      const long long n = (long long)N_out * K_in;
+      OT_TRY(launch_chunk_sum(sc.split_part, chunks, n, dW_S, 0, n, st));
+    }
   }
   if (t_hi > t_s && dW_NS) {
     const int G = t_hi - t_s, Bp = (int)pad64(B);
@@ -1093,8 +1135,8 @@ static onetrans_status weight_grad(const onetrans_model* m, GradRows Y, GradRows
     GradRows y0 = Y, x0 = X;
     y0.p = (const char*)Y.p + t_s * Y.row * (Y.f32 ? 4 : es);
     x0.p = (const char*)X.p + t_s * X.row * (X.f32 ? 4 : es);
-    OT_TRY(transpose(y0, ry, G, N_out, opA, Bp));
-    OT_TRY(transpose(x0, rx, G, K_in, opW, Bp));
+    OT_TRY(transpose(y0, ry, G, N_out, opA, Bp, Bp));
+    OT_TRY(transpose(x0, rx, G, K_in, opW, Bp, Bp));
     GemmDesc g = gdesc_base(m);
     g.mode = TILE_SAMPLES; g.M = N_out; g.G = G; g.g_lo = 0; g.grp_base = 0;
     g.K = Bp; g.A = opA; g.a_sm = Bp; g.a_sg = (long long)N_out * Bp; g.a_mext = N_out; g.a_gext = G;
@@ -1108,12 +1150,13 @@ static onetrans_status weight_grad(const onetrans_model* m, GradRows Y, GradRows
 // Bias gradient: column sums of float32 rows, the S set over all its rows and
 // each NS set over its token's rows.
 static onetrans_status bias_grad(const float* rows, long long row, long long samp, int C, int B, int t_lo, int t_s,
-                                 int t_hi, float* db_S, float* db_NS, cudaStream_t st) {
+                                 int t_hi, float* db_S, float* db_NS, float* part, cudaStream_t st) {
   if (t_s == t_lo && db_S) OT_TRY(cuda_ok(cudaMemsetAsync(db_S, 0, (size_t)C * 4, st)));
   if (t_s > t_lo && db_S)
-    OT_TRY(launch_colsum(rows + t_lo * row, rowset(0, samp, row, t_s - t_lo, B * (t_s - t_lo)), 1, C, db_S, 0, st));
+    OT_TRY(launch_colsum(rows + t_lo * row, rowset(0, samp, row, t_s - t_lo, B * (t_s - t_lo)), 1, C, db_S, 0, part,
+                         st));
   if (t_hi > t_s && db_NS)
-    OT_TRY(launch_colsum(rows + t_s * row, rowset(row, samp, 0, 1, B), t_hi - t_s, C, db_NS, C, st));
+    OT_TRY(launch_colsum(rows + t_s * row, rowset(row, samp, 0, 1, B), t_hi - t_s, C, db_NS, C, part, st));
   return ONETRANS_OK;
 }
 
@@ -1215,8 +1258,10 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
   Ln[0] = L0;
   for (int n = 1; n < NL; ++n) Ln[n] = Lq[n - 1];
   const int Lq0 = Lq[0];
-  const long long Mmax = pad64((long long)B * L0);
+  const long long Mmax = pad64((long long)B * L0) + 64LL * kSplitCtas;   // row chunks pad each to 64 rows
   const long long op_elems = std::max<long long>(Mmax, (long long)L_NS * pad64(B)) * std::max(3 * d, dff);
+  const long long split_elems = (long long)kSplitCtas * 128 * 256;      // chunks x N_out x K_in, at most
+  const long long col_elems = (cdiv((long long)B * L0, kColChunk) + cdiv(B, kColChunk) * L_NS) * std::max(3 * d, dff);
   const long long wt_elems = (long long)(1 + L_NS) * std::max(3 * d, dff) * d;
   Carve cv(ws, ws_bytes);
   std::vector<float*> X(NL, nullptr);   // float32 inputs of layers 1 .. NL-1
@@ -1245,7 +1290,11 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
   void* opW = cv.take((size_t)op_elems * es);
   void* wT = cv.take((size_t)wt_elems * es);
   void* dOb = cv.take((size_t)B * Lq0 * d * es);   // the attention output's gradient in the storage type
+  float* split_part = (float*)cv.take((size_t)split_elems * 4);
+  float* col_part = (float*)cv.take((size_t)col_elems * 4);
   if (need) { *need = cv.used; return ONETRANS_OK; }
+  TrainScratch sc;
+  sc.opA = opA; sc.opW = opW; sc.split_part = split_part; sc.col_part = col_part;
   const bool tc_attn = train_attn_tc(m);
   if (cv.overflow) return ONETRANS_ERR_CAPACITY;
 
@@ -1312,9 +1361,9 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     OT_TRY(recompute(n, x_in, x_f32));
     const long long Md = (long long)Lqn * d, Mf = (long long)Lqn * dff;
     // y = x1 + W2 z + b2
-    OT_TRY(bias_grad(g_cur, d, Md, d, B, 0, sq, Lqn, gr->b2_S[n], gr->b2_NS[n], st));
+    OT_TRY(bias_grad(g_cur, d, Md, d, B, 0, sq, Lqn, gr->b2_S[n], gr->b2_NS[n], col_part, st));
     OT_TRY(weight_grad<T>(m, GradRows{g_cur, d, Md, true}, GradRows{z, dff, Mf, false}, d, dff, B, 0, sq, Lqn,
-                          gr->W2_S[n], gr->W2_NS[n], opA, opW, st));
+                          gr->W2_S[n], gr->W2_NS[n], sc, st));
     void *wS, *wNS;
     OT_TRY(launch_cast<T>(g_cur, rowT, (long long)B * Md, st));
     OT_TRY(weights_T(m->W2_S[n], m->W2_NS[n], d, dff, wS, wNS));
@@ -1326,18 +1375,18 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
       gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 256), 256, 0, st>>>(dz, u, du32, (T*)du, nz);
     }
     OT_TRY(last_launch());
-    OT_TRY(bias_grad(du32, dff, Mf, dff, B, 0, sq, Lqn, gr->b1_S[n], gr->b1_NS[n], st));
+    OT_TRY(bias_grad(du32, dff, Mf, dff, B, 0, sq, Lqn, gr->b1_S[n], gr->b1_NS[n], col_part, st));
     OT_TRY(weight_grad<T>(m, GradRows{du, dff, Mf, false}, GradRows{h2, d, Md, false}, dff, d, B, 0, sq, Lqn,
-                          gr->W1_S[n], gr->W1_NS[n], opA, opW, st));
+                          gr->W1_S[n], gr->W1_NS[n], sc, st));
     OT_TRY(weights_T(m->W1_S[n], m->W1_NS[n], dff, d, wS, wNS));
     OT_TRY(mixed_rows_gemm<T>(m, du, dff, Mf, Lqn, B, 0, sq, Lqn, wS, wNS, dff, d, rmap32(dh2, Md, d), st));
     // h2 = RMSNorm(x1; g_ffn), x1 = x[tail] + W^O a
     OT_TRY(cuda_ok(cudaMemcpyAsync(dx1, g_cur, (size_t)B * Md * 4, cudaMemcpyDeviceToDevice, st)));
     OT_TRY((launch_rms_backward<T, float>(x1, Md, d, m->g_ffn[n], dh2, dx1, Md, d, pg, B * Lqn, Lqn, d,
                                          m->cfg.rms_eps, st)));
-    OT_TRY(launch_colsum(pg, rowset(0, Md, d, Lqn, B * Lqn), 1, d, gr->g_ffn[n], 0, st));
+    OT_TRY(launch_colsum(pg, rowset(0, Md, d, Lqn, B * Lqn), 1, d, gr->g_ffn[n], 0, col_part, st));
     OT_TRY(weight_grad<T>(m, GradRows{dx1, d, Md, true}, GradRows{a, d, Md, false}, d, d, B, 0, Lqn, Lqn,
-                          gr->Wo[n], nullptr, opA, opW, st));
+                          gr->Wo[n], nullptr, sc, st));
     OT_TRY(launch_cast<T>(dx1, rowT, (long long)B * Md, st));
     OT_TRY(weights_T(m->Wo[n], nullptr, d, d, wS, wNS));
     OT_TRY(mixed_rows_gemm<T>(m, rowT, d, Md, Lqn, B, 0, Lqn, Lqn, wS, nullptr, d, d, rmap32(da, Md, d), st));
@@ -1364,7 +1413,7 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     // (q, k, v) = W_i^{QKV} h_i
     const long long Mq = (long long)L * 3 * d;
     OT_TRY(weight_grad<T>(m, GradRows{dqkv, 3 * d, Mq, true}, GradRows{h, d, (long long)L * d, false}, 3 * d, d,
-                          B, 0, s, L, gr->Wqkv_S[n], gr->Wqkv_NS[n], opA, opW, st));
+                          B, 0, s, L, gr->Wqkv_S[n], gr->Wqkv_NS[n], sc, st));
     OT_TRY(launch_cast<T>(dqkv, rowT, (long long)B * Mq, st));
     OT_TRY(weights_T(m->Wqkv_S[n], m->Wqkv_NS[n], 3 * d, d, wS, wNS));
     OT_TRY(mixed_rows_gemm<T>(m, rowT, 3 * d, Mq, L, B, 0, s, L, wS, wNS, 3 * d, d,
@@ -1376,7 +1425,7 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     else
       OT_TRY((launch_rms_backward<T, T>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
                                        B * L, L, d, m->cfg.rms_eps, st)));
-    OT_TRY(launch_colsum(pg, rowset(0, (long long)L * d, d, L, B * L), 1, d, gr->g_attn[n], 0, st));
+    OT_TRY(launch_colsum(pg, rowset(0, (long long)L * d, d, L, B * L), 1, d, gr->g_attn[n], 0, col_part, st));
     g_cur = g_in;
   }
   return ONETRANS_OK;
