@@ -195,7 +195,7 @@ def forward_config(name: str, U: int, ws: int) -> dict:
 
 ALU_KERNELS = ("train_attn_rows",)   # kernel kinds that run on the CUDA cores' FMA pipes
 TRAIN_METRIC = "samples/sec of the training step (forward + backward with recomputation) on 1 B200"
-TRAIN_SAMPLES = 8
+TRAIN_SAMPLES = 64
 
 
 def train_config(U: int, ws: int) -> dict:
