@@ -7,7 +7,7 @@
 // sums (bias and gain gradients), the RMSNorm and GELU backward steps, and
 // attention forward / backward on rows recomputed from the layer input.
 #pragma once
-#include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace ot {
 
@@ -28,9 +28,10 @@ __device__ inline long long rowset_off(const RowSet& s, int g, int r) {
 // R <= r < R_pad), so that each chunk of Kc rows is its own K-major matrix
 // (Kc = R_pad: one chunk).  32 x 32 tiles through shared memory, so both the
 // reads and the writes are coalesced.
+// Any shape: 32 x 32 tiles, one element per thread and pass.
 template <typename Ti, typename To>
-__global__ void __launch_bounds__(256) transpose_rows_kernel(const Ti* __restrict__ src, RowSet s, int C,
-                                                             To* __restrict__ dst, int R_pad, int Kc) {
+__global__ void __launch_bounds__(256) transpose_rows_scalar_kernel(const Ti* __restrict__ src, RowSet s, int C,
+                                                                    To* __restrict__ dst, int R_pad, int Kc) {
   __shared__ float tile[32][33];
   const int g = blockIdx.z, c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -47,6 +48,56 @@ __global__ void __launch_bounds__(256) transpose_rows_kernel(const Ti* __restric
     if (c < C && r < R_pad) {
       const int ch = r / Kc;
       out[(long long)ch * C * Kc + (long long)c * Kc + (r - ch * Kc)] = from_f<To>(tile[tx][ty + 8 * i]);
+    }
+  }
+}
+
+// 64 x 64 tiles, 256 threads: each thread reads 4 columns of 4 rows (one
+// vector load per row, one row-offset computation per row) and writes 4 rows
+// of the transposed tile, 4 consecutive elements each.  Needs C % 4 == 0, the
+// row strides % 4 == 0, R_pad % 64 == 0 and Kc % 64 == 0 (the host checks).
+template <typename Ti, typename To>
+__global__ void __launch_bounds__(256) transpose_rows_kernel(const Ti* __restrict__ src, RowSet s, int C,
+                                                             To* __restrict__ dst, int R_pad, int Kc) {
+  __shared__ float tile[64][65];
+  const int g = blockIdx.z, c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  const int cq = (threadIdx.x & 15) * 4, rq = threadIdx.x >> 4;   // 16 column quads x 16 row lanes
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = rq + 16 * i, r = r0 + rr, c = c0 + cq;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (r < s.R && c < C) {
+      const Ti* p = src + rowset_off(s, g, r) + c;
+      if (sizeof(Ti) == 4) {
+        const float4 f = *(const float4*)p;
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+      } else {
+        const uint2 u = *(const uint2*)p;
+        const __nv_bfloat162* h = (const __nv_bfloat162*)&u;
+        const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tile[rr][cq + j] = v[j];
+  }
+  __syncthreads();
+  To* out = dst + (long long)g * C * R_pad;
+  const int ch = r0 / Kc, rin = r0 - ch * Kc + cq;   // the 64 rows of a tile lie in one chunk
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int cc = rq + 16 * i, c = c0 + cc;
+    if (c < C && r0 < R_pad) {
+      To* q = out + (long long)ch * C * Kc + (long long)c * Kc + rin;
+      if (sizeof(To) == 4) {
+        *(float4*)q = make_float4(tile[cq][cc], tile[cq + 1][cc], tile[cq + 2][cc], tile[cq + 3][cc]);
+      } else {
+        uint2 u;
+        __nv_bfloat162* h = (__nv_bfloat162*)&u;
+        h[0] = __floats2bfloat162_rn(tile[cq][cc], tile[cq + 1][cc]);
+        h[1] = __floats2bfloat162_rn(tile[cq + 2][cc], tile[cq + 3][cc]);
+        *(uint2*)q = u;
+      }
     }
   }
 }
@@ -124,7 +175,7 @@ __global__ void __launch_bounds__(256) rms_backward_kernel(const Tx* __restrict_
 // v = c (u + a u^3), c = sqrt(2/pi), a = 0.044715.
 __device__ inline float gelu_tanh_grad(float u) {
   const float c = 0.7978845608028654f, a = 0.044715f;
-  const float th = tanhf(c * (u + a * u * u * u));
+  const float th = tanh_fast(c * (u + a * u * u * u));   // MUFU tanh, relative error about 2^-11
   return 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * a * u * u);
 }
 
@@ -132,7 +183,7 @@ __device__ inline float gelu_tanh_grad(float u) {
 template <typename T>
 __global__ void gelu_forward_kernel(const float* __restrict__ u, T* __restrict__ z, long long n) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) z[i] = from_f<T>(gelu_tanh(u[i]));
+  if (i < n) z[i] = from_f<T>(gelu_fast(u[i]));   // MUFU tanh, as the inference path's FFN
 }
 
 // du = dz * GELU'(u): float32 (its column sums are db1) and the storage type

@@ -991,9 +991,16 @@ template <typename Ti, typename To>
 static onetrans_status launch_transpose(const void* src, const RowSet& s, int G, int C, void* dst, int R_pad,
                                         cudaStream_t st, int Kc = 0) {
   if (G <= 0 || C <= 0 || R_pad <= 0) return ONETRANS_OK;
+  const int kc = Kc > 0 ? Kc : R_pad;
   ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * ((double)s.R * sizeof(Ti) + (double)R_pad * sizeof(To)), st);
-  dim3 grid((unsigned)cdiv(C, 32), (unsigned)cdiv(R_pad, 32), (unsigned)G);
-  transpose_rows_kernel<Ti, To><<<grid, 256, 0, st>>>((const Ti*)src, s, C, (To*)dst, R_pad, Kc > 0 ? Kc : R_pad);
+  const bool vec = C % 4 == 0 && s.st % 4 == 0 && s.sb % 4 == 0 && s.gs % 4 == 0 && R_pad % 64 == 0 &&
+                   kc % 64 == 0 && (uintptr_t)src % 16 == 0 && (uintptr_t)dst % 16 == 0;
+  if (vec)
+    transpose_rows_kernel<Ti, To><<<dim3((unsigned)cdiv(C, 64), (unsigned)(R_pad / 64), (unsigned)G), 256, 0, st>>>(
+        (const Ti*)src, s, C, (To*)dst, R_pad, kc);
+  else
+    transpose_rows_scalar_kernel<Ti, To><<<dim3((unsigned)cdiv(C, 32), (unsigned)cdiv(R_pad, 32), (unsigned)G), 256,
+                                           0, st>>>((const Ti*)src, s, C, (To*)dst, R_pad, kc);
   return last_launch();
 }
 
