@@ -35,9 +35,10 @@ struct TrainAttnArgs {
 struct TrainAttnCfg {
   static constexpr int DH = 64, BM = 128, BN = 128, BOX = 16384, STAGES = 2;
   static constexpr int BAR_BYTES = 256;
-  // 6 tiles of 16 KB; the request is raised to 120 KB so that one CTA runs per
-  // SM (each takes all 512 TMEM columns)
-  static constexpr int SMEM = 6 * BOX + BAR_BYTES;
+  // 6 tiles of 16 KB, the barriers, a query tile's log-sum-exp and D (1 KB);
+  // the request is raised to 120 KB so that one CTA runs per SM (each takes
+  // all 512 TMEM columns)
+  static constexpr int SMEM = 6 * BOX + BAR_BYTES + 2 * BM * 4;
   static constexpr int SMEM_REQ = 120 * 1024;
 };
 
@@ -407,12 +408,22 @@ __global__ void __launch_bounds__(192, 1)
     const float c = 1.4426950408889634f * 0.125f;
     const float* lse = a.lse + ((long long)b * a.H + h) * a.Lq;
     const float* Dr = a.Dr + ((long long)b * a.H + h) * a.Lq;
+    // the query tile's log-sum-exp (base 2) and D, one column per softmax thread
+    float* s_lse = (float*)(smem + 6 * C::BOX + C::BAR_BYTES);
+    float* s_D = s_lse + C::BM;
     bool ok = true;
-    for (int i = 0; i < nq && ok; ++i) {
+    // every softmax thread passes both named barriers on every tile, even
+    // after a wait that gave up, so that none is left waiting at one
+    for (int i = 0; i < nq; ++i) {
       const int q0 = (it0 + i) * C::BM;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      s_lse[r] = q0 + r < a.Lq ? lse[q0 + r] * 1.4426950408889634f : 0.f;
+      s_D[r] = q0 + r < a.Lq ? Dr[q0 + r] : 0.f;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!ok) continue;
       ok = mbar_wait(s_full, i & 1);
       if (ok && i > 0) ok = mbar_wait(p_free, (i - 1) & 1);
-      if (!ok) break;
+      if (!ok) continue;
       tc_fence_after();
       // query column cc sees this key when q_off + q0 + cc >= j, and exists when q0 + cc < Lq
       const int lo = key_ok ? min(max(j - q_off - q0, 0), C::BM) : C::BM;
@@ -430,11 +441,9 @@ __global__ void __launch_bounds__(192, 1)
           for (int u = 0; u < 2; ++u) {
             const int cc = qq * 32 + 2 * e + u;
             const bool vis = cc >= lo && cc < hi;
-            const float ls = vis ? lse[q0 + cc] * 1.4426950408889634f : 0.f;
-            const float D = vis ? Dr[q0 + cc] : 0.f;
-            const float p = vis ? ex2_t(fmaf(sv[2 * e + u], c, -ls)) : 0.f;
+            const float p = vis ? ex2_t(fmaf(sv[2 * e + u], c, -s_lse[cc])) : 0.f;
             p2[u] = p;
-            d2[u] = p * (dp[2 * e + u] - D);
+            d2[u] = p * (dp[2 * e + u] - s_D[cc]);
           }
           pk[e] = pack_bf16x2(p2[0], p2[1]);
           dk[e] = pack_bf16x2(d2[0], d2[1]);
