@@ -1027,8 +1027,9 @@ static onetrans_status launch_colsum(const float* src, const RowSet& s, int G, i
 }
 
 // Row chunks of a weight-gradient GEMM: enough (weight tile, chunk) CTAs to
-// fill two waves of 148 SMs, chunks a multiple of 64 rows.
-constexpr int kSplitCtas = 296;
+// fill one wave of 148 SMs (more chunks mean more partial gradients to add),
+// chunks a multiple of 64 rows.
+constexpr int kSplitCtas = 148;
 static void split_rows(int R, int N_out, int K_in, int& chunks, int& Kc) {
   const int tiles = (int)(cdiv(N_out, 128) * cdiv(K_in, 256));
   const int want = std::max(1, std::min(kSplitCtas / std::max(tiles, 1), (int)(pad64(R) / 64)));
