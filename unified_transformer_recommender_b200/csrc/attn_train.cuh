@@ -29,7 +29,7 @@ struct TrainAttnArgs {
   float* lse_out;        // forward: written
   const float* Dr;       // [B, H, Lq] dO . O per query row (dQ, dK/dV)
   __nv_bfloat16* o;      // forward: output rows [B, Lq, d]
-  float* dqkv;           // [B, L, 3d]: dq into the q columns, dk / dv into k / v
+  __nv_bfloat16* dqkv;   // [B, L, 3d]: dq into the q columns, dk / dv into k / v (bf16: the next GEMMs' operand)
 };
 
 struct TrainAttnCfg {
@@ -284,10 +284,11 @@ __global__ void __launch_bounds__(192, 1)
         for (int cc = 0; cc < C::DH / 32; ++cc) store_bf16x32(dst + cc * 32, o + cc * 32);
         a.lse_out[si] = (m + log2f(l)) * 0.6931471805599453f;
       } else {
-        float* dst = a.dqkv + ((long long)b * a.L + pos) * 3 * a.d + h * C::DH;
+        __nv_bfloat16* dst = a.dqkv + ((long long)b * a.L + pos) * 3 * a.d + h * C::DH;
 #pragma unroll
-        for (int e = 0; e < C::DH; e += 4)
-          *(float4*)(dst + e) = make_float4(o[e] * 0.125f, o[e + 1] * 0.125f, o[e + 2] * 0.125f, o[e + 3] * 0.125f);
+        for (int e = 0; e < C::DH; ++e) o[e] *= 0.125f;
+#pragma unroll
+        for (int cc = 0; cc < C::DH / 32; ++cc) store_bf16x32(dst + cc * 32, o + cc * 32);
       }
     }
   }
@@ -466,12 +467,13 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld32(tDK + lb + cc * 32, dkv + cc * 32);
     }
     if (ok && key_ok) {
-      float* dst = a.dqkv + ((long long)b * a.L + j) * 3 * a.d + h * C::DH;
+      __nv_bfloat16* dst = a.dqkv + ((long long)b * a.L + j) * 3 * a.d + h * C::DH;
 #pragma unroll
-      for (int e = 0; e < C::DH; e += 4) {
-        *(float4*)(dst + a.d + e) = make_float4(dkv[e] * 0.125f, dkv[e + 1] * 0.125f, dkv[e + 2] * 0.125f,
-                                                dkv[e + 3] * 0.125f);
-        *(float4*)(dst + 2 * a.d + e) = make_float4(dv[e], dv[e + 1], dv[e + 2], dv[e + 3]);
+      for (int e = 0; e < C::DH; ++e) dkv[e] *= 0.125f;
+#pragma unroll
+      for (int cc = 0; cc < C::DH / 32; ++cc) {
+        store_bf16x32(dst + a.d + cc * 32, dkv + cc * 32);
+        store_bf16x32(dst + 2 * a.d + cc * 32, dv + cc * 32);
       }
     }
   }
@@ -482,8 +484,8 @@ __global__ void __launch_bounds__(192, 1)
 
 // D = dO . O per (sample, head, query row): the row term of the softmax's
 // backward.  One thread per (row, head).
-__global__ void attn_train_delta_kernel(const float* __restrict__ dO, const __nv_bfloat16* __restrict__ O, float* Dr,
-                                        int B, int Lq, int H, int dh) {
+__global__ void attn_train_delta_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
+                                        float* Dr, int B, int Lq, int H, int dh) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)B * Lq * H) return;
   const int h = (int)(i % H);
@@ -491,7 +493,7 @@ __global__ void attn_train_delta_kernel(const float* __restrict__ dO, const __nv
   const int t = (int)(bt % Lq), b = (int)(bt / Lq);
   const long long off = bt * H * dh + (long long)h * dh;
   float acc = 0.f;
-  for (int e = 0; e < dh; ++e) acc = fmaf(dO[off + e], __bfloat162float(O[off + e]), acc);
+  for (int e = 0; e < dh; ++e) acc = fmaf(__bfloat162float(dO[off + e]), __bfloat162float(O[off + e]), acc);
   Dr[((long long)b * H + h) * Lq + t] = acc;
 }
 

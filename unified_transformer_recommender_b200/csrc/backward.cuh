@@ -116,14 +116,15 @@ __global__ void chunk_sum_kernel(const float* __restrict__ part, int chunks, lon
 // blockIdx.z (kColChunk rows) of group g's rows into part[g][chunk][c], 32
 // columns per CTA and 8 row lanes per column; chunk_sum_kernel adds the chunks.
 constexpr int kColChunk = 256;
-__global__ void __launch_bounds__(256) colsum_kernel(const float* __restrict__ src, RowSet s, int C,
+template <typename Ti>
+__global__ void __launch_bounds__(256) colsum_kernel(const Ti* __restrict__ src, RowSet s, int C,
                                                      float* __restrict__ part) {
   __shared__ float red[8][33];
   const int g = blockIdx.y, ch = blockIdx.z, tx = threadIdx.x & 31, ty = threadIdx.x >> 5, c = blockIdx.x * 32 + tx;
   const int r_end = min(s.R, (ch + 1) * kColChunk);
   float acc = 0.f;
   if (c < C)
-    for (int r = ch * kColChunk + ty; r < r_end; r += 8) acc += src[rowset_off(s, g, r) + c];
+    for (int r = ch * kColChunk + ty; r < r_end; r += 8) acc += to_f(src[rowset_off(s, g, r) + c]);
   red[ty][tx] = acc;
   __syncthreads();
   if (ty == 0 && c < C) {
@@ -142,7 +143,8 @@ template <typename Tx, typename T>
 __global__ void __launch_bounds__(256) rms_backward_kernel(const Tx* __restrict__ x, long long x_sb, long long x_st,
                                                            const T* __restrict__ gamma, const float* __restrict__ dy,
                                                            float* __restrict__ dx, long long dx_sb, long long dx_st,
-                                                           float* __restrict__ pg, int rows, int fold, int d, float eps) {
+                                                           float* __restrict__ pg, int rows, int fold, int d, float eps,
+                                                           T* __restrict__ dx_copy) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -163,39 +165,77 @@ __global__ void __launch_bounds__(256) rms_backward_kernel(const Tx* __restrict_
   const float r = rsqrtf(ss / d + eps);
   const float c3 = r * r * r * sg / d;
   float* dxr = dx + b * dx_sb + t * dx_st;
+  T* cpr = dx_copy ? dx_copy + b * dx_sb + t * dx_st : nullptr;
   float* pgr = pg + (long long)row * d;
   for (int k = lane; k < d; k += 32) {
     const float xv = to_f(xr[k]), g = to_f(gamma[k]), dv = dyr[k];
-    dxr[k] += r * g * dv - xv * c3;
+    const float v = dxr[k] + (r * g * dv - xv * c3);
+    dxr[k] = v;
+    if (cpr) cpr[k] = from_f<T>(v);   // the finished row, as the next GEMM's operand
     pgr[k] = dv * xv * r;
   }
 }
 
-// d/du of GELU-tanh: 0.5 (1 + tanh(v)) + 0.5 u (1 - tanh^2(v)) c (1 + 3 a u^2),
-// v = c (u + a u^3), c = sqrt(2/pi), a = 0.044715.
-__device__ inline float gelu_tanh_grad(float u) {
+// GELU-tanh and its derivative from one tanh: with v = c (u + a u^3),
+// c = sqrt(2/pi), a = 0.044715, GELU(u) = 0.5 u (1 + tanh v) and
+// d/du = 0.5 (1 + tanh v) + 0.5 u (1 - tanh^2 v) c (1 + 3 a u^2).
+__device__ inline void gelu_tanh_and_grad(float u, float& z, float& g) {
   const float c = 0.7978845608028654f, a = 0.044715f;
   const float th = tanh_fast(c * (u + a * u * u * u));   // MUFU tanh, relative error about 2^-11
-  return 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * a * u * u);
+  z = 0.5f * u * (1.f + th);
+  g = 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * a * u * u);
 }
 
-// z = GELU(u) in the storage type (the FFN's hidden layer, recomputed).
-template <typename T>
-__global__ void gelu_forward_kernel(const float* __restrict__ u, T* __restrict__ z, long long n) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) z[i] = from_f<T>(gelu_fast(u[i]));   // MUFU tanh, as the inference path's FFN
+template <typename T> __device__ inline void ld4(const T* p, float v[4]);
+template <> __device__ inline void ld4<float>(const float* p, float v[4]) {
+  const float4 q = *reinterpret_cast<const float4*>(p);
+  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+}
+template <> __device__ inline void ld4<__nv_bfloat16>(const __nv_bfloat16* p, float v[4]) {
+  const uint2 q = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+template <typename T> __device__ inline void st4(T* p, const float v[4]);
+template <> __device__ inline void st4<float>(float* p, const float v[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <> __device__ inline void st4<__nv_bfloat16>(__nv_bfloat16* p, const float v[4]) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 q;
+  q.x = *reinterpret_cast<const uint32_t*>(&a);
+  q.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = q;
 }
 
-// du = dz * GELU'(u): float32 (its column sums are db1) and the storage type
-// (the operand of the next GEMMs).
+// du = dz * GELU'(u) and z = GELU(u), both in the storage type (du: the
+// operand of the next GEMMs and the rows whose column sums are db1; z: the
+// activation operand of dW2).  Four elements per thread; the buffers start
+// 16-byte aligned, so every full group of four is a vector access.
 template <typename T>
-__global__ void gelu_backward_kernel(const float* __restrict__ dz, const float* __restrict__ u,
-                                     float* __restrict__ du32, T* __restrict__ du, long long n) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) {
-    const float v = dz[i] * gelu_tanh_grad(u[i]);
-    du32[i] = v;
-    du[i] = from_f<T>(v);
+__global__ void __launch_bounds__(256) gelu_backward_kernel(const float* __restrict__ dz, const T* __restrict__ u,
+                                                            T* __restrict__ du, T* __restrict__ z, long long n) {
+  const long long i0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i0 >= n) return;
+  if (i0 + 4 <= n) {
+    float uv[4], dv[4], zv[4], gv[4];
+    ld4<T>(u + i0, uv);
+    ld4<float>(dz + i0, dv);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      gelu_tanh_and_grad(uv[k], zv[k], gv[k]);
+      gv[k] *= dv[k];
+    }
+    st4<T>(du + i0, gv);
+    st4<T>(z + i0, zv);
+  } else {
+    for (long long i = i0; i < n; ++i) {
+      float zz, g;
+      gelu_tanh_and_grad(to_f(u[i]), zz, g);
+      du[i] = from_f<T>(dz[i] * g);
+      z[i] = from_f<T>(zz);
+    }
   }
 }
 
@@ -258,11 +298,12 @@ __global__ void __launch_bounds__(64) attn_rows_forward_kernel(AttnRows a, T* __
 }
 
 // Per query row: D = dO . O, then dQ = sum_j P_j (dO . v_j - D) k_j / sqrt(d_h)
-// with P_j = exp(q . k_j / sqrt(d_h) - lse).  dq goes to dqkv's q columns.
+// with P_j = exp(q . k_j / sqrt(d_h) - lse).  dO in the storage type; dq goes
+// to dqkv's q columns in the storage type (the operand of the next GEMMs).
 template <typename T, int DH>
-__global__ void __launch_bounds__(64) attn_rows_dq_kernel(AttnRows a, const float* __restrict__ dout,
+__global__ void __launch_bounds__(64) attn_rows_dq_kernel(AttnRows a, const T* __restrict__ dout,
                                                           const T* __restrict__ out, const float* __restrict__ lse,
-                                                          float* __restrict__ Dr, float* __restrict__ dqkv) {
+                                                          float* __restrict__ Dr, T* __restrict__ dqkv) {
   const int t = blockIdx.x * 64 + threadIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (t >= a.Lq) return;
   const T* qkv = (const T*)a.qkv;
@@ -275,7 +316,7 @@ __global__ void __launch_bounds__(64) attn_rows_dq_kernel(AttnRows a, const floa
 #pragma unroll
   for (int e = 0; e < DH; ++e) {
     q[e] = to_f(qr[e]) * isq;
-    g[e] = dout[ro + e];
+    g[e] = to_f(dout[ro + e]);
     D = fmaf(g[e], to_f(out[ro + e]), D);
     dq[e] = 0.f;
   }
@@ -295,17 +336,17 @@ __global__ void __launch_bounds__(64) attn_rows_dq_kernel(AttnRows a, const floa
 #pragma unroll
     for (int e = 0; e < DH; ++e) dq[e] = fmaf(ds, to_f(kr[e]), dq[e]);
   }
-  float* dst = dqkv + ((long long)b * a.L + p) * 3 * a.d + (long long)h * DH;
+  T* dst = dqkv + ((long long)b * a.L + p) * 3 * a.d + (long long)h * DH;
 #pragma unroll
-  for (int e = 0; e < DH; ++e) dst[e] = dq[e];
+  for (int e = 0; e < DH; ++e) dst[e] = from_f<T>(dq[e]);
 }
 
 // Per key row j: dV = sum_t P_tj dO_t, dK = sum_t P_tj (dO_t . v_j - D_t) q_t / sqrt(d_h)
 // over the queries t that see key j.  dk, dv go to dqkv's k and v columns.
 template <typename T, int DH>
-__global__ void __launch_bounds__(64) attn_rows_dkdv_kernel(AttnRows a, const float* __restrict__ dout,
+__global__ void __launch_bounds__(64) attn_rows_dkdv_kernel(AttnRows a, const T* __restrict__ dout,
                                                             const float* __restrict__ lse, const float* __restrict__ Dr,
-                                                            float* __restrict__ dqkv) {
+                                                            T* __restrict__ dqkv) {
   const int j = blockIdx.x * 64 + threadIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (j >= a.L) return;
   const T* qkv = (const T*)a.qkv;
@@ -323,27 +364,27 @@ __global__ void __launch_bounds__(64) attn_rows_dkdv_kernel(AttnRows a, const fl
   const int q0 = a.L - a.Lq;
   for (int t = max(0, j - q0); t < a.Lq; ++t) {
     const T* qr = qkv + qkv_off(a, b, q0 + t, 0, h, DH);
-    const float* gr = dout + ((long long)b * a.Lq + t) * a.d + (long long)h * DH;
+    const T* gr = dout + ((long long)b * a.Lq + t) * a.d + (long long)h * DH;
     float s = 0.f, dp = 0.f;
 #pragma unroll
     for (int e = 0; e < DH; ++e) {
       s = fmaf(to_f(qr[e]), k[e], s);
-      dp = fmaf(gr[e], v[e], dp);
+      dp = fmaf(to_f(gr[e]), v[e], dp);
     }
     const long long si = ((long long)b * a.H + h) * a.Lq + t;
     const float pr = __expf(s - lse[si]);
     const float ds = pr * (dp - Dr[si]) * isq;
 #pragma unroll
     for (int e = 0; e < DH; ++e) {
-      dv[e] = fmaf(pr, gr[e], dv[e]);
+      dv[e] = fmaf(pr, to_f(gr[e]), dv[e]);
       dk[e] = fmaf(ds, to_f(qr[e]), dk[e]);
     }
   }
-  float* dst = dqkv + ((long long)b * a.L + j) * 3 * a.d + (long long)h * DH;
+  T* dst = dqkv + ((long long)b * a.L + j) * 3 * a.d + (long long)h * DH;
 #pragma unroll
   for (int e = 0; e < DH; ++e) {
-    dst[a.d + e] = dk[e];
-    dst[2 * a.d + e] = dv[e];
+    dst[a.d + e] = from_f<T>(dk[e]);
+    dst[2 * a.d + e] = from_f<T>(dv[e]);
   }
 }
 

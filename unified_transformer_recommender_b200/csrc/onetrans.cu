@@ -1012,15 +1012,17 @@ static onetrans_status launch_chunk_sum(const float* part, int chunks, long long
   return last_launch();
 }
 
-// Column sums of G row sets into dst[g * dst_gs + c]: chunks of kColChunk
-// rows in parallel into `part` (workspace), then the chunks added in order.
-static onetrans_status launch_colsum(const float* src, const RowSet& s, int G, int C, float* dst, long long dst_gs,
+// Column sums of G row sets (float32 or storage-type rows) into
+// dst[g * dst_gs + c]: chunks of kColChunk rows in parallel into `part`
+// (workspace), then the chunks added in order.
+template <typename Ti>
+static onetrans_status launch_colsum(const Ti* src, const RowSet& s, int G, int C, float* dst, long long dst_gs,
                                      float* part, cudaStream_t st) {
   if (G <= 0 || C <= 0) return ONETRANS_OK;
   const int chunks = (int)std::max<long long>(1, cdiv(s.R, kColChunk));
   {
-    ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * (s.R + chunks) * 4.0, st);
-    colsum_kernel<<<dim3((unsigned)cdiv(C, 32), (unsigned)G, (unsigned)chunks), 256, 0, st>>>(src, s, C, part);
+    ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * (s.R * sizeof(Ti) + chunks * 4.0), st);
+    colsum_kernel<Ti><<<dim3((unsigned)cdiv(C, 32), (unsigned)G, (unsigned)chunks), 256, 0, st>>>(src, s, C, part);
     OT_TRY(last_launch());
   }
   return launch_chunk_sum(part, chunks, (long long)G * C, dst, dst_gs, C, st);
@@ -1060,12 +1062,12 @@ static onetrans_status mixed_rows_gemm(const onetrans_model* m, const void* A, l
                                        int a_rows, int B, int t_lo, int t_s, int t_hi, const void* W_S,
                                        const void* W_NS, int K, int N, RowMap out, cudaStream_t st,
                                        const void* bias_S = nullptr, const void* bias_NS = nullptr,
-                                       RowMap res = RowMap{}) {
+                                       RowMap res = RowMap{}, int act = ACT_NONE) {
   if (t_s > t_lo) {
     GemmDesc g = gdesc_base(m);
     g.mode = TILE_ROWS; g.M = t_s - t_lo; g.m_lo = t_lo; g.G = B; g.g_lo = 0;
     g.K = K; g.A = A; g.a_sm = a_row; g.a_sg = a_samp; g.a_mext = a_rows; g.a_gext = B;
-    g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S;
+    g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S; g.act = act;
     g.out = out; g.res = res;
     OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
   }
@@ -1074,7 +1076,7 @@ static onetrans_status mixed_rows_gemm(const onetrans_model* m, const void* A, l
     g.mode = TILE_SAMPLES; g.M = B; g.G = t_hi - t_s; g.g_lo = t_s; g.grp_base = t_s;
     g.K = K; g.A = A; g.a_sm = a_samp; g.a_sg = a_row; g.a_mext = B; g.a_gext = a_rows;
     g.W = W_NS; g.w_sg = (long long)N * K; g.w_rows = N; g.w_groups = t_hi - t_s; g.N = N;
-    g.bias = bias_NS; g.bias_sg = bias_NS ? N : 0;
+    g.bias = bias_NS; g.bias_sg = bias_NS ? N : 0; g.act = act;
     g.out = out; g.res = res;
     OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
   }
@@ -1155,9 +1157,10 @@ static onetrans_status weight_grad(const onetrans_model* m, GradRows Y, GradRows
   return ONETRANS_OK;
 }
 
-// Bias gradient: column sums of float32 rows, the S set over all its rows and
-// each NS set over its token's rows.
-static onetrans_status bias_grad(const float* rows, long long row, long long samp, int C, int B, int t_lo, int t_s,
+// Bias gradient: column sums of rows (float32 or the storage type), the S set
+// over all its rows and each NS set over its token's rows.
+template <typename Ti>
+static onetrans_status bias_grad(const Ti* rows, long long row, long long samp, int C, int B, int t_lo, int t_s,
                                  int t_hi, float* db_S, float* db_NS, float* part, cudaStream_t st) {
   if (t_s == t_lo && db_S) OT_TRY(cuda_ok(cudaMemsetAsync(db_S, 0, (size_t)C * 4, st)));
   if (t_s > t_lo && db_S)
@@ -1171,31 +1174,34 @@ static onetrans_status bias_grad(const float* rows, long long row, long long sam
 template <typename T, typename Tx>
 static onetrans_status launch_rms_backward(const void* x, long long x_sb, long long x_st, const void* gamma,
                                            const float* dy, float* dx, long long dx_sb, long long dx_st, float* pg,
-                                           int rows, int fold, int d, float eps, cudaStream_t st) {
+                                           int rows, int fold, int d, float eps, void* dx_copy, cudaStream_t st) {
   if (rows <= 0) return ONETRANS_OK;
-  ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)rows * d * (sizeof(Tx) + 4.0 + 8.0 + 4.0), st);
-  rms_backward_kernel<Tx, T><<<(unsigned)cdiv(rows, 8), 256, 0, st>>>((const Tx*)x, x_sb, x_st, (const T*)gamma, dy,
-                                                                      dx, dx_sb, dx_st, pg, rows, fold, d, eps);
+  ProfScope prof(PK_TRAIN_ELEM, 0.0,
+                 (double)rows * d * (sizeof(Tx) + 4.0 + 8.0 + 4.0 + (dx_copy ? sizeof(T) : 0)), st);
+  rms_backward_kernel<Tx, T><<<(unsigned)cdiv(rows, 8), 256, 0, st>>>(
+      (const Tx*)x, x_sb, x_st, (const T*)gamma, dy, dx, dx_sb, dx_st, pg, rows, fold, d, eps, (T*)dx_copy);
   return last_launch();
 }
 
 template <typename T>
 static onetrans_status launch_attn_rows(const onetrans_model* m, int stage, const AttnRows& a, void* out,
-                                        float* lse, const float* dout, float* Dr, float* dqkv, cudaStream_t st) {
+                                        float* lse, const void* dout, float* Dr, void* dqkv, cudaStream_t st) {
   const int dh = m->dh;
   // visible (query, key) pairs x heads; FLOPs per pair: forward 2 x 2 d_h (q.k, p v), dq 3 x 2 d_h,
   // dk,dv 4 x 2 d_h; bytes: the q|k|v rows read once, the outputs written once
   const double pairs = (double)a.B * a.H * ((double)a.Lq * (a.L - a.Lq) + 0.5 * (double)a.Lq * (a.Lq + 1));
   const double fl = pairs * 2.0 * dh * (stage == 0 ? 2 : stage == 1 ? 3 : 4);
-  ProfScope prof(PK_TRAIN_ATTN, fl, (double)a.B * a.L * 3 * a.d * m->es + (double)a.B * a.Lq * a.d * 4, st);
+  ProfScope prof(PK_TRAIN_ATTN, fl, (double)a.B * a.L * 3 * a.d * m->es + (double)a.B * a.Lq * a.d * m->es, st);
 #define OT_ATTN_ROWS(DH)                                                                                   \
   if (stage == 0) {                                                                                         \
     attn_rows_forward_kernel<T, DH><<<dim3((unsigned)cdiv(a.Lq, 64), a.H, a.B), 64, 0, st>>>(a, (T*)out, lse); \
   } else if (stage == 1) {                                                                                  \
-    attn_rows_dq_kernel<T, DH><<<dim3((unsigned)cdiv(a.Lq, 64), a.H, a.B), 64, 0, st>>>(a, dout, (const T*)out, \
-                                                                                         lse, Dr, dqkv);    \
+    attn_rows_dq_kernel<T, DH><<<dim3((unsigned)cdiv(a.Lq, 64), a.H, a.B), 64, 0, st>>>(a, (const T*)dout,    \
+                                                                                         (const T*)out, lse, Dr, \
+                                                                                         (T*)dqkv);         \
   } else {                                                                                                  \
-    attn_rows_dkdv_kernel<T, DH><<<dim3((unsigned)cdiv(a.L, 64), a.H, a.B), 64, 0, st>>>(a, dout, lse, Dr, dqkv); \
+    attn_rows_dkdv_kernel<T, DH><<<dim3((unsigned)cdiv(a.L, 64), a.H, a.B), 64, 0, st>>>(a, (const T*)dout, lse, Dr, \
+                                                                                         (T*)dqkv);         \
   }
   switch (dh) {
     case 16: OT_ATTN_ROWS(16) break;
@@ -1216,7 +1222,7 @@ static bool train_attn_tc(const onetrans_model* m) {
 }
 
 static onetrans_status launch_attn_train_tc(const onetrans_model* m, int stage, const AttnRows& ar, void* o,
-                                            float* lse, float* Dr, const void* dOb, float* dqkv, cudaStream_t st) {
+                                            float* lse, float* Dr, const void* dOb, void* dqkv, cudaStream_t st) {
   using C = TrainAttnCfg;
   const int d = ar.d;
   CUtensorMap tq, tdo;
@@ -1230,10 +1236,10 @@ static onetrans_status launch_attn_train_tc(const onetrans_model* m, int stage, 
   TrainAttnArgs ta;
   std::memset(&ta, 0, sizeof(ta));
   ta.B = ar.B; ta.L = ar.L; ta.Lq = ar.Lq; ta.H = ar.H; ta.d = d;
-  ta.lse = lse; ta.lse_out = lse; ta.Dr = Dr; ta.o = (__nv_bfloat16*)o; ta.dqkv = dqkv;
+  ta.lse = lse; ta.lse_out = lse; ta.Dr = Dr; ta.o = (__nv_bfloat16*)o; ta.dqkv = (__nv_bfloat16*)dqkv;
   const double pairs = (double)ar.B * ar.H * ((double)ar.Lq * (ar.L - ar.Lq) + 0.5 * (double)ar.Lq * (ar.Lq + 1));
   ProfScope prof(PK_TRAIN_ATTN, pairs * 2.0 * C::DH * (stage == 0 ? 2 : stage == 1 ? 3 : 4),
-                 (double)ar.B * ar.L * 3 * d * 2 + (double)ar.B * ar.Lq * d * 4, st);
+                 (double)ar.B * ar.L * 3 * d * 2 + (double)ar.B * ar.Lq * d * 2, st);
   static bool attr[3] = {false, false, false};
   if (!attr[stage]) {
     cudaError_t e = stage == 0 ? cudaFuncSetAttribute(attn_train_q_kernel<false>,
@@ -1281,17 +1287,16 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
   float* Dr = (float*)cv.take((size_t)B * H * Lq0 * 4);
   float* x1 = (float*)cv.take((size_t)B * Lq0 * d * 4);
   void* h2 = cv.take((size_t)B * Lq0 * d * es);
-  float* u = (float*)cv.take((size_t)B * Lq0 * dff * 4);
+  void* u = cv.take((size_t)B * Lq0 * dff * es);   // W1 h2 + b1, recomputed for the backward only
   void* z = cv.take((size_t)B * Lq0 * dff * es);
   float* gbuf[2] = {(float*)cv.take((size_t)B * L0 * d * 4), (float*)cv.take((size_t)B * L0 * d * 4)};
+  void* gT = cv.take((size_t)B * L0 * d * es);      // the current output gradient in the storage type
   float* dx1 = (float*)cv.take((size_t)B * Lq0 * d * 4);
-  void* rowT = cv.take((size_t)B * L0 * 3 * d * es);   // a float32 gradient cast to the storage type
+  void* dx1T = cv.take((size_t)B * Lq0 * d * es);
   float* dz = (float*)cv.take((size_t)B * Lq0 * dff * 4);
-  float* du32 = (float*)cv.take((size_t)B * Lq0 * dff * 4);
   void* du = cv.take((size_t)B * Lq0 * dff * es);
   float* dh2 = (float*)cv.take((size_t)B * Lq0 * d * 4);
-  float* da = (float*)cv.take((size_t)B * Lq0 * d * 4);
-  float* dqkv = (float*)cv.take((size_t)B * L0 * 3 * d * 4);
+  void* dqkv = cv.take((size_t)B * L0 * 3 * d * es);
   float* dh = (float*)cv.take((size_t)B * L0 * d * 4);
   float* pg = (float*)cv.take((size_t)B * L0 * d * 4);
   void* opA = cv.take((size_t)op_elems * es);
@@ -1317,8 +1322,10 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     return ONETRANS_OK;
   };
 
-  // recompute layer n's intermediates from its input x_in (L rows per sample)
-  auto recompute = [&](int n, const void* x_in, bool x_f32) -> onetrans_status {
+  // recompute layer n's intermediates from its input x_in (L rows per sample):
+  // the forward pass needs z = GELU(W1 h2 + b1), the backward the
+  // pre-activation u (z then comes out of the GELU backward)
+  auto recompute = [&](int n, const void* x_in, bool x_f32, bool fwd) -> onetrans_status {
     const int L = Ln[n], Lqn = Lq[n], s = L - L_NS, sq = Lqn - L_NS, off = L - Lqn;
     if (x_f32) OT_TRY(rms_flat<T>(m, x_in, true, h, (long long)B * L, m->g_attn[n], st));
     else OT_TRY(rms_flat<T>(m, x_in, false, h, (long long)B * L, m->g_attn[n], st));
@@ -1340,50 +1347,48 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     go.rms = rmap(h2, (long long)Lqn * d, d);
     go.gamma = m->g_ffn[n];
     OT_TRY(launch_gemm<T>(m, go, st, PK_TRAIN));
-    // u = W1 h2 + b1 (float32), z = GELU(u)
-    OT_TRY(mixed_rows_gemm<T>(m, h2, d, (long long)Lqn * d, Lqn, B, 0, sq, Lqn, m->W1_S[n], m->W1_NS[n], d, dff,
-                              rmap32(u, (long long)Lqn * dff, dff), st, m->b1_S[n], m->b1_NS[n]));
-    const long long nz = (long long)B * Lqn * dff;
-    ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + es), st);
-    gelu_forward_kernel<T><<<(unsigned)cdiv(nz, 256), 256, 0, st>>>(u, (T*)z, nz);
-    return last_launch();
+    return mixed_rows_gemm<T>(m, h2, d, (long long)Lqn * d, Lqn, B, 0, sq, Lqn, m->W1_S[n], m->W1_NS[n], d, dff,
+                              rmap(fwd ? z : u, (long long)Lqn * dff, dff), st, m->b1_S[n], m->b1_NS[n], RowMap{},
+                              fwd ? ACT_GELU : ACT_NONE);
   };
 
   // ---- forward, keeping each layer's input
   for (int n = 0; n < NL; ++n) {
     const int Lqn = Lq[n], sq = Lqn - L_NS;
-    OT_TRY(recompute(n, n == 0 ? x0 : (const void*)X[n], n > 0));
+    OT_TRY(recompute(n, n == 0 ? x0 : (const void*)X[n], n > 0, true));
     float* y = n + 1 == NL ? out : X[n + 1];
     OT_TRY(mixed_rows_gemm<T>(m, z, dff, (long long)Lqn * dff, Lqn, B, 0, sq, Lqn, m->W2_S[n], m->W2_NS[n], dff, d,
                               rmap32(y, (long long)Lqn * d, d), st, m->b2_S[n], m->b2_NS[n],
                               rmap32(x1, (long long)Lqn * d, d)));
   }
 
-  // ---- backward, layer by layer
+  // ---- backward, layer by layer; the gradient of each layer's output is
+  // kept in float32 (g_cur, for the residual and the bias sums) and in the
+  // storage type (gT, the GEMM operand)
   const float* g_cur = dy;   // gradient of layer n's output, [B, Lq[n], d]
+  OT_TRY(launch_cast<T>(dy, gT, (long long)B * Lq[NL - 1] * d, st));
   for (int n = NL - 1; n >= 0; --n) {
     const int L = Ln[n], Lqn = Lq[n], s = L - L_NS, sq = Lqn - L_NS, off = L - Lqn;
     const bool x_f32 = n > 0;
     const void* x_in = n == 0 ? x0 : (const void*)X[n];
     float* g_in = n == 0 ? dx0 : gbuf[n % 2];   // gradient of layer n's input, [B, L, d]
-    OT_TRY(recompute(n, x_in, x_f32));
+    OT_TRY(recompute(n, x_in, x_f32, false));
     const long long Md = (long long)Lqn * d, Mf = (long long)Lqn * dff;
     // y = x1 + W2 z + b2
     OT_TRY(bias_grad(g_cur, d, Md, d, B, 0, sq, Lqn, gr->b2_S[n], gr->b2_NS[n], col_part, st));
-    OT_TRY(weight_grad<T>(m, GradRows{g_cur, d, Md, true}, GradRows{z, dff, Mf, false}, d, dff, B, 0, sq, Lqn,
-                          gr->W2_S[n], gr->W2_NS[n], sc, st));
     void *wS, *wNS;
-    OT_TRY(launch_cast<T>(g_cur, rowT, (long long)B * Md, st));
     OT_TRY(weights_T(m->W2_S[n], m->W2_NS[n], d, dff, wS, wNS));
-    OT_TRY(mixed_rows_gemm<T>(m, rowT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap32(dz, Mf, dff), st));
+    OT_TRY(mixed_rows_gemm<T>(m, gT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap32(dz, Mf, dff), st));
     // z = GELU(u), u = W1 h2 + b1
     const long long nz = (long long)B * Mf;
     {
-      ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (12.0 + es), st);
-      gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 256), 256, 0, st>>>(dz, u, du32, (T*)du, nz);
+      ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + 3.0 * es), st);
+      gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 1024), 256, 0, st>>>(dz, (const T*)u, (T*)du, (T*)z, nz);
     }
     OT_TRY(last_launch());
-    OT_TRY(bias_grad(du32, dff, Mf, dff, B, 0, sq, Lqn, gr->b1_S[n], gr->b1_NS[n], col_part, st));
+    OT_TRY(weight_grad<T>(m, GradRows{gT, d, Md, false}, GradRows{z, dff, Mf, false}, d, dff, B, 0, sq, Lqn,
+                          gr->W2_S[n], gr->W2_NS[n], sc, st));
+    OT_TRY(bias_grad((const T*)du, dff, Mf, dff, B, 0, sq, Lqn, gr->b1_S[n], gr->b1_NS[n], col_part, st));
     OT_TRY(weight_grad<T>(m, GradRows{du, dff, Mf, false}, GradRows{h2, d, Md, false}, dff, d, B, 0, sq, Lqn,
                           gr->W1_S[n], gr->W1_NS[n], sc, st));
     OT_TRY(weights_T(m->W1_S[n], m->W1_NS[n], dff, d, wS, wNS));
@@ -1391,48 +1396,46 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     // h2 = RMSNorm(x1; g_ffn), x1 = x[tail] + W^O a
     OT_TRY(cuda_ok(cudaMemcpyAsync(dx1, g_cur, (size_t)B * Md * 4, cudaMemcpyDeviceToDevice, st)));
     OT_TRY((launch_rms_backward<T, float>(x1, Md, d, m->g_ffn[n], dh2, dx1, Md, d, pg, B * Lqn, Lqn, d,
-                                         m->cfg.rms_eps, st)));
+                                         m->cfg.rms_eps, dx1T, st)));
     OT_TRY(launch_colsum(pg, rowset(0, Md, d, Lqn, B * Lqn), 1, d, gr->g_ffn[n], 0, col_part, st));
-    OT_TRY(weight_grad<T>(m, GradRows{dx1, d, Md, true}, GradRows{a, d, Md, false}, d, d, B, 0, Lqn, Lqn,
+    OT_TRY(weight_grad<T>(m, GradRows{dx1T, d, Md, false}, GradRows{a, d, Md, false}, d, d, B, 0, Lqn, Lqn,
                           gr->Wo[n], nullptr, sc, st));
-    OT_TRY(launch_cast<T>(dx1, rowT, (long long)B * Md, st));
     OT_TRY(weights_T(m->Wo[n], nullptr, d, d, wS, wNS));
-    OT_TRY(mixed_rows_gemm<T>(m, rowT, d, Md, Lqn, B, 0, Lqn, Lqn, wS, nullptr, d, d, rmap32(da, Md, d), st));
+    OT_TRY(mixed_rows_gemm<T>(m, dx1T, d, Md, Lqn, B, 0, Lqn, Lqn, wS, nullptr, d, d, rmap(dOb, Md, d), st));
     // the residual: the tail rows of the input receive dx1, the others start at 0
     OT_TRY(cuda_ok(cudaMemsetAsync(g_in, 0, (size_t)B * L * d * 4, st)));
     OT_TRY(cuda_ok(cudaMemcpy2DAsync(g_in + (size_t)off * d, (size_t)L * d * 4, dx1, (size_t)Md * 4, (size_t)Md * 4,
                                      B, cudaMemcpyDeviceToDevice, st)));
     // attention: dq, dk, dv of the recomputed rows
-    OT_TRY(cuda_ok(cudaMemsetAsync(dqkv, 0, (size_t)B * L * 3 * d * 4, st)));
+    OT_TRY(cuda_ok(cudaMemsetAsync(dqkv, 0, (size_t)B * L * 3 * d * es, st)));
     AttnRows ar;
     ar.qkv = qkv; ar.B = B; ar.L = L; ar.Lq = Lqn; ar.H = H; ar.d = d;
     if (tc_attn) {
-      OT_TRY(launch_cast<T>(da, dOb, (long long)B * Md, st));
       const long long nd = (long long)B * Lqn * H;
-      attn_train_delta_kernel<<<(unsigned)cdiv(nd, 256), 256, 0, st>>>(da, (const __nv_bfloat16*)a, Dr, B, Lqn, H,
-                                                                        m->dh);
+      attn_train_delta_kernel<<<(unsigned)cdiv(nd, 256), 256, 0, st>>>((const __nv_bfloat16*)dOb,
+                                                                        (const __nv_bfloat16*)a, Dr, B, Lqn, H, m->dh);
       OT_TRY(last_launch());
       OT_TRY(launch_attn_train_tc(m, 1, ar, a, lse, Dr, dOb, dqkv, st));
       OT_TRY(launch_attn_train_tc(m, 2, ar, a, lse, Dr, dOb, dqkv, st));
     } else {
-      OT_TRY(launch_attn_rows<T>(m, 1, ar, a, lse, da, Dr, dqkv, st));
-      OT_TRY(launch_attn_rows<T>(m, 2, ar, a, lse, da, Dr, dqkv, st));
+      OT_TRY(launch_attn_rows<T>(m, 1, ar, a, lse, dOb, Dr, dqkv, st));
+      OT_TRY(launch_attn_rows<T>(m, 2, ar, a, lse, dOb, Dr, dqkv, st));
     }
     // (q, k, v) = W_i^{QKV} h_i
     const long long Mq = (long long)L * 3 * d;
-    OT_TRY(weight_grad<T>(m, GradRows{dqkv, 3 * d, Mq, true}, GradRows{h, d, (long long)L * d, false}, 3 * d, d,
+    OT_TRY(weight_grad<T>(m, GradRows{dqkv, 3 * d, Mq, false}, GradRows{h, d, (long long)L * d, false}, 3 * d, d,
                           B, 0, s, L, gr->Wqkv_S[n], gr->Wqkv_NS[n], sc, st));
-    OT_TRY(launch_cast<T>(dqkv, rowT, (long long)B * Mq, st));
     OT_TRY(weights_T(m->Wqkv_S[n], m->Wqkv_NS[n], 3 * d, d, wS, wNS));
-    OT_TRY(mixed_rows_gemm<T>(m, rowT, 3 * d, Mq, L, B, 0, s, L, wS, wNS, 3 * d, d,
+    OT_TRY(mixed_rows_gemm<T>(m, dqkv, 3 * d, Mq, L, B, 0, s, L, wS, wNS, 3 * d, d,
                               rmap32(dh, (long long)L * d, d), st));
-    // h = RMSNorm(x; g_attn)
+    // h = RMSNorm(x; g_attn); the lower layer's output gradient also as its GEMM operand
+    void* g_copy = n > 0 ? gT : nullptr;
     if (x_f32)
       OT_TRY((launch_rms_backward<T, float>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
-                                           B * L, L, d, m->cfg.rms_eps, st)));
+                                           B * L, L, d, m->cfg.rms_eps, g_copy, st)));
     else
       OT_TRY((launch_rms_backward<T, T>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
-                                       B * L, L, d, m->cfg.rms_eps, st)));
+                                       B * L, L, d, m->cfg.rms_eps, g_copy, st)));
     OT_TRY(launch_colsum(pg, rowset(0, (long long)L * d, d, L, B * L), 1, d, gr->g_attn[n], 0, col_part, st));
     g_cur = g_in;
   }
