@@ -57,23 +57,12 @@ def run_train(b, X0, dY):
     return to_np(out), to_np(dx0), {k: [to_np(t) for t in v] for k, v in grads.items()}
 
 
-@pytest.mark.parametrize("dtype,policy,d,pyr", [("bf16", 0, 256, True), ("bf16", 1, 256, True),
-                                                ("fp32", 0, 256, True), ("bf16", 0, 256, False),
-                                                ("fp32", 0, 32, False), ("bf16", 0, 384, True)])
-def test_forward_backward_matches_oracle(dtype, policy, d, pyr):
-    ot.onetrans_set_kernel_policy(policy)
-    if d == 32:
-        sh = shape(n_layers=2, d=32, H=2, dff=128, L_NS=4)
-    elif d == 384:
-        sh = shape(n_layers=2, d=384, dff=1536, L_NS=16)
-    else:
-        sh = shape(n_layers=2)
-    L_S = 100
-    sched = linear_pyramid(L_S + sh.L_NS, sh.L_NS, 2) if pyr else None
-    b = build(sh, 250, dtype, pyramid=sched, std=attn_std(d))
-    X0 = gen_normal(251, (2, L_S + sh.L_NS, sh.d), dtype)
+def check_train(dtype, sh, B, L_S, pyr, seed):
+    sched = linear_pyramid(L_S + sh.L_NS, sh.L_NS, sh.n_layers) if pyr else None
+    b = build(sh, seed, dtype, pyramid=sched, std=attn_std(sh.d))
+    X0 = gen_normal(seed + 1, (B, L_S + sh.L_NS, sh.d), dtype)
     n_out = sched[-1] if pyr else L_S + sh.L_NS
-    dY = gen_normal(252, (2, n_out, sh.d), "fp32")
+    dY = gen_normal(seed + 2, (B, n_out, sh.d), "fp32")
     out, dx0, grads = run_train(b, X0, dY)
     Y, dX, dW = O.forward_backward(X0, b.W, sh.L_NS, sh.n_heads, EPS, sched, dY)
     assert rel_err(out, Y) <= TOL[dtype]
@@ -87,3 +76,25 @@ def test_forward_backward_matches_oracle(dtype, policy, d, pyr):
             errs[f"{k}[{l}]"] = grad_err(grads[k][l], dW[k][l], dtype)
     bad = {k: e for k, e in errs.items() if not e <= TOL[dtype]}
     assert not bad, (bad, errs)
+
+
+@pytest.mark.parametrize("dtype,policy,d,pyr", [("bf16", 0, 256, True), ("bf16", 1, 256, True),
+                                                ("fp32", 0, 256, True), ("bf16", 0, 256, False),
+                                                ("fp32", 0, 32, False), ("bf16", 0, 384, True)])
+def test_forward_backward_matches_oracle(dtype, policy, d, pyr):
+    ot.onetrans_set_kernel_policy(policy)
+    if d == 32:
+        sh = shape(n_layers=2, d=32, H=2, dff=128, L_NS=4)
+    elif d == 384:
+        sh = shape(n_layers=2, d=384, dff=1536, L_NS=16)
+    else:
+        sh = shape(n_layers=2)
+    check_train(dtype, sh, 2, 100, pyr, 250)
+
+
+def test_forward_backward_many_samples():
+    """66 samples of 70 S tokens: the weight gradients' row tiles span
+    several samples, the S set splits into many slices (partial gradients
+    added afterwards) and each NS set's rows (one per sample) fill one tile of
+    64 and part of a second."""
+    check_train("bf16", shape(n_layers=2, dff=512), 66, 70, False, 253)

@@ -19,6 +19,7 @@
 #include "ffn_tc.cuh"
 #include "backward.cuh"
 #include "attn_train.cuh"
+#include "gemm_wgrad.cuh"
 
 using namespace ot;
 
@@ -1101,10 +1102,68 @@ struct TrainScratch {
   float *split_part, *col_part;
 };
 
+// The same on the tensor cores straight from the row-major storage-type rows
+// (no transposed copies): the S set's row tiles split into slices that fill
+// one wave of CTAs, their partial gradients added in slice order; one slice
+// per NS set.
+static onetrans_status weight_grad_rows(GradRows Y, GradRows X, int N_out, int K_in, int B, int t_lo, int t_s,
+                                        int t_hi, float* dW_S, float* dW_NS, const TrainScratch& sc,
+                                        cudaStream_t st) {
+  const int es = 2;
+  const int tiles = (K_in / wgrad_pick_bn(K_in)) * (N_out / 128);
+  if (t_s == t_lo && dW_S) OT_TRY(cuda_ok(cudaMemsetAsync(dW_S, 0, (size_t)N_out * K_in * 4, st)));
+  if (t_s > t_lo && dW_S) {
+    const int Tn = t_s - t_lo;
+    WgradArgs wa;
+    wa.TC = (int)cdiv(Tn, 64);
+    wa.total = B * wa.TC;
+    const int want = std::max(1, std::min(kSplitCtas / std::max(tiles, 1), wa.total));
+    wa.per = (int)cdiv(wa.total, want);
+    const int Z = (int)cdiv(wa.total, wa.per);
+    CUtensorMap tY, tX, tO;
+    float* out = Z > 1 ? sc.split_part : dW_S;
+    int swx = 0;
+    if (!wgrad_rows_tmap(&tY, (const char*)Y.p + (size_t)t_lo * Y.row * es, N_out, Tn, B, Y.row, Y.samp, wa.swap) ||
+        !wgrad_rows_tmap(&tX, (const char*)X.p + (size_t)t_lo * X.row * es, K_in, Tn, B, X.row, X.samp, swx) ||
+        swx != wa.swap || !wgrad_out_tmap(&tO, out, N_out, K_in, Z))
+      return ONETRANS_ERR_CUDA;
+    {
+      ProfScope prof(PK_TRAIN, 2.0 * B * Tn * N_out * K_in, (double)B * Tn * (N_out + K_in) * es +
+                     (double)Z * N_out * K_in * 4, st);
+      OT_TRY(wgrad_launch(tY, tX, tO, N_out, K_in, Z, wa, st));
+    }
+    if (Z > 1) {
+      const long long n = (long long)N_out * K_in;
+      OT_TRY(launch_chunk_sum(sc.split_part, Z, n, dW_S, 0, n, st));
+    }
+  }
+  if (t_hi > t_s && dW_NS) {
+    const int G = t_hi - t_s;
+    WgradArgs wa;
+    wa.TC = (int)cdiv(B, 64);
+    wa.per = wa.TC;
+    wa.total = G * wa.TC;
+    CUtensorMap tY, tX, tO;
+    int swx = 0;
+    if (!wgrad_rows_tmap(&tY, (const char*)Y.p + (size_t)t_s * Y.row * es, N_out, B, G, Y.samp, Y.row, wa.swap) ||
+        !wgrad_rows_tmap(&tX, (const char*)X.p + (size_t)t_s * X.row * es, K_in, B, G, X.samp, X.row, swx) ||
+        swx != wa.swap || !wgrad_out_tmap(&tO, dW_NS, N_out, K_in, G))
+      return ONETRANS_ERR_CUDA;
+    ProfScope prof(PK_TRAIN, 2.0 * B * G * N_out * K_in, (double)B * G * (N_out + K_in) * es +
+                   (double)G * N_out * K_in * 4, st);
+    OT_TRY(wgrad_launch(tY, tX, tO, N_out, K_in, G, wa, st));
+  }
+  return ONETRANS_OK;
+}
+
 template <typename T>
 static onetrans_status weight_grad(const onetrans_model* m, GradRows Y, GradRows X, int N_out, int K_in, int B,
                                    int t_lo, int t_s, int t_hi, float* dW_S, float* dW_NS, const TrainScratch& sc,
                                    cudaStream_t st) {
+  if (m->bf16 && g_policy == 0 && !Y.f32 && !X.f32 && wgrad_supported(N_out, K_in) && encode_fn() &&
+      (uintptr_t)Y.p % 16 == 0 && (uintptr_t)X.p % 16 == 0 && Y.row % 8 == 0 && Y.samp % 8 == 0 &&
+      X.row % 8 == 0 && X.samp % 8 == 0)
+    return weight_grad_rows(Y, X, N_out, K_in, B, t_lo, t_s, t_hi, dW_S, dW_NS, sc, st);
   void *opA = sc.opA, *opW = sc.opW;
   const int es = m->es;
   auto transpose = [&](const GradRows& s, const RowSet& rs, int G, int C, void* dst, int R_pad, int Kc) {
