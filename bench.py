@@ -204,8 +204,9 @@ def train_config(U: int, ws: int) -> dict:
     sh = wl.shape
     return {"workload": f"train: the s_forward model ({sh.n_layers} layers d={sh.d} {sh.n_heads} heads FFN "
                         f"{sh.d_ff}, pyramid {wl.pyramid[0]}->{wl.pyramid[-1]}), {U} samples x ({wl.L_S} S + "
-                        f"{sh.L_NS} NS tokens): forward keeping each layer's input, backward with every layer "
-                        "recomputed; bf16 operands, float32 gradients of the input and of every weight",
+                        f"{sh.L_NS} NS tokens): forward keeping each layer's input, attention output and "
+                        "log-sum-exp, backward with the rest of each layer recomputed; bf16 operands, float32 "
+                        "gradients of the input and of every weight",
             "samples_per_gpu": U, "parallelism": f"samples sharded over {ws} GPU(s), no collective",
             "l2": "512 MB buffer written between timed steps (not timed)"}
 

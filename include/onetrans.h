@@ -353,8 +353,12 @@ ONETRANS_API onetrans_status onetrans_forward(const onetrans_model* m, const voi
  * time and memory with mixed precision and activation recomputation: [FR]
  * 7.5.3 system optimizations; paper-daily 4.3, the "+ mixed precision +
  * recomputation" row).  Forward over x0 [B, L_S + L_NS, d] (the mode's
- * type) keeping only each layer's input, then the backward layer by layer,
- * each layer's intermediates recomputed from its input.  The loss gradient
+ * type) keeping each layer's input and its attention output and
+ * log-sum-exp (O(L) per layer), then the backward layer by layer with the
+ * rest of each layer's intermediates (the normalised rows, q | k | v, the
+ * residual sum and the FFN pre-activation) recomputed from its input: a
+ * selective recomputation that skips the attention's second forward.  The
+ * loss gradient
  * enters as dy [B, L'_N, d] float32, the gradient of the output out
  * [B, L'_N, d] float32 (the rows onetrans_forward returns).  Writes out,
  * dx0 [B, L_S + L_NS, d] float32 (gradient of x0) and every weight gradient

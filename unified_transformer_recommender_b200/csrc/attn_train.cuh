@@ -482,19 +482,37 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 5) tmem_dealloc(tmem, 512);
 }
 
-// D = dO . O per (sample, head, query row): the row term of the softmax's
-// backward.  One thread per (row, head).
-__global__ void attn_train_delta_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
-                                        float* Dr, int B, int Lq, int H, int dh) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (long long)B * Lq * H) return;
-  const int h = (int)(i % H);
-  const long long bt = i / H;
-  const int t = (int)(bt % Lq), b = (int)(bt / Lq);
-  const long long off = bt * H * dh + (long long)h * dh;
-  float acc = 0.f;
-  for (int e = 0; e < dh; ++e) acc = fmaf(__bfloat162float(dO[off + e]), __bfloat162float(O[off + e]), acc);
-  Dr[((long long)b * H + h) * Lq + t] = acc;
+// D[b][h][t] = sum over e of dO[b, t, h, e] O[b, t, h, e] (d_h = 64): one
+// warp per row (b, t), each lane eight consecutive elements of dO and O (one
+// 16-byte load each), the eight lanes of a head added by shuffles.
+__global__ void __launch_bounds__(256) attn_train_delta_kernel(const __nv_bfloat16* __restrict__ dO,
+                                                               const __nv_bfloat16* __restrict__ O,
+                                                               float* __restrict__ Dr, int B, int Lq, int H) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= (long long)B * Lq) return;
+  const int d = H * 64;
+  const int b = (int)(row / Lq), t = (int)(row - (long long)b * Lq);
+  for (int base = 0; base < d; base += 256) {   // the same trip count in every lane
+    const int e0 = base + 8 * lane;
+    float acc = 0.f;
+    if (e0 < d) {
+      const uint4 a = *(const uint4*)(dO + row * d + e0);
+      const uint4 o = *(const uint4*)(O + row * d + e0);
+      const __nv_bfloat162* ah = (const __nv_bfloat162*)&a;
+      const __nv_bfloat162* oh = (const __nv_bfloat162*)&o;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 x = __bfloat1622float2(ah[j]), y = __bfloat1622float2(oh[j]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    if ((lane & 7) == 0 && e0 < d) Dr[((long long)b * H + e0 / 64) * Lq + t] = acc;
+  }
 }
 
 }  // namespace ot

@@ -1,11 +1,13 @@
 // Kernels of the training path: the backward pass of the block stack with
-// activation recomputation.  The contractions themselves run on the GEMM
-// kernels of the forward path (tcgen05 where the shape allows); these
-// kernels supply what the forward kernels do not: operand transposes (the
-// backward's GEMMs contract over rows, so their operands are the forward's
-// rows transposed, K-major, zero-padded to a multiple of 64 rows), column
-// sums (bias and gain gradients), the RMSNorm and GELU backward steps, and
-// attention forward / backward on rows recomputed from the layer input.
+// activation recomputation.  The contractions run on the GEMM kernels of
+// the forward path and, for the weight gradients, on the row-major
+// weight-gradient GEMM (tcgen05 where the shape allows); these kernels supply
+// the rest: operand transposes for the GEMMs that the tensor-core kernels do
+// not take (K-major, zero-padded to a multiple of 64 rows), column sums (bias
+// and gain gradients, two passes in a fixed order), the RMSNorm and GELU
+// backward steps (with the gain and shared-bias column sums folded in), and
+// attention forward / backward on CUDA cores for head widths the tensor-core
+// training attention does not take.
 #pragma once
 #include "tc_ptx.cuh"
 
@@ -22,6 +24,32 @@ __device__ inline long long rowset_off(const RowSet& s, int g, int r) {
   const int b = r / s.T, t = r - b * s.T;
   return (long long)g * s.gs + (long long)b * s.sb + (long long)t * s.st;
 }
+
+// Four consecutive elements as one vector access (16 bytes of float32, 8 of
+// bf16; the caller keeps the address aligned to that).
+template <typename T> __device__ inline void ld4(const T* p, float v[4]);
+template <> __device__ inline void ld4<float>(const float* p, float v[4]) {
+  const float4 q = *reinterpret_cast<const float4*>(p);
+  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+}
+template <> __device__ inline void ld4<__nv_bfloat16>(const __nv_bfloat16* p, float v[4]) {
+  const uint2 q = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+template <typename T> __device__ inline void st4(T* p, const float v[4]);
+template <> __device__ inline void st4<float>(float* p, const float v[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <> __device__ inline void st4<__nv_bfloat16>(__nv_bfloat16* p, const float v[4]) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 q;
+  q.x = *reinterpret_cast<const uint32_t*>(&a);
+  q.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = q;
+}
+
 
 // The K-major operand of a GEMM that contracts over rows: row r of group g,
 // column c goes to dst[g][r / Kc][c][r % Kc] (R_pad = chunks x Kc; 0 for
@@ -102,14 +130,27 @@ __global__ void __launch_bounds__(256) transpose_rows_kernel(const Ti* __restric
   }
 }
 
-// out[i] = sum over the chunks k of part[k * n + i], in chunk order.
-__global__ void chunk_sum_kernel(const float* __restrict__ part, int chunks, long long n, float* __restrict__ out,
-                                 long long out_stride, long long n_inner) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
+// out[(i / n_inner) * out_stride + i % n_inner] = sum over the chunks k of
+// part[k * n + i]: 32 outputs per CTA, warp w adding chunks w, w + 8, ...,
+// the eight warp sums then added in warp order (a fixed order: the result
+// does not depend on timing).
+__global__ void __launch_bounds__(256) chunk_sum_kernel(const float* __restrict__ part, int chunks, long long n,
+                                                        float* __restrict__ out, long long out_stride,
+                                                        long long n_inner) {
+  __shared__ float red[8][33];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const long long i = (long long)blockIdx.x * 32 + lane;
   float acc = 0.f;
-  for (int k = 0; k < chunks; ++k) acc += part[(long long)k * n + i];
-  out[(i / n_inner) * out_stride + i % n_inner] = acc;
+  if (i < n)
+    for (int k = w; k < chunks; k += 8) acc += part[(long long)k * n + i];
+  red[w][lane] = acc;
+  __syncthreads();
+  if (w == 0 && i < n) {
+    float t = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t += red[q][lane];
+    out[(i / n_inner) * out_stride + i % n_inner] = t;
+  }
 }
 
 // Column sums in two passes with a fixed order: this kernel sums chunk
@@ -132,6 +173,35 @@ __global__ void __launch_bounds__(256) colsum_kernel(const Ti* __restrict__ src,
 #pragma unroll
     for (int i = 0; i < 8; ++i) t += red[i][tx];
     part[((long long)ch * gridDim.y + g) * C + c] = t;
+  }
+}
+
+// The same, four columns per thread (one vector load per row): 128 columns
+// per CTA.  Needs C % 4 == 0, strides % 4 == 0 and a vector-aligned base.
+template <typename Ti>
+__global__ void __launch_bounds__(256) colsum4_kernel(const Ti* __restrict__ src, RowSet s, int C,
+                                                      float* __restrict__ part) {
+  __shared__ float red[8][129];
+  const int g = blockIdx.y, ch = blockIdx.z, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = blockIdx.x * 128 + 4 * lane;
+  const int r_end = min(s.R, (ch + 1) * kColChunk);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (c < C)
+    for (int r = ch * kColChunk + w; r < r_end; r += 8) {
+      float v[4];
+      ld4<Ti>(src + rowset_off(s, g, r) + c, v);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] += v[j];
+    }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) red[w][4 * lane + j] = acc[j];
+  __syncthreads();
+  const int cc = blockIdx.x * 128 + threadIdx.x;
+  if (threadIdx.x < 128 && cc < C) {
+    float t = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t += red[q][threadIdx.x];
+    part[((long long)ch * gridDim.y + g) * C + cc] = t;
   }
 }
 
@@ -176,6 +246,79 @@ __global__ void __launch_bounds__(256) rms_backward_kernel(const Tx* __restrict_
   }
 }
 
+// The same with the gain gradient folded in: warp w of CTA k takes rows
+// k*8 + w, then every (gridDim.x * 8)-th row after it; lane l the columns
+// 4l .. 4l+3 of every 128 (d = 128 NC4), as vector accesses.  The CTA's sums
+// of dy x r leave as one partial row part[k][d], the warps added in warp
+// order (chunk_sum_kernel then adds the CTAs' rows in CTA order).  Needs the
+// row strides % 4 == 0 and vector-aligned bases.
+template <typename Tx, typename T, int NC4>
+__global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restrict__ x, long long x_sb, long long x_st,
+                                                              const T* __restrict__ gamma,
+                                                              const float* __restrict__ dy, float* __restrict__ dx,
+                                                              long long dx_sb, long long dx_st, float* __restrict__ part,
+                                                              int rows, int fold, float eps, T* __restrict__ dx_copy) {
+  constexpr int d = 128 * NC4;
+  __shared__ float red[8][d];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  float gm[NC4][4], pg[NC4][4];
+#pragma unroll
+  for (int i = 0; i < NC4; ++i) {
+    ld4<T>(gamma + 128 * i + 4 * lane, gm[i]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) pg[i][j] = 0.f;
+  }
+  for (int row = blockIdx.x * 8 + w; row < rows; row += gridDim.x * 8) {
+    const int b = row / fold, t = row - b * fold;
+    const Tx* xr = x + b * x_sb + t * x_st;
+    const float* dyr = dy + (long long)row * d;
+    float xv[NC4][4], dv[NC4][4];
+    float ss = 0.f, sg = 0.f;
+#pragma unroll
+    for (int i = 0; i < NC4; ++i) {
+      ld4<Tx>(xr + 128 * i + 4 * lane, xv[i]);
+      ld4<float>(dyr + 128 * i + 4 * lane, dv[i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        ss = fmaf(xv[i][j], xv[i][j], ss);
+        sg = fmaf(gm[i][j] * dv[i][j], xv[i][j], sg);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      sg += __shfl_xor_sync(0xffffffffu, sg, o);
+    }
+    const float r = rsqrtf(ss / d + eps);
+    const float c3 = r * r * r * sg / d;
+    float* dxr = dx + b * dx_sb + t * dx_st;
+    T* cpr = dx_copy ? dx_copy + b * dx_sb + t * dx_st : nullptr;
+#pragma unroll
+    for (int i = 0; i < NC4; ++i) {
+      float o[4];
+      ld4<float>(dxr + 128 * i + 4 * lane, o);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        o[j] += r * gm[i][j] * dv[i][j] - xv[i][j] * c3;
+        pg[i][j] = fmaf(dv[i][j], xv[i][j] * r, pg[i][j]);
+      }
+      st4<float>(dxr + 128 * i + 4 * lane, o);
+      if (cpr) st4<T>(cpr + 128 * i + 4 * lane, o);   // the finished row, as the next GEMM's operand
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NC4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) red[w][128 * i + 4 * lane + j] = pg[i][j];
+  __syncthreads();
+  for (int c = threadIdx.x; c < d; c += 256) {
+    float t = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t += red[q][c];
+    part[(long long)blockIdx.x * d + c] = t;
+  }
+}
+
 // GELU-tanh and its derivative from one tanh: with v = c (u + a u^3),
 // c = sqrt(2/pi), a = 0.044715, GELU(u) = 0.5 u (1 + tanh v) and
 // d/du = 0.5 (1 + tanh v) + 0.5 u (1 - tanh^2 v) c (1 + 3 a u^2).
@@ -184,29 +327,6 @@ __device__ inline void gelu_tanh_and_grad(float u, float& z, float& g) {
   const float th = tanh_fast(c * (u + a * u * u * u));   // MUFU tanh, relative error about 2^-11
   z = 0.5f * u * (1.f + th);
   g = 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * a * u * u);
-}
-
-template <typename T> __device__ inline void ld4(const T* p, float v[4]);
-template <> __device__ inline void ld4<float>(const float* p, float v[4]) {
-  const float4 q = *reinterpret_cast<const float4*>(p);
-  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-}
-template <> __device__ inline void ld4<__nv_bfloat16>(const __nv_bfloat16* p, float v[4]) {
-  const uint2 q = *reinterpret_cast<const uint2*>(p);
-  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
-  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
-  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-}
-template <typename T> __device__ inline void st4(T* p, const float v[4]);
-template <> __device__ inline void st4<float>(float* p, const float v[4]) {
-  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-}
-template <> __device__ inline void st4<__nv_bfloat16>(__nv_bfloat16* p, const float v[4]) {
-  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
-  uint2 q;
-  q.x = *reinterpret_cast<const uint32_t*>(&a);
-  q.y = *reinterpret_cast<const uint32_t*>(&b);
-  *reinterpret_cast<uint2*>(p) = q;
 }
 
 // du = dz * GELU'(u) and z = GELU(u), both in the storage type (du: the
@@ -236,6 +356,52 @@ __global__ void __launch_bounds__(256) gelu_backward_kernel(const float* __restr
       du[i] = from_f<T>(dz[i] * g);
       z[i] = from_f<T>(zz);
     }
+  }
+}
+
+// The same over whole rows of dff columns with the column sums of du over
+// the S rows folded in (the gradient of the shared set's b1): CTA k takes
+// rows [k*rows_per, (k+1)*rows_per) of the B x Lq rows (row t of a sample is
+// an S row for t < sq), thread i the columns 4i .. 4i+3 of every 1024
+// (dff <= 1024 J, dff % 4 == 0); the sums (of du before its rounding to the
+// storage type) leave as part[k][dff].
+template <typename T, int J>
+__global__ void __launch_bounds__(256) gelu_backward_bias_kernel(const float* __restrict__ dz,
+                                                                 const T* __restrict__ u, T* __restrict__ du,
+                                                                 T* __restrict__ z, int rows, int Lq, int sq, int dff,
+                                                                 int rows_per, float* __restrict__ part) {
+  float acc[J][4];
+#pragma unroll
+  for (int j = 0; j < J; ++j)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
+  const int r0 = blockIdx.x * rows_per, r1 = min(rows, r0 + rows_per);
+#pragma unroll 2
+  for (int r = r0; r < r1; ++r) {
+    const bool s_row = (r % Lq) < sq;
+    const long long base = (long long)r * dff;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int c = 1024 * j + 4 * threadIdx.x;
+      if (c < dff) {
+        float uv[4], dv[4], zv[4], gv[4];
+        ld4<T>(u + base + c, uv);
+        ld4<float>(dz + base + c, dv);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gelu_tanh_and_grad(uv[q], zv[q], gv[q]);
+          gv[q] *= dv[q];
+          if (s_row) acc[j][q] += gv[q];
+        }
+        st4<T>(du + base + c, gv);
+        st4<T>(z + base + c, zv);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int c = 1024 * j + 4 * threadIdx.x;
+    if (c < dff) st4<float>(part + (long long)blockIdx.x * dff + c, acc[j]);
   }
 }
 

@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -1009,8 +1010,19 @@ static onetrans_status launch_chunk_sum(const float* part, int chunks, long long
                                         long long n_inner, cudaStream_t st) {
   if (n <= 0) return ONETRANS_OK;
   ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)n * (chunks + 1) * 4.0, st);
-  chunk_sum_kernel<<<(unsigned)cdiv(n, 256), 256, 0, st>>>(part, chunks, n, out, out_stride, n_inner);
+  chunk_sum_kernel<<<(unsigned)cdiv(n, 32), 256, 0, st>>>(part, chunks, n, out, out_stride, n_inner);
   return last_launch();
+}
+
+// CTAs of the row-parallel reductions that leave one partial row per CTA
+// (gain and bias gradients): four per SM of a 148-SM part.
+constexpr int kRedCtas = 4 * 148;
+
+static bool vec4_ok(const void* p, size_t align, std::initializer_list<long long> strides) {
+  if ((uintptr_t)p % align) return false;
+  for (long long v : strides)
+    if (v % 4) return false;
+  return true;
 }
 
 // Column sums of G row sets (float32 or storage-type rows) into
@@ -1023,7 +1035,11 @@ static onetrans_status launch_colsum(const Ti* src, const RowSet& s, int G, int 
   const int chunks = (int)std::max<long long>(1, cdiv(s.R, kColChunk));
   {
     ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)G * C * (s.R * sizeof(Ti) + chunks * 4.0), st);
-    colsum_kernel<Ti><<<dim3((unsigned)cdiv(C, 32), (unsigned)G, (unsigned)chunks), 256, 0, st>>>(src, s, C, part);
+    if (C % 4 == 0 && vec4_ok(src, 4 * sizeof(Ti), {s.gs, s.sb, s.st}))
+      colsum4_kernel<Ti><<<dim3((unsigned)cdiv(C, 128), (unsigned)G, (unsigned)chunks), 256, 0, st>>>(src, s, C,
+                                                                                                      part);
+    else
+      colsum_kernel<Ti><<<dim3((unsigned)cdiv(C, 32), (unsigned)G, (unsigned)chunks), 256, 0, st>>>(src, s, C, part);
     OT_TRY(last_launch());
   }
   return launch_chunk_sum(part, chunks, (long long)G * C, dst, dst_gs, C, st);
@@ -1230,16 +1246,49 @@ static onetrans_status bias_grad(const Ti* rows, long long row, long long samp, 
   return ONETRANS_OK;
 }
 
+// RMSNorm backward of `rows` rows (dx += ..., optional storage-type copy of
+// each finished dx row) and the gain gradient dg = sum over the rows of
+// dy x r: folded into the row kernel (one partial row per CTA, added in CTA
+// order) where d is a multiple of 128 up to 512 and the rows allow vector
+// access, else through per-row products and column sums.
 template <typename T, typename Tx>
 static onetrans_status launch_rms_backward(const void* x, long long x_sb, long long x_st, const void* gamma,
                                            const float* dy, float* dx, long long dx_sb, long long dx_st, float* pg,
-                                           int rows, int fold, int d, float eps, void* dx_copy, cudaStream_t st) {
-  if (rows <= 0) return ONETRANS_OK;
-  ProfScope prof(PK_TRAIN_ELEM, 0.0,
-                 (double)rows * d * (sizeof(Tx) + 4.0 + 8.0 + 4.0 + (dx_copy ? sizeof(T) : 0)), st);
-  rms_backward_kernel<Tx, T><<<(unsigned)cdiv(rows, 8), 256, 0, st>>>(
-      (const Tx*)x, x_sb, x_st, (const T*)gamma, dy, dx, dx_sb, dx_st, pg, rows, fold, d, eps, (T*)dx_copy);
-  return last_launch();
+                                           int rows, int fold, int d, float eps, void* dx_copy, float* dg,
+                                           float* part, cudaStream_t st) {
+  if (rows <= 0) return dg ? cuda_ok(cudaMemsetAsync(dg, 0, (size_t)d * 4, st)) : ONETRANS_OK;
+  const bool fused = d % 128 == 0 && d <= 512 && vec4_ok(x, 4 * sizeof(Tx), {x_sb, x_st}) &&
+                     vec4_ok(dx, 16, {dx_sb, dx_st}) && vec4_ok(dy, 16, {}) && vec4_ok(gamma, 4 * sizeof(T), {}) &&
+                     vec4_ok(dx_copy, 4 * sizeof(T), {});
+  if (fused) {
+    const int ctas = (int)std::min<long long>(cdiv(rows, 8), kRedCtas);
+    {
+      ProfScope prof(PK_TRAIN_ELEM, 0.0,
+                     (double)rows * d * (sizeof(Tx) + 4.0 + 8.0 + (dx_copy ? sizeof(T) : 0)) + (double)ctas * d * 4,
+                     st);
+#define OT_RMS_DG(NC4)                                                                                             \
+  rms_backward_dg_kernel<Tx, T, NC4><<<(unsigned)ctas, 256, 0, st>>>((const Tx*)x, x_sb, x_st, (const T*)gamma, dy, \
+                                                                    dx, dx_sb, dx_st, part, rows, fold, eps,       \
+                                                                    (T*)dx_copy)
+      switch (d / 128) {
+        case 1: OT_RMS_DG(1); break;
+        case 2: OT_RMS_DG(2); break;
+        case 3: OT_RMS_DG(3); break;
+        default: OT_RMS_DG(4); break;
+      }
+#undef OT_RMS_DG
+      OT_TRY(last_launch());
+    }
+    return launch_chunk_sum(part, ctas, d, dg, 0, d, st);
+  }
+  {
+    ProfScope prof(PK_TRAIN_ELEM, 0.0,
+                   (double)rows * d * (sizeof(Tx) + 4.0 + 8.0 + 4.0 + (dx_copy ? sizeof(T) : 0)), st);
+    rms_backward_kernel<Tx, T><<<(unsigned)cdiv(rows, 8), 256, 0, st>>>(
+        (const Tx*)x, x_sb, x_st, (const T*)gamma, dy, dx, dx_sb, dx_st, pg, rows, fold, d, eps, (T*)dx_copy);
+    OT_TRY(last_launch());
+  }
+  return launch_colsum(pg, rowset(0, (long long)fold * d, d, fold, rows), 1, d, dg, 0, part, st);
 }
 
 template <typename T>
@@ -1334,15 +1383,21 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
   const long long Mmax = pad64((long long)B * L0) + 64LL * kSplitCtas;   // row chunks pad each to 64 rows
   const long long op_elems = std::max<long long>(Mmax, (long long)L_NS * pad64(B)) * std::max(3 * d, dff);
   const long long split_elems = (long long)kSplitCtas * 128 * 256;      // chunks x N_out x K_in, at most
-  const long long col_elems = (cdiv((long long)B * L0, kColChunk) + cdiv(B, kColChunk) * L_NS) * std::max(3 * d, dff);
+  const long long col_elems = std::max<long long>(cdiv((long long)B * L0, kColChunk) + cdiv(B, kColChunk) * L_NS,
+                                                  kRedCtas) * std::max(3 * d, dff);
   const long long wt_elems = (long long)(1 + L_NS) * std::max(3 * d, dff) * d;
   Carve cv(ws, ws_bytes);
   std::vector<float*> X(NL, nullptr);   // float32 inputs of layers 1 .. NL-1
   for (int n = 1; n < NL; ++n) X[n] = (float*)cv.take((size_t)B * Ln[n] * d * 4);
   void* h = cv.take((size_t)B * L0 * d * es);
   void* qkv = cv.take((size_t)B * L0 * 3 * d * es);
-  void* a = cv.take((size_t)B * Lq0 * d * es);
-  float* lse = (float*)cv.take((size_t)B * H * Lq0 * 4);
+  // each layer's attention output and log-sum-exp, kept from the forward
+  std::vector<void*> Aout(NL);
+  std::vector<float*> LSE(NL);
+  for (int n = 0; n < NL; ++n) {
+    Aout[n] = cv.take((size_t)B * Lq[n] * d * es);
+    LSE[n] = (float*)cv.take((size_t)B * H * Lq[n] * 4);
+  }
   float* Dr = (float*)cv.take((size_t)B * H * Lq0 * 4);
   float* x1 = (float*)cv.take((size_t)B * Lq0 * d * 4);
   void* h2 = cv.take((size_t)B * Lq0 * d * es);
@@ -1381,20 +1436,25 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     return ONETRANS_OK;
   };
 
-  // recompute layer n's intermediates from its input x_in (L rows per sample):
-  // the forward pass needs z = GELU(W1 h2 + b1), the backward the
-  // pre-activation u (z then comes out of the GELU backward)
+  // layer n's intermediates from its input x_in (L rows per sample).  The
+  // forward pass computes the attention output and its log-sum-exp, kept
+  // for the backward, and z = GELU(W1 h2 + b1); the backward recomputes the
+  // rest (h, q | k | v, x1, h2 and the pre-activation u; z then comes out of
+  // the GELU backward).
   auto recompute = [&](int n, const void* x_in, bool x_f32, bool fwd) -> onetrans_status {
     const int L = Ln[n], Lqn = Lq[n], s = L - L_NS, sq = Lqn - L_NS, off = L - Lqn;
+    void* a = Aout[n];
     if (x_f32) OT_TRY(rms_flat<T>(m, x_in, true, h, (long long)B * L, m->g_attn[n], st));
     else OT_TRY(rms_flat<T>(m, x_in, false, h, (long long)B * L, m->g_attn[n], st));
     // q | k | v of every row (q unscaled)
     OT_TRY(mixed_rows_gemm<T>(m, h, d, (long long)L * d, L, B, 0, s, L, m->Wqkv_S[n], m->Wqkv_NS[n], d, 3 * d,
                               rmap(qkv, (long long)L * 3 * d, 3 * d), st));
-    AttnRows ar;
-    ar.qkv = qkv; ar.B = B; ar.L = L; ar.Lq = Lqn; ar.H = H; ar.d = d;
-    if (tc_attn) OT_TRY(launch_attn_train_tc(m, 0, ar, a, lse, nullptr, nullptr, nullptr, st));
-    else OT_TRY(launch_attn_rows<T>(m, 0, ar, a, lse, nullptr, nullptr, nullptr, st));
+    if (fwd) {
+      AttnRows ar;
+      ar.qkv = qkv; ar.B = B; ar.L = L; ar.Lq = Lqn; ar.H = H; ar.d = d;
+      if (tc_attn) OT_TRY(launch_attn_train_tc(m, 0, ar, a, LSE[n], nullptr, nullptr, nullptr, st));
+      else OT_TRY(launch_attn_rows<T>(m, 0, ar, a, LSE[n], nullptr, nullptr, nullptr, st));
+    }
     // x1 = x[tail] + W^O a, h2 = RMSNorm(x1)
     GemmDesc go = gdesc_base(m);
     go.mode = TILE_FLAT; go.M = B * Lqn; go.fold = Lqn; go.G = 1;
@@ -1428,6 +1488,8 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
   OT_TRY(launch_cast<T>(dy, gT, (long long)B * Lq[NL - 1] * d, st));
   for (int n = NL - 1; n >= 0; --n) {
     const int L = Ln[n], Lqn = Lq[n], s = L - L_NS, sq = Lqn - L_NS, off = L - Lqn;
+    void* a = Aout[n];
+    float* lse = LSE[n];
     const bool x_f32 = n > 0;
     const void* x_in = n == 0 ? x0 : (const void*)X[n];
     float* g_in = n == 0 ? dx0 : gbuf[n % 2];   // gradient of layer n's input, [B, L, d]
@@ -1440,14 +1502,36 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     OT_TRY(mixed_rows_gemm<T>(m, gT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap32(dz, Mf, dff), st));
     // z = GELU(u), u = W1 h2 + b1
     const long long nz = (long long)B * Mf;
-    {
+    const int rows = B * Lqn;
+    const bool gelu_fused = gr->b1_S[n] && dff % 4 == 0 && dff <= 4096;
+    if (gelu_fused) {
+      // du, z and the S rows' column sums of du (db1 of the shared set) in one pass
+      const int ctas0 = (int)std::min<long long>(cdiv(rows, 8), kRedCtas);
+      const int rows_per = (int)cdiv(rows, ctas0), ctas = (int)cdiv(rows, rows_per);
+      {
+        ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + 3.0 * es) + (double)ctas * dff * 4, st);
+#define OT_GELU_B(J)                                                                                        \
+  gelu_backward_bias_kernel<T, J><<<(unsigned)ctas, 256, 0, st>>>(dz, (const T*)u, (T*)du, (T*)z, rows, Lqn, sq, \
+                                                                   dff, rows_per, col_part)
+        switch ((dff + 1023) / 1024) {
+          case 1: OT_GELU_B(1); break;
+          case 2: OT_GELU_B(2); break;
+          case 3: OT_GELU_B(3); break;
+          default: OT_GELU_B(4); break;
+        }
+#undef OT_GELU_B
+        OT_TRY(last_launch());
+      }
+      OT_TRY(launch_chunk_sum(col_part, ctas, dff, gr->b1_S[n], 0, dff, st));
+    } else {
       ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + 3.0 * es), st);
       gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 1024), 256, 0, st>>>(dz, (const T*)u, (T*)du, (T*)z, nz);
+      OT_TRY(last_launch());
     }
-    OT_TRY(last_launch());
     OT_TRY(weight_grad<T>(m, GradRows{gT, d, Md, false}, GradRows{z, dff, Mf, false}, d, dff, B, 0, sq, Lqn,
                           gr->W2_S[n], gr->W2_NS[n], sc, st));
-    OT_TRY(bias_grad((const T*)du, dff, Mf, dff, B, 0, sq, Lqn, gr->b1_S[n], gr->b1_NS[n], col_part, st));
+    OT_TRY(bias_grad((const T*)du, dff, Mf, dff, B, 0, sq, Lqn, gelu_fused ? nullptr : gr->b1_S[n], gr->b1_NS[n],
+                     col_part, st));
     OT_TRY(weight_grad<T>(m, GradRows{du, dff, Mf, false}, GradRows{h2, d, Md, false}, dff, d, B, 0, sq, Lqn,
                           gr->W1_S[n], gr->W1_NS[n], sc, st));
     OT_TRY(weights_T(m->W1_S[n], m->W1_NS[n], dff, d, wS, wNS));
@@ -1455,8 +1539,7 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     // h2 = RMSNorm(x1; g_ffn), x1 = x[tail] + W^O a
     OT_TRY(cuda_ok(cudaMemcpyAsync(dx1, g_cur, (size_t)B * Md * 4, cudaMemcpyDeviceToDevice, st)));
     OT_TRY((launch_rms_backward<T, float>(x1, Md, d, m->g_ffn[n], dh2, dx1, Md, d, pg, B * Lqn, Lqn, d,
-                                         m->cfg.rms_eps, dx1T, st)));
-    OT_TRY(launch_colsum(pg, rowset(0, Md, d, Lqn, B * Lqn), 1, d, gr->g_ffn[n], 0, col_part, st));
+                                         m->cfg.rms_eps, dx1T, gr->g_ffn[n], col_part, st)));
     OT_TRY(weight_grad<T>(m, GradRows{dx1T, d, Md, false}, GradRows{a, d, Md, false}, d, d, B, 0, Lqn, Lqn,
                           gr->Wo[n], nullptr, sc, st));
     OT_TRY(weights_T(m->Wo[n], nullptr, d, d, wS, wNS));
@@ -1470,9 +1553,11 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     AttnRows ar;
     ar.qkv = qkv; ar.B = B; ar.L = L; ar.Lq = Lqn; ar.H = H; ar.d = d;
     if (tc_attn) {
-      const long long nd = (long long)B * Lqn * H;
-      attn_train_delta_kernel<<<(unsigned)cdiv(nd, 256), 256, 0, st>>>((const __nv_bfloat16*)dOb,
-                                                                        (const __nv_bfloat16*)a, Dr, B, Lqn, H, m->dh);
+      {
+        ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)B * Lqn * d * 4.0 + (double)B * Lqn * H * 4.0, st);
+        attn_train_delta_kernel<<<(unsigned)cdiv((long long)B * Lqn, 8), 256, 0, st>>>(
+            (const __nv_bfloat16*)dOb, (const __nv_bfloat16*)a, Dr, B, Lqn, H);
+      }
       OT_TRY(last_launch());
       OT_TRY(launch_attn_train_tc(m, 1, ar, a, lse, Dr, dOb, dqkv, st));
       OT_TRY(launch_attn_train_tc(m, 2, ar, a, lse, Dr, dOb, dqkv, st));
@@ -1491,11 +1576,10 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     void* g_copy = n > 0 ? gT : nullptr;
     if (x_f32)
       OT_TRY((launch_rms_backward<T, float>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
-                                           B * L, L, d, m->cfg.rms_eps, g_copy, st)));
+                                           B * L, L, d, m->cfg.rms_eps, g_copy, gr->g_attn[n], col_part, st)));
     else
       OT_TRY((launch_rms_backward<T, T>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
-                                       B * L, L, d, m->cfg.rms_eps, g_copy, st)));
-    OT_TRY(launch_colsum(pg, rowset(0, (long long)L * d, d, L, B * L), 1, d, gr->g_attn[n], 0, col_part, st));
+                                       B * L, L, d, m->cfg.rms_eps, g_copy, gr->g_attn[n], col_part, st)));
     g_cur = g_in;
   }
   return ONETRANS_OK;
