@@ -131,24 +131,45 @@ __global__ void __launch_bounds__(256) transpose_rows_kernel(const Ti* __restric
 }
 
 // out[(i / n_inner) * out_stride + i % n_inner] = sum over the chunks k of
-// part[k * n + i]: 32 outputs per CTA, warp w adding chunks w, w + 8, ...,
-// the eight warp sums then added in warp order (a fixed order: the result
-// does not depend on timing).
-__global__ void __launch_bounds__(256) chunk_sum_kernel(const float* __restrict__ part, int chunks, long long n,
-                                                        float* __restrict__ out, long long out_stride,
-                                                        long long n_inner) {
-  __shared__ float red[8][33];
+// part[k * n + i], chunk by chunk in order.  Few chunks (the row slices of a
+// weight gradient): one thread per four outputs, vector loads.  Many chunks
+// (the per-CTA partial rows of a gain or bias gradient): 32 outputs per CTA,
+// warp w adding chunks w, w + NW, ..., the NW warp sums then added in warp
+// order.  Both orders are fixed: the result does not depend on timing.
+__global__ void __launch_bounds__(256) chunk_sum4_kernel(const float* __restrict__ part, int chunks, long long n,
+                                                         float* __restrict__ out, long long out_stride,
+                                                         long long n_inner) {
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i >= n) return;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int k = 0; k < chunks; ++k) {
+    float v[4];
+    ld4<float>(part + (long long)k * n + i, v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j] += v[j];
+  }
+  st4<float>(out + (i / n_inner) * out_stride + i % n_inner, acc);
+}
+
+template <int NW>
+__global__ void __launch_bounds__(NW * 32) chunk_sum_kernel(const float* __restrict__ part, int chunks, long long n,
+                                                            float* __restrict__ out, long long out_stride,
+                                                            long long n_inner) {
+  __shared__ float red[NW][33];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const long long i = (long long)blockIdx.x * 32 + lane;
   float acc = 0.f;
-  if (i < n)
-    for (int k = w; k < chunks; k += 8) acc += part[(long long)k * n + i];
+  if (i < n) {
+#pragma unroll 4
+    for (int k = w; k < chunks; k += NW) acc += part[(long long)k * n + i];
+  }
   red[w][lane] = acc;
   __syncthreads();
   if (w == 0 && i < n) {
     float t = 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) t += red[q][lane];
+    for (int q = 0; q < NW; ++q) t += red[q][lane];
     out[(i / n_inner) * out_stride + i % n_inner] = t;
   }
 }
@@ -250,12 +271,17 @@ __global__ void __launch_bounds__(256) rms_backward_kernel(const Tx* __restrict_
 // k*8 + w, then every (gridDim.x * 8)-th row after it; lane l the columns
 // 4l .. 4l+3 of every 128 (d = 128 NC4), as vector accesses.  The CTA's sums
 // of dy x r leave as one partial row part[k][d], the warps added in warp
-// order (chunk_sum_kernel then adds the CTAs' rows in CTA order).  Needs the
-// row strides % 4 == 0 and vector-aligned bases.
+// order (chunk_sum_kernel then adds the CTAs' rows in CTA order).  dx is
+// written, not accumulated: the gradient that reaches x around the norm (the
+// residual branch) is read from `res`, row t - r_off of the sample (0 for
+// t < r_off or without res).  Needs the row strides % 4 == 0 and
+// vector-aligned bases.
 template <typename Tx, typename T, int NC4>
 __global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restrict__ x, long long x_sb, long long x_st,
                                                               const T* __restrict__ gamma,
-                                                              const float* __restrict__ dy, float* __restrict__ dx,
+                                                              const float* __restrict__ dy,
+                                                              const float* __restrict__ res, long long r_sb,
+                                                              long long r_st, int r_off, float* __restrict__ dx,
                                                               long long dx_sb, long long dx_st, float* __restrict__ part,
                                                               int rows, int fold, float eps, T* __restrict__ dx_copy) {
   constexpr int d = 128 * NC4;
@@ -293,10 +319,11 @@ __global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restri
     const float c3 = r * r * r * sg / d;
     float* dxr = dx + b * dx_sb + t * dx_st;
     T* cpr = dx_copy ? dx_copy + b * dx_sb + t * dx_st : nullptr;
+    const float* rr = (res && t >= r_off) ? res + b * r_sb + (t - r_off) * r_st : nullptr;
 #pragma unroll
     for (int i = 0; i < NC4; ++i) {
-      float o[4];
-      ld4<float>(dxr + 128 * i + 4 * lane, o);
+      float o[4] = {0.f, 0.f, 0.f, 0.f};
+      if (rr) ld4<float>(rr + 128 * i + 4 * lane, o);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         o[j] += r * gm[i][j] * dv[i][j] - xv[i][j] * c3;
@@ -319,15 +346,6 @@ __global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restri
   }
 }
 
-// GELU-tanh and its derivative from one tanh: with v = c (u + a u^3),
-// c = sqrt(2/pi), a = 0.044715, GELU(u) = 0.5 u (1 + tanh v) and
-// d/du = 0.5 (1 + tanh v) + 0.5 u (1 - tanh^2 v) c (1 + 3 a u^2).
-__device__ inline void gelu_tanh_and_grad(float u, float& z, float& g) {
-  const float c = 0.7978845608028654f, a = 0.044715f;
-  const float th = tanh_fast(c * (u + a * u * u * u));   // MUFU tanh, relative error about 2^-11
-  z = 0.5f * u * (1.f + th);
-  g = 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * a * u * u);
-}
 
 // du = dz * GELU'(u) and z = GELU(u), both in the storage type (du: the
 // operand of the next GEMMs and the rows whose column sums are db1; z: the

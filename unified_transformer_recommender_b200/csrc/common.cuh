@@ -17,7 +17,10 @@ namespace ot {
 
 enum TileMode : int { TILE_ROWS = 0, TILE_SAMPLES = 1, TILE_FLAT = 2 };
 enum OutKind : int { OUT_ROWS = 0, OUT_KV = 1 };
-enum Act : int { ACT_NONE = 0, ACT_GELU = 1 };
+// ACT_GELU_BWD (the FFN backward): the product is dz, the gradient of
+// GELU's output; the epilogue reads the pre-activation u (act_in), stores
+// du = dz * GELU'(u) as the output and GELU(u) through act_out.
+enum Act : int { ACT_NONE = 0, ACT_GELU = 1, ACT_GELU_BWD = 2 };
 
 // Address of element (b, t, n) = base + b*sb + t*st + (n / split)*sc + n % split
 // (in elements).  `split` lets one GEMM write column blocks to separate
@@ -66,6 +69,7 @@ struct GemmDesc {
   KVStore kv;
   int scale_cols;     // output columns n < scale_cols are multiplied by col_scale
   float col_scale;    // (queries leave the GEMM pre-scaled by 1/sqrt(d_h) * log2(e))
+  RowMap act_in, act_out;  // ACT_GELU_BWD: u read, GELU(u) written (storage type)
 };
 
 // Queries arrive pre-scaled by 1/sqrt(d_h) * log2(e) (the producing GEMM's

@@ -184,6 +184,9 @@ __global__ void __launch_bounds__(BresCfg::THREADS, 1)
       tc_fence_after();
       // this thread's 128 columns of the tile (its half), as bf16 pairs
       uint32_t pk[64];
+      int ob = 0, ot_ = 0;   // (b, t) of this thread's output row
+      const bool row_ok = mt0 + r < d.m_lo + d.M;
+      if (d.act == ACT_GELU_BWD && row_ok) row_of(d, mt0 + r, g, ob, ot_);
       const uint32_t tacc = tmem + (uint32_t)(acc * C::BN + half * (C::BN / 2)) + lb;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -199,6 +202,17 @@ __global__ void __launch_bounds__(BresCfg::THREADS, 1)
         if (d.act == ACT_GELU) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = gelu_fast(v[i]);
+        } else if (d.act == ACT_GELU_BWD && row_ok) {
+          // v = dz; u from its rows: du = dz GELU'(u) leaves as the output, GELU(u) through act_out
+          float uv[32];
+          load_row32(d.act_in, rm_off(d.act_in, ob, ot_, n), uv);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float g;
+            gelu_tanh_and_grad(uv[i], uv[i], g);
+            v[i] *= g;
+          }
+          store_row32(d.act_out, rm_off(d.act_out, ob, ot_, n), uv);
         }
         if (n < d.scale_cols) {
 #pragma unroll

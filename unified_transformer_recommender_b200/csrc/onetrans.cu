@@ -218,6 +218,7 @@ static double gemm_bytes(const onetrans_model* m, const GemmDesc& d) {
   b += rows * d.N * (d.out_kind == OUT_KV ? es : (d.out.f32 ? 4 : es));
   if (d.res.base) b += rows * d.N * (d.res.f32 ? 4 : es);
   if (d.rms.base) b += rows * d.N * es;
+  if (d.act == ACT_GELU_BWD) b += 2.0 * rows * d.N * es;
   return b;
 }
 
@@ -227,6 +228,11 @@ static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, c
   if (d.M <= 0 || d.G <= 0 || d.N <= 0) return ONETRANS_OK;
   if (cdiv(d.M, 64) > 65535 || d.G > 65535) return ONETRANS_ERR_SHAPE;
   ProfScope prof(kind, 2.0 * d.M * d.G * (double)d.N * d.K, gemm_bytes(m, d), st);
+  if (d.act == ACT_GELU_BWD) {
+    // the GELU-backward epilogue exists in the weight-resident kernel only
+    if (!(m->bf16 && g_policy == 0 && tc_gemm_supported(d) && tc_bres_supported(d))) return ONETRANS_ERR_UNSUPPORTED;
+    return tc_bres_launch(d, device_sm_count(), st);
+  }
   if (m->bf16 && g_policy == 0 && tc_gemm_supported(d)) {
     if (tc_bres_supported(d)) {
       const onetrans_status r = tc_bres_launch(d, device_sm_count(), st);
@@ -1010,7 +1016,13 @@ static onetrans_status launch_chunk_sum(const float* part, int chunks, long long
                                         long long n_inner, cudaStream_t st) {
   if (n <= 0) return ONETRANS_OK;
   ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)n * (chunks + 1) * 4.0, st);
-  chunk_sum_kernel<<<(unsigned)cdiv(n, 32), 256, 0, st>>>(part, chunks, n, out, out_stride, n_inner);
+  if (chunks <= 32 && n % 4 == 0 && n_inner % 4 == 0 && out_stride % 4 == 0 && (uintptr_t)part % 16 == 0 &&
+      (uintptr_t)out % 16 == 0)
+    chunk_sum4_kernel<<<(unsigned)cdiv(n / 4, 256), 256, 0, st>>>(part, chunks, n, out, out_stride, n_inner);
+  else if (chunks <= 64)
+    chunk_sum_kernel<8><<<(unsigned)cdiv(n, 32), 256, 0, st>>>(part, chunks, n, out, out_stride, n_inner);
+  else
+    chunk_sum_kernel<32><<<(unsigned)cdiv(n, 32), 1024, 0, st>>>(part, chunks, n, out, out_stride, n_inner);
   return last_launch();
 }
 
@@ -1074,18 +1086,32 @@ static onetrans_status launch_cast(const float* src, void* dst, long long n, cud
 // t < t_s use the shared S weights W_S [N, K], rows t >= t_s the set of NS
 // token t - t_s of W_NS [L_NS, N, K].  A element (b, t, k) = A + b*a_samp +
 // t*a_row + k; output rows through `out`; optional bias sets and residual.
+// When the range is every row of densely stored samples, the shared-weight
+// launch runs over all rows as one flat row set (whole 128-row tiles across
+// sample boundaries, and one weight slice for the weight-resident kernel);
+// the NS launch after it then rewrites the NS rows with their own weights.
+// The output must not alias the residual or act_in rows.
 template <typename T>
 static onetrans_status mixed_rows_gemm(const onetrans_model* m, const void* A, long long a_row, long long a_samp,
                                        int a_rows, int B, int t_lo, int t_s, int t_hi, const void* W_S,
                                        const void* W_NS, int K, int N, RowMap out, cudaStream_t st,
                                        const void* bias_S = nullptr, const void* bias_NS = nullptr,
-                                       RowMap res = RowMap{}, int act = ACT_NONE) {
-  if (t_s > t_lo) {
+                                       RowMap res = RowMap{}, int act = ACT_NONE, RowMap act_in = RowMap{},
+                                       RowMap act_out = RowMap{}) {
+  const bool flat = t_lo == 0 && t_hi == a_rows && a_samp == (long long)a_rows * a_row;
+  if (t_s > t_lo && flat) {
+    GemmDesc g = gdesc_base(m);
+    g.mode = TILE_FLAT; g.M = B * a_rows; g.fold = a_rows; g.G = 1;
+    g.K = K; g.A = A; g.a_sm = a_row; g.a_mext = (long long)B * a_rows; g.a_gext = 1;
+    g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S; g.act = act;
+    g.out = out; g.res = res; g.act_in = act_in; g.act_out = act_out;
+    OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
+  } else if (t_s > t_lo) {
     GemmDesc g = gdesc_base(m);
     g.mode = TILE_ROWS; g.M = t_s - t_lo; g.m_lo = t_lo; g.G = B; g.g_lo = 0;
     g.K = K; g.A = A; g.a_sm = a_row; g.a_sg = a_samp; g.a_mext = a_rows; g.a_gext = B;
     g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S; g.act = act;
-    g.out = out; g.res = res;
+    g.out = out; g.res = res; g.act_in = act_in; g.act_out = act_out;
     OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
   }
   if (t_hi > t_s) {
@@ -1094,7 +1120,7 @@ static onetrans_status mixed_rows_gemm(const onetrans_model* m, const void* A, l
     g.K = K; g.A = A; g.a_sm = a_samp; g.a_sg = a_row; g.a_mext = B; g.a_gext = a_rows;
     g.W = W_NS; g.w_sg = (long long)N * K; g.w_rows = N; g.w_groups = t_hi - t_s; g.N = N;
     g.bias = bias_NS; g.bias_sg = bias_NS ? N : 0; g.act = act;
-    g.out = out; g.res = res;
+    g.out = out; g.res = res; g.act_in = act_in; g.act_out = act_out;
     OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
   }
   return ONETRANS_OK;
@@ -1246,20 +1272,24 @@ static onetrans_status bias_grad(const Ti* rows, long long row, long long samp, 
   return ONETRANS_OK;
 }
 
-// RMSNorm backward of `rows` rows (dx += ..., optional storage-type copy of
-// each finished dx row) and the gain gradient dg = sum over the rows of
-// dy x r: folded into the row kernel (one partial row per CTA, added in CTA
-// order) where d is a multiple of 128 up to 512 and the rows allow vector
-// access, else through per-row products and column sums.
+// RMSNorm backward of `rows` rows (`fold` per sample) into dx (dense
+// [B][fold][d] rows): dx = (residual gradient: row t - r_off of `res`, 0 for
+// t < r_off) + the norm's backward, with an optional storage-type copy of
+// each finished row, and the gain gradient dg = sum over the rows of dy x r.
+// Where d is a multiple of 128 up to 512 and the rows allow vector access
+// one row kernel does it all (dg as one partial row per CTA, added in CTA
+// order); else dx is filled from `res` first and the per-row products are
+// column-summed.
 template <typename T, typename Tx>
 static onetrans_status launch_rms_backward(const void* x, long long x_sb, long long x_st, const void* gamma,
-                                           const float* dy, float* dx, long long dx_sb, long long dx_st, float* pg,
-                                           int rows, int fold, int d, float eps, void* dx_copy, float* dg,
-                                           float* part, cudaStream_t st) {
+                                           const float* dy, const float* res, long long r_sb, long long r_st,
+                                           int r_off, float* dx, float* pg, int rows, int fold, int d, float eps,
+                                           void* dx_copy, float* dg, float* part, cudaStream_t st) {
   if (rows <= 0) return dg ? cuda_ok(cudaMemsetAsync(dg, 0, (size_t)d * 4, st)) : ONETRANS_OK;
+  const long long dx_sb = (long long)fold * d, dx_st = d;
   const bool fused = d % 128 == 0 && d <= 512 && vec4_ok(x, 4 * sizeof(Tx), {x_sb, x_st}) &&
-                     vec4_ok(dx, 16, {dx_sb, dx_st}) && vec4_ok(dy, 16, {}) && vec4_ok(gamma, 4 * sizeof(T), {}) &&
-                     vec4_ok(dx_copy, 4 * sizeof(T), {});
+                     vec4_ok(dx, 16, {}) && vec4_ok(res, 16, {r_sb, r_st}) && vec4_ok(dy, 16, {}) &&
+                     vec4_ok(gamma, 4 * sizeof(T), {}) && vec4_ok(dx_copy, 4 * sizeof(T), {});
   if (fused) {
     const int ctas = (int)std::min<long long>(cdiv(rows, 8), kRedCtas);
     {
@@ -1268,8 +1298,8 @@ static onetrans_status launch_rms_backward(const void* x, long long x_sb, long l
                      st);
 #define OT_RMS_DG(NC4)                                                                                             \
   rms_backward_dg_kernel<Tx, T, NC4><<<(unsigned)ctas, 256, 0, st>>>((const Tx*)x, x_sb, x_st, (const T*)gamma, dy, \
-                                                                    dx, dx_sb, dx_st, part, rows, fold, eps,       \
-                                                                    (T*)dx_copy)
+                                                                    res, r_sb, r_st, r_off, dx, dx_sb, dx_st, part, \
+                                                                    rows, fold, eps, (T*)dx_copy)
       switch (d / 128) {
         case 1: OT_RMS_DG(1); break;
         case 2: OT_RMS_DG(2); break;
@@ -1281,6 +1311,11 @@ static onetrans_status launch_rms_backward(const void* x, long long x_sb, long l
     }
     return launch_chunk_sum(part, ctas, d, dg, 0, d, st);
   }
+  // dx starts as the residual gradient
+  OT_TRY(cuda_ok(cudaMemsetAsync(dx, 0, (size_t)rows * d * 4, st)));
+  if (res && fold > r_off)
+    OT_TRY(cuda_ok(cudaMemcpy2DAsync(dx + (size_t)r_off * d, (size_t)dx_sb * 4, res, (size_t)r_sb * 4,
+                                     (size_t)(fold - r_off) * d * 4, rows / fold, cudaMemcpyDeviceToDevice, st)));
   {
     ProfScope prof(PK_TRAIN_ELEM, 0.0,
                    (double)rows * d * (sizeof(Tx) + 4.0 + 8.0 + 4.0 + (dx_copy ? sizeof(T) : 0)), st);
@@ -1499,34 +1534,47 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     OT_TRY(bias_grad(g_cur, d, Md, d, B, 0, sq, Lqn, gr->b2_S[n], gr->b2_NS[n], col_part, st));
     void *wS, *wNS;
     OT_TRY(weights_T(m->W2_S[n], m->W2_NS[n], d, dff, wS, wNS));
-    OT_TRY(mixed_rows_gemm<T>(m, gT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap32(dz, Mf, dff), st));
-    // z = GELU(u), u = W1 h2 + b1
-    const long long nz = (long long)B * Mf;
-    const int rows = B * Lqn;
-    const bool gelu_fused = gr->b1_S[n] && dff % 4 == 0 && dff <= 4096;
-    if (gelu_fused) {
-      // du, z and the S rows' column sums of du (db1 of the shared set) in one pass
-      const int ctas0 = (int)std::min<long long>(cdiv(rows, 8), kRedCtas);
-      const int rows_per = (int)cdiv(rows, ctas0), ctas = (int)cdiv(rows, rows_per);
-      {
-        ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + 3.0 * es) + (double)ctas * dff * 4, st);
+    // z = GELU(u), u = W1 h2 + b1: the dz GEMM's epilogue applies the GELU
+    // backward where the weight-resident kernel takes the shape (du and z
+    // in the storage type, dz never stored); otherwise dz in float32 and a
+    // GELU-backward pass that also sums the S rows' du
+    const onetrans_status fz =
+        m->bf16 && g_policy == 0
+            ? mixed_rows_gemm<T>(m, gT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap(du, Mf, dff), st, nullptr,
+                                 nullptr, RowMap{}, ACT_GELU_BWD, rmap(u, Mf, dff), rmap(z, Mf, dff))
+            : ONETRANS_ERR_UNSUPPORTED;
+    if (fz != ONETRANS_OK && fz != ONETRANS_ERR_UNSUPPORTED) return fz;
+    const bool gelu_in_gemm = fz == ONETRANS_OK;
+    bool gelu_fused = false;
+    if (!gelu_in_gemm) {
+      OT_TRY(mixed_rows_gemm<T>(m, gT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap32(dz, Mf, dff), st));
+      const long long nz = (long long)B * Mf;
+      const int rows = B * Lqn;
+      gelu_fused = gr->b1_S[n] && dff % 4 == 0 && dff <= 4096;
+      if (gelu_fused) {
+        // du, z and the S rows' column sums of du (db1 of the shared set) in one pass
+        const int ctas0 = (int)std::min<long long>(cdiv(rows, 8), kRedCtas);
+        const int rows_per = (int)cdiv(rows, ctas0), ctas = (int)cdiv(rows, rows_per);
+        {
+          ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + 3.0 * es) + (double)ctas * dff * 4, st);
 #define OT_GELU_B(J)                                                                                        \
   gelu_backward_bias_kernel<T, J><<<(unsigned)ctas, 256, 0, st>>>(dz, (const T*)u, (T*)du, (T*)z, rows, Lqn, sq, \
                                                                    dff, rows_per, col_part)
-        switch ((dff + 1023) / 1024) {
-          case 1: OT_GELU_B(1); break;
-          case 2: OT_GELU_B(2); break;
-          case 3: OT_GELU_B(3); break;
-          default: OT_GELU_B(4); break;
-        }
+          switch ((dff + 1023) / 1024) {
+            case 1: OT_GELU_B(1); break;
+            case 2: OT_GELU_B(2); break;
+            case 3: OT_GELU_B(3); break;
+            default: OT_GELU_B(4); break;
+          }
 #undef OT_GELU_B
+          OT_TRY(last_launch());
+        }
+        OT_TRY(launch_chunk_sum(col_part, ctas, dff, gr->b1_S[n], 0, dff, st));
+      } else {
+        ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + 3.0 * es), st);
+        gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 1024), 256, 0, st>>>(dz, (const T*)u, (T*)du, (T*)z, nz);
         OT_TRY(last_launch());
       }
-      OT_TRY(launch_chunk_sum(col_part, ctas, dff, gr->b1_S[n], 0, dff, st));
-    } else {
-      ProfScope prof(PK_TRAIN_ELEM, 0.0, (double)nz * (4.0 + 3.0 * es), st);
-      gelu_backward_kernel<T><<<(unsigned)cdiv(nz, 1024), 256, 0, st>>>(dz, (const T*)u, (T*)du, (T*)z, nz);
-      OT_TRY(last_launch());
     }
     OT_TRY(weight_grad<T>(m, GradRows{gT, d, Md, false}, GradRows{z, dff, Mf, false}, d, dff, B, 0, sq, Lqn,
                           gr->W2_S[n], gr->W2_NS[n], sc, st));
@@ -1536,18 +1584,13 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
                           gr->W1_S[n], gr->W1_NS[n], sc, st));
     OT_TRY(weights_T(m->W1_S[n], m->W1_NS[n], dff, d, wS, wNS));
     OT_TRY(mixed_rows_gemm<T>(m, du, dff, Mf, Lqn, B, 0, sq, Lqn, wS, wNS, dff, d, rmap32(dh2, Md, d), st));
-    // h2 = RMSNorm(x1; g_ffn), x1 = x[tail] + W^O a
-    OT_TRY(cuda_ok(cudaMemcpyAsync(dx1, g_cur, (size_t)B * Md * 4, cudaMemcpyDeviceToDevice, st)));
-    OT_TRY((launch_rms_backward<T, float>(x1, Md, d, m->g_ffn[n], dh2, dx1, Md, d, pg, B * Lqn, Lqn, d,
+    // h2 = RMSNorm(x1; g_ffn), x1 = x[tail] + W^O a; y's gradient reaches x1 around the FFN
+    OT_TRY((launch_rms_backward<T, float>(x1, Md, d, m->g_ffn[n], dh2, g_cur, Md, d, 0, dx1, pg, B * Lqn, Lqn, d,
                                          m->cfg.rms_eps, dx1T, gr->g_ffn[n], col_part, st)));
     OT_TRY(weight_grad<T>(m, GradRows{dx1T, d, Md, false}, GradRows{a, d, Md, false}, d, d, B, 0, Lqn, Lqn,
                           gr->Wo[n], nullptr, sc, st));
     OT_TRY(weights_T(m->Wo[n], nullptr, d, d, wS, wNS));
     OT_TRY(mixed_rows_gemm<T>(m, dx1T, d, Md, Lqn, B, 0, Lqn, Lqn, wS, nullptr, d, d, rmap(dOb, Md, d), st));
-    // the residual: the tail rows of the input receive dx1, the others start at 0
-    OT_TRY(cuda_ok(cudaMemsetAsync(g_in, 0, (size_t)B * L * d * 4, st)));
-    OT_TRY(cuda_ok(cudaMemcpy2DAsync(g_in + (size_t)off * d, (size_t)L * d * 4, dx1, (size_t)Md * 4, (size_t)Md * 4,
-                                     B, cudaMemcpyDeviceToDevice, st)));
     // attention: dq, dk, dv of the recomputed rows
     OT_TRY(cuda_ok(cudaMemsetAsync(dqkv, 0, (size_t)B * L * 3 * d * es, st)));
     AttnRows ar;
@@ -1572,13 +1615,14 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     OT_TRY(weights_T(m->Wqkv_S[n], m->Wqkv_NS[n], 3 * d, d, wS, wNS));
     OT_TRY(mixed_rows_gemm<T>(m, dqkv, 3 * d, Mq, L, B, 0, s, L, wS, wNS, 3 * d, d,
                               rmap32(dh, (long long)L * d, d), st));
-    // h = RMSNorm(x; g_attn); the lower layer's output gradient also as its GEMM operand
+    // h = RMSNorm(x; g_attn); x1's gradient reaches the tail rows of x around
+    // the attention; the lower layer's output gradient also as its GEMM operand
     void* g_copy = n > 0 ? gT : nullptr;
     if (x_f32)
-      OT_TRY((launch_rms_backward<T, float>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
+      OT_TRY((launch_rms_backward<T, float>(x_in, (long long)L * d, d, m->g_attn[n], dh, dx1, Md, d, off, g_in, pg,
                                            B * L, L, d, m->cfg.rms_eps, g_copy, gr->g_attn[n], col_part, st)));
     else
-      OT_TRY((launch_rms_backward<T, T>(x_in, (long long)L * d, d, m->g_attn[n], dh, g_in, (long long)L * d, d, pg,
+      OT_TRY((launch_rms_backward<T, T>(x_in, (long long)L * d, d, m->g_attn[n], dh, dx1, Md, d, off, g_in, pg,
                                        B * L, L, d, m->cfg.rms_eps, g_copy, gr->g_attn[n], col_part, st)));
     g_cur = g_in;
   }

@@ -287,6 +287,15 @@ __device__ inline float gelu_fast(float x) {
   const float hx = 0.5f * x;
   return fmaf(hx, tanh_fast(x * fmaf(k01, x * x, k0)), hx);
 }
+// GELU-tanh and its derivative from one tanh: with v = c (u + a u^3),
+// c = sqrt(2/pi), a = 0.044715, GELU(u) = 0.5 u (1 + tanh v) and
+// d/du = 0.5 (1 + tanh v) + 0.5 u (1 - tanh^2 v) c (1 + 3 a u^2).
+__device__ inline void gelu_tanh_and_grad(float u, float& z, float& g) {
+  const float c = 0.7978845608028654f, a = 0.044715f;
+  const float th = tanh_fast(c * (u + a * u * u * u));   // MUFU tanh, relative error about 2^-11
+  z = 0.5f * u * (1.f + th);
+  g = 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * a * u * u);
+}
 // The same for a pair (x0, x1) = (a0 + b0, a1 + b1), returned as bf16x2: the
 // fp32 arithmetic on packed pairs, the two tanh on the MUFU.
 __device__ inline uint32_t gelu_bias_bf16x2(float a0, float a1, float b0, float b1) {
