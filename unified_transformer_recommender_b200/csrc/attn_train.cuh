@@ -35,9 +35,10 @@ struct TrainAttnArgs {
 struct TrainAttnCfg {
   static constexpr int DH = 64, BM = 128, BN = 128, BOX = 16384, STAGES = 2;
   static constexpr int BAR_BYTES = 256;
-  // 6 tiles of 16 KB, the barriers, a query tile's log-sum-exp and D (1 KB);
-  // the request is raised to 120 KB so that one CTA runs per SM (each takes
-  // all 512 TMEM columns)
+  // 6 tiles of 16 KB, the barriers, a query tile's log-sum-exp and D (1 KB).
+  // The forward takes 256 TMEM columns and this request (two CTAs per SM);
+  // dQ and dK/dV take all 512 columns and raise the request to 120 KB, so
+  // that one CTA runs per SM
   static constexpr int SMEM = 6 * BOX + BAR_BYTES + 2 * BM * 4;
   static constexpr int SMEM_REQ = 120 * 1024;
 };
@@ -54,7 +55,7 @@ __device__ inline float fmax3_t(float a, float b, float c) {
 }
 
 template <bool DQ>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, DQ ? 1 : 2)
     attn_train_q_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                         const TrainAttnArgs a) {
   using C = TrainAttnCfg;
@@ -95,12 +96,14 @@ __global__ void __launch_bounds__(192, 1)
     prefetch_tmap(&tmQKV);
     if (DQ) prefetch_tmap(&tmDO);
   }
-  if (warp == 5) tmem_alloc(tmem_slot, 512);
+  constexpr uint32_t kCols = DQ ? 512 : 256;
+  if (warp == 5) tmem_alloc(tmem_slot, kCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tX = tmem + 128, tP = tmem + 256, tQ = tmem + 320;  // tX: O (forward) or dP
+  // forward: S 0-127, O 128-191, P 192-255; dQ: S 0-127, dP 128-255, dS 256-319, dQ 320-383
+  const uint32_t tS = tmem, tX = tmem + 128, tP = tmem + (DQ ? 256 : 192), tQ = tmem + 320;
   grid_dep_wait();
   grid_dep_launch();
 
@@ -294,10 +297,17 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) tmem_dealloc(tmem, 512);
+  if (warp == 5) tmem_dealloc(tmem, kCols);
 }
 
-__global__ void __launch_bounds__(192, 1)
+// dK, dV: one CTA per 128 keys of one head, two CTAs per SM.  Each query
+// tile is taken in two halves of 64 queries: S^T = K Q^T and dP^T = V dO^T
+// (N = 64) into TMEM, then P^T and dS^T written as bf16 over the S^T and
+// dP^T columns already read (so 256 TMEM columns hold S^T, dP^T, dV and
+// dK), then dV += P^T dO and dK += dS^T Q with the A operands from TMEM.  The
+// next half's products wait for those two (their commit), so one CTA runs
+// its products and its softmax in turn and the SM's other CTA fills the gaps.
+__global__ void __launch_bounds__(192, 2)
     attn_train_kv_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                          const TrainAttnArgs a) {
   using C = TrainAttnCfg;
@@ -309,12 +319,11 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* kv_ready = bars;
   uint64_t* qd_full = bars + 1;              // [STAGES]
   uint64_t* qd_empty = qd_full + C::STAGES;  // [STAGES]
-  uint64_t* s_full = qd_empty + C::STAGES;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* p_free = s_full + 3;
-  uint64_t* o_done = s_full + 4;
-  uint32_t* tmem_slot = (uint32_t*)(s_full + 5);
+  uint64_t* s_full = qd_empty + C::STAGES;   // S^T and dP^T of a half are in TMEM
+  uint64_t* p_full = s_full + 1;             // P^T and dS^T of a half are in TMEM
+  uint64_t* p_free = s_full + 2;             // dV and dK of a half are done
+  uint64_t* o_done = s_full + 3;
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 4);
   if (smem_u32(smem) & 1023) {
     if (threadIdx.x == 0) flag_error(kErrSmemAlign);
     return;
@@ -328,7 +337,6 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(kv_ready, 1);
     for (int i = 0; i < C::STAGES; ++i) { mbar_init(&qd_full[i], 1); mbar_init(&qd_empty[i], 1); }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
     mbar_init(o_done, 1);
@@ -338,13 +346,13 @@ __global__ void __launch_bounds__(192, 1)
     prefetch_tmap(&tmQKV);
     prefetch_tmap(&tmDO);
   }
-  if (warp == 5) tmem_alloc(tmem_slot, 512);
+  if (warp == 5) tmem_alloc(tmem_slot, 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 128, tP = tmem + 256, tDS = tmem + 320, tDV = tmem + 384,
-                 tDK = tmem + 448;
+  // S^T 0-63 (P^T over its first 32), dP^T 64-127 (dS^T over its first 32), dV 128-191, dK 192-255
+  const uint32_t tS = tmem, tDP = tmem + 64, tDV = tmem + 128, tDK = tmem + 192;
   grid_dep_wait();
   grid_dep_launch();
 
@@ -364,7 +372,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      constexpr uint32_t id_ss = idesc_bf16(128, 128);
+      constexpr uint32_t id_ss = idesc_bf16(128, 64);
       constexpr uint32_t id_ts = idesc_bf16(128, C::DH, false, true);
       const uint64_t dk = sdesc_k128(smem_u32(sK)), dv = sdesc_k128(smem_u32(sV));
       const uint64_t dq0 = sdesc_k128(smem_u32(sQD)), ddo0 = sdesc_k128(smem_u32(sQD + C::BOX));
@@ -373,30 +381,36 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = 0; i < nq && ok; ++i) {
         const int s = i % C::STAGES;
         ok = mbar_wait(&qd_full[s], (i / C::STAGES) & 1);
-        if (ok && i > 0) ok = mbar_wait(s_free, (i - 1) & 1);
         if (!ok) break;
-        tc_fence_after();
-        const uint32_t so = s * 2 * C::BOX;
-        // S^T = K Q^T and dP^T = V dO^T: keys on the TMEM lanes, queries on the columns
+        for (int qh = 0; qh < 2 && ok; ++qh) {
+          const int hf = 2 * i + qh;
+          // the previous half's dV, dK have read P^T and dS^T from these columns
+          if (hf > 0) ok = mbar_wait(p_free, (hf - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          // rows qh*64 .. of the Q and dO tiles: 64 rows x 128 B further in
+          const uint32_t so = s * 2 * C::BOX + qh * 8192;
+          // S^T = K Q^T and dP^T = V dO^T: keys on the TMEM lanes, 64 queries on the columns
 #pragma unroll
-        for (int k = 0; k < C::DH / 16; ++k)
-          umma_bf16(tS, desc_add(dk, k * 32), desc_add(desc_add(dq0, so), k * 32), id_ss, k ? 1u : 0u);
+          for (int k = 0; k < C::DH / 16; ++k)
+            umma_bf16(tS, desc_add(dk, k * 32), desc_add(desc_add(dq0, so), k * 32), id_ss, k ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < C::DH / 16; ++k)
-          umma_bf16(tDP, desc_add(dv, k * 32), desc_add(desc_add(ddo0, so), k * 32), id_ss, k ? 1u : 0u);
-        umma_commit(s_full);
-        ok = mbar_wait(p_full, i & 1);
-        if (!ok) break;
-        tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q: A from TMEM (16 queries per step), B MN-major
-        const uint64_t mdo = desc_add(mdo0, so), mq = desc_add(mq0, so);
+          for (int k = 0; k < C::DH / 16; ++k)
+            umma_bf16(tDP, desc_add(dv, k * 32), desc_add(desc_add(ddo0, so), k * 32), id_ss, k ? 1u : 0u);
+          umma_commit(s_full);
+          ok = mbar_wait(p_full, hf & 1);
+          if (!ok) break;
+          tc_fence_after();
+          // dV += P^T dO, dK += dS^T Q: A from TMEM (16 queries per step), B MN-major
+          const uint64_t mdo = desc_add(mdo0, so), mq = desc_add(mq0, so);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ts(tDV, tP + kk * 8, desc_add(mdo, kk * 2048), id_ts, (i || kk) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ts(tDV, tS + kk * 8, desc_add(mdo, kk * 2048), id_ts, (hf || kk) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ts(tDK, tDS + kk * 8, desc_add(mq, kk * 2048), id_ts, (i || kk) ? 1u : 0u);
-        umma_commit(p_free);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ts(tDK, tDP + kk * 8, desc_add(mq, kk * 2048), id_ts, (hf || kk) ? 1u : 0u);
+          umma_commit(p_free);
+        }
         umma_commit(&qd_empty[s]);
       }
       umma_commit(o_done);
@@ -421,42 +435,42 @@ __global__ void __launch_bounds__(192, 1)
       s_lse[r] = q0 + r < a.Lq ? lse[q0 + r] * 1.4426950408889634f : 0.f;
       s_D[r] = q0 + r < a.Lq ? Dr[q0 + r] : 0.f;
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (!ok) continue;
-      ok = mbar_wait(s_full, i & 1);
-      if (ok && i > 0) ok = mbar_wait(p_free, (i - 1) & 1);
-      if (!ok) continue;
-      tc_fence_after();
-      // query column cc sees this key when q_off + q0 + cc >= j, and exists when q0 + cc < Lq
+      // query column cc of the tile sees this key when q_off + q0 + cc >= j, and exists when q0 + cc < Lq
       const int lo = key_ok ? min(max(j - q_off - q0, 0), C::BM) : C::BM;
       const int hi = min(max(a.Lq - q0, 0), C::BM);
+      for (int qh = 0; qh < 2; ++qh) {
+        if (!ok) continue;
+        ok = mbar_wait(s_full, (2 * i + qh) & 1);
+        if (!ok) continue;
+        tc_fence_after();
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        float sv[32], dp[32];
-        tmem_ld32(tS + lb + qq * 32, sv);
-        tmem_ld32(tDP + lb + qq * 32, dp);
-        uint32_t pk[16], dk[16];
+        for (int qq = 0; qq < 2; ++qq) {
+          float sv[32], dp[32];
+          tmem_ld32(tS + lb + qq * 32, sv);
+          tmem_ld32(tDP + lb + qq * 32, dp);
+          uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float p2[2], d2[2];
+          for (int e = 0; e < 16; ++e) {
+            float p2[2], d2[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int cc = qq * 32 + 2 * e + u;
-            const bool vis = cc >= lo && cc < hi;
-            const float p = vis ? ex2_t(fmaf(sv[2 * e + u], c, -s_lse[cc])) : 0.f;
-            p2[u] = p;
-            d2[u] = p * (dp[2 * e + u] - s_D[cc]);
+            for (int u = 0; u < 2; ++u) {
+              const int cc = qh * 64 + qq * 32 + 2 * e + u;
+              const bool vis = cc >= lo && cc < hi;
+              const float p = vis ? ex2_t(fmaf(sv[2 * e + u], c, -s_lse[cc])) : 0.f;
+              p2[u] = p;
+              d2[u] = p * (dp[2 * e + u] - s_D[cc]);
+            }
+            pk[e] = pack_bf16x2(p2[0], p2[1]);
+            dk[e] = pack_bf16x2(d2[0], d2[1]);
           }
-          pk[e] = pack_bf16x2(p2[0], p2[1]);
-          dk[e] = pack_bf16x2(d2[0], d2[1]);
+          // over columns already read: chunk qq's 16 packed columns land on S^T / dP^T columns 16 qq ..
+          tmem_st16(tS + lb + qq * 16, pk);
+          tmem_st16(tDP + lb + qq * 16, dk);
         }
-        tmem_st16(tP + lb + qq * 16, pk);
-        tmem_st16(tDS + lb + qq * 16, dk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full);
       }
-      tc_fence_before();
-      mbar_arrive(s_free);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(p_full);
     }
     ok = ok && mbar_wait(o_done, 0);
     tc_fence_after();
@@ -479,7 +493,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) tmem_dealloc(tmem, 512);
+  if (warp == 5) tmem_dealloc(tmem, 256);
 }
 
 // D[b][h][t] = sum over e of dO[b, t, h, e] O[b, t, h, e] (d_h = 64): one
