@@ -1385,19 +1385,19 @@ static onetrans_status launch_attn_train_tc(const onetrans_model* m, int stage, 
                  (double)ar.B * ar.L * 3 * d * 2 + (double)ar.B * ar.Lq * d * 2, st);
   static bool attr[3] = {false, false, false};
   if (!attr[stage]) {
-    cudaError_t e = stage == 0 ? cudaFuncSetAttribute(attn_train_q_kernel<false>,
+    cudaError_t e = stage == 0 ? cudaFuncSetAttribute(attn_train_fwd_kernel,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)
-                    : stage == 1 ? cudaFuncSetAttribute(attn_train_q_kernel<true>,
-                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_REQ)
+                    : stage == 1 ? cudaFuncSetAttribute(attn_train_dq_kernel,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)
                                  : cudaFuncSetAttribute(attn_train_kv_kernel,
                                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return ONETRANS_ERR_CUDA;
     attr[stage] = true;
   }
   if (stage == 0)
-    attn_train_q_kernel<false><<<dim3((unsigned)cdiv(ar.Lq, C::BM), ar.H, ar.B), 192, C::SMEM, st>>>(tq, tdo, ta);
+    attn_train_fwd_kernel<<<dim3((unsigned)cdiv(ar.Lq, C::BM), ar.H, ar.B), 192, C::SMEM, st>>>(tq, ta);
   else if (stage == 1)
-    attn_train_q_kernel<true><<<dim3((unsigned)cdiv(ar.Lq, C::BM), ar.H, ar.B), 192, C::SMEM_REQ, st>>>(tq, tdo, ta);
+    attn_train_dq_kernel<<<dim3((unsigned)cdiv(ar.Lq, C::BM), ar.H, ar.B), 192, C::SMEM, st>>>(tq, tdo, ta);
   else
     attn_train_kv_kernel<<<dim3((unsigned)cdiv(ar.L, C::BN), ar.H, ar.B), 192, C::SMEM, st>>>(tq, tdo, ta);
   return last_launch();
