@@ -12,8 +12,13 @@
 //
 // Plain row outputs whose rows TMA can address leave through shared memory
 // (the stage buffers are idle once the accumulator is complete) and TMA
-// stores; K/V pages and outputs that feed the in-epilogue RMSNorm are stored
-// per thread.
+// stores.  Float32 row outputs with a float32 residual and / or the
+// in-epilogue RMSNorm take the staged path end to end (`rows_tma`): the
+// residual comes in by TMA into the stage buffers, 16 KB boxes of 32 columns
+// at a time, each thread adds its row's values and writes the sum back in
+// place, the boxes leave by TMA; the RMSNorm pass then brings the stored row
+// block back by TMA (from L2) and sends the normalised bf16 rows out the same
+// way.  K/V pages and the remaining cases are stored per thread.
 //
 // Warp roles (192 threads): warps 0-3 epilogue, warp 4 TMA producer,
 // warp 5 TMEM allocator and MMA issuer.
@@ -37,10 +42,114 @@ struct TcGemmCfg {
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
+// Epilogue of rows_tma: `slots` 16 KB boxes of the stage area; pass 1 adds
+// the residual and stores the float32 rows, pass 2 (RMSNorm) normalises them.
+template <int BN>
+__device__ inline void rows_tma_epilogue(uint8_t* smem, int slots, uint64_t* ebar, const CUtensorMap* tmOut,
+                                         const CUtensorMap* tmRes, const CUtensorMap* tmRms, const GemmDesc& d,
+                                         uint32_t trow, int r, bool done, int n0, int mt0, int g, int grp,
+                                         int out_swap) {
+  const __nv_bfloat16* bias = (const __nv_bfloat16*)d.bias;
+  const bool lead = threadIdx.x == 0;
+  uint32_t ph = 0;   // parity of ebar's next completion
+  float ss = 0.f;
+  const int c1 = out_swap ? g : mt0, c2 = out_swap ? mt0 : g;   // the tile's row coordinates
+  bool ok = done;
+  constexpr int NBOX = BN / 32;
+  for (int q0 = 0; q0 < NBOX; q0 += slots) {
+    const int nb = min(slots, NBOX - q0);
+    if (d.res.base) {
+      if (lead) {
+        mbar_expect_tx(ebar, nb * 16384);
+        for (int i = 0; i < nb; ++i) tma_load_3d(tmRes, ebar, smem + i * 16384, n0 + (q0 + i) * 32, c1, c2);
+      }
+      ok = mbar_wait(ebar, ph) && ok;
+      ph ^= 1;
+    }
+    for (int i = 0; i < nb; ++i) {
+      const int c0 = (q0 + i) * 32, n = n0 + c0;
+      float v[32];
+      tmem_ld32(trow + c0, v);
+      if (bias) {
+        float bv[32];
+        load_bf16x32(bias + (long long)grp * d.bias_sg + d.n_lo + n, bv);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] += bv[e];
+      }
+      if (d.act == ACT_GELU) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = gelu_fast(v[e]);
+      }
+      if (d.res.base) {
+        float rv[32];
+        ld_sw128_f32(smem, i, r, rv);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] += rv[e];
+      }
+      if (n < d.scale_cols) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] *= d.col_scale;
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
+      st_sw128_f32(smem, i, r, v);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (lead && ok) {
+      for (int i = 0; i < nb; ++i) tma_store_3d(tmOut, smem + i * 16384, n0 + (q0 + i) * 32, c1, c2);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    // the stores have read the boxes before anyone writes them again (and,
+    // for the RMSNorm pass, the rows are in global memory)
+    if (lead) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
+  if (!d.rms.base) return;
+  // pass 2: h = x r g, r = (mean(x^2) + eps)^(-1/2); per group of h boxes (64
+  // bf16 columns) the two x boxes of each come back into slots 2j, 2j+1 and
+  // h goes out of slots from 2 * per on
+  const float rr = rsqrtf(ss / d.N + d.eps);
+  const __nv_bfloat16* gm = (const __nv_bfloat16*)d.gamma;
+  constexpr int NH = BN / 64;
+  const int per = max(1, slots / 3);
+  for (int j0 = 0; j0 < NH; j0 += per) {
+    const int nj = min(per, NH - j0);
+    if (lead) {
+      // the rows were stored by this CTA's own TMA stores (complete above)
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      mbar_expect_tx(ebar, nj * 2 * 16384);
+      for (int i = 0; i < 2 * nj; ++i) tma_load_3d(tmOut, ebar, smem + i * 16384, n0 + (2 * j0 + i) * 32, c1, c2);
+    }
+    ok = mbar_wait(ebar, ph) && ok;
+    ph ^= 1;
+    for (int j = 0; j < nj; ++j) {
+      float xv[64], gv[64];
+      ld_sw128_f32(smem, 2 * j, r, xv);
+      ld_sw128_f32(smem, 2 * j + 1, r, xv + 32);
+      load_bf16x32(gm + (j0 + j) * 64, gv);
+      load_bf16x32(gm + (j0 + j) * 64 + 32, gv + 32);
+#pragma unroll
+      for (int e = 0; e < 64; ++e) xv[e] = xv[e] * rr * gv[e];
+      st_sw128_32(smem + 2 * per * 16384 + j * 16384, 16384, r, 0, xv);
+      st_sw128_32(smem + 2 * per * 16384 + j * 16384, 16384, r, 32, xv + 32);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (lead && ok) {
+      for (int j = 0; j < nj; ++j) tma_store_3d(tmRms, smem + 2 * per * 16384 + j * 16384, n0 + (j0 + j) * 64, c1, c2);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    if (lead) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmOut, const GemmDesc d, const int a_swap,
+                   const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmRes,
+                   const __grid_constant__ CUtensorMap tmRms, const GemmDesc d, const int a_swap,
                    const int out_tma, const int out_swap) {
   using C = TcGemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -48,7 +157,8 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
   uint64_t* full = (uint64_t*)(smem + C::STAGES * C::STAGE_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
-  uint32_t* tmem_slot = (uint32_t*)(accf + 1);
+  uint64_t* ebar = accf + 1;   // rows_tma epilogue: residual / row-block loads
+  uint32_t* tmem_slot = (uint32_t*)(ebar + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN;
@@ -63,6 +173,7 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
+    mbar_init(ebar, 1);
     fence_barrier_init();
   }
   if (warp == 4 && lane == 0) {
@@ -123,6 +234,10 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
     const bool done = mbar_wait(accf, 0);
     tc_fence_after();
     const int r = warp * 32 + lane;
+    if (out_tma == 2) {
+      rows_tma_epilogue<BN>(smem, C::STAGES * C::STAGE_BYTES / 16384, ebar, &tmOut, &tmRes, &tmRms, d,
+                            tmem + ((uint32_t)(warp * 32) << 16), r, done, n0, mt0, g, grp, out_swap);
+    } else {
     const int m = mt0 + r;
     const bool valid = done && m < d.m_lo + d.M;
     int b = 0, t = 0;
@@ -201,6 +316,7 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
         store_row32(d.rms, rm_off(d.rms, b, t, c0), v);
       }
     }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -234,12 +350,12 @@ inline bool tc_gemm_supported(const GemmDesc& d) {
 
 // TMA map over the plain output rows of a GEMM (columns [0, N)), when the
 // rows form a strided 2-D set and the whole tile fits in the stage buffers.
-inline bool make_gemm_out_tmap(CUtensorMap* map, const GemmDesc& d, int bn, int stage_bytes, int& swap) {
-  const RowMap& r = d.out;
+// TMA map over the rows of a GEMM (columns [0, N)) held by RowMap r, boxes
+// of 128 rows x `bc` columns, when the rows form a strided 2-D set.
+inline bool make_rows_tmap(CUtensorMap* map, const GemmDesc& d, const RowMap& r, uint32_t bc, int& swap) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn || d.out_kind != OUT_ROWS || d.rms.base || r.split < d.N || ((uintptr_t)r.base % 16)) return false;
+  if (!fn || !r.base || r.split < d.N || ((uintptr_t)r.base % 16)) return false;
   const uint64_t es = r.f32 ? 4 : 2;
-  if ((uint64_t)128 * bn * es > (uint64_t)stage_bytes) return false;
   const uint64_t m_ext = (uint64_t)(d.m_lo + d.M), g_ext = (uint64_t)(d.g_lo + d.G);
   uint64_t s_m, s_g;
   if (d.mode == TILE_ROWS) { s_m = r.st; s_g = r.sb; }
@@ -250,7 +366,6 @@ inline bool make_gemm_out_tmap(CUtensorMap* map, const GemmDesc& d, int bn, int 
   }
   if (g_ext == 1) s_g = m_ext * s_m;
   swap = (g_ext > 1 && s_g < s_m) ? 1 : 0;
-  const uint32_t bc = r.f32 ? 32 : 64;
   const cuuint64_t dims[3] = {(cuuint64_t)d.N, swap ? g_ext : m_ext, swap ? m_ext : g_ext};
   const cuuint64_t strides[2] = {(swap ? s_g : s_m) * es, (swap ? s_m : s_g) * es};
   const cuuint32_t box[3] = {bc, swap ? 1u : 128u, swap ? 128u : 1u};
@@ -261,10 +376,71 @@ inline bool make_gemm_out_tmap(CUtensorMap* map, const GemmDesc& d, int bn, int 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// TMA map over the plain output rows of a GEMM, when the whole tile fits in
+// the stage buffers.
+inline bool make_gemm_out_tmap(CUtensorMap* map, const GemmDesc& d, int bn, int stage_bytes, int& swap) {
+  if (d.out_kind != OUT_ROWS || d.rms.base) return false;
+  const uint64_t es = d.out.f32 ? 4 : 2;
+  if ((uint64_t)128 * bn * es > (uint64_t)stage_bytes) return false;
+  return make_rows_tmap(map, d, d.out, d.out.f32 ? 32 : 64, swap);
+}
+
+// The staged float32-rows epilogue (rows_tma): float32 output rows, an
+// optional float32 residual, an optional RMSNorm of the whole row (bf16),
+// all three TMA-addressable with the same row geometry.
+inline bool make_rows_tma_maps(CUtensorMap* tout, CUtensorMap* tres, CUtensorMap* trms, const GemmDesc& d, int bn,
+                               int& swap) {
+  if (d.out_kind != OUT_ROWS || !d.out.f32 || d.act == ACT_GELU_BWD) return false;
+  if (d.res.base && !d.res.f32) return false;
+  if (d.rms.base && (bn != d.N || d.rms.f32 || (uintptr_t)d.gamma % 16)) return false;
+  int s_out = 0, s_res = 0, s_rms = 0;
+  if (!make_rows_tmap(tout, d, d.out, 32, s_out)) return false;
+  if (d.res.base && !make_rows_tmap(tres, d, d.res, 32, s_res)) return false;
+  if (d.rms.base && !make_rows_tmap(trms, d, d.rms, 64, s_rms)) return false;
+  if ((d.res.base && s_res != s_out) || (d.rms.base && s_rms != s_out)) return false;
+  swap = s_out;
+  return true;
+}
+
+// A flat row set (rows of B samples back to back, `fold` per sample) as
+// per-sample tiles, for an epilogue whose residual rows do not fold the same
+// way (the pyramid's tail rows of a longer input).  Taken when the last tile
+// of a sample wastes at most an eighth of the sample's rows.
+inline bool flat_to_rows(GemmDesc& g) {
+  if (g.mode != TILE_FLAT || g.G != 1 || g.m_lo != 0 || g.a_gext != 1 || g.fold < 128 || g.M % g.fold) return false;
+  const int waste = (g.fold + 127) / 128 * 128 - g.fold;
+  if (8 * waste > g.fold) return false;
+  const int B = g.M / g.fold;
+  g.mode = TILE_ROWS;
+  g.a_sg = (long long)g.fold * g.a_sm;
+  g.a_mext = g.fold;
+  g.a_gext = B;
+  g.M = g.fold;
+  g.G = B;
+  g.g_lo = 0;
+  return true;
+}
+
 template <int BN>
-inline onetrans_status tc_gemm_launch_bn(const GemmDesc& d, cudaStream_t st) {
+inline onetrans_status tc_gemm_launch_bn(const GemmDesc& d_in, cudaStream_t st) {
   using C = TcGemmCfg<BN>;
-  CUtensorMap ta, tb, tout;
+  CUtensorMap ta, tb, tout, tres, trms;
+  // the epilogue decides the row tiling: the staged float32 rows path where
+  // the output (and residual / RMSNorm rows) allow it, else the plain staged
+  // output, else per-thread stores
+  GemmDesc d = d_in;
+  int out_swap = 0, out_tma = 0;
+  if (make_rows_tma_maps(&tout, &tres, &trms, d, BN, out_swap)) {
+    out_tma = 2;
+  } else {
+    GemmDesc dr = d_in;
+    if (dr.res.base && flat_to_rows(dr) && make_rows_tma_maps(&tout, &tres, &trms, dr, BN, out_swap)) {
+      d = dr;
+      out_tma = 2;
+    } else if (make_gemm_out_tmap(&tout, d, BN, C::STAGES * C::STAGE_BYTES, out_swap)) {
+      out_tma = 1;
+    }
+  }
   const uint64_t mext = (uint64_t)d.a_mext, gext = (uint64_t)d.a_gext;
   const uint64_t s_m = (uint64_t)d.a_sm, s_g = gext > 1 ? (uint64_t)d.a_sg : mext * (uint64_t)d.a_sm;
   const int a_swap = (gext > 1 && d.a_sg < d.a_sm) ? 1 : 0;
@@ -281,11 +457,12 @@ inline onetrans_status tc_gemm_launch_bn(const GemmDesc& d, cudaStream_t st) {
       return ONETRANS_ERR_CUDA;
     attr_set = true;
   }
-  int out_swap = 0;
-  const int out_tma = make_gemm_out_tmap(&tout, d, BN, C::STAGES * C::STAGE_BYTES, out_swap) ? 1 : 0;
   if (!out_tma) tout = ta;
+  if (!d.res.base || out_tma != 2) tres = ta;
+  if (!d.rms.base || out_tma != 2) trms = ta;
   dim3 grid((unsigned)(d.N / BN), (unsigned)((d.M + 127) / 128), (unsigned)d.G);
-  launch_dependent(gemm_tc_kernel<BN>, grid, dim3(192), C::SMEM, st, ta, tb, tout, d, a_swap, out_tma, out_swap);
+  launch_dependent(gemm_tc_kernel<BN>, grid, dim3(192), C::SMEM, st, ta, tb, tout, tres, trms, d, a_swap, out_tma,
+                   out_swap);
   return cudaGetLastError() == cudaSuccess ? ONETRANS_OK : ONETRANS_ERR_CUDA;
 }
 
