@@ -56,12 +56,22 @@ __device__ inline void rows_tma_epilogue(uint8_t* smem, int slots, uint64_t* eba
   const int c1 = out_swap ? g : mt0, c2 = out_swap ? mt0 : g;   // the tile's row coordinates
   bool ok = done;
   constexpr int NBOX = BN / 32;
-  for (int q0 = 0; q0 < NBOX; q0 += slots) {
-    const int nb = min(slots, NBOX - q0);
+  // a bf16 residual arrives as boxes of 64 columns in the slots after the
+  // group's output boxes (one per two of them)
+  const bool res16 = d.res.base && !d.res.f32;
+  const int gmax = res16 ? (2 * slots / 3) & ~1 : slots;
+  for (int q0 = 0; q0 < NBOX; q0 += gmax) {
+    const int nb = min(gmax, NBOX - q0);
     if (d.res.base) {
       if (lead) {
-        mbar_expect_tx(ebar, nb * 16384);
-        for (int i = 0; i < nb; ++i) tma_load_3d(tmRes, ebar, smem + i * 16384, n0 + (q0 + i) * 32, c1, c2);
+        if (res16) {
+          mbar_expect_tx(ebar, (nb / 2) * 16384);
+          for (int j = 0; j < nb / 2; ++j)
+            tma_load_3d(tmRes, ebar, smem + (nb + j) * 16384, n0 + q0 * 32 + j * 64, c1, c2);
+        } else {
+          mbar_expect_tx(ebar, nb * 16384);
+          for (int i = 0; i < nb; ++i) tma_load_3d(tmRes, ebar, smem + i * 16384, n0 + (q0 + i) * 32, c1, c2);
+        }
       }
       ok = mbar_wait(ebar, ph) && ok;
       ph ^= 1;
@@ -82,7 +92,8 @@ __device__ inline void rows_tma_epilogue(uint8_t* smem, int slots, uint64_t* eba
       }
       if (d.res.base) {
         float rv[32];
-        ld_sw128_f32(smem, i, r, rv);
+        if (res16) ld_sw128_bf16_half(smem, nb + i / 2, r, i & 1, rv);
+        else ld_sw128_f32(smem, i, r, rv);
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] += rv[e];
       }
@@ -391,11 +402,10 @@ inline bool make_gemm_out_tmap(CUtensorMap* map, const GemmDesc& d, int bn, int 
 inline bool make_rows_tma_maps(CUtensorMap* tout, CUtensorMap* tres, CUtensorMap* trms, const GemmDesc& d, int bn,
                                int& swap) {
   if (d.out_kind != OUT_ROWS || !d.out.f32 || d.act == ACT_GELU_BWD) return false;
-  if (d.res.base && !d.res.f32) return false;
   if (d.rms.base && (bn != d.N || d.rms.f32 || (uintptr_t)d.gamma % 16)) return false;
   int s_out = 0, s_res = 0, s_rms = 0;
   if (!make_rows_tmap(tout, d, d.out, 32, s_out)) return false;
-  if (d.res.base && !make_rows_tmap(tres, d, d.res, 32, s_res)) return false;
+  if (d.res.base && !make_rows_tmap(tres, d, d.res, d.res.f32 ? 32 : 64, s_res)) return false;
   if (d.rms.base && !make_rows_tmap(trms, d, d.rms, 64, s_rms)) return false;
   if ((d.res.base && s_res != s_out) || (d.rms.base && s_rms != s_out)) return false;
   swap = s_out;

@@ -409,6 +409,21 @@ __device__ inline void ld_sw128_bf16(const uint8_t* tile, int box, int r, float*
     }
   }
 }
+// 32 bf16 values (to fp32): half `half` (columns 32 half .. +31) of row r of
+// a staged 64-column bf16 box.
+__device__ inline void ld_sw128_bf16_half(const uint8_t* tile, int box, int r, int half, float* v) {
+  const uint8_t* rowp = tile + box * 16384 + r * 128;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint4 u = *(const uint4*)(rowp + (((half * 4 + k) ^ (r & 7)) << 4));
+    const __nv_bfloat162* h = (const __nv_bfloat162*)&u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      v[8 * k + 2 * j] = f.x; v[8 * k + 2 * j + 1] = f.y;
+    }
+  }
+}
 __device__ inline void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
                "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
