@@ -53,10 +53,13 @@ struct GemmDesc {
   // A element (m, g, k) = A + m*a_sm + g*a_sg + k; extents for the TMA map
   const void* A;
   long long a_sm, a_sg, a_mext, a_gext;
-  // W element (grp, n, k) = W + grp*w_sg + (n_lo + n)*K + k
+  // W element (grp, n, k) = W + grp*w_sg + (n_lo + n)*K + k, or with w_mn set
+  // (a weight stored [K][w_rows], as dX = dY W reads the forward's W)
+  // W + grp*w_sg + k*w_rows + n_lo + n
   const void* W;
   long long w_sg;
   int w_rows, w_groups;
+  int w_mn;
   const void* bias;  // bias[grp*bias_sg + n_lo + n], or null
   long long bias_sg;
   int act;

@@ -109,9 +109,18 @@ __global__ void __launch_bounds__(BresCfg::THREADS, 1)
   if (warp == C::EPI_WARPS && lane == 0) {
     const uint64_t keep = l2_evict_last();
     mbar_expect_tx(w_full, C::W_BYTES);
+    if (d.w_mn) {
+      // [K][N] weight rows: per k-block four boxes of 64 columns x 64 rows (MN-major)
 #pragma unroll
-    for (int kb = 0; kb < C::KB; ++kb)
-      tma_load_3d_hint(&tmB, w_full, sW + kb * C::B_BYTES, kb * 64, d.n_lo + n0, grp, keep);
+      for (int kb = 0; kb < C::KB; ++kb)
+#pragma unroll
+        for (int c = 0; c < C::BN / 64; ++c)
+          tma_load_3d_hint(&tmB, w_full, sW + kb * C::B_BYTES + c * 8192, d.n_lo + n0 + c * 64, kb * 64, grp, keep);
+    } else {
+#pragma unroll
+      for (int kb = 0; kb < C::KB; ++kb)
+        tma_load_3d_hint(&tmB, w_full, sW + kb * C::B_BYTES, kb * 64, d.n_lo + n0, grp, keep);
+    }
   }
   grid_dep_wait();
   grid_dep_launch();
@@ -141,8 +150,10 @@ __global__ void __launch_bounds__(BresCfg::THREADS, 1)
   } else if (warp == C::EPI_WARPS + 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, C::BN);
-      const uint64_t da0 = sdesc_k128(smem_u32(sA)), dw0 = sdesc_k128(smem_u32(sW));
+      const uint32_t idesc = d.w_mn ? idesc_bf16(128, C::BN, false, true) : idesc_bf16(128, C::BN);
+      const uint64_t da0 = sdesc_k128(smem_u32(sA));
+      const uint64_t dw0 = d.w_mn ? sdesc_mn128(smem_u32(sW), 8192) : sdesc_k128(smem_u32(sW));
+      const uint32_t kstep = d.w_mn ? 2048 : 32;   // 16 k: 16 rows of 128 B, or 32 bytes of a row
       bool ok = mbar_wait(w_full, 0);
       if (ok) tc_fence_after();
       int q = 0, j = 0;
@@ -163,7 +174,7 @@ __global__ void __launch_bounds__(BresCfg::THREADS, 1)
           const uint64_t da = desc_add(da0, s * C::A_BYTES), dw = desc_add(dw0, kb * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            umma_bf16(tacc, desc_add(da, k * 32), desc_add(dw, k * 32), idesc, (kb | k) ? 1u : 0u);
+            umma_bf16(tacc, desc_add(da, k * 32), desc_add(dw, k * kstep), idesc, (kb | k) ? 1u : 0u);
           umma_commit(&a_empty[s]);
         }
         if (ok) umma_commit(&acc_full[acc]);
@@ -281,7 +292,8 @@ inline onetrans_status tc_bres_launch(const GemmDesc& d, int sm_count, cudaStrea
                    : make_tmap_3d(&ta, d.A, d.K, mext, gext, s_m, s_g, 64, 128, 1);
   const uint64_t wg = (uint64_t)d.w_groups;
   const uint64_t w_sg = wg > 1 ? (uint64_t)d.w_sg : (uint64_t)d.w_rows * d.K;
-  ok = ok && make_tmap_3d(&tb, d.W, d.K, d.w_rows, wg, d.K, w_sg, 64, C::BN, 1);
+  if (d.w_mn) ok = ok && make_tmap_3d(&tb, d.W, d.w_rows, d.K, wg, d.w_rows, w_sg, 64, 64, 1);
+  else ok = ok && make_tmap_3d(&tb, d.W, d.K, d.w_rows, wg, d.K, w_sg, 64, C::BN, 1);
   if (!ok) return ONETRANS_ERR_CUDA;
   static bool attr_set = false;
   if (!attr_set) {

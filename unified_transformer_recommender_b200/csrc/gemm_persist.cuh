@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(PersistCfg::THREADS, 1)
 
 // ------------------------------------------------------------------ host --
 inline bool tc_persist_supported(const GemmDesc& d) {
-  return d.out_kind == OUT_ROWS && !d.res.base && !d.rms.base && !d.out.f32 && d.N % PersistCfg::BN == 0 &&
+  return d.out_kind == OUT_ROWS && !d.res.base && !d.rms.base && !d.out.f32 && !d.w_mn && d.N % PersistCfg::BN == 0 &&
          tc_gemm_supported(d);
 }
 

@@ -33,8 +33,10 @@ struct TcGemmCfg {
   static constexpr int UN = BN <= 256 ? BN : BN / 2;  // N of one tcgen05.mma
   static constexpr int NSUB = BN / UN;
   static constexpr int BOX_N = BN <= 256 ? BN : BN / 2;  // TMA box rows of W (<= 256)
-  // two CTAs per SM for BN <= 256 (one's epilogue overlaps the other's loads and MMAs)
-  static constexpr int STAGES = BN <= 256 ? 2 : 3;
+  // two CTAs per SM for BN = 256 (one's epilogue overlaps the other's loads
+  // and MMAs); BN = 128 takes the small grids (a handful of tiles with a long
+  // K), where a deeper ring hides the load latency of the serial k-loop
+  static constexpr int STAGES = BN == 128 ? 4 : BN <= 256 ? 2 : 3;
   static constexpr int A_BYTES = 128 * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -211,15 +213,26 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
         mbar_expect_tx(&full[s], C::STAGE_BYTES);
         if (a_swap) tma_load_3d_hint(&tmA, &full[s], sa, kb * 64, g, mt0, stream);
         else tma_load_3d_hint(&tmA, &full[s], sa, kb * 64, mt0, g, stream);
+        if (d.w_mn) {
+          // 64 columns of N x the k-block's 64 rows per box (MN-major)
 #pragma unroll
-        for (int c = 0; c < BN / C::BOX_N; ++c)
-          tma_load_3d_hint(&tmB, &full[s], sb + c * C::BOX_N * 128, kb * 64, d.n_lo + n0 + c * C::BOX_N, grp, keep);
+          for (int c = 0; c < BN / 64; ++c)
+            tma_load_3d_hint(&tmB, &full[s], sb + c * 8192, d.n_lo + n0 + c * 64, kb * 64, grp, keep);
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN / C::BOX_N; ++c)
+            tma_load_3d_hint(&tmB, &full[s], sb + c * C::BOX_N * 128, kb * 64, d.n_lo + n0 + c * C::BOX_N, grp, keep);
+        }
       }
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, C::UN);
+      const uint32_t idesc = d.w_mn ? idesc_bf16(128, C::UN, false, true) : idesc_bf16(128, C::UN);
       const uint64_t d0 = sdesc_k128(smem_u32(smem));  // stage 0's A tile
+      // stage 0's B tile: K-major (16 k per 32 bytes), or MN-major (64-column
+      // boxes 8 KB apart, 16 k per 2 KB)
+      const uint64_t b0 = d.w_mn ? sdesc_mn128(smem_u32(smem + C::A_BYTES), 8192) : desc_add(d0, C::A_BYTES);
+      const uint32_t kstep = d.w_mn ? 2048 : 32;
       bool ok = true;
       for (int kb = 0; kb < KB && ok; ++kb) {
         const int s = kb % C::STAGES;
@@ -227,14 +240,14 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
         ok = mbar_wait(&full[s], ph);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t da = desc_add(d0, s * C::STAGE_BYTES);
+        const uint64_t da = desc_add(d0, s * C::STAGE_BYTES), db = desc_add(b0, s * C::STAGE_BYTES);
         const uint32_t acc0 = kb ? 1u : 0u;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
 #pragma unroll
           for (int j = 0; j < C::NSUB; ++j)
-            umma_bf16(tmem + j * C::UN, desc_add(da, k * 32), desc_add(da, C::A_BYTES + j * C::UN * 128 + k * 32),
-                      idesc, k ? 1u : acc0);
+            umma_bf16(tmem + j * C::UN, desc_add(da, k * 32), desc_add(db, j * C::UN * 128 + k * kstep), idesc,
+                      k ? 1u : acc0);
         }
         umma_commit(&empty[s]);
       }
@@ -337,6 +350,9 @@ __global__ void __launch_bounds__(192, BN <= 256 ? 2 : 1)
 // ------------------------------------------------------------------ host --
 inline int tc_pick_bn(const GemmDesc& d) {
   if (d.rms.base) return (d.N == 128 || d.N == 256 || d.N == 384) ? d.N : 0;
+  // a grid far below one wave with a long reduction: narrower tiles, more CTAs
+  const long long tiles256 = (long long)((d.N + 255) / 256) * ((d.M + 127) / 128) * d.G;
+  if (d.N % 128 == 0 && d.K >= 512 && 2 * tiles256 <= 148) return 128;
   if (d.N % 256 == 0) return 256;
   if (d.N % 384 == 0) return 384;
   if (d.N % 128 == 0) return 128;
@@ -348,6 +364,7 @@ inline bool tc_gemm_supported(const GemmDesc& d) {
   if (d.K <= 0 || d.K % 64 || !tc_pick_bn(d)) return false;
   if ((uintptr_t)d.A % 16 || (uintptr_t)d.W % 16) return false;
   if (d.a_sm % 8 || d.a_sg % 8 || d.w_sg % 8) return false;
+  if (d.w_mn && (d.w_rows % 64 || d.n_lo % 64)) return false;
   if (d.bias && ((d.bias_sg % 8) || (d.n_lo % 8) || ((uintptr_t)d.bias % 16))) return false;
   if (d.res.base && !rowmap_vec_ok(d.res)) return false;
   if (d.rms.base && (!rowmap_vec_ok(d.rms) || (uintptr_t)d.gamma % 16)) return false;
@@ -458,7 +475,8 @@ inline onetrans_status tc_gemm_launch_bn(const GemmDesc& d_in, cudaStream_t st) 
                    : make_tmap_3d(&ta, d.A, d.K, mext, gext, s_m, s_g, 64, 128, 1);
   const uint64_t wg = (uint64_t)d.w_groups;
   const uint64_t w_sg = wg > 1 ? (uint64_t)d.w_sg : (uint64_t)d.w_rows * d.K;
-  ok = ok && make_tmap_3d(&tb, d.W, d.K, d.w_rows, wg, d.K, w_sg, 64, C::BOX_N, 1);
+  if (d.w_mn) ok = ok && make_tmap_3d(&tb, d.W, d.w_rows, d.K, wg, d.w_rows, w_sg, 64, 64, 1);
+  else ok = ok && make_tmap_3d(&tb, d.W, d.K, d.w_rows, wg, d.K, w_sg, 64, C::BOX_N, 1);
   if (!ok) return ONETRANS_ERR_CUDA;
   static bool attr_set = false;
   if (!attr_set) {

@@ -244,6 +244,7 @@ static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, c
     }
     return tc_gemm_launch(d, st);
   }
+  if (d.w_mn) return ONETRANS_ERR_UNSUPPORTED;   // the callers transpose the weight instead
   dim3 grid((unsigned)cdiv(d.N, 64), (unsigned)cdiv(d.M, 64), (unsigned)d.G);
   gemm_simt_kernel<T><<<grid, 256, 0, st>>>(d);
   OT_TRY(last_launch());
@@ -1097,20 +1098,20 @@ static onetrans_status mixed_rows_gemm(const onetrans_model* m, const void* A, l
                                        const void* W_NS, int K, int N, RowMap out, cudaStream_t st,
                                        const void* bias_S = nullptr, const void* bias_NS = nullptr,
                                        RowMap res = RowMap{}, int act = ACT_NONE, RowMap act_in = RowMap{},
-                                       RowMap act_out = RowMap{}) {
+                                       RowMap act_out = RowMap{}, int w_mn = 0) {
   const bool flat = t_lo == 0 && t_hi == a_rows && a_samp == (long long)a_rows * a_row;
   if (t_s > t_lo && flat) {
     GemmDesc g = gdesc_base(m);
     g.mode = TILE_FLAT; g.M = B * a_rows; g.fold = a_rows; g.G = 1;
     g.K = K; g.A = A; g.a_sm = a_row; g.a_mext = (long long)B * a_rows; g.a_gext = 1;
-    g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S; g.act = act;
+    g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S; g.act = act; g.w_mn = w_mn;
     g.out = out; g.res = res; g.act_in = act_in; g.act_out = act_out;
     OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
   } else if (t_s > t_lo) {
     GemmDesc g = gdesc_base(m);
     g.mode = TILE_ROWS; g.M = t_s - t_lo; g.m_lo = t_lo; g.G = B; g.g_lo = 0;
     g.K = K; g.A = A; g.a_sm = a_row; g.a_sg = a_samp; g.a_mext = a_rows; g.a_gext = B;
-    g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S; g.act = act;
+    g.W = W_S; g.w_rows = N; g.N = N; g.bias = bias_S; g.act = act; g.w_mn = w_mn;
     g.out = out; g.res = res; g.act_in = act_in; g.act_out = act_out;
     OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
   }
@@ -1119,7 +1120,7 @@ static onetrans_status mixed_rows_gemm(const onetrans_model* m, const void* A, l
     g.mode = TILE_SAMPLES; g.M = B; g.G = t_hi - t_s; g.g_lo = t_s; g.grp_base = t_s;
     g.K = K; g.A = A; g.a_sm = a_samp; g.a_sg = a_row; g.a_mext = B; g.a_gext = a_rows;
     g.W = W_NS; g.w_sg = (long long)N * K; g.w_rows = N; g.w_groups = t_hi - t_s; g.N = N;
-    g.bias = bias_NS; g.bias_sg = bias_NS ? N : 0; g.act = act;
+    g.bias = bias_NS; g.bias_sg = bias_NS ? N : 0; g.act = act; g.w_mn = w_mn;
     g.out = out; g.res = res; g.act_in = act_in; g.act_out = act_out;
     OT_TRY(launch_gemm<T>(m, g, st, PK_TRAIN));
   }
@@ -1471,6 +1472,22 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     return ONETRANS_OK;
   };
 
+  // dX = dY W over a mixed row set (rows t < t_s use W_S, the others their NS
+  // token's set of W_NS; W [N_out = K][K_in = N] as the forward stores it):
+  // the tensor-core GEMMs read W as an MN-major operand; kernels that do not
+  // take one get the weights transposed
+  auto dx_gemm = [&](const void* A, long long a_row, long long a_samp, int rows, int t_s, const void* W_S,
+                     const void* W_NS, int K, int N, RowMap out, int act = ACT_NONE, RowMap act_in = RowMap{},
+                     RowMap act_out = RowMap{}) -> onetrans_status {
+    const onetrans_status r = mixed_rows_gemm<T>(m, A, a_row, a_samp, rows, B, 0, t_s, rows, W_S, W_NS, K, N, out, st,
+                                                 nullptr, nullptr, RowMap{}, act, act_in, act_out, 1);
+    if (r != ONETRANS_ERR_UNSUPPORTED) return r;
+    void *wS, *wNS;
+    OT_TRY(weights_T(W_S, W_NS, K, N, wS, wNS));
+    return mixed_rows_gemm<T>(m, A, a_row, a_samp, rows, B, 0, t_s, rows, wS, W_NS ? wNS : nullptr, K, N, out, st,
+                              nullptr, nullptr, RowMap{}, act, act_in, act_out, 0);
+  };
+
   // layer n's intermediates from its input x_in (L rows per sample).  The
   // forward pass computes the attention output and its log-sum-exp, kept
   // for the backward, and z = GELU(W1 h2 + b1); the backward recomputes the
@@ -1532,22 +1549,20 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     const long long Md = (long long)Lqn * d, Mf = (long long)Lqn * dff;
     // y = x1 + W2 z + b2
     OT_TRY(bias_grad(g_cur, d, Md, d, B, 0, sq, Lqn, gr->b2_S[n], gr->b2_NS[n], col_part, st));
-    void *wS, *wNS;
-    OT_TRY(weights_T(m->W2_S[n], m->W2_NS[n], d, dff, wS, wNS));
     // z = GELU(u), u = W1 h2 + b1: the dz GEMM's epilogue applies the GELU
     // backward where the weight-resident kernel takes the shape (du and z
     // in the storage type, dz never stored); otherwise dz in float32 and a
     // GELU-backward pass that also sums the S rows' du
     const onetrans_status fz =
         m->bf16 && g_policy == 0
-            ? mixed_rows_gemm<T>(m, gT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap(du, Mf, dff), st, nullptr,
-                                 nullptr, RowMap{}, ACT_GELU_BWD, rmap(u, Mf, dff), rmap(z, Mf, dff))
+            ? dx_gemm(gT, d, Md, Lqn, sq, m->W2_S[n], m->W2_NS[n], d, dff, rmap(du, Mf, dff), ACT_GELU_BWD,
+                      rmap(u, Mf, dff), rmap(z, Mf, dff))
             : ONETRANS_ERR_UNSUPPORTED;
     if (fz != ONETRANS_OK && fz != ONETRANS_ERR_UNSUPPORTED) return fz;
     const bool gelu_in_gemm = fz == ONETRANS_OK;
     bool gelu_fused = false;
     if (!gelu_in_gemm) {
-      OT_TRY(mixed_rows_gemm<T>(m, gT, d, Md, Lqn, B, 0, sq, Lqn, wS, wNS, d, dff, rmap32(dz, Mf, dff), st));
+      OT_TRY(dx_gemm(gT, d, Md, Lqn, sq, m->W2_S[n], m->W2_NS[n], d, dff, rmap32(dz, Mf, dff)));
       const long long nz = (long long)B * Mf;
       const int rows = B * Lqn;
       gelu_fused = gr->b1_S[n] && dff % 4 == 0 && dff <= 4096;
@@ -1582,15 +1597,13 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
                      col_part, st));
     OT_TRY(weight_grad<T>(m, GradRows{du, dff, Mf, false}, GradRows{h2, d, Md, false}, dff, d, B, 0, sq, Lqn,
                           gr->W1_S[n], gr->W1_NS[n], sc, st));
-    OT_TRY(weights_T(m->W1_S[n], m->W1_NS[n], dff, d, wS, wNS));
-    OT_TRY(mixed_rows_gemm<T>(m, du, dff, Mf, Lqn, B, 0, sq, Lqn, wS, wNS, dff, d, rmap32(dh2, Md, d), st));
+    OT_TRY(dx_gemm(du, dff, Mf, Lqn, sq, m->W1_S[n], m->W1_NS[n], dff, d, rmap32(dh2, Md, d)));
     // h2 = RMSNorm(x1; g_ffn), x1 = x[tail] + W^O a; y's gradient reaches x1 around the FFN
     OT_TRY((launch_rms_backward<T, float>(x1, Md, d, m->g_ffn[n], dh2, g_cur, Md, d, 0, dx1, pg, B * Lqn, Lqn, d,
                                          m->cfg.rms_eps, dx1T, gr->g_ffn[n], col_part, st)));
     OT_TRY(weight_grad<T>(m, GradRows{dx1T, d, Md, false}, GradRows{a, d, Md, false}, d, d, B, 0, Lqn, Lqn,
                           gr->Wo[n], nullptr, sc, st));
-    OT_TRY(weights_T(m->Wo[n], nullptr, d, d, wS, wNS));
-    OT_TRY(mixed_rows_gemm<T>(m, dx1T, d, Md, Lqn, B, 0, Lqn, Lqn, wS, nullptr, d, d, rmap(dOb, Md, d), st));
+    OT_TRY(dx_gemm(dx1T, d, Md, Lqn, Lqn, m->Wo[n], nullptr, d, d, rmap(dOb, Md, d)));
     // attention: dq, dk, dv of the recomputed rows
     OT_TRY(cuda_ok(cudaMemsetAsync(dqkv, 0, (size_t)B * L * 3 * d * es, st)));
     AttnRows ar;
@@ -1612,9 +1625,7 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     const long long Mq = (long long)L * 3 * d;
     OT_TRY(weight_grad<T>(m, GradRows{dqkv, 3 * d, Mq, false}, GradRows{h, d, (long long)L * d, false}, 3 * d, d,
                           B, 0, s, L, gr->Wqkv_S[n], gr->Wqkv_NS[n], sc, st));
-    OT_TRY(weights_T(m->Wqkv_S[n], m->Wqkv_NS[n], 3 * d, d, wS, wNS));
-    OT_TRY(mixed_rows_gemm<T>(m, dqkv, 3 * d, Mq, L, B, 0, s, L, wS, wNS, 3 * d, d,
-                              rmap32(dh, (long long)L * d, d), st));
+    OT_TRY(dx_gemm(dqkv, 3 * d, Mq, L, s, m->Wqkv_S[n], m->Wqkv_NS[n], 3 * d, d, rmap32(dh, (long long)L * d, d)));
     // h = RMSNorm(x; g_attn); x1's gradient reaches the tail rows of x around
     // the attention; the lower layer's output gradient also as its GEMM operand
     void* g_copy = n > 0 ? gT : nullptr;
