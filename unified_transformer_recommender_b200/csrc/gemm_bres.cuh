@@ -12,7 +12,10 @@
 // thread issues the 128 x 256 tcgen05.mma steps into one of two TMEM
 // accumulators, so the MMAs of tile i+1 run while eight epilogue warps drain
 // tile i (tcgen05.ld, bias / GELU / column scale, bf16) and send it out by TMA
-// stores through a 32 KB staging area, half a tile at a time.
+// stores through a 32 KB staging area, half a tile at a time.  The training
+// step's dz GEMM adds the GELU backward to the epilogue (ACT_GELU_BWD: u read
+// per row, du out by TMA, GELU(u) stored per row), and its dX GEMMs load the
+// slice from the forward's [K][N] weight as MN-major boxes (w_mn).
 //
 // Warp roles (320 threads): warps 0-7 epilogue (warp w and w+4 share TMEM
 // lanes 32*(w%4).. and take one half of the tile's columns each), warp 8 TMA
