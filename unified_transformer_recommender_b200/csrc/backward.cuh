@@ -274,8 +274,10 @@ __global__ void __launch_bounds__(256) rms_backward_kernel(const Tx* __restrict_
 // order (chunk_sum_kernel then adds the CTAs' rows in CTA order).  dx is
 // written, not accumulated: the gradient that reaches x around the norm (the
 // residual branch) is read from `res`, row t - r_off of the sample (0 for
-// t < r_off or without res).  Needs the row strides % 4 == 0 and
-// vector-aligned bases.
+// t < r_off or without res).  With part_s, the CTA also leaves the column
+// sums of the finished dx rows with t < s_rows as part_s[k][d] (the shared
+// b2 gradient of the layer below, whose output x is).  Needs the row strides
+// % 4 == 0 and vector-aligned bases.
 template <typename Tx, typename T, int NC4>
 __global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restrict__ x, long long x_sb, long long x_st,
                                                               const T* __restrict__ gamma,
@@ -283,16 +285,17 @@ __global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restri
                                                               const float* __restrict__ res, long long r_sb,
                                                               long long r_st, int r_off, float* __restrict__ dx,
                                                               long long dx_sb, long long dx_st, float* __restrict__ part,
-                                                              int rows, int fold, float eps, T* __restrict__ dx_copy) {
+                                                              int rows, int fold, float eps, T* __restrict__ dx_copy,
+                                                              float* __restrict__ part_s, int s_rows) {
   constexpr int d = 128 * NC4;
   __shared__ float red[8][d];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  float gm[NC4][4], pg[NC4][4];
+  float gm[NC4][4], pg[NC4][4], ps[NC4][4];
 #pragma unroll
   for (int i = 0; i < NC4; ++i) {
     ld4<T>(gamma + 128 * i + 4 * lane, gm[i]);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) pg[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) pg[i][j] = ps[i][j] = 0.f;
   }
   for (int row = blockIdx.x * 8 + w; row < rows; row += gridDim.x * 8) {
     const int b = row / fold, t = row - b * fold;
@@ -320,6 +323,7 @@ __global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restri
     float* dxr = dx + b * dx_sb + t * dx_st;
     T* cpr = dx_copy ? dx_copy + b * dx_sb + t * dx_st : nullptr;
     const float* rr = (res && t >= r_off) ? res + b * r_sb + (t - r_off) * r_st : nullptr;
+    const bool s_row = t < s_rows;
 #pragma unroll
     for (int i = 0; i < NC4; ++i) {
       float o[4] = {0.f, 0.f, 0.f, 0.f};
@@ -328,6 +332,7 @@ __global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restri
       for (int j = 0; j < 4; ++j) {
         o[j] += r * gm[i][j] * dv[i][j] - xv[i][j] * c3;
         pg[i][j] = fmaf(dv[i][j], xv[i][j] * r, pg[i][j]);
+        if (s_row) ps[i][j] += o[j];
       }
       st4<float>(dxr + 128 * i + 4 * lane, o);
       if (cpr) st4<T>(cpr + 128 * i + 4 * lane, o);   // the finished row, as the next GEMM's operand
@@ -343,6 +348,19 @@ __global__ void __launch_bounds__(256) rms_backward_dg_kernel(const Tx* __restri
 #pragma unroll
     for (int q = 0; q < 8; ++q) t += red[q][c];
     part[(long long)blockIdx.x * d + c] = t;
+  }
+  if (!part_s) return;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < NC4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) red[w][128 * i + 4 * lane + j] = ps[i][j];
+  __syncthreads();
+  for (int c = threadIdx.x; c < d; c += 256) {
+    float t = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t += red[q][c];
+    part_s[(long long)blockIdx.x * d + c] = t;
   }
 }
 

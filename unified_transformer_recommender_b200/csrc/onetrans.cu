@@ -1285,7 +1285,11 @@ template <typename T, typename Tx>
 static onetrans_status launch_rms_backward(const void* x, long long x_sb, long long x_st, const void* gamma,
                                            const float* dy, const float* res, long long r_sb, long long r_st,
                                            int r_off, float* dx, float* pg, int rows, int fold, int d, float eps,
-                                           void* dx_copy, float* dg, float* part, cudaStream_t st) {
+                                           void* dx_copy, float* dg, float* part, cudaStream_t st,
+                                           float* db_s = nullptr, int s_rows = 0, bool* db_s_done = nullptr) {
+  // db_s (optional): the column sums of the finished dx rows with t < s_rows,
+  // taken in the fused row kernel only (*db_s_done tells the caller)
+  if (db_s_done) *db_s_done = false;
   if (rows <= 0) return dg ? cuda_ok(cudaMemsetAsync(dg, 0, (size_t)d * 4, st)) : ONETRANS_OK;
   const long long dx_sb = (long long)fold * d, dx_st = d;
   const bool fused = d % 128 == 0 && d <= 512 && vec4_ok(x, 4 * sizeof(Tx), {x_sb, x_st}) &&
@@ -1293,6 +1297,7 @@ static onetrans_status launch_rms_backward(const void* x, long long x_sb, long l
                      vec4_ok(gamma, 4 * sizeof(T), {}) && vec4_ok(dx_copy, 4 * sizeof(T), {});
   if (fused) {
     const int ctas = (int)std::min<long long>(cdiv(rows, 8), kRedCtas);
+    float* part_s = db_s ? part + (size_t)kRedCtas * d : nullptr;
     {
       ProfScope prof(PK_TRAIN_ELEM, 0.0,
                      (double)rows * d * (sizeof(Tx) + 4.0 + 8.0 + (dx_copy ? sizeof(T) : 0)) + (double)ctas * d * 4,
@@ -1300,7 +1305,7 @@ static onetrans_status launch_rms_backward(const void* x, long long x_sb, long l
 #define OT_RMS_DG(NC4)                                                                                             \
   rms_backward_dg_kernel<Tx, T, NC4><<<(unsigned)ctas, 256, 0, st>>>((const Tx*)x, x_sb, x_st, (const T*)gamma, dy, \
                                                                     res, r_sb, r_st, r_off, dx, dx_sb, dx_st, part, \
-                                                                    rows, fold, eps, (T*)dx_copy)
+                                                                    rows, fold, eps, (T*)dx_copy, part_s, s_rows)
       switch (d / 128) {
         case 1: OT_RMS_DG(1); break;
         case 2: OT_RMS_DG(2); break;
@@ -1310,7 +1315,12 @@ static onetrans_status launch_rms_backward(const void* x, long long x_sb, long l
 #undef OT_RMS_DG
       OT_TRY(last_launch());
     }
-    return launch_chunk_sum(part, ctas, d, dg, 0, d, st);
+    OT_TRY(launch_chunk_sum(part, ctas, d, dg, 0, d, st));
+    if (db_s) {
+      OT_TRY(launch_chunk_sum(part_s, ctas, d, db_s, 0, d, st));
+      if (db_s_done) *db_s_done = true;
+    }
+    return ONETRANS_OK;
   }
   // dx starts as the residual gradient
   OT_TRY(cuda_ok(cudaMemsetAsync(dx, 0, (size_t)rows * d * 4, st)));
@@ -1537,6 +1547,7 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
   // kept in float32 (g_cur, for the residual and the bias sums) and in the
   // storage type (gT, the GEMM operand)
   const float* g_cur = dy;   // gradient of layer n's output, [B, Lq[n], d]
+  bool b2s_done = false;     // db2 of the shared set of layer n already summed by the layer above
   OT_TRY(launch_cast<T>(dy, gT, (long long)B * Lq[NL - 1] * d, st));
   for (int n = NL - 1; n >= 0; --n) {
     const int L = Ln[n], Lqn = Lq[n], s = L - L_NS, sq = Lqn - L_NS, off = L - Lqn;
@@ -1548,7 +1559,7 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     OT_TRY(recompute(n, x_in, x_f32, false));
     const long long Md = (long long)Lqn * d, Mf = (long long)Lqn * dff;
     // y = x1 + W2 z + b2
-    OT_TRY(bias_grad(g_cur, d, Md, d, B, 0, sq, Lqn, gr->b2_S[n], gr->b2_NS[n], col_part, st));
+    OT_TRY(bias_grad(g_cur, d, Md, d, B, 0, sq, Lqn, b2s_done ? nullptr : gr->b2_S[n], gr->b2_NS[n], col_part, st));
     // z = GELU(u), u = W1 h2 + b1: the dz GEMM's epilogue applies the GELU
     // backward where the weight-resident kernel takes the shape (du and z
     // in the storage type, dz never stored); otherwise dz in float32 and a
@@ -1629,9 +1640,12 @@ static onetrans_status train_impl(const onetrans_model* m, const void* x0, int B
     // h = RMSNorm(x; g_attn); x1's gradient reaches the tail rows of x around
     // the attention; the lower layer's output gradient also as its GEMM operand
     void* g_copy = n > 0 ? gT : nullptr;
+    // the lower layer's db2 (shared set: its S rows t < L - L_NS) from the same pass
+    float* db2_below = n > 0 ? gr->b2_S[n - 1] : nullptr;
     if (x_f32)
       OT_TRY((launch_rms_backward<T, float>(x_in, (long long)L * d, d, m->g_attn[n], dh, dx1, Md, d, off, g_in, pg,
-                                           B * L, L, d, m->cfg.rms_eps, g_copy, gr->g_attn[n], col_part, st)));
+                                           B * L, L, d, m->cfg.rms_eps, g_copy, gr->g_attn[n], col_part, st,
+                                           db2_below, L - L_NS, &b2s_done)));
     else
       OT_TRY((launch_rms_backward<T, T>(x_in, (long long)L * d, d, m->g_attn[n], dh, dx1, Md, d, off, g_in, pg,
                                        B * L, L, d, m->cfg.rms_eps, g_copy, gr->g_attn[n], col_part, st)));
