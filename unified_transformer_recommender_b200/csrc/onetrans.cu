@@ -95,6 +95,8 @@ struct ProfScope {
     if (!rec.e0 || !rec.e1) return;
     on = cudaEventRecord(rec.e0, st) == cudaSuccess;
   }
+  // the scope launched nothing after all (a kernel refused the shape): no record
+  void cancel() { on = false; }
   ~ProfScope() {
     if (!on) return;
     std::lock_guard<std::mutex> lk(g_prof.mu);
@@ -230,8 +232,13 @@ static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, c
   ProfScope prof(kind, 2.0 * d.M * d.G * (double)d.N * d.K, gemm_bytes(m, d), st);
   if (d.act == ACT_GELU_BWD) {
     // the GELU-backward epilogue exists in the weight-resident kernel only
-    if (!(m->bf16 && g_policy == 0 && tc_gemm_supported(d) && tc_bres_supported(d))) return ONETRANS_ERR_UNSUPPORTED;
-    return tc_bres_launch(d, device_sm_count(), st);
+    if (!(m->bf16 && g_policy == 0 && tc_gemm_supported(d) && tc_bres_supported(d))) {
+      prof.cancel();
+      return ONETRANS_ERR_UNSUPPORTED;
+    }
+    const onetrans_status r = tc_bres_launch(d, device_sm_count(), st);
+    if (r == ONETRANS_ERR_UNSUPPORTED) prof.cancel();
+    return r;
   }
   if (m->bf16 && g_policy == 0 && tc_gemm_supported(d)) {
     if (tc_bres_supported(d)) {
@@ -244,7 +251,10 @@ static onetrans_status launch_gemm(const onetrans_model* m, const GemmDesc& d, c
     }
     return tc_gemm_launch(d, st);
   }
-  if (d.w_mn) return ONETRANS_ERR_UNSUPPORTED;   // the callers transpose the weight instead
+  if (d.w_mn) {   // the callers transpose the weight instead
+    prof.cancel();
+    return ONETRANS_ERR_UNSUPPORTED;
+  }
   dim3 grid((unsigned)cdiv(d.N, 64), (unsigned)cdiv(d.M, 64), (unsigned)d.G);
   gemm_simt_kernel<T><<<grid, 256, 0, st>>>(d);
   OT_TRY(last_launch());
