@@ -4,11 +4,10 @@ Mistakes are planted in the oracle's backward, on the CPU: the RMSNorm
 backward without its mean term (the r^3 x sum(g dy x)/d part), the softmax
 backward without its row term D = rowsum(dP P), and the GELU derivative
 without its second term.  Each moves some gradient of the stack by more
-than twice the norm-wise bf16 bar of `test_gpu_train.py` (on these inputs
-by 0.27, 1.36 and 0.37 of the gradient's norm)
-(||got - ref|| / ||ref|| <= 2e-2), so a kernel with that mistake fails it,
-while bf16 rounding of the operands costs about 5e-3 norm-wise (the bar's
-derivation).  Weights at std 1/sqrt(d), as in the GPU training tests."""
+than twice the norm-wise bf16 bar of `test_gpu_train.py`
+(||got - ref|| / ||ref|| <= 2e-2; on these inputs by 0.27, 1.36 and 0.37),
+so a kernel with that mistake fails it, while bf16 rounding of the operands
+costs about 5e-3 norm-wise (the bar's derivation).  Weights at std 1/sqrt(d), as in the GPU training tests."""
 import numpy as np
 import pytest
 
