@@ -354,4 +354,8 @@ def test_forward_backward_argument_errors_before_any_launch():
     assert fb(fm.h, FAKE, 2, 1178, FAKE, FAKE, FAKE, ctypes.byref(g), FAKE, big, None) == ot.ERR_INVALID_ARG
     out = ot.SZ(0)
     assert ot.lib.onetrans_workspace_size(fm.h, ot.OP_TRAIN, 2, 1178, ctypes.byref(out)) == ot.OK
-    assert out.value > 2 * 1190 * 256 * 4 * 5                       # at least the kept layer inputs
+    # at least what the forward keeps: the float32 inputs of layers 1..5 and
+    # every layer's bf16 attention output and float32 log-sum-exp
+    kept = sum(2 * sched[n - 1] * 256 * 4 for n in range(1, 6))
+    kept += sum(2 * q * 256 * 2 + 2 * 4 * q * 4 for q in sched)
+    assert out.value > kept
