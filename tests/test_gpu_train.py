@@ -1,5 +1,7 @@
-"""The training step (forward keeping each layer's input, backward with each
-layer recomputed from it) through the C ABI against the oracle's backward:
+"""The training step (forward keeping each layer's input, attention output and
+log-sum-exp; backward with the rest of each layer recomputed) through the C
+ABI against the oracle's backward (which recomputes whole layers; the
+gradients are the same):
 the output, the input gradient and every weight gradient.  Weights at std
 1/sqrt(d), so attention is far from uniform and its backward matters.
 
